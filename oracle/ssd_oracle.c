@@ -1,0 +1,341 @@
+/*
+ * ssd_oracle.c -- plain, slow, float64 CPU oracle of the Mamba-2 SSD layer core.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path links, loads or calls
+ * this file: only the test-suite, the smoke check and the benchmark's CPU
+ * baseline leg use it.  It shares no code, header, table or helper with the
+ * CUDA library; it is written from the method's definition, not from kernels.
+ *
+ * What it computes (per batch b and head h, state of size N x P):
+ *
+ *   dt_t = softplus(dt_raw[t,h] + dt_bias[h])
+ *   h_t  = exp(dt_t * A[h]) * h_{t-1} + dt_t * B_t x_t^T          (N x P)
+ *   y_t  = C_t^T h_t + D[h] * x_t                                  (P)
+ *
+ * Sources (titles of the pages the method is described on):
+ *  - "Mamba3" (Telegram post, ai_machinelearning_big_data), paragraph on
+ *    Mamba-2: the state transition matrix is a scalar times the identity; and
+ *    section "New discretisation scheme": Mamba-1/2 discretise with a mix of
+ *    ZOH (here exp(dt*A) on the state) and Euler (here dt*B on the input).
+ *  - "Mamba-3 : SSM optimise inference" (call-informatique.fr), section
+ *    "Du training-first a l'inference-first": transition reduced to a scalar
+ *    times identity.
+ *  - "Mamba-2 vs Transformers / SSD" (axiomlogica.com), section "Mamba-2 and
+ *    the SSD paper: what changed in practice": the layer is a semiseparable
+ *    matrix; SSM recurrence and masked attention are two contraction orders of
+ *    it; the blocked algorithm splits the sequence into chunks processed in
+ *    parallel and recombines the per-chunk states.
+ *
+ * Readings where the pages are silent (every one is also listed in the design doc):
+ *  - y_t uses the state AFTER the token-t update (so the diagonal of the
+ *    semiseparable mask is exp(0) = 1).
+ *  - softplus(z) = log(1 + e^z), evaluated exactly (no threshold).
+ *  - head h reads group g = h / (H / G) of B and C (contiguous head blocks).
+ *  - D and dt_bias are one scalar per head; NULL means zero.
+ *  - init_state NULL means a zero initial state.
+ *
+ * Layouts (row-major, last index fastest):
+ *   x, y [b][L][H][P]; dt_raw [b][L][H]; B, C [b][L][G][N];
+ *   dt_bias, A, D [H]; init_state, final_state [b][H][N][P].
+ *   Decode step: x, y [b][H][P]; dt_raw [b][H]; B, C [b][G][N]; state [b][H][N][P].
+ *
+ * All functions return 0 on success, -1 on invalid arguments.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* softplus(z) = log(1 + exp(z)), written so that it neither overflows for
+ * large z nor loses digits for very negative z. */
+static double sp(double z) { return fmax(z, 0.0) + log1p(exp(-fabs(z))); }
+
+double oracle_softplus(double z) { return sp(z); }
+
+/* Round a double to the nearest bfloat16 value (8 significant bits, 8-bit
+ * exponent like IEEE binary32), ties to even.  Used only where the API stores
+ * a state in bf16 (the reading of "the oracle runs on the bf16-rounded
+ * values" for a bf16 decode state). */
+double oracle_round_bf16(double v) {
+    if (v == 0.0 || !isfinite(v)) return v;
+    int e2;
+    (void)frexp(v, &e2);           /* |v| in [2^(e2-1), 2^e2) */
+    int e = e2 - 1;
+    if (e < -126) e = -126;        /* subnormal range: fixed spacing 2^-133 */
+    double spacing = ldexp(1.0, e - 7);
+    double q = nearbyint(v / spacing);   /* default mode: ties to even */
+    double r = q * spacing;
+    const double bf16_max = ldexp(255.0 / 128.0, 127);  /* (2 - 2^-7) * 2^127 */
+    if (fabs(r) > bf16_max) return v > 0 ? INFINITY : -INFINITY;
+    return r;
+}
+
+static int set_threads(int nthreads) {
+#ifdef _OPENMP
+    if (nthreads > 0) return nthreads;
+    return omp_get_max_threads();
+#else
+    (void)nthreads;
+    return 1;
+#endif
+}
+
+int oracle_num_threads(void) { return set_threads(0); }
+
+static int check_dims(int64_t b, int64_t L, int64_t H, int64_t P, int64_t N, int64_t G) {
+    if (b <= 0 || L < 0 || H <= 0 || P <= 0 || N <= 0 || G <= 0) return -1;
+    if (H % G != 0) return -1;
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* 1. Sequential recurrence: the definition itself.                          */
+/* ------------------------------------------------------------------------ */
+int oracle_ssd_recurrent(int64_t batch, int64_t seqlen, int64_t nheads, int64_t headdim,
+                         int64_t dstate, int64_t ngroups,
+                         const double* x, const double* dt_raw, const double* dt_bias,
+                         const double* A, const double* B, const double* C, const double* D,
+                         const double* init_state, double* y, double* final_state,
+                         int nthreads) {
+    if (check_dims(batch, seqlen, nheads, headdim, dstate, ngroups)) return -1;
+    if (!x || !dt_raw || !A || !B || !C) return -1;
+    const int64_t H = nheads, P = headdim, N = dstate, G = ngroups, L = seqlen;
+    const int64_t heads_per_group = H / G;
+    const int nt = set_threads(nthreads);
+    int64_t pair;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nt)
+    for (pair = 0; pair < batch * H; ++pair) {
+        const int64_t b = pair / H, h = pair % H, g = h / heads_per_group;
+        double* st = (double*)malloc(sizeof(double) * N * P);
+        if (init_state) memcpy(st, init_state + (b * H + h) * N * P, sizeof(double) * N * P);
+        else memset(st, 0, sizeof(double) * N * P);
+        const double bias = dt_bias ? dt_bias[h] : 0.0;
+        const double d_skip = D ? D[h] : 0.0;
+        for (int64_t t = 0; t < L; ++t) {
+            const double dt = sp(dt_raw[(b * L + t) * H + h] + bias);
+            const double decay = exp(dt * A[h]);
+            const double* xt = x + ((b * L + t) * H + h) * P;
+            const double* Bt = B + ((b * L + t) * G + g) * N;
+            const double* Ct = C + ((b * L + t) * G + g) * N;
+            /* h_t = decay * h_{t-1} + dt * B_t x_t^T */
+            for (int64_t n = 0; n < N; ++n) {
+                const double coef = dt * Bt[n];
+                double* row = st + n * P;
+                for (int64_t p = 0; p < P; ++p) row[p] = decay * row[p] + coef * xt[p];
+            }
+            /* y_t = C_t^T h_t + D x_t */
+            if (y) {
+                double* yt = y + ((b * L + t) * H + h) * P;
+                for (int64_t p = 0; p < P; ++p) {
+                    double acc = 0.0;
+                    for (int64_t n = 0; n < N; ++n) acc += Ct[n] * st[n * P + p];
+                    yt[p] = acc + d_skip * xt[p];
+                }
+            }
+        }
+        if (final_state) memcpy(final_state + (b * H + h) * N * P, st, sizeof(double) * N * P);
+        free(st);
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* 2. Quadratic ("masked attention") form of the same semiseparable matrix:  */
+/*    y = (Lmask o C B^T)(dt x) + D x + exp(cs_i) C_i^T h0,                  */
+/*    Lmask[i][j] = exp(cs_i - cs_j) for j <= i, else 0,                     */
+/*    cs_i = sum_{k<=i} dt_k A  (inclusive).                                 */
+/*    final_state = exp(cs_{L-1}) h0 + sum_j exp(cs_{L-1}-cs_j) dt_j B_j x_j^T */
+/* ------------------------------------------------------------------------ */
+int oracle_ssd_quadratic(int64_t batch, int64_t seqlen, int64_t nheads, int64_t headdim,
+                         int64_t dstate, int64_t ngroups,
+                         const double* x, const double* dt_raw, const double* dt_bias,
+                         const double* A, const double* B, const double* C, const double* D,
+                         const double* init_state, double* y, double* final_state,
+                         int nthreads) {
+    if (check_dims(batch, seqlen, nheads, headdim, dstate, ngroups)) return -1;
+    if (!x || !dt_raw || !A || !B || !C) return -1;
+    const int64_t H = nheads, P = headdim, N = dstate, G = ngroups, L = seqlen;
+    const int64_t heads_per_group = H / G;
+    const int nt = set_threads(nthreads);
+    int64_t pair;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nt)
+    for (pair = 0; pair < batch * H; ++pair) {
+        const int64_t b = pair / H, h = pair % H, g = h / heads_per_group;
+        const double bias = dt_bias ? dt_bias[h] : 0.0;
+        const double d_skip = D ? D[h] : 0.0;
+        double* dt = (double*)malloc(sizeof(double) * (L + 1));
+        double* cs = (double*)malloc(sizeof(double) * (L + 1));
+        double run = 0.0;
+        for (int64_t t = 0; t < L; ++t) {
+            dt[t] = sp(dt_raw[(b * L + t) * H + h] + bias);
+            run += dt[t] * A[h];
+            cs[t] = run;
+        }
+        const double* h0 = init_state ? init_state + (b * H + h) * N * P : NULL;
+        for (int64_t i = 0; y && i < L; ++i) {
+            const double* Ci = C + ((b * L + i) * G + g) * N;
+            double* yi = y + ((b * L + i) * H + h) * P;
+            for (int64_t p = 0; p < P; ++p) yi[p] = 0.0;
+            for (int64_t j = 0; j <= i; ++j) {
+                const double* Bj = B + ((b * L + j) * G + g) * N;
+                const double* xj = x + ((b * L + j) * H + h) * P;
+                double cb = 0.0;
+                for (int64_t n = 0; n < N; ++n) cb += Ci[n] * Bj[n];
+                const double m = exp(cs[i] - cs[j]) * cb * dt[j];
+                for (int64_t p = 0; p < P; ++p) yi[p] += m * xj[p];
+            }
+            if (h0) {
+                const double e = exp(cs[i]);
+                for (int64_t p = 0; p < P; ++p) {
+                    double acc = 0.0;
+                    for (int64_t n = 0; n < N; ++n) acc += Ci[n] * h0[n * P + p];
+                    yi[p] += e * acc;
+                }
+            }
+            const double* xi = x + ((b * L + i) * H + h) * P;
+            for (int64_t p = 0; p < P; ++p) yi[p] += d_skip * xi[p];
+        }
+        if (final_state) {
+            double* hf = final_state + (b * H + h) * N * P;
+            const double last = L > 0 ? cs[L - 1] : 0.0;
+            for (int64_t k = 0; k < N * P; ++k) hf[k] = h0 ? exp(last) * h0[k] : 0.0;
+            for (int64_t j = 0; j < L; ++j) {
+                const double w = exp(last - cs[j]) * dt[j];
+                const double* Bj = B + ((b * L + j) * G + g) * N;
+                const double* xj = x + ((b * L + j) * H + h) * P;
+                for (int64_t n = 0; n < N; ++n)
+                    for (int64_t p = 0; p < P; ++p) hf[n * P + p] += w * Bj[n] * xj[p];
+            }
+        }
+        free(dt);
+        free(cs);
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* 3. Chunked (blocked two-pass) restatement: the sequence is cut into       */
+/*    chunks of `chunk` tokens (the last one may be shorter).  Per chunk:    */
+/*    acs_l = chunk-local inclusive cumsum of dt*A;                          */
+/*    intra-chunk quadratic block; chunk state                               */
+/*    S_c = sum_s exp(acs_last - acs_s) dt_s B_s x_s^T;                      */
+/*    state passing h_in[c+1] = exp(acs_last) h_in[c] + S_c (h_in[0] = h0);  */
+/*    off-diagonal output exp(acs_l) C_l^T h_in[c].                          */
+/* ------------------------------------------------------------------------ */
+int oracle_ssd_chunked(int64_t batch, int64_t seqlen, int64_t nheads, int64_t headdim,
+                       int64_t dstate, int64_t ngroups, int64_t chunk,
+                       const double* x, const double* dt_raw, const double* dt_bias,
+                       const double* A, const double* B, const double* C, const double* D,
+                       const double* init_state, double* y, double* final_state,
+                       int nthreads) {
+    if (check_dims(batch, seqlen, nheads, headdim, dstate, ngroups)) return -1;
+    if (chunk <= 0 || !x || !dt_raw || !A || !B || !C) return -1;
+    const int64_t H = nheads, P = headdim, N = dstate, G = ngroups, L = seqlen, Q = chunk;
+    const int64_t heads_per_group = H / G;
+    const int64_t nchunks = (L + Q - 1) / Q;
+    const int nt = set_threads(nthreads);
+    int64_t pair;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nt)
+    for (pair = 0; pair < batch * H; ++pair) {
+        const int64_t b = pair / H, h = pair % H, g = h / heads_per_group;
+        const double bias = dt_bias ? dt_bias[h] : 0.0;
+        const double d_skip = D ? D[h] : 0.0;
+        double* dt = (double*)malloc(sizeof(double) * (Q + 1));
+        double* acs = (double*)malloc(sizeof(double) * (Q + 1));
+        double* hin = (double*)malloc(sizeof(double) * N * P);   /* state entering the chunk */
+        double* sc = (double*)malloc(sizeof(double) * N * P);    /* chunk's own state S_c */
+        if (init_state) memcpy(hin, init_state + (b * H + h) * N * P, sizeof(double) * N * P);
+        else memset(hin, 0, sizeof(double) * N * P);
+        for (int64_t c = 0; c < nchunks; ++c) {
+            const int64_t t0 = c * Q;
+            const int64_t len = (t0 + Q <= L) ? Q : L - t0;
+            double run = 0.0;
+            for (int64_t l = 0; l < len; ++l) {
+                dt[l] = sp(dt_raw[(b * L + t0 + l) * H + h] + bias);
+                run += dt[l] * A[h];
+                acs[l] = run;
+            }
+            /* outputs of the chunk: intra-chunk block + off-diagonal term + skip */
+            for (int64_t l = 0; y && l < len; ++l) {
+                const double* Cl = C + ((b * L + t0 + l) * G + g) * N;
+                const double* xl = x + ((b * L + t0 + l) * H + h) * P;
+                double* yl = y + ((b * L + t0 + l) * H + h) * P;
+                for (int64_t p = 0; p < P; ++p) yl[p] = d_skip * xl[p];
+                for (int64_t s = 0; s <= l; ++s) {
+                    const double* Bs = B + ((b * L + t0 + s) * G + g) * N;
+                    const double* xs = x + ((b * L + t0 + s) * H + h) * P;
+                    double cb = 0.0;
+                    for (int64_t n = 0; n < N; ++n) cb += Cl[n] * Bs[n];
+                    const double m = cb * exp(acs[l] - acs[s]) * dt[s];
+                    for (int64_t p = 0; p < P; ++p) yl[p] += m * xs[p];
+                }
+                const double e = exp(acs[l]);
+                for (int64_t p = 0; p < P; ++p) {
+                    double acc = 0.0;
+                    for (int64_t n = 0; n < N; ++n) acc += Cl[n] * hin[n * P + p];
+                    yl[p] += e * acc;
+                }
+            }
+            /* chunk state S_c */
+            memset(sc, 0, sizeof(double) * N * P);
+            for (int64_t s = 0; s < len; ++s) {
+                const double w = exp(acs[len - 1] - acs[s]) * dt[s];
+                const double* Bs = B + ((b * L + t0 + s) * G + g) * N;
+                const double* xs = x + ((b * L + t0 + s) * H + h) * P;
+                for (int64_t n = 0; n < N; ++n)
+                    for (int64_t p = 0; p < P; ++p) sc[n * P + p] += w * Bs[n] * xs[p];
+            }
+            /* state passing to the next chunk */
+            const double chunk_decay = exp(acs[len - 1]);
+            for (int64_t k = 0; k < N * P; ++k) hin[k] = chunk_decay * hin[k] + sc[k];
+        }
+        if (final_state) memcpy(final_state + (b * H + h) * N * P, hin, sizeof(double) * N * P);
+        free(dt);
+        free(acs);
+        free(hin);
+        free(sc);
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* 4. One decode step (recurrent mode, one token per sequence), in place on  */
+/*    the state.  If round_state_bf16 != 0 the stored state is rounded to    */
+/*    bf16 after the update (the API's bf16 state storage); y is taken from  */
+/*    the unrounded float64 update.                                          */
+/* ------------------------------------------------------------------------ */
+int oracle_ssd_decode_step(int64_t batch, int64_t nheads, int64_t headdim, int64_t dstate,
+                           int64_t ngroups, double* state, const double* x,
+                           const double* dt_raw, const double* dt_bias, const double* A,
+                           const double* B, const double* C, const double* D, double* y,
+                           int round_state_bf16, int nthreads) {
+    if (check_dims(batch, 1, nheads, headdim, dstate, ngroups)) return -1;
+    if (!state || !x || !dt_raw || !A || !B || !C) return -1;
+    const int64_t H = nheads, P = headdim, N = dstate, G = ngroups;
+    const int64_t heads_per_group = H / G;
+    const int nt = set_threads(nthreads);
+    int64_t pair;
+#pragma omp parallel for schedule(static) num_threads(nt)
+    for (pair = 0; pair < batch * H; ++pair) {
+        const int64_t b = pair / H, h = pair % H, g = h / heads_per_group;
+        const double dt = sp(dt_raw[b * H + h] + (dt_bias ? dt_bias[h] : 0.0));
+        const double decay = exp(dt * A[h]);
+        const double* xt = x + (b * H + h) * P;
+        const double* Bt = B + (b * G + g) * N;
+        const double* Ct = C + (b * G + g) * N;
+        double* st = state + (b * H + h) * N * P;
+        double* yt = y ? y + (b * H + h) * P : NULL;
+        if (yt) for (int64_t p = 0; p < P; ++p) yt[p] = (D ? D[h] : 0.0) * xt[p];
+        for (int64_t n = 0; n < N; ++n) {
+            for (int64_t p = 0; p < P; ++p) {
+                const double v = decay * st[n * P + p] + dt * Bt[n] * xt[p];
+                if (yt) yt[p] += Ct[n] * v;
+                st[n * P + p] = round_state_bf16 ? oracle_round_bf16(v) : v;
+            }
+        }
+    }
+    return 0;
+}

@@ -1,0 +1,83 @@
+"""The oracle's pins catch plausible mistakes.
+
+Each case plants one slip in a temporary copy of the oracle's C source (on the
+CPU, never on a GPU), rebuilds it, and reruns the pins of
+``test_oracle_pins.py`` against the mutant: at least one pin must fail.
+"""
+import importlib.util
+import os
+import sys
+
+import pytest
+
+import tests.test_oracle_pins as pins
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "ssd_oracle.c")
+
+# (name, original text, mutated text); every original must occur in the source
+MUTATIONS = [
+    ("y_before_state_update",   # recurrence: read the state before the token-t update
+     "            /* h_t = decay * h_{t-1} + dt * B_t x_t^T */\n",
+     "            if (y) { double* yt0 = y + ((b * L + t) * H + h) * P; for (int64_t p = 0; p < P; ++p) { double a0 = 0.0; for (int64_t n = 0; n < N; ++n) a0 += Ct[n] * st[n * P + p]; yt0[p] = a0 + d_skip * xt[p]; } }\n            if (0)\n"),
+    ("decay_sign", "const double decay = exp(dt * A[h]);\n            const double* xt = x + ((b * L + t)",
+     "const double decay = exp(-dt * A[h]);\n            const double* xt = x + ((b * L + t)"),
+    ("b_c_swapped_in_recurrence", "const double coef = dt * Bt[n];", "const double coef = dt * Ct[n];"),
+    ("skip_term_dropped", "yt[p] = acc + d_skip * xt[p];", "yt[p] = acc;"),
+    ("group_map_modulo", "for (pair = 0; pair < batch * H; ++pair) {\n        const int64_t b = pair / H, h = pair % H, g = h / heads_per_group;\n        double* st",
+     "for (pair = 0; pair < batch * H; ++pair) {\n        const int64_t b = pair / H, h = pair % H, g = h % G;\n        double* st"),
+    ("euler_dt_missing", "const double coef = dt * Bt[n];", "const double coef = Bt[n];"),
+    ("quadratic_exclusive_cumsum", "            run += dt[t] * A[h];\n            cs[t] = run;",
+     "            cs[t] = run;\n            run += dt[t] * A[h];"),
+    ("chunked_offdiag_dropped", "yl[p] += e * acc;", "yl[p] += 0.0 * e * acc;"),
+    ("chunked_state_decay_wrong", "const double w = exp(acs[len - 1] - acs[s]) * dt[s];",
+     "const double w = exp(acs[len - 1]) * dt[s];"),
+    ("softplus_bias_dropped", "const double dt = sp(dt_raw[(b * L + t) * H + h] + bias);",
+     "const double dt = sp(dt_raw[(b * L + t) * H + h]);"),
+    ("decode_state_not_decayed", "const double v = decay * st[n * P + p] + dt * Bt[n] * xt[p];",
+     "const double v = st[n * P + p] + dt * Bt[n] * xt[p];"),
+]
+
+PIN_TESTS = [
+    lambda: pins.test_recurrent_equals_quadratic(2, True),
+    lambda: pins.test_recurrent_equals_chunked(50, 16),
+    pins.test_a_zero_is_causal_linear_attention,
+    lambda: pins.test_dt_to_zero("recurrent"),
+    lambda: pins.test_scalar_geometric_series("recurrent"),
+    lambda: pins.test_scalar_geometric_series("quadratic"),
+    lambda: pins.test_scalar_geometric_series("chunked"),
+    lambda: pins.test_impulse_response_varying_dt("recurrent"),
+    lambda: pins.test_impulse_response_varying_dt("quadratic"),
+    lambda: pins.test_impulse_response_varying_dt("chunked"),
+    pins.test_group_mapping,
+    pins.test_decode_steps_equal_prefill,
+]
+
+
+def _load_mutant(tmp_path, name, old, new):
+    src = open(SRC).read()
+    assert src.count(old) >= 1, f"mutation {name}: anchor text not found"
+    pkg = tmp_path / f"oracle_{name}"
+    pkg.mkdir()
+    init = open(os.path.join(ROOT, "oracle", "__init__.py")).read()
+    (pkg / "__init__.py").write_text(init.replace('"-Werror",', ""))  # mutants may leave unused names
+    (pkg / "ssd_oracle.c").write_text(src.replace(old, new, 1))
+    spec = importlib.util.spec_from_file_location(f"oracle_{name}", pkg / "__init__.py",
+                                                  submodule_search_locations=[str(pkg)])
+    mod = importlib.util.module_from_spec(spec)
+    sys.modules[spec.name] = mod
+    spec.loader.exec_module(mod)
+    return mod
+
+
+@pytest.mark.parametrize("name,old,new", MUTATIONS, ids=[m[0] for m in MUTATIONS])
+def test_pins_catch_mutation(tmp_path, monkeypatch, name, old, new):
+    mutant = _load_mutant(tmp_path, name, old, new)
+    monkeypatch.setattr(pins, "oracle", mutant)
+    caught = 0
+    for t in PIN_TESTS:
+        try:
+            t()
+        except (AssertionError, ValueError):
+            caught += 1
+    assert caught > 0, f"no pin failed for mutation {name}"
