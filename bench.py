@@ -1,0 +1,378 @@
+#!/usr/bin/env python
+"""Benchmark of libssd (Mamba-2 SSD layer core) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one ssd_chunk_scan_fwd over the Mamba-2 1.3B-shaped layer (batch 4,
+seqlen 2048, 64 heads x P=64, N=128, 1 group, chunk 256; bf16 inputs, fp32
+accumulation, y and final_state in fp32) on synthetic seeded inputs resident in
+HBM.  The same run also times K decode steps (ssd_state_update, batch 256, 128
+heads, P=64, N=128, 8 groups, fp32 state) and reports them under "decode".
+
+Timing: W untimed warm-up steps, then exactly K steps between a barrier +
+cudaDeviceSynchronize on both sides, CUDA events on the launching stream, max
+over ranks.  Three input sets (x 67 MB each) rotate so that consecutive steps
+never find their inputs in the 126 MB L2.  Multi-GPU: one process per GPU
+(torchrun), each rank runs its own batch shard (weak scaling, no collective on
+the data path); value = tokens of all ranks / max time over ranks.
+
+--impl reference times the float64 CPU oracle (the reference arm of this
+build) on a bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "SSD prefill tokens/s + TFLOP/s; decode tokens/s + state GB/s (1 B200)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ counts
+def prefill_flops(b, L, H, P, N, G, Q):
+    """Full-block algorithmic flops of the chunked contraction:
+    b * nchunks * [G * 2 Q^2 N  (C B^T per group)  +  H * (2 Q^2 P + 4 Q N P)]."""
+    nc = -(-L // Q)
+    return b * nc * (G * 2 * Q * Q * N + H * (2 * Q * Q * P + 4 * Q * N * P))
+
+
+def prefill_bytes(b, L, H, P, N, G, io_bytes, y_bytes, state_bytes, with_init=False):
+    """Algorithmic bytes: x + y + B + C + dt_raw + final_state (+ init_state)."""
+    tok = b * L
+    n = tok * H * P * io_bytes + tok * H * P * y_bytes + 2 * tok * G * N * io_bytes + tok * H * io_bytes
+    n += b * H * N * P * state_bytes * (2 if with_init else 1)
+    return n
+
+
+def decode_bytes(b, H, P, N, G, io_bytes, y_bytes, state_bytes):
+    """State read + write, plus x, y, B, C, dt_raw."""
+    return 2 * b * H * N * P * state_bytes + b * H * P * (io_bytes + y_bytes) + 2 * b * G * N * io_bytes + b * H * io_bytes
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """Samples SM clock, power and clock-event reasons with NVML every ~2 ms in a thread."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, device_index_uuid):
+        self.samples = []
+        self.ok = False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(device_index_uuid)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # NVML unavailable: report no clocks rather than guess
+            self.err = repr(e)
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                pw = nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0
+                self.samples.append((mhz, rs, pw))
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": getattr(self, "max_mhz", None), "reasons": [],
+                    "samples": 0, "note": getattr(self, "err", "no samples")}
+        mhz = [s[0] for s in self.samples]
+        bits = 0
+        for s in self.samples:
+            bits |= s[1]
+        reasons = [name for bit, name in self.REASONS.items() if bits & bit and name != "gpu_idle"]
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(self.samples), "power_w_max": max(s[2] for s in self.samples)}
+
+
+# ------------------------------------------------------------------ reference arm
+def run_reference(args, rank):
+    """The float64 CPU oracle on a bounded sample of the prefill workload."""
+    if rank != 0:
+        return
+    import numpy as np
+
+    import oracle
+    from mamba_ssd_scan_chunked_b200 import inputs as I
+    s = I.MAMBA2_1P3B
+    heads = list(range(4))          # per step: batch 0, 4 of 64 heads, all 2048 tokens
+    inp = s.inputs(batches=[0])
+    f = {k: I.to_f64(v) for k, v in inp.items()}
+    sl = dict(x=f["x"][:, :, heads], dt_raw=f["dt_raw"][:, :, heads], dt_bias=f["dt_bias"][heads],
+              A=f["A"][heads], B=f["B"], C=f["C"], D=f["D"][heads])
+    for _ in range(args.warmup):
+        oracle.recurrent(**sl)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.recurrent(**sl)
+    dt = time.perf_counter() - t0
+    tok_equiv = s.seqlen * len(heads) / s.nheads        # full-layer tokens per step
+    value = tok_equiv * args.steps / dt
+    cores = oracle.num_threads()
+    sample = f"batch 0, heads 0-3 of 64, seqlen 2048 (= {tok_equiv:.0f} full-layer tokens) per step"
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": s.name, "global_batch": s.batch, "seq_len": s.seqlen, "parallelism": "host cores"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ our arm
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+
+    import numpy as np
+    import torch
+
+    from mamba_ssd_scan_chunked_b200 import dist
+    from mamba_ssd_scan_chunked_b200 import inputs as I
+    from mamba_ssd_scan_chunked_b200 import ssd
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    pg = dist.init(world, rank, local_rank)
+
+    peaks, peak_kind = load_peaks()
+    s = I.MAMBA2_1P3B
+    my_batches = dist.shard(s.batch * world, rank, world)   # weak scaling: each rank its own 4 sequences
+
+    def to_dev(a):
+        if a.dtype == np.uint16:
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+    # three rotating input sets (different sequences) so steps do not hit L2-resident inputs
+    NSETS = 3
+    sets = []
+    for k in range(NSETS):
+        batches = [b + k * s.batch * world for b in my_batches]
+        inp = I.prefill_inputs(s.batch, s.seqlen, s.nheads, s.headdim, s.dstate, s.ngroups, s.seed, s.dtype,
+                               batches=batches)
+        sets.append({kk: to_dev(v) for kk, v in inp.items()})
+    y = torch.empty((s.batch, s.seqlen, s.nheads, s.headdim), dtype=torch.float32, device=dev)
+    fs = torch.empty((s.batch, s.nheads, s.dstate, s.headdim), dtype=torch.float32, device=dev)
+    desc = ssd.prefill_desc(sets[0]["x"], sets[0]["B"], s.chunk, torch.float32, torch.float32)
+    path = ssd.ssd_chunk_scan_path(desc)
+    ws = torch.empty(ssd.ssd_chunk_scan_workspace_size(desc), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    launches_per_prefill = 2          # decay-cumsum kernel + chunk kernel
+
+    def prefill(k):
+        d = sets[k % NSETS]
+        st = ssd.ssd_chunk_scan_fwd(desc, d["x"].data_ptr(), d["dt_raw"].data_ptr(), d["dt_bias"].data_ptr(),
+                                    d["A"].data_ptr(), d["B"].data_ptr(), d["C"].data_ptr(), d["D"].data_ptr(), 0,
+                                    y.data_ptr(), fs.data_ptr(), ws.data_ptr(), ws.numel(), stream.cuda_stream)
+        if st:
+            raise ssd.SsdError(st, "ssd_chunk_scan_fwd")
+
+    uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    for k in range(args.warmup):
+        prefill(k)
+    dist.barrier(pg)
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    with ClockSampler(uuid) as clk:
+        ev[0].record(stream)
+        for k in range(args.steps):
+            prefill(k)
+        ev[1].record(stream)
+        torch.cuda.synchronize()
+    dist.barrier(pg)
+    ms_local = ev[0].elapsed_time(ev[1]) / args.steps
+    ms = dist.max_over_ranks(pg, ms_local)
+    st_err, detail = ssd.ssd_get_device_error(stream.cuda_stream)
+    if st_err:
+        raise RuntimeError(f"device error word {detail:#x} after the timed prefill")
+
+    tokens_rank = s.batch * s.seqlen
+    value = tokens_rank * world / (ms * 1e-3)
+    flops = prefill_flops(s.batch, s.seqlen, s.nheads, s.headdim, s.dstate, s.ngroups, s.chunk)
+    nbytes = prefill_bytes(s.batch, s.seqlen, s.nheads, s.headdim, s.dstate, s.ngroups, 2, 4, 4)
+    tflops = flops / (ms * 1e-3) / 1e12
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    t_tc = flops / (peaks["bf16_tflops"] * 1e12)
+    bound = "hbm" if t_hbm >= t_tc else "tensor"
+    if bound == "hbm":
+        roofline = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": gbs / peaks["hbm_gbs"]}
+    else:
+        roofline = {"bound": "tensor", "achieved": tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                    "frac": tflops / peaks["bf16_tflops"]}
+    roofline.update({"traffic": None, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json)" if peak_kind == "measured"
+                     else "fallback", "kernel": "ssd_chunk_scan_fwd (decay cumsum + tcgen05 chunk kernel)",
+                     "algorithmic_bytes_per_launch": nbytes, "algorithmic_flops_per_launch": flops,
+                     "roofline_time_us": 1e6 * max(t_hbm, t_tc)})
+
+    # ---------------- decode (batch 256 x 128 heads, fp32 state), timed the same way
+    dcfg = I.DECODE_B256
+    dec_batches = dist.shard(dcfg.batch * world, rank, world)
+    state = torch.from_numpy(np.stack([I.draw_decode_state(b, dcfg.nheads, dcfg.headdim, dcfg.dstate, dcfg.seed,
+                                                           dcfg.state_dtype) for b in dec_batches])).to(dev)
+    prm = {k: to_dev(v) for k, v in I.draw_head_params(dcfg.nheads, dcfg.seed).items()}
+    nsteps_in = 8
+    dsteps = []
+    for t in range(nsteps_in):
+        st = I.draw_decode_step(t, dcfg.batch, dcfg.nheads, dcfg.headdim, dcfg.dstate, dcfg.ngroups, dcfg.seed,
+                                dcfg.io_dtype)
+        dsteps.append({k: to_dev(v) for k, v in st.items()})
+    yd = torch.empty((dcfg.batch, dcfg.nheads, dcfg.headdim), dtype=torch.float32, device=dev)
+    ddesc = ssd.DecodeDesc(dcfg.batch, dcfg.nheads, dcfg.headdim, dcfg.dstate, dcfg.ngroups, ssd.SSD_BF16,
+                           ssd.SSD_F32, ssd.SSD_F32)
+
+    def decode(t):
+        d = dsteps[t % nsteps_in]
+        st = ssd.ssd_state_update(ddesc, state.data_ptr(), d["x"].data_ptr(), d["dt_raw"].data_ptr(),
+                                  prm["dt_bias"].data_ptr(), prm["A"].data_ptr(), d["B"].data_ptr(),
+                                  d["C"].data_ptr(), prm["D"].data_ptr(), yd.data_ptr(), stream.cuda_stream)
+        if st:
+            raise ssd.SsdError(st, "ssd_state_update")
+
+    for t in range(args.warmup):
+        decode(t)
+    dist.barrier(pg)
+    torch.cuda.synchronize()
+    with ClockSampler(uuid) as dclk:
+        ev[0].record(stream)
+        for t in range(args.steps):
+            decode(t)
+        ev[1].record(stream)
+        torch.cuda.synchronize()
+    dist.barrier(pg)
+    dms = dist.max_over_ranks(pg, ev[0].elapsed_time(ev[1]) / args.steps)
+    dbytes = decode_bytes(dcfg.batch, dcfg.nheads, dcfg.headdim, dcfg.dstate, dcfg.ngroups, 2, 4, 4)
+    dgbs = dbytes / (dms * 1e-3) / 1e9
+    decode_line = {"workload": dcfg.name, "tokens_per_s": dcfg.batch * world / (dms * 1e-3),
+                   "ms_per_step": dms, "state_gbs": 2 * dcfg.batch * dcfg.nheads * dcfg.dstate * dcfg.headdim * 4
+                   / (dms * 1e-3) / 1e9,
+                   "roofline": {"bound": "hbm", "achieved": dgbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                "frac": dgbs / peaks["hbm_gbs"], "traffic": None,
+                                "algorithmic_bytes_per_launch": dbytes, "kernel": "state_update_kernel"},
+                   "clocks": dclk.summary()}
+
+    # ---------------- end to end through the public API with host buffers
+    e2e = None
+    if rank == 0 or world > 1:
+        host = {k: v.cpu().pin_memory() for k, v in sets[0].items() if k in ("x", "dt_raw", "B", "C")}
+        y_h = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+        fs_h = torch.empty(fs.shape, dtype=fs.dtype).pin_memory()
+        dbuf = {k: torch.empty_like(sets[0][k]) for k in host}
+        h2d = sum(v.numel() * v.element_size() for v in host.values())
+        d2h = y_h.numel() * 4 + fs_h.numel() * 4
+        e2e_steps = max(3, min(args.steps, 10))
+
+        def e2e_step():
+            for k, v in host.items():
+                dbuf[k].copy_(v, non_blocking=True)
+            st = ssd.ssd_chunk_scan_fwd(desc, dbuf["x"].data_ptr(), dbuf["dt_raw"].data_ptr(),
+                                        sets[0]["dt_bias"].data_ptr(), sets[0]["A"].data_ptr(),
+                                        dbuf["B"].data_ptr(), dbuf["C"].data_ptr(), sets[0]["D"].data_ptr(), 0,
+                                        y.data_ptr(), fs.data_ptr(), ws.data_ptr(), ws.numel(), stream.cuda_stream)
+            if st:
+                raise ssd.SsdError(st, "ssd_chunk_scan_fwd")
+            y_h.copy_(y, non_blocking=True)
+            fs_h.copy_(fs, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        ev[0].record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        ev[1].record(stream)
+        torch.cuda.synchronize()
+        ems = dist.max_over_ranks(pg, ev[0].elapsed_time(ev[1]) / e2e_steps)
+        e2e = {"value": tokens_rank * world / (ems * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": ems, "steps": e2e_steps}
+
+    # ---------------- CPU baseline (oracle) on a bounded sample, rank 0 at N=1 only
+    cpu_baseline = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        heads = list(range(16))
+        inp = s.inputs(batches=[0])
+        f = {k: I.to_f64(v) for k, v in inp.items()}
+        t0 = time.perf_counter()
+        oracle.recurrent(f["x"][:, :, heads], f["dt_raw"][:, :, heads], f["dt_bias"][heads], f["A"][heads], f["B"],
+                         f["C"], f["D"][heads])
+        cdt = time.perf_counter() - t0
+        tok_equiv = s.seqlen * len(heads) / s.nheads
+        cpu_baseline = {"value": tok_equiv / cdt, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+                        "sample": f"batch 0, heads 0-15 of 64, seqlen 2048 (= {tok_equiv:.0f} full-layer tokens), "
+                                  f"{cdt:.1f} s"}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": s.name, "global_batch": s.batch * world, "seq_len": s.seqlen,
+                           "nheads": s.nheads, "headdim": s.headdim, "dstate": s.dstate, "ngroups": s.ngroups,
+                           "chunk": s.chunk, "inputs": "bf16", "accumulate": "fp32", "y": "fp32",
+                           "final_state": "fp32", "parallelism": f"dp{world}" if world > 1 else "single",
+                           "l2": "3 rotating input sets (x 67 MB each); inputs larger than L2 across steps",
+                           "kernel_path": "tensor cores" if path == 0 else "cuda cores"},
+                "tflops": tflops, "gbs": gbs, "roofline": roofline, "decode": decode_line,
+                "cpu_baseline": cpu_baseline, "e2e": e2e,
+                "gpu_launches": launches_per_prefill * args.steps + args.steps,
+                "clocks": clk.summary()}
+        print(json.dumps(line), flush=True)
+    dist.finish(pg)
+
+
+if __name__ == "__main__":
+    main()

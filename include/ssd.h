@@ -1,0 +1,199 @@
+/*
+ * libssd -- Mamba-2 SSD (structured state-space duality) layer core on one
+ * NVIDIA B200 (sm_100a).  C ABI: plain pointers, sizes and status codes; no
+ * C++ or framework types cross this boundary.
+ *
+ * The operation (per batch element b and head h; the state is N x P):
+ *
+ *   dt_t = softplus(dt_raw[t,h] + dt_bias[h])
+ *   h_t  = exp(dt_t * A[h]) * h_{t-1} + dt_t * B_t x_t^T
+ *   y_t  = C_t^T h_t + D[h] * x_t
+ *
+ * Where it is defined (page titles and sections; the pages print no formula,
+ * these are the statements the formula above follows):
+ *  - transition = a scalar times the identity: "Mamba3" (Telegram post,
+ *    ai_machinelearning_big_data), first paragraph; "Mamba-3 : SSM optimise
+ *    inference", section "Du training-first a l'inference-first".
+ *  - ZOH on the state, Euler on the input: "Mamba3", section "New
+ *    discretisation scheme" (Mamba-1 and Mamba-2 mix ZOH and Euler).
+ *  - two paths: the blocked (chunked) contraction of the semiseparable matrix
+ *    for a whole sequence, and the O(1) recurrent step at generation time:
+ *    "Mamba-2 vs Transformers / SSD", sections "Mamba-2 and the SSD paper:
+ *    what changed in practice" and "How to decide..." (table: streaming
+ *    inference, O(1) recurrent step).
+ *
+ * Readings where the pages are silent:
+ *  - y_t reads the state after the token-t update.
+ *  - head h uses group g = h / (nheads / ngroups) of B and C.
+ *  - dt_bias, A and D are one fp32 scalar per head; a NULL dt_bias or D means 0.
+ *  - no clamp and no threshold on dt (softplus is exact up to fp32 rounding).
+ *
+ * Layouts (row-major, last index fastest, every tensor densely packed):
+ *   prefill: x, y [batch][seqlen][nheads][headdim]; dt_raw [batch][seqlen][nheads];
+ *            B, C [batch][seqlen][ngroups][dstate];
+ *            init_state, final_state [batch][nheads][dstate][headdim].
+ *   decode:  x, y [batch][nheads][headdim]; dt_raw [batch][nheads];
+ *            B, C [batch][ngroups][dstate]; state [batch][nheads][dstate][headdim].
+ *
+ * Conventions shared by every call:
+ *  - Ownership: the caller owns every pointer, all device memory and the
+ *    stream.  The library allocates no device memory; the prefill takes a
+ *    caller-owned workspace of at least ssd_chunk_scan_workspace_size() bytes.
+ *  - All tensor pointers are device pointers.  dt_bias, A and D are device
+ *    pointers too.  `stream` is a cudaStream_t (NULL = legacy default stream).
+ *  - Asynchrony: the compute calls only enqueue work on `stream` and never
+ *    synchronise; SSD_OK means "enqueued".  Results are ready when the stream
+ *    is.
+ *  - Validation happens on the host before anything is enqueued; on any error
+ *    nothing is launched and no memory is touched.
+ *  - Alignment: every tensor base pointer must be 16-byte aligned
+ *    (SSD_ERR_ALIGNMENT otherwise).
+ *  - Reentrancy: the library keeps no per-call host state; concurrent calls on
+ *    different streams must use different workspaces.
+ */
+#ifndef LIBSSD_SSD_H
+#define LIBSSD_SSD_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SSD_OK = 0,
+    SSD_ERR_INVALID_ARG = 1,     /* NULL required pointer, bad dimension, bad dtype, aliasing */
+    SSD_ERR_UNSUPPORTED = 2,     /* valid request this build does not implement */
+    SSD_ERR_ALIGNMENT = 3,       /* a tensor base pointer is not 16-byte aligned */
+    SSD_ERR_WORKSPACE = 4,       /* workspace NULL or smaller than required */
+    SSD_ERR_CUDA = 5,            /* a CUDA runtime/driver call failed (launch, attribute, ...) */
+    SSD_ERR_DEVICE_TIMEOUT = 6   /* a bounded device-side wait gave up (see ssd_get_device_error) */
+} ssd_status_t;
+
+typedef enum {
+    SSD_F32 = 0,   /* IEEE binary32 */
+    SSD_BF16 = 1   /* bfloat16 (stored as 16-bit patterns; results rounded to nearest even) */
+} ssd_dtype_t;
+
+/* Prefill problem description.  Enum fields are int32_t holding ssd_dtype_t. */
+typedef struct {
+    int64_t batch;      /* >= 0; 0 is a no-op */
+    int64_t seqlen;     /* >= 0; 0 writes final_state = init_state (or zeros) */
+    int64_t nheads;     /* H >= 1 */
+    int64_t headdim;    /* P, multiple of 8, <= 256 */
+    int64_t dstate;     /* N, multiple of 8, <= 256 */
+    int64_t ngroups;    /* G >= 1, nheads % ngroups == 0 */
+    int64_t chunk;      /* Q: power of two in [16, 256]; seqlen need not be a multiple */
+    int32_t io_dtype;   /* dtype of x, dt_raw, B, C */
+    int32_t y_dtype;    /* dtype of y */
+    int32_t state_dtype;/* dtype of init_state and final_state */
+} ssd_prefill_desc_t;
+
+/* Decode (single-token state update) problem description. */
+typedef struct {
+    int64_t batch;      /* >= 0; 0 is a no-op */
+    int64_t nheads;
+    int64_t headdim;    /* P, multiple of 8, <= 256 */
+    int64_t dstate;     /* N, multiple of 8, <= 256 */
+    int64_t ngroups;
+    int32_t io_dtype;   /* dtype of x, dt_raw, B, C */
+    int32_t y_dtype;    /* dtype of y */
+    int32_t state_dtype;/* dtype of the in-place state */
+} ssd_decode_desc_t;
+
+/* Library version as MAJOR * 10000 + MINOR * 100 + PATCH. */
+int ssd_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* ssd_status_string(ssd_status_t status);
+
+/*
+ * Bytes of device workspace ssd_chunk_scan_fwd needs for `desc` (written to
+ * *bytes).  Pure host function: touches no device.  The workspace holds the
+ * per-token dt and chunk-local decay cumsum (fp32), the in-flight fp32 chunk
+ * states of the inter-chunk state-passing scan, and its progress flags.
+ * Errors: SSD_ERR_INVALID_ARG / SSD_ERR_UNSUPPORTED as for ssd_chunk_scan_fwd.
+ */
+ssd_status_t ssd_chunk_scan_workspace_size(const ssd_prefill_desc_t* desc, size_t* bytes);
+
+/*
+ * Which kernel path ssd_chunk_scan_fwd takes for `desc` (written to *path):
+ *   0 = tensor-core path (bf16 inputs; tcgen05 MMAs with TMEM accumulators fed
+ *       by TMA; fp32 accumulation and fp32 state passing),
+ *   1 = CUDA-core fp32 path (fp32 inputs, or shapes the tensor-core path does
+ *       not cover).
+ * Pure host function.
+ */
+ssd_status_t ssd_chunk_scan_path(const ssd_prefill_desc_t* desc, int32_t* path);
+
+/*
+ * Chunked prefill scan over whole sequences: the semiseparable matrix is
+ * contracted chunk by chunk ("Mamba-2 vs Transformers / SSD", section "Mamba-2
+ * and the SSD paper: what changed in practice": chunks processed in parallel,
+ * then the per-chunk SSM states recombined).  Per chunk of Q tokens it
+ * computes the chunk-local decay cumsum, the intra-chunk block
+ * (C B^T o L)(dt x), the chunk state B^T(decay dt x) and the off-diagonal
+ * term exp(cumsum) C h_in; an fp32 scan over chunks carries the state.
+ *
+ *  (x, dt_raw, B, C and y may be NULL when batch == 0 or seqlen == 0)
+ *  x           [b][L][H][P]   io_dtype   required
+ *  dt_raw      [b][L][H]      io_dtype   required
+ *  dt_bias     [H]            fp32       nullable (= 0)
+ *  A           [H]            fp32       required (taken as given; A <= 0 is the intended use)
+ *  B, C        [b][L][G][N]   io_dtype   required
+ *  D           [H]            fp32       nullable (= 0)
+ *  init_state  [b][H][N][P]   state_dtype nullable (= zero state, not read)
+ *  y           [b][L][H][P]   y_dtype    required, written; must not overlap x
+ *  final_state [b][H][N][P]   state_dtype nullable (not written), else written
+ *  workspace   >= ssd_chunk_scan_workspace_size bytes, 256-byte aligned; its
+ *              contents on entry are irrelevant; clobbered
+ * Errors: SSD_ERR_INVALID_ARG, SSD_ERR_UNSUPPORTED, SSD_ERR_ALIGNMENT,
+ *         SSD_ERR_WORKSPACE (nothing launched), SSD_ERR_CUDA (launch failed;
+ *         outputs undefined).
+ */
+ssd_status_t ssd_chunk_scan_fwd(const ssd_prefill_desc_t* desc,
+                                const void* x, const void* dt_raw, const float* dt_bias,
+                                const float* A, const void* B, const void* C, const float* D,
+                                const void* init_state, void* y, void* final_state,
+                                void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Single-token decode step, in place on the state ("Mamba-2 vs Transformers /
+ * SSD", section "How to decide...": O(1) recurrent step; "Mamba3", section on
+ * Mamba-2: decoding moves the state between memory levels rather than
+ * computing -- the step is one streaming read-modify-write of the state):
+ *
+ *   state[b,h] <- exp(dt A) state[b,h] + dt B x^T;  y = C^T state[b,h] + D x
+ *
+ *  state  [b][H][N][P]  state_dtype  required, read and written in place
+ *                                     (bf16 state is rounded to nearest even)
+ *  x      [b][H][P]     io_dtype     required
+ *  dt_raw [b][H]        io_dtype     required
+ *  dt_bias, A, D [H]    fp32         dt_bias, D nullable
+ *  B, C   [b][G][N]     io_dtype     required
+ *  y      [b][H][P]     y_dtype      required; must not overlap state or x
+ * Errors: as ssd_chunk_scan_fwd (no workspace).
+ */
+ssd_status_t ssd_state_update(const ssd_decode_desc_t* desc, void* state, const void* x,
+                              const void* dt_raw, const float* dt_bias, const float* A,
+                              const void* B, const void* C, const float* D, void* y,
+                              void* stream);
+
+/*
+ * Synchronises `stream`, then reports (and clears) the device-side error word
+ * of the current device.  Kernels never trap: a bounded wait that gives up
+ * (the inter-chunk state hand-off of the prefill waits for the previous
+ * chunk's state with an iteration limit) records it there and returns.
+ * Returns SSD_OK, SSD_ERR_DEVICE_TIMEOUT, or SSD_ERR_CUDA if synchronisation
+ * itself failed.  If `detail` is not NULL it receives the raw error bits.
+ * The word is shared by all streams of the device: call it when no other
+ * libssd work is in flight.
+ */
+ssd_status_t ssd_get_device_error(void* stream, uint32_t* detail);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LIBSSD_SSD_H */

@@ -1,0 +1,230 @@
+// libssd C ABI: argument validation, workspace layout and dispatch.
+// Declarations and the contract of every entry point are in include/ssd.h.
+#include <atomic>
+#include <mutex>
+
+#include "../../include/ssd.h"
+#include "ssd_common.cuh"
+#include "ssd_internal.h"
+
+namespace ssd {
+
+// Device-side error word (bits kErr*), one per device that loads the library.
+__device__ unsigned g_device_error;
+
+static std::mutex g_err_mutex;
+static unsigned* g_err_ptr[64];
+
+static cudaError_t device_error_ptr(unsigned** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lk(g_err_mutex);
+    if (!g_err_ptr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_device_error);
+        if (e != cudaSuccess) return e;
+        g_err_ptr[dev] = (unsigned*)p;
+    }
+    *out = g_err_ptr[dev];
+    return cudaSuccess;
+}
+
+static inline size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+static bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+    if (!a || !b || na == 0 || nb == 0) return false;
+    const uintptr_t a0 = (uintptr_t)a, b0 = (uintptr_t)b;
+    return a0 < b0 + nb && b0 < a0 + na;
+}
+
+static bool valid_dtype(int32_t d) { return d == SSD_F32 || d == SSD_BF16; }
+static size_t dsize(int32_t d) { return d == SSD_BF16 ? 2 : 4; }
+
+static bool is_pow2(int64_t v) { return v > 0 && (v & (v - 1)) == 0; }
+
+static ssd_status_t check_prefill_desc(const ssd_prefill_desc_t* d) {
+    if (!d) return SSD_ERR_INVALID_ARG;
+    if (d->batch < 0 || d->seqlen < 0 || d->nheads < 1 || d->headdim < 1 || d->dstate < 1 ||
+        d->ngroups < 1 || d->chunk < 1)
+        return SSD_ERR_INVALID_ARG;
+    if (d->nheads % d->ngroups != 0) return SSD_ERR_INVALID_ARG;
+    if (!valid_dtype(d->io_dtype) || !valid_dtype(d->y_dtype) || !valid_dtype(d->state_dtype))
+        return SSD_ERR_INVALID_ARG;
+    if (!is_pow2(d->chunk) || d->chunk < 16 || d->chunk > 256) return SSD_ERR_UNSUPPORTED;
+    if (d->headdim % 8 != 0 || d->dstate % 8 != 0 || d->headdim > 256 || d->dstate > 256)
+        return SSD_ERR_UNSUPPORTED;
+    if (d->nheads > (1 << 20) || d->batch > (1 << 24) || d->seqlen > ((int64_t)1 << 31))
+        return SSD_ERR_UNSUPPORTED;
+    return SSD_OK;
+}
+
+static PrefillLayout prefill_layout(const ssd_prefill_desc_t* d, bool tc) {
+    PrefillLayout lay{};
+    const int64_t BH = d->batch * d->nheads;
+    lay.nchunks = (d->seqlen + d->chunk - 1) / d->chunk;
+    lay.Lpad = lay.nchunks * d->chunk;
+    size_t off = 0;
+    lay.off_dt = off;
+    off = align256(off + sizeof(float) * (size_t)BH * lay.Lpad);
+    lay.off_acs = off;
+    off = align256(off + sizeof(float) * (size_t)BH * lay.Lpad);
+    lay.off_states = off;
+    const size_t state_elems = (size_t)d->dstate * d->headdim;
+    off = align256(off + sizeof(float) * state_elems * (size_t)BH * (tc ? 1 : lay.nchunks));
+    lay.off_flags = off;
+    off = align256(off + sizeof(int) * ((size_t)BH + 64));
+    lay.total = off;
+    return lay;
+}
+
+static int prefill_path(const ssd_prefill_desc_t* d) {
+    return tc_path_supports(d->headdim, d->dstate, d->chunk, d->io_dtype == SSD_BF16) ? 0 : 1;
+}
+
+// copies (or zero-fills) init_state into final_state for seqlen == 0
+template <typename S, typename D>
+__global__ void copy_state_kernel(const S* __restrict__ src, D* __restrict__ dst, int64_t n) {
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+        dst[i] = from_f32<D>(src ? to_f32(src[i]) : 0.f);
+}
+
+}  // namespace ssd
+
+using namespace ssd;
+
+extern "C" {
+
+int ssd_version(void) { return 100; }
+
+const char* ssd_status_string(ssd_status_t s) {
+    switch (s) {
+        case SSD_OK: return "SSD_OK";
+        case SSD_ERR_INVALID_ARG: return "SSD_ERR_INVALID_ARG: invalid argument";
+        case SSD_ERR_UNSUPPORTED: return "SSD_ERR_UNSUPPORTED: shape or dtype not implemented";
+        case SSD_ERR_ALIGNMENT: return "SSD_ERR_ALIGNMENT: tensor base not 16-byte aligned";
+        case SSD_ERR_WORKSPACE: return "SSD_ERR_WORKSPACE: workspace missing or too small";
+        case SSD_ERR_CUDA: return "SSD_ERR_CUDA: CUDA call failed";
+        case SSD_ERR_DEVICE_TIMEOUT: return "SSD_ERR_DEVICE_TIMEOUT: a device-side wait gave up";
+    }
+    return "SSD_ERR_UNKNOWN";
+}
+
+ssd_status_t ssd_chunk_scan_workspace_size(const ssd_prefill_desc_t* desc, size_t* bytes) {
+    if (!bytes) return SSD_ERR_INVALID_ARG;
+    const ssd_status_t st = check_prefill_desc(desc);
+    if (st != SSD_OK) return st;
+    *bytes = prefill_layout(desc, prefill_path(desc) == 0).total;
+    return SSD_OK;
+}
+
+ssd_status_t ssd_chunk_scan_path(const ssd_prefill_desc_t* desc, int32_t* path) {
+    if (!path) return SSD_ERR_INVALID_ARG;
+    const ssd_status_t st = check_prefill_desc(desc);
+    if (st != SSD_OK) return st;
+    *path = prefill_path(desc);
+    return SSD_OK;
+}
+
+ssd_status_t ssd_chunk_scan_fwd(const ssd_prefill_desc_t* d, const void* x, const void* dt_raw,
+                                const float* dt_bias, const float* A, const void* B, const void* C,
+                                const float* D, const void* init_state, void* y, void* final_state,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+    ssd_status_t st = check_prefill_desc(d);
+    if (st != SSD_OK) return st;
+    const bool empty = d->batch == 0 || d->seqlen == 0;   // token tensors may then be NULL
+    if (!A || (!empty && (!x || !dt_raw || !B || !C || !y))) return SSD_ERR_INVALID_ARG;
+    const void* ptrs[] = {x, dt_raw, dt_bias, A, B, C, D, init_state, y, final_state};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return SSD_ERR_ALIGNMENT;
+    const size_t tok = (size_t)d->batch * d->seqlen;
+    const size_t x_bytes = tok * d->nheads * d->headdim * dsize(d->io_dtype);
+    const size_t y_bytes = tok * d->nheads * d->headdim * dsize(d->y_dtype);
+    const size_t s_bytes = (size_t)d->batch * d->nheads * d->dstate * d->headdim * dsize(d->state_dtype);
+    const size_t bc_bytes = tok * d->ngroups * d->dstate * dsize(d->io_dtype);
+    if (overlaps(y, y_bytes, x, x_bytes) || overlaps(y, y_bytes, B, bc_bytes) ||
+        overlaps(y, y_bytes, C, bc_bytes) || overlaps(final_state, s_bytes, y, y_bytes) ||
+        overlaps(final_state, s_bytes, x, x_bytes))
+        return SSD_ERR_INVALID_ARG;
+    const bool tc = prefill_path(d) == 0;
+    const PrefillLayout lay = prefill_layout(d, tc);
+    if (d->batch == 0) return SSD_OK;
+    if (d->seqlen > 0 && (!workspace || workspace_bytes < lay.total)) return SSD_ERR_WORKSPACE;
+    if (workspace && ((uintptr_t)workspace & 255u)) return SSD_ERR_ALIGNMENT;
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e;
+    if (d->seqlen == 0) {
+        if (!final_state) return SSD_OK;
+        const int64_t n = (int64_t)d->batch * d->nheads * d->dstate * d->headdim;
+        const unsigned grid = (unsigned)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
+        const bool sb = d->state_dtype == SSD_BF16;
+        if (sb) copy_state_kernel<bf16, bf16><<<grid, 256, 0, s>>>((const bf16*)init_state, (bf16*)final_state, n);
+        else copy_state_kernel<float, float><<<grid, 256, 0, s>>>((const float*)init_state, (float*)final_state, n);
+        return cudaGetLastError() == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
+    }
+    PrefillArgs a{};
+    a.batch = d->batch; a.L = d->seqlen; a.H = d->nheads; a.P = d->headdim; a.N = d->dstate;
+    a.G = d->ngroups; a.Q = d->chunk;
+    a.io_bf16 = d->io_dtype == SSD_BF16; a.y_bf16 = d->y_dtype == SSD_BF16;
+    a.state_bf16 = d->state_dtype == SSD_BF16;
+    a.x = x; a.dt_raw = dt_raw; a.B = B; a.C = C; a.dt_bias = dt_bias; a.A = A; a.D = D;
+    a.init_state = init_state; a.y = y; a.final_state = final_state;
+    a.ws = (char*)workspace; a.lay = lay;
+    e = device_error_ptr(&a.dev_err);
+    if (e != cudaSuccess) return SSD_ERR_CUDA;
+    e = launch_dt_cumsum(a, s);
+    if (e != cudaSuccess) return SSD_ERR_CUDA;
+    e = tc ? launch_prefill_tc(a, s) : launch_prefill_simt(a, s);
+    return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
+}
+
+ssd_status_t ssd_state_update(const ssd_decode_desc_t* d, void* state, const void* x, const void* dt_raw,
+                              const float* dt_bias, const float* A, const void* B, const void* C,
+                              const float* D, void* y, void* stream) {
+    if (!d) return SSD_ERR_INVALID_ARG;
+    if (d->batch < 0 || d->nheads < 1 || d->headdim < 1 || d->dstate < 1 || d->ngroups < 1 ||
+        d->nheads % d->ngroups != 0)
+        return SSD_ERR_INVALID_ARG;
+    if (!valid_dtype(d->io_dtype) || !valid_dtype(d->y_dtype) || !valid_dtype(d->state_dtype))
+        return SSD_ERR_INVALID_ARG;
+    if (d->headdim % 8 != 0 || d->dstate % 8 != 0 || d->headdim > 256 || d->dstate > 256)
+        return SSD_ERR_UNSUPPORTED;
+    if (d->batch * d->nheads > (int64_t)0x7fffffff) return SSD_ERR_UNSUPPORTED;
+    if (!state || !x || !dt_raw || !A || !B || !C || !y) return SSD_ERR_INVALID_ARG;
+    const void* ptrs[] = {state, x, dt_raw, dt_bias, A, B, C, D, y};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return SSD_ERR_ALIGNMENT;
+    const size_t bh = (size_t)d->batch * d->nheads;
+    const size_t s_bytes = bh * d->dstate * d->headdim * dsize(d->state_dtype);
+    const size_t y_bytes = bh * d->headdim * dsize(d->y_dtype);
+    const size_t x_bytes = bh * d->headdim * dsize(d->io_dtype);
+    if (overlaps(y, y_bytes, state, s_bytes) || overlaps(y, y_bytes, x, x_bytes) ||
+        overlaps(state, s_bytes, x, x_bytes))
+        return SSD_ERR_INVALID_ARG;
+    if (d->batch == 0) return SSD_OK;
+    DecodeArgs a{};
+    a.batch = d->batch; a.H = d->nheads; a.P = d->headdim; a.N = d->dstate; a.G = d->ngroups;
+    a.io_bf16 = d->io_dtype == SSD_BF16; a.y_bf16 = d->y_dtype == SSD_BF16;
+    a.state_bf16 = d->state_dtype == SSD_BF16;
+    a.state = state; a.x = x; a.dt_raw = dt_raw; a.B = B; a.C = C;
+    a.dt_bias = dt_bias; a.A = A; a.D = D; a.y = y;
+    const cudaError_t e = launch_state_update(a, (cudaStream_t)stream);
+    return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
+}
+
+ssd_status_t ssd_get_device_error(void* stream, uint32_t* detail) {
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return SSD_ERR_CUDA;
+    unsigned v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(v)) != cudaSuccess) return SSD_ERR_CUDA;
+    if (v) {
+        const unsigned zero = 0;
+        if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess) return SSD_ERR_CUDA;
+    }
+    if (detail) *detail = v;
+    return v ? SSD_ERR_DEVICE_TIMEOUT : SSD_OK;
+}
+
+}  // extern "C"

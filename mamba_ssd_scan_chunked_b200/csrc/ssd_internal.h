@@ -1,0 +1,53 @@
+// Host-side declarations shared by the libssd translation units (not part of
+// the public C ABI in include/ssd.h).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace ssd {
+
+struct DecodeArgs {
+    int64_t batch, H, P, N, G;
+    bool io_bf16, y_bf16, state_bf16;
+    void* state;
+    const void *x, *dt_raw, *B, *C;
+    const float *dt_bias, *A, *D;
+    void* y;
+};
+
+cudaError_t launch_state_update(const DecodeArgs& a, cudaStream_t stream);
+
+// Workspace carve-up of the prefill (all offsets 256-byte aligned).
+struct PrefillLayout {
+    int64_t nchunks;       // ceil(L / Q)
+    int64_t Lpad;          // nchunks * Q
+    size_t off_dt, off_acs;        // fp32 [b][H][Lpad] each
+    size_t off_states;             // fp32 chunk states (CUDA-core path) or chain slots
+    size_t off_flags;              // int32 [b][H] chain progress + 64 control words
+    size_t total;
+};
+
+struct PrefillArgs {
+    int64_t batch, L, H, P, N, G, Q;
+    bool io_bf16, y_bf16, state_bf16;
+    const void *x, *dt_raw, *B, *C;
+    const float *dt_bias, *A, *D;
+    const void* init_state;
+    void* y;
+    void* final_state;
+    char* ws;
+    PrefillLayout lay;
+    unsigned* dev_err;     // device error word of the current device
+};
+
+// chunk-local dt / decay cumsum (shared by both prefill paths)
+cudaError_t launch_dt_cumsum(const PrefillArgs& a, cudaStream_t s);
+// CUDA-core fp32 prefill path (chunk states, state passing, chunk outputs)
+cudaError_t launch_prefill_simt(const PrefillArgs& a, cudaStream_t s);
+// tensor-core prefill path; returns cudaErrorNotSupported when the shape is not covered
+bool tc_path_supports(int64_t P, int64_t N, int64_t Q, bool io_bf16);
+cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s);
+
+}  // namespace ssd

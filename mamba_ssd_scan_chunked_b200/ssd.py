@@ -1,0 +1,221 @@
+"""Thin Python binding of libssd (include/ssd.h).
+
+Argument marshalling only: every step of the SSD computation runs in the CUDA
+kernels of ``libssd.so``.  PyTorch serves as the allocator of device memory and
+the source of streams.  There is no fallback: if ``libssd.so`` is missing the
+first call raises.
+
+Raw names mirror the C ABI (``ssd_chunk_scan_fwd``, ``ssd_state_update``, ...)
+and take integer device pointers; ``chunk_scan_fwd`` and ``state_update`` are
+the tensor-level conveniences (shape checks, output and workspace allocation).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libssd.so")
+
+SSD_F32 = 0
+SSD_BF16 = 1
+
+STATUS = {0: "SSD_OK", 1: "SSD_ERR_INVALID_ARG", 2: "SSD_ERR_UNSUPPORTED", 3: "SSD_ERR_ALIGNMENT",
+          4: "SSD_ERR_WORKSPACE", 5: "SSD_ERR_CUDA", 6: "SSD_ERR_DEVICE_TIMEOUT"}
+
+# every symbol include/ssd.h declares
+EXPORTS = ("ssd_version", "ssd_status_string", "ssd_chunk_scan_workspace_size", "ssd_chunk_scan_path",
+           "ssd_chunk_scan_fwd", "ssd_state_update", "ssd_get_device_error")
+
+
+class SsdError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS.get(status, status)}")
+
+
+class PrefillDesc(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int64), ("seqlen", ctypes.c_int64), ("nheads", ctypes.c_int64),
+                ("headdim", ctypes.c_int64), ("dstate", ctypes.c_int64), ("ngroups", ctypes.c_int64),
+                ("chunk", ctypes.c_int64), ("io_dtype", ctypes.c_int32), ("y_dtype", ctypes.c_int32),
+                ("state_dtype", ctypes.c_int32)]
+
+
+class DecodeDesc(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int64), ("nheads", ctypes.c_int64), ("headdim", ctypes.c_int64),
+                ("dstate", ctypes.c_int64), ("ngroups", ctypes.c_int64), ("io_dtype", ctypes.c_int32),
+                ("y_dtype", ctypes.c_int32), ("state_dtype", ctypes.c_int32)]
+
+
+_lock = threading.Lock()
+_lib = None
+_VP = ctypes.c_void_p
+
+
+def lib():
+    """The loaded libssd.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                                   "`python -m mamba_ssd_scan_chunked_b200.build` (there is no fallback path)")
+            L = ctypes.CDLL(LIB_PATH)
+            L.ssd_version.restype = ctypes.c_int
+            L.ssd_version.argtypes = []
+            L.ssd_status_string.restype = ctypes.c_char_p
+            L.ssd_status_string.argtypes = [ctypes.c_int]
+            L.ssd_chunk_scan_workspace_size.restype = ctypes.c_int
+            L.ssd_chunk_scan_workspace_size.argtypes = [ctypes.POINTER(PrefillDesc), ctypes.POINTER(ctypes.c_size_t)]
+            L.ssd_chunk_scan_path.restype = ctypes.c_int
+            L.ssd_chunk_scan_path.argtypes = [ctypes.POINTER(PrefillDesc), ctypes.POINTER(ctypes.c_int32)]
+            L.ssd_chunk_scan_fwd.restype = ctypes.c_int
+            L.ssd_chunk_scan_fwd.argtypes = [ctypes.POINTER(PrefillDesc)] + [_VP] * 10 + [_VP, ctypes.c_size_t, _VP]
+            L.ssd_state_update.restype = ctypes.c_int
+            L.ssd_state_update.argtypes = [ctypes.POINTER(DecodeDesc)] + [_VP] * 10
+            L.ssd_get_device_error.restype = ctypes.c_int
+            L.ssd_get_device_error.argtypes = [_VP, ctypes.POINTER(ctypes.c_uint32)]
+            _lib = L
+    return _lib
+
+
+# --------------------------------------------------------------------------
+# raw C-ABI calls (integer device pointers; 0 = NULL)
+# --------------------------------------------------------------------------
+def ssd_version() -> int:
+    return lib().ssd_version()
+
+
+def ssd_status_string(status: int) -> str:
+    return lib().ssd_status_string(status).decode()
+
+
+def ssd_chunk_scan_workspace_size(desc: PrefillDesc) -> int:
+    n = ctypes.c_size_t(0)
+    st = lib().ssd_chunk_scan_workspace_size(ctypes.byref(desc), ctypes.byref(n))
+    if st:
+        raise SsdError(st, "ssd_chunk_scan_workspace_size")
+    return n.value
+
+
+def ssd_chunk_scan_path(desc: PrefillDesc) -> int:
+    p = ctypes.c_int32(-1)
+    st = lib().ssd_chunk_scan_path(ctypes.byref(desc), ctypes.byref(p))
+    if st:
+        raise SsdError(st, "ssd_chunk_scan_path")
+    return p.value
+
+
+def ssd_chunk_scan_fwd(desc, x, dt_raw, dt_bias, A, B, C, D, init_state, y, final_state,
+                       workspace, workspace_bytes, stream) -> int:
+    """Raw call; returns the status code (0 = enqueued)."""
+    return lib().ssd_chunk_scan_fwd(ctypes.byref(desc), x or None, dt_raw or None, dt_bias or None, A or None,
+                                     B or None, C or None, D or None, init_state or None, y or None,
+                                     final_state or None, workspace or None, int(workspace_bytes), stream or None)
+
+
+def ssd_state_update(desc, state, x, dt_raw, dt_bias, A, B, C, D, y, stream) -> int:
+    """Raw call; returns the status code (0 = enqueued)."""
+    return lib().ssd_state_update(ctypes.byref(desc), state or None, x or None, dt_raw or None, dt_bias or None,
+                                  A or None, B or None, C or None, D or None, y or None, stream or None)
+
+
+def ssd_get_device_error(stream=None):
+    """Synchronise ``stream`` and return (status, detail bits) of the device error word."""
+    d = ctypes.c_uint32(0)
+    st = lib().ssd_get_device_error(stream or None, ctypes.byref(d))
+    return st, d.value
+
+
+# --------------------------------------------------------------------------
+# tensor-level conveniences
+# --------------------------------------------------------------------------
+def _dtype_code(t) -> int:
+    import torch
+    if t == torch.float32:
+        return SSD_F32
+    if t == torch.bfloat16:
+        return SSD_BF16
+    raise TypeError(f"unsupported dtype {t}; libssd takes float32 or bfloat16")
+
+
+def _torch_dtype(code: int):
+    import torch
+    return torch.bfloat16 if code == SSD_BF16 else torch.float32
+
+
+def _ptr(t) -> int:
+    return 0 if t is None else int(t.data_ptr())
+
+
+def _stream(stream) -> int:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def prefill_desc(x, B, chunk, y_dtype=None, state_dtype=None) -> PrefillDesc:
+    import torch
+    b, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    io = _dtype_code(x.dtype)
+    return PrefillDesc(b, L, H, P, N, G, int(chunk), io,
+                       _dtype_code(y_dtype) if y_dtype is not None else io,
+                       _dtype_code(state_dtype) if state_dtype is not None else SSD_F32)
+
+
+def workspace_bytes(x, B, chunk, y_dtype=None, state_dtype=None) -> int:
+    return ssd_chunk_scan_workspace_size(prefill_desc(x, B, chunk, y_dtype, state_dtype))
+
+
+def chunk_scan_fwd(x, dt_raw, dt_bias, A, B, C, D, chunk, init_state=None, *, y=None, final_state=None,
+                   y_dtype=None, state_dtype=None, want_final_state=True, workspace=None, stream=None):
+    """Chunked prefill scan.  Shapes: x [b,L,H,P], dt_raw [b,L,H], B/C [b,L,G,N], dt_bias/A/D [H] (fp32).
+
+    Returns (y, final_state).  Outputs and workspace are allocated with torch
+    when not given; ``state_dtype`` defaults to init_state's dtype, else fp32.
+    """
+    import torch
+    if state_dtype is None:
+        state_dtype = init_state.dtype if init_state is not None else torch.float32
+    desc = prefill_desc(x, B, chunk, y_dtype, state_dtype)
+    b, L, H, P = x.shape
+    N = B.shape[3]
+    for t in (x, dt_raw, B, C, dt_bias, A, D, init_state, y, final_state):
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("libssd takes contiguous CUDA tensors")
+    if y is None:
+        y = torch.empty((b, L, H, P), dtype=_torch_dtype(desc.y_dtype), device=x.device)
+    if final_state is None and want_final_state:
+        final_state = torch.empty((b, H, N, P), dtype=_torch_dtype(desc.state_dtype), device=x.device)
+    need = ssd_chunk_scan_workspace_size(desc)
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
+    st = ssd_chunk_scan_fwd(desc, _ptr(x), _ptr(dt_raw), _ptr(dt_bias), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                            _ptr(init_state), _ptr(y), _ptr(final_state), _ptr(workspace), workspace.numel(),
+                            _stream(stream))
+    if st:
+        raise SsdError(st, "ssd_chunk_scan_fwd")
+    return y, final_state
+
+
+def state_update(state, x, dt_raw, dt_bias, A, B, C, D, *, y=None, y_dtype=None, stream=None):
+    """Decode step in place on ``state`` [b,H,N,P].  x [b,H,P], dt_raw [b,H], B/C [b,G,N].  Returns y."""
+    import torch
+    b, H, P = x.shape
+    G, N = B.shape[1], B.shape[2]
+    io = _dtype_code(x.dtype)
+    desc = DecodeDesc(b, H, P, N, G, io, _dtype_code(y_dtype) if y_dtype is not None else io,
+                      _dtype_code(state.dtype))
+    for t in (state, x, dt_raw, B, C, dt_bias, A, D, y):
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("libssd takes contiguous CUDA tensors")
+    if y is None:
+        y = torch.empty((b, H, P), dtype=_torch_dtype(desc.y_dtype), device=x.device)
+    st = ssd_state_update(desc, _ptr(state), _ptr(x), _ptr(dt_raw), _ptr(dt_bias), _ptr(A), _ptr(B), _ptr(C),
+                          _ptr(D), _ptr(y), _stream(stream))
+    if st:
+        raise SsdError(st, "ssd_state_update")
+    return y

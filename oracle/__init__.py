@@ -74,6 +74,8 @@ def _load():
             lib.oracle_ssd_decode_step.restype = ctypes.c_int
             lib.oracle_round_bf16.argtypes = [ctypes.c_double]
             lib.oracle_round_bf16.restype = ctypes.c_double
+            lib.oracle_round_bf16_array.argtypes = [_D, _D, _I64]
+            lib.oracle_round_bf16_array.restype = None
             lib.oracle_softplus.argtypes = [ctypes.c_double]
             lib.oracle_softplus.restype = ctypes.c_double
             lib.oracle_num_threads.argtypes = []
@@ -105,10 +107,10 @@ def softplus(z: float) -> float:
 
 def round_bf16(v) -> np.ndarray:
     """Round float64 values to the nearest bfloat16 (ties to even), as float64."""
-    lib = _load()
-    a = np.asarray(v, dtype=np.float64)
-    out = np.array([lib.oracle_round_bf16(float(t)) for t in a.ravel()], dtype=np.float64)
-    return out.reshape(a.shape)
+    a = np.ascontiguousarray(v, dtype=np.float64)
+    out = np.empty_like(a)
+    _load().oracle_round_bf16_array(_ptr(a), _ptr(out), a.size)
+    return out
 
 
 def _run_prefill(fn_name, x, dt_raw, dt_bias, A, B, C, D, init_state, extra=(), nthreads=0,

@@ -73,6 +73,11 @@ double oracle_round_bf16(double v) {
     return r;
 }
 
+/* Element-wise oracle_round_bf16 over an array (out may equal in). */
+void oracle_round_bf16_array(const double* in, double* out, int64_t n) {
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_round_bf16(in[i]);
+}
+
 static int set_threads(int nthreads) {
 #ifdef _OPENMP
     if (nthreads > 0) return nthreads;

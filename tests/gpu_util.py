@@ -1,0 +1,104 @@
+"""Helpers of the GPU parity tests: move the seeded storage arrays to the
+device, run libssd through its C ABI (ssd.py marshals only), run the float64
+oracle on the same values, and measure max|err| / rms(oracle)."""
+import numpy as np
+
+import oracle
+from mamba_ssd_scan_chunked_b200 import inputs as I
+from mamba_ssd_scan_chunked_b200 import ssd
+
+# tolerances stated for the method: max|err| / rms(y_oracle)
+TOL_F32 = 1e-4
+TOL_BF16 = 2e-2
+
+
+def torch():
+    import torch as t
+    return t
+
+
+def to_dev(a: np.ndarray):
+    t = torch()
+    if a.dtype == np.uint16:
+        return t.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(t.bfloat16).cuda()
+    return t.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def to_host64(x) -> np.ndarray:
+    t = torch()
+    x = x.detach()
+    if x.dtype == t.bfloat16:
+        return I.to_f64(x.view(t.int16).cpu().numpy().view(np.uint16))
+    return x.cpu().numpy().astype(np.float64)
+
+
+def metric(got: np.ndarray, ref: np.ndarray) -> float:
+    rms = float(np.sqrt(np.mean(ref * ref)))
+    return float(np.max(np.abs(got - ref))) / max(rms, 1e-300)
+
+
+def bf16_excess_metric(got: np.ndarray, ref: np.ndarray) -> float:
+    """max(|err| - half a bf16 spacing of the reference) / rms: the error a
+    bf16 output adds beyond rounding the exact value to its own format."""
+    rms = float(np.sqrt(np.mean(ref * ref)))
+    mag = np.maximum(np.abs(ref), 2.0 ** -126)
+    half_ulp = 2.0 ** (np.floor(np.log2(mag)) - 8)
+    return float(np.max(np.maximum(np.abs(got - ref) - half_ulp, 0.0))) / max(rms, 1e-300)
+
+
+def bf16_state_metric(got: np.ndarray, ref: np.ndarray) -> float:
+    """For states STORED in bf16 on both sides: the kernel decides each bf16
+    rounding from an fp32 value, the oracle from a float64 one, so a stored
+    element may sit one bf16 step from the oracle's; beyond that one step the
+    error is measured against rms(ref) as usual."""
+    rms = float(np.sqrt(np.mean(ref * ref)))
+    mag = np.maximum(np.abs(ref), 2.0 ** -126)
+    ulp = 2.0 ** (np.floor(np.log2(mag)) - 7)
+    return float(np.max(np.maximum(np.abs(got - ref) - ulp, 0.0))) / max(rms, 1e-300)
+
+
+def record(name: str, **values):
+    """Append measured parity metrics to $SSD_PARITY_LOG (JSON lines), if set."""
+    import json
+    import os
+    path = os.environ.get("SSD_PARITY_LOG")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps({"test": name, **values}) + "\n")
+
+
+def gpu_prefill(inp: dict, chunk: int, init_state=None, y_dtype="f32", state_dtype="f32"):
+    """Run ssd_chunk_scan_fwd on storage arrays; returns (y, final_state) as float64 numpy."""
+    t = torch()
+    dev = {k: to_dev(v) for k, v in inp.items()}
+    init = to_dev(init_state) if init_state is not None else None
+    ydt = t.float32 if y_dtype == "f32" else t.bfloat16
+    sdt = t.float32 if state_dtype == "f32" else t.bfloat16
+    y, fs = ssd.chunk_scan_fwd(dev["x"], dev["dt_raw"], dev["dt_bias"], dev["A"], dev["B"], dev["C"], dev["D"],
+                               chunk, init, y_dtype=ydt, state_dtype=sdt)
+    t.cuda.synchronize()
+    st, detail = ssd.ssd_get_device_error(0)
+    assert st == 0, f"device error word {detail:#x}"
+    return to_host64(y), to_host64(fs)
+
+
+def oracle_prefill(inp: dict, init_state=None, heads=None):
+    """float64 oracle on the exact stored values; `heads` restricts to a subset of heads."""
+    f = {k: I.to_f64(v) for k, v in inp.items()}
+    h0 = I.to_f64(init_state) if init_state is not None else None
+    if heads is None:
+        return oracle.recurrent(f["x"], f["dt_raw"], f["dt_bias"], f["A"], f["B"], f["C"], f["D"], init_state=h0)
+    H, G = f["x"].shape[2], f["B"].shape[2]
+    ys, ss = [], []
+    for h in heads:
+        g = h // (H // G)
+        y, s = oracle.recurrent(f["x"][:, :, h:h + 1], f["dt_raw"][:, :, h:h + 1], f["dt_bias"][h:h + 1],
+                                f["A"][h:h + 1], f["B"][:, :, g:g + 1], f["C"][:, :, g:g + 1], f["D"][h:h + 1],
+                                init_state=None if h0 is None else h0[:, h:h + 1])
+        ys.append(y)
+        ss.append(s)
+    return np.concatenate(ys, axis=2), np.concatenate(ss, axis=1)
+
+
+def random_state(shape, seed, dtype, std=0.5):
+    return I.to_storage(np.random.default_rng(seed).normal(0, std, shape), dtype)

@@ -1,0 +1,141 @@
+"""The C ABI boundary, checked without a GPU.
+
+libssd.so must load on a machine without a GPU, export every function
+include/ssd.h declares, and reject invalid requests on the host before it
+touches a device (all calls below return before any CUDA call).
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from mamba_ssd_scan_chunked_b200 import build as B
+from mamba_ssd_scan_chunked_b200 import ssd
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ssd.h")
+
+OK, INVALID, UNSUPPORTED, ALIGN, WORKSPACE = 0, 1, 2, 3, 4
+FAKE = 0x7f0000000000          # 16-byte aligned fake device address (never dereferenced)
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    B.build()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ssd_[a-z_]+)\s*\(", text)))
+
+
+def test_header_matches_binding_exports():
+    assert declared_functions() == sorted(ssd.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol():
+    out = subprocess.run(["nm", "-D", "--defined-only", ssd.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(re.findall(r"\bT (ssd_\w+)", out))
+    for name in declared_functions():
+        assert name in exported, name
+        assert hasattr(ctypes.CDLL(ssd.LIB_PATH), name)
+
+
+def test_version_and_status_strings():
+    assert ssd.ssd_version() == 100
+    for code in range(7):
+        assert ssd.ssd_status_string(code).startswith(ssd.STATUS[code])
+    assert ssd.ssd_status_string(99) == "SSD_ERR_UNKNOWN"
+
+
+def desc(**kw):
+    d = dict(batch=2, seqlen=512, nheads=4, headdim=64, dstate=128, ngroups=2, chunk=256,
+             io_dtype=ssd.SSD_BF16, y_dtype=ssd.SSD_F32, state_dtype=ssd.SSD_F32)
+    d.update(kw)
+    return ssd.PrefillDesc(**d)
+
+
+def test_workspace_size_and_path():
+    d = desc()
+    n = ssd.ssd_chunk_scan_workspace_size(d)
+    BH, Lpad = 2 * 4, 512
+    # dt + cumsum (fp32 per token and head) + one fp32 state slot per (b, h) + flags
+    assert n >= 2 * 4 * BH * Lpad + 4 * BH * 128 * 64
+    assert ssd.ssd_chunk_scan_path(d) == 0                       # bf16, N=128: tensor cores
+    assert ssd.ssd_chunk_scan_path(desc(io_dtype=ssd.SSD_F32)) == 1   # fp32: CUDA cores
+    # the CUDA-core path keeps one fp32 state per chunk
+    n32 = ssd.ssd_chunk_scan_workspace_size(desc(io_dtype=ssd.SSD_F32))
+    assert n32 >= 4 * BH * 2 * 128 * 64
+    # ragged sequence: chunks are rounded up
+    assert ssd.ssd_chunk_scan_workspace_size(desc(seqlen=513)) > n
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(nheads=4, ngroups=3), INVALID),
+    (dict(batch=-1), INVALID),
+    (dict(nheads=0), INVALID),
+    (dict(io_dtype=7), INVALID),
+    (dict(y_dtype=-1), INVALID),
+    (dict(chunk=48), UNSUPPORTED),
+    (dict(chunk=512), UNSUPPORTED),
+    (dict(chunk=8), UNSUPPORTED),
+    (dict(headdim=12), UNSUPPORTED),
+    (dict(dstate=264), UNSUPPORTED),
+])
+def test_descriptor_validation(kw, code):
+    with pytest.raises(ssd.SsdError) as e:
+        ssd.ssd_chunk_scan_workspace_size(desc(**kw))
+    assert e.value.status == code
+
+
+def fwd(d, **ptrs):
+    p = dict(x=FAKE, dt_raw=FAKE + 0x1000000, dt_bias=0, A=FAKE + 0x2000000, B=FAKE + 0x3000000,
+             C=FAKE + 0x4000000, D=0, init_state=0, y=FAKE + 0x10000000, final_state=0, workspace=0,
+             workspace_bytes=0, stream=0)
+    p.update(ptrs)
+    return ssd.ssd_chunk_scan_fwd(d, p["x"], p["dt_raw"], p["dt_bias"], p["A"], p["B"], p["C"], p["D"],
+                                  p["init_state"], p["y"], p["final_state"], p["workspace"], p["workspace_bytes"],
+                                  p["stream"])
+
+
+def test_prefill_host_validation_codes():
+    d = desc()
+    assert fwd(d, x=0) == INVALID
+    assert fwd(d, A=0) == INVALID
+    assert fwd(d, y=0) == INVALID
+    assert fwd(d, x=FAKE + 8) == ALIGN
+    assert fwd(d, D=FAKE + 0x5000004) == ALIGN
+    assert fwd(d, y=FAKE) == INVALID                       # y aliases x
+    assert fwd(d) == WORKSPACE                             # no workspace
+    need = ssd.ssd_chunk_scan_workspace_size(d)
+    assert fwd(d, workspace=FAKE + 0x20000000, workspace_bytes=need - 1) == WORKSPACE
+    assert fwd(d, workspace=FAKE + 0x20000010, workspace_bytes=need) == ALIGN   # workspace wants 256-byte alignment
+    assert fwd(desc(batch=0)) == OK                        # empty batch: nothing to do, nothing launched
+    assert fwd(desc(chunk=100)) == UNSUPPORTED
+
+
+def test_decode_host_validation_codes():
+    def dd(**kw):
+        d = dict(batch=8, nheads=4, headdim=64, dstate=128, ngroups=2, io_dtype=ssd.SSD_BF16,
+                 y_dtype=ssd.SSD_F32, state_dtype=ssd.SSD_F32)
+        d.update(kw)
+        return ssd.DecodeDesc(**d)
+
+    def call(d, **ptrs):
+        p = dict(state=FAKE, x=FAKE + 0x1000000, dt_raw=FAKE + 0x2000000, dt_bias=0, A=FAKE + 0x3000000,
+                 B=FAKE + 0x4000000, C=FAKE + 0x5000000, D=0, y=FAKE + 0x6000000, stream=0)
+        p.update(ptrs)
+        return ssd.ssd_state_update(d, p["state"], p["x"], p["dt_raw"], p["dt_bias"], p["A"], p["B"], p["C"],
+                                    p["D"], p["y"], p["stream"])
+
+    assert call(dd(ngroups=3)) == INVALID
+    assert call(dd(headdim=10)) == UNSUPPORTED
+    assert call(dd(state_dtype=5)) == INVALID
+    assert call(dd(), state=0) == INVALID
+    assert call(dd(), x=FAKE + 0x1000004) == ALIGN
+    assert call(dd(), y=FAKE) == INVALID                   # y overlaps the state
+    assert call(dd(batch=0)) == OK

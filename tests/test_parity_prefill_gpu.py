@@ -1,0 +1,120 @@
+"""GPU parity of ssd_chunk_scan_fwd against the float64 oracle (small and
+medium shapes: several chunks, ragged tails, both kernel paths, all dtype
+combinations, initial states, cross-path invariants)."""
+import numpy as np
+import pytest
+
+from mamba_ssd_scan_chunked_b200 import inputs as I
+from mamba_ssd_scan_chunked_b200 import ssd
+from tests.gpu_util import (TOL_BF16, TOL_F32, bf16_excess_metric, gpu_prefill, metric, oracle_prefill,
+                            random_state, to_dev, to_host64, torch)
+
+pytestmark = pytest.mark.gpu
+
+
+def shape_inputs(b, L, H, P, N, G, dtype, seed):
+    return I.prefill_inputs(b, L, H, P, N, G, seed, dtype)
+
+
+def path_of(inp, chunk):
+    t = torch()
+    x = to_dev(inp["x"][:, :1])
+    Bm = to_dev(inp["B"][:, :1])
+    return ssd.ssd_chunk_scan_path(ssd.prefill_desc(x, Bm, chunk))
+
+
+# (b, L, H, P, N, G, chunk, dtype) -- L is not a multiple of the chunk in most cases
+CASES = [
+    (2, 300, 4, 64, 16, 2, 64, I.F32),      # fp32, CUDA cores, ragged tail
+    (1, 256, 4, 64, 16, 1, 64, I.F32),
+    (2, 200, 3, 32, 24, 3, 32, I.F32),      # odd head count, G = H
+    (1, 130, 2, 64, 64, 1, 16, I.F32),
+    (2, 600, 4, 64, 128, 2, 256, I.BF16),   # bf16, tensor cores: 3 chunks, last has 88 tokens
+    (2, 384, 4, 64, 128, 1, 128, I.BF16),   # tensor cores, chunk 128
+    (1, 1000, 6, 64, 128, 3, 256, I.BF16),  # tensor cores, 4 chunks, ragged 232-token tail
+    (2, 333, 4, 64, 64, 2, 64, I.BF16),     # bf16 on CUDA cores
+    (1, 257, 2, 128, 256, 1, 128, I.BF16),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: "b{}_L{}_H{}_P{}_N{}_G{}_Q{}_{}".format(*c))
+@pytest.mark.parametrize("with_init", [False, True])
+def test_prefill_matches_oracle(case, with_init):
+    b, L, H, P, N, G, Q, dt = case
+    inp = shape_inputs(b, L, H, P, N, G, dt, seed=11 + L)
+    h0 = random_state((b, H, N, P), 5 + L, I.F32) if with_init else None
+    y, fs = gpu_prefill(inp, Q, h0)
+    y_ref, fs_ref = oracle_prefill(inp, h0)
+    tol = TOL_F32 if dt == I.F32 else TOL_BF16
+    assert metric(y, y_ref) <= tol
+    assert metric(fs, fs_ref) <= tol
+
+
+def test_tensor_core_path_is_taken_for_bf16_dstate128():
+    inp = shape_inputs(1, 256, 2, 64, 128, 1, I.BF16, 3)
+    assert path_of(inp, 256) == 0
+    assert path_of(inp, 128) == 0
+    inp32 = shape_inputs(1, 256, 2, 64, 128, 1, I.F32, 3)
+    assert path_of(inp32, 256) == 1
+
+
+def test_tensor_core_error_budget_is_far_inside_the_bound():
+    # the hi/lo split keeps the tensor-core path ~100x inside the 2e-2 bound
+    inp = shape_inputs(2, 1024, 8, 64, 128, 2, I.BF16, 77)
+    y, fs = gpu_prefill(inp, 256)
+    y_ref, fs_ref = oracle_prefill(inp)
+    assert metric(y, y_ref) < 2e-3
+    assert metric(fs, fs_ref) < 2e-3
+
+
+@pytest.mark.parametrize("Q", [256, 64])
+def test_bf16_outputs(Q):
+    """y and final_state stored in bf16: the error beyond the output's own rounding stays in bounds."""
+    N = 128 if Q == 256 else 64
+    inp = shape_inputs(2, 512, 4, 64, N, 2, I.BF16, 21)
+    h0 = random_state((2, 4, N, 64), 22, I.BF16)
+    y, fs = gpu_prefill(inp, Q, h0, y_dtype="bf16", state_dtype="bf16")
+    y_ref, fs_ref = oracle_prefill(inp, h0)
+    assert bf16_excess_metric(y, y_ref) <= TOL_BF16
+    assert bf16_excess_metric(fs, fs_ref) <= TOL_BF16
+
+
+def test_zero_init_buffer_equals_null_init():
+    inp = shape_inputs(1, 512, 4, 64, 128, 2, I.BF16, 31)
+    y0, f0 = gpu_prefill(inp, 256)
+    z = np.zeros((1, 4, 128, 64), np.float32)
+    y1, f1 = gpu_prefill(inp, 256, z)
+    assert np.array_equal(y0, y1) and np.array_equal(f0, f1)
+
+
+@pytest.mark.parametrize("dt", [I.F32, I.BF16])
+def test_split_prefill_handoff(dt):
+    """prefill(L) == prefill(L1) then prefill(L - L1) from its final state."""
+    b, L, H, P, N, G, Q = 2, 768, 4, 64, 128, 2, 256
+    inp = shape_inputs(b, L, H, P, N, G, dt, 41)
+    y, fs = gpu_prefill(inp, Q)
+    L1 = 512
+    first = {k: (v[:, :L1] if k in ("x", "dt_raw", "B", "C") else v) for k, v in inp.items()}
+    second = {k: (np.ascontiguousarray(v[:, L1:]) if k in ("x", "dt_raw", "B", "C") else v) for k, v in inp.items()}
+    first = {k: np.ascontiguousarray(v) for k, v in first.items()}
+    y1, f1 = gpu_prefill(first, Q)
+    y2, f2 = gpu_prefill(second, Q, f1.astype(np.float32))
+    tol = TOL_F32 if dt == I.F32 else TOL_BF16
+    assert metric(np.concatenate([y1, y2], axis=1), y) <= tol
+    assert metric(f2, fs) <= tol
+
+
+def test_empty_sequence_copies_init_state():
+    t = torch()
+    inp = shape_inputs(2, 0, 4, 64, 128, 2, I.BF16, 51)
+    h0 = random_state((2, 4, 128, 64), 52, I.F32)
+    y, fs = gpu_prefill(inp, 256, h0)
+    assert y.shape == (2, 0, 4, 64)
+    assert np.array_equal(fs, I.to_f64(h0))
+    _, fz = gpu_prefill(inp, 256, None)
+    assert not np.any(fz)
+
+
+def test_device_error_word_clear_after_runs():
+    st, detail = ssd.ssd_get_device_error(0)
+    assert st == 0 and detail == 0
