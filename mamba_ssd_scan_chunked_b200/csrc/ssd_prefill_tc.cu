@@ -12,12 +12,12 @@
 // relative to the block start:
 //
 //   S    = C B^T                      (tcgen05, A=C K-major, B=B K-major, fp32 in TMEM)
-//   M    = S o [s<=l] 2^(r_l-r_s) dt_s   (CUDA cores, TMEM -> regs -> TMEM)
+//   M    = S o [s<=l] 2^(r_l-r_s) dt_s   (CUDA cores, TMEM -> regs -> TMEM in place)
 //   Y    = M X                        (tcgen05, A=M from TMEM, B=X MN-major)
 //   S_c  = B^T (w o X), w_s = 2^(r_last-r_s) dt_s     (tcgen05, A=B MN-major)
 //   h'   = 2^(r_last) h + S_c          (fp32, CUDA cores; the inter-chunk scan)
 //   Yoff = C h                         (tcgen05, A=C K-major, B=h MN-major)
-//   y    = Y + 2^(r_l) Yoff + D x      (fp32 epilogue)
+//   y    = Y + 2^(r_l) Yoff + D x      (fp32 epilogue, staged in smem, TMA store)
 //
 // Precision: the operands computed in-kernel (M, w o X, h) are split into a
 // bf16 pair hi + lo (hi = bf16(v), lo = bf16(v - hi)) and contracted with two
@@ -33,9 +33,10 @@
 // for flags[b,h] >= c, reads the fp32 state slot, updates it in place and sets
 // flags[b,h] = c+1.  A CTA allocates TMEM before taking a ticket, so a ticket
 // holder never waits for TMEM.  Every wait is bounded by a 2 s globaltimer
-// deadline; on expiry the kernel sets the device error word, makes every other
-// wait of the launch return at once, finishes its (in-bounds) work and frees
-// its TMEM.  Nothing traps.
+// deadline.  A hand-off wait that expires sets the device error word and a
+// launch-wide abort word that ends every other hand-off wait at once; the CTA
+// then finishes its (in-bounds) work -- still waiting for its own TMA and MMA
+// completions -- and frees its TMEM.  Nothing traps.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -49,7 +50,9 @@ namespace tc {
 
 constexpr int SUB = 128;        // tokens per block (MMA M)
 constexpr int PD = 64;          // headdim handled by this path
-constexpr int THREADS = 256;    // 8 warps; warps w and w+4 share TMEM lanes 32*(w%4)..+31
+constexpr int PIPES = 2;        // independent block pipelines per CTA (one CTA per SM)
+constexpr int PTHREADS = 256;   // threads of a pipeline: 8 warps; warps w and w+4 share TMEM lanes 32*(w%4)..+31
+constexpr int THREADS = PIPES * PTHREADS;
 constexpr uint32_t TILE = SUB * 128;   // [128 rows x 64 bf16] SW128 tile = 16 KB
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr unsigned long long WAIT_NS = 2000000000ull;   // bound of every device-side wait
@@ -58,7 +61,8 @@ constexpr unsigned long long WAIT_NS = 2000000000ull;   // bound of every device
 constexpr uint32_t COL_R = 0;     // S (fp32 128) -> M hi|lo (bf16x2 64+64) -> Yoff (fp32 64)
 constexpr uint32_t COL_Y = 128;   // Y accumulator (fp32 64)
 constexpr uint32_t COL_ST = 192;  // chunk-state accumulator (fp32 64, lanes = n)
-constexpr uint32_t TMEM_COLS = 256;
+constexpr uint32_t PIPE_COLS = 256;              // TMEM columns of one pipeline
+constexpr uint32_t TMEM_COLS = PIPES * PIPE_COLS;
 
 // control words after the per-(b,h) flags
 constexpr int CTRL_TICKET = 0;
@@ -70,14 +74,15 @@ struct Cfg {
     static constexpr uint32_t OFF_C = 0;
     static constexpr uint32_t OFF_B = OFF_C + KB * TILE;
     static constexpr uint32_t OFF_X = OFF_B + KB * TILE;
-    static constexpr uint32_t OFF_W = OFF_X + TILE;          // w o X, then h (MN-major)
+    // W1/W2: hi/lo halves of w o X, then of h (MN-major operands), then the y staging tile
     static constexpr uint32_t W_BYTES = (N > SUB ? N : SUB) * 128;
-    static constexpr uint32_t OFF_R = OFF_W + W_BYTES;       // r[128]
-    static constexpr uint32_t OFF_DT = OFF_R + 512;          // dt[128]
-    static constexpr uint32_t OFF_BAR = OFF_DT + 512;        // mbarriers
-    static constexpr uint32_t OFF_MISC = OFF_BAR + 64;       // tmem base, ticket, abort
-    static constexpr uint32_t BYTES = OFF_MISC + 64;
-    static constexpr uint32_t SMEM = BYTES + 1024;           // + alignment slack
+    static constexpr uint32_t OFF_W1 = OFF_X + TILE;
+    static constexpr uint32_t OFF_W2 = OFF_W1 + W_BYTES;
+    static constexpr uint32_t OFF_CS = OFF_W2 + W_BYTES;      // log2(dt_s) - r_s [128]
+    static constexpr uint32_t OFF_BAR = OFF_CS + 512;        // mbarriers
+    static constexpr uint32_t OFF_MISC = OFF_BAR + 64;       // tmem base, tickets
+    static constexpr uint32_t PIPE_SMEM = (OFF_MISC + 64 + 1023) / 1024 * 1024;   // one pipeline's region
+    static constexpr uint32_t SMEM = PIPES * PIPE_SMEM;      // 1024-byte aligned base (checked)
     static constexpr uint32_t TX = (2 * KB + 1) * TILE;      // TMA bytes per block
 };
 
@@ -133,6 +138,21 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* tm,
         "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], [%6];"
         ::"r"(dst), "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar)
         : "memory");
+}
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap* tm, uint32_t src, int c0, int c1, int c2, int c3) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];"
+        ::"l"(reinterpret_cast<uint64_t>(tm)), "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+        : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// 2^x on the SFU (approximate, flushes subnormal results to zero; 2^-inf = 0)
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 __device__ __forceinline__ void mma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
     asm volatile(
@@ -214,51 +234,81 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
 }
 
 // ---------------------------------------------------------------- the kernel
+// Persistent: each CTA takes work items by ticket until none are left, and
+// prefetches the next 128-token block (of the same item or of its next item)
+// while it finishes the current one.  Two CTAs share an SM.
 template <int N>
-__global__ void __launch_bounds__(THREADS, 2)
+__global__ void __launch_bounds__(THREADS, 1)
 ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
-              const __grid_constant__ CUtensorMap tmC, const Params p) {
+              const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmY, const Params p) {
     using K = Cfg<N>;
     static_assert(N == 128, "this instantiation covers dstate 128");
-    extern __shared__ uint8_t smem_raw[];
-    const uint32_t raw = smem_u32(smem_raw);
-    const uint32_t base = (raw + 1023u) & ~1023u;
-    uint8_t* sm = smem_raw + (base - raw);
+    extern __shared__ __align__(1024) uint8_t smem_all[];
+    const int pipe = threadIdx.x / PTHREADS;          // this thread's pipeline
+    uint8_t* sm = smem_all + pipe * K::PIPE_SMEM;     // the pipeline's own smem region
+    const uint32_t base = smem_u32(sm);
+    const uint32_t base_all = smem_u32(smem_all);
 
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int tid = threadIdx.x % PTHREADS, warp = tid >> 5, lane = tid & 31;
     const int half = warp >> 2;                       // column half of the tiles
     const int row = (warp & 3) * 32 + lane;           // TMEM lane = tile row
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
 
-    float* sr = reinterpret_cast<float*>(sm + K::OFF_R);
-    float* sdt = reinterpret_cast<float*>(sm + K::OFF_DT);
-    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + K::OFF_MISC);
-    int* s_ticket = reinterpret_cast<int*>(sm + K::OFF_MISC + 4);
-    enum { BAR_TMA = 0, BAR_S, BAR_ST1, BAR_Y, BAR_ST2, BAR_OFF1, BAR_OFF2, NBAR };
+    float* scs = reinterpret_cast<float*>(sm + K::OFF_CS);
+    int* s_ticket = reinterpret_cast<int*>(sm + K::OFF_MISC + 4);     // item of the current block
+    int* s_next = reinterpret_cast<int*>(sm + K::OFF_MISC + 8);       // item of the next item
+    enum { BAR_TMA = 0, BAR_S, BAR_ST, BAR_Y, BAR_OFF, NBAR };
     auto bar = [&](int i) -> uint32_t { return base + K::OFF_BAR + 8u * (uint32_t)i; };
     volatile int* g_abort = reinterpret_cast<volatile int*>(p.flags + p.BH + CTRL_ABORT);
+    const int total = p.nchunks * p.BH;
+    unsigned err = 0;
 
-    // TMEM first, then the ticket (a ticket holder never waits for TMEM)
-    if (warp == 0) {
+    // the 128-byte swizzle of TMA and of the MMA descriptors assumes 1024-byte
+    // aligned tiles; refuse to run (and say so) if the runtime did not align
+    if (base_all & 1023u) {
+        if (threadIdx.x == 0) atomicOr(p.dev_err, kErrAsyncTimeout);
+        return;
+    }
+    // TMEM first, then tickets (a ticket holder never waits for TMEM)
+    if (threadIdx.x < 32) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
-                     ::"r"(base + K::OFF_MISC), "r"(TMEM_COLS) : "memory");
+                     ::"r"(base_all + K::OFF_MISC), "r"(TMEM_COLS) : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     if (tid == 32) {
         for (int i = 0; i < NBAR; ++i) mbar_init(bar(i), 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (tid == 0) *s_ticket = atomicAdd(p.flags + p.BH + CTRL_TICKET, 1);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = *s_tmem;
-    const int item = *s_ticket;
-    const int c = item / p.BH, bh = item % p.BH;
-    const int b = bh / p.H, h = bh % p.H, g = h / (p.H / p.G);
-    unsigned err = 0;
+    // the pipeline's 256 columns of the CTA's allocation (address = lane << 16 | column)
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem_all + K::OFF_MISC) + PIPE_COLS * pipe;
+    // barrier of this pipeline's 256 threads (named barrier 1 or 2; 0 is __syncthreads)
+    auto psync = [&]() { asm volatile("bar.sync %0, %1;" ::"r"(1 + pipe), "r"(PTHREADS) : "memory"); };
+
     auto wait = [&](int i, uint32_t ph) {
         if (!mbar_wait(bar(i), ph)) err |= kErrAsyncTimeout;
+    };
+    // (item, block) -> coordinates
+    auto nblocks = [&](int it) -> int {
+        const long long rem = p.L - (long long)(it / p.BH) * p.Q;
+        const int n = (int)((rem + SUB - 1) / SUB);
+        return n < p.Q / SUB ? n : p.Q / SUB;
+    };
+    // TMA of block j of item `it` (thread 0)
+    auto issue_loads = [&](int it, int j) {
+        const int c_ = it / p.BH, bh_ = it % p.BH;
+        const int b_ = bh_ / p.H, h_ = bh_ % p.H, g_ = h_ / (p.H / p.G);
+        const int t0_ = c_ * p.Q + j * SUB;
+        fence_proxy_async();
+        mbar_expect_tx(bar(BAR_TMA), K::TX);
+#pragma unroll
+        for (int kb = 0; kb < K::KB; ++kb) {
+            tma_load_4d(base + K::OFF_C + kb * TILE, &tmC, kb * 64, g_, t0_, b_, bar(BAR_TMA));
+            tma_load_4d(base + K::OFF_B + kb * TILE, &tmB, kb * 64, g_, t0_, b_, bar(BAR_TMA));
+        }
+        tma_load_4d(base + K::OFF_X, &tmX, 0, h_, t0_, b_, bar(BAR_TMA));
     };
 
     // instruction descriptors
@@ -266,42 +316,41 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
     constexpr uint32_t ID_ST = idesc_bf16(128, PD, true, true);     // B^T (MN-major) x wX (MN-major)
     constexpr uint32_t ID_Y = idesc_bf16(128, PD, false, true);     // M (TMEM) x X (MN-major)
     constexpr uint32_t ID_OFF = idesc_bf16(128, PD, false, true);   // C (K-major) x h (MN-major)
+    const float NEG_INF = __int_as_float(0xff800000u);
 
-    // a ticket beyond the grid cannot happen when the control words were reset
-    // by the decay-cumsum kernel; guard anyway so no index leaves its buffer
-    const bool valid_item = item >= 0 && item < p.nchunks * p.BH;
-    const long long tok0 = (long long)c * p.Q;
-    const int nsub_all = p.Q / SUB;
-    const long long rem = p.L - tok0;
-    const int nsub = !valid_item ? 0
-                     : ((int)((rem + SUB - 1) / SUB) < nsub_all ? (int)((rem + SUB - 1) / SUB) : nsub_all);
-    const float dsk = p.D ? p.D[h] : 0.f;
-    float hreg[32];                                   // state h (row `row`, cols half*32..+31)
+    if (tid == 0) {
+        const int it = atomicAdd(p.flags + p.BH + CTRL_TICKET, 1);
+        *s_ticket = it;
+        if (it < total) issue_loads(it, 0);
+    }
+    psync();
+    int item = *s_ticket;
+    int j = 0;
+    uint32_t blk = 0;      // blocks processed by this CTA: phase of every mbarrier
 
-    for (int j = 0; j < nsub; ++j) {
-        const uint32_t ph = (uint32_t)(j & 1);
-        const long long t0 = tok0 + (long long)j * SUB;
-        // ---- stage the block: TMA for C, B, X; dt and decay cumsum by threads
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
+    while (item < total) {
+        const uint32_t ph = blk & 1u;
+        const int c = item / p.BH, bh = item % p.BH;
+        const int b = bh / p.H, h = bh % p.H;
+        const int nsub = nblocks(item);
+        const bool last_block = (j == nsub - 1);
+        const long long t0 = (long long)c * p.Q + (long long)j * SUB;
+
+        // ---- per-token decay terms of the block (r relative to the block start, log2 units)
+        const long long o_bh = (long long)bh * p.Lpad;
+        const float r0 = (j == 0) ? 0.f : p.acsw[o_bh + t0 - 1];
+        const float rl = (p.acsw[o_bh + t0 + row] - r0) * LOG2E;           // this row
+        const float rlast = (p.acsw[o_bh + t0 + SUB - 1] - r0) * LOG2E;    // block end
+        if (half == 0) {
+            const float d = p.dtw[o_bh + t0 + row];
+            // dt folded into the exponent: dt_s 2^(x - r_s) = 2^(x + log2(dt_s) - r_s); dt_s = 0 gives 0
+            scs[row] = (d > 0.f ? __log2f(d) : NEG_INF) - rl;
+        }
         if (tid == 0) {
-            fence_proxy_async();
-            mbar_expect_tx(bar(BAR_TMA), K::TX);
-#pragma unroll
-            for (int kb = 0; kb < K::KB; ++kb) {
-                tma_load_4d(base + K::OFF_C + kb * TILE, &tmC, kb * 64, g, (int)t0, b, bar(BAR_TMA));
-                tma_load_4d(base + K::OFF_B + kb * TILE, &tmB, kb * 64, g, (int)t0, b, bar(BAR_TMA));
-            }
-            tma_load_4d(base + K::OFF_X, &tmX, 0, h, (int)t0, b, bar(BAR_TMA));
+            bulk_wait_read0();                                // previous y store done reading W1/W2
+            if (last_block) *s_next = atomicAdd(p.flags + p.BH + CTRL_TICKET, 1);
         }
-        if (tid < SUB) {
-            const long long o = (long long)bh * p.Lpad + t0 + tid;
-            const float r0 = (j == 0) ? 0.f : p.acsw[(long long)bh * p.Lpad + t0 - 1];
-            sr[tid] = (p.acsw[o] - r0) * LOG2E;
-            sdt[tid] = p.dtw[o];
-        }
-        __syncthreads();
+        psync();
         wait(BAR_TMA, ph);
 
         // ---- S = C B^T (K = N)
@@ -315,115 +364,109 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
             }
             mma_commit(bar(BAR_S));
         }
-
-        // ---- w o X (hi into smem now, lo kept in registers)
-        const float rlast = sr[SUB - 1];
-        uint32_t wlo[16];
+        // ---- w o X split hi -> W1, lo -> W2; then both state passes back to back
         {
-            const int s = row;
-            const float w = exp2f(rlast - sr[s]) * sdt[s];
+            const float w = ex2(rlast + scs[row]);
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                const uint32_t o = swz(s, half * 4 + q);
+                const uint32_t o = swz(row, half * 4 + q);
                 const uint4 xv = *reinterpret_cast<const uint4*>(sm + K::OFF_X + o);
                 const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-                uint32_t hw[4];
+                uint32_t hw[4], lw[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const float v0 = bf16_lo(xw[e]) * w, v1 = bf16_hi(xw[e]) * w;
                     hw[e] = pack_bf16(v0, v1);
-                    wlo[q * 4 + e] = pack_bf16(v0 - bf16_lo(hw[e]), v1 - bf16_hi(hw[e]));
+                    lw[e] = pack_bf16(v0 - bf16_lo(hw[e]), v1 - bf16_hi(hw[e]));
                 }
-                *reinterpret_cast<uint4*>(sm + K::OFF_W + o) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                *reinterpret_cast<uint4*>(sm + K::OFF_W1 + o) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                *reinterpret_cast<uint4*>(sm + K::OFF_W2 + o) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
             }
         }
         fence_proxy_async();
-        __syncthreads();
-        // ---- chunk state, hi part: S_c = B^T (w o X)_hi   (K = 128 tokens)
+        psync();
         if (tid == 0) {
             tc_fence_after();
 #pragma unroll
             for (int k = 0; k < SUB / 16; ++k)
                 mma_ss(tmem + COL_ST, sdesc(base + K::OFF_B + k * 2048, TILE, 1024),
-                       sdesc(base + K::OFF_W + k * 2048, TILE, 1024), ID_ST, k > 0);
-            mma_commit(bar(BAR_ST1));
+                       sdesc(base + K::OFF_W1 + k * 2048, TILE, 1024), ID_ST, k > 0);
+#pragma unroll
+            for (int k = 0; k < SUB / 16; ++k)
+                mma_ss(tmem + COL_ST, sdesc(base + K::OFF_B + k * 2048, TILE, 1024),
+                       sdesc(base + K::OFF_W2 + k * 2048, TILE, 1024), ID_ST, 1);
+            mma_commit(bar(BAR_ST));
         }
 
-        // ---- M = S o mask o 2^(r_l - r_s) dt_s, split hi/lo, back into TMEM
+        // ---- M = S o [s<=l] 2^(r_l - r_s) dt_s, split hi/lo, written back in place:
+        // for every 16-column K step k of the MMA, hi goes to columns [16k, 16k+8)
+        // and lo to [16k+8, 16k+16) -- the very S columns this thread just read,
+        // so no other thread's input is overwritten.
         wait(BAR_S, ph);
         tc_fence_after();
-        {
-            uint32_t mh[32], ml[32];
-            const float rl = sr[row];
 #pragma unroll
-            for (int part = 0; part < 2; ++part) {
-                uint32_t sv[32];
-                tmem_ld32(tmem + lane_off + COL_R + half * 64 + part * 32, sv);
-                tmem_wait_ld();
+        for (int part = 0; part < 2; ++part) {
+            const int c0 = half * 64 + part * 32;
+            uint32_t v[32], o[32];
+            tmem_ld32(tmem + lane_off + COL_R + c0, v);
+            tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const int s0 = half * 64 + part * 32 + 2 * i;
-                    const float m0 = (s0 <= row) ? __uint_as_float(sv[2 * i]) * exp2f(rl - sr[s0]) * sdt[s0] : 0.f;
-                    const float m1 =
-                        (s0 + 1 <= row) ? __uint_as_float(sv[2 * i + 1]) * exp2f(rl - sr[s0 + 1]) * sdt[s0 + 1] : 0.f;
+            for (int g = 0; g < 2; ++g) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int s0 = c0 + g * 16 + 2 * i;
+                    const float e0 = ex2(s0 <= row ? rl + scs[s0] : NEG_INF);
+                    const float e1 = ex2(s0 + 1 <= row ? rl + scs[s0 + 1] : NEG_INF);
+                    const float m0 = __uint_as_float(v[g * 16 + 2 * i]) * e0;
+                    const float m1 = __uint_as_float(v[g * 16 + 2 * i + 1]) * e1;
                     const uint32_t hi = pack_bf16(m0, m1);
-                    mh[part * 16 + i] = hi;
-                    ml[part * 16 + i] = pack_bf16(m0 - bf16_lo(hi), m1 - bf16_hi(hi));
+                    o[g * 16 + i] = hi;
+                    o[g * 16 + 8 + i] = pack_bf16(m0 - bf16_lo(hi), m1 - bf16_hi(hi));
                 }
             }
-            tc_fence_before();
-            __syncthreads();            // every S column read before any is overwritten
-            tc_fence_after();
-            tmem_st32(tmem + lane_off + COL_R + half * 32, mh);        // M hi: packed cols [0, 64)
-            tmem_st32(tmem + lane_off + COL_R + 64 + half * 32, ml);   // M lo: packed cols [64, 128)
-            tmem_wait_st();
+            tmem_st32(tmem + lane_off + COL_R + c0, o);
         }
+        tmem_wait_st();
         tc_fence_before();
-        __syncthreads();
+        psync();
         // ---- Y = M_hi X + M_lo X   (K = 128 tokens, A from TMEM)
         if (tid == 0) {
             tc_fence_after();
 #pragma unroll
             for (int k = 0; k < SUB / 16; ++k)
-                mma_ts(tmem + COL_Y, tmem + COL_R + 8 * k, sdesc(base + K::OFF_X + k * 2048, TILE, 1024), ID_Y, k > 0);
+                mma_ts(tmem + COL_Y, tmem + COL_R + 16 * k, sdesc(base + K::OFF_X + k * 2048, TILE, 1024), ID_Y, k > 0);
 #pragma unroll
             for (int k = 0; k < SUB / 16; ++k)
-                mma_ts(tmem + COL_Y, tmem + COL_R + 64 + 8 * k, sdesc(base + K::OFF_X + k * 2048, TILE, 1024), ID_Y, 1);
+                mma_ts(tmem + COL_Y, tmem + COL_R + 16 * k + 8, sdesc(base + K::OFF_X + k * 2048, TILE, 1024), ID_Y, 1);
             mma_commit(bar(BAR_Y));
         }
 
-        // ---- chunk state, lo part
-        wait(BAR_ST1, ph);
+        // ---- x of this thread's outputs (for D x), kept before sX is reloaded
+        uint32_t xr[16];
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-            *reinterpret_cast<uint4*>(sm + K::OFF_W + swz(row, half * 4 + q)) =
-                make_uint4(wlo[q * 4], wlo[q * 4 + 1], wlo[q * 4 + 2], wlo[q * 4 + 3]);
-        fence_proxy_async();
-        __syncthreads();
-        if (tid == 0) {
-            tc_fence_after();
-#pragma unroll
-            for (int k = 0; k < SUB / 16; ++k)
-                mma_ss(tmem + COL_ST, sdesc(base + K::OFF_B + k * 2048, TILE, 1024),
-                       sdesc(base + K::OFF_W + k * 2048, TILE, 1024), ID_ST, 1);
-            mma_commit(bar(BAR_ST2));
+        for (int q = 0; q < 4; ++q) {
+            const uint4 xv = *reinterpret_cast<const uint4*>(sm + K::OFF_X + swz(row, half * 4 + q));
+            xr[4 * q] = xv.x; xr[4 * q + 1] = xv.y; xr[4 * q + 2] = xv.z; xr[4 * q + 3] = xv.w;
         }
 
-        // ---- h entering this block
+        // ---- h entering this block: the initial state, the previous chunk's
+        // published state, or the state this CTA left in the slot after its
+        // previous block of the same item (same thread, same addresses)
         float hin[32];
-        if (j == 0) {
-            if (c == 0) {
-                if (p.init_state) {
-                    const long long o = ((long long)bh * N + row) * PD + half * 32;
+        float* slot = p.slots + ((long long)bh * N + row) * PD + half * 32;
+        if (j == 0 && c == 0) {
+            if (p.init_state) {
+                const long long o = ((long long)bh * N + row) * PD + half * 32;
 #pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        hin[i] = p.state_bf16 ? __bfloat162float(reinterpret_cast<const bf16*>(p.init_state)[o + i])
-                                              : reinterpret_cast<const float*>(p.init_state)[o + i];
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) hin[i] = 0.f;
-                }
+                for (int i = 0; i < 32; ++i)
+                    hin[i] = p.state_bf16 ? __bfloat162float(reinterpret_cast<const bf16*>(p.init_state)[o + i])
+                                          : reinterpret_cast<const float*>(p.init_state)[o + i];
             } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) hin[i] = 0.f;
+            }
+        } else {
+            if (j == 0) {
                 if (tid == 0) {
                     // bounded wait for chunk c-1 of this (b, h); a wait that gives
                     // up raises the launch-wide abort word so the others stop at once
@@ -443,150 +486,145 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                         __nanosleep(64);
                     }
                 }
-                __syncthreads();
-                const float* slot = p.slots + ((long long)bh * N + row) * PD + half * 32;
-#pragma unroll
-                for (int i = 0; i < 32; i += 4) {
-                    const float4 v = __ldcg(reinterpret_cast<const float4*>(slot + i));
-                    hin[i] = v.x; hin[i + 1] = v.y; hin[i + 2] = v.z; hin[i + 3] = v.w;
-                }
+                psync();
             }
-        } else {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) hin[i] = hreg[i];
+            for (int i = 0; i < 32; i += 4) {
+                const float4 v = __ldcg(reinterpret_cast<const float4*>(slot + i));
+                hin[i] = v.x; hin[i + 1] = v.y; hin[i + 2] = v.z; hin[i + 3] = v.w;
+            }
         }
 
-        // ---- h' = 2^(r_last) h + S_c; publish after the last block of the item
-        wait(BAR_ST2, ph);   // also orders after the Y MMAs (issued earlier)
+        // ---- h' = 2^(r_last) h + S_c (fp32): into the slot (for the next block, or
+        // published for the next chunk after the last block), or final_state
+        wait(BAR_ST, ph);
         tc_fence_after();
         {
             uint32_t sv[32];
             tmem_ld32(tmem + lane_off + COL_ST + half * 32, sv);
             tmem_wait_ld();
-            const float dl = exp2f(rlast);
+            const float dl = ex2(rlast);
+            float ho[32];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) hreg[i] = fmaf(dl, hin[i], __uint_as_float(sv[i]));
-        }
-        const bool last_block = (j == nsub - 1);
-        if (last_block) {
-            if (c == p.nchunks - 1) {
+            for (int i = 0; i < 32; ++i) ho[i] = fmaf(dl, hin[i], __uint_as_float(sv[i]));
+            if (last_block && c == p.nchunks - 1) {
                 if (p.final_state) {
                     const long long o = ((long long)bh * N + row) * PD + half * 32;
                     if (p.state_bf16) {
                         bf16* fs = reinterpret_cast<bf16*>(p.final_state) + o;
 #pragma unroll
-                        for (int i = 0; i < 32; i += 8) {
-                            float v8[8];
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) v8[e] = hreg[i + e];
-                            Vec16<bf16>::store(fs + i, v8);
-                        }
+                        for (int i = 0; i < 32; i += 8) Vec16<bf16>::store(fs + i, ho + i);
                     } else {
                         float* fs = reinterpret_cast<float*>(p.final_state) + o;
 #pragma unroll
                         for (int i = 0; i < 32; i += 4)
-                            *reinterpret_cast<float4*>(fs + i) = make_float4(hreg[i], hreg[i + 1], hreg[i + 2], hreg[i + 3]);
+                            *reinterpret_cast<float4*>(fs + i) = make_float4(ho[i], ho[i + 1], ho[i + 2], ho[i + 3]);
                     }
                 }
             } else {
-                float* slot = p.slots + ((long long)bh * N + row) * PD + half * 32;
 #pragma unroll
                 for (int i = 0; i < 32; i += 4)
-                    __stcg(reinterpret_cast<float4*>(slot + i), make_float4(hreg[i], hreg[i + 1], hreg[i + 2], hreg[i + 3]));
-                __threadfence();
+                    __stcg(reinterpret_cast<float4*>(slot + i), make_float4(ho[i], ho[i + 1], ho[i + 2], ho[i + 3]));
             }
         }
-        // h (entering the block) split for C h: hi into smem, lo kept
-        uint32_t hlo[16];
+        // ---- h (entering the block) split hi -> W1, lo -> W2 (free: the state MMAs are done)
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-            uint32_t hw[4];
+            uint32_t hw[4], lw[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const float v0 = hin[q * 8 + 2 * e], v1 = hin[q * 8 + 2 * e + 1];
                 hw[e] = pack_bf16(v0, v1);
-                hlo[q * 4 + e] = pack_bf16(v0 - bf16_lo(hw[e]), v1 - bf16_hi(hw[e]));
+                lw[e] = pack_bf16(v0 - bf16_lo(hw[e]), v1 - bf16_hi(hw[e]));
             }
-            *reinterpret_cast<uint4*>(sm + K::OFF_W + swz(row, half * 4 + q)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+            const uint32_t o = swz(row, half * 4 + q);
+            *reinterpret_cast<uint4*>(sm + K::OFF_W1 + o) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+            *reinterpret_cast<uint4*>(sm + K::OFF_W2 + o) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
         }
         fence_proxy_async();
         tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
+        psync();
+        // next block: the same item's next block, or the first block of the next ticket
+        const int next_item = last_block ? *s_next : item;
+        const int next_j = last_block ? 0 : j + 1;
         if (tid == 0) {
-            if (last_block && c < p.nchunks - 1)
+            tc_fence_after();
+            if (last_block && c < p.nchunks - 1) {
+                // every thread's slot stores precede the barrier above; the fence
+                // and release make them visible before the flag
+                __threadfence();
                 asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p.flags + bh), "r"(c + 1) : "memory");
-            // ---- Yoff = C h_hi (K = N), into the freed region R
-#pragma unroll
-            for (int k = 0; k < N / 16; ++k) {
-                const uint32_t off = (uint32_t)(k >> 2) * TILE + (uint32_t)(k & 3) * 32u;
-                mma_ss(tmem + COL_R, sdesc(base + K::OFF_C + off, 16, 1024), sdesc(base + K::OFF_W + k * 2048, TILE, 1024),
-                       ID_OFF, k > 0);
             }
-            mma_commit(bar(BAR_OFF1));
-        }
-        wait(BAR_OFF1, ph);
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-            *reinterpret_cast<uint4*>(sm + K::OFF_W + swz(row, half * 4 + q)) =
-                make_uint4(hlo[q * 4], hlo[q * 4 + 1], hlo[q * 4 + 2], hlo[q * 4 + 3]);
-        fence_proxy_async();
-        __syncthreads();
-        if (tid == 0) {
+            // ---- Yoff = C h_hi + C h_lo (K = N) into region R, once Y has consumed M
+            wait(BAR_Y, ph);
             tc_fence_after();
 #pragma unroll
             for (int k = 0; k < N / 16; ++k) {
                 const uint32_t off = (uint32_t)(k >> 2) * TILE + (uint32_t)(k & 3) * 32u;
-                mma_ss(tmem + COL_R, sdesc(base + K::OFF_C + off, 16, 1024), sdesc(base + K::OFF_W + k * 2048, TILE, 1024),
-                       ID_OFF, 1);
+                mma_ss(tmem + COL_R, sdesc(base + K::OFF_C + off, 16, 1024),
+                       sdesc(base + K::OFF_W1 + k * 2048, TILE, 1024), ID_OFF, k > 0);
             }
-            mma_commit(bar(BAR_OFF2));
+#pragma unroll
+            for (int k = 0; k < N / 16; ++k) {
+                const uint32_t off = (uint32_t)(k >> 2) * TILE + (uint32_t)(k & 3) * 32u;
+                mma_ss(tmem + COL_R, sdesc(base + K::OFF_C + off, 16, 1024),
+                       sdesc(base + K::OFF_W2 + k * 2048, TILE, 1024), ID_OFF, 1);
+            }
+            mma_commit(bar(BAR_OFF));
         }
 
-        // ---- y = Y + 2^(r_l) Yoff + D x
-        wait(BAR_OFF2, ph);
+        // ---- y = Y + 2^(r_l) Yoff + D x; the next block's loads overlap this epilogue
+        wait(BAR_OFF, ph);
         tc_fence_after();
+        if (tid == 0 && next_item < total) issue_loads(next_item, next_j);   // C, B, X all free now
         {
             uint32_t yv[32], ov[32];
             tmem_ld32(tmem + lane_off + COL_Y + half * 32, yv);
             tmem_ld32(tmem + lane_off + COL_R + half * 32, ov);
             tmem_wait_ld();
-            const long long t = t0 + row;
-            if (t < p.L) {
-                const float el = exp2f(sr[row]);
-                float out[32];
+            const float el = ex2(rl);
+            const float dsk = p.D ? p.D[h] : 0.f;
+            float out[32];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const uint4 xv = *reinterpret_cast<const uint4*>(sm + K::OFF_X + swz(row, half * 4 + q));
-                    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+            for (int e = 0; e < 16; ++e) {
+                out[2 * e] = __uint_as_float(yv[2 * e]) + el * __uint_as_float(ov[2 * e]) + dsk * bf16_lo(xr[e]);
+                out[2 * e + 1] =
+                    __uint_as_float(yv[2 * e + 1]) + el * __uint_as_float(ov[2 * e + 1]) + dsk * bf16_hi(xr[e]);
+            }
+            // staging tiles: W1 (and W2 for the second fp32 half), free since OFF completed
+            if (p.y_bf16) {
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int i = q * 8 + 2 * e;
-                        out[i] = __uint_as_float(yv[i]) + el * __uint_as_float(ov[i]) + dsk * bf16_lo(xw[e]);
-                        out[i + 1] = __uint_as_float(yv[i + 1]) + el * __uint_as_float(ov[i + 1]) + dsk * bf16_hi(xw[e]);
-                    }
-                }
-                const long long o = (((long long)b * p.L + t) * p.H + h) * PD + half * 32;
-                if (p.y_bf16) {
-                    bf16* yp = reinterpret_cast<bf16*>(p.y) + o;
+                for (int q = 0; q < 4; ++q)
+                    *reinterpret_cast<uint4*>(sm + K::OFF_W1 + swz(row, half * 4 + q)) = Vec16<bf16>::pack(out + 8 * q);
+            } else {
+                uint8_t* tile = sm + (half ? K::OFF_W2 : K::OFF_W1);
 #pragma unroll
-                    for (int i = 0; i < 32; i += 8) Vec16<bf16>::store(yp + i, out + i);
-                } else {
-                    float* yp = reinterpret_cast<float*>(p.y) + o;
-#pragma unroll
-                    for (int i = 0; i < 32; i += 4)
-                        __stcs(reinterpret_cast<float4*>(yp + i), make_float4(out[i], out[i + 1], out[i + 2], out[i + 3]));
-                }
+                for (int q = 0; q < 8; ++q)
+                    *reinterpret_cast<float4*>(tile + swz(row, q)) =
+                        make_float4(out[4 * q], out[4 * q + 1], out[4 * q + 2], out[4 * q + 3]);
             }
         }
+        fence_proxy_async();
+        tc_fence_before();
+        psync();
+        if (tid == 0) {
+            tma_store_4d(&tmY, base + K::OFF_W1, 0, h, (int)t0, b);
+            if (!p.y_bf16) tma_store_4d(&tmY, base + K::OFF_W2, 32, h, (int)t0, b);
+            bulk_commit();
+        }
+        item = next_item;
+        j = next_j;
+        ++blk;
     }
 
+    if (tid == 0) bulk_wait0();   // the last y store is complete before the CTA leaves
     if (err) atomicOr(p.dev_err, err);
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) {
+    if (threadIdx.x < 32) {
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
+        const uint32_t tmem_all = *reinterpret_cast<volatile uint32_t*>(smem_all + K::OFF_MISC);
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_all), "r"(TMEM_COLS) : "memory");
     }
 }
 
@@ -604,15 +642,19 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// 4-D bf16 tensor map (inner, d1, d2, d3), box {64, 1, 128, 1}, 128-byte swizzle
-static bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t d1, uint64_t d2, uint64_t d3) {
+// 4-D tensor map (inner, d1, d2, d3) with a {128 bytes, 1, 128, 1} box and
+// 128-byte swizzle: 64 bf16 or 32 fp32 elements per row of the box
+static bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t d1, uint64_t d2, uint64_t d3,
+                     bool fp32 = false) {
     auto fn = encode_fn();
     if (!fn) return false;
+    const uint64_t es = fp32 ? 4 : 2;
     cuuint64_t dims[4] = {inner, d1, d2, d3};
-    cuuint64_t strides[3] = {inner * 2, inner * d1 * 2, inner * d1 * d2 * 2};
-    cuuint32_t box[4] = {64, 1, (cuuint32_t)SUB, 1};
+    cuuint64_t strides[3] = {inner * es, inner * d1 * es, inner * d1 * d2 * es};
+    cuuint32_t box[4] = {(cuuint32_t)(128 / es), 1, (cuuint32_t)SUB, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estr,
+    return fn(m, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+              const_cast<void*>(ptr), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -620,22 +662,30 @@ static bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t d
 template <int N>
 static cudaError_t launch_n(const PrefillArgs& a, cudaStream_t s) {
     using K = Cfg<N>;
-    CUtensorMap mx, mb, mc;
-    if (!make_map(&mx, a.x, (uint64_t)a.P, (uint64_t)a.H, (uint64_t)a.L, (uint64_t)a.batch) ||
+    CUtensorMap mx, mb, mc, my;
+    if (!make_map(&my, a.y, (uint64_t)a.P, (uint64_t)a.H, (uint64_t)a.L, (uint64_t)a.batch, !a.y_bf16) ||
+        !make_map(&mx, a.x, (uint64_t)a.P, (uint64_t)a.H, (uint64_t)a.L, (uint64_t)a.batch) ||
         !make_map(&mb, a.B, (uint64_t)a.N, (uint64_t)a.G, (uint64_t)a.L, (uint64_t)a.batch) ||
         !make_map(&mc, a.C, (uint64_t)a.N, (uint64_t)a.G, (uint64_t)a.L, (uint64_t)a.batch))
         return cudaErrorInvalidValue;
+    // persistent grid: as many CTAs as can be resident (one per SM), never more than items
     static std::mutex mu;
-    static bool attr_set[64] = {};
+    static int resident[64] = {};
     int dev = 0;
-    cudaGetDevice(&dev);
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     {
         std::lock_guard<std::mutex> lk(mu);
-        if (dev < 64 && !attr_set[dev]) {
-            cudaError_t e = cudaFuncSetAttribute(ssd_tc_kernel<N>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 (int)K::SMEM);
+        if (!resident[dev]) {
+            e = cudaFuncSetAttribute(ssd_tc_kernel<N>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)K::SMEM);
             if (e != cudaSuccess) return e;
-            attr_set[dev] = true;
+            int per_sm = 0, sms = 0;
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ssd_tc_kernel<N>, THREADS, K::SMEM);
+            if (e != cudaSuccess) return e;
+            e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+            if (e != cudaSuccess) return e;
+            resident[dev] = (per_sm > 0 ? per_sm : 1) * sms;
         }
     }
     Params p{};
@@ -659,7 +709,9 @@ static cudaError_t launch_n(const PrefillArgs& a, cudaStream_t s) {
     p.y_bf16 = a.y_bf16;
     const long long items = (long long)p.nchunks * p.BH;
     if (items > 0x7fffffffLL) return cudaErrorInvalidValue;
-    ssd_tc_kernel<N><<<(unsigned)items, THREADS, K::SMEM, s>>>(mx, mb, mc, p);
+    const long long want = (items + PIPES - 1) / PIPES;   // each CTA runs PIPES ticket streams
+    const unsigned grid = (unsigned)(want < resident[dev] ? want : resident[dev]);
+    ssd_tc_kernel<N><<<grid, THREADS, K::SMEM, s>>>(mx, mb, mc, my, p);
     return cudaGetLastError();
 }
 
