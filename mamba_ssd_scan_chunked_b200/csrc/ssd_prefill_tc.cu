@@ -51,8 +51,11 @@ namespace tc {
 constexpr int SUB = 128;        // tokens per block (MMA M)
 constexpr int PD = 64;          // headdim handled by this path
 constexpr int PIPES = 2;        // independent block pipelines per CTA (one CTA per SM)
-constexpr int PTHREADS = 256;   // threads of a pipeline: 8 warps; warps w and w+4 share TMEM lanes 32*(w%4)..+31
-constexpr int THREADS = PIPES * PTHREADS;
+constexpr int NCOMPUTE = 256;   // compute threads of a pipeline: 8 warps; warps w and w+4 share TMEM lanes 32*(w%4)..+31
+// thread layout: warps 8p..8p+7 compute for pipeline p, then one control warp per
+// pipeline.  A warp may only touch TMEM lanes 32*(warp % 4), so compute warps
+// must start at a multiple of 4 warps: they come first.
+constexpr int THREADS = PIPES * (NCOMPUTE + 32);
 constexpr uint32_t TILE = SUB * 128;   // [128 rows x 64 bf16] SW128 tile = 16 KB
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr unsigned long long WAIT_NS = 2000000000ull;   // bound of every device-side wait
@@ -71,6 +74,7 @@ constexpr int CTRL_ABORT = 1;
 template <int N>
 struct Cfg {
     static constexpr int KB = N / 64;                       // 64-wide K blocks of C, B
+    // tiles of one pipeline (1024-byte aligned, 128-byte swizzle)
     static constexpr uint32_t OFF_C = 0;
     static constexpr uint32_t OFF_B = OFF_C + KB * TILE;
     static constexpr uint32_t OFF_X = OFF_B + KB * TILE;
@@ -78,12 +82,16 @@ struct Cfg {
     static constexpr uint32_t W_BYTES = (N > SUB ? N : SUB) * 128;
     static constexpr uint32_t OFF_W1 = OFF_X + TILE;
     static constexpr uint32_t OFF_W2 = OFF_W1 + W_BYTES;
-    static constexpr uint32_t OFF_CS = OFF_W2 + W_BYTES;      // log2(dt_s) - r_s [128]
-    static constexpr uint32_t OFF_BAR = OFF_CS + 512;        // mbarriers
-    static constexpr uint32_t OFF_MISC = OFF_BAR + 64;       // tmem base, tickets
-    static constexpr uint32_t PIPE_SMEM = (OFF_MISC + 64 + 1023) / 1024 * 1024;   // one pipeline's region
-    static constexpr uint32_t SMEM = PIPES * PIPE_SMEM;      // 1024-byte aligned base (checked)
-    static constexpr uint32_t TX = (2 * KB + 1) * TILE;      // TMA bytes per block
+    static constexpr uint32_t TILES = OFF_W2 + W_BYTES;
+    // small area of one pipeline (after the tiles of all pipelines)
+    static constexpr uint32_t OFF_ACS = 0;                   // chunk-local cumsum of the block [128] (TMA)
+    static constexpr uint32_t OFF_DTCS = OFF_ACS + 512;      // dt [128] (TMA), turned into log2(dt_s) - r_s
+    static constexpr uint32_t OFF_BAR = OFF_DTCS + 512;      // mbarriers
+    static constexpr uint32_t OFF_MISC = OFF_BAR + 80;       // tmem base, block coordinates
+    static constexpr uint32_t SMALL = OFF_MISC + 64;
+    static constexpr uint32_t SMEM = PIPES * (TILES + SMALL);
+    static constexpr uint32_t TX = (2 * KB + 1) * TILE + 2 * SUB * 4;   // TMA bytes per block
+    static_assert(TILES % 1024 == 0 && SMALL % 16 == 0, "alignment");
 };
 
 struct Params {
@@ -145,6 +153,14 @@ __device__ __forceinline__ void tma_store_4d(const CUtensorMap* tm, uint32_t src
         ::"l"(reinterpret_cast<uint64_t>(tm)), "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
         : "memory");
 }
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+// 1-D bulk copy global -> shared (16-byte aligned addresses, size a multiple of 16)
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
+}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
@@ -154,15 +170,20 @@ __device__ __forceinline__ float ex2(float x) {
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
-__device__ __forceinline__ void mma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+// one tcgen05.mma (kind::f16, A and B from shared memory); IDESC and ACC are
+// compile-time constants so an issue costs the MMA and two address adds
+template <uint32_t IDESC, int ACC>
+__device__ __forceinline__ void mma_ss(uint32_t d, uint64_t a, uint64_t b) {
     asm volatile(
         "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n"
-        ::"r"(d), "l"(a), "l"(b), "r"(idesc), "r"(acc) : "memory");
+        ::"r"(d), "l"(a), "l"(b), "n"(IDESC), "n"(ACC) : "memory");
 }
-__device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
+// one tcgen05.mma with the A operand in tensor memory
+template <uint32_t IDESC, int ACC>
+__device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a_tmem, uint64_t b) {
     asm volatile(
         "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n"
-        ::"r"(d), "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc) : "memory");
+        ::"r"(d), "r"(a_tmem), "l"(b), "n"(IDESC), "n"(ACC) : "memory");
 }
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
@@ -186,6 +207,20 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
         "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
         "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};"
         ::"r"(taddr), SSD_W8(0), SSD_W8(8), SSD_W8(16), SSD_W8(24)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15}, [%16];"
+        : SSD_R8(0), SSD_R8(8)
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16};"
+        ::"r"(taddr), SSD_W8(0), SSD_W8(8)
         : "memory");
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
@@ -234,9 +269,12 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
 }
 
 // ---------------------------------------------------------------- the kernel
-// Persistent: each CTA takes work items by ticket until none are left, and
-// prefetches the next 128-token block (of the same item or of its next item)
-// while it finishes the current one.  Two CTAs share an SM.
+// Persistent, one CTA per SM, PIPES independent block pipelines per CTA.  A
+// pipeline = 8 compute warps (256 threads; thread = one TMEM lane/tile row and
+// one half of its columns) + 1 control warp whose lane 0 takes tickets,
+// issues every TMA and MMA, waits for the previous chunk of the chain and
+// publishes.  Compute and control meet only at mbarriers; the control warp
+// loads block n+1 as soon as the MMAs of block n are done.
 template <int N>
 __global__ void __launch_bounds__(THREADS, 1)
 ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
@@ -244,21 +282,26 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
     using K = Cfg<N>;
     static_assert(N == 128, "this instantiation covers dstate 128");
     extern __shared__ __align__(1024) uint8_t smem_all[];
-    const int pipe = threadIdx.x / PTHREADS;          // this thread's pipeline
-    uint8_t* sm = smem_all + pipe * K::PIPE_SMEM;     // the pipeline's own smem region
+    const bool control = threadIdx.x >= PIPES * NCOMPUTE;   // a pipeline's control warp
+    const int pipe = control ? (threadIdx.x - PIPES * NCOMPUTE) / 32 : threadIdx.x / NCOMPUTE;
+    uint8_t* sm = smem_all + pipe * K::TILES;         // the pipeline's own tiles
+    uint8_t* ss = smem_all + PIPES * K::TILES + pipe * K::SMALL;   // and its small area
     const uint32_t base = smem_u32(sm);
+    const uint32_t sbase = smem_u32(ss);
     const uint32_t base_all = smem_u32(smem_all);
-
-    const int tid = threadIdx.x % PTHREADS, warp = tid >> 5, lane = tid & 31;
-    const int half = warp >> 2;                       // column half of the tiles
-    const int row = (warp & 3) * 32 + lane;           // TMEM lane = tile row
+    const int tid = threadIdx.x % NCOMPUTE;           // compute thread index within its pipeline
+    const int warp = tid >> 5, lane = threadIdx.x & 31;
+    const int half = (warp >> 2) & 1;                 // column half of the tiles
+    const int row = (warp & 3) * 32 + lane;           // TMEM lane = tile row; warp % 4 == CTA warp % 4
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
 
-    float* scs = reinterpret_cast<float*>(sm + K::OFF_CS);
-    int* s_ticket = reinterpret_cast<int*>(sm + K::OFF_MISC + 4);     // item of the current block
-    int* s_next = reinterpret_cast<int*>(sm + K::OFF_MISC + 8);       // item of the next item
-    enum { BAR_TMA = 0, BAR_S, BAR_ST, BAR_Y, BAR_OFF, NBAR };
-    auto bar = [&](int i) -> uint32_t { return base + K::OFF_BAR + 8u * (uint32_t)i; };
+    float* scs = reinterpret_cast<float*>(ss + K::OFF_DTCS);           // dt, then log2(dt) - r
+    const float* s_acs = reinterpret_cast<const float*>(ss + K::OFF_ACS);
+    volatile int* s_item = reinterpret_cast<volatile int*>(ss + K::OFF_MISC + 4);
+    volatile int* s_j = reinterpret_cast<volatile int*>(ss + K::OFF_MISC + 8);
+    uint8_t* s_tmem_slot = smem_all + PIPES * K::TILES + K::OFF_MISC;    // pipeline 0's misc word
+    enum { BAR_TMA = 0, BAR_S, BAR_WX, BAR_ST, BAR_M, BAR_CHAIN, BAR_Y, BAR_H, BAR_OFF, BAR_EPI, NBAR };
+    auto bar = [&](int i) -> uint32_t { return sbase + K::OFF_BAR + 8u * (uint32_t)i; };
     volatile int* g_abort = reinterpret_cast<volatile int*>(p.flags + p.BH + CTRL_ABORT);
     const int total = p.nchunks * p.BH;
     unsigned err = 0;
@@ -272,204 +315,91 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
     // TMEM first, then tickets (a ticket holder never waits for TMEM)
     if (threadIdx.x < 32) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
-                     ::"r"(base_all + K::OFF_MISC), "r"(TMEM_COLS) : "memory");
+                     ::"r"(smem_u32(s_tmem_slot)), "r"(TMEM_COLS) : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
-    if (tid == 32) {
-        for (int i = 0; i < NBAR; ++i) mbar_init(bar(i), 1);
+    if (!control && tid == 0) {
+        const uint32_t cnt[NBAR] = {1, 1, NCOMPUTE, 1, NCOMPUTE, 1, 1, NCOMPUTE, 1, NCOMPUTE};
+        for (int i = 0; i < NBAR; ++i) mbar_init(bar(i), cnt[i]);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     // the pipeline's 256 columns of the CTA's allocation (address = lane << 16 | column)
-    const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem_all + K::OFF_MISC) + PIPE_COLS * pipe;
-    // barrier of this pipeline's 256 threads (named barrier 1 or 2; 0 is __syncthreads)
-    auto psync = [&]() { asm volatile("bar.sync %0, %1;" ::"r"(1 + pipe), "r"(PTHREADS) : "memory"); };
-
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(s_tmem_slot) + PIPE_COLS * pipe;
     auto wait = [&](int i, uint32_t ph) {
         if (!mbar_wait(bar(i), ph)) err |= kErrAsyncTimeout;
     };
-    // (item, block) -> coordinates
     auto nblocks = [&](int it) -> int {
         const long long rem = p.L - (long long)(it / p.BH) * p.Q;
         const int n = (int)((rem + SUB - 1) / SUB);
         return n < p.Q / SUB ? n : p.Q / SUB;
     };
-    // TMA of block j of item `it` (thread 0)
-    auto issue_loads = [&](int it, int j) {
-        const int c_ = it / p.BH, bh_ = it % p.BH;
-        const int b_ = bh_ / p.H, h_ = bh_ % p.H, g_ = h_ / (p.H / p.G);
-        const int t0_ = c_ * p.Q + j * SUB;
-        fence_proxy_async();
-        mbar_expect_tx(bar(BAR_TMA), K::TX);
-#pragma unroll
-        for (int kb = 0; kb < K::KB; ++kb) {
-            tma_load_4d(base + K::OFF_C + kb * TILE, &tmC, kb * 64, g_, t0_, b_, bar(BAR_TMA));
-            tma_load_4d(base + K::OFF_B + kb * TILE, &tmB, kb * 64, g_, t0_, b_, bar(BAR_TMA));
-        }
-        tma_load_4d(base + K::OFF_X, &tmX, 0, h_, t0_, b_, bar(BAR_TMA));
-    };
 
-    // instruction descriptors
-    constexpr uint32_t ID_S = idesc_bf16(128, 128, false, false);   // C (K-major) x B^T (K-major)
-    constexpr uint32_t ID_ST = idesc_bf16(128, PD, true, true);     // B^T (MN-major) x wX (MN-major)
-    constexpr uint32_t ID_Y = idesc_bf16(128, PD, false, true);     // M (TMEM) x X (MN-major)
-    constexpr uint32_t ID_OFF = idesc_bf16(128, PD, false, true);   // C (K-major) x h (MN-major)
-    const float NEG_INF = __int_as_float(0xff800000u);
-
-    if (tid == 0) {
-        const int it = atomicAdd(p.flags + p.BH + CTRL_TICKET, 1);
-        *s_ticket = it;
-        if (it < total) issue_loads(it, 0);
-    }
-    psync();
-    int item = *s_ticket;
-    int j = 0;
-    uint32_t blk = 0;      // blocks processed by this CTA: phase of every mbarrier
-
-    while (item < total) {
-        const uint32_t ph = blk & 1u;
-        const int c = item / p.BH, bh = item % p.BH;
-        const int b = bh / p.H, h = bh % p.H;
-        const int nsub = nblocks(item);
-        const bool last_block = (j == nsub - 1);
-        const long long t0 = (long long)c * p.Q + (long long)j * SUB;
-
-        // ---- per-token decay terms of the block (r relative to the block start, log2 units)
-        const long long o_bh = (long long)bh * p.Lpad;
-        const float r0 = (j == 0) ? 0.f : p.acsw[o_bh + t0 - 1];
-        const float rl = (p.acsw[o_bh + t0 + row] - r0) * LOG2E;           // this row
-        const float rlast = (p.acsw[o_bh + t0 + SUB - 1] - r0) * LOG2E;    // block end
-        if (half == 0) {
-            const float d = p.dtw[o_bh + t0 + row];
-            // dt folded into the exponent: dt_s 2^(x - r_s) = 2^(x + log2(dt_s) - r_s); dt_s = 0 gives 0
-            scs[row] = (d > 0.f ? __log2f(d) : NEG_INF) - rl;
-        }
-        if (tid == 0) {
-            bulk_wait_read0();                                // previous y store done reading W1/W2
-            if (last_block) *s_next = atomicAdd(p.flags + p.BH + CTRL_TICKET, 1);
-        }
-        psync();
-        wait(BAR_TMA, ph);
-
-        // ---- S = C B^T (K = N)
-        if (tid == 0) {
-            tc_fence_after();
-#pragma unroll
-            for (int k = 0; k < N / 16; ++k) {
-                const uint32_t off = (uint32_t)(k >> 2) * TILE + (uint32_t)(k & 3) * 32u;
-                mma_ss(tmem + COL_R, sdesc(base + K::OFF_C + off, 16, 1024), sdesc(base + K::OFF_B + off, 16, 1024),
-                       ID_S, k > 0);
-            }
-            mma_commit(bar(BAR_S));
-        }
-        // ---- w o X split hi -> W1, lo -> W2; then both state passes back to back
-        {
-            const float w = ex2(rlast + scs[row]);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const uint32_t o = swz(row, half * 4 + q);
-                const uint4 xv = *reinterpret_cast<const uint4*>(sm + K::OFF_X + o);
-                const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-                uint32_t hw[4], lw[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float v0 = bf16_lo(xw[e]) * w, v1 = bf16_hi(xw[e]) * w;
-                    hw[e] = pack_bf16(v0, v1);
-                    lw[e] = pack_bf16(v0 - bf16_lo(hw[e]), v1 - bf16_hi(hw[e]));
+    if (control) {
+        // ==================================================== control warp
+        if (lane == 0) {
+            constexpr uint32_t ID_S = idesc_bf16(128, 128, false, false);   // C (K-major) x B^T (K-major)
+            constexpr uint32_t ID_ST = idesc_bf16(128, PD, true, true);     // B^T (MN-major) x wX (MN-major)
+            constexpr uint32_t ID_Y = idesc_bf16(128, PD, false, true);     // M (TMEM) x X (MN-major)
+            constexpr uint32_t ID_OFF = idesc_bf16(128, PD, false, true);   // C (K-major) x h (MN-major)
+            // publish the block's coordinates, then load its operands and per-token terms
+            auto load_block = [&](int it, int j) {
+                *s_item = it;
+                *s_j = j;
+                if (it >= total) {                      // no more work: release the compute warps
+                    mbar_arrive(bar(BAR_TMA));
+                    return;
                 }
-                *reinterpret_cast<uint4*>(sm + K::OFF_W1 + o) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-                *reinterpret_cast<uint4*>(sm + K::OFF_W2 + o) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-            }
-        }
-        fence_proxy_async();
-        psync();
-        if (tid == 0) {
-            tc_fence_after();
+                const int c_ = it / p.BH, bh_ = it % p.BH;
+                const int b_ = bh_ / p.H, h_ = bh_ % p.H, g_ = h_ / (p.H / p.G);
+                const int t0_ = c_ * p.Q + j * SUB;
+                fence_proxy_async();
+                mbar_expect_tx(bar(BAR_TMA), K::TX);
 #pragma unroll
-            for (int k = 0; k < SUB / 16; ++k)
-                mma_ss(tmem + COL_ST, sdesc(base + K::OFF_B + k * 2048, TILE, 1024),
-                       sdesc(base + K::OFF_W1 + k * 2048, TILE, 1024), ID_ST, k > 0);
-#pragma unroll
-            for (int k = 0; k < SUB / 16; ++k)
-                mma_ss(tmem + COL_ST, sdesc(base + K::OFF_B + k * 2048, TILE, 1024),
-                       sdesc(base + K::OFF_W2 + k * 2048, TILE, 1024), ID_ST, 1);
-            mma_commit(bar(BAR_ST));
-        }
-
-        // ---- M = S o [s<=l] 2^(r_l - r_s) dt_s, split hi/lo, written back in place:
-        // for every 16-column K step k of the MMA, hi goes to columns [16k, 16k+8)
-        // and lo to [16k+8, 16k+16) -- the very S columns this thread just read,
-        // so no other thread's input is overwritten.
-        wait(BAR_S, ph);
-        tc_fence_after();
-#pragma unroll
-        for (int part = 0; part < 2; ++part) {
-            const int c0 = half * 64 + part * 32;
-            uint32_t v[32], o[32];
-            tmem_ld32(tmem + lane_off + COL_R + c0, v);
-            tmem_wait_ld();
-#pragma unroll
-            for (int g = 0; g < 2; ++g) {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int s0 = c0 + g * 16 + 2 * i;
-                    const float e0 = ex2(s0 <= row ? rl + scs[s0] : NEG_INF);
-                    const float e1 = ex2(s0 + 1 <= row ? rl + scs[s0 + 1] : NEG_INF);
-                    const float m0 = __uint_as_float(v[g * 16 + 2 * i]) * e0;
-                    const float m1 = __uint_as_float(v[g * 16 + 2 * i + 1]) * e1;
-                    const uint32_t hi = pack_bf16(m0, m1);
-                    o[g * 16 + i] = hi;
-                    o[g * 16 + 8 + i] = pack_bf16(m0 - bf16_lo(hi), m1 - bf16_hi(hi));
+                for (int kb = 0; kb < K::KB; ++kb) {
+                    tma_load_4d(base + K::OFF_C + kb * TILE, &tmC, kb * 64, g_, t0_, b_, bar(BAR_TMA));
+                    tma_load_4d(base + K::OFF_B + kb * TILE, &tmB, kb * 64, g_, t0_, b_, bar(BAR_TMA));
                 }
-            }
-            tmem_st32(tmem + lane_off + COL_R + c0, o);
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        psync();
-        // ---- Y = M_hi X + M_lo X   (K = 128 tokens, A from TMEM)
-        if (tid == 0) {
-            tc_fence_after();
+                tma_load_4d(base + K::OFF_X, &tmX, 0, h_, t0_, b_, bar(BAR_TMA));
+                const long long o = (long long)bh_ * p.Lpad + t0_;
+                bulk_load(sbase + K::OFF_ACS, p.acsw + o, SUB * 4, bar(BAR_TMA));
+                bulk_load(sbase + K::OFF_DTCS, p.dtw + o, SUB * 4, bar(BAR_TMA));
+            };
+            // Shared-memory descriptors, built once: a K step of a K-major operand
+            // advances the start address by 32 B (+2 in the descriptor), a 64-wide
+            // K block by one tile (+TILE/16); a K step of an MN-major operand by 16
+            // rows of 128 B (+128).  The 14-bit address field cannot overflow:
+            // every shared address is below 2^18.
+            const uint64_t dC = sdesc(base + K::OFF_C, 16, 1024);       // K-major (S, Yoff)
+            const uint64_t dBk = sdesc(base + K::OFF_B, 16, 1024);      // K-major (S)
+            const uint64_t dBm = sdesc(base + K::OFF_B, TILE, 1024);    // MN-major (state)
+            const uint64_t dX = sdesc(base + K::OFF_X, TILE, 1024);     // MN-major (Y)
+            const uint64_t dW1 = sdesc(base + K::OFF_W1, TILE, 1024);   // MN-major (state, Yoff)
+            const uint64_t dW2 = sdesc(base + K::OFF_W2, TILE, 1024);
+            constexpr uint32_t KSTEP_K = 2, KBLOCK_K = TILE >> 4, KSTEP_MN = 2048 >> 4;
+            int item = atomicAdd(p.flags + p.BH + CTRL_TICKET, 1);
+            int j = 0;
+            load_block(item, 0);
+            uint32_t blk = 0;
+            while (item < total) {
+                const uint32_t ph = blk & 1u;
+                const int c = item / p.BH, bh = item % p.BH;
+                const bool last_block = (j == nblocks(item) - 1);
+                wait(BAR_TMA, ph);
+                if (blk > 0) wait(BAR_EPI, ph ^ 1u);   // block n-1 finished reading TMEM
+                tc_fence_after();
+                // ---- S = C B^T (K = N)
 #pragma unroll
-            for (int k = 0; k < SUB / 16; ++k)
-                mma_ts(tmem + COL_Y, tmem + COL_R + 16 * k, sdesc(base + K::OFF_X + k * 2048, TILE, 1024), ID_Y, k > 0);
-#pragma unroll
-            for (int k = 0; k < SUB / 16; ++k)
-                mma_ts(tmem + COL_Y, tmem + COL_R + 16 * k + 8, sdesc(base + K::OFF_X + k * 2048, TILE, 1024), ID_Y, 1);
-            mma_commit(bar(BAR_Y));
-        }
-
-        // ---- x of this thread's outputs (for D x), kept before sX is reloaded
-        uint32_t xr[16];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const uint4 xv = *reinterpret_cast<const uint4*>(sm + K::OFF_X + swz(row, half * 4 + q));
-            xr[4 * q] = xv.x; xr[4 * q + 1] = xv.y; xr[4 * q + 2] = xv.z; xr[4 * q + 3] = xv.w;
-        }
-
-        // ---- h entering this block: the initial state, the previous chunk's
-        // published state, or the state this CTA left in the slot after its
-        // previous block of the same item (same thread, same addresses)
-        float hin[32];
-        float* slot = p.slots + ((long long)bh * N + row) * PD + half * 32;
-        if (j == 0 && c == 0) {
-            if (p.init_state) {
-                const long long o = ((long long)bh * N + row) * PD + half * 32;
-#pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    hin[i] = p.state_bf16 ? __bfloat162float(reinterpret_cast<const bf16*>(p.init_state)[o + i])
-                                          : reinterpret_cast<const float*>(p.init_state)[o + i];
-            } else {
-#pragma unroll
-                for (int i = 0; i < 32; ++i) hin[i] = 0.f;
-            }
-        } else {
-            if (j == 0) {
-                if (tid == 0) {
-                    // bounded wait for chunk c-1 of this (b, h); a wait that gives
-                    // up raises the launch-wide abort word so the others stop at once
+                for (int k = 0; k < N / 16; ++k) {
+                    const uint32_t o = (uint32_t)(k >> 2) * KBLOCK_K + (uint32_t)(k & 3) * KSTEP_K;
+                    if (k == 0) mma_ss<ID_S, 0>(tmem + COL_R, dC + o, dBk + o);
+                    else mma_ss<ID_S, 1>(tmem + COL_R, dC + o, dBk + o);
+                }
+                mma_commit(bar(BAR_S));
+                // ---- the chain: chunk c-1 of this (b, h) must have published its state
+                if (j == 0 && c > 0) {
                     const int* f = p.flags + bh;
                     const unsigned long long deadline = gtimer() + WAIT_NS;
                     uint32_t spins = 0;
@@ -486,144 +416,296 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                         __nanosleep(64);
                     }
                 }
-                psync();
-            }
+                mbar_arrive(bar(BAR_CHAIN));
+                // ---- chunk state S_c = B^T (w o X): hi pass then lo pass (K = 128 tokens)
+                wait(BAR_WX, ph);
+                tc_fence_after();
 #pragma unroll
-            for (int i = 0; i < 32; i += 4) {
-                const float4 v = __ldcg(reinterpret_cast<const float4*>(slot + i));
-                hin[i] = v.x; hin[i + 1] = v.y; hin[i + 2] = v.z; hin[i + 3] = v.w;
+                for (int k = 0; k < SUB / 16; ++k)
+                    if (k == 0) mma_ss<ID_ST, 0>(tmem + COL_ST, dBm, dW1);
+                    else mma_ss<ID_ST, 1>(tmem + COL_ST, dBm + k * KSTEP_MN, dW1 + k * KSTEP_MN);
+#pragma unroll
+                for (int k = 0; k < SUB / 16; ++k)
+                    mma_ss<ID_ST, 1>(tmem + COL_ST, dBm + k * KSTEP_MN, dW2 + k * KSTEP_MN);
+                mma_commit(bar(BAR_ST));
+                // ---- Y = M_hi X + M_lo X (A from TMEM, hi/lo interleaved per K step)
+                wait(BAR_M, ph);
+                tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < SUB / 16; ++k)
+                    if (k == 0) mma_ts<ID_Y, 0>(tmem + COL_Y, tmem + COL_R, dX);
+                    else mma_ts<ID_Y, 1>(tmem + COL_Y, tmem + COL_R + 16 * k, dX + k * KSTEP_MN);
+#pragma unroll
+                for (int k = 0; k < SUB / 16; ++k)
+                    mma_ts<ID_Y, 1>(tmem + COL_Y, tmem + COL_R + 16 * k + 8, dX + k * KSTEP_MN);
+                mma_commit(bar(BAR_Y));
+                // ---- publish (the compute warps stored the state before arriving), then Yoff = C h
+                wait(BAR_H, ph);
+                if (last_block && c < p.nchunks - 1) {
+                    __threadfence();
+                    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p.flags + bh), "r"(c + 1) : "memory");
+                }
+                wait(BAR_Y, ph);                      // Y has consumed M: region R is free
+                tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < N / 16; ++k) {
+                    const uint32_t o = (uint32_t)(k >> 2) * KBLOCK_K + (uint32_t)(k & 3) * KSTEP_K;
+                    if (k == 0) mma_ss<ID_OFF, 0>(tmem + COL_R, dC, dW1);
+                    else mma_ss<ID_OFF, 1>(tmem + COL_R, dC + o, dW1 + k * KSTEP_MN);
+                }
+#pragma unroll
+                for (int k = 0; k < N / 16; ++k) {
+                    const uint32_t o = (uint32_t)(k >> 2) * KBLOCK_K + (uint32_t)(k & 3) * KSTEP_K;
+                    mma_ss<ID_OFF, 1>(tmem + COL_R, dC + o, dW2 + k * KSTEP_MN);
+                }
+                mma_commit(bar(BAR_OFF));
+                // ---- next block: C, B, X, dt and the cumsum are all free once these MMAs are done
+                wait(BAR_OFF, ph);
+                if (!last_block) {
+                    ++j;
+                } else {
+                    item = atomicAdd(p.flags + p.BH + CTRL_TICKET, 1);
+                    j = 0;
+                }
+                load_block(item, j);
+                ++blk;
             }
         }
+    } else {
+        // ==================================================== compute warps
+        const float NEG_INF = __int_as_float(0xff800000u);
+        auto csync = [&]() { asm volatile("bar.sync %0, %1;" ::"r"(1 + pipe), "r"(NCOMPUTE) : "memory"); };
+        uint32_t blk = 0;
+        float prev_last = 0.f;   // raw cumsum at the end of the previous block of the same item
+        while (true) {
+            const uint32_t ph = blk & 1u;
+            wait(BAR_TMA, ph);
+            const int item = *s_item, j = *s_j;
+            if (item >= total) break;
+            const int c = item / p.BH, bh = item % p.BH;
+            const int b = bh / p.H, h = bh % p.H;
+            const bool last_block = (j == nblocks(item) - 1);
+            const long long t0 = (long long)c * p.Q + (long long)j * SUB;
 
-        // ---- h' = 2^(r_last) h + S_c (fp32): into the slot (for the next block, or
-        // published for the next chunk after the last block), or final_state
-        wait(BAR_ST, ph);
-        tc_fence_after();
-        {
-            uint32_t sv[32];
-            tmem_ld32(tmem + lane_off + COL_ST + half * 32, sv);
-            tmem_wait_ld();
-            const float dl = ex2(rlast);
-            float ho[32];
+            // ---- per-token decay terms (r relative to the block start, log2 units)
+            const float r0 = (j == 0) ? 0.f : prev_last;
+            const float rl = (s_acs[row] - r0) * LOG2E;
+            const float rlast = (s_acs[SUB - 1] - r0) * LOG2E;
+            if (half == 0) {
+                // dt folded into the exponent: dt_s 2^(x - r_s) = 2^(x + log2(dt_s) - r_s); dt_s = 0
+                // gives 0.  In place: this thread alone reads and writes element `row`.
+                const float d = scs[row];
+                scs[row] = (d > 0.f ? __log2f(d) : NEG_INF) - rl;
+            }
+            if (tid == 0) bulk_wait_read0();          // previous y store has read W1/W2
+            csync();
+            prev_last = s_acs[SUB - 1];
+
+            // ---- w o X split hi -> W1, lo -> W2
+            {
+                const float w = ex2(rlast + scs[row]);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) ho[i] = fmaf(dl, hin[i], __uint_as_float(sv[i]));
-            if (last_block && c == p.nchunks - 1) {
-                if (p.final_state) {
-                    const long long o = ((long long)bh * N + row) * PD + half * 32;
-                    if (p.state_bf16) {
-                        bf16* fs = reinterpret_cast<bf16*>(p.final_state) + o;
+                for (int q = 0; q < 4; ++q) {
+                    const uint32_t o = swz(row, half * 4 + q);
+                    const uint4 xv = *reinterpret_cast<const uint4*>(sm + K::OFF_X + o);
+                    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+                    uint32_t hw[4], lw[4];
 #pragma unroll
-                        for (int i = 0; i < 32; i += 8) Vec16<bf16>::store(fs + i, ho + i);
-                    } else {
-                        float* fs = reinterpret_cast<float*>(p.final_state) + o;
-#pragma unroll
-                        for (int i = 0; i < 32; i += 4)
-                            *reinterpret_cast<float4*>(fs + i) = make_float4(ho[i], ho[i + 1], ho[i + 2], ho[i + 3]);
+                    for (int e = 0; e < 4; ++e) {
+                        const float v0 = bf16_lo(xw[e]) * w, v1 = bf16_hi(xw[e]) * w;
+                        hw[e] = pack_bf16(v0, v1);
+                        lw[e] = pack_bf16(v0 - bf16_lo(hw[e]), v1 - bf16_hi(hw[e]));
                     }
+                    *reinterpret_cast<uint4*>(sm + K::OFF_W1 + o) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                    *reinterpret_cast<uint4*>(sm + K::OFF_W2 + o) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+                }
+            }
+            fence_proxy_async();
+            mbar_arrive(bar(BAR_WX));
+
+            // ---- M = S o [s<=l] 2^(r_l - r_s) dt_s, split hi/lo, written back in place:
+            // for every 16-column K step k of the MMA, hi goes to columns [16k, 16k+8)
+            // and lo to [16k+8, 16k+16) -- the S columns this thread just read.
+            // Column parts entirely above the diagonal for the whole warp are zero.
+            wait(BAR_S, ph);
+            tc_fence_after();
+            const int row_lo = (warp & 3) * 32;       // first row of this warp
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+                const int c0 = half * 64 + g * 16;    // one K step of the MMA: 16 columns
+                uint32_t v[16], o[16];
+                tmem_ld16(tmem + lane_off + COL_R + c0, v);
+                tmem_wait_ld();
+                if (c0 > row_lo + 31) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) o[i] = 0u;
+                } else {
+                    const float4* cs4 = reinterpret_cast<const float4*>(scs + c0);
+#pragma unroll
+                    for (int i4 = 0; i4 < 4; ++i4) {
+                        const float4 cv = cs4[i4];
+                        const float cvv[4] = {cv.x, cv.y, cv.z, cv.w};
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh) {
+                            const int i = i4 * 2 + hh;
+                            const int s0 = c0 + 2 * i;
+                            const float e0 = ex2(s0 <= row ? rl + cvv[2 * hh] : NEG_INF);
+                            const float e1 = ex2(s0 + 1 <= row ? rl + cvv[2 * hh + 1] : NEG_INF);
+                            const float m0 = __uint_as_float(v[2 * i]) * e0;
+                            const float m1 = __uint_as_float(v[2 * i + 1]) * e1;
+                            const uint32_t hi = pack_bf16(m0, m1);
+                            o[i] = hi;
+                            o[8 + i] = pack_bf16(m0 - bf16_lo(hi), m1 - bf16_hi(hi));
+                        }
+                    }
+                }
+                tmem_st16(tmem + lane_off + COL_R + c0, o);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar(BAR_M));
+
+            // ---- x of this thread's outputs (for D x), read before sX is reloaded
+            uint32_t xr[16];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const uint4 xv = *reinterpret_cast<const uint4*>(sm + K::OFF_X + swz(row, half * 4 + q));
+                xr[4 * q] = xv.x; xr[4 * q + 1] = xv.y; xr[4 * q + 2] = xv.z; xr[4 * q + 3] = xv.w;
+            }
+
+            // ---- h entering this block: the initial state, the previous chunk's
+            // published state, or the slot this thread wrote in the previous block of
+            // the same item (loads in flight while the state MMAs finish)
+            float hin[32];
+            float* slot = p.slots + ((long long)bh * N + row) * PD + half * 32;
+            wait(BAR_CHAIN, ph);
+            if (j == 0 && c == 0) {
+                if (p.init_state) {
+                    const long long o = ((long long)bh * N + row) * PD + half * 32;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        hin[i] = p.state_bf16 ? __bfloat162float(reinterpret_cast<const bf16*>(p.init_state)[o + i])
+                                              : reinterpret_cast<const float*>(p.init_state)[o + i];
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) hin[i] = 0.f;
                 }
             } else {
 #pragma unroll
-                for (int i = 0; i < 32; i += 4)
-                    __stcg(reinterpret_cast<float4*>(slot + i), make_float4(ho[i], ho[i + 1], ho[i + 2], ho[i + 3]));
+                for (int i = 0; i < 32; i += 4) {
+                    const float4 v = __ldcg(reinterpret_cast<const float4*>(slot + i));
+                    hin[i] = v.x; hin[i + 1] = v.y; hin[i + 2] = v.z; hin[i + 3] = v.w;
+                }
             }
-        }
-        // ---- h (entering the block) split hi -> W1, lo -> W2 (free: the state MMAs are done)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            uint32_t hw[4], lw[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float v0 = hin[q * 8 + 2 * e], v1 = hin[q * 8 + 2 * e + 1];
-                hw[e] = pack_bf16(v0, v1);
-                lw[e] = pack_bf16(v0 - bf16_lo(hw[e]), v1 - bf16_hi(hw[e]));
-            }
-            const uint32_t o = swz(row, half * 4 + q);
-            *reinterpret_cast<uint4*>(sm + K::OFF_W1 + o) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-            *reinterpret_cast<uint4*>(sm + K::OFF_W2 + o) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-        }
-        fence_proxy_async();
-        tc_fence_before();
-        psync();
-        // next block: the same item's next block, or the first block of the next ticket
-        const int next_item = last_block ? *s_next : item;
-        const int next_j = last_block ? 0 : j + 1;
-        if (tid == 0) {
-            tc_fence_after();
-            if (last_block && c < p.nchunks - 1) {
-                // every thread's slot stores precede the barrier above; the fence
-                // and release make them visible before the flag
-                __threadfence();
-                asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p.flags + bh), "r"(c + 1) : "memory");
-            }
-            // ---- Yoff = C h_hi + C h_lo (K = N) into region R, once Y has consumed M
-            wait(BAR_Y, ph);
-            tc_fence_after();
-#pragma unroll
-            for (int k = 0; k < N / 16; ++k) {
-                const uint32_t off = (uint32_t)(k >> 2) * TILE + (uint32_t)(k & 3) * 32u;
-                mma_ss(tmem + COL_R, sdesc(base + K::OFF_C + off, 16, 1024),
-                       sdesc(base + K::OFF_W1 + k * 2048, TILE, 1024), ID_OFF, k > 0);
-            }
-#pragma unroll
-            for (int k = 0; k < N / 16; ++k) {
-                const uint32_t off = (uint32_t)(k >> 2) * TILE + (uint32_t)(k & 3) * 32u;
-                mma_ss(tmem + COL_R, sdesc(base + K::OFF_C + off, 16, 1024),
-                       sdesc(base + K::OFF_W2 + k * 2048, TILE, 1024), ID_OFF, 1);
-            }
-            mma_commit(bar(BAR_OFF));
-        }
 
-        // ---- y = Y + 2^(r_l) Yoff + D x; the next block's loads overlap this epilogue
-        wait(BAR_OFF, ph);
-        tc_fence_after();
-        if (tid == 0 && next_item < total) issue_loads(next_item, next_j);   // C, B, X all free now
-        {
-            uint32_t yv[32], ov[32];
-            tmem_ld32(tmem + lane_off + COL_Y + half * 32, yv);
-            tmem_ld32(tmem + lane_off + COL_R + half * 32, ov);
-            tmem_wait_ld();
-            const float el = ex2(rl);
-            const float dsk = p.D ? p.D[h] : 0.f;
-            float out[32];
+            // ---- h' = 2^(r_last) h + S_c (fp32) -> slot or final_state; h split -> W1/W2
+            wait(BAR_ST, ph);
+            tc_fence_after();
+            {
+                const float dl = ex2(rlast);
+                const bool to_final = last_block && c == p.nchunks - 1;
+                const long long fo = ((long long)bh * N + row) * PD + half * 32;
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                out[2 * e] = __uint_as_float(yv[2 * e]) + el * __uint_as_float(ov[2 * e]) + dsk * bf16_lo(xr[e]);
-                out[2 * e + 1] =
-                    __uint_as_float(yv[2 * e + 1]) + el * __uint_as_float(ov[2 * e + 1]) + dsk * bf16_hi(xr[e]);
+                for (int pc = 0; pc < 2; ++pc) {
+                    uint32_t sv[16];
+                    tmem_ld16(tmem + lane_off + COL_ST + half * 32 + pc * 16, sv);
+                    tmem_wait_ld();
+                    float ho[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) ho[i] = fmaf(dl, hin[pc * 16 + i], __uint_as_float(sv[i]));
+                    if (to_final) {
+                        if (p.final_state) {
+                            if (p.state_bf16) {
+                                bf16* fs = reinterpret_cast<bf16*>(p.final_state) + fo + pc * 16;
+                                Vec16<bf16>::store(fs, ho);
+                                Vec16<bf16>::store(fs + 8, ho + 8);
+                            } else {
+                                float* fs = reinterpret_cast<float*>(p.final_state) + fo + pc * 16;
+#pragma unroll
+                                for (int i = 0; i < 16; i += 4)
+                                    *reinterpret_cast<float4*>(fs + i) = make_float4(ho[i], ho[i + 1], ho[i + 2], ho[i + 3]);
+                            }
+                        }
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 16; i += 4)
+                            __stcg(reinterpret_cast<float4*>(slot + pc * 16 + i),
+                                   make_float4(ho[i], ho[i + 1], ho[i + 2], ho[i + 3]));
+                    }
+                }
             }
-            // staging tiles: W1 (and W2 for the second fp32 half), free since OFF completed
-            if (p.y_bf16) {
 #pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    *reinterpret_cast<uint4*>(sm + K::OFF_W1 + swz(row, half * 4 + q)) = Vec16<bf16>::pack(out + 8 * q);
-            } else {
-                uint8_t* tile = sm + (half ? K::OFF_W2 : K::OFF_W1);
+            for (int q = 0; q < 4; ++q) {
+                uint32_t hw[4], lw[4];
 #pragma unroll
-                for (int q = 0; q < 8; ++q)
-                    *reinterpret_cast<float4*>(tile + swz(row, q)) =
-                        make_float4(out[4 * q], out[4 * q + 1], out[4 * q + 2], out[4 * q + 3]);
+                for (int e = 0; e < 4; ++e) {
+                    const float v0 = hin[q * 8 + 2 * e], v1 = hin[q * 8 + 2 * e + 1];
+                    hw[e] = pack_bf16(v0, v1);
+                    lw[e] = pack_bf16(v0 - bf16_lo(hw[e]), v1 - bf16_hi(hw[e]));
+                }
+                const uint32_t o = swz(row, half * 4 + q);
+                *reinterpret_cast<uint4*>(sm + K::OFF_W1 + o) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                *reinterpret_cast<uint4*>(sm + K::OFF_W2 + o) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
             }
+            fence_proxy_async();
+            mbar_arrive(bar(BAR_H));
+
+            // ---- y = Y + 2^(r_l) Yoff + D x, staged in W1/W2, TMA store
+            wait(BAR_OFF, ph);
+            tc_fence_after();
+            {
+                const float el = ex2(rl);
+                const float dsk = p.D ? p.D[h] : 0.f;
+#pragma unroll
+                for (int pc = 0; pc < 2; ++pc) {
+                    uint32_t yv[16], ov[16];
+                    tmem_ld16(tmem + lane_off + COL_Y + half * 32 + pc * 16, yv);
+                    tmem_ld16(tmem + lane_off + COL_R + half * 32 + pc * 16, ov);
+                    tmem_wait_ld();
+                    if (pc == 1) {
+                        tc_fence_before();
+                        mbar_arrive(bar(BAR_EPI));    // TMEM of this block may be reused
+                    }
+                    float out[16];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const uint32_t xw = xr[pc * 8 + e];
+                        out[2 * e] = __uint_as_float(yv[2 * e]) + el * __uint_as_float(ov[2 * e]) + dsk * bf16_lo(xw);
+                        out[2 * e + 1] =
+                            __uint_as_float(yv[2 * e + 1]) + el * __uint_as_float(ov[2 * e + 1]) + dsk * bf16_hi(xw);
+                    }
+                    if (p.y_bf16) {
+#pragma unroll
+                        for (int q = 0; q < 2; ++q)
+                            *reinterpret_cast<uint4*>(sm + K::OFF_W1 + swz(row, half * 4 + pc * 2 + q)) =
+                                Vec16<bf16>::pack(out + 8 * q);
+                    } else {
+                        uint8_t* tile = sm + (half ? K::OFF_W2 : K::OFF_W1);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            *reinterpret_cast<float4*>(tile + swz(row, pc * 4 + q)) =
+                                make_float4(out[4 * q], out[4 * q + 1], out[4 * q + 2], out[4 * q + 3]);
+                    }
+                }
+            }
+            fence_proxy_async();
+            csync();
+            if (tid == 0) {
+                tma_store_4d(&tmY, base + K::OFF_W1, 0, h, (int)t0, b);
+                if (!p.y_bf16) tma_store_4d(&tmY, base + K::OFF_W2, 32, h, (int)t0, b);
+                bulk_commit();
+            }
+            ++blk;
         }
-        fence_proxy_async();
-        tc_fence_before();
-        psync();
-        if (tid == 0) {
-            tma_store_4d(&tmY, base + K::OFF_W1, 0, h, (int)t0, b);
-            if (!p.y_bf16) tma_store_4d(&tmY, base + K::OFF_W2, 32, h, (int)t0, b);
-            bulk_commit();
-        }
-        item = next_item;
-        j = next_j;
-        ++blk;
+        if (tid == 0) bulk_wait0();   // the last y store is complete before the CTA leaves
     }
 
-    if (tid == 0) bulk_wait0();   // the last y store is complete before the CTA leaves
     if (err) atomicOr(p.dev_err, err);
     tc_fence_before();
     __syncthreads();
     if (threadIdx.x < 32) {
         tc_fence_after();
-        const uint32_t tmem_all = *reinterpret_cast<volatile uint32_t*>(smem_all + K::OFF_MISC);
+        const uint32_t tmem_all = *reinterpret_cast<volatile uint32_t*>(s_tmem_slot);
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_all), "r"(TMEM_COLS) : "memory");
     }
 }
