@@ -59,6 +59,10 @@ static ssd_status_t check_prefill_desc(const ssd_prefill_desc_t* d) {
         return SSD_ERR_UNSUPPORTED;
     if (d->nheads > (1 << 20) || d->batch > (1 << 24) || d->seqlen > ((int64_t)1 << 31))
         return SSD_ERR_UNSUPPORTED;
+    // 1-D grids: blocks over (batch*heads) x chunks x tiles must stay below 2^31
+    const int64_t nchunks = (d->seqlen + d->chunk - 1) / d->chunk;
+    const int64_t tiles = ((d->dstate + 63) / 64) * ((d->headdim + 63) / 64) * ((d->chunk + 63) / 64);
+    if (d->batch * d->nheads * nchunks * tiles >= ((int64_t)1 << 31)) return SSD_ERR_UNSUPPORTED;
     return SSD_OK;
 }
 

@@ -23,21 +23,22 @@
 namespace ssd {
 
 // --------------------------------------------------------------------------
-// dt and chunk-local decay cumsum.  grid (nchunks, b*H), block Q threads.
+// dt and chunk-local decay cumsum.  1-D grid over (b*H) x nchunks, block
+// max(Q, 32) threads.
 // --------------------------------------------------------------------------
 template <typename IoT>
 __global__ void dt_cumsum_kernel(const IoT* __restrict__ dt_raw, const float* __restrict__ dt_bias,
                                  const float* __restrict__ A, float* __restrict__ dt_out,
                                  float* __restrict__ acs_out, int* __restrict__ flags,
-                                 int64_t L, int64_t Lpad, int H, int Q, int nflags) {
+                                 int64_t L, int64_t Lpad, int H, int Q, int nflags, int nchunks, int BH) {
     __shared__ float warp_tot[32];
-    const int c = blockIdx.x;
-    const int bh = blockIdx.y;
+    const int c = (int)(blockIdx.x % (unsigned)nchunks);
+    const int bh = (int)(blockIdx.x / (unsigned)nchunks);
     const int b = bh / H, h = bh % H;
     const int l = threadIdx.x;
     const int64_t t = (int64_t)c * Q + l;
     float dt = 0.f, a = 0.f;
-    if (t < L) {
+    if (l < Q && t < L) {
         dt = softplus_f32(to_f32(dt_raw[((int64_t)b * L + t) * H + h]) + (dt_bias ? dt_bias[h] : 0.f));
         a = dt * A[h];
     }
@@ -64,11 +65,13 @@ __global__ void dt_cumsum_kernel(const IoT* __restrict__ dt_raw, const float* __
     __syncthreads();
     if (warp > 0) v += warp_tot[warp - 1];
     const int64_t o = (int64_t)bh * Lpad + t;
-    dt_out[o] = dt;
-    acs_out[o] = v;
+    if (l < Q) {
+        dt_out[o] = dt;
+        acs_out[o] = v;
+    }
     // reset the inter-chunk progress flags and control words of this launch
     if (c == 0) {
-        const int per = (nflags + gridDim.y - 1) / gridDim.y;
+        const int per = (nflags + BH - 1) / BH;
         for (int i = l; i < per; i += blockDim.x) {
             const int k = bh * per + i;
             if (k < nflags) flags[k] = 0;
@@ -82,9 +85,11 @@ static cudaError_t launch_dt_t(const PrefillArgs& a, cudaStream_t s) {
     float* acs = (float*)(a.ws + a.lay.off_acs);
     int* flags = (int*)(a.ws + a.lay.off_flags);
     const int nflags = (int)(a.batch * a.H + 64);
-    dim3 grid((unsigned)a.lay.nchunks, (unsigned)(a.batch * a.H));
-    dt_cumsum_kernel<IoT><<<grid, (unsigned)a.Q, 0, s>>>((const IoT*)a.dt_raw, a.dt_bias, a.A, dt, acs, flags,
-                                                        a.L, a.lay.Lpad, (int)a.H, (int)a.Q, nflags);
+    const unsigned blocks = (unsigned)(a.lay.nchunks * a.batch * a.H);
+    const unsigned threads = (unsigned)(a.Q < 32 ? 32 : a.Q);   // whole warps for the shuffles
+    dt_cumsum_kernel<IoT><<<blocks, threads, 0, s>>>((const IoT*)a.dt_raw, a.dt_bias, a.A, dt, acs, flags, a.L,
+                                                    a.lay.Lpad, (int)a.H, (int)a.Q, nflags, (int)a.lay.nchunks,
+                                                    (int)(a.batch * a.H));
     return cudaGetLastError();
 }
 
@@ -113,21 +118,23 @@ __device__ __forceinline__ void tile_fma(const float (*At)[TM + TPAD], const flo
 }
 
 // --------------------------------------------------------------------------
-// chunk_state.  grid (nchunks, b*H, ceil(N/64)*ceil(P/64)), block 256.
+// chunk_state.  1-D grid over nchunks x (b*H) x ceil(N/64)*ceil(P/64), block 256.
 // states[(bh*nchunks + c)][n][p] (fp32).
 // --------------------------------------------------------------------------
 template <typename IoT>
 __global__ void __launch_bounds__(256)
 chunk_state_kernel(const IoT* __restrict__ x, const IoT* __restrict__ Bm, const float* __restrict__ dtw,
                    const float* __restrict__ acsw, float* __restrict__ states, int64_t L, int64_t Lpad,
-                   int H, int P, int N, int G, int Q, int nchunks) {
+                   int H, int P, int N, int G, int Q, int nchunks, int ntiles) {
     __shared__ __align__(16) float At[TK][TM + TPAD];   // [s][n]
     __shared__ __align__(16) float Bt[TK][TM + TPAD];   // [s][p] scaled by w_s
     __shared__ float ws[256];
-    const int c = blockIdx.x, bh = blockIdx.y;
+    const int tile = (int)(blockIdx.x % (unsigned)ntiles);
+    const int c = (int)((blockIdx.x / (unsigned)ntiles) % (unsigned)nchunks);
+    const int bh = (int)(blockIdx.x / ((unsigned)ntiles * (unsigned)nchunks));
     const int b = bh / H, h = bh % H, g = h / (H / G);
     const int ptiles = (P + TM - 1) / TM;
-    const int n0 = (blockIdx.z / ptiles) * TM, p0 = (blockIdx.z % ptiles) * TM;
+    const int n0 = (tile / ptiles) * TM, p0 = (tile % ptiles) * TM;
     const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
     const int64_t base_t = (int64_t)c * Q;
     const float* dtc = dtw + (int64_t)bh * Lpad + base_t;
@@ -196,7 +203,7 @@ state_pass_kernel(float* __restrict__ states, const float* __restrict__ acsw,
 }
 
 // --------------------------------------------------------------------------
-// chunk_scan.  grid (nchunks * ceil(Q/64), b*H, ceil(P/64)), block 256.
+// chunk_scan.  1-D grid over nchunks*ceil(Q/64) x (b*H) x ceil(P/64), block 256.
 // --------------------------------------------------------------------------
 template <typename IoT, typename YT>
 __global__ void __launch_bounds__(256)
@@ -204,16 +211,18 @@ chunk_scan_kernel(const IoT* __restrict__ x, const IoT* __restrict__ Bm, const I
                   const float* __restrict__ Dv, const float* __restrict__ dtw,
                   const float* __restrict__ acsw, const float* __restrict__ states,
                   YT* __restrict__ y, int64_t L, int64_t Lpad, int H, int P, int N, int G, int Q,
-                  int nchunks) {
+                  int nchunks, int ptiles) {
     __shared__ __align__(16) float At[TK][TM + TPAD];
     __shared__ __align__(16) float Bt[TK][TM + TPAD];
     __shared__ __align__(16) float Mt[TM][TM + TPAD];   // [s][l] masked decay matrix
     __shared__ __align__(16) float Xs[TM][TM + TPAD];   // [s][p]
     __shared__ float acs_l[TM], acs_s[TM], dt_s[TM];
     const int rtiles = (Q + TM - 1) / TM;
-    const int c = blockIdx.x / rtiles, rt = blockIdx.x % rtiles;
-    const int bh = blockIdx.y, b = bh / H, h = bh % H, g = h / (H / G);
-    const int p0 = blockIdx.z * TM;
+    const unsigned crt = (unsigned)(nchunks * rtiles);
+    const int cr = (int)((blockIdx.x / (unsigned)ptiles) % crt);
+    const int c = cr / rtiles, rt = cr % rtiles;
+    const int bh = (int)(blockIdx.x / ((unsigned)ptiles * crt)), b = bh / H, h = bh % H, g = h / (H / G);
+    const int p0 = (int)(blockIdx.x % (unsigned)ptiles) * TM;
     const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
     const int l0 = rt * TM;                       // chunk-local first row of the tile
     const int64_t base_t = (int64_t)c * Q;
@@ -312,8 +321,8 @@ static cudaError_t launch_simt_t(const PrefillArgs& a, cudaStream_t s) {
     const int H = (int)a.H, P = (int)a.P, N = (int)a.N, G = (int)a.G, Q = (int)a.Q;
     const unsigned BH = (unsigned)(a.batch * a.H);
     const unsigned tiles_np = (unsigned)(((N + TM - 1) / TM) * ((P + TM - 1) / TM));
-    chunk_state_kernel<IoT><<<dim3(nc, BH, tiles_np), 256, 0, s>>>(
-        (const IoT*)a.x, (const IoT*)a.B, dt, acs, states, a.L, a.lay.Lpad, H, P, N, G, Q, nc);
+    chunk_state_kernel<IoT><<<(unsigned)(nc * BH * tiles_np), 256, 0, s>>>(
+        (const IoT*)a.x, (const IoT*)a.B, dt, acs, states, a.L, a.lay.Lpad, H, P, N, G, Q, nc, (int)tiles_np);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const int NP = N * P;
@@ -322,9 +331,10 @@ static cudaError_t launch_simt_t(const PrefillArgs& a, cudaStream_t s) {
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const unsigned rtiles = (unsigned)((Q + TM - 1) / TM);
-    chunk_scan_kernel<IoT, YT><<<dim3(nc * rtiles, BH, (unsigned)((P + TM - 1) / TM)), 256, 0, s>>>(
+    const unsigned ptiles = (unsigned)((P + TM - 1) / TM);
+    chunk_scan_kernel<IoT, YT><<<nc * rtiles * BH * ptiles, 256, 0, s>>>(
         (const IoT*)a.x, (const IoT*)a.B, (const IoT*)a.C, a.D, dt, acs, states, (YT*)a.y, a.L,
-        a.lay.Lpad, H, P, N, G, Q, nc);
+        a.lay.Lpad, H, P, N, G, Q, nc, (int)ptiles);
     return cudaGetLastError();
 }
 
