@@ -158,6 +158,39 @@ ssd_status_t ssd_chunk_scan_fwd(const ssd_prefill_desc_t* desc,
                                 const void* init_state, void* y, void* final_state,
                                 void* workspace, size_t workspace_bytes, void* stream);
 
+/* Size of the scratch array ssd_chunk_scan_fwd_noalloc uses (32 MiB per GPU). */
+#define SSD_NOALLOC_WORKSPACE_BYTES ((size_t)32 << 20)
+
+/*
+ * ssd_chunk_scan_fwd without a caller workspace, for callers that cannot
+ * allocate device memory: code that may only touch the input and output
+ * buffers it is given (for example a plugin inside a framework that owns all
+ * device memory), or a path where cudaMalloc -- which can synchronise the
+ * device -- is not allowed.  The pages describe no such variant; this is a
+ * convenience of the library.
+ *
+ * Arguments and results are exactly those of ssd_chunk_scan_fwd minus the
+ * workspace.  The scratch is a fixed array of SSD_NOALLOC_WORKSPACE_BYTES in
+ * the library's own device memory, reserved on every GPU that loads the
+ * library until the process exits; nothing is allocated per call (no
+ * cudaMalloc, cudaFree or allocating library routine).
+ *  - Problems whose ssd_chunk_scan_workspace_size exceeds the scratch are
+ *    rejected with SSD_ERR_WORKSPACE before anything is launched (the 1.3B-
+ *    shaped layer, batch 4 x 2048 tokens, needs about 12.6 MiB).
+ *  - The first call with a given device current looks up the scratch's device
+ *    address on that device; make that first call before any stream capture.
+ *  - Every call on a device shares the one scratch array, which keeps the last
+ *    call's contents (the kernels reset what must start at zero themselves).
+ *    Calls that overlap on the GPU -- on different streams, or from different
+ *    threads -- race on it: serialise them.
+ * Errors: as ssd_chunk_scan_fwd, plus SSD_ERR_WORKSPACE for a problem too
+ * large for the scratch, SSD_ERR_CUDA if the scratch cannot be located.
+ */
+ssd_status_t ssd_chunk_scan_fwd_noalloc(const ssd_prefill_desc_t* desc,
+                                        const void* x, const void* dt_raw, const float* dt_bias,
+                                        const float* A, const void* B, const void* C, const float* D,
+                                        const void* init_state, void* y, void* final_state, void* stream);
+
 /*
  * Single-token decode step, in place on the state ("Mamba-2 vs Transformers /
  * SSD", section "How to decide...": O(1) recurrent step; "Mamba3", section on

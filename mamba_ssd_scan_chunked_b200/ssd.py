@@ -26,7 +26,10 @@ STATUS = {0: "SSD_OK", 1: "SSD_ERR_INVALID_ARG", 2: "SSD_ERR_UNSUPPORTED", 3: "S
 
 # every symbol include/ssd.h declares
 EXPORTS = ("ssd_version", "ssd_status_string", "ssd_chunk_scan_workspace_size", "ssd_chunk_scan_path",
-           "ssd_chunk_scan_fwd", "ssd_state_update", "ssd_get_device_error")
+           "ssd_chunk_scan_fwd", "ssd_chunk_scan_fwd_noalloc", "ssd_state_update", "ssd_get_device_error")
+
+# scratch size of ssd_chunk_scan_fwd_noalloc (SSD_NOALLOC_WORKSPACE_BYTES)
+NOALLOC_WORKSPACE_BYTES = 32 << 20
 
 
 class SsdError(RuntimeError):
@@ -72,6 +75,8 @@ def lib():
             L.ssd_chunk_scan_path.argtypes = [ctypes.POINTER(PrefillDesc), ctypes.POINTER(ctypes.c_int32)]
             L.ssd_chunk_scan_fwd.restype = ctypes.c_int
             L.ssd_chunk_scan_fwd.argtypes = [ctypes.POINTER(PrefillDesc)] + [_VP] * 10 + [_VP, ctypes.c_size_t, _VP]
+            L.ssd_chunk_scan_fwd_noalloc.restype = ctypes.c_int
+            L.ssd_chunk_scan_fwd_noalloc.argtypes = [ctypes.POINTER(PrefillDesc)] + [_VP] * 11
             L.ssd_state_update.restype = ctypes.c_int
             L.ssd_state_update.argtypes = [ctypes.POINTER(DecodeDesc)] + [_VP] * 10
             L.ssd_get_device_error.restype = ctypes.c_int
@@ -113,6 +118,13 @@ def ssd_chunk_scan_fwd(desc, x, dt_raw, dt_bias, A, B, C, D, init_state, y, fina
     return lib().ssd_chunk_scan_fwd(ctypes.byref(desc), x or None, dt_raw or None, dt_bias or None, A or None,
                                      B or None, C or None, D or None, init_state or None, y or None,
                                      final_state or None, workspace or None, int(workspace_bytes), stream or None)
+
+
+def ssd_chunk_scan_fwd_noalloc(desc, x, dt_raw, dt_bias, A, B, C, D, init_state, y, final_state, stream) -> int:
+    """Raw call of the variant without a caller workspace; returns the status code."""
+    return lib().ssd_chunk_scan_fwd_noalloc(ctypes.byref(desc), x or None, dt_raw or None, dt_bias or None, A or None,
+                                            B or None, C or None, D or None, init_state or None, y or None,
+                                            final_state or None, stream or None)
 
 
 def ssd_state_update(desc, state, x, dt_raw, dt_bias, A, B, C, D, y, stream) -> int:
