@@ -86,7 +86,7 @@ struct Cfg {
     // small area of one pipeline (after the tiles of all pipelines)
     static constexpr uint32_t OFF_ACS = 0;                   // chunk-local cumsum of the block [128] (TMA)
     static constexpr uint32_t OFF_DTCS = OFF_ACS + 512;      // dt [128] (TMA), turned into log2(dt_s) - r_s
-    static constexpr uint32_t OFF_BAR = OFF_DTCS + 512;      // mbarriers
+    static constexpr uint32_t OFF_BAR = OFF_DTCS + 512;      // mbarriers (10)
     static constexpr uint32_t OFF_MISC = OFF_BAR + 80;       // tmem base, block coordinates
     static constexpr uint32_t SMALL = OFF_MISC + 64;
     static constexpr uint32_t SMEM = PIPES * (TILES + SMALL);
@@ -273,8 +273,14 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
 // pipeline = 8 compute warps (256 threads; thread = one TMEM lane/tile row and
 // one half of its columns) + 1 control warp whose lane 0 takes tickets,
 // issues every TMA and MMA, waits for the previous chunk of the chain and
-// publishes.  Compute and control meet only at mbarriers; the control warp
-// loads block n+1 as soon as the MMAs of block n are done.
+// publishes.  Compute and control meet only at mbarriers.
+//
+// Per 128-token block the state accumulator (TMEM) is first loaded with
+// 2^(r_last) h and the chunk-state MMAs accumulate onto it, so h' stays in
+// TMEM for the next block of the item; C h is computed first into the Y
+// accumulator, scaled by 2^(r_l) in place, and M X accumulates on top.  Region
+// R only holds S/M, so the next block's loads and C B^T start as soon as Y is
+// done, overlapping this block's epilogue.
 template <int N>
 __global__ void __launch_bounds__(THREADS, 1)
 ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
@@ -300,7 +306,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
     volatile int* s_item = reinterpret_cast<volatile int*>(ss + K::OFF_MISC + 4);
     volatile int* s_j = reinterpret_cast<volatile int*>(ss + K::OFF_MISC + 8);
     uint8_t* s_tmem_slot = smem_all + PIPES * K::TILES + K::OFF_MISC;    // pipeline 0's misc word
-    enum { BAR_TMA = 0, BAR_S, BAR_WX, BAR_ST, BAR_M, BAR_CHAIN, BAR_Y, BAR_H, BAR_OFF, BAR_EPI, NBAR };
+    enum { BAR_TMA = 0, BAR_S, BAR_CHAIN, BAR_H, BAR_OFF, BAR_WX, BAR_M, BAR_Y, BAR_PUB, BAR_EPI, NBAR };
     auto bar = [&](int i) -> uint32_t { return sbase + K::OFF_BAR + 8u * (uint32_t)i; };
     volatile int* g_abort = reinterpret_cast<volatile int*>(p.flags + p.BH + CTRL_ABORT);
     const int total = p.nchunks * p.BH;
@@ -319,7 +325,8 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     if (!control && tid == 0) {
-        const uint32_t cnt[NBAR] = {1, 1, NCOMPUTE, 1, NCOMPUTE, 1, 1, NCOMPUTE, 1, NCOMPUTE};
+        //                        TMA S  CHAIN H         OFF WX        M         Y  PUB       EPI
+        const uint32_t cnt[NBAR] = {1, 1, 1, NCOMPUTE, 1, NCOMPUTE, NCOMPUTE, 1, NCOMPUTE, NCOMPUTE};
         for (int i = 0; i < NBAR; ++i) mbar_init(bar(i), cnt[i]);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -344,6 +351,18 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
             constexpr uint32_t ID_ST = idesc_bf16(128, PD, true, true);     // B^T (MN-major) x wX (MN-major)
             constexpr uint32_t ID_Y = idesc_bf16(128, PD, false, true);     // M (TMEM) x X (MN-major)
             constexpr uint32_t ID_OFF = idesc_bf16(128, PD, false, true);   // C (K-major) x h (MN-major)
+            // Shared-memory descriptors, built once: a K step of a K-major operand
+            // advances the start address by 32 B (+2 in the descriptor), a 64-wide
+            // K block by one tile (+TILE/16); a K step of an MN-major operand by 16
+            // rows of 128 B (+128).  The 14-bit address field cannot overflow:
+            // every shared address is below 2^18.
+            const uint64_t dC = sdesc(base + K::OFF_C, 16, 1024);       // K-major (S, Yoff)
+            const uint64_t dBk = sdesc(base + K::OFF_B, 16, 1024);      // K-major (S)
+            const uint64_t dBm = sdesc(base + K::OFF_B, TILE, 1024);    // MN-major (state)
+            const uint64_t dX = sdesc(base + K::OFF_X, TILE, 1024);     // MN-major (Y)
+            const uint64_t dW1 = sdesc(base + K::OFF_W1, TILE, 1024);   // MN-major (state, Yoff)
+            const uint64_t dW2 = sdesc(base + K::OFF_W2, TILE, 1024);
+            constexpr uint32_t KSTEP_K = 2, KBLOCK_K = TILE >> 4, KSTEP_MN = 2048 >> 4;
             // publish the block's coordinates, then load its operands and per-token terms
             auto load_block = [&](int it, int j) {
                 *s_item = it;
@@ -367,18 +386,6 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                 bulk_load(sbase + K::OFF_ACS, p.acsw + o, SUB * 4, bar(BAR_TMA));
                 bulk_load(sbase + K::OFF_DTCS, p.dtw + o, SUB * 4, bar(BAR_TMA));
             };
-            // Shared-memory descriptors, built once: a K step of a K-major operand
-            // advances the start address by 32 B (+2 in the descriptor), a 64-wide
-            // K block by one tile (+TILE/16); a K step of an MN-major operand by 16
-            // rows of 128 B (+128).  The 14-bit address field cannot overflow:
-            // every shared address is below 2^18.
-            const uint64_t dC = sdesc(base + K::OFF_C, 16, 1024);       // K-major (S, Yoff)
-            const uint64_t dBk = sdesc(base + K::OFF_B, 16, 1024);      // K-major (S)
-            const uint64_t dBm = sdesc(base + K::OFF_B, TILE, 1024);    // MN-major (state)
-            const uint64_t dX = sdesc(base + K::OFF_X, TILE, 1024);     // MN-major (Y)
-            const uint64_t dW1 = sdesc(base + K::OFF_W1, TILE, 1024);   // MN-major (state, Yoff)
-            const uint64_t dW2 = sdesc(base + K::OFF_W2, TILE, 1024);
-            constexpr uint32_t KSTEP_K = 2, KBLOCK_K = TILE >> 4, KSTEP_MN = 2048 >> 4;
             int item = atomicAdd(p.flags + p.BH + CTRL_TICKET, 1);
             int j = 0;
             load_block(item, 0);
@@ -388,9 +395,8 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                 const int c = item / p.BH, bh = item % p.BH;
                 const bool last_block = (j == nblocks(item) - 1);
                 wait(BAR_TMA, ph);
-                if (blk > 0) wait(BAR_EPI, ph ^ 1u);   // block n-1 finished reading TMEM
                 tc_fence_after();
-                // ---- S = C B^T (K = N)
+                // ---- S = C B^T (K = N) into region R (free: the previous Y is done)
 #pragma unroll
                 for (int k = 0; k < N / 16; ++k) {
                     const uint32_t o = (uint32_t)(k >> 2) * KBLOCK_K + (uint32_t)(k & 3) * KSTEP_K;
@@ -417,50 +423,47 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                     }
                 }
                 mbar_arrive(bar(BAR_CHAIN));
-                // ---- chunk state S_c = B^T (w o X): hi pass then lo pass (K = 128 tokens)
+                // ---- Yoff = C h_hi + C h_lo into the Y accumulator (once the previous
+                // block's epilogue has read it)
+                if (blk > 0) wait(BAR_EPI, ph ^ 1u);
+                wait(BAR_H, ph);
+                tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < N / 16; ++k) {
+                    const uint32_t o = (uint32_t)(k >> 2) * KBLOCK_K + (uint32_t)(k & 3) * KSTEP_K;
+                    if (k == 0) mma_ss<ID_OFF, 0>(tmem + COL_Y, dC, dW1);
+                    else mma_ss<ID_OFF, 1>(tmem + COL_Y, dC + o, dW1 + k * KSTEP_MN);
+                }
+#pragma unroll
+                for (int k = 0; k < N / 16; ++k) {
+                    const uint32_t o = (uint32_t)(k >> 2) * KBLOCK_K + (uint32_t)(k & 3) * KSTEP_K;
+                    mma_ss<ID_OFF, 1>(tmem + COL_Y, dC + o, dW2 + k * KSTEP_MN);
+                }
+                mma_commit(bar(BAR_OFF));
+                // ---- state: onto 2^(r_last) h (written by the compute warps) accumulate
+                // B^T (w o X)_hi and B^T (w o X)_lo (K = 128 tokens)
                 wait(BAR_WX, ph);
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < SUB / 16; ++k)
-                    if (k == 0) mma_ss<ID_ST, 0>(tmem + COL_ST, dBm, dW1);
-                    else mma_ss<ID_ST, 1>(tmem + COL_ST, dBm + k * KSTEP_MN, dW1 + k * KSTEP_MN);
+                    mma_ss<ID_ST, 1>(tmem + COL_ST, dBm + k * KSTEP_MN, dW1 + k * KSTEP_MN);
 #pragma unroll
                 for (int k = 0; k < SUB / 16; ++k)
                     mma_ss<ID_ST, 1>(tmem + COL_ST, dBm + k * KSTEP_MN, dW2 + k * KSTEP_MN);
-                mma_commit(bar(BAR_ST));
-                // ---- Y = M_hi X + M_lo X (A from TMEM, hi/lo interleaved per K step)
+                // ---- Y += M_hi X + M_lo X onto the scaled Yoff (A from TMEM)
                 wait(BAR_M, ph);
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < SUB / 16; ++k)
-                    if (k == 0) mma_ts<ID_Y, 0>(tmem + COL_Y, tmem + COL_R, dX);
-                    else mma_ts<ID_Y, 1>(tmem + COL_Y, tmem + COL_R + 16 * k, dX + k * KSTEP_MN);
+                    mma_ts<ID_Y, 1>(tmem + COL_Y, tmem + COL_R + 16 * k, dX + k * KSTEP_MN);
 #pragma unroll
                 for (int k = 0; k < SUB / 16; ++k)
                     mma_ts<ID_Y, 1>(tmem + COL_Y, tmem + COL_R + 16 * k + 8, dX + k * KSTEP_MN);
                 mma_commit(bar(BAR_Y));
-                // ---- publish (the compute warps stored the state before arriving), then Yoff = C h
-                wait(BAR_H, ph);
-                if (last_block && c < p.nchunks - 1) {
-                    __threadfence();
-                    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p.flags + bh), "r"(c + 1) : "memory");
-                }
-                wait(BAR_Y, ph);                      // Y has consumed M: region R is free
-                tc_fence_after();
-#pragma unroll
-                for (int k = 0; k < N / 16; ++k) {
-                    const uint32_t o = (uint32_t)(k >> 2) * KBLOCK_K + (uint32_t)(k & 3) * KSTEP_K;
-                    if (k == 0) mma_ss<ID_OFF, 0>(tmem + COL_R, dC, dW1);
-                    else mma_ss<ID_OFF, 1>(tmem + COL_R, dC + o, dW1 + k * KSTEP_MN);
-                }
-#pragma unroll
-                for (int k = 0; k < N / 16; ++k) {
-                    const uint32_t o = (uint32_t)(k >> 2) * KBLOCK_K + (uint32_t)(k & 3) * KSTEP_K;
-                    mma_ss<ID_OFF, 1>(tmem + COL_R, dC + o, dW2 + k * KSTEP_MN);
-                }
-                mma_commit(bar(BAR_OFF));
-                // ---- next block: C, B, X, dt and the cumsum are all free once these MMAs are done
-                wait(BAR_OFF, ph);
+                // ---- next block: C, B, X, dt and the cumsum are free once Y is done
+                wait(BAR_Y, ph);
+                const int cur_item = item;
+                const int cur_c = c, cur_bh = bh;
                 if (!last_block) {
                     ++j;
                 } else {
@@ -468,6 +471,14 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                     j = 0;
                 }
                 load_block(item, j);
+                // ---- publish after the compute warps stored the state of the item's last block
+                wait(BAR_PUB, ph);
+                if (last_block && cur_c < p.nchunks - 1) {
+                    __threadfence();
+                    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p.flags + cur_bh), "r"(cur_c + 1)
+                                 : "memory");
+                }
+                (void)cur_item;
                 ++blk;
             }
         }
@@ -501,27 +512,62 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
             csync();
             prev_last = s_acs[SUB - 1];
 
-            // ---- w o X split hi -> W1, lo -> W2
+            // ---- h entering the block: the initial state or the previous chunk's
+            // published state (first block of an item), else the state the
+            // previous block left in the TMEM accumulator.  Split hi -> W1, lo -> W2
+            // for C h; 2^(r_last) h -> the state accumulator.
             {
-                const float w = ex2(rlast + scs[row]);
+                const float dl = ex2(rlast);
+                float* slot = p.slots + ((long long)bh * N + row) * PD + half * 32;
+                if (j == 0) wait(BAR_CHAIN, ph);
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const uint32_t o = swz(row, half * 4 + q);
-                    const uint4 xv = *reinterpret_cast<const uint4*>(sm + K::OFF_X + o);
-                    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-                    uint32_t hw[4], lw[4];
+                for (int pc = 0; pc < 2; ++pc) {
+                    float hv[16];
+                    if (j > 0) {
+                        uint32_t v[16];
+                        tmem_ld16(tmem + lane_off + COL_ST + half * 32 + pc * 16, v);
+                        tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float v0 = bf16_lo(xw[e]) * w, v1 = bf16_hi(xw[e]) * w;
-                        hw[e] = pack_bf16(v0, v1);
-                        lw[e] = pack_bf16(v0 - bf16_lo(hw[e]), v1 - bf16_hi(hw[e]));
+                        for (int i = 0; i < 16; ++i) hv[i] = __uint_as_float(v[i]);
+                    } else if (c > 0) {
+#pragma unroll
+                        for (int i = 0; i < 16; i += 4) {
+                            const float4 v = __ldcg(reinterpret_cast<const float4*>(slot + pc * 16 + i));
+                            hv[i] = v.x; hv[i + 1] = v.y; hv[i + 2] = v.z; hv[i + 3] = v.w;
+                        }
+                    } else if (p.init_state) {
+                        const long long o = ((long long)bh * N + row) * PD + half * 32 + pc * 16;
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            hv[i] = p.state_bf16 ? __bfloat162float(reinterpret_cast<const bf16*>(p.init_state)[o + i])
+                                                 : reinterpret_cast<const float*>(p.init_state)[o + i];
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) hv[i] = 0.f;
                     }
-                    *reinterpret_cast<uint4*>(sm + K::OFF_W1 + o) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-                    *reinterpret_cast<uint4*>(sm + K::OFF_W2 + o) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+                    uint32_t sc[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) sc[i] = __float_as_uint(dl * hv[i]);
+                    tmem_st16(tmem + lane_off + COL_ST + half * 32 + pc * 16, sc);
+#pragma unroll
+                    for (int q = 0; q < 2; ++q) {
+                        uint32_t hw[4], lw[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float v0 = hv[q * 8 + 2 * e], v1 = hv[q * 8 + 2 * e + 1];
+                            hw[e] = pack_bf16(v0, v1);
+                            lw[e] = pack_bf16(v0 - bf16_lo(hw[e]), v1 - bf16_hi(hw[e]));
+                        }
+                        const uint32_t o = swz(row, half * 4 + pc * 2 + q);
+                        *reinterpret_cast<uint4*>(sm + K::OFF_W1 + o) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                        *reinterpret_cast<uint4*>(sm + K::OFF_W2 + o) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+                    }
                 }
+                tmem_wait_st();
+                fence_proxy_async();
+                tc_fence_before();
+                mbar_arrive(bar(BAR_H));
             }
-            fence_proxy_async();
-            mbar_arrive(bar(BAR_WX));
 
             // ---- M = S o [s<=l] 2^(r_l - r_s) dt_s, split hi/lo, written back in place:
             // for every 16-column K step k of the MMA, hi goes to columns [16k, 16k+8)
@@ -561,60 +607,64 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                 }
                 tmem_st16(tmem + lane_off + COL_R + c0, o);
             }
+
+            // ---- scale Yoff by 2^(r_l) in place (the Y MMAs accumulate on top)
+            const float el = ex2(rl);
+            wait(BAR_OFF, ph);
+            tc_fence_after();
+#pragma unroll
+            for (int pc = 0; pc < 2; ++pc) {
+                uint32_t v[16];
+                tmem_ld16(tmem + lane_off + COL_Y + half * 32 + pc * 16, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(el * __uint_as_float(v[i]));
+                tmem_st16(tmem + lane_off + COL_Y + half * 32 + pc * 16, v);
+            }
+            // ---- w o X split hi -> W1, lo -> W2 (free: C h is done); x kept for D x
+            uint32_t xr[16];
+            {
+                const float w = ex2(rlast + scs[row]);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const uint32_t o = swz(row, half * 4 + q);
+                    const uint4 xv = *reinterpret_cast<const uint4*>(sm + K::OFF_X + o);
+                    xr[4 * q] = xv.x; xr[4 * q + 1] = xv.y; xr[4 * q + 2] = xv.z; xr[4 * q + 3] = xv.w;
+                    uint32_t hw[4], lw[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float v0 = bf16_lo(xr[4 * q + e]) * w, v1 = bf16_hi(xr[4 * q + e]) * w;
+                        hw[e] = pack_bf16(v0, v1);
+                        lw[e] = pack_bf16(v0 - bf16_lo(hw[e]), v1 - bf16_hi(hw[e]));
+                    }
+                    *reinterpret_cast<uint4*>(sm + K::OFF_W1 + o) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                    *reinterpret_cast<uint4*>(sm + K::OFF_W2 + o) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+                }
+            }
             tmem_wait_st();
+            fence_proxy_async();
             tc_fence_before();
+            mbar_arrive(bar(BAR_WX));
             mbar_arrive(bar(BAR_M));
 
-            // ---- x of this thread's outputs (for D x), read before sX is reloaded
-            uint32_t xr[16];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const uint4 xv = *reinterpret_cast<const uint4*>(sm + K::OFF_X + swz(row, half * 4 + q));
-                xr[4 * q] = xv.x; xr[4 * q + 1] = xv.y; xr[4 * q + 2] = xv.z; xr[4 * q + 3] = xv.w;
-            }
-
-            // ---- h entering this block: the initial state, the previous chunk's
-            // published state, or the slot this thread wrote in the previous block of
-            // the same item (loads in flight while the state MMAs finish)
-            float hin[32];
-            float* slot = p.slots + ((long long)bh * N + row) * PD + half * 32;
-            wait(BAR_CHAIN, ph);
-            if (j == 0 && c == 0) {
-                if (p.init_state) {
-                    const long long o = ((long long)bh * N + row) * PD + half * 32;
-#pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        hin[i] = p.state_bf16 ? __bfloat162float(reinterpret_cast<const bf16*>(p.init_state)[o + i])
-                                              : reinterpret_cast<const float*>(p.init_state)[o + i];
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) hin[i] = 0.f;
-                }
-            } else {
-#pragma unroll
-                for (int i = 0; i < 32; i += 4) {
-                    const float4 v = __ldcg(reinterpret_cast<const float4*>(slot + i));
-                    hin[i] = v.x; hin[i + 1] = v.y; hin[i + 2] = v.z; hin[i + 3] = v.w;
-                }
-            }
-
-            // ---- h' = 2^(r_last) h + S_c (fp32) -> slot or final_state; h split -> W1/W2
-            wait(BAR_ST, ph);
+            // ---- after Y (and the state MMAs before it): publish the item's state,
+            // then y = (2^(r_l) Yoff + M X) + D x, staged in W1/W2, TMA store
+            wait(BAR_Y, ph);
             tc_fence_after();
-            {
-                const float dl = ex2(rlast);
-                const bool to_final = last_block && c == p.nchunks - 1;
+            if (last_block) {
+                const bool to_final = c == p.nchunks - 1;
                 const long long fo = ((long long)bh * N + row) * PD + half * 32;
+                float* slot = p.slots + fo;
 #pragma unroll
                 for (int pc = 0; pc < 2; ++pc) {
                     uint32_t sv[16];
                     tmem_ld16(tmem + lane_off + COL_ST + half * 32 + pc * 16, sv);
                     tmem_wait_ld();
-                    float ho[16];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) ho[i] = fmaf(dl, hin[pc * 16 + i], __uint_as_float(sv[i]));
                     if (to_final) {
                         if (p.final_state) {
+                            float ho[16];
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) ho[i] = __uint_as_float(sv[i]);
                             if (p.state_bf16) {
                                 bf16* fs = reinterpret_cast<bf16*>(p.final_state) + fo + pc * 16;
                                 Vec16<bf16>::store(fs, ho);
@@ -630,49 +680,29 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
 #pragma unroll
                         for (int i = 0; i < 16; i += 4)
                             __stcg(reinterpret_cast<float4*>(slot + pc * 16 + i),
-                                   make_float4(ho[i], ho[i + 1], ho[i + 2], ho[i + 3]));
+                                   make_float4(__uint_as_float(sv[i]), __uint_as_float(sv[i + 1]),
+                                               __uint_as_float(sv[i + 2]), __uint_as_float(sv[i + 3])));
                     }
                 }
             }
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                uint32_t hw[4], lw[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float v0 = hin[q * 8 + 2 * e], v1 = hin[q * 8 + 2 * e + 1];
-                    hw[e] = pack_bf16(v0, v1);
-                    lw[e] = pack_bf16(v0 - bf16_lo(hw[e]), v1 - bf16_hi(hw[e]));
-                }
-                const uint32_t o = swz(row, half * 4 + q);
-                *reinterpret_cast<uint4*>(sm + K::OFF_W1 + o) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-                *reinterpret_cast<uint4*>(sm + K::OFF_W2 + o) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-            }
-            fence_proxy_async();
-            mbar_arrive(bar(BAR_H));
-
-            // ---- y = Y + 2^(r_l) Yoff + D x, staged in W1/W2, TMA store
-            wait(BAR_OFF, ph);
-            tc_fence_after();
+            mbar_arrive(bar(BAR_PUB));
             {
-                const float el = ex2(rl);
                 const float dsk = p.D ? p.D[h] : 0.f;
 #pragma unroll
                 for (int pc = 0; pc < 2; ++pc) {
-                    uint32_t yv[16], ov[16];
+                    uint32_t yv[16];
                     tmem_ld16(tmem + lane_off + COL_Y + half * 32 + pc * 16, yv);
-                    tmem_ld16(tmem + lane_off + COL_R + half * 32 + pc * 16, ov);
                     tmem_wait_ld();
                     if (pc == 1) {
                         tc_fence_before();
-                        mbar_arrive(bar(BAR_EPI));    // TMEM of this block may be reused
+                        mbar_arrive(bar(BAR_EPI));    // the Y accumulator may be reused
                     }
                     float out[16];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         const uint32_t xw = xr[pc * 8 + e];
-                        out[2 * e] = __uint_as_float(yv[2 * e]) + el * __uint_as_float(ov[2 * e]) + dsk * bf16_lo(xw);
-                        out[2 * e + 1] =
-                            __uint_as_float(yv[2 * e + 1]) + el * __uint_as_float(ov[2 * e + 1]) + dsk * bf16_hi(xw);
+                        out[2 * e] = __uint_as_float(yv[2 * e]) + dsk * bf16_lo(xw);
+                        out[2 * e + 1] = __uint_as_float(yv[2 * e + 1]) + dsk * bf16_hi(xw);
                     }
                     if (p.y_bf16) {
 #pragma unroll
