@@ -106,6 +106,7 @@ struct Params {
     unsigned* dev_err;
     long long L, Lpad;
     int H, G, Q, nchunks, BH;
+    int K, nruns;           // a work item = one (b, h) and a run of K consecutive chunks
     int state_bf16, y_bf16;
 };
 
@@ -309,7 +310,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
     enum { BAR_TMA = 0, BAR_S, BAR_CHAIN, BAR_H, BAR_OFF, BAR_WX, BAR_M, BAR_Y, BAR_PUB, BAR_EPI, NBAR };
     auto bar = [&](int i) -> uint32_t { return sbase + K::OFF_BAR + 8u * (uint32_t)i; };
     volatile int* g_abort = reinterpret_cast<volatile int*>(p.flags + p.BH + CTRL_ABORT);
-    const int total = p.nchunks * p.BH;
+    const int total = p.nruns * p.BH;
     unsigned err = 0;
 
     // the 128-byte swizzle of TMA and of the MMA descriptors assumes 1024-byte
@@ -338,10 +339,12 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
     auto wait = [&](int i, uint32_t ph) {
         if (!mbar_wait(bar(i), ph)) err |= kErrAsyncTimeout;
     };
-    auto nblocks = [&](int it) -> int {
-        const long long rem = p.L - (long long)(it / p.BH) * p.Q;
-        const int n = (int)((rem + SUB - 1) / SUB);
-        return n < p.Q / SUB ? n : p.Q / SUB;
+    // item = run r (chunks [rK, rK+K)) of sequence bh; tickets are run-major, so
+    // run r-1 of the same sequence always holds an earlier ticket
+    auto nblocks = [&](int it) -> int {       // 128-token blocks of the run (never straddle a chunk)
+        const long long t_first = (long long)(it / p.BH) * p.K * p.Q;
+        const long long len = p.L - t_first < (long long)p.K * p.Q ? p.L - t_first : (long long)p.K * p.Q;
+        return (int)((len + SUB - 1) / SUB);
     };
 
     if (control) {
@@ -371,9 +374,9 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                     mbar_arrive(bar(BAR_TMA));
                     return;
                 }
-                const int c_ = it / p.BH, bh_ = it % p.BH;
+                const int r_ = it / p.BH, bh_ = it % p.BH;
                 const int b_ = bh_ / p.H, h_ = bh_ % p.H, g_ = h_ / (p.H / p.G);
-                const int t0_ = c_ * p.Q + j * SUB;
+                const int t0_ = r_ * p.K * p.Q + j * SUB;
                 fence_proxy_async();
                 mbar_expect_tx(bar(BAR_TMA), K::TX);
 #pragma unroll
@@ -392,7 +395,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
             uint32_t blk = 0;
             while (item < total) {
                 const uint32_t ph = blk & 1u;
-                const int c = item / p.BH, bh = item % p.BH;
+                const int c = item / p.BH, bh = item % p.BH;   // c: the run index
                 const bool last_block = (j == nblocks(item) - 1);
                 wait(BAR_TMA, ph);
                 tc_fence_after();
@@ -473,7 +476,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                 load_block(item, j);
                 // ---- publish after the compute warps stored the state of the item's last block
                 wait(BAR_PUB, ph);
-                if (last_block && cur_c < p.nchunks - 1) {
+                if (last_block && cur_c < p.nruns - 1) {
                     __threadfence();
                     asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p.flags + cur_bh), "r"(cur_c + 1)
                                  : "memory");
@@ -493,13 +496,14 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
             wait(BAR_TMA, ph);
             const int item = *s_item, j = *s_j;
             if (item >= total) break;
-            const int c = item / p.BH, bh = item % p.BH;
+            const int c = item / p.BH, bh = item % p.BH;   // c: the run index
             const int b = bh / p.H, h = bh % p.H;
             const bool last_block = (j == nblocks(item) - 1);
-            const long long t0 = (long long)c * p.Q + (long long)j * SUB;
+            const long long t0 = (long long)c * p.K * p.Q + (long long)j * SUB;
+            const bool chunk_start = (t0 % p.Q) == 0;    // the decay cumsum restarts at every chunk
 
             // ---- per-token decay terms (r relative to the block start, log2 units)
-            const float r0 = (j == 0) ? 0.f : prev_last;
+            const float r0 = chunk_start ? 0.f : prev_last;
             const float rl = (s_acs[row] - r0) * LOG2E;
             const float rlast = (s_acs[SUB - 1] - r0) * LOG2E;
             if (half == 0) {
@@ -652,7 +656,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
             wait(BAR_Y, ph);
             tc_fence_after();
             if (last_block) {
-                const bool to_final = c == p.nchunks - 1;
+                const bool to_final = c == p.nruns - 1;
                 const long long fo = ((long long)bh * N + row) * PD + half * 32;
                 float* slot = p.slots + fo;
 #pragma unroll
@@ -817,9 +821,21 @@ static cudaError_t launch_n(const PrefillArgs& a, cudaStream_t s) {
     p.Q = (int)a.Q;
     p.nchunks = (int)a.lay.nchunks;
     p.BH = (int)(a.batch * a.H);
+    // Runs: with as many sequences as pipelines, one item walks a whole
+    // sequence and the state never leaves the SM.  With fewer sequences the
+    // chunks are cut into runs chained through the fp32 slots.
+    {
+        const long long pipes = (long long)resident[dev] * PIPES;
+        const long long nc = p.nchunks;
+        long long Kc = nc;
+        if (2LL * p.BH < pipes) Kc = (nc * p.BH + pipes - 1) / pipes;
+        if (Kc < 1) Kc = 1;
+        p.K = (int)Kc;
+        p.nruns = (int)((nc + Kc - 1) / Kc);
+    }
     p.state_bf16 = a.state_bf16;
     p.y_bf16 = a.y_bf16;
-    const long long items = (long long)p.nchunks * p.BH;
+    const long long items = (long long)p.nruns * p.BH;
     if (items > 0x7fffffffLL) return cudaErrorInvalidValue;
     const long long want = (items + PIPES - 1) / PIPES;   // each CTA runs PIPES ticket streams
     const unsigned grid = (unsigned)(want < resident[dev] ? want : resident[dev]);
