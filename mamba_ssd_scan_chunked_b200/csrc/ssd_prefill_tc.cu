@@ -148,6 +148,11 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* tm,
         ::"r"(dst), "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar)
         : "memory");
 }
+// L2 prefetch of a tile (no shared-memory destination, no completion)
+__device__ __forceinline__ void tma_prefetch_4d(const CUtensorMap* tm, int c0, int c1, int c2, int c3) {
+    asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];"
+                 ::"l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(c2), "r"(c3) : "memory");
+}
 __device__ __forceinline__ void tma_store_4d(const CUtensorMap* tm, uint32_t src, int c0, int c1, int c2, int c3) {
     asm volatile(
         "cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];"
@@ -165,6 +170,11 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ uint32_t elect_one() {
+    uint32_t p;
+    asm volatile("{\n .reg .pred P;\n elect.sync _|P, 0xffffffff;\n selp.u32 %0, 1, 0, P;\n}\n" : "=r"(p));
+    return p;
+}
 // 2^x on the SFU (approximate, flushes subnormal results to zero; 2^-inf = 0)
 __device__ __forceinline__ float ex2(float x) {
     float y;
@@ -349,7 +359,8 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
 
     if (control) {
         // ==================================================== control warp
-        if (lane == 0) {
+        {
+            const uint32_t lead = elect_one();
             constexpr uint32_t ID_S = idesc_bf16(128, 128, false, false);   // C (K-major) x B^T (K-major)
             constexpr uint32_t ID_ST = idesc_bf16(128, PD, true, true);     // B^T (MN-major) x wX (MN-major)
             constexpr uint32_t ID_Y = idesc_bf16(128, PD, false, true);     // M (TMEM) x X (MN-major)
@@ -368,12 +379,17 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
             constexpr uint32_t KSTEP_K = 2, KBLOCK_K = TILE >> 4, KSTEP_MN = 2048 >> 4;
             // publish the block's coordinates, then load its operands and per-token terms
             auto load_block = [&](int it, int j) {
-                *s_item = it;
-                *s_j = j;
+                __syncwarp();
+                if (lead) {
+                    *s_item = it;
+                    *s_j = j;
+                }
+                __syncwarp();
                 if (it >= total) {                      // no more work: release the compute warps
-                    mbar_arrive(bar(BAR_TMA));
+                    if (lead) mbar_arrive(bar(BAR_TMA));
                     return;
                 }
+                if (!lead) return;
                 const int r_ = it / p.BH, bh_ = it % p.BH;
                 const int b_ = bh_ / p.H, h_ = bh_ % p.H, g_ = h_ / (p.H / p.G);
                 const int t0_ = r_ * p.K * p.Q + j * SUB;
@@ -388,8 +404,19 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                 const long long o = (long long)bh_ * p.Lpad + t0_;
                 bulk_load(sbase + K::OFF_ACS, p.acsw + o, SUB * 4, bar(BAR_TMA));
                 bulk_load(sbase + K::OFF_DTCS, p.dtw + o, SUB * 4, bar(BAR_TMA));
+                // the next block of the item into L2 while this one is processed
+                if (j + 1 < nblocks(it)) {
+#pragma unroll
+                    for (int kb = 0; kb < K::KB; ++kb) {
+                        tma_prefetch_4d(&tmC, kb * 64, g_, t0_ + SUB, b_);
+                        tma_prefetch_4d(&tmB, kb * 64, g_, t0_ + SUB, b_);
+                    }
+                    tma_prefetch_4d(&tmX, 0, h_, t0_ + SUB, b_);
+                }
             };
-            int item = atomicAdd(p.flags + p.BH + CTRL_TICKET, 1);
+            int item = 0;
+            if (lead) item = atomicAdd(p.flags + p.BH + CTRL_TICKET, 1);
+            item = __shfl_sync(0xffffffffu, item, __ffs(__ballot_sync(0xffffffffu, lead)) - 1);
             int j = 0;
             load_block(item, 0);
             uint32_t blk = 0;
@@ -399,14 +426,15 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                 const bool last_block = (j == nblocks(item) - 1);
                 wait(BAR_TMA, ph);
                 tc_fence_after();
+                __syncwarp();
                 // ---- S = C B^T (K = N) into region R (free: the previous Y is done)
 #pragma unroll
                 for (int k = 0; k < N / 16; ++k) {
                     const uint32_t o = (uint32_t)(k >> 2) * KBLOCK_K + (uint32_t)(k & 3) * KSTEP_K;
-                    if (k == 0) mma_ss<ID_S, 0>(tmem + COL_R, dC + o, dBk + o);
-                    else mma_ss<ID_S, 1>(tmem + COL_R, dC + o, dBk + o);
+                    if (k == 0) { if (lead) mma_ss<ID_S, 0>(tmem + COL_R, dC + o, dBk + o);
+                    } else if (lead) mma_ss<ID_S, 1>(tmem + COL_R, dC + o, dBk + o);
                 }
-                mma_commit(bar(BAR_S));
+                if (lead) mma_commit(bar(BAR_S));
                 // ---- the chain: chunk c-1 of this (b, h) must have published its state
                 if (j == 0 && c > 0) {
                     const int* f = p.flags + bh;
@@ -425,44 +453,48 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                         __nanosleep(64);
                     }
                 }
-                mbar_arrive(bar(BAR_CHAIN));
+                __syncwarp();
+                if (lead) mbar_arrive(bar(BAR_CHAIN));
                 // ---- Yoff = C h_hi + C h_lo into the Y accumulator (once the previous
                 // block's epilogue has read it)
                 if (blk > 0) wait(BAR_EPI, ph ^ 1u);
                 wait(BAR_H, ph);
                 tc_fence_after();
+                __syncwarp();
 #pragma unroll
                 for (int k = 0; k < N / 16; ++k) {
                     const uint32_t o = (uint32_t)(k >> 2) * KBLOCK_K + (uint32_t)(k & 3) * KSTEP_K;
-                    if (k == 0) mma_ss<ID_OFF, 0>(tmem + COL_Y, dC, dW1);
-                    else mma_ss<ID_OFF, 1>(tmem + COL_Y, dC + o, dW1 + k * KSTEP_MN);
+                    if (k == 0) { if (lead) mma_ss<ID_OFF, 0>(tmem + COL_Y, dC, dW1);
+                    } else if (lead) mma_ss<ID_OFF, 1>(tmem + COL_Y, dC + o, dW1 + k * KSTEP_MN);
                 }
 #pragma unroll
                 for (int k = 0; k < N / 16; ++k) {
                     const uint32_t o = (uint32_t)(k >> 2) * KBLOCK_K + (uint32_t)(k & 3) * KSTEP_K;
-                    mma_ss<ID_OFF, 1>(tmem + COL_Y, dC + o, dW2 + k * KSTEP_MN);
+                    if (lead) mma_ss<ID_OFF, 1>(tmem + COL_Y, dC + o, dW2 + k * KSTEP_MN);
                 }
-                mma_commit(bar(BAR_OFF));
+                if (lead) mma_commit(bar(BAR_OFF));
                 // ---- state: onto 2^(r_last) h (written by the compute warps) accumulate
                 // B^T (w o X)_hi and B^T (w o X)_lo (K = 128 tokens)
                 wait(BAR_WX, ph);
                 tc_fence_after();
+                __syncwarp();
 #pragma unroll
                 for (int k = 0; k < SUB / 16; ++k)
-                    mma_ss<ID_ST, 1>(tmem + COL_ST, dBm + k * KSTEP_MN, dW1 + k * KSTEP_MN);
+                    if (lead) mma_ss<ID_ST, 1>(tmem + COL_ST, dBm + k * KSTEP_MN, dW1 + k * KSTEP_MN);
 #pragma unroll
                 for (int k = 0; k < SUB / 16; ++k)
-                    mma_ss<ID_ST, 1>(tmem + COL_ST, dBm + k * KSTEP_MN, dW2 + k * KSTEP_MN);
+                    if (lead) mma_ss<ID_ST, 1>(tmem + COL_ST, dBm + k * KSTEP_MN, dW2 + k * KSTEP_MN);
                 // ---- Y += M_hi X + M_lo X onto the scaled Yoff (A from TMEM)
                 wait(BAR_M, ph);
                 tc_fence_after();
+                __syncwarp();
 #pragma unroll
                 for (int k = 0; k < SUB / 16; ++k)
-                    mma_ts<ID_Y, 1>(tmem + COL_Y, tmem + COL_R + 16 * k, dX + k * KSTEP_MN);
+                    if (lead) mma_ts<ID_Y, 1>(tmem + COL_Y, tmem + COL_R + 16 * k, dX + k * KSTEP_MN);
 #pragma unroll
                 for (int k = 0; k < SUB / 16; ++k)
-                    mma_ts<ID_Y, 1>(tmem + COL_Y, tmem + COL_R + 16 * k + 8, dX + k * KSTEP_MN);
-                mma_commit(bar(BAR_Y));
+                    if (lead) mma_ts<ID_Y, 1>(tmem + COL_Y, tmem + COL_R + 16 * k + 8, dX + k * KSTEP_MN);
+                if (lead) mma_commit(bar(BAR_Y));
                 // ---- next block: C, B, X, dt and the cumsum are free once Y is done
                 wait(BAR_Y, ph);
                 const int cur_item = item;
@@ -470,13 +502,15 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                 if (!last_block) {
                     ++j;
                 } else {
-                    item = atomicAdd(p.flags + p.BH + CTRL_TICKET, 1);
+                    int nx = 0;
+                    if (lead) nx = atomicAdd(p.flags + p.BH + CTRL_TICKET, 1);
+                    item = __shfl_sync(0xffffffffu, nx, __ffs(__ballot_sync(0xffffffffu, lead)) - 1);
                     j = 0;
                 }
                 load_block(item, j);
                 // ---- publish after the compute warps stored the state of the item's last block
                 wait(BAR_PUB, ph);
-                if (last_block && cur_c < p.nruns - 1) {
+                if (last_block && cur_c < p.nruns - 1 && lead) {
                     __threadfence();
                     asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p.flags + cur_bh), "r"(cur_c + 1)
                                  : "memory");
