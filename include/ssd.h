@@ -225,6 +225,25 @@ ssd_status_t ssd_state_update(const ssd_decode_desc_t* desc, void* state, const 
  */
 ssd_status_t ssd_get_device_error(void* stream, uint32_t* detail);
 
+/* Fault-injection bits for ssd_debug_inject. */
+#define SSD_FAULT_DROP_RUN_PUBLISH 0x1u
+
+/*
+ * Test hook for the device-side failure path; never needed in normal use.
+ * Sets the faults injected into every following launch until called again
+ * with 0 (process-wide, all devices).
+ *  SSD_FAULT_DROP_RUN_PUBLISH: on the tensor-core prefill path, a run of
+ *    chunks that hands its state to the next run of the same sequence never
+ *    signals it.  The next run's bounded wait (2 s) then expires: the launch
+ *    still completes (its outputs are undefined), and ssd_get_device_error
+ *    reports SSD_ERR_DEVICE_TIMEOUT with bit 0x1 (a hand-off wait timed out)
+ *    and possibly 0x2 (other waits cut short) in *detail.  Nothing traps and
+ *    the CUDA context stays usable.  Runs are used only when a prefill has
+ *    fewer (batch x head) sequences than SMs.
+ * Errors: SSD_ERR_INVALID_ARG for unknown bits (nothing changed).
+ */
+ssd_status_t ssd_debug_inject(uint32_t faults);
+
 #ifdef __cplusplus
 }
 #endif

@@ -13,6 +13,9 @@ namespace ssd {
 __device__ unsigned g_device_error;
 
 static std::mutex g_err_mutex;
+static std::atomic<uint32_t> g_debug_faults{0};
+
+uint32_t debug_faults() { return g_debug_faults.load(std::memory_order_relaxed); }
 static unsigned* g_err_ptr[64];
 
 static cudaError_t device_error_ptr(unsigned** out) {
@@ -177,6 +180,7 @@ ssd_status_t ssd_chunk_scan_fwd(const ssd_prefill_desc_t* d, const void* x, cons
     a.x = x; a.dt_raw = dt_raw; a.B = B; a.C = C; a.dt_bias = dt_bias; a.A = A; a.D = D;
     a.init_state = init_state; a.y = y; a.final_state = final_state;
     a.ws = (char*)workspace; a.lay = lay;
+    a.drop_publish = (debug_faults() & SSD_FAULT_DROP_RUN_PUBLISH) ? 1 : 0;
     e = device_error_ptr(&a.dev_err);
     if (e != cudaSuccess) return SSD_ERR_CUDA;
     e = launch_dt_cumsum(a, s);
@@ -217,6 +221,12 @@ ssd_status_t ssd_state_update(const ssd_decode_desc_t* d, void* state, const voi
     a.dt_bias = dt_bias; a.A = A; a.D = D; a.y = y;
     const cudaError_t e = launch_state_update(a, (cudaStream_t)stream);
     return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
+}
+
+ssd_status_t ssd_debug_inject(uint32_t faults) {
+    if (faults & ~(uint32_t)SSD_FAULT_DROP_RUN_PUBLISH) return SSD_ERR_INVALID_ARG;
+    g_debug_faults.store(faults, std::memory_order_relaxed);
+    return SSD_OK;
 }
 
 ssd_status_t ssd_get_device_error(void* stream, uint32_t* detail) {

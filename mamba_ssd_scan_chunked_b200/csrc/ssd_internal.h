@@ -40,6 +40,7 @@ struct PrefillArgs {
     char* ws;
     PrefillLayout lay;
     unsigned* dev_err;     // device error word of the current device
+    int drop_publish;      // fault injection (ssd_debug_inject): runs do not publish their state
 };
 
 // chunk-local dt / decay cumsum (shared by both prefill paths)
@@ -49,5 +50,8 @@ cudaError_t launch_prefill_simt(const PrefillArgs& a, cudaStream_t s);
 // tensor-core prefill path; returns cudaErrorNotSupported when the shape is not covered
 bool tc_path_supports(int64_t P, int64_t N, int64_t Q, bool io_bf16);
 cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s);
+
+// fault-injection bits set by ssd_debug_inject (read at every launch)
+uint32_t debug_faults();
 
 }  // namespace ssd

@@ -108,6 +108,7 @@ struct Params {
     int H, G, Q, nchunks, BH;
     int K, nruns;           // a work item = one (b, h) and a run of K consecutive chunks
     int state_bf16, y_bf16;
+    int drop_publish;       // test hook: runs never publish their state (successors time out)
 };
 
 // ---------------------------------------------------------------- PTX helpers
@@ -510,7 +511,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                 load_block(item, j);
                 // ---- publish after the compute warps stored the state of the item's last block
                 wait(BAR_PUB, ph);
-                if (last_block && cur_c < p.nruns - 1 && lead) {
+                if (last_block && cur_c < p.nruns - 1 && lead && !p.drop_publish) {
                     __threadfence();
                     asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p.flags + cur_bh), "r"(cur_c + 1)
                                  : "memory");
@@ -869,6 +870,7 @@ static cudaError_t launch_n(const PrefillArgs& a, cudaStream_t s) {
     }
     p.state_bf16 = a.state_bf16;
     p.y_bf16 = a.y_bf16;
+    p.drop_publish = a.drop_publish;
     const long long items = (long long)p.nruns * p.BH;
     if (items > 0x7fffffffLL) return cudaErrorInvalidValue;
     const long long want = (items + PIPES - 1) / PIPES;   // each CTA runs PIPES ticket streams

@@ -26,7 +26,11 @@ STATUS = {0: "SSD_OK", 1: "SSD_ERR_INVALID_ARG", 2: "SSD_ERR_UNSUPPORTED", 3: "S
 
 # every symbol include/ssd.h declares
 EXPORTS = ("ssd_version", "ssd_status_string", "ssd_chunk_scan_workspace_size", "ssd_chunk_scan_path",
-           "ssd_chunk_scan_fwd", "ssd_chunk_scan_fwd_noalloc", "ssd_state_update", "ssd_get_device_error")
+           "ssd_chunk_scan_fwd", "ssd_chunk_scan_fwd_noalloc", "ssd_state_update", "ssd_get_device_error",
+           "ssd_debug_inject")
+
+# fault-injection bits of ssd_debug_inject
+SSD_FAULT_DROP_RUN_PUBLISH = 0x1
 
 # scratch size of ssd_chunk_scan_fwd_noalloc (SSD_NOALLOC_WORKSPACE_BYTES)
 NOALLOC_WORKSPACE_BYTES = 32 << 20
@@ -81,6 +85,8 @@ def lib():
             L.ssd_state_update.argtypes = [ctypes.POINTER(DecodeDesc)] + [_VP] * 10
             L.ssd_get_device_error.restype = ctypes.c_int
             L.ssd_get_device_error.argtypes = [_VP, ctypes.POINTER(ctypes.c_uint32)]
+            L.ssd_debug_inject.restype = ctypes.c_int
+            L.ssd_debug_inject.argtypes = [ctypes.c_uint32]
             _lib = L
     return _lib
 
@@ -138,6 +144,11 @@ def ssd_get_device_error(stream=None):
     d = ctypes.c_uint32(0)
     st = lib().ssd_get_device_error(stream or None, ctypes.byref(d))
     return st, d.value
+
+
+def ssd_debug_inject(faults: int) -> int:
+    """Test hook: fault bits injected into every following launch (0 clears)."""
+    return lib().ssd_debug_inject(int(faults))
 
 
 # --------------------------------------------------------------------------
