@@ -180,6 +180,104 @@ def run_reference(args, rank):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------ the other workloads
+def measure_workloads(torch, ssd, I, dev, peaks, max_call_s=2.0):
+    """Times the long-sequence / state-size sweep and the batch-512 prefill + bf16-state
+    decode hand-off on seeded device-generated inputs with the workloads' value
+    distributions (x, B, C, dt_raw ~ N(0,1); dt_bias = log(expm1(U[1e-3,1e-1]));
+    A = -U[1,16]; D ~ N(0,1)).  Parity of these workloads against the oracle is
+    checked by tests/test_configs_gpu.py; here only time is measured: 1 warm-up
+    call, then calls until 3 are timed or max_call_s is spent.  Algorithmic bytes
+    and the roofline fraction follow the main line's convention."""
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(2)
+    hbm = peaks["hbm_gbs"]
+
+    def normal(shape, dtype):
+        return torch.randn(shape, generator=gen, device=dev, dtype=torch.float32).to(dtype)
+
+    def heads(H):
+        u = torch.rand(H, generator=gen, device=dev) * (0.1 - 1e-3) + 1e-3
+        return torch.log(torch.expm1(u)), -(torch.rand(H, generator=gen, device=dev) * 15 + 1), normal((H,), torch.float32)
+
+    def timed(call):
+        call()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n, t_total = 0, 0.0
+        while n < 3 and t_total < max_call_s:
+            e0.record()
+            call()
+            e1.record()
+            torch.cuda.synchronize()
+            t_total += e0.elapsed_time(e1) * 1e-3
+            n += 1
+        return t_total / n
+
+    out = {}
+    bf16 = torch.bfloat16
+    shapes = I.long_sequence_sweep() + [I.HANDOFF_PREFILL]
+    for sh in shapes:
+        b, L, H, P, N, G, Q = sh.batch, sh.seqlen, sh.nheads, sh.headdim, sh.dstate, sh.ngroups, sh.chunk
+        handoff = sh is I.HANDOFF_PREFILL
+        x = normal((b, L, H, P), bf16)
+        dtr = normal((b, L, H), bf16)
+        Bm = normal((b, L, G, N), bf16)
+        Cm = normal((b, L, G, N), bf16)
+        dtb, A, D = heads(H)
+        sdt = bf16 if handoff else torch.float32
+        y = torch.empty((b, L, H, P), dtype=torch.float32, device=dev)
+        fs = torch.empty((b, H, N, P), dtype=sdt, device=dev)
+        desc = ssd.prefill_desc(x, Bm, Q, torch.float32, sdt)
+        ws = torch.empty(ssd.ssd_chunk_scan_workspace_size(desc), dtype=torch.uint8, device=dev)
+        stream = torch.cuda.current_stream(dev).cuda_stream
+
+        def call():
+            st = ssd.ssd_chunk_scan_fwd(desc, x.data_ptr(), dtr.data_ptr(), dtb.data_ptr(), A.data_ptr(),
+                                        Bm.data_ptr(), Cm.data_ptr(), D.data_ptr(), 0, y.data_ptr(), fs.data_ptr(),
+                                        ws.data_ptr(), ws.numel(), stream)
+            if st:
+                raise ssd.SsdError(st, "ssd_chunk_scan_fwd")
+
+        sec = timed(call)
+        nbytes = prefill_bytes(b, L, H, P, N, G, 2, 4, 2 if handoff else 4)
+        flops = prefill_flops(b, L, H, P, N, G, Q)
+        t_hbm = nbytes / (hbm * 1e9)
+        t_tc = flops / (peaks["bf16_tflops"] * 1e12)
+        out[sh.name] = {"kind": "prefill", "path": "tensor cores" if ssd.ssd_chunk_scan_path(desc) == 0 else "cuda cores",
+                        "tokens_per_s": b * L / sec, "ms_per_call": sec * 1e3, "tflops": flops / sec / 1e12,
+                        "gbs": nbytes / sec / 1e9, "bound": "hbm" if t_hbm >= t_tc else "tensor",
+                        "frac": max(t_hbm, t_tc) / sec}
+        if handoff:
+            # the bf16 final state feeds decode steps at batch 512
+            dsh = I.HANDOFF_DECODE
+            state = fs
+            xs = normal((b, H, P), bf16)
+            dts = normal((b, H), bf16)
+            Bs = normal((b, G, N), bf16)
+            Cs = normal((b, G, N), bf16)
+            yd = torch.empty((b, H, P), dtype=torch.float32, device=dev)
+            ddesc = ssd.DecodeDesc(b, H, P, N, G, ssd.SSD_BF16, ssd.SSD_F32, ssd.SSD_BF16)
+
+            def dcall():
+                st = ssd.ssd_state_update(ddesc, state.data_ptr(), xs.data_ptr(), dts.data_ptr(), dtb.data_ptr(),
+                                          A.data_ptr(), Bs.data_ptr(), Cs.data_ptr(), D.data_ptr(), yd.data_ptr(),
+                                          stream)
+                if st:
+                    raise ssd.SsdError(st, "ssd_state_update")
+
+            dsec = timed(dcall)
+            dbytes = decode_bytes(b, H, P, N, G, 2, 4, 2)
+            out[dsh.name] = {"kind": "decode", "tokens_per_s": b / dsec, "ms_per_call": dsec * 1e3,
+                             "gbs": dbytes / dsec / 1e9, "bound": "hbm", "frac": dbytes / dsec / 1e9 / hbm}
+        del x, dtr, Bm, Cm, y, fs, ws
+        torch.cuda.empty_cache()
+    st_err, detail = ssd.ssd_get_device_error(torch.cuda.current_stream(dev).cuda_stream)
+    if st_err:
+        raise RuntimeError(f"device error word {detail:#x} after the workload sweep")
+    return out
+
+
 # ------------------------------------------------------------------ our arm
 def main():
     ap = argparse.ArgumentParser()
@@ -188,6 +286,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip timing the other benchmark workloads (long-sequence sweep, batch-512 hand-off)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     rank = int(os.environ.get("RANK", "0"))
@@ -379,6 +479,10 @@ def main():
                         "kind": "oracle",
                         "sample": f"the full workload ({tokens_rank} tokens x 64 heads) run {reps} times, {cdt:.1f} s"}
 
+    workloads = None
+    if rank == 0 and world == 1 and not args.no_workloads:
+        workloads = measure_workloads(torch, ssd, I, dev, peaks)
+
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -390,7 +494,7 @@ def main():
                            "l2": "3 rotating input sets (x 67 MB each); inputs larger than L2 across steps",
                            "kernel_path": "tensor cores" if path == 0 else "cuda cores"},
                 "tflops": tflops, "gbs": gbs, "roofline": roofline, "decode": decode_line,
-                "cpu_baseline": cpu_baseline, "e2e": e2e,
+                "cpu_baseline": cpu_baseline, "e2e": e2e, "workloads": workloads,
                 "gpu_launches": launches_per_prefill * args.steps + args.steps,
                 "clocks": clk.summary()}
         print(json.dumps(line), flush=True)
