@@ -32,6 +32,14 @@ __device__ __forceinline__ float softplus_f32(float z) {
 template <typename T> struct Vec16;
 template <> struct Vec16<float> {
     static constexpr int N = 4;
+    __device__ __forceinline__ static void unpack(uint4 v, float* out) {
+        out[0] = __uint_as_float(v.x); out[1] = __uint_as_float(v.y);
+        out[2] = __uint_as_float(v.z); out[3] = __uint_as_float(v.w);
+    }
+    __device__ __forceinline__ static uint4 pack(const float* in) {
+        return make_uint4(__float_as_uint(in[0]), __float_as_uint(in[1]), __float_as_uint(in[2]),
+                          __float_as_uint(in[3]));
+    }
     __device__ __forceinline__ static void load(const float* p, float* out) {
         float4 v = *reinterpret_cast<const float4*>(p);
         out[0] = v.x; out[1] = v.y; out[2] = v.z; out[3] = v.w;

@@ -40,7 +40,8 @@ def oracle_decode(state0, steps, params, round_bf16):
 
 
 @pytest.mark.parametrize("b,H,P,N,G", [(3, 4, 64, 128, 2), (2, 6, 32, 16, 3), (4, 8, 64, 64, 1),
-                                       (1, 2, 128, 256, 2), (2, 4, 8, 8, 4)])
+                                       (1, 2, 128, 256, 2), (2, 4, 8, 8, 4), (2, 3, 24, 32, 1),
+                                       (1, 3, 256, 64, 1), (3, 5, 16, 24, 5)])
 @pytest.mark.parametrize("io,state", [(I.F32, I.F32), (I.BF16, I.F32), (I.BF16, I.BF16)])
 def test_decode_matches_oracle(b, H, P, N, G, io, state):
     params = I.draw_head_params(H, seed=7)
