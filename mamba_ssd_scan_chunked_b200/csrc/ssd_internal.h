@@ -24,8 +24,8 @@ struct PrefillLayout {
     int64_t nchunks;       // ceil(L / Q)
     int64_t Lpad;          // nchunks * Q
     size_t off_dt, off_acs;        // fp32 [b][H][Lpad] each
-    size_t off_states;             // fp32 chunk states (CUDA-core path) or chain slots
-    size_t off_flags;              // int32 [b][H] chain progress + 64 control words
+    size_t off_states;             // fp32 chunk states (CUDA-core path) or run-entry states
+    size_t off_flags;              // int32 [b][H] run-entry states published + 64 control words
     size_t total;
 };
 
@@ -40,7 +40,7 @@ struct PrefillArgs {
     char* ws;
     PrefillLayout lay;
     unsigned* dev_err;     // device error word of the current device
-    int drop_publish;      // fault injection (ssd_debug_inject): runs do not publish their state
+    int drop_publish;      // fault injection (ssd_debug_inject): run-entry states are never published
 };
 
 // chunk-local dt / decay cumsum (shared by both prefill paths)
@@ -49,6 +49,8 @@ cudaError_t launch_dt_cumsum(const PrefillArgs& a, cudaStream_t s);
 cudaError_t launch_prefill_simt(const PrefillArgs& a, cudaStream_t s);
 // tensor-core prefill path; returns cudaErrorNotSupported when the shape is not covered
 bool tc_path_supports(int64_t P, int64_t N, int64_t Q, bool io_bf16);
+// runs per sequence of the tensor-core path (1 = every work item is a whole sequence)
+int64_t tc_runs(int64_t BH, int64_t nchunks);
 cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s);
 
 // fault-injection bits set by ssd_debug_inject (read at every launch)

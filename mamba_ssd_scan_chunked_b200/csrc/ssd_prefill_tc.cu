@@ -1,6 +1,6 @@
 // Tensor-core prefill of the SSD layer core for sm_100a: tcgen05 MMAs with
 // TMEM accumulators, operands staged by TMA, fp32 state passing between
-// chunks through a chained (ticketed) hand-off.
+// runs of chunks through a chained (ticketed) hand-off.
 //
 // The chunked contraction of the semiseparable matrix ("Mamba-2 vs
 // Transformers / SSD", section "Mamba-2 and the SSD paper: what changed in
@@ -27,16 +27,25 @@
 // outputs reach 60x their rms (tokens with large dt).  C B^T uses the exact
 // inputs and needs one pass.
 //
-// Chained state passing: items are handed out by an atomic ticket in
-// chunk-major order, so the item of chunk c-1 of the same (b, h) always holds
-// an earlier ticket and is already running; item c waits (bounded, see below)
-// for flags[b,h] >= c, reads the fp32 state slot, updates it in place and sets
-// flags[b,h] = c+1.  A CTA allocates TMEM before taking a ticket, so a ticket
-// holder never waits for TMEM.  Every wait is bounded by a 2 s globaltimer
-// deadline.  A hand-off wait that expires sets the device error word and a
-// launch-wide abort word that ends every other hand-off wait at once; the CTA
-// then finishes its (in-bounds) work -- still waiting for its own TMA and MMA
-// completions -- and frees its TMEM.  Nothing traps.
+// Work items and state passing: a work item is one (b, h) sequence, or a run of
+// K consecutive chunks of it when there are too few sequences to fill the
+// block pipelines.  With runs, every run after the first needs the state that
+// enters it, so the ticket stream first hands out state items (run r < nruns-1
+// of a sequence: only the chunk-state MMAs, from a zero state, giving the
+// run's own contribution dS_r and its total decay R_r), then output items (run
+// r: the whole block chain from the entry state h_in(r)).  A state item ends
+// with the one sequential step, h_in(r+1) = 2^(R_r) h_in(r) + dS_r, for which
+// it waits (bounded) until flags[b,h] >= r, i.e. until state item r-1 has
+// published h_in(r); it then writes h_in(r+1) to its fp32 slot and sets
+// flags[b,h] = r+1.  An output item r > 0 waits for flags[b,h] >= r before its
+// first block.  Tickets are handed out in order and an item only ever waits for
+// an item with an earlier ticket, which is running or done and waits only on
+// earlier ones: no cycle.  A CTA allocates TMEM before taking a ticket, so a
+// ticket holder never waits for TMEM.  Every wait is bounded by a 2 s
+// globaltimer deadline.  A hand-off wait that expires sets the device error
+// word and a launch-wide abort word that ends every other hand-off wait at
+// once; the CTA then finishes its (in-bounds) work -- still waiting for its own
+// TMA and MMA completions -- and frees its TMEM.  Nothing traps.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -91,13 +100,14 @@ struct Cfg {
     static constexpr uint32_t SMALL = OFF_MISC + 64;
     static constexpr uint32_t SMEM = PIPES * (TILES + SMALL);
     static constexpr uint32_t TX = (2 * KB + 1) * TILE + 2 * SUB * 4;   // TMA bytes per block
+    static constexpr uint32_t TX_ST = (KB + 1) * TILE + 2 * SUB * 4;    // ... of a state item (no C)
     static_assert(TILES % 1024 == 0 && SMALL % 16 == 0, "alignment");
 };
 
 struct Params {
     const float* dtw;       // [BH][Lpad]
     const float* acsw;      // [BH][Lpad] chunk-local inclusive cumsum of dt*A
-    float* slots;           // [BH][N][PD] fp32 state slots of the chain
+    float* slots;           // [BH][nruns-1][N][PD] fp32 entry states of runs 1..nruns-1
     int* flags;             // [BH] chunks published, then control words
     const void* init_state; // [BH][N][PD] state dtype or NULL
     void* final_state;      // [BH][N][PD] state dtype or NULL
@@ -106,9 +116,10 @@ struct Params {
     unsigned* dev_err;
     long long L, Lpad;
     int H, G, Q, nchunks, BH;
-    int K, nruns;           // a work item = one (b, h) and a run of K consecutive chunks
+    int K, nruns;           // a run = K consecutive chunks of one (b, h)
+    int nstate;             // state items ((nruns - 1) * BH), ahead of the nruns * BH output items
     int state_bf16, y_bf16;
-    int drop_publish;       // test hook: runs never publish their state (successors time out)
+    int drop_publish;       // test hook: state items never publish (their successors time out)
 };
 
 // ---------------------------------------------------------------- PTX helpers
@@ -283,9 +294,10 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
 // ---------------------------------------------------------------- the kernel
 // Persistent, one CTA per SM, PIPES independent block pipelines per CTA.  A
 // pipeline = 8 compute warps (256 threads; thread = one TMEM lane/tile row and
-// one half of its columns) + 1 control warp whose lane 0 takes tickets,
-// issues every TMA and MMA, waits for the previous chunk of the chain and
-// publishes.  Compute and control meet only at mbarriers.
+// one half of its columns) + 1 control warp, converged, whose elected lane
+// takes tickets, issues every TMA and MMA, waits for run-entry states and
+// publishes them.  Compute and control meet only at mbarriers; a state item
+// still completes every barrier once per block, so phases stay in step.
 //
 // Per 128-token block the state accumulator (TMEM) is first loaded with
 // 2^(r_last) h and the chunk-state MMAs accumulate onto it, so h' stays in
@@ -321,7 +333,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
     enum { BAR_TMA = 0, BAR_S, BAR_CHAIN, BAR_H, BAR_OFF, BAR_WX, BAR_M, BAR_Y, BAR_PUB, BAR_EPI, NBAR };
     auto bar = [&](int i) -> uint32_t { return sbase + K::OFF_BAR + 8u * (uint32_t)i; };
     volatile int* g_abort = reinterpret_cast<volatile int*>(p.flags + p.BH + CTRL_ABORT);
-    const int total = p.nruns * p.BH;
+    const int total = p.nstate + p.nruns * p.BH;
     unsigned err = 0;
 
     // the 128-byte swizzle of TMA and of the MMA descriptors assumes 1024-byte
@@ -350,12 +362,24 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
     auto wait = [&](int i, uint32_t ph) {
         if (!mbar_wait(bar(i), ph)) err |= kErrAsyncTimeout;
     };
-    // item = run r (chunks [rK, rK+K)) of sequence bh; tickets are run-major, so
-    // run r-1 of the same sequence always holds an earlier ticket
+    // ticket -> (state item?, run r (chunks [rK, rK+K)), sequence bh); both kinds
+    // are run-major, so item r-1 of a sequence holds an earlier ticket than item r
+    struct Item { int st, r, bh; };
+    auto decode = [&](int it) -> Item {
+        Item d;
+        d.st = it < p.nstate;
+        const int k = d.st ? it : it - p.nstate;
+        d.r = k / p.BH;
+        d.bh = k % p.BH;
+        return d;
+    };
     auto nblocks = [&](int it) -> int {       // 128-token blocks of the run (never straddle a chunk)
-        const long long t_first = (long long)(it / p.BH) * p.K * p.Q;
+        const long long t_first = (long long)decode(it).r * p.K * p.Q;
         const long long len = p.L - t_first < (long long)p.K * p.Q ? p.L - t_first : (long long)p.K * p.Q;
         return (int)((len + SUB - 1) / SUB);
+    };
+    auto slot_of = [&](int bh, int r) -> float* {   // entry state of run r >= 1
+        return p.slots + (long long)(bh * (p.nruns - 1) + r - 1) * N * PD;
     };
 
     if (control) {
@@ -391,14 +415,15 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                     return;
                 }
                 if (!lead) return;
-                const int r_ = it / p.BH, bh_ = it % p.BH;
+                const Item d_ = decode(it);
+                const int bh_ = d_.bh;
                 const int b_ = bh_ / p.H, h_ = bh_ % p.H, g_ = h_ / (p.H / p.G);
-                const int t0_ = r_ * p.K * p.Q + j * SUB;
+                const int t0_ = d_.r * p.K * p.Q + j * SUB;
                 fence_proxy_async();
-                mbar_expect_tx(bar(BAR_TMA), K::TX);
+                mbar_expect_tx(bar(BAR_TMA), d_.st ? K::TX_ST : K::TX);   // a state item needs no C
 #pragma unroll
                 for (int kb = 0; kb < K::KB; ++kb) {
-                    tma_load_4d(base + K::OFF_C + kb * TILE, &tmC, kb * 64, g_, t0_, b_, bar(BAR_TMA));
+                    if (!d_.st) tma_load_4d(base + K::OFF_C + kb * TILE, &tmC, kb * 64, g_, t0_, b_, bar(BAR_TMA));
                     tma_load_4d(base + K::OFF_B + kb * TILE, &tmB, kb * 64, g_, t0_, b_, bar(BAR_TMA));
                 }
                 tma_load_4d(base + K::OFF_X, &tmX, 0, h_, t0_, b_, bar(BAR_TMA));
@@ -409,7 +434,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                 if (j + 1 < nblocks(it)) {
 #pragma unroll
                     for (int kb = 0; kb < K::KB; ++kb) {
-                        tma_prefetch_4d(&tmC, kb * 64, g_, t0_ + SUB, b_);
+                        if (!d_.st) tma_prefetch_4d(&tmC, kb * 64, g_, t0_ + SUB, b_);
                         tma_prefetch_4d(&tmB, kb * 64, g_, t0_ + SUB, b_);
                     }
                     tma_prefetch_4d(&tmX, 0, h_, t0_ + SUB, b_);
@@ -421,85 +446,110 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
             int j = 0;
             load_block(item, 0);
             uint32_t blk = 0;
+            // bounded wait until sequence bh has published the entry state of run r
+            auto chain_wait = [&](int bh, int r) {
+                const int* f = p.flags + bh;
+                const unsigned long long deadline = gtimer() + WAIT_NS;
+                uint32_t spins = 0;
+                while (true) {
+                    int v;
+                    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
+                    if (v >= r) break;
+                    if (*g_abort) { err |= kErrChainAborted; break; }
+                    if ((++spins & 255u) == 0 && gtimer() > deadline) {
+                        err |= kErrChainTimeout;
+                        atomicExch(p.flags + p.BH + CTRL_ABORT, 1);
+                        break;
+                    }
+                    __nanosleep(64);
+                }
+            };
             while (item < total) {
                 const uint32_t ph = blk & 1u;
-                const int c = item / p.BH, bh = item % p.BH;   // c: the run index
+                const Item d = decode(item);
                 const bool last_block = (j == nblocks(item) - 1);
                 wait(BAR_TMA, ph);
                 tc_fence_after();
                 __syncwarp();
-                // ---- S = C B^T (K = N) into region R (free: the previous Y is done)
+                if (d.st) {
+                    // ---- state item: only the chunk-state MMAs (no S, Yoff, M, Y or y);
+                    // the barriers of the skipped steps still complete once per block
+                    if (lead) mbar_arrive(bar(BAR_S));
+                    if (blk > 0) wait(BAR_EPI, ph ^ 1u);
+                    wait(BAR_H, ph);
+                    if (lead) mbar_arrive(bar(BAR_OFF));
+                    wait(BAR_WX, ph);
+                    tc_fence_after();
+                    __syncwarp();
 #pragma unroll
-                for (int k = 0; k < N / 16; ++k) {
-                    const uint32_t o = (uint32_t)(k >> 2) * KBLOCK_K + (uint32_t)(k & 3) * KSTEP_K;
-                    if (k == 0) { if (lead) mma_ss<ID_S, 0>(tmem + COL_R, dC + o, dBk + o);
-                    } else if (lead) mma_ss<ID_S, 1>(tmem + COL_R, dC + o, dBk + o);
-                }
-                if (lead) mma_commit(bar(BAR_S));
-                // ---- the chain: chunk c-1 of this (b, h) must have published its state
-                if (j == 0 && c > 0) {
-                    const int* f = p.flags + bh;
-                    const unsigned long long deadline = gtimer() + WAIT_NS;
-                    uint32_t spins = 0;
-                    while (true) {
-                        int v;
-                        asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
-                        if (v >= c) break;
-                        if (*g_abort) { err |= kErrChainAborted; break; }
-                        if ((++spins & 255u) == 0 && gtimer() > deadline) {
-                            err |= kErrChainTimeout;
-                            atomicExch(p.flags + p.BH + CTRL_ABORT, 1);
-                            break;
-                        }
-                        __nanosleep(64);
+                    for (int k = 0; k < SUB / 16; ++k)
+                        if (lead) mma_ss<ID_ST, 1>(tmem + COL_ST, dBm + k * KSTEP_MN, dW1 + k * KSTEP_MN);
+#pragma unroll
+                    for (int k = 0; k < SUB / 16; ++k)
+                        if (lead) mma_ss<ID_ST, 1>(tmem + COL_ST, dBm + k * KSTEP_MN, dW2 + k * KSTEP_MN);
+                    wait(BAR_M, ph);
+                    if (lead) mma_commit(bar(BAR_Y));
+                    // the combine of the last block needs h_in(r), published by state
+                    // item r-1 (this item's MMAs are already issued)
+                    if (last_block && d.r > 0 && lead) chain_wait(d.bh, d.r);
+                    __syncwarp();
+                    if (lead) mbar_arrive(bar(BAR_CHAIN));
+                } else {
+                    // ---- S = C B^T (K = N) into region R (free: the previous Y is done)
+#pragma unroll
+                    for (int k = 0; k < N / 16; ++k) {
+                        const uint32_t o = (uint32_t)(k >> 2) * KBLOCK_K + (uint32_t)(k & 3) * KSTEP_K;
+                        if (k == 0) { if (lead) mma_ss<ID_S, 0>(tmem + COL_R, dC + o, dBk + o);
+                        } else if (lead) mma_ss<ID_S, 1>(tmem + COL_R, dC + o, dBk + o);
                     }
+                    if (lead) mma_commit(bar(BAR_S));
+                    // ---- an output item starts from the entry state of its run
+                    if (j == 0 && d.r > 0 && lead) chain_wait(d.bh, d.r);
+                    __syncwarp();
+                    if (lead) mbar_arrive(bar(BAR_CHAIN));
+                    // ---- Yoff = C h_hi + C h_lo into the Y accumulator (once the previous
+                    // block's epilogue has read it)
+                    if (blk > 0) wait(BAR_EPI, ph ^ 1u);
+                    wait(BAR_H, ph);
+                    tc_fence_after();
+                    __syncwarp();
+#pragma unroll
+                    for (int k = 0; k < N / 16; ++k) {
+                        const uint32_t o = (uint32_t)(k >> 2) * KBLOCK_K + (uint32_t)(k & 3) * KSTEP_K;
+                        if (k == 0) { if (lead) mma_ss<ID_OFF, 0>(tmem + COL_Y, dC, dW1);
+                        } else if (lead) mma_ss<ID_OFF, 1>(tmem + COL_Y, dC + o, dW1 + k * KSTEP_MN);
+                    }
+#pragma unroll
+                    for (int k = 0; k < N / 16; ++k) {
+                        const uint32_t o = (uint32_t)(k >> 2) * KBLOCK_K + (uint32_t)(k & 3) * KSTEP_K;
+                        if (lead) mma_ss<ID_OFF, 1>(tmem + COL_Y, dC + o, dW2 + k * KSTEP_MN);
+                    }
+                    if (lead) mma_commit(bar(BAR_OFF));
+                    // ---- state: onto 2^(r_last) h (written by the compute warps) accumulate
+                    // B^T (w o X)_hi and B^T (w o X)_lo (K = 128 tokens)
+                    wait(BAR_WX, ph);
+                    tc_fence_after();
+                    __syncwarp();
+#pragma unroll
+                    for (int k = 0; k < SUB / 16; ++k)
+                        if (lead) mma_ss<ID_ST, 1>(tmem + COL_ST, dBm + k * KSTEP_MN, dW1 + k * KSTEP_MN);
+#pragma unroll
+                    for (int k = 0; k < SUB / 16; ++k)
+                        if (lead) mma_ss<ID_ST, 1>(tmem + COL_ST, dBm + k * KSTEP_MN, dW2 + k * KSTEP_MN);
+                    // ---- Y += M_hi X + M_lo X onto the scaled Yoff (A from TMEM)
+                    wait(BAR_M, ph);
+                    tc_fence_after();
+                    __syncwarp();
+#pragma unroll
+                    for (int k = 0; k < SUB / 16; ++k)
+                        if (lead) mma_ts<ID_Y, 1>(tmem + COL_Y, tmem + COL_R + 16 * k, dX + k * KSTEP_MN);
+#pragma unroll
+                    for (int k = 0; k < SUB / 16; ++k)
+                        if (lead) mma_ts<ID_Y, 1>(tmem + COL_Y, tmem + COL_R + 16 * k + 8, dX + k * KSTEP_MN);
+                    if (lead) mma_commit(bar(BAR_Y));
                 }
-                __syncwarp();
-                if (lead) mbar_arrive(bar(BAR_CHAIN));
-                // ---- Yoff = C h_hi + C h_lo into the Y accumulator (once the previous
-                // block's epilogue has read it)
-                if (blk > 0) wait(BAR_EPI, ph ^ 1u);
-                wait(BAR_H, ph);
-                tc_fence_after();
-                __syncwarp();
-#pragma unroll
-                for (int k = 0; k < N / 16; ++k) {
-                    const uint32_t o = (uint32_t)(k >> 2) * KBLOCK_K + (uint32_t)(k & 3) * KSTEP_K;
-                    if (k == 0) { if (lead) mma_ss<ID_OFF, 0>(tmem + COL_Y, dC, dW1);
-                    } else if (lead) mma_ss<ID_OFF, 1>(tmem + COL_Y, dC + o, dW1 + k * KSTEP_MN);
-                }
-#pragma unroll
-                for (int k = 0; k < N / 16; ++k) {
-                    const uint32_t o = (uint32_t)(k >> 2) * KBLOCK_K + (uint32_t)(k & 3) * KSTEP_K;
-                    if (lead) mma_ss<ID_OFF, 1>(tmem + COL_Y, dC + o, dW2 + k * KSTEP_MN);
-                }
-                if (lead) mma_commit(bar(BAR_OFF));
-                // ---- state: onto 2^(r_last) h (written by the compute warps) accumulate
-                // B^T (w o X)_hi and B^T (w o X)_lo (K = 128 tokens)
-                wait(BAR_WX, ph);
-                tc_fence_after();
-                __syncwarp();
-#pragma unroll
-                for (int k = 0; k < SUB / 16; ++k)
-                    if (lead) mma_ss<ID_ST, 1>(tmem + COL_ST, dBm + k * KSTEP_MN, dW1 + k * KSTEP_MN);
-#pragma unroll
-                for (int k = 0; k < SUB / 16; ++k)
-                    if (lead) mma_ss<ID_ST, 1>(tmem + COL_ST, dBm + k * KSTEP_MN, dW2 + k * KSTEP_MN);
-                // ---- Y += M_hi X + M_lo X onto the scaled Yoff (A from TMEM)
-                wait(BAR_M, ph);
-                tc_fence_after();
-                __syncwarp();
-#pragma unroll
-                for (int k = 0; k < SUB / 16; ++k)
-                    if (lead) mma_ts<ID_Y, 1>(tmem + COL_Y, tmem + COL_R + 16 * k, dX + k * KSTEP_MN);
-#pragma unroll
-                for (int k = 0; k < SUB / 16; ++k)
-                    if (lead) mma_ts<ID_Y, 1>(tmem + COL_Y, tmem + COL_R + 16 * k + 8, dX + k * KSTEP_MN);
-                if (lead) mma_commit(bar(BAR_Y));
                 // ---- next block: C, B, X, dt and the cumsum are free once Y is done
                 wait(BAR_Y, ph);
-                const int cur_item = item;
-                const int cur_c = c, cur_bh = bh;
                 if (!last_block) {
                     ++j;
                 } else {
@@ -509,14 +559,13 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                     j = 0;
                 }
                 load_block(item, j);
-                // ---- publish after the compute warps stored the state of the item's last block
+                // ---- a state item publishes h_in(r+1) once the compute warps stored it
                 wait(BAR_PUB, ph);
-                if (last_block && cur_c < p.nruns - 1 && lead && !p.drop_publish) {
+                if (d.st && last_block && lead && !p.drop_publish) {
                     __threadfence();
-                    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p.flags + cur_bh), "r"(cur_c + 1)
+                    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p.flags + d.bh), "r"(d.r + 1)
                                  : "memory");
                 }
-                (void)cur_item;
                 ++blk;
             }
         }
@@ -526,12 +575,14 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
         auto csync = [&]() { asm volatile("bar.sync %0, %1;" ::"r"(1 + pipe), "r"(NCOMPUTE) : "memory"); };
         uint32_t blk = 0;
         float prev_last = 0.f;   // raw cumsum at the end of the previous block of the same item
+        float run_decay = 0.f;   // log2 decay over a state item's blocks so far (its R_r at the end)
         while (true) {
             const uint32_t ph = blk & 1u;
             wait(BAR_TMA, ph);
             const int item = *s_item, j = *s_j;
             if (item >= total) break;
-            const int c = item / p.BH, bh = item % p.BH;   // c: the run index
+            const Item d = decode(item);
+            const int c = d.r, bh = d.bh;
             const int b = bh / p.H, h = bh % p.H;
             const bool last_block = (j == nblocks(item) - 1);
             const long long t0 = (long long)c * p.K * p.Q + (long long)j * SUB;
@@ -544,20 +595,122 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
             if (half == 0) {
                 // dt folded into the exponent: dt_s 2^(x - r_s) = 2^(x + log2(dt_s) - r_s); dt_s = 0
                 // gives 0.  In place: this thread alone reads and writes element `row`.
-                const float d = scs[row];
-                scs[row] = (d > 0.f ? __log2f(d) : NEG_INF) - rl;
+                const float dtv = scs[row];
+                scs[row] = (dtv > 0.f ? __log2f(dtv) : NEG_INF) - rl;
             }
             if (tid == 0) bulk_wait_read0();          // previous y store has read W1/W2
             csync();
             prev_last = s_acs[SUB - 1];
 
-            // ---- h entering the block: the initial state or the previous chunk's
-            // published state (first block of an item), else the state the
-            // previous block left in the TMEM accumulator.  Split hi -> W1, lo -> W2
-            // for C h; 2^(r_last) h -> the state accumulator.
+            // h_in(r) of this thread's row and 16 of its columns: the initial state
+            // (r = 0) or the run's entry-state slot
+            auto load_entry = [&](int r, int pc, float (&hv)[16]) {
+                if (r > 0) {
+                    const float* slot = slot_of(bh, r) + row * PD + half * 32 + pc * 16;
+#pragma unroll
+                    for (int i = 0; i < 16; i += 4) {
+                        const float4 v = __ldcg(reinterpret_cast<const float4*>(slot + i));
+                        hv[i] = v.x; hv[i + 1] = v.y; hv[i + 2] = v.z; hv[i + 3] = v.w;
+                    }
+                } else if (p.init_state) {
+                    const long long o = ((long long)bh * N + row) * PD + half * 32 + pc * 16;
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        hv[i] = p.state_bf16 ? __bfloat162float(reinterpret_cast<const bf16*>(p.init_state)[o + i])
+                                             : reinterpret_cast<const float*>(p.init_state)[o + i];
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) hv[i] = 0.f;
+                }
+            };
+            // w o X split hi -> W1, lo -> W2; the raw x words are returned for D x
+            auto write_wx = [&](uint32_t (&xr)[16]) {
+                const float w = ex2(rlast + scs[row]);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const uint32_t o = swz(row, half * 4 + q);
+                    const uint4 xv = *reinterpret_cast<const uint4*>(sm + K::OFF_X + o);
+                    xr[4 * q] = xv.x; xr[4 * q + 1] = xv.y; xr[4 * q + 2] = xv.z; xr[4 * q + 3] = xv.w;
+                    uint32_t hw[4], lw[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float v0 = bf16_lo(xr[4 * q + e]) * w, v1 = bf16_hi(xr[4 * q + e]) * w;
+                        hw[e] = pack_bf16(v0, v1);
+                        lw[e] = pack_bf16(v0 - bf16_lo(hw[e]), v1 - bf16_hi(hw[e]));
+                    }
+                    *reinterpret_cast<uint4*>(sm + K::OFF_W1 + o) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                    *reinterpret_cast<uint4*>(sm + K::OFF_W2 + o) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+                }
+            };
+
+            if (d.st) {
+                // ==== state item: the run's own state from zero, dS_r, and its
+                // log2 decay R_r; the last block combines h_in(r+1) = 2^(R_r) h_in(r) + dS_r
+                run_decay = (j == 0 ? 0.f : run_decay) + rlast;
+                {
+                    const float dl = ex2(rlast);
+#pragma unroll
+                    for (int pc = 0; pc < 2; ++pc) {
+                        uint32_t v[16];
+                        if (j > 0) {
+                            tmem_ld16(tmem + lane_off + COL_ST + half * 32 + pc * 16, v);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(dl * __uint_as_float(v[i]));
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) v[i] = 0u;
+                        }
+                        tmem_st16(tmem + lane_off + COL_ST + half * 32 + pc * 16, v);
+                    }
+                    tmem_wait_st();
+                    tc_fence_before();
+                    mbar_arrive(bar(BAR_H));
+                }
+                wait(BAR_S, ph);
+                wait(BAR_OFF, ph);
+                {
+                    uint32_t xr[16];
+                    write_wx(xr);
+                }
+                fence_proxy_async();
+                mbar_arrive(bar(BAR_WX));
+                mbar_arrive(bar(BAR_M));
+                wait(BAR_Y, ph);
+                tc_fence_after();
+                if (last_block) {
+                    wait(BAR_CHAIN, ph);              // h_in(r) is published
+                    const float dr = ex2(run_decay);
+#pragma unroll
+                    for (int pc = 0; pc < 2; ++pc) {
+                        uint32_t sv[16];
+                        tmem_ld16(tmem + lane_off + COL_ST + half * 32 + pc * 16, sv);
+                        tmem_wait_ld();
+                        float hin[16];
+                        load_entry(c, pc, hin);
+                        float* slot = slot_of(bh, c + 1) + row * PD + half * 32 + pc * 16;
+#pragma unroll
+                        for (int i = 0; i < 16; i += 4)
+                            __stcg(reinterpret_cast<float4*>(slot + i),
+                                   make_float4(fmaf(dr, hin[i], __uint_as_float(sv[i])),
+                                               fmaf(dr, hin[i + 1], __uint_as_float(sv[i + 1])),
+                                               fmaf(dr, hin[i + 2], __uint_as_float(sv[i + 2])),
+                                               fmaf(dr, hin[i + 3], __uint_as_float(sv[i + 3]))));
+                    }
+                }
+                mbar_arrive(bar(BAR_PUB));
+                tc_fence_before();
+                mbar_arrive(bar(BAR_EPI));            // no output: the Y accumulator is free
+                ++blk;
+                continue;
+            }
+
+            // ==== output item
+            // ---- h entering the block: the run's entry state (first block), else the
+            // state the previous block left in the TMEM accumulator.  Split hi -> W1,
+            // lo -> W2 for C h; 2^(r_last) h -> the state accumulator.
             {
                 const float dl = ex2(rlast);
-                float* slot = p.slots + ((long long)bh * N + row) * PD + half * 32;
                 if (j == 0) wait(BAR_CHAIN, ph);
 #pragma unroll
                 for (int pc = 0; pc < 2; ++pc) {
@@ -568,21 +721,8 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                         tmem_wait_ld();
 #pragma unroll
                         for (int i = 0; i < 16; ++i) hv[i] = __uint_as_float(v[i]);
-                    } else if (c > 0) {
-#pragma unroll
-                        for (int i = 0; i < 16; i += 4) {
-                            const float4 v = __ldcg(reinterpret_cast<const float4*>(slot + pc * 16 + i));
-                            hv[i] = v.x; hv[i + 1] = v.y; hv[i + 2] = v.z; hv[i + 3] = v.w;
-                        }
-                    } else if (p.init_state) {
-                        const long long o = ((long long)bh * N + row) * PD + half * 32 + pc * 16;
-#pragma unroll
-                        for (int i = 0; i < 16; ++i)
-                            hv[i] = p.state_bf16 ? __bfloat162float(reinterpret_cast<const bf16*>(p.init_state)[o + i])
-                                                 : reinterpret_cast<const float*>(p.init_state)[o + i];
                     } else {
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) hv[i] = 0.f;
+                        load_entry(c, pc, hv);
                     }
                     uint32_t sc[16];
 #pragma unroll
@@ -660,67 +800,39 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                 for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(el * __uint_as_float(v[i]));
                 tmem_st16(tmem + lane_off + COL_Y + half * 32 + pc * 16, v);
             }
-            // ---- w o X split hi -> W1, lo -> W2 (free: C h is done); x kept for D x
+            // ---- w o X (free: C h is done); x kept for D x
             uint32_t xr[16];
-            {
-                const float w = ex2(rlast + scs[row]);
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const uint32_t o = swz(row, half * 4 + q);
-                    const uint4 xv = *reinterpret_cast<const uint4*>(sm + K::OFF_X + o);
-                    xr[4 * q] = xv.x; xr[4 * q + 1] = xv.y; xr[4 * q + 2] = xv.z; xr[4 * q + 3] = xv.w;
-                    uint32_t hw[4], lw[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float v0 = bf16_lo(xr[4 * q + e]) * w, v1 = bf16_hi(xr[4 * q + e]) * w;
-                        hw[e] = pack_bf16(v0, v1);
-                        lw[e] = pack_bf16(v0 - bf16_lo(hw[e]), v1 - bf16_hi(hw[e]));
-                    }
-                    *reinterpret_cast<uint4*>(sm + K::OFF_W1 + o) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-                    *reinterpret_cast<uint4*>(sm + K::OFF_W2 + o) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-                }
-            }
+            write_wx(xr);
             tmem_wait_st();
             fence_proxy_async();
             tc_fence_before();
             mbar_arrive(bar(BAR_WX));
             mbar_arrive(bar(BAR_M));
 
-            // ---- after Y (and the state MMAs before it): publish the item's state,
-            // then y = (2^(r_l) Yoff + M X) + D x, staged in W1/W2, TMA store
+            // ---- after Y (and the state MMAs before it): the final state after the
+            // last block of the last run, then y = (2^(r_l) Yoff + M X) + D x, staged
+            // in W1/W2, TMA store
             wait(BAR_Y, ph);
             tc_fence_after();
-            if (last_block) {
-                const bool to_final = c == p.nruns - 1;
+            if (last_block && c == p.nruns - 1 && p.final_state) {
                 const long long fo = ((long long)bh * N + row) * PD + half * 32;
-                float* slot = p.slots + fo;
 #pragma unroll
                 for (int pc = 0; pc < 2; ++pc) {
                     uint32_t sv[16];
                     tmem_ld16(tmem + lane_off + COL_ST + half * 32 + pc * 16, sv);
                     tmem_wait_ld();
-                    if (to_final) {
-                        if (p.final_state) {
-                            float ho[16];
+                    float ho[16];
 #pragma unroll
-                            for (int i = 0; i < 16; ++i) ho[i] = __uint_as_float(sv[i]);
-                            if (p.state_bf16) {
-                                bf16* fs = reinterpret_cast<bf16*>(p.final_state) + fo + pc * 16;
-                                Vec16<bf16>::store(fs, ho);
-                                Vec16<bf16>::store(fs + 8, ho + 8);
-                            } else {
-                                float* fs = reinterpret_cast<float*>(p.final_state) + fo + pc * 16;
-#pragma unroll
-                                for (int i = 0; i < 16; i += 4)
-                                    *reinterpret_cast<float4*>(fs + i) = make_float4(ho[i], ho[i + 1], ho[i + 2], ho[i + 3]);
-                            }
-                        }
+                    for (int i = 0; i < 16; ++i) ho[i] = __uint_as_float(sv[i]);
+                    if (p.state_bf16) {
+                        bf16* fs = reinterpret_cast<bf16*>(p.final_state) + fo + pc * 16;
+                        Vec16<bf16>::store(fs, ho);
+                        Vec16<bf16>::store(fs + 8, ho + 8);
                     } else {
+                        float* fs = reinterpret_cast<float*>(p.final_state) + fo + pc * 16;
 #pragma unroll
                         for (int i = 0; i < 16; i += 4)
-                            __stcg(reinterpret_cast<float4*>(slot + pc * 16 + i),
-                                   make_float4(__uint_as_float(sv[i]), __uint_as_float(sv[i + 1]),
-                                               __uint_as_float(sv[i + 2]), __uint_as_float(sv[i + 3])));
+                            *reinterpret_cast<float4*>(fs + i) = make_float4(ho[i], ho[i + 1], ho[i + 2], ho[i + 3]);
                     }
                 }
             }
@@ -856,22 +968,14 @@ static cudaError_t launch_n(const PrefillArgs& a, cudaStream_t s) {
     p.Q = (int)a.Q;
     p.nchunks = (int)a.lay.nchunks;
     p.BH = (int)(a.batch * a.H);
-    // Runs: with as many sequences as pipelines, one item walks a whole
-    // sequence and the state never leaves the SM.  With fewer sequences the
-    // chunks are cut into runs chained through the fp32 slots.
-    {
-        const long long pipes = (long long)resident[dev] * PIPES;
-        const long long nc = p.nchunks;
-        long long Kc = nc;
-        if (2LL * p.BH < pipes) Kc = (nc * p.BH + pipes - 1) / pipes;
-        if (Kc < 1) Kc = 1;
-        p.K = (int)Kc;
-        p.nruns = (int)((nc + Kc - 1) / Kc);
-    }
+    const long long nruns = tc_runs(p.BH, p.nchunks);
+    p.nruns = (int)nruns;
+    p.K = (int)((p.nchunks + nruns - 1) / nruns);
+    p.nstate = (int)((nruns - 1) * p.BH);
     p.state_bf16 = a.state_bf16;
     p.y_bf16 = a.y_bf16;
     p.drop_publish = a.drop_publish;
-    const long long items = (long long)p.nruns * p.BH;
+    const long long items = (long long)p.nstate + (long long)p.nruns * p.BH;
     if (items > 0x7fffffffLL) return cudaErrorInvalidValue;
     const long long want = (items + PIPES - 1) / PIPES;   // each CTA runs PIPES ticket streams
     const unsigned grid = (unsigned)(want < resident[dev] ? want : resident[dev]);
@@ -880,6 +984,21 @@ static cudaError_t launch_n(const PrefillArgs& a, cudaStream_t s) {
 }
 
 }  // namespace tc
+
+// Runs per sequence.  With at least half as many sequences as the block
+// pipelines of a 148-SM part (2 per SM), every item is a whole sequence and the
+// state never leaves the SM.  Otherwise sequences are cut into runs so that
+// about 3 output items fall to each pipeline: fewer, longer items measured
+// faster than finer balance (each item pays a pipeline fill and drain, and
+// every run but the last one extra, light state item).  A pure function of the
+// shape, so that the workspace size does not depend on the device.
+int64_t tc_runs(int64_t BH, int64_t nchunks) {
+    constexpr int64_t kPipes = 148 * tc::PIPES;
+    if (nchunks <= 1 || 2 * BH >= kPipes) return 1;
+    int64_t k = (nchunks * BH + 3 * kPipes - 1) / (3 * kPipes);   // chunks per run
+    if (k < 1) k = 1;
+    return (nchunks + k - 1) / k;
+}
 
 bool tc_path_supports(int64_t P, int64_t N, int64_t Q, bool io_bf16) {
     return io_bf16 && P == tc::PD && N == 128 && (Q == 128 || Q == 256);

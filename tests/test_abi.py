@@ -63,7 +63,8 @@ def test_workspace_size_and_path():
     d = desc()
     n = ssd.ssd_chunk_scan_workspace_size(d)
     BH, Lpad = 2 * 4, 512
-    # dt + cumsum (fp32 per token and head) + one fp32 state slot per (b, h) + flags
+    # dt + cumsum (fp32 per token and head) + the fp32 entry state of every run after
+    # the first (8 sequences of 2 chunks: 2 runs each) + flags
     assert n >= 2 * 4 * BH * Lpad + 4 * BH * 128 * 64
     assert ssd.ssd_chunk_scan_path(d) == 0                       # bf16, N=128: tensor cores
     assert ssd.ssd_chunk_scan_path(desc(io_dtype=ssd.SSD_F32)) == 1   # fp32: CUDA cores

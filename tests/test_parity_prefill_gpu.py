@@ -34,6 +34,7 @@ CASES = [
     (1, 1000, 6, 64, 128, 3, 256, I.BF16),  # tensor cores, 4 chunks, ragged 232-token tail
     (2, 333, 4, 64, 64, 2, 64, I.BF16),     # bf16 on CUDA cores
     (1, 257, 2, 128, 256, 1, 128, I.BF16),
+    (1, 3918, 100, 64, 128, 4, 128, I.BF16),  # tensor cores, runs of 2 chunks, the last run 1 chunk
 ]
 
 
