@@ -120,7 +120,8 @@ ssd_status_t ssd_chunk_scan_workspace_size(const ssd_prefill_desc_t* desc, size_
 /*
  * Which kernel path ssd_chunk_scan_fwd takes for `desc` (written to *path):
  *   0 = tensor-core path (bf16 inputs; tcgen05 MMAs with TMEM accumulators fed
- *       by TMA; fp32 accumulation and fp32 state passing),
+ *       by TMA; fp32 accumulation and fp32 state passing): headdim 64,
+ *       dstate 64, 128 or 256, chunk 128 or 256,
  *   1 = CUDA-core fp32 path (fp32 inputs, or shapes the tensor-core path does
  *       not cover).
  * Pure host function.

@@ -83,7 +83,7 @@ static PrefillLayout prefill_layout(const ssd_prefill_desc_t* d, bool tc) {
     const size_t state_elems = (size_t)d->dstate * d->headdim;
     // CUDA-core path: one state per chunk; tensor-core path: the entry state of
     // every run after the first
-    const int64_t nstates = tc ? tc_runs(BH, lay.nchunks) - 1 : lay.nchunks;
+    const int64_t nstates = tc ? tc_runs(BH, lay.nchunks, d->dstate) - 1 : lay.nchunks;
     off = align256(off + sizeof(float) * state_elems * (size_t)BH * (size_t)nstates);
     lay.off_flags = off;
     off = align256(off + sizeof(int) * ((size_t)BH + 64));

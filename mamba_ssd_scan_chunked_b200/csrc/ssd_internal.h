@@ -50,7 +50,7 @@ cudaError_t launch_prefill_simt(const PrefillArgs& a, cudaStream_t s);
 // tensor-core prefill path; returns cudaErrorNotSupported when the shape is not covered
 bool tc_path_supports(int64_t P, int64_t N, int64_t Q, bool io_bf16);
 // runs per sequence of the tensor-core path (1 = every work item is a whole sequence)
-int64_t tc_runs(int64_t BH, int64_t nchunks);
+int64_t tc_runs(int64_t BH, int64_t nchunks, int64_t N);
 cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s);
 
 // fault-injection bits set by ssd_debug_inject (read at every launch)

@@ -59,36 +59,44 @@ namespace tc {
 
 constexpr int SUB = 128;        // tokens per block (MMA M)
 constexpr int PD = 64;          // headdim handled by this path
-constexpr int PIPES = 2;        // independent block pipelines per CTA (one CTA per SM)
 constexpr int NCOMPUTE = 256;   // compute threads of a pipeline: 8 warps; warps w and w+4 share TMEM lanes 32*(w%4)..+31
 // thread layout: warps 8p..8p+7 compute for pipeline p, then one control warp per
 // pipeline.  A warp may only touch TMEM lanes 32*(warp % 4), so compute warps
 // must start at a multiple of 4 warps: they come first.
-constexpr int THREADS = PIPES * (NCOMPUTE + 32);
 constexpr uint32_t TILE = SUB * 128;   // [128 rows x 64 bf16] SW128 tile = 16 KB
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr unsigned long long WAIT_NS = 2000000000ull;   // bound of every device-side wait
 
-// TMEM columns (256 allocated)
-constexpr uint32_t COL_R = 0;     // S (fp32 128) -> M hi|lo (bf16x2 64+64) -> Yoff (fp32 64)
-constexpr uint32_t COL_Y = 128;   // Y accumulator (fp32 64)
-constexpr uint32_t COL_ST = 192;  // chunk-state accumulator (fp32 64, lanes = n)
-constexpr uint32_t PIPE_COLS = 256;              // TMEM columns of one pipeline
-constexpr uint32_t TMEM_COLS = PIPES * PIPE_COLS;
+// TMEM columns of a pipeline
+constexpr uint32_t COL_R = 0;     // S (fp32 128) -> M hi|lo (bf16x2 64+64)
+constexpr uint32_t COL_Y = 128;   // Yoff, then Y (fp32 64)
+constexpr uint32_t COL_ST = 192;  // chunk-state accumulator: fp32 64 per 128 state rows (lane = n % 128)
 
 // control words after the per-(b,h) flags
 constexpr int CTRL_TICKET = 0;
 constexpr int CTRL_ABORT = 1;
 
+// dstate N = 64, 128 or 256.  dstate 64 keeps the layout of 128 with B
+// zero-padded: its chunk state is an M=128 MMA whose upper 64 rows stay zero,
+// while C B^T and C h take only the 4 valid K steps.  dstate 256 needs 208 KB of
+// tiles, so it runs one pipeline per CTA, with the state in two 128-row halves.
 template <int N>
 struct Cfg {
-    static constexpr int KB = N / 64;                       // 64-wide K blocks of C, B
+    static constexpr int NP = N < 128 ? 128 : N;            // state rows held (padded)
+    static constexpr int KB = NP / 64;                      // 64-wide K blocks of C, B in smem
+    static constexpr int KBV = N / 64;                      // ... of them loaded (the rest stays zero)
+    static constexpr int NB = NP / 128;                     // 128-row blocks of the state
+    static constexpr int PIPES = N > 128 ? 1 : 2;           // block pipelines per CTA (one CTA per SM)
+    static constexpr int THREADS = PIPES * (NCOMPUTE + 32);
+    static constexpr uint32_t PIPE_COLS = COL_ST + 64 * NB <= 256 ? 256 : 512;   // TMEM columns of a pipeline
+    static constexpr uint32_t TMEM_COLS = PIPES * PIPE_COLS;
+    static_assert(TMEM_COLS <= 512, "TMEM");
     // tiles of one pipeline (1024-byte aligned, 128-byte swizzle)
     static constexpr uint32_t OFF_C = 0;
     static constexpr uint32_t OFF_B = OFF_C + KB * TILE;
     static constexpr uint32_t OFF_X = OFF_B + KB * TILE;
     // W1/W2: hi/lo halves of w o X, then of h (MN-major operands), then the y staging tile
-    static constexpr uint32_t W_BYTES = (N > SUB ? N : SUB) * 128;
+    static constexpr uint32_t W_BYTES = NP * 128;
     static constexpr uint32_t OFF_W1 = OFF_X + TILE;
     static constexpr uint32_t OFF_W2 = OFF_W1 + W_BYTES;
     static constexpr uint32_t TILES = OFF_W2 + W_BYTES;
@@ -99,9 +107,10 @@ struct Cfg {
     static constexpr uint32_t OFF_MISC = OFF_BAR + 80;       // tmem base, block coordinates
     static constexpr uint32_t SMALL = OFF_MISC + 64;
     static constexpr uint32_t SMEM = PIPES * (TILES + SMALL);
-    static constexpr uint32_t TX = (2 * KB + 1) * TILE + 2 * SUB * 4;   // TMA bytes per block
-    static constexpr uint32_t TX_ST = (KB + 1) * TILE + 2 * SUB * 4;    // ... of a state item (no C)
+    static constexpr uint32_t TX = (2 * KBV + 1) * TILE + 2 * SUB * 4;   // TMA bytes per block
+    static constexpr uint32_t TX_ST = (KBV + 1) * TILE + 2 * SUB * 4;    // ... of a state item (no C)
     static_assert(TILES % 1024 == 0 && SMALL % 16 == 0, "alignment");
+    static_assert(SMEM <= 232448, "shared memory per CTA");
 };
 
 struct Params {
@@ -292,7 +301,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
 }
 
 // ---------------------------------------------------------------- the kernel
-// Persistent, one CTA per SM, PIPES independent block pipelines per CTA.  A
+// Persistent, one CTA per SM, Cfg::PIPES independent block pipelines per CTA.  A
 // pipeline = 8 compute warps (256 threads; thread = one TMEM lane/tile row and
 // one half of its columns) + 1 control warp, converged, whose elected lane
 // takes tickets, issues every TMA and MMA, waits for run-entry states and
@@ -306,11 +315,12 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
 // R only holds S/M, so the next block's loads and C B^T start as soon as Y is
 // done, overlapping this block's epilogue.
 template <int N>
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(Cfg<N>::THREADS, 1)
 ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
               const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmY, const Params p) {
     using K = Cfg<N>;
-    static_assert(N == 128, "this instantiation covers dstate 128");
+    static_assert(N == 64 || N == 128 || N == 256, "dstate 64, 128 or 256");
+    constexpr int PIPES = K::PIPES;
     extern __shared__ __align__(1024) uint8_t smem_all[];
     const bool control = threadIdx.x >= PIPES * NCOMPUTE;   // a pipeline's control warp
     const int pipe = control ? (threadIdx.x - PIPES * NCOMPUTE) / 32 : threadIdx.x / NCOMPUTE;
@@ -345,8 +355,14 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
     // TMEM first, then tickets (a ticket holder never waits for TMEM)
     if (threadIdx.x < 32) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
-                     ::"r"(smem_u32(s_tmem_slot)), "r"(TMEM_COLS) : "memory");
+                     ::"r"(smem_u32(s_tmem_slot)), "r"(K::TMEM_COLS) : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    // dstate 64: the B tile of state rows 64..127 is never loaded; zero it once
+    if (K::KBV < K::KB && !control) {
+        uint4* z = reinterpret_cast<uint4*>(sm + K::OFF_B + K::KBV * TILE);
+        for (int i = tid; i < (K::KB - K::KBV) * (int)TILE / 16; i += NCOMPUTE) z[i] = make_uint4(0u, 0u, 0u, 0u);
+        fence_proxy_async();
     }
     if (!control && tid == 0) {
         //                        TMA S  CHAIN H         OFF WX        M         Y  PUB       EPI
@@ -358,7 +374,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
     __syncthreads();
     tc_fence_after();
     // the pipeline's 256 columns of the CTA's allocation (address = lane << 16 | column)
-    const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(s_tmem_slot) + PIPE_COLS * pipe;
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(s_tmem_slot) + K::PIPE_COLS * pipe;
     auto wait = [&](int i, uint32_t ph) {
         if (!mbar_wait(bar(i), ph)) err |= kErrAsyncTimeout;
     };
@@ -402,6 +418,20 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
             const uint64_t dW1 = sdesc(base + K::OFF_W1, TILE, 1024);   // MN-major (state, Yoff)
             const uint64_t dW2 = sdesc(base + K::OFF_W2, TILE, 1024);
             constexpr uint32_t KSTEP_K = 2, KBLOCK_K = TILE >> 4, KSTEP_MN = 2048 >> 4;
+            // chunk-state MMAs: onto the state accumulator, B^T (w o X)_hi and
+            // B^T (w o X)_lo (K = 128 tokens), one M=128 MMA per 128 state rows
+            auto issue_state = [&]() {
+#pragma unroll
+                for (int nb = 0; nb < K::NB; ++nb) {
+                    const uint64_t a0 = dBm + (uint64_t)((2u * TILE * nb) >> 4);   // B tiles 2nb, 2nb+1
+#pragma unroll
+                    for (int k = 0; k < SUB / 16; ++k)
+                        if (lead) mma_ss<ID_ST, 1>(tmem + COL_ST + 64 * nb, a0 + k * KSTEP_MN, dW1 + k * KSTEP_MN);
+#pragma unroll
+                    for (int k = 0; k < SUB / 16; ++k)
+                        if (lead) mma_ss<ID_ST, 1>(tmem + COL_ST + 64 * nb, a0 + k * KSTEP_MN, dW2 + k * KSTEP_MN);
+                }
+            };
             // publish the block's coordinates, then load its operands and per-token terms
             auto load_block = [&](int it, int j) {
                 __syncwarp();
@@ -422,7 +452,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                 fence_proxy_async();
                 mbar_expect_tx(bar(BAR_TMA), d_.st ? K::TX_ST : K::TX);   // a state item needs no C
 #pragma unroll
-                for (int kb = 0; kb < K::KB; ++kb) {
+                for (int kb = 0; kb < K::KBV; ++kb) {
                     if (!d_.st) tma_load_4d(base + K::OFF_C + kb * TILE, &tmC, kb * 64, g_, t0_, b_, bar(BAR_TMA));
                     tma_load_4d(base + K::OFF_B + kb * TILE, &tmB, kb * 64, g_, t0_, b_, bar(BAR_TMA));
                 }
@@ -433,7 +463,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                 // the next block of the item into L2 while this one is processed
                 if (j + 1 < nblocks(it)) {
 #pragma unroll
-                    for (int kb = 0; kb < K::KB; ++kb) {
+                    for (int kb = 0; kb < K::KBV; ++kb) {
                         if (!d_.st) tma_prefetch_4d(&tmC, kb * 64, g_, t0_ + SUB, b_);
                         tma_prefetch_4d(&tmB, kb * 64, g_, t0_ + SUB, b_);
                     }
@@ -481,12 +511,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                     wait(BAR_WX, ph);
                     tc_fence_after();
                     __syncwarp();
-#pragma unroll
-                    for (int k = 0; k < SUB / 16; ++k)
-                        if (lead) mma_ss<ID_ST, 1>(tmem + COL_ST, dBm + k * KSTEP_MN, dW1 + k * KSTEP_MN);
-#pragma unroll
-                    for (int k = 0; k < SUB / 16; ++k)
-                        if (lead) mma_ss<ID_ST, 1>(tmem + COL_ST, dBm + k * KSTEP_MN, dW2 + k * KSTEP_MN);
+                    issue_state();
                     wait(BAR_M, ph);
                     if (lead) mma_commit(bar(BAR_Y));
                     // the combine of the last block needs h_in(r), published by state
@@ -530,12 +555,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                     wait(BAR_WX, ph);
                     tc_fence_after();
                     __syncwarp();
-#pragma unroll
-                    for (int k = 0; k < SUB / 16; ++k)
-                        if (lead) mma_ss<ID_ST, 1>(tmem + COL_ST, dBm + k * KSTEP_MN, dW1 + k * KSTEP_MN);
-#pragma unroll
-                    for (int k = 0; k < SUB / 16; ++k)
-                        if (lead) mma_ss<ID_ST, 1>(tmem + COL_ST, dBm + k * KSTEP_MN, dW2 + k * KSTEP_MN);
+                    issue_state();
                     // ---- Y += M_hi X + M_lo X onto the scaled Yoff (A from TMEM)
                     wait(BAR_M, ph);
                     tc_fence_after();
@@ -602,18 +622,23 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
             csync();
             prev_last = s_acs[SUB - 1];
 
-            // h_in(r) of this thread's row and 16 of its columns: the initial state
-            // (r = 0) or the run's entry-state slot
-            auto load_entry = [&](int r, int pc, float (&hv)[16]) {
-                if (r > 0) {
-                    const float* slot = slot_of(bh, r) + row * PD + half * 32 + pc * 16;
+            // h_in(r) of state row n = row + 128 nb and 16 of this thread's columns:
+            // the initial state (r = 0) or the run's entry-state slot; 0 for the
+            // padding rows n >= N
+            auto load_entry = [&](int r, int nb, int pc, float (&hv)[16]) {
+                const int n = row + 128 * nb;
+                if (n >= N) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) hv[i] = 0.f;
+                } else if (r > 0) {
+                    const float* slot = slot_of(bh, r) + n * PD + half * 32 + pc * 16;
 #pragma unroll
                     for (int i = 0; i < 16; i += 4) {
                         const float4 v = __ldcg(reinterpret_cast<const float4*>(slot + i));
                         hv[i] = v.x; hv[i + 1] = v.y; hv[i + 2] = v.z; hv[i + 3] = v.w;
                     }
                 } else if (p.init_state) {
-                    const long long o = ((long long)bh * N + row) * PD + half * 32 + pc * 16;
+                    const long long o = ((long long)bh * N + n) * PD + half * 32 + pc * 16;
 #pragma unroll
                     for (int i = 0; i < 16; ++i)
                         hv[i] = p.state_bf16 ? __bfloat162float(reinterpret_cast<const bf16*>(p.init_state)[o + i])
@@ -650,10 +675,11 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                 {
                     const float dl = ex2(rlast);
 #pragma unroll
-                    for (int pc = 0; pc < 2; ++pc) {
+                    for (int q = 0; q < 2 * K::NB; ++q) {   // (row block, 16-column part)
+                        const uint32_t col = COL_ST + 64 * (q >> 1) + half * 32 + (q & 1) * 16;
                         uint32_t v[16];
                         if (j > 0) {
-                            tmem_ld16(tmem + lane_off + COL_ST + half * 32 + pc * 16, v);
+                            tmem_ld16(tmem + lane_off + col, v);
                             tmem_wait_ld();
 #pragma unroll
                             for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(dl * __uint_as_float(v[i]));
@@ -661,7 +687,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
 #pragma unroll
                             for (int i = 0; i < 16; ++i) v[i] = 0u;
                         }
-                        tmem_st16(tmem + lane_off + COL_ST + half * 32 + pc * 16, v);
+                        tmem_st16(tmem + lane_off + col, v);
                     }
                     tmem_wait_st();
                     tc_fence_before();
@@ -682,13 +708,15 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                     wait(BAR_CHAIN, ph);              // h_in(r) is published
                     const float dr = ex2(run_decay);
 #pragma unroll
-                    for (int pc = 0; pc < 2; ++pc) {
+                    for (int q = 0; q < 2 * K::NB; ++q) {
+                        const int nb = q >> 1, pc = q & 1;
+                        if (row + 128 * nb >= N) continue;     // padding rows (warp-uniform: N % 32 == 0)
                         uint32_t sv[16];
-                        tmem_ld16(tmem + lane_off + COL_ST + half * 32 + pc * 16, sv);
+                        tmem_ld16(tmem + lane_off + COL_ST + 64 * nb + half * 32 + pc * 16, sv);
                         tmem_wait_ld();
                         float hin[16];
-                        load_entry(c, pc, hin);
-                        float* slot = slot_of(bh, c + 1) + row * PD + half * 32 + pc * 16;
+                        load_entry(c, nb, pc, hin);
+                        float* slot = slot_of(bh, c + 1) + (row + 128 * nb) * PD + half * 32 + pc * 16;
 #pragma unroll
                         for (int i = 0; i < 16; i += 4)
                             __stcg(reinterpret_cast<float4*>(slot + i),
@@ -713,21 +741,23 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                 const float dl = ex2(rlast);
                 if (j == 0) wait(BAR_CHAIN, ph);
 #pragma unroll
-                for (int pc = 0; pc < 2; ++pc) {
+                for (int qq = 0; qq < 2 * K::NB; ++qq) {   // (row block, 16-column part)
+                    const int nb = qq >> 1, pc = qq & 1;
+                    const uint32_t col = COL_ST + 64 * nb + half * 32 + pc * 16;
                     float hv[16];
                     if (j > 0) {
                         uint32_t v[16];
-                        tmem_ld16(tmem + lane_off + COL_ST + half * 32 + pc * 16, v);
+                        tmem_ld16(tmem + lane_off + col, v);
                         tmem_wait_ld();
 #pragma unroll
                         for (int i = 0; i < 16; ++i) hv[i] = __uint_as_float(v[i]);
                     } else {
-                        load_entry(c, pc, hv);
+                        load_entry(c, nb, pc, hv);
                     }
                     uint32_t sc[16];
 #pragma unroll
                     for (int i = 0; i < 16; ++i) sc[i] = __float_as_uint(dl * hv[i]);
-                    tmem_st16(tmem + lane_off + COL_ST + half * 32 + pc * 16, sc);
+                    tmem_st16(tmem + lane_off + col, sc);
 #pragma unroll
                     for (int q = 0; q < 2; ++q) {
                         uint32_t hw[4], lw[4];
@@ -737,7 +767,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                             hw[e] = pack_bf16(v0, v1);
                             lw[e] = pack_bf16(v0 - bf16_lo(hw[e]), v1 - bf16_hi(hw[e]));
                         }
-                        const uint32_t o = swz(row, half * 4 + pc * 2 + q);
+                        const uint32_t o = swz(row + 128 * nb, half * 4 + pc * 2 + q);
                         *reinterpret_cast<uint4*>(sm + K::OFF_W1 + o) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
                         *reinterpret_cast<uint4*>(sm + K::OFF_W2 + o) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
                     }
@@ -815,11 +845,14 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
             wait(BAR_Y, ph);
             tc_fence_after();
             if (last_block && c == p.nruns - 1 && p.final_state) {
-                const long long fo = ((long long)bh * N + row) * PD + half * 32;
 #pragma unroll
-                for (int pc = 0; pc < 2; ++pc) {
+                for (int q = 0; q < 2 * K::NB; ++q) {
+                    const int nb = q >> 1, pc = q & 1;
+                    const int n = row + 128 * nb;
+                    if (n >= N) continue;                 // padding rows (warp-uniform: N % 32 == 0)
+                    const long long fo = ((long long)bh * N + n) * PD + half * 32;
                     uint32_t sv[16];
-                    tmem_ld16(tmem + lane_off + COL_ST + half * 32 + pc * 16, sv);
+                    tmem_ld16(tmem + lane_off + COL_ST + 64 * nb + half * 32 + pc * 16, sv);
                     tmem_wait_ld();
                     float ho[16];
 #pragma unroll
@@ -887,7 +920,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
     if (threadIdx.x < 32) {
         tc_fence_after();
         const uint32_t tmem_all = *reinterpret_cast<volatile uint32_t*>(s_tmem_slot);
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_all), "r"(TMEM_COLS) : "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_all), "r"(K::TMEM_COLS) : "memory");
     }
 }
 
@@ -944,7 +977,7 @@ static cudaError_t launch_n(const PrefillArgs& a, cudaStream_t s) {
             e = cudaFuncSetAttribute(ssd_tc_kernel<N>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)K::SMEM);
             if (e != cudaSuccess) return e;
             int per_sm = 0, sms = 0;
-            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ssd_tc_kernel<N>, THREADS, K::SMEM);
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ssd_tc_kernel<N>, K::THREADS, K::SMEM);
             if (e != cudaSuccess) return e;
             e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
             if (e != cudaSuccess) return e;
@@ -968,7 +1001,7 @@ static cudaError_t launch_n(const PrefillArgs& a, cudaStream_t s) {
     p.Q = (int)a.Q;
     p.nchunks = (int)a.lay.nchunks;
     p.BH = (int)(a.batch * a.H);
-    const long long nruns = tc_runs(p.BH, p.nchunks);
+    const long long nruns = tc_runs(p.BH, p.nchunks, N);
     p.nruns = (int)nruns;
     p.K = (int)((p.nchunks + nruns - 1) / nruns);
     p.nstate = (int)((nruns - 1) * p.BH);
@@ -977,23 +1010,23 @@ static cudaError_t launch_n(const PrefillArgs& a, cudaStream_t s) {
     p.drop_publish = a.drop_publish;
     const long long items = (long long)p.nstate + (long long)p.nruns * p.BH;
     if (items > 0x7fffffffLL) return cudaErrorInvalidValue;
-    const long long want = (items + PIPES - 1) / PIPES;   // each CTA runs PIPES ticket streams
+    const long long want = (items + K::PIPES - 1) / K::PIPES;   // each CTA runs PIPES ticket streams
     const unsigned grid = (unsigned)(want < resident[dev] ? want : resident[dev]);
-    ssd_tc_kernel<N><<<grid, THREADS, K::SMEM, s>>>(mx, mb, mc, my, p);
+    ssd_tc_kernel<N><<<grid, K::THREADS, K::SMEM, s>>>(mx, mb, mc, my, p);
     return cudaGetLastError();
 }
 
 }  // namespace tc
 
 // Runs per sequence.  With at least half as many sequences as the block
-// pipelines of a 148-SM part (2 per SM), every item is a whole sequence and the
+// pipelines of a 148-SM part (1 or 2 per SM), every item is a whole sequence and the
 // state never leaves the SM.  Otherwise sequences are cut into runs so that
 // about 3 output items fall to each pipeline: fewer, longer items measured
 // faster than finer balance (each item pays a pipeline fill and drain, and
 // every run but the last one extra, light state item).  A pure function of the
 // shape, so that the workspace size does not depend on the device.
-int64_t tc_runs(int64_t BH, int64_t nchunks) {
-    constexpr int64_t kPipes = 148 * tc::PIPES;
+int64_t tc_runs(int64_t BH, int64_t nchunks, int64_t N) {
+    const int64_t kPipes = 148 * (N > 128 ? tc::Cfg<256>::PIPES : tc::Cfg<128>::PIPES);
     if (nchunks <= 1 || 2 * BH >= kPipes) return 1;
     int64_t k = (nchunks * BH + 3 * kPipes - 1) / (3 * kPipes);   // chunks per run
     if (k < 1) k = 1;
@@ -1001,12 +1034,16 @@ int64_t tc_runs(int64_t BH, int64_t nchunks) {
 }
 
 bool tc_path_supports(int64_t P, int64_t N, int64_t Q, bool io_bf16) {
-    return io_bf16 && P == tc::PD && N == 128 && (Q == 128 || Q == 256);
+    return io_bf16 && P == tc::PD && (N == 64 || N == 128 || N == 256) && (Q == 128 || Q == 256);
 }
 
 cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
     if (!tc_path_supports(a.P, a.N, a.Q, a.io_bf16)) return cudaErrorNotSupported;
-    return tc::launch_n<128>(a, s);
+    switch (a.N) {
+        case 64: return tc::launch_n<64>(a, s);
+        case 128: return tc::launch_n<128>(a, s);
+        default: return tc::launch_n<256>(a, s);
+    }
 }
 
 }  // namespace ssd

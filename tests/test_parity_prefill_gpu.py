@@ -34,7 +34,11 @@ CASES = [
     (1, 1000, 6, 64, 128, 3, 256, I.BF16),  # tensor cores, 4 chunks, ragged 232-token tail
     (2, 333, 4, 64, 64, 2, 64, I.BF16),     # bf16 on CUDA cores
     (1, 257, 2, 128, 256, 1, 128, I.BF16),
-    (1, 3918, 100, 64, 128, 4, 128, I.BF16),  # tensor cores, runs of 2 chunks, the last run 1 chunk
+    (1, 3918, 100, 64, 128, 4, 128, I.BF16),  # tensor cores, runs of 4 chunks, the last run 3 chunks
+    (2, 600, 4, 64, 64, 2, 256, I.BF16),    # dstate 64 on tensor cores (zero-padded B), runs
+    (1, 2100, 90, 64, 64, 3, 256, I.BF16),  # dstate 64, 90 sequences cut into runs of 1 chunk
+    (1, 1000, 6, 64, 256, 3, 128, I.BF16),  # dstate 256: one pipeline per SM, two state halves, runs
+    (2, 1500, 80, 64, 256, 8, 256, I.BF16), # dstate 256, whole sequences, 160 items on 148 CTAs
 ]
 
 
@@ -51,12 +55,15 @@ def test_prefill_matches_oracle(case, with_init):
     assert metric(fs, fs_ref) <= tol
 
 
-def test_tensor_core_path_is_taken_for_bf16_dstate128():
-    inp = shape_inputs(1, 256, 2, 64, 128, 1, I.BF16, 3)
+@pytest.mark.parametrize("N", [64, 128, 256])
+def test_tensor_core_path_is_taken_for_bf16_headdim64(N):
+    inp = shape_inputs(1, 256, 2, 64, N, 1, I.BF16, 3)
     assert path_of(inp, 256) == 0
     assert path_of(inp, 128) == 0
-    inp32 = shape_inputs(1, 256, 2, 64, 128, 1, I.F32, 3)
+    assert path_of(inp, 64) == 1                      # chunk 64: CUDA cores
+    inp32 = shape_inputs(1, 256, 2, 64, N, 1, I.F32, 3)
     assert path_of(inp32, 256) == 1
+    assert path_of(shape_inputs(1, 256, 2, 64, 32, 1, I.BF16, 3), 256) == 1   # dstate 32: CUDA cores
 
 
 def test_tensor_core_error_budget_is_far_inside_the_bound():
