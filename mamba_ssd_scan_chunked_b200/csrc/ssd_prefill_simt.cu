@@ -23,60 +23,71 @@
 namespace ssd {
 
 // --------------------------------------------------------------------------
-// dt and chunk-local decay cumsum.  1-D grid over (b*H) x nchunks, block
-// max(Q, 32) threads.
+// dt and chunk-local decay cumsum.  One block per (batch b, chunk c, group of
+// DT_HG consecutive heads); thread l = token l of the chunk.  A thread reads
+// its token's DT_HG heads (contiguous in dt_raw [b][L][H]; independent loads,
+// all in flight at once), applies softplus and dt * A, and the block scans the
+// DT_HG columns over its tokens at once: warp shuffles, then the warp totals
+// through shared memory.  dt and the cumsum go out as coalesced rows of
+// [b*H][Lpad] (a warp writes 32 consecutive tokens of one head).
 // --------------------------------------------------------------------------
+constexpr int DT_HG = 8;         // heads per block
+
 template <typename IoT>
-__global__ void dt_cumsum_kernel(const IoT* __restrict__ dt_raw, const float* __restrict__ dt_bias,
-                                 const float* __restrict__ A, float* __restrict__ dt_out,
-                                 float* __restrict__ acs_out, int* __restrict__ flags,
-                                 int64_t L, int64_t Lpad, int H, int Q, int nflags, int nchunks, int BH) {
-    __shared__ float warp_tot[32];
-    const int c = (int)(blockIdx.x % (unsigned)nchunks);
-    const int bh = (int)(blockIdx.x / (unsigned)nchunks);
-    const int b = bh / H, h = bh % H;
-    const int l = threadIdx.x;
-    const int64_t t = (int64_t)c * Q + l;
-    float dt = 0.f, a = 0.f;
-    if (l < Q && t < L) {
-        dt = softplus_f32(to_f32(dt_raw[((int64_t)b * L + t) * H + h]) + (dt_bias ? dt_bias[h] : 0.f));
-        a = dt * A[h];
-    }
-    // inclusive block scan of a (warp shuffles, then a scan of warp totals)
+__global__ void __launch_bounds__(256)
+dt_cumsum_kernel(const IoT* __restrict__ dt_raw, const float* __restrict__ dt_bias,
+                 const float* __restrict__ A, float* __restrict__ dt_out,
+                 float* __restrict__ acs_out, int* __restrict__ flags,
+                 int64_t L, int64_t Lpad, int H, int Q, int nflags, int nchunks, int hgroups) {
+    __shared__ float warp_tot[8][DT_HG];       // Q <= 256: at most 8 warps
+    const int hg = (int)(blockIdx.x % (unsigned)hgroups);
+    const int c = (int)((blockIdx.x / (unsigned)hgroups) % (unsigned)nchunks);
+    const int b = (int)(blockIdx.x / ((unsigned)hgroups * (unsigned)nchunks));
+    const int h0 = hg * DT_HG;
+    const int l = threadIdx.x;                 // token within the chunk (blockDim = max(Q, 32))
     const int lane = l & 31, warp = l >> 5;
-    float v = a;
+    const int64_t t = (int64_t)c * Q + l;
+    const bool live = l < Q && t < L;
+    float raw[DT_HG];
+#pragma unroll
+    for (int k = 0; k < DT_HG; ++k)
+        raw[k] = (live && h0 + k < H) ? to_f32(dt_raw[((int64_t)b * L + t) * H + h0 + k]) : 0.f;
+    float dt[DT_HG], v[DT_HG];
+#pragma unroll
+    for (int k = 0; k < DT_HG; ++k) {
+        const int h = h0 + k;
+        dt[k] = (live && h < H) ? softplus_f32(raw[k] + (dt_bias ? dt_bias[h] : 0.f)) : 0.f;
+        v[k] = h < H ? dt[k] * A[h] : 0.f;
+    }
+    // inclusive scan over the tokens, DT_HG columns at once
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-        const float u = __shfl_up_sync(0xffffffffu, v, o);
-        if (lane >= o) v += u;
-    }
-    if (lane == 31) warp_tot[warp] = v;
-    __syncthreads();
-    if (warp == 0) {
-        const int nw = (Q + 31) / 32;
-        float w = lane < nw ? warp_tot[lane] : 0.f;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const float u = __shfl_up_sync(0xffffffffu, w, o);
-            if (lane >= o) w += u;
+        for (int k = 0; k < DT_HG; ++k) {
+            const float u = __shfl_up_sync(0xffffffffu, v[k], o);
+            if (lane >= o) v[k] += u;
         }
-        if (lane < nw) warp_tot[lane] = w;
     }
+    if (lane == 31)
+#pragma unroll
+        for (int k = 0; k < DT_HG; ++k) warp_tot[warp][k] = v[k];
     __syncthreads();
-    if (warp > 0) v += warp_tot[warp - 1];
-    const int64_t o = (int64_t)bh * Lpad + t;
+    for (int w = 0; w < warp; ++w)
+#pragma unroll
+        for (int k = 0; k < DT_HG; ++k) v[k] += warp_tot[w][k];
     if (l < Q) {
-        dt_out[o] = dt;
-        acs_out[o] = v;
-    }
-    // reset the inter-chunk progress flags and control words of this launch
-    if (c == 0) {
-        const int per = (nflags + BH - 1) / BH;
-        for (int i = l; i < per; i += blockDim.x) {
-            const int k = bh * per + i;
-            if (k < nflags) flags[k] = 0;
+#pragma unroll
+        for (int k = 0; k < DT_HG; ++k) {
+            if (h0 + k >= H) break;
+            const int64_t o = ((int64_t)b * H + h0 + k) * Lpad + t;
+            dt_out[o] = dt[k];
+            acs_out[o] = v[k];
         }
     }
+    // reset the run hand-off flags and control words of this launch (a slice per block)
+    const int per = (int)((nflags + gridDim.x - 1) / gridDim.x);
+    const int f0 = (int)blockIdx.x * per;
+    for (int i = f0 + l; i < nflags && i < f0 + per; i += blockDim.x) flags[i] = 0;
 }
 
 template <typename IoT>
@@ -85,11 +96,13 @@ static cudaError_t launch_dt_t(const PrefillArgs& a, cudaStream_t s) {
     float* acs = (float*)(a.ws + a.lay.off_acs);
     int* flags = (int*)(a.ws + a.lay.off_flags);
     const int nflags = (int)(a.batch * a.H + 64);
-    const unsigned blocks = (unsigned)(a.lay.nchunks * a.batch * a.H);
+    const int hgroups = (int)((a.H + DT_HG - 1) / DT_HG);
+    const long long blocks = a.lay.nchunks * a.batch * hgroups;
+    if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
     const unsigned threads = (unsigned)(a.Q < 32 ? 32 : a.Q);   // whole warps for the shuffles
-    dt_cumsum_kernel<IoT><<<blocks, threads, 0, s>>>((const IoT*)a.dt_raw, a.dt_bias, a.A, dt, acs, flags, a.L,
-                                                    a.lay.Lpad, (int)a.H, (int)a.Q, nflags, (int)a.lay.nchunks,
-                                                    (int)(a.batch * a.H));
+    dt_cumsum_kernel<IoT><<<(unsigned)blocks, threads, 0, s>>>(
+        (const IoT*)a.dt_raw, a.dt_bias, a.A, dt, acs, flags, a.L, a.lay.Lpad, (int)a.H, (int)a.Q, nflags,
+        (int)a.lay.nchunks, hgroups);
     return cudaGetLastError();
 }
 

@@ -314,7 +314,8 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
 // accumulator, scaled by 2^(r_l) in place, and M X accumulates on top.  Region
 // R only holds S/M, so the next block's loads and C B^T start as soon as Y is
 // done, overlapping this block's epilogue.
-template <int N>
+// RUNS: sequences are cut into runs (state items and run hand-offs present)
+template <int N, bool RUNS>
 __global__ void __launch_bounds__(Cfg<N>::THREADS, 1)
 ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
               const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmY, const Params p) {
@@ -383,7 +384,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
     struct Item { int st, r, bh; };
     auto decode = [&](int it) -> Item {
         Item d;
-        d.st = it < p.nstate;
+        d.st = RUNS && it < p.nstate;
         const int k = d.st ? it : it - p.nstate;
         d.r = k / p.BH;
         d.bh = k % p.BH;
@@ -529,7 +530,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                     }
                     if (lead) mma_commit(bar(BAR_S));
                     // ---- an output item starts from the entry state of its run
-                    if (j == 0 && d.r > 0 && lead) chain_wait(d.bh, d.r);
+                    if (RUNS && j == 0 && d.r > 0 && lead) chain_wait(d.bh, d.r);
                     __syncwarp();
                     if (lead) mbar_arrive(bar(BAR_CHAIN));
                     // ---- Yoff = C h_hi + C h_lo into the Y accumulator (once the previous
@@ -627,10 +628,10 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
             // padding rows n >= N
             auto load_entry = [&](int r, int nb, int pc, float (&hv)[16]) {
                 const int n = row + 128 * nb;
-                if (n >= N) {
+                if (N < 128 && n >= N) {
 #pragma unroll
                     for (int i = 0; i < 16; ++i) hv[i] = 0.f;
-                } else if (r > 0) {
+                } else if (RUNS && r > 0) {
                     const float* slot = slot_of(bh, r) + n * PD + half * 32 + pc * 16;
 #pragma unroll
                     for (int i = 0; i < 16; i += 4) {
@@ -710,7 +711,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
 #pragma unroll
                     for (int q = 0; q < 2 * K::NB; ++q) {
                         const int nb = q >> 1, pc = q & 1;
-                        if (row + 128 * nb >= N) continue;     // padding rows (warp-uniform: N % 32 == 0)
+                        if (N < 128 && row + 128 * nb >= N) continue;   // padding rows (warp-uniform: N % 32 == 0)
                         uint32_t sv[16];
                         tmem_ld16(tmem + lane_off + COL_ST + 64 * nb + half * 32 + pc * 16, sv);
                         tmem_wait_ld();
@@ -849,7 +850,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                 for (int q = 0; q < 2 * K::NB; ++q) {
                     const int nb = q >> 1, pc = q & 1;
                     const int n = row + 128 * nb;
-                    if (n >= N) continue;                 // padding rows (warp-uniform: N % 32 == 0)
+                    if (N < 128 && n >= N) continue;     // padding rows (warp-uniform: N % 32 == 0)
                     const long long fo = ((long long)bh * N + n) * PD + half * 32;
                     uint32_t sv[16];
                     tmem_ld16(tmem + lane_off + COL_ST + 64 * nb + half * 32 + pc * 16, sv);
@@ -974,10 +975,12 @@ static cudaError_t launch_n(const PrefillArgs& a, cudaStream_t s) {
     {
         std::lock_guard<std::mutex> lk(mu);
         if (!resident[dev]) {
-            e = cudaFuncSetAttribute(ssd_tc_kernel<N>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)K::SMEM);
+            e = cudaFuncSetAttribute(ssd_tc_kernel<N, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)K::SMEM);
+            if (e != cudaSuccess) return e;
+            e = cudaFuncSetAttribute(ssd_tc_kernel<N, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)K::SMEM);
             if (e != cudaSuccess) return e;
             int per_sm = 0, sms = 0;
-            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ssd_tc_kernel<N>, K::THREADS, K::SMEM);
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ssd_tc_kernel<N, false>, K::THREADS, K::SMEM);
             if (e != cudaSuccess) return e;
             e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
             if (e != cudaSuccess) return e;
@@ -1012,7 +1015,10 @@ static cudaError_t launch_n(const PrefillArgs& a, cudaStream_t s) {
     if (items > 0x7fffffffLL) return cudaErrorInvalidValue;
     const long long want = (items + K::PIPES - 1) / K::PIPES;   // each CTA runs PIPES ticket streams
     const unsigned grid = (unsigned)(want < resident[dev] ? want : resident[dev]);
-    ssd_tc_kernel<N><<<grid, K::THREADS, K::SMEM, s>>>(mx, mb, mc, my, p);
+    // whole sequences (one run each) take the instantiation without state items
+    // or hand-off waits: the code of the block loop is then that alone
+    if (p.nruns > 1) ssd_tc_kernel<N, true><<<grid, K::THREADS, K::SMEM, s>>>(mx, mb, mc, my, p);
+    else ssd_tc_kernel<N, false><<<grid, K::THREADS, K::SMEM, s>>>(mx, mb, mc, my, p);
     return cudaGetLastError();
 }
 
