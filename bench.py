@@ -39,8 +39,8 @@ METRIC = "SSD prefill tokens/s + TFLOP/s; decode tokens/s + state GB/s (1 B200)"
 # of the SHA-256 of the kernel's source file at capture time: a changed kernel
 # reports null until it is captured again (summaries under profiles/).
 NCU_TRAFFIC = {
-    "ssd_prefill_tc.cu": ("ef07cdd0586c7e9a", 75557632 + 88305920),
-    "ssd_decode.cu": ("85bad38e2a990c89", 1079074000 + 1023788000),
+    "ssd_prefill_tc.cu": ("7e67b905026fb3cb", 75557632 + 88568320),
+    "ssd_decode.cu": ("cba348ad46ab41a0", 1079097000 + 1024990000),
 }
 
 
