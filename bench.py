@@ -7,7 +7,9 @@ One step = one ssd_chunk_scan_fwd over the Mamba-2 1.3B-shaped layer (batch 4,
 seqlen 2048, 64 heads x P=64, N=128, 1 group, chunk 256; bf16 inputs, fp32
 accumulation, y and final_state in fp32) on synthetic seeded inputs resident in
 HBM.  The same run also times K decode steps (ssd_state_update, batch 256, 128
-heads, P=64, N=128, 8 groups, fp32 state) and reports them under "decode".
+heads, P=64, N=128, 8 groups, fp32 state) and reports them under "decode",
+with the same steps replayed from a checkpoint and a 16-token buffer
+(ssd_replay_step) under "decode"."replay".
 
 Timing: W untimed warm-up steps, then exactly K steps between a barrier +
 cudaDeviceSynchronize on both sides, CUDA events on the launching stream, max
@@ -426,6 +428,50 @@ def main():
                                 "algorithmic_bytes_per_launch": dbytes, "kernel": "state_update_kernel"},
                    "clocks": dclk.summary()}
 
+    # ---------------- replayed decode of the same steps: checkpoint + a buffer of
+    # RK tokens, the checkpoint written back once per RK steps
+    RK = 16
+    rdesc = ssd.ReplayDesc(dcfg.batch, dcfg.nheads, dcfg.headdim, dcfg.dstate, dcfg.ngroups, ssd.SSD_BF16,
+                           ssd.SSD_F32, ssd.SSD_F32, RK)
+    rbuf = torch.empty(max(ssd.ssd_replay_buffer_size(rdesc), 1), dtype=torch.uint8, device=dev)
+    rfill = [0]
+
+    def replay(t):
+        d = dsteps[t % nsteps_in]
+        st = ssd.ssd_replay_step(rdesc, state.data_ptr(), rbuf.data_ptr(), rfill[0], d["x"].data_ptr(),
+                                 d["dt_raw"].data_ptr(), prm["dt_bias"].data_ptr(), prm["A"].data_ptr(),
+                                 d["B"].data_ptr(), d["C"].data_ptr(), prm["D"].data_ptr(), yd.data_ptr(),
+                                 stream.cuda_stream)
+        if st:
+            raise ssd.SsdError(st, "ssd_replay_step")
+        rfill[0] = (rfill[0] + 1) % RK
+
+    rsteps = RK * max(1, args.steps // RK)      # whole buffer cycles: every RK-th step folds
+    for t in range(RK):
+        replay(t)
+    dist.barrier(pg)
+    torch.cuda.synchronize()
+    ev[0].record(stream)
+    for t in range(rsteps):
+        replay(t)
+    ev[1].record(stream)
+    torch.cuda.synchronize()
+    dist.barrier(pg)
+    rms = dist.max_over_ranks(pg, ev[0].elapsed_time(ev[1]) / rsteps)
+    sbytes = dcfg.batch * dcfg.nheads * dcfg.dstate * dcfg.headdim * 4
+    # per step: the checkpoint read, its write once per RK steps, the step's io,
+    # and the buffered x_s (per head) and B_s (per group) read back, (RK-1)/2 on average
+    io_bytes = decode_bytes(dcfg.batch, dcfg.nheads, dcfg.headdim, dcfg.dstate, dcfg.ngroups, 2, 4, 4) - 2 * sbytes
+    buf_bytes = (RK - 1) / 2 * (dcfg.batch * dcfg.nheads * dcfg.headdim * 2
+                                + dcfg.batch * dcfg.nheads * dcfg.dstate * 2)
+    rbytes = sbytes * (1 + 1 / RK) + io_bytes + buf_bytes + dcfg.batch * dcfg.nheads * dcfg.headdim * 2
+    rgbs = rbytes / (rms * 1e-3) / 1e9
+    decode_line["replay"] = {"capacity": RK, "tokens_per_s": dcfg.batch * world / (rms * 1e-3), "ms_per_step": rms,
+                             "speedup_vs_state_update": dms / rms,
+                             "roofline": {"bound": "hbm", "achieved": rgbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                          "frac": rgbs / peaks["hbm_gbs"], "algorithmic_bytes_per_step": rbytes,
+                                          "kernel": "replay_step_kernel"}}
+
     # ---------------- end to end through the public API with host buffers
     e2e = None
     if rank == 0 or world > 1:
@@ -495,7 +541,7 @@ def main():
                            "kernel_path": "tensor cores" if path == 0 else "cuda cores"},
                 "tflops": tflops, "gbs": gbs, "roofline": roofline, "decode": decode_line,
                 "cpu_baseline": cpu_baseline, "e2e": e2e, "workloads": workloads,
-                "gpu_launches": launches_per_prefill * args.steps + args.steps,
+                "gpu_launches": launches_per_prefill * args.steps + args.steps + rsteps,
                 "clocks": clk.summary()}
         print(json.dumps(line), flush=True)
     dist.finish(pg)

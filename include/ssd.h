@@ -102,6 +102,20 @@ typedef struct {
     int32_t state_dtype;/* dtype of the in-place state */
 } ssd_decode_desc_t;
 
+/* Replayed decode (checkpoint + buffer of recent tokens) problem description. */
+typedef struct {
+    int64_t batch;      /* >= 0; 0 is a no-op */
+    int64_t nheads;
+    int64_t headdim;    /* P: 8, 16, 32, 64 or 128 */
+    int64_t dstate;     /* N, multiple of 8, <= 256 */
+    int64_t ngroups;
+    int32_t io_dtype;   /* dtype of x, dt_raw, B, C (and of their buffered copies) */
+    int32_t y_dtype;    /* dtype of y */
+    int32_t state_dtype;/* dtype of the checkpoint */
+    int32_t capacity;   /* K, 1..16: tokens after the checkpoint the buffer holds; the
+                           step that brings it to K folds them into the checkpoint */
+} ssd_replay_desc_t;
+
 /* Library version as MAJOR * 10000 + MINOR * 100 + PATCH. */
 int ssd_version(void);
 
@@ -215,6 +229,50 @@ ssd_status_t ssd_state_update(const ssd_decode_desc_t* desc, void* state, const 
                               void* stream);
 
 /*
+ * Bytes of the replay buffer ssd_replay_step needs for `desc` (written to
+ * *bytes).  Pure host function.  Errors: SSD_ERR_INVALID_ARG /
+ * SSD_ERR_UNSUPPORTED as for ssd_replay_step.
+ */
+ssd_status_t ssd_replay_buffer_size(const ssd_replay_desc_t* desc, size_t* bytes);
+
+/*
+ * One decode step on a state held as a checkpoint plus a buffer of the tokens
+ * after it ("Mamba3" (Telegram post) and "Mamba-3 : SSM optimise inference",
+ * ReplaySSM: outputs are computed from the checkpoint and the buffered inputs
+ * on most steps; the state is written back only when the buffer fills).
+ *
+ * Before the call the state of sequence (b, h) is the checkpoint advanced by
+ * the `fill` buffered tokens; the call takes token t and returns
+ *   y_t = C_t^T h_t + D x_t,   h_t = exp(dt_t A) h_{t-1} + dt_t B_t x_t^T
+ * (the decode step of ssd_state_update, up to rounding).  If fill + 1 <
+ * capacity, token t is appended to the buffer and the checkpoint is only read
+ * (the caller's next fill is fill + 1); if fill + 1 == capacity, all buffered
+ * tokens and t are folded into the checkpoint, which then holds h_t (the
+ * caller's next fill is 0).  A bf16 checkpoint is rounded (to nearest even) at
+ * those folds only.  Averaged over capacity steps, the state is read once per
+ * step and written once per capacity steps.
+ *
+ *  checkpoint [b][H][N][P]  state_dtype  required; read every step, written
+ *                                        on the folding step
+ *  buffer     ssd_replay_buffer_size bytes, 256-byte aligned, caller-owned;
+ *             its layout is the library's; its contents are irrelevant when
+ *             fill == 0 and must be left as the previous call left them otherwise
+ *  fill       0 <= fill < capacity: tokens currently buffered (host value);
+ *             start a sequence with the initial state in the checkpoint and fill 0
+ *  x [b][H][P], dt_raw [b][H], B, C [b][G][N]: io_dtype, required
+ *  dt_bias, A, D [H] fp32 (dt_bias, D nullable); y [b][H][P] y_dtype, required
+ * Calls on one buffer must be ordered on one stream (each step reads what the
+ * previous one appended).
+ * Errors: SSD_ERR_INVALID_ARG (bad descriptor, fill out of range, NULL
+ * pointers, y/x/checkpoint/buffer overlapping), SSD_ERR_UNSUPPORTED
+ * (headdim not 8/16/32/64/128, dstate, capacity > 16), SSD_ERR_ALIGNMENT,
+ * SSD_ERR_CUDA; nothing is launched on a host-side error.
+ */
+ssd_status_t ssd_replay_step(const ssd_replay_desc_t* desc, void* checkpoint, void* buffer, int32_t fill,
+                             const void* x, const void* dt_raw, const float* dt_bias, const float* A,
+                             const void* B, const void* C, const float* D, void* y, void* stream);
+
+/*
  * Synchronises `stream`, then reports (and clears) the device-side error word
  * of the current device.  Kernels never trap: a bounded wait that gives up
  * (the inter-chunk state hand-off of the prefill waits for the previous
@@ -233,14 +291,15 @@ ssd_status_t ssd_get_device_error(void* stream, uint32_t* detail);
  * Test hook for the device-side failure path; never needed in normal use.
  * Sets the faults injected into every following launch until called again
  * with 0 (process-wide, all devices).
- *  SSD_FAULT_DROP_RUN_PUBLISH: on the tensor-core prefill path, a run of
- *    chunks that hands its state to the next run of the same sequence never
- *    signals it.  The next run's bounded wait (2 s) then expires: the launch
- *    still completes (its outputs are undefined), and ssd_get_device_error
- *    reports SSD_ERR_DEVICE_TIMEOUT with bit 0x1 (a hand-off wait timed out)
- *    and possibly 0x2 (other waits cut short) in *detail.  Nothing traps and
- *    the CUDA context stays usable.  Runs are used only when a prefill has
- *    fewer (batch x head) sequences than SMs.
+ *  SSD_FAULT_DROP_RUN_PUBLISH: on the tensor-core prefill path, the state
+ *    item that computes the entry state of a run of chunks never signals it.
+ *    The bounded waits (2 s) of the items that need it then expire: the
+ *    launch still completes (its outputs are undefined), and
+ *    ssd_get_device_error reports SSD_ERR_DEVICE_TIMEOUT with bit 0x1 (a
+ *    hand-off wait timed out) and possibly 0x2 (other waits cut short) in
+ *    *detail.  Nothing traps and the CUDA context stays usable.  Sequences
+ *    are cut into runs only when a prefill has fewer (batch x head) sequences
+ *    than half the block pipelines (148 on a 148-SM part, 74 at dstate 256).
  * Errors: SSD_ERR_INVALID_ARG for unknown bits (nothing changed).
  */
 ssd_status_t ssd_debug_inject(uint32_t faults);

@@ -95,6 +95,35 @@ static int prefill_path(const ssd_prefill_desc_t* d) {
     return tc_path_supports(d->headdim, d->dstate, d->chunk, d->io_dtype == SSD_BF16) ? 0 : 1;
 }
 
+// replay descriptor checks shared by ssd_replay_buffer_size and ssd_replay_step
+static ssd_status_t check_replay_desc(const ssd_replay_desc_t* d) {
+    if (!d) return SSD_ERR_INVALID_ARG;
+    if (d->batch < 0 || d->nheads < 1 || d->headdim < 1 || d->dstate < 1 || d->ngroups < 1 ||
+        d->nheads % d->ngroups != 0 || d->capacity < 1)
+        return SSD_ERR_INVALID_ARG;
+    if (!valid_dtype(d->io_dtype) || !valid_dtype(d->y_dtype) || !valid_dtype(d->state_dtype))
+        return SSD_ERR_INVALID_ARG;
+    // a lane owns 4 columns of a state row and the lanes of a warp cover whole rows
+    const int64_t P = d->headdim;
+    if (!(P == 8 || P == 16 || P == 32 || P == 64 || P == 128)) return SSD_ERR_UNSUPPORTED;
+    if (d->dstate % 8 != 0 || d->dstate > 256 || d->capacity > 16) return SSD_ERR_UNSUPPORTED;
+    if (d->batch * d->nheads > (int64_t)0x7fffffff) return SSD_ERR_UNSUPPORTED;
+    return SSD_OK;
+}
+
+static ReplayLayout replay_layout(const ssd_replay_desc_t* d) {
+    ReplayLayout l{};
+    const size_t K = (size_t)d->capacity, e = dsize(d->io_dtype);
+    const size_t bh = (size_t)d->batch * d->nheads, bg = (size_t)d->batch * d->ngroups;
+    l.off_x = 0;
+    l.off_B = align256(l.off_x + bh * K * d->headdim * e);
+    l.off_dt = align256(l.off_B + bg * K * d->dstate * e);
+    l.off_cum = align256(l.off_dt + bh * K * sizeof(float));
+    l.off_cb = align256(l.off_cum + bh * K * sizeof(float));
+    l.total = align256(l.off_cb + bg * 16 * sizeof(float));
+    return l;
+}
+
 // copies (or zero-fills) init_state into final_state for seqlen == 0
 template <typename S, typename D>
 __global__ void copy_state_kernel(const S* __restrict__ src, D* __restrict__ dst, int64_t n) {
@@ -223,6 +252,51 @@ ssd_status_t ssd_state_update(const ssd_decode_desc_t* d, void* state, const voi
     a.state = state; a.x = x; a.dt_raw = dt_raw; a.B = B; a.C = C;
     a.dt_bias = dt_bias; a.A = A; a.D = D; a.y = y;
     const cudaError_t e = launch_state_update(a, (cudaStream_t)stream);
+    return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
+}
+
+ssd_status_t ssd_replay_buffer_size(const ssd_replay_desc_t* desc, size_t* bytes) {
+    if (!bytes) return SSD_ERR_INVALID_ARG;
+    const ssd_status_t st = check_replay_desc(desc);
+    if (st != SSD_OK) return st;
+    *bytes = replay_layout(desc).total;
+    return SSD_OK;
+}
+
+ssd_status_t ssd_replay_step(const ssd_replay_desc_t* d, void* checkpoint, void* buffer, int32_t fill,
+                             const void* x, const void* dt_raw, const float* dt_bias, const float* A,
+                             const void* B, const void* C, const float* D, void* y, void* stream) {
+    ssd_status_t st = check_replay_desc(d);
+    if (st != SSD_OK) return st;
+    if (fill < 0 || fill >= d->capacity) return SSD_ERR_INVALID_ARG;
+    if (!checkpoint || !buffer || !x || !dt_raw || !A || !B || !C || !y) return SSD_ERR_INVALID_ARG;
+    const void* ptrs[] = {checkpoint, x, dt_raw, dt_bias, A, B, C, D, y};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return SSD_ERR_ALIGNMENT;
+    if ((uintptr_t)buffer & 255u) return SSD_ERR_ALIGNMENT;
+    const ReplayLayout lay = replay_layout(d);
+    const size_t bh = (size_t)d->batch * d->nheads;
+    const size_t s_bytes = bh * d->dstate * d->headdim * dsize(d->state_dtype);
+    const size_t y_bytes = bh * d->headdim * dsize(d->y_dtype);
+    const size_t x_bytes = bh * d->headdim * dsize(d->io_dtype);
+    if (overlaps(y, y_bytes, checkpoint, s_bytes) || overlaps(y, y_bytes, x, x_bytes) ||
+        overlaps(checkpoint, s_bytes, x, x_bytes) || overlaps(buffer, lay.total, checkpoint, s_bytes) ||
+        overlaps(buffer, lay.total, y, y_bytes) || overlaps(buffer, lay.total, x, x_bytes))
+        return SSD_ERR_INVALID_ARG;
+    if (d->batch == 0) return SSD_OK;
+    ReplayArgs a{};
+    a.batch = d->batch; a.H = d->nheads; a.P = d->headdim; a.N = d->dstate; a.G = d->ngroups;
+    a.K = d->capacity; a.fill = fill;
+    a.io_bf16 = d->io_dtype == SSD_BF16; a.y_bf16 = d->y_dtype == SSD_BF16;
+    a.state_bf16 = d->state_dtype == SSD_BF16;
+    a.ckpt = checkpoint;
+    a.xb = (char*)buffer + lay.off_x;
+    a.Bb = (char*)buffer + lay.off_B;
+    a.dtb = (float*)((char*)buffer + lay.off_dt);
+    a.cumb = (float*)((char*)buffer + lay.off_cum);
+    a.cb = (float*)((char*)buffer + lay.off_cb);
+    a.x = x; a.dt_raw = dt_raw; a.B = B; a.C = C; a.dt_bias = dt_bias; a.A = A; a.D = D; a.y = y;
+    const cudaError_t e = launch_replay_step(a, (cudaStream_t)stream);
     return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
 }
 

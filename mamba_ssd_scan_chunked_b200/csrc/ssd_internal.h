@@ -19,6 +19,26 @@ struct DecodeArgs {
 
 cudaError_t launch_state_update(const DecodeArgs& a, cudaStream_t stream);
 
+// Replayed decode step: checkpoint + buffer of the last tokens (ssd_replay.cu).
+struct ReplayArgs {
+    int64_t batch, H, P, N, G, K, fill;
+    bool io_bf16, y_bf16, state_bf16;
+    void* ckpt;
+    void *xb, *Bb;                 // buffered x [b][H][K][P], B [b][G][K][N] (io dtype)
+    float *dtb, *cumb;             // buffered dt, log-decay cumsum [b][H][K]
+    float* cb;                     // the step's C_t . B_s [b][G][16]
+    const void *x, *dt_raw, *B, *C;
+    const float *dt_bias, *A, *D;
+    void* y;
+};
+
+// Byte offsets of the replay buffer's parts (all 256-byte aligned) and its size.
+struct ReplayLayout {
+    size_t off_x, off_B, off_dt, off_cum, off_cb, total;
+};
+
+cudaError_t launch_replay_step(const ReplayArgs& a, cudaStream_t stream);
+
 // Workspace carve-up of the prefill (all offsets 256-byte aligned).
 struct PrefillLayout {
     int64_t nchunks;       // ceil(L / Q)

@@ -26,8 +26,8 @@ STATUS = {0: "SSD_OK", 1: "SSD_ERR_INVALID_ARG", 2: "SSD_ERR_UNSUPPORTED", 3: "S
 
 # every symbol include/ssd.h declares
 EXPORTS = ("ssd_version", "ssd_status_string", "ssd_chunk_scan_workspace_size", "ssd_chunk_scan_path",
-           "ssd_chunk_scan_fwd", "ssd_chunk_scan_fwd_noalloc", "ssd_state_update", "ssd_get_device_error",
-           "ssd_debug_inject")
+           "ssd_chunk_scan_fwd", "ssd_chunk_scan_fwd_noalloc", "ssd_state_update", "ssd_replay_buffer_size",
+           "ssd_replay_step", "ssd_get_device_error", "ssd_debug_inject")
 
 # fault-injection bits of ssd_debug_inject
 SSD_FAULT_DROP_RUN_PUBLISH = 0x1
@@ -53,6 +53,12 @@ class DecodeDesc(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int64), ("nheads", ctypes.c_int64), ("headdim", ctypes.c_int64),
                 ("dstate", ctypes.c_int64), ("ngroups", ctypes.c_int64), ("io_dtype", ctypes.c_int32),
                 ("y_dtype", ctypes.c_int32), ("state_dtype", ctypes.c_int32)]
+
+
+class ReplayDesc(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int64), ("nheads", ctypes.c_int64), ("headdim", ctypes.c_int64),
+                ("dstate", ctypes.c_int64), ("ngroups", ctypes.c_int64), ("io_dtype", ctypes.c_int32),
+                ("y_dtype", ctypes.c_int32), ("state_dtype", ctypes.c_int32), ("capacity", ctypes.c_int32)]
 
 
 _lock = threading.Lock()
@@ -83,6 +89,10 @@ def lib():
             L.ssd_chunk_scan_fwd_noalloc.argtypes = [ctypes.POINTER(PrefillDesc)] + [_VP] * 11
             L.ssd_state_update.restype = ctypes.c_int
             L.ssd_state_update.argtypes = [ctypes.POINTER(DecodeDesc)] + [_VP] * 10
+            L.ssd_replay_buffer_size.restype = ctypes.c_int
+            L.ssd_replay_buffer_size.argtypes = [ctypes.POINTER(ReplayDesc), ctypes.POINTER(ctypes.c_size_t)]
+            L.ssd_replay_step.restype = ctypes.c_int
+            L.ssd_replay_step.argtypes = [ctypes.POINTER(ReplayDesc), _VP, _VP, ctypes.c_int32] + [_VP] * 9
             L.ssd_get_device_error.restype = ctypes.c_int
             L.ssd_get_device_error.argtypes = [_VP, ctypes.POINTER(ctypes.c_uint32)]
             L.ssd_debug_inject.restype = ctypes.c_int
@@ -137,6 +147,21 @@ def ssd_state_update(desc, state, x, dt_raw, dt_bias, A, B, C, D, y, stream) -> 
     """Raw call; returns the status code (0 = enqueued)."""
     return lib().ssd_state_update(ctypes.byref(desc), state or None, x or None, dt_raw or None, dt_bias or None,
                                   A or None, B or None, C or None, D or None, y or None, stream or None)
+
+
+def ssd_replay_buffer_size(desc: ReplayDesc) -> int:
+    n = ctypes.c_size_t(0)
+    st = lib().ssd_replay_buffer_size(ctypes.byref(desc), ctypes.byref(n))
+    if st:
+        raise SsdError(st, "ssd_replay_buffer_size")
+    return n.value
+
+
+def ssd_replay_step(desc, checkpoint, buffer, fill, x, dt_raw, dt_bias, A, B, C, D, y, stream) -> int:
+    """Raw call; returns the status code (0 = enqueued)."""
+    return lib().ssd_replay_step(ctypes.byref(desc), checkpoint or None, buffer or None, int(fill), x or None,
+                                 dt_raw or None, dt_bias or None, A or None, B or None, C or None, D or None,
+                                 y or None, stream or None)
 
 
 def ssd_get_device_error(stream=None):
@@ -242,3 +267,37 @@ def state_update(state, x, dt_raw, dt_bias, A, B, C, D, *, y=None, y_dtype=None,
     if st:
         raise SsdError(st, "ssd_state_update")
     return y
+
+
+def replay_desc(checkpoint, x, B, capacity, y_dtype=None) -> ReplayDesc:
+    b, H, P = x.shape
+    G, N = B.shape[1], B.shape[2]
+    io = _dtype_code(x.dtype)
+    return ReplayDesc(b, H, P, N, G, io, _dtype_code(y_dtype) if y_dtype is not None else io,
+                      _dtype_code(checkpoint.dtype), int(capacity))
+
+
+def replay_buffer(checkpoint, x, B, capacity):
+    """A device buffer of the size ssd_replay_step needs (uint8, 256-byte aligned by the allocator)."""
+    import torch
+    n = ssd_replay_buffer_size(replay_desc(checkpoint, x, B, capacity))
+    return torch.empty(max(n, 1), dtype=torch.uint8, device=x.device)
+
+
+def replay_step(checkpoint, buffer, fill, capacity, x, dt_raw, dt_bias, A, B, C, D, *, y=None, y_dtype=None,
+                stream=None):
+    """Replayed decode step: checkpoint [b,H,N,P] + buffer (``replay_buffer``) holding ``fill``
+    tokens; x [b,H,P], dt_raw [b,H], B/C [b,G,N].  Returns (y, next fill)."""
+    import torch
+    desc = replay_desc(checkpoint, x, B, capacity, y_dtype)
+    for t in (checkpoint, buffer, x, dt_raw, B, C, dt_bias, A, D, y):
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("libssd takes contiguous CUDA tensors")
+    b, H, P = x.shape
+    if y is None:
+        y = torch.empty((b, H, P), dtype=_torch_dtype(desc.y_dtype), device=x.device)
+    st = ssd_replay_step(desc, _ptr(checkpoint), _ptr(buffer), fill, _ptr(x), _ptr(dt_raw), _ptr(dt_bias), _ptr(A),
+                         _ptr(B), _ptr(C), _ptr(D), _ptr(y), _stream(stream))
+    if st:
+        raise SsdError(st, "ssd_replay_step")
+    return y, (fill + 1) % int(capacity)

@@ -140,3 +140,47 @@ def test_decode_host_validation_codes():
     assert call(dd(), x=FAKE + 0x1000004) == ALIGN
     assert call(dd(), y=FAKE) == INVALID                   # y overlaps the state
     assert call(dd(batch=0)) == OK
+
+
+def replay_d(**kw):
+    d = dict(batch=8, nheads=4, headdim=64, dstate=128, ngroups=2, io_dtype=ssd.SSD_BF16,
+             y_dtype=ssd.SSD_F32, state_dtype=ssd.SSD_F32, capacity=16)
+    d.update(kw)
+    return ssd.ReplayDesc(**d)
+
+
+def test_replay_buffer_size():
+    # x [b][H][K][P] + B [b][G][K][N] (io dtype) + dt, cumsum [b][H][K] fp32 + the step's
+    # C.B_s [b][G][16] fp32, each part 256-byte aligned
+    b, H, P, N, G, K = 8, 4, 64, 128, 2, 16
+    assert ssd.ssd_replay_buffer_size(replay_d()) == \
+        b * H * K * P * 2 + b * G * K * N * 2 + 2 * b * H * K * 4 + 256 * ((b * G * 16 * 4 + 255) // 256)
+    assert ssd.ssd_replay_buffer_size(replay_d(io_dtype=ssd.SSD_F32)) == \
+        b * H * K * P * 4 + b * G * K * N * 4 + 2 * b * H * K * 4 + 256 * ((b * G * 16 * 4 + 255) // 256)
+    assert ssd.ssd_replay_buffer_size(replay_d(batch=0)) == 0
+    for kw, code in [(dict(capacity=0), INVALID), (dict(capacity=17), UNSUPPORTED), (dict(headdim=96), UNSUPPORTED),
+                     (dict(headdim=256), UNSUPPORTED), (dict(dstate=12), UNSUPPORTED), (dict(ngroups=3), INVALID),
+                     (dict(y_dtype=4), INVALID)]:
+        with pytest.raises(ssd.SsdError) as e:
+            ssd.ssd_replay_buffer_size(replay_d(**kw))
+        assert e.value.status == code, kw
+
+
+def test_replay_host_validation_codes():
+    def call(d, fill=0, **ptrs):
+        p = dict(ckpt=FAKE, buf=FAKE + 0x8000000, x=FAKE + 0x1000000, dt_raw=FAKE + 0x2000000, dt_bias=0,
+                 A=FAKE + 0x3000000, B=FAKE + 0x4000000, C=FAKE + 0x5000000, D=0, y=FAKE + 0x6000000, stream=0)
+        p.update(ptrs)
+        return ssd.ssd_replay_step(d, p["ckpt"], p["buf"], fill, p["x"], p["dt_raw"], p["dt_bias"], p["A"], p["B"],
+                                   p["C"], p["D"], p["y"], p["stream"])
+
+    assert call(replay_d(), fill=16) == INVALID            # fill must be below the capacity
+    assert call(replay_d(), fill=-1) == INVALID
+    assert call(replay_d(), buf=0) == INVALID
+    assert call(replay_d(), ckpt=0) == INVALID
+    assert call(replay_d(), buf=FAKE + 0x8000010) == ALIGN   # the buffer wants 256-byte alignment
+    assert call(replay_d(), x=FAKE + 0x1000008) == ALIGN
+    assert call(replay_d(), y=FAKE) == INVALID              # y overlaps the checkpoint
+    assert call(replay_d(), buf=FAKE + 0x100) == INVALID    # the buffer overlaps the checkpoint
+    assert call(replay_d(headdim=48)) == UNSUPPORTED
+    assert call(replay_d(batch=0)) == OK                   # nothing to do, nothing launched
