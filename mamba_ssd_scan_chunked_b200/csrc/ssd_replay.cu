@@ -21,8 +21,11 @@
 //
 // Mapping: one warp per (batch, head), as the decode kernel.  A lane owns a
 // 4-element column vector of the state (16 bytes fp32, 8 bytes bf16) so that
-// the flush can keep x_s of all K buffered tokens for its columns in
-// registers.
+// the fold can keep x_s of all K buffered tokens for its columns in registers
+// (paired fp32 FMAs: two columns per instruction).  The dot products C_t . B_s
+// of an ordinary step are per (batch, group) and come from a small kernel run
+// before it.  The fold's coefficients beta_s B_s[n] are staged per warp in
+// shared memory, rows of 17 floats (conflict-free writes and reads).
 #include "ssd_common.cuh"
 #include "ssd_internal.h"
 
@@ -116,29 +119,23 @@ replay_dots_kernel(const IoT* __restrict__ Bb, const IoT* __restrict__ Bm, const
     }
 }
 
-// x_s of the 16 token slots for a lane's 4 columns, held through the fold:
-// packed bf16 pairs (32 registers) for bf16 inputs, fp32 (64) otherwise.
-template <typename IoT> struct XSlots;
-template <> struct XSlots<float> {
-    float v[16][RP_VEC];
-    __device__ __forceinline__ void set(int s, const float* x) {
-#pragma unroll
-        for (int j = 0; j < RP_VEC; ++j) v[s][j] = x[j];
-    }
-    __device__ __forceinline__ float get(int s, int j) const { return v[s][j]; }
-};
-template <> struct XSlots<bf16> {
-    uint32_t v[16][RP_VEC / 2];
-    // x is exactly representable: it holds bf16 inputs widened to fp32 (or 0)
-    __device__ __forceinline__ void set(int s, const float* x) {
-#pragma unroll
-        for (int j = 0; j < RP_VEC / 2; ++j)
-            v[s][j] = (__float_as_uint(x[2 * j]) >> 16) | (__float_as_uint(x[2 * j + 1]) & 0xffff0000u);
-    }
-    __device__ __forceinline__ float get(int s, int j) const {
-        return (j & 1) ? __uint_as_float(v[s][j >> 1] & 0xffff0000u) : __uint_as_float(v[s][j >> 1] << 16);
-    }
-};
+// Packed fp32 pairs (low half = first element) and the sm_100 paired FMA:
+// one instruction updates two columns of a state row.
+__device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
+    return (uint64_t)__float_as_uint(lo) | ((uint64_t)__float_as_uint(hi) << 32);
+}
+__device__ __forceinline__ float f2lo(uint64_t v) { return __uint_as_float((uint32_t)v); }
+__device__ __forceinline__ float f2hi(uint64_t v) { return __uint_as_float((uint32_t)(v >> 32)); }
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
 
 // FLUSH: this step fills the buffer (fill == K - 1) and is folded into the
 // checkpoint.  Buffers: xb [b][H][K][P], Bb [b][G][K][N] (io dtype), dtb and
@@ -168,7 +165,7 @@ replay_step_kernel(StateT* __restrict__ ckpt, IoT* __restrict__ xb, IoT* __restr
     const int p0 = vc * RP_VEC;
     StateT* base = ckpt + (size_t)bh * N * P + p0;
     // state vectors in flight per lane (the fold holds x_s of 16 tokens as well)
-    constexpr int U = FLUSH ? (sizeof(IoT) == 2 ? 8 : 4) : RP_U;
+    constexpr int U = FLUSH ? 4 : RP_U;
 
     const float dt = softplus_f32(to_f32(dt_raw[bh]) + (dt_bias ? dt_bias[h] : 0.f));
     const float cum_t = (fill > 0 ? cumb[(size_t)bh * K + fill - 1] : 0.f) + dt * A[h];
@@ -220,7 +217,7 @@ replay_step_kernel(StateT* __restrict__ ckpt, IoT* __restrict__ xb, IoT* __restr
         }
     } else {
         // x_s of the K buffered tokens for this lane's columns (s == fill: x_t)
-        XSlots<IoT> xs;
+        uint64_t xs[16][2];                    // x_s[cols] as fp32 pairs
 #pragma unroll
         for (int s = 0; s < 16; ++s) {
             float xv[RP_VEC];
@@ -229,8 +226,10 @@ replay_step_kernel(StateT* __restrict__ ckpt, IoT* __restrict__ xb, IoT* __restr
 #pragma unroll
                 for (int j = 0; j < RP_VEC; ++j) xv[j] = s == fill ? xt[j] : 0.f;
             }
-            xs.set(s, xv);
+            xs[s][0] = f2pack(xv[0], xv[1]);
+            xs[s][1] = f2pack(xv[2], xv[3]);
         }
+        const uint64_t al2 = f2pack(alpha, alpha);
         // h <- alpha h + sum_s g[n][s] x_s[cols]; acc = sum_n C[n] h_new[n][cols]
         for (int r0 = r_off; r0 < N; r0 += U * rstep) {
             float hv[U][RP_VEC];
@@ -243,18 +242,18 @@ replay_step_kernel(StateT* __restrict__ ckpt, IoT* __restrict__ xb, IoT* __restr
             for (int u = 0; u < U; ++u) {
                 const int r = r0 + u * rstep;
                 if (r < N) {
-                    float v[RP_VEC];
-#pragma unroll
-                    for (int j = 0; j < RP_VEC; ++j) v[j] = alpha * hv[u][j];
+                    uint64_t v2[2] = {fmul2(al2, f2pack(hv[u][0], hv[u][1])), fmul2(al2, f2pack(hv[u][2], hv[u][3]))};
                     const float* gr = gs + r * 17;
 #pragma unroll
                     for (int t = 0; t < 16; ++t) {
                         if (t < K) {
                             const float gv = gr[t];
-#pragma unroll
-                            for (int j = 0; j < RP_VEC; ++j) v[j] = fmaf(gv, xs.get(t, j), v[j]);
+                            const uint64_t g2 = f2pack(gv, gv);
+                            v2[0] = ffma2(g2, xs[t][0], v2[0]);
+                            v2[1] = ffma2(g2, xs[t][1], v2[1]);
                         }
                     }
+                    const float v[RP_VEC] = {f2lo(v2[0]), f2hi(v2[0]), f2lo(v2[1]), f2hi(v2[1])};
                     Vec4<StateT>::store(base + (size_t)r * P, v);   // bf16: rounded to nearest even
                     const float c = cs[r];
 #pragma unroll
