@@ -44,6 +44,9 @@ dt_cumsum_kernel(const IoT* __restrict__ dt_raw, const float* __restrict__ dt_bi
     const int c = (int)((blockIdx.x / (unsigned)hgroups) % (unsigned)nchunks);
     const int b = (int)(blockIdx.x / ((unsigned)hgroups * (unsigned)nchunks));
     const int h0 = hg * DT_HG;
+    // the tensor-core kernel launched after this one may start now: it waits for
+    // this grid to complete before it reads anything written here
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int l = threadIdx.x;                 // token within the chunk (blockDim = max(Q, 32))
     const int lane = l & 31, warp = l >> 5;
     const int64_t t = (int64_t)c * Q + l;

@@ -471,6 +471,10 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                     tma_prefetch_4d(&tmX, 0, h_, t0_ + SUB, b_);
                 }
             };
+            // this launch may start while the decay-cumsum kernel before it is still
+            // running (programmatic dependent launch): wait for it to finish -- its
+            // dt, cumsum and reset flags -- before the first ticket
+            asm volatile("griddepcontrol.wait;" ::: "memory");
             int item = 0;
             if (lead) item = atomicAdd(p.flags + p.BH + CTRL_TICKET, 1);
             item = __shfl_sync(0xffffffffu, item, __ffs(__ballot_sync(0xffffffffu, lead)) - 1);
@@ -1016,10 +1020,22 @@ static cudaError_t launch_n(const PrefillArgs& a, cudaStream_t s) {
     const long long want = (items + K::PIPES - 1) / K::PIPES;   // each CTA runs PIPES ticket streams
     const unsigned grid = (unsigned)(want < resident[dev] ? want : resident[dev]);
     // whole sequences (one run each) take the instantiation without state items
-    // or hand-off waits: the code of the block loop is then that alone
-    if (p.nruns > 1) ssd_tc_kernel<N, true><<<grid, K::THREADS, K::SMEM, s>>>(mx, mb, mc, my, p);
-    else ssd_tc_kernel<N, false><<<grid, K::THREADS, K::SMEM, s>>>(mx, mb, mc, my, p);
-    return cudaGetLastError();
+    // or hand-off waits: the code of the block loop is then that alone.  The
+    // launch is a programmatic dependent of the decay-cumsum kernel before it on
+    // the stream: its prologue overlaps that kernel, and its control warps wait
+    // for it (griddepcontrol.wait) before reading what it wrote.
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(K::THREADS);
+    cfg.dynamicSmemBytes = K::SMEM;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (p.nruns > 1) return cudaLaunchKernelEx(&cfg, ssd_tc_kernel<N, true>, mx, mb, mc, my, p);
+    return cudaLaunchKernelEx(&cfg, ssd_tc_kernel<N, false>, mx, mb, mc, my, p);
 }
 
 }  // namespace tc
