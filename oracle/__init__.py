@@ -72,6 +72,8 @@ def _load():
             lib.oracle_ssd_chunked.restype = ctypes.c_int
             lib.oracle_ssd_decode_step.argtypes = [_I64] * 5 + [_D] * 9 + [ctypes.c_int, ctypes.c_int]
             lib.oracle_ssd_decode_step.restype = ctypes.c_int
+            lib.oracle_ssd_decode_step_mimo.argtypes = [_I64] * 6 + [_D] * 9 + [ctypes.c_int, ctypes.c_int]
+            lib.oracle_ssd_decode_step_mimo.restype = ctypes.c_int
             lib.oracle_round_bf16.argtypes = [ctypes.c_double]
             lib.oracle_round_bf16.restype = ctypes.c_double
             lib.oracle_round_bf16_array.argtypes = [_D, _D, _I64]
@@ -167,4 +169,24 @@ def decode_step(state, x, dt_raw, dt_bias, A, B, C, D, round_state_bf16=False, n
                                         int(bool(round_state_bf16)), int(nthreads))
     if rc != 0:
         raise ValueError("oracle_ssd_decode_step: invalid arguments")
+    return y
+
+
+def decode_step_mimo(state, x, dt_raw, dt_bias, A, B, C, D, round_state_bf16=False, nthreads=0):
+    """One MIMO (rank-R) recurrent step in place on ``state`` [b,H,N,P] (float64, modified).
+
+    x [b,H,R,P], dt_raw [b,H], B,C [b,G,R,N].  Returns y [b,H,R,P].
+    """
+    if state.dtype != np.float64 or not state.flags.c_contiguous:
+        raise TypeError("state must be a C-contiguous float64 array (updated in place)")
+    x, dt_raw, dt_bias, A, B, C, D = map(_f64, (x, dt_raw, dt_bias, A, B, C, D))
+    b, H, R, P = x.shape
+    G, N = B.shape[1], B.shape[3]
+    assert state.shape == (b, H, N, P) and dt_raw.shape == (b, H) and B.shape == (b, G, R, N) and C.shape == B.shape
+    y = np.empty((b, H, R, P), dtype=np.float64)
+    rc = _load().oracle_ssd_decode_step_mimo(b, H, P, N, G, R, _ptr(state), _ptr(x), _ptr(dt_raw), _ptr(dt_bias),
+                                             _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(y),
+                                             int(bool(round_state_bf16)), int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle_ssd_decode_step_mimo: invalid arguments")
     return y

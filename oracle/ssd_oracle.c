@@ -38,6 +38,7 @@
  *   x, y [b][L][H][P]; dt_raw [b][L][H]; B, C [b][L][G][N];
  *   dt_bias, A, D [H]; init_state, final_state [b][H][N][P].
  *   Decode step: x, y [b][H][P]; dt_raw [b][H]; B, C [b][G][N]; state [b][H][N][P].
+ *   MIMO decode step (rank R): x, y [b][H][R][P]; B, C [b][G][R][N].
  *
  * All functions return 0 on success, -1 on invalid arguments.
  */
@@ -338,6 +339,55 @@ int oracle_ssd_decode_step(int64_t batch, int64_t nheads, int64_t headdim, int64
             for (int64_t p = 0; p < P; ++p) {
                 const double v = decay * st[n * P + p] + dt * Bt[n] * xt[p];
                 if (yt) yt[p] += Ct[n] * v;
+                st[n * P + p] = round_state_bf16 ? oracle_round_bf16(v) : v;
+            }
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* 5. One MIMO decode step: B, C widened to rank R ("Mamba3" (Telegram post), */
+/*    section on the switch from SISO to MIMO: outer products become matrix  */
+/*    products, the state size stays the same; "Mamba-3 : SSM optimise       */
+/*    inference", section "Mode MIMO": several SSMs in parallel with extended */
+/*    B and C matrices).  Reading, per (b, h), with X_t = [x_0 .. x_{R-1}]:   */
+/*      h_t = exp(dt A) h_{t-1} + dt * sum_r B_r x_r^T                        */
+/*      y_r = C_r^T h_t + D x_r          (r = 0 .. R-1)                       */
+/*    Layouts: x, y [b][H][R][P]; dt_raw [b][H]; B, C [b][G][R][N].  R = 1 is */
+/*    the decode step above.  round_state_bf16 as there.                      */
+/* ------------------------------------------------------------------------ */
+int oracle_ssd_decode_step_mimo(int64_t batch, int64_t nheads, int64_t headdim, int64_t dstate,
+                                int64_t ngroups, int64_t rank, double* state, const double* x,
+                                const double* dt_raw, const double* dt_bias, const double* A,
+                                const double* B, const double* C, const double* D, double* y,
+                                int round_state_bf16, int nthreads) {
+    if (check_dims(batch, 1, nheads, headdim, dstate, ngroups) || rank < 1) return -1;
+    if (!state || !x || !dt_raw || !A || !B || !C) return -1;
+    const int64_t H = nheads, P = headdim, N = dstate, G = ngroups, R = rank;
+    const int64_t heads_per_group = H / G;
+    const int nt = set_threads(nthreads);
+    int64_t pair;
+#pragma omp parallel for schedule(static) num_threads(nt)
+    for (pair = 0; pair < batch * H; ++pair) {
+        const int64_t b = pair / H, h = pair % H, g = h / heads_per_group;
+        const double dt = sp(dt_raw[b * H + h] + (dt_bias ? dt_bias[h] : 0.0));
+        const double decay = exp(dt * A[h]);
+        const double* Xt = x + (b * H + h) * R * P;          /* [R][P] */
+        const double* Bt = B + (b * G + g) * R * N;          /* [R][N] */
+        const double* Ct = C + (b * G + g) * R * N;
+        double* st = state + (b * H + h) * N * P;
+        double* yt = y ? y + (b * H + h) * R * P : NULL;
+        if (yt)
+            for (int64_t r = 0; r < R; ++r)
+                for (int64_t p = 0; p < P; ++p) yt[r * P + p] = (D ? D[h] : 0.0) * Xt[r * P + p];
+        for (int64_t n = 0; n < N; ++n) {
+            for (int64_t p = 0; p < P; ++p) {
+                double in = 0.0;                              /* sum_r B_r[n] x_r[p] */
+                for (int64_t r = 0; r < R; ++r) in += Bt[r * N + n] * Xt[r * P + p];
+                const double v = decay * st[n * P + p] + dt * in;
+                if (yt)
+                    for (int64_t r = 0; r < R; ++r) yt[r * P + p] += Ct[r * N + n] * v;
                 st[n * P + p] = round_state_bf16 ? oracle_round_bf16(v) : v;
             }
         }

@@ -36,6 +36,12 @@ MUTATIONS = [
      "const double dt = sp(dt_raw[(b * L + t) * H + h]);"),
     ("decode_state_not_decayed", "const double v = decay * st[n * P + p] + dt * Bt[n] * xt[p];",
      "const double v = st[n * P + p] + dt * Bt[n] * xt[p];"),
+    ("mimo_input_reads_C", "for (int64_t r = 0; r < R; ++r) in += Bt[r * N + n] * Xt[r * P + p];",
+     "for (int64_t r = 0; r < R; ++r) in += Ct[r * N + n] * Xt[r * P + p];"),
+    ("mimo_only_first_rank", "for (int64_t r = 0; r < R; ++r) in += Bt[r * N + n] * Xt[r * P + p];",
+     "for (int64_t r = 0; r < 1; ++r) in += Bt[r * N + n] * Xt[r * P + p];"),
+    ("mimo_output_rank_swapped", "for (int64_t r = 0; r < R; ++r) yt[r * P + p] += Ct[r * N + n] * v;",
+     "for (int64_t r = 0; r < R; ++r) yt[r * P + p] += Ct[(R - 1 - r) * N + n] * v;"),
 ]
 
 PIN_TESTS = [
@@ -51,6 +57,8 @@ PIN_TESTS = [
     lambda: pins.test_impulse_response_varying_dt("chunked"),
     pins.test_group_mapping,
     pins.test_decode_steps_equal_prefill,
+    lambda: pins.test_mimo_step_is_a_chain_of_single_input_steps(2),
+    lambda: pins.test_mimo_step_is_a_chain_of_single_input_steps(4),
 ]
 
 

@@ -310,3 +310,49 @@ def test_golden_regression():
                              init_state=h0)
     assert rel(y.ravel(), np.array(gold["y"])) < 1e-14
     assert rel(fs.ravel(), np.array(gold["final_state"])) < 1e-14
+
+
+# MIMO decode (rank R): pinned by compositions of the (pinned) single-input step.
+def _mimo_case(rng, b=2, H=4, P=3, N=5, G=2, R=3):
+    return dict(state=rng.standard_normal((b, H, N, P)), x=rng.standard_normal((b, H, R, P)),
+                dt_raw=rng.standard_normal((b, H)), dt_bias=np.log(np.expm1(rng.uniform(1e-2, 0.5, H))),
+                A=-rng.uniform(0.5, 4.0, H), B=rng.standard_normal((b, G, R, N)),
+                C=rng.standard_normal((b, G, R, N)), D=rng.standard_normal(H))
+
+
+def test_mimo_rank1_is_the_decode_step():
+    c = _mimo_case(np.random.default_rng(31), R=1)
+    st1, st2 = c["state"].copy(), c["state"].copy()
+    y1 = oracle.decode_step_mimo(st1, c["x"], c["dt_raw"], c["dt_bias"], c["A"], c["B"], c["C"], c["D"])
+    y2 = oracle.decode_step(st2, c["x"][:, :, 0], c["dt_raw"], c["dt_bias"], c["A"], c["B"][:, :, 0],
+                            c["C"][:, :, 0], c["D"])
+    assert rel(y1[:, :, 0], y2) < 1e-14 and rel(st1, st2) < 1e-14
+
+
+@pytest.mark.parametrize("R", [2, 4])
+def test_mimo_step_is_a_chain_of_single_input_steps(R):
+    """h <- exp(dt A) h + dt sum_r B_r x_r^T is one single-input step with input 0
+    followed by R-1 single-input steps with A = 0 (no decay) and the same dt; output
+    r is the last output of such a chain that ends with input r and reads C_r."""
+    c = _mimo_case(np.random.default_rng(40 + R), R=R)
+    st = c["state"].copy()
+    y = oracle.decode_step_mimo(st, c["x"], c["dt_raw"], c["dt_bias"], c["A"], c["B"], c["C"], c["D"])
+    zeroA = np.zeros_like(c["A"])
+    for r_last in range(R):
+        order = [r for r in range(R) if r != r_last] + [r_last]
+        chain = c["state"].copy()
+        for i, r in enumerate(order):
+            yc = oracle.decode_step(chain, c["x"][:, :, r], c["dt_raw"], c["dt_bias"], c["A"] if i == 0 else zeroA,
+                                    c["B"][:, :, r], c["C"][:, :, r_last], c["D"])
+        assert rel(chain, st) < 1e-13
+        assert rel(yc, y[:, :, r_last]) < 1e-13
+
+
+def test_mimo_bf16_state_rounding():
+    c = _mimo_case(np.random.default_rng(52), R=2)
+    exact, rounded = c["state"].copy(), c["state"].copy()
+    y1 = oracle.decode_step_mimo(exact, c["x"], c["dt_raw"], c["dt_bias"], c["A"], c["B"], c["C"], c["D"])
+    y2 = oracle.decode_step_mimo(rounded, c["x"], c["dt_raw"], c["dt_bias"], c["A"], c["B"], c["C"], c["D"],
+                                 round_state_bf16=True)
+    assert np.array_equal(y1, y2)
+    assert np.array_equal(rounded, oracle.round_bf16(exact))
