@@ -9,7 +9,8 @@ accumulation, y and final_state in fp32) on synthetic seeded inputs resident in
 HBM.  The same run also times K decode steps (ssd_state_update, batch 256, 128
 heads, P=64, N=128, 8 groups, fp32 state) and reports them under "decode",
 with the same steps replayed from a checkpoint and a 16-token buffer
-(ssd_replay_step) under "decode"."replay".
+(ssd_replay_step) under "decode"."replay" and rank-4 MIMO steps
+(ssd_state_update_mimo) on the same state under "decode"."mimo".
 
 Timing: W untimed warm-up steps, then exactly K steps between a barrier +
 cudaDeviceSynchronize on both sides, CUDA events on the launching stream, max
@@ -472,6 +473,46 @@ def main():
                                           "frac": rgbs / peaks["hbm_gbs"], "algorithmic_bytes_per_step": rbytes,
                                           "kernel": "replay_step_kernel"}}
 
+    # ---------------- MIMO decode (rank 4) on the same state: 4x the flops of a
+    # step for the same state traffic
+    MR = 4
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(dcfg.seed)
+    mx_ = (torch.randn((dcfg.batch, dcfg.nheads, MR, dcfg.headdim), generator=gen, device=dev)).bfloat16()
+    mB = (torch.randn((dcfg.batch, dcfg.ngroups, MR, dcfg.dstate), generator=gen, device=dev)).bfloat16()
+    mC = (torch.randn((dcfg.batch, dcfg.ngroups, MR, dcfg.dstate), generator=gen, device=dev)).bfloat16()
+    my_ = torch.empty((dcfg.batch, dcfg.nheads, MR, dcfg.headdim), dtype=torch.float32, device=dev)
+    mdesc = ssd.MimoDesc(dcfg.batch, dcfg.nheads, dcfg.headdim, dcfg.dstate, dcfg.ngroups, MR, ssd.SSD_BF16,
+                         ssd.SSD_F32, ssd.SSD_F32)
+
+    def mimo(t):
+        d = dsteps[t % nsteps_in]
+        st = ssd.ssd_state_update_mimo(mdesc, state.data_ptr(), mx_.data_ptr(), d["dt_raw"].data_ptr(),
+                                       prm["dt_bias"].data_ptr(), prm["A"].data_ptr(), mB.data_ptr(), mC.data_ptr(),
+                                       prm["D"].data_ptr(), my_.data_ptr(), stream.cuda_stream)
+        if st:
+            raise ssd.SsdError(st, "ssd_state_update_mimo")
+
+    for t in range(args.warmup):
+        mimo(t)
+    dist.barrier(pg)
+    torch.cuda.synchronize()
+    ev[0].record(stream)
+    for t in range(args.steps):
+        mimo(t)
+    ev[1].record(stream)
+    torch.cuda.synchronize()
+    dist.barrier(pg)
+    mms = dist.max_over_ranks(pg, ev[0].elapsed_time(ev[1]) / args.steps)
+    mbytes = (2 * sbytes + dcfg.batch * dcfg.nheads * MR * dcfg.headdim * (2 + 4)
+              + 2 * dcfg.batch * dcfg.ngroups * MR * dcfg.dstate * 2 + dcfg.batch * dcfg.nheads * 2)
+    mgbs = mbytes / (mms * 1e-3) / 1e9
+    decode_line["mimo"] = {"rank": MR, "tokens_per_s": dcfg.batch * world / (mms * 1e-3), "ms_per_step": mms,
+                           "time_vs_state_update": mms / dms,
+                           "roofline": {"bound": "hbm", "achieved": mgbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                        "frac": mgbs / peaks["hbm_gbs"], "algorithmic_bytes_per_step": mbytes,
+                                        "kernel": "mimo_step_kernel"}}
+
     # ---------------- end to end through the public API with host buffers
     e2e = None
     if rank == 0 or world > 1:
@@ -541,7 +582,7 @@ def main():
                            "kernel_path": "tensor cores" if path == 0 else "cuda cores"},
                 "tflops": tflops, "gbs": gbs, "roofline": roofline, "decode": decode_line,
                 "cpu_baseline": cpu_baseline, "e2e": e2e, "workloads": workloads,
-                "gpu_launches": launches_per_prefill * args.steps + args.steps + rsteps,
+                "gpu_launches": launches_per_prefill * args.steps + 2 * args.steps + rsteps,
                 "clocks": clk.summary()}
         print(json.dumps(line), flush=True)
     dist.finish(pg)

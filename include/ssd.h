@@ -102,6 +102,19 @@ typedef struct {
     int32_t state_dtype;/* dtype of the in-place state */
 } ssd_decode_desc_t;
 
+/* MIMO (rank-R) decode problem description. */
+typedef struct {
+    int64_t batch;      /* >= 0; 0 is a no-op */
+    int64_t nheads;
+    int64_t headdim;    /* P: 8, 16, 32, 64 or 128 */
+    int64_t dstate;     /* N, multiple of 8, <= 256 */
+    int64_t ngroups;
+    int64_t rank;       /* R: 1, 2, 4 or 8 */
+    int32_t io_dtype;   /* dtype of x, dt_raw, B, C */
+    int32_t y_dtype;    /* dtype of y */
+    int32_t state_dtype;/* dtype of the in-place state */
+} ssd_mimo_desc_t;
+
 /* Replayed decode (checkpoint + buffer of recent tokens) problem description. */
 typedef struct {
     int64_t batch;      /* >= 0; 0 is a no-op */
@@ -227,6 +240,33 @@ ssd_status_t ssd_state_update(const ssd_decode_desc_t* desc, void* state, const 
                               const void* dt_raw, const float* dt_bias, const float* A,
                               const void* B, const void* C, const float* D, void* y,
                               void* stream);
+
+/*
+ * MIMO decode step, in place on the state: B and C widened to rank R, the
+ * state keeps its N x P size ("Mamba3" (Telegram post), section on the switch
+ * from SISO to MIMO: the outer products become matrix products; "Mamba-3 :
+ * SSM optimise inference", section "Mode MIMO": several SSMs in parallel with
+ * extended B and C, more arithmetic for the same decode memory traffic).
+ * Per (b, h), with the R inputs x_r and outputs y_r of a token:
+ *
+ *   state <- exp(dt A) state + dt sum_r B_r x_r^T;   y_r = C_r^T state + D x_r
+ *
+ * rank 1 is ssd_state_update.
+ *  state  [b][H][N][P]     state_dtype  required, read and written in place
+ *                                        (bf16 state is rounded to nearest even)
+ *  x      [b][H][R][P]     io_dtype     required
+ *  dt_raw [b][H]           io_dtype     required (one dt per head and token)
+ *  dt_bias, A, D [H]       fp32         dt_bias, D nullable
+ *  B, C   [b][G][R][N]     io_dtype     required
+ *  y      [b][H][R][P]     y_dtype      required; must not overlap state or x
+ * Errors: SSD_ERR_INVALID_ARG, SSD_ERR_UNSUPPORTED (headdim not 8/16/32/64/128,
+ * rank not 1/2/4/8, dstate), SSD_ERR_ALIGNMENT, SSD_ERR_CUDA; nothing is
+ * launched on a host-side error.
+ */
+ssd_status_t ssd_state_update_mimo(const ssd_mimo_desc_t* desc, void* state, const void* x,
+                                   const void* dt_raw, const float* dt_bias, const float* A,
+                                   const void* B, const void* C, const float* D, void* y,
+                                   void* stream);
 
 /*
  * Bytes of the replay buffer ssd_replay_step needs for `desc` (written to

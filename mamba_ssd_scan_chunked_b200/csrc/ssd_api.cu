@@ -255,6 +255,42 @@ ssd_status_t ssd_state_update(const ssd_decode_desc_t* d, void* state, const voi
     return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
 }
 
+ssd_status_t ssd_state_update_mimo(const ssd_mimo_desc_t* d, void* state, const void* x, const void* dt_raw,
+                                   const float* dt_bias, const float* A, const void* B, const void* C,
+                                   const float* D, void* y, void* stream) {
+    if (!d) return SSD_ERR_INVALID_ARG;
+    if (d->batch < 0 || d->nheads < 1 || d->headdim < 1 || d->dstate < 1 || d->ngroups < 1 || d->rank < 1 ||
+        d->nheads % d->ngroups != 0)
+        return SSD_ERR_INVALID_ARG;
+    if (!valid_dtype(d->io_dtype) || !valid_dtype(d->y_dtype) || !valid_dtype(d->state_dtype))
+        return SSD_ERR_INVALID_ARG;
+    const int64_t P = d->headdim, R = d->rank;
+    if (!(P == 8 || P == 16 || P == 32 || P == 64 || P == 128)) return SSD_ERR_UNSUPPORTED;
+    if (!(R == 1 || R == 2 || R == 4 || R == 8)) return SSD_ERR_UNSUPPORTED;
+    if (d->dstate % 8 != 0 || d->dstate > 256) return SSD_ERR_UNSUPPORTED;
+    if (d->batch * d->nheads > (int64_t)0x7fffffff) return SSD_ERR_UNSUPPORTED;
+    if (!state || !x || !dt_raw || !A || !B || !C || !y) return SSD_ERR_INVALID_ARG;
+    const void* ptrs[] = {state, x, dt_raw, dt_bias, A, B, C, D, y};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return SSD_ERR_ALIGNMENT;
+    const size_t bh = (size_t)d->batch * d->nheads;
+    const size_t s_bytes = bh * d->dstate * P * dsize(d->state_dtype);
+    const size_t y_bytes = bh * R * P * dsize(d->y_dtype);
+    const size_t x_bytes = bh * R * P * dsize(d->io_dtype);
+    if (overlaps(y, y_bytes, state, s_bytes) || overlaps(y, y_bytes, x, x_bytes) ||
+        overlaps(state, s_bytes, x, x_bytes))
+        return SSD_ERR_INVALID_ARG;
+    if (d->batch == 0) return SSD_OK;
+    MimoArgs a{};
+    a.batch = d->batch; a.H = d->nheads; a.P = P; a.N = d->dstate; a.G = d->ngroups; a.R = R;
+    a.io_bf16 = d->io_dtype == SSD_BF16; a.y_bf16 = d->y_dtype == SSD_BF16;
+    a.state_bf16 = d->state_dtype == SSD_BF16;
+    a.state = state; a.x = x; a.dt_raw = dt_raw; a.B = B; a.C = C;
+    a.dt_bias = dt_bias; a.A = A; a.D = D; a.y = y;
+    const cudaError_t e = launch_mimo_step(a, (cudaStream_t)stream);
+    return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
+}
+
 ssd_status_t ssd_replay_buffer_size(const ssd_replay_desc_t* desc, size_t* bytes) {
     if (!bytes) return SSD_ERR_INVALID_ARG;
     const ssd_status_t st = check_replay_desc(desc);

@@ -39,6 +39,18 @@ struct ReplayLayout {
 
 cudaError_t launch_replay_step(const ReplayArgs& a, cudaStream_t stream);
 
+// MIMO (rank-R) decode step (ssd_mimo.cu).
+struct MimoArgs {
+    int64_t batch, H, P, N, G, R;
+    bool io_bf16, y_bf16, state_bf16;
+    void* state;
+    const void *x, *dt_raw, *B, *C;   // x [b][H][R][P]; B, C [b][G][R][N]
+    const float *dt_bias, *A, *D;
+    void* y;                          // [b][H][R][P]
+};
+
+cudaError_t launch_mimo_step(const MimoArgs& a, cudaStream_t stream);
+
 // Workspace carve-up of the prefill (all offsets 256-byte aligned).
 struct PrefillLayout {
     int64_t nchunks;       // ceil(L / Q)

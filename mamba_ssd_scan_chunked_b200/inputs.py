@@ -108,6 +108,17 @@ def draw_decode_step(t: int, batch: int, nheads: int, headdim: int, dstate: int,
     return {k: to_storage(v, dtype) for k, v in (("x", x), ("dt_raw", dt_raw), ("B", Bm), ("C", Cm))}
 
 
+def draw_mimo_step(t: int, batch: int, nheads: int, headdim: int, dstate: int,
+                   ngroups: int, rank: int, seed: int, dtype: str) -> dict:
+    """x [b,H,R,P], dt_raw [b,H], B [b,G,R,N], C [b,G,R,N] of a rank-R decode step t."""
+    rng = np.random.default_rng([seed, 4, t])
+    x = rng.standard_normal((batch, nheads, rank, headdim))
+    dt_raw = rng.standard_normal((batch, nheads))
+    Bm = rng.standard_normal((batch, ngroups, rank, dstate))
+    Cm = rng.standard_normal((batch, ngroups, rank, dstate))
+    return {k: to_storage(v, dtype) for k, v in (("x", x), ("dt_raw", dt_raw), ("B", Bm), ("C", Cm))}
+
+
 def prefill_inputs(batch: int, seqlen: int, nheads: int, headdim: int, dstate: int,
                    ngroups: int, seed: int, dtype: str, batches=None) -> dict:
     """Whole prefill input set (or the listed batch elements, in that order)."""

@@ -26,7 +26,8 @@ STATUS = {0: "SSD_OK", 1: "SSD_ERR_INVALID_ARG", 2: "SSD_ERR_UNSUPPORTED", 3: "S
 
 # every symbol include/ssd.h declares
 EXPORTS = ("ssd_version", "ssd_status_string", "ssd_chunk_scan_workspace_size", "ssd_chunk_scan_path",
-           "ssd_chunk_scan_fwd", "ssd_chunk_scan_fwd_noalloc", "ssd_state_update", "ssd_replay_buffer_size",
+           "ssd_chunk_scan_fwd", "ssd_chunk_scan_fwd_noalloc", "ssd_state_update", "ssd_state_update_mimo",
+           "ssd_replay_buffer_size",
            "ssd_replay_step", "ssd_get_device_error", "ssd_debug_inject")
 
 # fault-injection bits of ssd_debug_inject
@@ -53,6 +54,12 @@ class DecodeDesc(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int64), ("nheads", ctypes.c_int64), ("headdim", ctypes.c_int64),
                 ("dstate", ctypes.c_int64), ("ngroups", ctypes.c_int64), ("io_dtype", ctypes.c_int32),
                 ("y_dtype", ctypes.c_int32), ("state_dtype", ctypes.c_int32)]
+
+
+class MimoDesc(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int64), ("nheads", ctypes.c_int64), ("headdim", ctypes.c_int64),
+                ("dstate", ctypes.c_int64), ("ngroups", ctypes.c_int64), ("rank", ctypes.c_int64),
+                ("io_dtype", ctypes.c_int32), ("y_dtype", ctypes.c_int32), ("state_dtype", ctypes.c_int32)]
 
 
 class ReplayDesc(ctypes.Structure):
@@ -89,6 +96,8 @@ def lib():
             L.ssd_chunk_scan_fwd_noalloc.argtypes = [ctypes.POINTER(PrefillDesc)] + [_VP] * 11
             L.ssd_state_update.restype = ctypes.c_int
             L.ssd_state_update.argtypes = [ctypes.POINTER(DecodeDesc)] + [_VP] * 10
+            L.ssd_state_update_mimo.restype = ctypes.c_int
+            L.ssd_state_update_mimo.argtypes = [ctypes.POINTER(MimoDesc)] + [_VP] * 10
             L.ssd_replay_buffer_size.restype = ctypes.c_int
             L.ssd_replay_buffer_size.argtypes = [ctypes.POINTER(ReplayDesc), ctypes.POINTER(ctypes.c_size_t)]
             L.ssd_replay_step.restype = ctypes.c_int
@@ -147,6 +156,12 @@ def ssd_state_update(desc, state, x, dt_raw, dt_bias, A, B, C, D, y, stream) -> 
     """Raw call; returns the status code (0 = enqueued)."""
     return lib().ssd_state_update(ctypes.byref(desc), state or None, x or None, dt_raw or None, dt_bias or None,
                                   A or None, B or None, C or None, D or None, y or None, stream or None)
+
+
+def ssd_state_update_mimo(desc, state, x, dt_raw, dt_bias, A, B, C, D, y, stream) -> int:
+    """Raw call; returns the status code (0 = enqueued)."""
+    return lib().ssd_state_update_mimo(ctypes.byref(desc), state or None, x or None, dt_raw or None, dt_bias or None,
+                                       A or None, B or None, C or None, D or None, y or None, stream or None)
 
 
 def ssd_replay_buffer_size(desc: ReplayDesc) -> int:
@@ -301,3 +316,23 @@ def replay_step(checkpoint, buffer, fill, capacity, x, dt_raw, dt_bias, A, B, C,
     if st:
         raise SsdError(st, "ssd_replay_step")
     return y, (fill + 1) % int(capacity)
+
+
+def state_update_mimo(state, x, dt_raw, dt_bias, A, B, C, D, *, y=None, y_dtype=None, stream=None):
+    """MIMO decode step in place on ``state`` [b,H,N,P].  x [b,H,R,P], dt_raw [b,H], B/C [b,G,R,N].  Returns y."""
+    import torch
+    b, H, R, P = x.shape
+    G, N = B.shape[1], B.shape[3]
+    io = _dtype_code(x.dtype)
+    desc = MimoDesc(b, H, P, N, G, R, io, _dtype_code(y_dtype) if y_dtype is not None else io,
+                    _dtype_code(state.dtype))
+    for t in (state, x, dt_raw, B, C, dt_bias, A, D, y):
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("libssd takes contiguous CUDA tensors")
+    if y is None:
+        y = torch.empty((b, H, R, P), dtype=_torch_dtype(desc.y_dtype), device=x.device)
+    st = ssd_state_update_mimo(desc, _ptr(state), _ptr(x), _ptr(dt_raw), _ptr(dt_bias), _ptr(A), _ptr(B), _ptr(C),
+                               _ptr(D), _ptr(y), _stream(stream))
+    if st:
+        raise SsdError(st, "ssd_state_update_mimo")
+    return y

@@ -184,3 +184,28 @@ def test_replay_host_validation_codes():
     assert call(replay_d(), buf=FAKE + 0x100) == INVALID    # the buffer overlaps the checkpoint
     assert call(replay_d(headdim=48)) == UNSUPPORTED
     assert call(replay_d(batch=0)) == OK                   # nothing to do, nothing launched
+
+
+def test_mimo_host_validation_codes():
+    def md(**kw):
+        d = dict(batch=8, nheads=4, headdim=64, dstate=128, ngroups=2, rank=4, io_dtype=ssd.SSD_BF16,
+                 y_dtype=ssd.SSD_F32, state_dtype=ssd.SSD_F32)
+        d.update(kw)
+        return ssd.MimoDesc(**d)
+
+    def call(d, **ptrs):
+        p = dict(state=FAKE, x=FAKE + 0x1000000, dt_raw=FAKE + 0x2000000, dt_bias=0, A=FAKE + 0x3000000,
+                 B=FAKE + 0x4000000, C=FAKE + 0x5000000, D=0, y=FAKE + 0x6000000, stream=0)
+        p.update(ptrs)
+        return ssd.ssd_state_update_mimo(d, p["state"], p["x"], p["dt_raw"], p["dt_bias"], p["A"], p["B"], p["C"],
+                                         p["D"], p["y"], p["stream"])
+
+    assert call(md(rank=3)) == UNSUPPORTED
+    assert call(md(rank=16)) == UNSUPPORTED
+    assert call(md(rank=0)) == INVALID
+    assert call(md(headdim=256)) == UNSUPPORTED
+    assert call(md(ngroups=3)) == INVALID
+    assert call(md(), B=0) == INVALID
+    assert call(md(), x=FAKE + 0x1000008) == ALIGN
+    assert call(md(), y=FAKE + 0x1000000) == INVALID        # y overlaps x
+    assert call(md(batch=0)) == OK
