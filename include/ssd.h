@@ -186,6 +186,27 @@ ssd_status_t ssd_chunk_scan_fwd(const ssd_prefill_desc_t* desc,
                                 const void* init_state, void* y, void* final_state,
                                 void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * ssd_chunk_scan_fwd for a batch of variable-length, left-padded sequences
+ * (one of the adjacent steps the pages list with the Mamba-3 variants; the
+ * Hugging Face integration they cite batches with left padding).  Sequence b
+ * starts at token pad_left[b]: the tokens before it are absent from the
+ * recurrence (dt = 0 there: no decay, no input), so final_state[b] and y[b]
+ * from pad_left[b] on equal those of the unpadded sequence alone, started
+ * from init_state[b].  y at the padding positions is computed as if dt = 0
+ * (C_t^T h + D x_t with h the initial state); callers ignore it.
+ *  pad_left  [b] int32, device, required when batch > 0, 4-byte aligned;
+ *            values outside [0, seqlen] are clamped by their effect (a value
+ *            >= seqlen pads the whole sequence, a negative one nothing)
+ * All other arguments and errors as ssd_chunk_scan_fwd.
+ */
+ssd_status_t ssd_chunk_scan_fwd_varlen(const ssd_prefill_desc_t* desc,
+                                       const void* x, const void* dt_raw, const float* dt_bias,
+                                       const float* A, const void* B, const void* C, const float* D,
+                                       const void* init_state, const int32_t* pad_left, void* y,
+                                       void* final_state, void* workspace, size_t workspace_bytes,
+                                       void* stream);
+
 /* Size of the scratch array ssd_chunk_scan_fwd_noalloc uses (32 MiB per GPU). */
 #define SSD_NOALLOC_WORKSPACE_BYTES ((size_t)32 << 20)
 

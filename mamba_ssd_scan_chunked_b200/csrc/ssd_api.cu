@@ -168,10 +168,11 @@ ssd_status_t ssd_chunk_scan_path(const ssd_prefill_desc_t* desc, int32_t* path) 
     return SSD_OK;
 }
 
-ssd_status_t ssd_chunk_scan_fwd(const ssd_prefill_desc_t* d, const void* x, const void* dt_raw,
-                                const float* dt_bias, const float* A, const void* B, const void* C,
-                                const float* D, const void* init_state, void* y, void* final_state,
-                                void* workspace, size_t workspace_bytes, void* stream) {
+// ssd_chunk_scan_fwd and its variable-length form (pad_left NULL = no padding)
+static ssd_status_t prefill(const ssd_prefill_desc_t* d, const void* x, const void* dt_raw,
+                            const float* dt_bias, const float* A, const void* B, const void* C,
+                            const float* D, const void* init_state, const int32_t* pad_left, void* y,
+                            void* final_state, void* workspace, size_t workspace_bytes, void* stream) {
     ssd_status_t st = check_prefill_desc(d);
     if (st != SSD_OK) return st;
     const bool empty = d->batch == 0 || d->seqlen == 0;   // token tensors may then be NULL
@@ -211,6 +212,7 @@ ssd_status_t ssd_chunk_scan_fwd(const ssd_prefill_desc_t* d, const void* x, cons
     a.state_bf16 = d->state_dtype == SSD_BF16;
     a.x = x; a.dt_raw = dt_raw; a.B = B; a.C = C; a.dt_bias = dt_bias; a.A = A; a.D = D;
     a.init_state = init_state; a.y = y; a.final_state = final_state;
+    a.pad_left = pad_left;
     a.ws = (char*)workspace; a.lay = lay;
     a.drop_publish = (debug_faults() & SSD_FAULT_DROP_RUN_PUBLISH) ? 1 : 0;
     e = device_error_ptr(&a.dev_err);
@@ -219,6 +221,25 @@ ssd_status_t ssd_chunk_scan_fwd(const ssd_prefill_desc_t* d, const void* x, cons
     if (e != cudaSuccess) return SSD_ERR_CUDA;
     e = tc ? launch_prefill_tc(a, s) : launch_prefill_simt(a, s);
     return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
+}
+
+ssd_status_t ssd_chunk_scan_fwd(const ssd_prefill_desc_t* d, const void* x, const void* dt_raw,
+                                const float* dt_bias, const float* A, const void* B, const void* C,
+                                const float* D, const void* init_state, void* y, void* final_state,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+    return prefill(d, x, dt_raw, dt_bias, A, B, C, D, init_state, nullptr, y, final_state, workspace,
+                   workspace_bytes, stream);
+}
+
+ssd_status_t ssd_chunk_scan_fwd_varlen(const ssd_prefill_desc_t* d, const void* x, const void* dt_raw,
+                                       const float* dt_bias, const float* A, const void* B, const void* C,
+                                       const float* D, const void* init_state, const int32_t* pad_left, void* y,
+                                       void* final_state, void* workspace, size_t workspace_bytes,
+                                       void* stream) {
+    if (!pad_left && d && d->batch > 0) return SSD_ERR_INVALID_ARG;
+    if (pad_left && ((uintptr_t)pad_left & 3u)) return SSD_ERR_ALIGNMENT;
+    return prefill(d, x, dt_raw, dt_bias, A, B, C, D, init_state, pad_left, y, final_state, workspace,
+                   workspace_bytes, stream);
 }
 
 ssd_status_t ssd_state_update(const ssd_decode_desc_t* d, void* state, const void* x, const void* dt_raw,

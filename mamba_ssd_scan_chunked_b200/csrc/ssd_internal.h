@@ -71,6 +71,7 @@ struct PrefillArgs {
     void* final_state;
     char* ws;
     PrefillLayout lay;
+    const int32_t* pad_left;  // [batch] leading tokens to treat as absent (dt = 0), or NULL
     unsigned* dev_err;     // device error word of the current device
     int drop_publish;      // fault injection (ssd_debug_inject): run-entry states are never published
 };

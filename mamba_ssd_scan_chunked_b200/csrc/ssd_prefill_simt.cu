@@ -37,7 +37,7 @@ template <typename IoT>
 __global__ void __launch_bounds__(256)
 dt_cumsum_kernel(const IoT* __restrict__ dt_raw, const float* __restrict__ dt_bias,
                  const float* __restrict__ A, float* __restrict__ dt_out,
-                 float* __restrict__ acs_out, int* __restrict__ flags,
+                 float* __restrict__ acs_out, int* __restrict__ flags, const int32_t* __restrict__ pad_left,
                  int64_t L, int64_t Lpad, int H, int Q, int nflags, int nchunks, int hgroups) {
     __shared__ float warp_tot[8][DT_HG];       // Q <= 256: at most 8 warps
     const int hg = (int)(blockIdx.x % (unsigned)hgroups);
@@ -50,7 +50,8 @@ dt_cumsum_kernel(const IoT* __restrict__ dt_raw, const float* __restrict__ dt_bi
     const int l = threadIdx.x;                 // token within the chunk (blockDim = max(Q, 32))
     const int lane = l & 31, warp = l >> 5;
     const int64_t t = (int64_t)c * Q + l;
-    const bool live = l < Q && t < L;
+    // tokens before pad_left[b] are absent: dt = 0 (no decay, no input)
+    const bool live = l < Q && t < L && (!pad_left || t >= (int64_t)pad_left[b]);
     float raw[DT_HG];
 #pragma unroll
     for (int k = 0; k < DT_HG; ++k)
@@ -104,7 +105,7 @@ static cudaError_t launch_dt_t(const PrefillArgs& a, cudaStream_t s) {
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
     const unsigned threads = (unsigned)(a.Q < 32 ? 32 : a.Q);   // whole warps for the shuffles
     dt_cumsum_kernel<IoT><<<(unsigned)blocks, threads, 0, s>>>(
-        (const IoT*)a.dt_raw, a.dt_bias, a.A, dt, acs, flags, a.L, a.lay.Lpad, (int)a.H, (int)a.Q, nflags,
+        (const IoT*)a.dt_raw, a.dt_bias, a.A, dt, acs, flags, a.pad_left, a.L, a.lay.Lpad, (int)a.H, (int)a.Q, nflags,
         (int)a.lay.nchunks, hgroups);
     return cudaGetLastError();
 }

@@ -26,7 +26,7 @@ STATUS = {0: "SSD_OK", 1: "SSD_ERR_INVALID_ARG", 2: "SSD_ERR_UNSUPPORTED", 3: "S
 
 # every symbol include/ssd.h declares
 EXPORTS = ("ssd_version", "ssd_status_string", "ssd_chunk_scan_workspace_size", "ssd_chunk_scan_path",
-           "ssd_chunk_scan_fwd", "ssd_chunk_scan_fwd_noalloc", "ssd_state_update", "ssd_state_update_mimo",
+           "ssd_chunk_scan_fwd", "ssd_chunk_scan_fwd_varlen", "ssd_chunk_scan_fwd_noalloc", "ssd_state_update", "ssd_state_update_mimo",
            "ssd_replay_buffer_size",
            "ssd_replay_step", "ssd_get_device_error", "ssd_debug_inject")
 
@@ -92,6 +92,8 @@ def lib():
             L.ssd_chunk_scan_path.argtypes = [ctypes.POINTER(PrefillDesc), ctypes.POINTER(ctypes.c_int32)]
             L.ssd_chunk_scan_fwd.restype = ctypes.c_int
             L.ssd_chunk_scan_fwd.argtypes = [ctypes.POINTER(PrefillDesc)] + [_VP] * 10 + [_VP, ctypes.c_size_t, _VP]
+            L.ssd_chunk_scan_fwd_varlen.restype = ctypes.c_int
+            L.ssd_chunk_scan_fwd_varlen.argtypes = [ctypes.POINTER(PrefillDesc)] + [_VP] * 11 + [_VP, ctypes.c_size_t, _VP]
             L.ssd_chunk_scan_fwd_noalloc.restype = ctypes.c_int
             L.ssd_chunk_scan_fwd_noalloc.argtypes = [ctypes.POINTER(PrefillDesc)] + [_VP] * 11
             L.ssd_state_update.restype = ctypes.c_int
@@ -143,6 +145,15 @@ def ssd_chunk_scan_fwd(desc, x, dt_raw, dt_bias, A, B, C, D, init_state, y, fina
     return lib().ssd_chunk_scan_fwd(ctypes.byref(desc), x or None, dt_raw or None, dt_bias or None, A or None,
                                      B or None, C or None, D or None, init_state or None, y or None,
                                      final_state or None, workspace or None, int(workspace_bytes), stream or None)
+
+
+def ssd_chunk_scan_fwd_varlen(desc, x, dt_raw, dt_bias, A, B, C, D, init_state, pad_left, y, final_state,
+                              workspace, workspace_bytes, stream) -> int:
+    """Raw call of the left-padded variable-length variant; returns the status code."""
+    return lib().ssd_chunk_scan_fwd_varlen(ctypes.byref(desc), x or None, dt_raw or None, dt_bias or None, A or None,
+                                           B or None, C or None, D or None, init_state or None, pad_left or None,
+                                           y or None, final_state or None, workspace or None, int(workspace_bytes),
+                                           stream or None)
 
 
 def ssd_chunk_scan_fwd_noalloc(desc, x, dt_raw, dt_bias, A, B, C, D, init_state, y, final_state, stream) -> int:
@@ -234,8 +245,9 @@ def workspace_bytes(x, B, chunk, y_dtype=None, state_dtype=None) -> int:
 
 
 def chunk_scan_fwd(x, dt_raw, dt_bias, A, B, C, D, chunk, init_state=None, *, y=None, final_state=None,
-                   y_dtype=None, state_dtype=None, want_final_state=True, workspace=None, stream=None):
-    """Chunked prefill scan.  Shapes: x [b,L,H,P], dt_raw [b,L,H], B/C [b,L,G,N], dt_bias/A/D [H] (fp32).
+                   y_dtype=None, state_dtype=None, want_final_state=True, workspace=None, pad_left=None, stream=None):
+    """Chunked prefill scan.  Shapes: x [b,L,H,P], dt_raw [b,L,H], B/C [b,L,G,N], dt_bias/A/D [H] (fp32);
+    ``pad_left`` (int32 [b], CUDA) marks left-padded variable-length sequences.
 
     Returns (y, final_state).  Outputs and workspace are allocated with torch
     when not given; ``state_dtype`` defaults to init_state's dtype, else fp32.
@@ -256,9 +268,16 @@ def chunk_scan_fwd(x, dt_raw, dt_bias, A, B, C, D, chunk, init_state=None, *, y=
     need = ssd_chunk_scan_workspace_size(desc)
     if workspace is None or workspace.numel() < need:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
-    st = ssd_chunk_scan_fwd(desc, _ptr(x), _ptr(dt_raw), _ptr(dt_bias), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
-                            _ptr(init_state), _ptr(y), _ptr(final_state), _ptr(workspace), workspace.numel(),
-                            _stream(stream))
+    if pad_left is None:
+        st = ssd_chunk_scan_fwd(desc, _ptr(x), _ptr(dt_raw), _ptr(dt_bias), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                                _ptr(init_state), _ptr(y), _ptr(final_state), _ptr(workspace), workspace.numel(),
+                                _stream(stream))
+    else:
+        if pad_left.dtype != torch.int32 or not pad_left.is_cuda or not pad_left.is_contiguous():
+            raise ValueError("pad_left must be a contiguous int32 CUDA tensor [batch]")
+        st = ssd_chunk_scan_fwd_varlen(desc, _ptr(x), _ptr(dt_raw), _ptr(dt_bias), _ptr(A), _ptr(B), _ptr(C),
+                                       _ptr(D), _ptr(init_state), _ptr(pad_left), _ptr(y), _ptr(final_state),
+                                       _ptr(workspace), workspace.numel(), _stream(stream))
     if st:
         raise SsdError(st, "ssd_chunk_scan_fwd")
     return y, final_state

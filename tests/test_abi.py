@@ -209,3 +209,22 @@ def test_mimo_host_validation_codes():
     assert call(md(), x=FAKE + 0x1000008) == ALIGN
     assert call(md(), y=FAKE + 0x1000000) == INVALID        # y overlaps x
     assert call(md(batch=0)) == OK
+
+
+def test_varlen_host_validation_codes():
+    d = desc()
+    need = ssd.ssd_chunk_scan_workspace_size(d)
+
+    def call(pad_left, **kw):
+        p = dict(x=FAKE, dt_raw=FAKE + 0x1000000, dt_bias=0, A=FAKE + 0x2000000, B=FAKE + 0x3000000,
+                 C=FAKE + 0x4000000, D=0, init_state=0, y=FAKE + 0x10000000, final_state=0,
+                 workspace=0, workspace_bytes=0, stream=0)
+        p.update(kw)
+        return ssd.ssd_chunk_scan_fwd_varlen(d, p["x"], p["dt_raw"], p["dt_bias"], p["A"], p["B"], p["C"], p["D"],
+                                             p["init_state"], pad_left, p["y"], p["final_state"], p["workspace"],
+                                             p["workspace_bytes"], p["stream"])
+
+    assert call(0) == INVALID                              # pad_left is required
+    assert call(FAKE + 0x30000002) == ALIGN                # int32 array: 4-byte aligned
+    assert call(FAKE + 0x30000000) == WORKSPACE            # otherwise the checks of ssd_chunk_scan_fwd
+    assert need > 0
