@@ -42,7 +42,7 @@ METRIC = "SSD prefill tokens/s + TFLOP/s; decode tokens/s + state GB/s (1 B200)"
 # of the SHA-256 of the kernel's source file at capture time: a changed kernel
 # reports null until it is captured again (summaries under profiles/).
 NCU_TRAFFIC = {
-    "ssd_prefill_tc.cu": ("7e67b905026fb3cb", 75557632 + 88568320),
+    "ssd_prefill_tc.cu": ("ef13bab91c33b8b7", 75555072 + 87655680),
     "ssd_decode.cu": ("cba348ad46ab41a0", 1079097000 + 1024990000),
 }
 
