@@ -323,7 +323,10 @@ ssd_status_t ssd_replay_buffer_size(const ssd_replay_desc_t* desc, size_t* bytes
  *  x [b][H][P], dt_raw [b][H], B, C [b][G][N]: io_dtype, required
  *  dt_bias, A, D [H] fp32 (dt_bias, D nullable); y [b][H][P] y_dtype, required
  * Calls on one buffer must be ordered on one stream (each step reads what the
- * previous one appended).
+ * previous one appended).  Rollback (speculative decoding, which the pages name
+ * as a use): until the buffer is folded the checkpoint is only read, so the
+ * last k buffered tokens are dropped by calling again with fill - k; tokens
+ * already folded into the checkpoint cannot be dropped.
  * Errors: SSD_ERR_INVALID_ARG (bad descriptor, fill out of range, NULL
  * pointers, y/x/checkpoint/buffer overlapping), SSD_ERR_UNSUPPORTED
  * (headdim not 8/16/32/64/128, dstate, capacity > 16), SSD_ERR_ALIGNMENT,

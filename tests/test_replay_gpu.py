@@ -85,3 +85,40 @@ def test_capacity_one_equals_state_update():
     # fp32 either way; only the rounding order differs (alpha h + (beta B_n) x_p
     # here, one fma of exp(dt A) h and dt B_n x_p there), over five steps
     assert metric(to_host64(s_replay), to_host64(s_plain)) <= 1e-5
+
+
+def test_rollback_by_lowering_fill():
+    """Speculative decoding: the checkpoint is only read until the buffer fills,
+    so dropping the last k buffered tokens is a call with fill - k.  Steps 0..5
+    are taken, steps 4 and 5 are rejected, and two other tokens follow; the
+    outputs must be the oracle's for the accepted sequence 0..3, 6, 7."""
+    t = torch()
+    b, H, P, N, G, K = 2, 4, 64, 128, 2, 16
+    params = I.draw_head_params(H, seed=71)
+    st0 = np.stack([I.draw_decode_state(i, H, P, N, seed=72, dtype=I.F32) for i in range(b)])
+    steps = [I.draw_decode_step(s, b, H, P, N, G, seed=73, dtype=I.BF16) for s in range(8)]
+    ckpt = to_dev(st0)
+    prm = {k: to_dev(v) for k, v in params.items()}
+    dev = [{k: to_dev(v) for k, v in s.items()} for s in steps]
+    buf = ssd.replay_buffer(ckpt, dev[0]["x"], dev[0]["B"], K)
+
+    def step(i, fill):
+        d = dev[i]
+        return ssd.replay_step(ckpt, buf, fill, K, d["x"], d["dt_raw"], prm["dt_bias"], prm["A"], d["B"], d["C"],
+                               prm["D"], y_dtype=t.float32)
+
+    fill = 0
+    for i in range(6):                          # 0..3 accepted, 4 and 5 speculative
+        _, fill = step(i, fill)
+    fill -= 2                                   # reject 4 and 5
+    ys = [step(i, f)[0] for i, f in ((6, fill), (7, fill + 1))]
+    ref = I.to_f64(st0).copy()
+    f = {k: I.to_f64(v) for k, v in params.items()}
+    y_ref = None
+    for i in (0, 1, 2, 3, 6, 7):
+        g = {k: I.to_f64(v) for k, v in steps[i].items()}
+        y_ref = oracle.decode_step(ref, g["x"], g["dt_raw"], f["dt_bias"], f["A"], g["B"], g["C"], f["D"])
+        if i == 6:
+            y6_ref = y_ref
+    assert metric(to_host64(ys[0]), y6_ref) <= TOL_BF16
+    assert metric(to_host64(ys[1]), y_ref) <= TOL_BF16
