@@ -20,6 +20,10 @@ C file's header:
 - ``chunked``    -- the blocked two-pass contraction with per-chunk states
   recombined across chunks (same page, same section, and its table row
   "Mamba-2 SSD layer | Blocked two-pass contraction").
+- ``backward``   -- reverse-mode gradients of the recurrence (the pages only
+  say that end-to-end training also needs the backward pass: "Mamba-3 : SSM
+  optimise inference", opening paragraph; the gradients follow from the
+  forward definition).
 - ``decode_step`` -- one token of the recurrent mode, in place on the state
   (same page, table "Evaluation criteria": O(1) recurrent step at inference).
 
@@ -74,6 +78,8 @@ def _load():
             lib.oracle_ssd_decode_step.restype = ctypes.c_int
             lib.oracle_ssd_decode_step_mimo.argtypes = [_I64] * 6 + [_D] * 9 + [ctypes.c_int, ctypes.c_int]
             lib.oracle_ssd_decode_step_mimo.restype = ctypes.c_int
+            lib.oracle_ssd_backward.argtypes = sig6 + [_D] * 18 + [ctypes.c_int]
+            lib.oracle_ssd_backward.restype = ctypes.c_int
             lib.oracle_round_bf16.argtypes = [ctypes.c_double]
             lib.oracle_round_bf16.restype = ctypes.c_double
             lib.oracle_round_bf16_array.argtypes = [_D, _D, _I64]
@@ -190,3 +196,27 @@ def decode_step_mimo(state, x, dt_raw, dt_bias, A, B, C, D, round_state_bf16=Fal
     if rc != 0:
         raise ValueError("oracle_ssd_decode_step_mimo: invalid arguments")
     return y
+
+
+def backward(x, dt_raw, dt_bias, A, B, C, D, init_state, dy, dfinal=None, nthreads=0):
+    """Gradients of sum<dy, y> + <dfinal, final_state> through the recurrence.
+
+    Shapes as in ``recurrent``; dy [b,L,H,P], dfinal [b,H,N,P] or None.
+    Returns a dict of float64 arrays: dx, ddt_raw, ddt_bias, dA, dB, dC, dD,
+    dinit_state (same shapes as the forward inputs).
+    """
+    x, dt_raw, dt_bias, A, B, C, D, init_state, dy, dfinal = map(
+        _f64, (x, dt_raw, dt_bias, A, B, C, D, init_state, dy, dfinal))
+    b, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    assert dt_raw.shape == (b, L, H) and B.shape == C.shape == (b, L, G, N) and dy.shape == x.shape
+    out = {"dx": np.empty_like(x), "ddt_raw": np.empty_like(dt_raw), "ddt_bias": np.empty(H),
+           "dA": np.empty(H), "dB": np.empty_like(B), "dC": np.empty_like(C), "dD": np.empty(H),
+           "dinit_state": np.empty((b, H, N, P))}
+    rc = _load().oracle_ssd_backward(b, L, H, P, N, G, _ptr(x), _ptr(dt_raw), _ptr(dt_bias), _ptr(A), _ptr(B),
+                                     _ptr(C), _ptr(D), _ptr(init_state), _ptr(dy), _ptr(dfinal),
+                                     *(_ptr(out[k]) for k in ("dx", "ddt_raw", "ddt_bias", "dA", "dB", "dC",
+                                                             "dD", "dinit_state")), int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle_ssd_backward: invalid arguments")
+    return out

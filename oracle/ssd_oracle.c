@@ -394,3 +394,161 @@ int oracle_ssd_decode_step_mimo(int64_t batch, int64_t nheads, int64_t headdim, 
     }
     return 0;
 }
+
+/* ------------------------------------------------------------------------ */
+/* 6. Backward pass: reverse-mode gradients of the sequential recurrence.    */
+/* ------------------------------------------------------------------------ */
+/* The pages only say that end-to-end training also needs the backward pass
+ * ("Mamba-3 : SSM optimise inference", opening paragraph); what it computes is
+ * fixed by the forward definition above.  For the scalar loss
+ *     loss = sum_t <dy_t, y_t> + <dfinal, h_{L-1}>
+ * the adjoint of the state, G_t = d loss / d h_t (N x P), obeys
+ *     G_{L-1} = dfinal + C_{L-1} dy_{L-1}^T,
+ *     G_t     = C_t dy_t^T + exp(dt_{t+1} A) G_{t+1},
+ * and every gradient is a local product at token t (with hp = h_{t-1}):
+ *     dx_t   = dt_t B_t^T G_t + D dy_t
+ *     dB_t  += dt_t G_t x_t                 (summed over the heads of a group)
+ *     dC_t  += h_t dy_t                     (same)
+ *     d(dt A)_t = exp(dt_t A) <G_t, hp>
+ *     d dt_t = <G_t, B_t x_t^T> + A d(dt A)_t
+ *     d dt_raw_t = d dt_t * sigmoid(dt_raw_t + dt_bias)   (softplus' = sigmoid)
+ *     dA += dt_t d(dt A)_t;  d dt_bias += d dt_raw_t;  dD += <dy_t, x_t>
+ *     d init_state = exp(dt_0 A) G_0.
+ * The states h_t are not all kept: one every SEG tokens is, and each segment
+ * is recomputed from its checkpoint during the reverse sweep.
+ * dinit, ddt_bias and dD may be NULL (not computed); dfinal, init_state, D and
+ * dt_bias may be NULL (zero). */
+#define ORACLE_BWD_SEG 64
+
+static void step_state(double* dst, const double* src, double decay, double dt, const double* Bt,
+                       const double* xt, int64_t N, int64_t P) {
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t p = 0; p < P; ++p) dst[n * P + p] = decay * src[n * P + p] + dt * Bt[n] * xt[p];
+}
+
+int oracle_ssd_backward(int64_t batch, int64_t seqlen, int64_t nheads, int64_t headdim, int64_t dstate,
+                        int64_t ngroups, const double* x, const double* dt_raw, const double* dt_bias,
+                        const double* A, const double* B, const double* C, const double* D,
+                        const double* init_state, const double* dy, const double* dfinal, double* dx,
+                        double* ddt_raw, double* ddt_bias, double* dA, double* dB, double* dC, double* dD,
+                        double* dinit, int nthreads) {
+    if (check_dims(batch, seqlen, nheads, headdim, dstate, ngroups)) return -1;
+    if (!x || !dt_raw || !A || !B || !C || !dy || !dx || !ddt_raw || !dA || !dB || !dC) return -1;
+    const int64_t H = nheads, P = headdim, N = dstate, G = ngroups, L = seqlen, NP = N * P;
+    const int64_t heads_per_group = H / G, S = ORACLE_BWD_SEG, nseg = (L + S - 1) / S;
+    /* per-head dB, dC and per-(b, h) partial sums, reduced in a fixed order below */
+    double* dBh = (double*)calloc((size_t)(batch * L * H * N) + 1, sizeof(double));
+    double* dCh = (double*)calloc((size_t)(batch * L * H * N) + 1, sizeof(double));
+    double* part = (double*)calloc((size_t)(3 * batch * H), sizeof(double));
+    if (!dBh || !dCh || !part) { free(dBh); free(dCh); free(part); return -1; }
+    const int nt = set_threads(nthreads);
+    int64_t pair;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nt)
+    for (pair = 0; pair < batch * H; ++pair) {
+        const int64_t b = pair / H, h = pair % H, g = h / heads_per_group;
+        const double bias = dt_bias ? dt_bias[h] : 0.0, d_skip = D ? D[h] : 0.0, Ah = A[h];
+        double* ck = (double*)malloc(sizeof(double) * (size_t)((nseg + 1) * NP));   /* h before each segment */
+        double* seg = (double*)malloc(sizeof(double) * (size_t)((S + 1) * NP));     /* h_{t0-1} .. h_{t1-1} */
+        double* Gs = (double*)malloc(sizeof(double) * (size_t)NP);
+        /* forward sweep: keep the state entering every segment */
+        double* cur = seg;
+        if (init_state) memcpy(cur, init_state + (b * H + h) * NP, sizeof(double) * NP);
+        else memset(cur, 0, sizeof(double) * NP);
+        for (int64_t t = 0; t < L; ++t) {
+            if (t % S == 0) memcpy(ck + (t / S) * NP, cur, sizeof(double) * NP);
+            const double dt = sp(dt_raw[(b * L + t) * H + h] + bias);
+            step_state(seg + NP, cur, exp(dt * Ah), dt, B + ((b * L + t) * G + g) * N,
+                       x + ((b * L + t) * H + h) * P, N, P);
+            memcpy(cur, seg + NP, sizeof(double) * NP);
+        }
+        /* reverse sweep */
+        if (dfinal) memcpy(Gs, dfinal + (b * H + h) * NP, sizeof(double) * NP);
+        else memset(Gs, 0, sizeof(double) * NP);
+        double sum_dA = 0.0, sum_dbias = 0.0, sum_dD = 0.0;
+        for (int64_t k = nseg - 1; k >= 0; --k) {
+            const int64_t t0 = k * S, t1 = (t0 + S < L) ? t0 + S : L;
+            memcpy(seg, ck + k * NP, sizeof(double) * NP);
+            for (int64_t t = t0; t < t1; ++t) {
+                const double dt = sp(dt_raw[(b * L + t) * H + h] + bias);
+                step_state(seg + (t - t0 + 1) * NP, seg + (t - t0) * NP, exp(dt * Ah), dt,
+                           B + ((b * L + t) * G + g) * N, x + ((b * L + t) * H + h) * P, N, P);
+            }
+            for (int64_t t = t1 - 1; t >= t0; --t) {
+                const double* hp = seg + (t - t0) * NP;       /* h_{t-1} */
+                const double* hc = seg + (t - t0 + 1) * NP;   /* h_t */
+                const double z = dt_raw[(b * L + t) * H + h] + bias;
+                const double dt = sp(z), decay = exp(dt * Ah);
+                const double* xt = x + ((b * L + t) * H + h) * P;
+                const double* dyt = dy + ((b * L + t) * H + h) * P;
+                const double* Bt = B + ((b * L + t) * G + g) * N;
+                const double* Ct = C + ((b * L + t) * G + g) * N;
+                /* y_t reads h_t: G_t gains C_t dy_t^T */
+                for (int64_t n = 0; n < N; ++n)
+                    for (int64_t p = 0; p < P; ++p) Gs[n * P + p] += Ct[n] * dyt[p];
+                double* dxt = dx + ((b * L + t) * H + h) * P;
+                for (int64_t p = 0; p < P; ++p) {
+                    double acc = 0.0;
+                    for (int64_t n = 0; n < N; ++n) acc += Bt[n] * Gs[n * P + p];
+                    dxt[p] = dt * acc + d_skip * dyt[p];
+                }
+                double* dBt = dBh + ((b * L + t) * H + h) * N;
+                double* dCt = dCh + ((b * L + t) * H + h) * N;
+                double gbx = 0.0, gh = 0.0;
+                for (int64_t n = 0; n < N; ++n) {
+                    double gx = 0.0, hy = 0.0;
+                    for (int64_t p = 0; p < P; ++p) {
+                        gx += Gs[n * P + p] * xt[p];
+                        hy += hc[n * P + p] * dyt[p];
+                        gh += Gs[n * P + p] * hp[n * P + p];
+                    }
+                    dBt[n] = dt * gx;
+                    dCt[n] = hy;
+                    gbx += Bt[n] * gx;
+                }
+                const double dlogdecay = decay * gh;            /* d loss / d (dt_t A) */
+                const double ddt = gbx + Ah * dlogdecay;
+                const double dz = ddt / (1.0 + exp(-z));
+                ddt_raw[(b * L + t) * H + h] = dz;
+                sum_dA += dt * dlogdecay;
+                sum_dbias += dz;
+                for (int64_t p = 0; p < P; ++p) sum_dD += dyt[p] * xt[p];
+                /* G_{t-1} part that flows through the transition */
+                for (int64_t i = 0; i < NP; ++i) Gs[i] *= decay;
+            }
+        }
+        if (dinit) memcpy(dinit + (b * H + h) * NP, Gs, sizeof(double) * NP);
+        part[3 * pair + 0] = sum_dA;
+        part[3 * pair + 1] = sum_dbias;
+        part[3 * pair + 2] = sum_dD;
+        free(ck);
+        free(seg);
+        free(Gs);
+    }
+    for (int64_t bt = 0; bt < batch * L; ++bt)
+        for (int64_t g = 0; g < G; ++g)
+            for (int64_t n = 0; n < N; ++n) {
+                double sb = 0.0, sc = 0.0;
+                for (int64_t j = 0; j < heads_per_group; ++j) {
+                    const int64_t h = g * heads_per_group + j;
+                    sb += dBh[(bt * H + h) * N + n];
+                    sc += dCh[(bt * H + h) * N + n];
+                }
+                dB[(bt * G + g) * N + n] = sb;
+                dC[(bt * G + g) * N + n] = sc;
+            }
+    for (int64_t h = 0; h < H; ++h) {
+        double sa = 0.0, sbias = 0.0, sd = 0.0;
+        for (int64_t b = 0; b < batch; ++b) {
+            sa += part[3 * (b * H + h) + 0];
+            sbias += part[3 * (b * H + h) + 1];
+            sd += part[3 * (b * H + h) + 2];
+        }
+        dA[h] = sa;
+        if (ddt_bias) ddt_bias[h] = sbias;
+        if (dD) dD[h] = sd;
+    }
+    free(dBh);
+    free(dCh);
+    free(part);
+    return 0;
+}

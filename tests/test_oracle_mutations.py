@@ -2,7 +2,7 @@
 
 Each case plants one slip in a temporary copy of the oracle's C source (on the
 CPU, never on a GPU), rebuilds it, and reruns the pins of
-``test_oracle_pins.py`` against the mutant: at least one pin must fail.
+``test_oracle_pins.py`` and ``test_oracle_bwd_pins.py`` against the mutant: at least one pin must fail.
 """
 import importlib.util
 import os
@@ -10,6 +10,7 @@ import sys
 
 import pytest
 
+import tests.test_oracle_bwd_pins as bwd_pins
 import tests.test_oracle_pins as pins
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -42,6 +43,15 @@ MUTATIONS = [
      "for (int64_t r = 0; r < 1; ++r) in += Bt[r * N + n] * Xt[r * P + p];"),
     ("mimo_output_rank_swapped", "for (int64_t r = 0; r < R; ++r) yt[r * P + p] += Ct[r * N + n] * v;",
      "for (int64_t r = 0; r < R; ++r) yt[r * P + p] += Ct[(R - 1 - r) * N + n] * v;"),
+    ("bwd_final_seed_dropped", "if (dfinal) memcpy(Gs, dfinal", "if (0) memcpy(Gs, dfinal"),
+    ("bwd_adjoint_not_decayed", "for (int64_t i = 0; i < NP; ++i) Gs[i] *= decay;",
+     "for (int64_t i = 0; i < NP; ++i) Gs[i] *= 1.0;"),
+    ("bwd_softplus_derivative_dropped", "const double dz = ddt / (1.0 + exp(-z));", "const double dz = ddt;"),
+    ("bwd_dB_missing_dt", "dBt[n] = dt * gx;", "dBt[n] = gx;"),
+    ("bwd_dC_reads_previous_state", "hy += hc[n * P + p] * dyt[p];", "hy += hp[n * P + p] * dyt[p];"),
+    ("bwd_decay_path_of_dt_dropped", "const double ddt = gbx + Ah * dlogdecay;", "const double ddt = gbx;"),
+    ("bwd_wrong_segment_checkpoint", "memcpy(seg, ck + k * NP, sizeof(double) * NP);",
+     "memcpy(seg, ck + (k > 0 ? k - 1 : 0) * NP, sizeof(double) * NP);"),
 ]
 
 PIN_TESTS = [
@@ -59,6 +69,9 @@ PIN_TESTS = [
     pins.test_decode_steps_equal_prefill,
     lambda: pins.test_mimo_step_is_a_chain_of_single_input_steps(2),
     lambda: pins.test_mimo_step_is_a_chain_of_single_input_steps(4),
+    lambda: bwd_pins.test_backward_elementwise_finite_differences(2),
+    lambda: bwd_pins.test_backward_directional_finite_differences(True, True),
+    bwd_pins.test_backward_single_token_closed_form,
 ]
 
 
@@ -82,6 +95,7 @@ def _load_mutant(tmp_path, name, old, new):
 def test_pins_catch_mutation(tmp_path, monkeypatch, name, old, new):
     mutant = _load_mutant(tmp_path, name, old, new)
     monkeypatch.setattr(pins, "oracle", mutant)
+    monkeypatch.setattr(bwd_pins, "oracle", mutant)
     caught = 0
     for t in PIN_TESTS:
         try:
