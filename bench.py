@@ -10,7 +10,9 @@ HBM.  The same run also times K decode steps (ssd_state_update, batch 256, 128
 heads, P=64, N=128, 8 groups, fp32 state) and reports them under "decode",
 with the same steps replayed from a checkpoint and a 16-token buffer
 (ssd_replay_step) under "decode"."replay" and rank-4 MIMO steps
-(ssd_state_update_mimo) on the same state under "decode"."mimo".
+(ssd_state_update_mimo) on the same state under "decode"."mimo", and the
+backward pass of the prefill (ssd_chunk_scan_bwd, fp32 gradients, with a
+final-state gradient) under "backward".
 
 Timing: W untimed warm-up steps, then exactly K steps between a barrier +
 cudaDeviceSynchronize on both sides, CUDA events on the launching stream, max
@@ -83,6 +85,21 @@ def prefill_bytes(b, L, H, P, N, G, io_bytes, y_bytes, state_bytes, with_init=Fa
     n = tok * H * P * io_bytes + tok * H * P * y_bytes + 2 * tok * G * N * io_bytes + tok * H * io_bytes
     n += b * H * N * P * state_bytes * (2 if with_init else 1)
     return n
+
+
+def backward_bytes(b, L, H, P, N, G, io_bytes, grad_bytes, state_bytes):
+    """Algorithmic bytes of the backward pass: x, dy, dt_raw, B, C read (io
+    dtype) and dfinal_state read; dx, ddt_raw, dB, dC written (gradient dtype)."""
+    tok = b * L
+    ins = tok * (2 * H * P + H + 2 * G * N) * io_bytes + b * H * N * P * state_bytes
+    outs = tok * (H * P + H + 2 * G * N) * grad_bytes
+    return ins + outs
+
+
+def backward_flops(b, L, H, P, N, G, Q):
+    """The backward's three chunked scans: the state adjoint (the forward's
+    shape) and two transposed scans (headdim N, dstate P, one group per head)."""
+    return prefill_flops(b, L, H, P, N, G, Q) + 2 * prefill_flops(b, L, H, N, P, H, Q)
 
 
 def decode_bytes(b, H, P, N, G, io_bytes, y_bytes, state_bytes):
@@ -513,6 +530,65 @@ def main():
                                         "frac": mgbs / peaks["hbm_gbs"], "algorithmic_bytes_per_step": mbytes,
                                         "kernel": "mimo_step_kernel"}}
 
+    # ---------------- backward pass of the same layer, timed the same way
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1000 + rank)
+    dyb = torch.randn((s.batch, s.seqlen, s.nheads, s.headdim), generator=gen, device=dev).to(torch.bfloat16)
+    dfin = 0.1 * torch.randn((s.batch, s.nheads, s.dstate, s.headdim), generator=gen, device=dev)
+    bdesc = ssd.prefill_desc(sets[0]["x"], sets[0]["B"], s.chunk, torch.float32, torch.float32)
+    bws = torch.empty(ssd.ssd_chunk_scan_bwd_workspace_size(bdesc), dtype=torch.uint8, device=dev)
+    gx = torch.empty((s.batch, s.seqlen, s.nheads, s.headdim), dtype=torch.float32, device=dev)
+    gdt = torch.empty((s.batch, s.seqlen, s.nheads), dtype=torch.float32, device=dev)
+    gB = torch.empty((s.batch, s.seqlen, s.ngroups, s.dstate), dtype=torch.float32, device=dev)
+    gC = torch.empty_like(gB)
+    gpar = torch.empty((3, s.nheads), dtype=torch.float32, device=dev)
+    launches_per_bwd = ssd.ssd_chunk_scan_bwd_launches(bdesc, True)
+
+    def backward(k):
+        d = sets[k % NSETS]
+        st = ssd.ssd_chunk_scan_bwd(bdesc, d["x"].data_ptr(), d["dt_raw"].data_ptr(), d["dt_bias"].data_ptr(),
+                                    d["A"].data_ptr(), d["B"].data_ptr(), d["C"].data_ptr(), d["D"].data_ptr(), 0,
+                                    dyb.data_ptr(), dfin.data_ptr(), gx.data_ptr(), gdt.data_ptr(),
+                                    gpar[0].data_ptr(), gpar[1].data_ptr(), gB.data_ptr(), gC.data_ptr(),
+                                    gpar[2].data_ptr(), 0, bws.data_ptr(), bws.numel(), stream.cuda_stream)
+        if st:
+            raise ssd.SsdError(st, "ssd_chunk_scan_bwd")
+
+    bsteps = max(3, min(args.steps, 10))
+    for k in range(args.warmup):
+        backward(k)
+    dist.barrier(pg)
+    torch.cuda.synchronize()
+    ev[0].record(stream)
+    for k in range(bsteps):
+        backward(k)
+    ev[1].record(stream)
+    torch.cuda.synchronize()
+    dist.barrier(pg)
+    bms = dist.max_over_ranks(pg, ev[0].elapsed_time(ev[1]) / bsteps)
+    st_err, detail = ssd.ssd_get_device_error(stream.cuda_stream)
+    if st_err:
+        raise RuntimeError(f"device error word {detail:#x} after the timed backward")
+    bbytes = backward_bytes(s.batch, s.seqlen, s.nheads, s.headdim, s.dstate, s.ngroups, 2, 4, 4)
+    bflops = backward_flops(s.batch, s.seqlen, s.nheads, s.headdim, s.dstate, s.ngroups, s.chunk)
+    bt_hbm = bbytes / (peaks["hbm_gbs"] * 1e9)
+    bt_tc = bflops / (peaks["bf16_tflops"] * 1e12)
+    bgbs = bbytes / (bms * 1e-3) / 1e9
+    btf = bflops / (bms * 1e-3) / 1e12
+    if bt_hbm >= bt_tc:
+        broof = {"bound": "hbm", "achieved": bgbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                 "frac": bgbs / peaks["hbm_gbs"]}
+    else:
+        broof = {"bound": "tensor", "achieved": btf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                 "frac": btf / peaks["bf16_tflops"]}
+    backward_line = {"tokens_per_s": tokens_rank * world / (bms * 1e-3), "ms_per_step": bms, "steps": bsteps,
+                     "launches_per_step": launches_per_bwd, "gradients": "fp32", "dfinal_state": "given",
+                     "gbs": bgbs, "tflops": btf,
+                     "roofline": {**broof,
+                                  "algorithmic_bytes_per_call": bbytes, "algorithmic_flops_per_call": bflops,
+                                  "roofline_time_us": 1e6 * max(bt_hbm, bt_tc),
+                                  "kernel": "ssd_chunk_scan_bwd (three chunked scans + copies + finishing)"}}
+
     # ---------------- end to end through the public API with host buffers
     e2e = None
     if rank == 0 or world > 1:
@@ -618,8 +694,10 @@ def main():
                            "l2": "3 rotating input sets (x 67 MB each); inputs larger than L2 across steps",
                            "kernel_path": "tensor cores" if path == 0 else "cuda cores"},
                 "tflops": tflops, "gbs": gbs, "roofline": roofline, "decode": decode_line,
+                "backward": backward_line,
                 "cpu_baseline": cpu_baseline, "e2e": e2e, "workloads": workloads,
                 "gpu_launches": launches_per_prefill * args.steps + 2 * args.steps + rsteps,
+                "gpu_launches_backward": launches_per_bwd * bsteps,
                 "clocks": clk.summary()}
         print(json.dumps(line), flush=True)
     dist.finish(pg)

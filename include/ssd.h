@@ -207,6 +207,54 @@ ssd_status_t ssd_chunk_scan_fwd_varlen(const ssd_prefill_desc_t* desc,
                                        void* final_state, void* workspace, size_t workspace_bytes,
                                        void* stream);
 
+/*
+ * Backward pass of ssd_chunk_scan_fwd (training).  The pages only state that
+ * end-to-end training also needs it ("Mamba-3 : SSM optimise inference",
+ * opening paragraph); it is the gradient of
+ *     loss = sum_t <dy_t, y_t> + <dfinal_state, final_state>
+ * with respect to every input of the forward call for the same descriptor.
+ * The state adjoint G_t = C_t dy_t^T + exp(dt_{t+1} A) G_{t+1} is computed as
+ * the forward's chunked scan run backwards in time; G_t x_t and h_t dy_t as
+ * the same scan on transposed states; the decay gradients from the identity
+ * d loss / d (cumulative log-decay at u) = dy_u.(y_u - D x_u) - dt_u x_u.(B_u^T G_u)
+ * (+ <dfinal, h_{L-1}> at u = L-1), suffix-summed over the sequence.
+ *
+ *  inputs: exactly those of ssd_chunk_scan_fwd (same layouts and dtypes), plus
+ *  dy           [b][L][H][P]   io_dtype    required (NULL allowed if empty)
+ *  dfinal_state [b][H][N][P]   state_dtype nullable (= 0, final state not used)
+ *  outputs (every one written, none may overlap an input or another output):
+ *  dx           [b][L][H][P]   y_dtype     required
+ *  ddt_raw      [b][L][H]      y_dtype     required
+ *  dB, dC       [b][L][G][N]   y_dtype     required (summed over a group's heads)
+ *  dA           [H]            fp32        required (summed over batch and tokens)
+ *  ddt_bias, dD [H]            fp32        nullable (not written)
+ *  dinit_state  [b][H][N][P]   state_dtype nullable (not written)
+ *  workspace    >= ssd_chunk_scan_bwd_workspace_size bytes, 256-byte aligned,
+ *               clobbered
+ * The path (tensor-core or CUDA-core) follows ssd_chunk_scan_path for the
+ * adjoint scan; the transposed scans (headdim N in 64-column slices, dstate
+ * P) take the tensor-core path when bf16 inputs have headdim 64.
+ * Errors: as ssd_chunk_scan_fwd; the parameter gradients are plain fp32 sums
+ * (deterministic: no atomics).
+ */
+ssd_status_t ssd_chunk_scan_bwd(const ssd_prefill_desc_t* desc,
+                                const void* x, const void* dt_raw, const float* dt_bias,
+                                const float* A, const void* B, const void* C, const float* D,
+                                const void* init_state, const void* dy, const void* dfinal_state,
+                                void* dx, void* ddt_raw, float* ddt_bias, float* dA, void* dB, void* dC,
+                                float* dD, void* dinit_state, void* workspace, size_t workspace_bytes,
+                                void* stream);
+
+/* Workspace bytes ssd_chunk_scan_bwd needs for `desc`.  Pure host function. */
+ssd_status_t ssd_chunk_scan_bwd_workspace_size(const ssd_prefill_desc_t* desc, size_t* bytes);
+
+/*
+ * Number of kernels one ssd_chunk_scan_bwd call launches for `desc`
+ * (has_states: dfinal_state or init_state given).  Pure host function.
+ */
+ssd_status_t ssd_chunk_scan_bwd_launches(const ssd_prefill_desc_t* desc, int32_t has_states,
+                                         int32_t* launches);
+
 /* Size of the scratch array ssd_chunk_scan_fwd_noalloc uses (32 MiB per GPU). */
 #define SSD_NOALLOC_WORKSPACE_BYTES ((size_t)32 << 20)
 

@@ -242,6 +242,101 @@ ssd_status_t ssd_chunk_scan_fwd_varlen(const ssd_prefill_desc_t* d, const void* 
                    workspace_bytes, stream);
 }
 
+// the descriptor of the transposed scans of the backward (headdim and dstate
+// swapped, one group per head, N cut into column slices)
+static ssd_prefill_desc_t transposed_desc(const ssd_prefill_desc_t* d, int64_t pw) {
+    ssd_prefill_desc_t t = *d;
+    t.headdim = pw;
+    t.dstate = d->headdim;
+    t.ngroups = d->nheads;
+    t.y_dtype = SSD_F32;
+    t.state_dtype = SSD_F32;
+    return t;
+}
+
+static ssd_status_t check_backward_desc(const ssd_prefill_desc_t* d, BackwardLayout* lay) {
+    ssd_status_t st = check_prefill_desc(d);
+    if (st != SSD_OK) return st;
+    const BackwardLayout l = backward_layout(d->batch, d->seqlen, d->nheads, d->headdim, d->dstate, d->ngroups,
+                                             d->chunk, d->io_dtype == SSD_BF16);
+    const ssd_prefill_desc_t t = transposed_desc(d, l.pw);
+    st = check_prefill_desc(&t);
+    if (st != SSD_OK) return st;
+    if (d->batch * d->seqlen * d->nheads > ((int64_t)1 << 31) / 8) return SSD_ERR_UNSUPPORTED;
+    if (lay) *lay = l;
+    return SSD_OK;
+}
+
+ssd_status_t ssd_chunk_scan_bwd_workspace_size(const ssd_prefill_desc_t* desc, size_t* bytes) {
+    if (!bytes) return SSD_ERR_INVALID_ARG;
+    BackwardLayout l;
+    const ssd_status_t st = check_backward_desc(desc, &l);
+    if (st != SSD_OK) return st;
+    *bytes = l.total;
+    return SSD_OK;
+}
+
+ssd_status_t ssd_chunk_scan_bwd(const ssd_prefill_desc_t* d, const void* x, const void* dt_raw,
+                                const float* dt_bias, const float* A, const void* B, const void* C,
+                                const float* D, const void* init_state, const void* dy,
+                                const void* dfinal_state, void* dx, void* ddt_raw, float* ddt_bias, float* dA,
+                                void* dB, void* dC, float* dD, void* dinit_state, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+    BackwardLayout lay;
+    ssd_status_t st = check_backward_desc(d, &lay);
+    if (st != SSD_OK) return st;
+    const bool empty = d->batch == 0 || d->seqlen == 0;
+    if (!A || !dA) return SSD_ERR_INVALID_ARG;
+    if (!empty && (!x || !dt_raw || !B || !C || !dy || !dx || !ddt_raw || !dB || !dC)) return SSD_ERR_INVALID_ARG;
+    const void* ptrs[] = {x, dt_raw, dt_bias, A, B, C, D, init_state, dy, dfinal_state,
+                          dx, ddt_raw, ddt_bias, dA, dB, dC, dD, dinit_state};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return SSD_ERR_ALIGNMENT;
+    const size_t tok = (size_t)d->batch * d->seqlen;
+    const size_t ei = dsize(d->io_dtype), eg = dsize(d->y_dtype), es = dsize(d->state_dtype);
+    const size_t hp = (size_t)d->nheads * d->headdim, gn = (size_t)d->ngroups * d->dstate;
+    const size_t sb = (size_t)d->batch * d->nheads * d->dstate * d->headdim * es, hb = sizeof(float) * d->nheads;
+    // no output may overlap an input or another output
+    const struct { const void* p; size_t n; } in[] = {
+        {x, tok * hp * ei}, {dt_raw, tok * d->nheads * ei}, {dt_bias, hb}, {A, hb}, {B, tok * gn * ei},
+        {C, tok * gn * ei}, {D, hb}, {init_state, sb}, {dy, tok * hp * ei}, {dfinal_state, sb}};
+    const struct { const void* p; size_t n; } out[] = {
+        {dx, tok * hp * eg}, {ddt_raw, tok * d->nheads * eg}, {ddt_bias, hb}, {dA, hb}, {dB, tok * gn * eg},
+        {dC, tok * gn * eg}, {dD, hb}, {dinit_state, sb}};
+    for (size_t i = 0; i < sizeof(out) / sizeof(out[0]); ++i) {
+        for (const auto& r : in)
+            if (overlaps(out[i].p, out[i].n, r.p, r.n)) return SSD_ERR_INVALID_ARG;
+        for (size_t j = i + 1; j < sizeof(out) / sizeof(out[0]); ++j)
+            if (overlaps(out[i].p, out[i].n, out[j].p, out[j].n)) return SSD_ERR_INVALID_ARG;
+    }
+    if (!empty && (!workspace || workspace_bytes < lay.total)) return SSD_ERR_WORKSPACE;
+    if (workspace && ((uintptr_t)workspace & 255u)) return SSD_ERR_ALIGNMENT;
+    BackwardArgs a{};
+    a.batch = d->batch; a.L = d->seqlen; a.H = d->nheads; a.P = d->headdim; a.N = d->dstate;
+    a.G = d->ngroups; a.Q = d->chunk;
+    a.io_bf16 = d->io_dtype == SSD_BF16; a.grad_bf16 = d->y_dtype == SSD_BF16;
+    a.state_bf16 = d->state_dtype == SSD_BF16;
+    a.x = x; a.dt_raw = dt_raw; a.B = B; a.C = C; a.dy = dy;
+    a.dt_bias = dt_bias; a.A = A; a.D = D; a.init_state = init_state; a.dfinal = dfinal_state;
+    a.dx = dx; a.ddt_raw = ddt_raw; a.dB = dB; a.dC = dC; a.dinit = dinit_state;
+    a.ddt_bias = ddt_bias; a.dA = dA; a.dD = dD;
+    a.ws = (char*)workspace; a.lay = lay;
+    cudaError_t e = device_error_ptr(&a.dev_err);
+    if (e != cudaSuccess) return SSD_ERR_CUDA;
+    cudaStream_t s = (cudaStream_t)stream;
+    e = empty ? launch_backward_empty(a, s) : launch_backward(a, s);
+    return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
+}
+
+ssd_status_t ssd_chunk_scan_bwd_launches(const ssd_prefill_desc_t* desc, int32_t has_states, int32_t* launches) {
+    if (!launches) return SSD_ERR_INVALID_ARG;
+    BackwardLayout l;
+    const ssd_status_t st = check_backward_desc(desc, &l);
+    if (st != SSD_OK) return st;
+    *launches = (desc->batch == 0 || desc->seqlen == 0) ? 1 : backward_launches(l, has_states != 0);
+    return SSD_OK;
+}
+
 ssd_status_t ssd_state_update(const ssd_decode_desc_t* d, void* state, const void* x, const void* dt_raw,
                               const float* dt_bias, const float* A, const void* B, const void* C,
                               const float* D, void* y, void* stream) {

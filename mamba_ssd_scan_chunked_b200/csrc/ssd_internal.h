@@ -86,6 +86,46 @@ bool tc_path_supports(int64_t P, int64_t N, int64_t Q, bool io_bf16);
 int64_t tc_runs(int64_t BH, int64_t nchunks, int64_t N);
 cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s);
 
+// Backward pass of the prefill (ssd_backward.cu).  Workspace carve-up, all
+// offsets 256-byte aligned; "slice" strides separate the column slices of the
+// transposed scans.
+struct BackwardLayout {
+    int64_t nchunks, Lpad;
+    int64_t pw, nblk;              // column-slice width of the transposed scans, slices
+    bool tc_main, tc_t;            // tensor-core path for the adjoint scan / transposed scans
+    size_t off_dtf, off_acsf, off_dtr, off_acsr;   // fp32 [b*H][Lpad]: forward and reversed
+    size_t off_states, off_flags;                  // shared by the scans (run one after another)
+    size_t off_dyr, off_xr, off_Cr, off_Br;        // io dtype, reversed in time
+    size_t off_Cer, off_Be, slice_io;              // io dtype [slice][b][L][H][pw]
+    size_t off_dfin, off_G0;                       // fp32 [b][H][N][P]
+    size_t off_dfinT, off_h0T, off_hfT, slice_st;  // fp32 [slice][b][H][P][pw]
+    size_t off_y1, off_y2, off_y3, slice_y;        // fp32 scan outputs
+    size_t off_tok, off_part;                      // fp32 per-token and per-sequence scalars
+    size_t total;
+};
+
+BackwardLayout backward_layout(int64_t batch, int64_t L, int64_t H, int64_t P, int64_t N, int64_t G, int64_t Q,
+                               bool io_bf16);
+
+struct BackwardArgs {
+    int64_t batch, L, H, P, N, G, Q;
+    bool io_bf16, grad_bf16, state_bf16;
+    const void *x, *dt_raw, *B, *C, *dy;
+    const float *dt_bias, *A, *D;
+    const void *init_state, *dfinal;
+    void *dx, *ddt_raw, *dB, *dC, *dinit;
+    float *ddt_bias, *dA, *dD;
+    char* ws;
+    BackwardLayout lay;
+    unsigned* dev_err;
+};
+
+cudaError_t launch_backward(const BackwardArgs& a, cudaStream_t s);
+// seqlen 0 (or batch 0): zero parameter gradients, d init_state = dfinal
+cudaError_t launch_backward_empty(const BackwardArgs& a, cudaStream_t s);
+// kernels one ssd_chunk_scan_bwd call launches
+int backward_launches(const BackwardLayout& l, bool has_states);
+
 // fault-injection bits set by ssd_debug_inject (read at every launch)
 uint32_t debug_faults();
 

@@ -119,6 +119,16 @@ def draw_mimo_step(t: int, batch: int, nheads: int, headdim: int, dstate: int,
     return {k: to_storage(v, dtype) for k, v in (("x", x), ("dt_raw", dt_raw), ("B", Bm), ("C", Cm))}
 
 
+def draw_output_grads(batch: int, seqlen: int, nheads: int, headdim: int, dstate: int, seed: int,
+                      dtype: str, state_dtype: str) -> dict:
+    """Seeds of a backward pass: dy [b,L,H,P] (unit normal) and dfinal [b,H,N,P]
+    (normal, std 0.1, like the states)."""
+    rng = np.random.default_rng([seed, 5])
+    dy = rng.standard_normal((batch, seqlen, nheads, headdim))
+    dfinal = 0.1 * rng.standard_normal((batch, nheads, dstate, headdim))
+    return {"dy": to_storage(dy, dtype), "dfinal": to_storage(dfinal, state_dtype)}
+
+
 def prefill_inputs(batch: int, seqlen: int, nheads: int, headdim: int, dstate: int,
                    ngroups: int, seed: int, dtype: str, batches=None) -> dict:
     """Whole prefill input set (or the listed batch elements, in that order)."""

@@ -26,7 +26,8 @@ STATUS = {0: "SSD_OK", 1: "SSD_ERR_INVALID_ARG", 2: "SSD_ERR_UNSUPPORTED", 3: "S
 
 # every symbol include/ssd.h declares
 EXPORTS = ("ssd_version", "ssd_status_string", "ssd_chunk_scan_workspace_size", "ssd_chunk_scan_path",
-           "ssd_chunk_scan_fwd", "ssd_chunk_scan_fwd_varlen", "ssd_chunk_scan_fwd_noalloc", "ssd_state_update", "ssd_state_update_mimo",
+           "ssd_chunk_scan_fwd", "ssd_chunk_scan_fwd_varlen", "ssd_chunk_scan_fwd_noalloc",
+           "ssd_chunk_scan_bwd", "ssd_chunk_scan_bwd_workspace_size", "ssd_chunk_scan_bwd_launches", "ssd_state_update", "ssd_state_update_mimo",
            "ssd_replay_buffer_size",
            "ssd_replay_step", "ssd_get_device_error", "ssd_debug_inject")
 
@@ -96,6 +97,14 @@ def lib():
             L.ssd_chunk_scan_fwd_varlen.argtypes = [ctypes.POINTER(PrefillDesc)] + [_VP] * 11 + [_VP, ctypes.c_size_t, _VP]
             L.ssd_chunk_scan_fwd_noalloc.restype = ctypes.c_int
             L.ssd_chunk_scan_fwd_noalloc.argtypes = [ctypes.POINTER(PrefillDesc)] + [_VP] * 11
+            L.ssd_chunk_scan_bwd.restype = ctypes.c_int
+            L.ssd_chunk_scan_bwd.argtypes = [ctypes.POINTER(PrefillDesc)] + [_VP] * 19 + [ctypes.c_size_t, _VP]
+            L.ssd_chunk_scan_bwd_workspace_size.restype = ctypes.c_int
+            L.ssd_chunk_scan_bwd_workspace_size.argtypes = [ctypes.POINTER(PrefillDesc),
+                                                            ctypes.POINTER(ctypes.c_size_t)]
+            L.ssd_chunk_scan_bwd_launches.restype = ctypes.c_int
+            L.ssd_chunk_scan_bwd_launches.argtypes = [ctypes.POINTER(PrefillDesc), ctypes.c_int32,
+                                                      ctypes.POINTER(ctypes.c_int32)]
             L.ssd_state_update.restype = ctypes.c_int
             L.ssd_state_update.argtypes = [ctypes.POINTER(DecodeDesc)] + [_VP] * 10
             L.ssd_state_update_mimo.restype = ctypes.c_int
@@ -154,6 +163,31 @@ def ssd_chunk_scan_fwd_varlen(desc, x, dt_raw, dt_bias, A, B, C, D, init_state, 
                                            B or None, C or None, D or None, init_state or None, pad_left or None,
                                            y or None, final_state or None, workspace or None, int(workspace_bytes),
                                            stream or None)
+
+
+def ssd_chunk_scan_bwd(desc, x, dt_raw, dt_bias, A, B, C, D, init_state, dy, dfinal_state, dx, ddt_raw, ddt_bias, dA,
+                       dB, dC, dD, dinit_state, workspace, workspace_bytes, stream) -> int:
+    """Raw call of the backward pass; returns the status code (0 = enqueued)."""
+    ptrs = (x, dt_raw, dt_bias, A, B, C, D, init_state, dy, dfinal_state, dx, ddt_raw, ddt_bias, dA, dB, dC, dD,
+            dinit_state, workspace)
+    return lib().ssd_chunk_scan_bwd(ctypes.byref(desc), *(p or None for p in ptrs), int(workspace_bytes),
+                                     stream or None)
+
+
+def ssd_chunk_scan_bwd_workspace_size(desc: PrefillDesc) -> int:
+    n = ctypes.c_size_t(0)
+    st = lib().ssd_chunk_scan_bwd_workspace_size(ctypes.byref(desc), ctypes.byref(n))
+    if st:
+        raise SsdError(st, "ssd_chunk_scan_bwd_workspace_size")
+    return int(n.value)
+
+
+def ssd_chunk_scan_bwd_launches(desc: PrefillDesc, has_states: bool) -> int:
+    n = ctypes.c_int32(0)
+    st = lib().ssd_chunk_scan_bwd_launches(ctypes.byref(desc), int(bool(has_states)), ctypes.byref(n))
+    if st:
+        raise SsdError(st, "ssd_chunk_scan_bwd_launches")
+    return int(n.value)
 
 
 def ssd_chunk_scan_fwd_noalloc(desc, x, dt_raw, dt_bias, A, B, C, D, init_state, y, final_state, stream) -> int:
@@ -281,6 +315,47 @@ def chunk_scan_fwd(x, dt_raw, dt_bias, A, B, C, D, chunk, init_state=None, *, y=
     if st:
         raise SsdError(st, "ssd_chunk_scan_fwd")
     return y, final_state
+
+
+def chunk_scan_bwd(x, dt_raw, dt_bias, A, B, C, D, chunk, dy, init_state=None, dfinal_state=None, *,
+                   grad_dtype=None, state_dtype=None, want_dinit=True, workspace=None, stream=None):
+    """Backward pass of ``chunk_scan_fwd``: gradients of sum<dy, y> + <dfinal_state, final_state>.
+
+    Returns a dict of CUDA tensors: dx, ddt_raw, dB, dC (``grad_dtype``, default
+    x's dtype), dA, ddt_bias, dD (fp32 [H]) and dinit_state (state dtype, or
+    None when ``want_dinit`` is false).
+    """
+    import torch
+    if state_dtype is None:
+        src = init_state if init_state is not None else dfinal_state
+        state_dtype = src.dtype if src is not None else torch.float32
+    desc = prefill_desc(x, B, chunk, grad_dtype, state_dtype)
+    b, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    for t in (x, dt_raw, B, C, dt_bias, A, D, init_state, dy, dfinal_state):
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("libssd takes contiguous CUDA tensors")
+    gd, dev = _torch_dtype(desc.y_dtype), x.device
+    out = {"dx": torch.empty((b, L, H, P), dtype=gd, device=dev),
+           "ddt_raw": torch.empty((b, L, H), dtype=gd, device=dev),
+           "dB": torch.empty((b, L, G, N), dtype=gd, device=dev),
+           "dC": torch.empty((b, L, G, N), dtype=gd, device=dev),
+           "dA": torch.empty(H, dtype=torch.float32, device=dev),
+           "ddt_bias": torch.empty(H, dtype=torch.float32, device=dev),
+           "dD": torch.empty(H, dtype=torch.float32, device=dev),
+           "dinit_state": (torch.empty((b, H, N, P), dtype=_torch_dtype(desc.state_dtype), device=dev)
+                           if want_dinit else None)}
+    need = ssd_chunk_scan_bwd_workspace_size(desc)
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    st = ssd_chunk_scan_bwd(desc, _ptr(x), _ptr(dt_raw), _ptr(dt_bias), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                            _ptr(init_state), _ptr(dy), _ptr(dfinal_state), _ptr(out["dx"]), _ptr(out["ddt_raw"]),
+                            _ptr(out["ddt_bias"]), _ptr(out["dA"]), _ptr(out["dB"]), _ptr(out["dC"]),
+                            _ptr(out["dD"]), _ptr(out["dinit_state"]), _ptr(workspace), workspace.numel(),
+                            _stream(stream))
+    if st:
+        raise SsdError(st, "ssd_chunk_scan_bwd")
+    return out
 
 
 def state_update(state, x, dt_raw, dt_bias, A, B, C, D, *, y=None, y_dtype=None, stream=None):

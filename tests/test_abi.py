@@ -228,3 +228,51 @@ def test_varlen_host_validation_codes():
     assert call(FAKE + 0x30000002) == ALIGN                # int32 array: 4-byte aligned
     assert call(FAKE + 0x30000000) == WORKSPACE            # otherwise the checks of ssd_chunk_scan_fwd
     assert need > 0
+
+
+def bwd(d, **ptrs):
+    # distinct 16 MB windows per tensor (the test shapes stay far below that)
+    names = ("x", "dt_raw", "dt_bias", "A", "B", "C", "D", "init_state", "dy", "dfinal_state", "dx", "ddt_raw",
+             "ddt_bias", "dA", "dB", "dC", "dD", "dinit_state")
+    p = {k: FAKE + 0x1000000 * i for i, k in enumerate(names)}
+    for k in ("dt_bias", "D", "init_state", "dfinal_state", "ddt_bias", "dD", "dinit_state"):
+        p[k] = 0
+    p.update(workspace=0, workspace_bytes=0, stream=0)
+    p.update(ptrs)
+    return ssd.ssd_chunk_scan_bwd(d, *(p[k] for k in names), p["workspace"], p["workspace_bytes"], p["stream"])
+
+
+def test_backward_workspace_and_launches():
+    d = desc()
+    n = ssd.ssd_chunk_scan_bwd_workspace_size(d)
+    # at least the forward's workspace plus the reversed copies and fp32 scan outputs
+    assert n > ssd.ssd_chunk_scan_workspace_size(d)
+    b, L, H, P, N = 2, 512, 4, 64, 128
+    assert n >= 4 * b * L * H * P + 2 * 4 * b * L * H * N
+    # tensor-core path: dstate 128 in two 64-column slices for the transposed scans
+    assert ssd.ssd_chunk_scan_bwd_launches(d, False) == 1 + 2 * 2 + 2 + 2 * 2 + 4
+    assert ssd.ssd_chunk_scan_bwd_launches(d, True) == 1 + 1 + 2 * 2 + 2 + 2 * 2 + 4
+    # fp32 inputs: CUDA-core scans (three launches each), no slicing
+    assert ssd.ssd_chunk_scan_bwd_launches(desc(io_dtype=ssd.SSD_F32), False) == 1 + 4 + 1 + 3 + 4 + 4
+    with pytest.raises(ssd.SsdError) as e:
+        ssd.ssd_chunk_scan_bwd_workspace_size(desc(chunk=100))
+    assert e.value.status == UNSUPPORTED
+
+
+def test_backward_host_validation_codes():
+    d = desc()
+    need = ssd.ssd_chunk_scan_bwd_workspace_size(d)
+    ws = FAKE + 0x40000000
+    assert bwd(d, x=0) == INVALID
+    assert bwd(d, dy=0) == INVALID
+    assert bwd(d, dA=0) == INVALID
+    assert bwd(d, dB=0) == INVALID
+    assert bwd(d, dy=FAKE + 0x8000008) == ALIGN
+    assert bwd(d, dx=FAKE) == INVALID                            # dx aliases x
+    assert bwd(d, dC=FAKE + 0xa000000) == INVALID                # dC aliases dx
+    assert bwd(d, dD=FAKE + 0xd000000) == INVALID                # dD aliases dA
+    assert bwd(d) == WORKSPACE
+    assert bwd(d, workspace=ws, workspace_bytes=need - 1) == WORKSPACE
+    assert bwd(d, workspace=ws + 16, workspace_bytes=need) == ALIGN
+    assert bwd(desc(chunk=100)) == UNSUPPORTED
+    assert bwd(desc(nheads=4, ngroups=3)) == INVALID
