@@ -213,71 +213,64 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
-// dx and the per-token scalars x.dxu, C.(h dy) and x.dy; one warp per (b, t, h).
+// Everything local to one token row (b, t), one block per row: per head (a
+// warp each) dx and the scalars x.dxu, C.(h dy) and x.dy; per (group, n) dB and
+// dC summed over the group's heads.  The row's scan outputs (y1, y2, y3) are
+// read once from HBM (y3 twice, the second time from L1/L2).  The scalars go
+// out as tok[3][b*L][H].
 template <typename IoT, typename GT>
 __global__ void __launch_bounds__(256)
-bwd_token_kernel(const IoT* __restrict__ x, const IoT* __restrict__ dy, const IoT* __restrict__ C,
-                 const float* __restrict__ D, const float* __restrict__ dtf, const float* __restrict__ y1,
-                 const float* __restrict__ y3, GT* __restrict__ dx, float* __restrict__ tok, int64_t batch,
-                 int64_t L, int64_t Lpad, int H, int P, int N, int G, int pw, int64_t slice_y) {
-    const int64_t nwarps = batch * L * H;
-    const int lane = threadIdx.x & 31;
-    const int64_t BHL = batch * H * L;
-    for (int64_t wi = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5; wi < nwarps;
-         wi += ((int64_t)gridDim.x * blockDim.x) >> 5) {
-        const int h = (int)(wi % H);
-        const int64_t r = wi / H, b = r / L, t = r % L;
-        const int64_t bh = b * H + h;
-        const int64_t row = r * H + h;                          // (b, t, h)
-        const int64_t rrow = (b * L + (L - 1 - t)) * H + h;     // (b, L-1-t, h)
-        const float dt = dtf[bh * Lpad + t];
-        const float dsk = D ? D[h] : 0.f;
-        float xdxu = 0.f, xdy = 0.f, ydy = 0.f;
-        for (int p = lane; p < P; p += 32) {
-            const float xv = to_f32(x[row * P + p]), dyv = to_f32(dy[row * P + p]);
-            const float dxu = y1[rrow * P + p];
-            dx[row * P + p] = from_f32<GT>(dt * dxu + dsk * dyv);
-            xdxu += xv * dxu;
-            xdy += xv * dyv;
-        }
-        const int64_t crow = (r * G + h / (H / G)) * N;
-        for (int n = lane; n < N; n += 32) {
-            const int j = n / pw, k = n % pw;
-            ydy += to_f32(C[crow + n]) * y3[j * slice_y + row * pw + k];
-        }
-        xdxu = warp_sum(xdxu);
-        xdy = warp_sum(xdy);
-        ydy = warp_sum(ydy);
-        if (lane == 0) {
-            tok[bh * L + t] = xdxu;
-            tok[BHL + bh * L + t] = ydy;
-            tok[2 * BHL + bh * L + t] = xdy;
-        }
-    }
-}
-
-// dB and dC: one thread per (b, t, g, n), summing the group's heads.
-template <typename GT>
-__global__ void __launch_bounds__(256)
-bwd_dbdc_kernel(const float* __restrict__ dtf, const float* __restrict__ y2, const float* __restrict__ y3,
-                GT* __restrict__ dB, GT* __restrict__ dC, int64_t batch, int64_t L, int64_t Lpad, int H, int N,
-                int G, int pw, int64_t slice_y) {
-    const int64_t n_all = batch * L * G * N;
+bwd_row_kernel(const IoT* __restrict__ x, const IoT* __restrict__ dy, const IoT* __restrict__ C,
+               const float* __restrict__ D, const float* __restrict__ dtf, const float* __restrict__ y1,
+               const float* __restrict__ y2, const float* __restrict__ y3, GT* __restrict__ dx, GT* __restrict__ dB,
+               GT* __restrict__ dC, float* __restrict__ tok, int64_t batch, int64_t L, int64_t Lpad, int H, int P,
+               int N, int G, int pw, int64_t slice_y) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
     const int hpg = H / G;
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n_all; i += (int64_t)gridDim.x * blockDim.x) {
-        const int n = (int)(i % N);
-        const int g = (int)((i / N) % G);
-        const int64_t r = i / ((int64_t)N * G), b = r / L, t = r % L;
-        const int j = n / pw, k = n % pw;
-        const int64_t rr = b * L + (L - 1 - t);
-        float sb = 0.f, sc = 0.f;
-        for (int q = 0; q < hpg; ++q) {
-            const int h = g * hpg + q;
-            sb += dtf[(b * H + h) * Lpad + t] * y2[j * slice_y + (rr * H + h) * pw + k];
-            sc += y3[j * slice_y + (r * H + h) * pw + k];
+    const int64_t rows = batch * L;
+    for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+        const int64_t b = r / L, t = r - b * L;
+        const int64_t rr = b * L + (L - 1 - t);              // the row's index in reversed time
+        for (int h = warp; h < H; h += nwarps) {
+            const float dt = dtf[(b * H + h) * Lpad + t];
+            const float dsk = D ? D[h] : 0.f;
+            const int64_t row = r * H + h, rrow = rr * H + h;
+            float xdxu = 0.f, xdy = 0.f, ydy = 0.f;
+            for (int p = lane; p < P; p += 32) {
+                const float xv = to_f32(x[row * P + p]), dyv = to_f32(dy[row * P + p]);
+                const float dxu = y1[rrow * P + p];
+                dx[row * P + p] = from_f32<GT>(dt * dxu + dsk * dyv);
+                xdxu += xv * dxu;
+                xdy += xv * dyv;
+            }
+            const IoT* Cg = C + (r * G + h / hpg) * N;
+            for (int n = lane; n < N; n += 32) {
+                const int j = n / pw;
+                ydy += to_f32(Cg[n]) * y3[j * slice_y + row * pw + (n - j * pw)];
+            }
+            xdxu = warp_sum(xdxu);
+            xdy = warp_sum(xdy);
+            ydy = warp_sum(ydy);
+            if (lane == 0) {
+                tok[row] = xdxu;
+                tok[rows * H + row] = ydy;
+                tok[2 * rows * H + row] = xdy;
+            }
         }
-        dB[i] = from_f32<GT>(sb);
-        dC[i] = from_f32<GT>(sc);
+        for (int i = threadIdx.x; i < G * N; i += blockDim.x) {
+            const int g = i / N, n = i - g * N, j = n / pw, k = n - j * pw;
+            const float* y2r = y2 + j * slice_y + (rr * H + g * hpg) * pw + k;
+            const float* y3r = y3 + j * slice_y + (r * H + g * hpg) * pw + k;
+            const float* dtr = dtf + (b * H + g * hpg) * Lpad + t;
+            float sb = 0.f, sc = 0.f;
+#pragma unroll 8
+            for (int q = 0; q < hpg; ++q) {
+                sb += dtr[q * Lpad] * y2r[q * pw];
+                sc += y3r[q * pw];
+            }
+            dB[r * G * N + i] = from_f32<GT>(sb);
+            dC[r * G * N + i] = from_f32<GT>(sc);
+        }
     }
 }
 
@@ -327,10 +320,11 @@ bwd_decay_kernel(const IoT* __restrict__ dt_raw, const float* __restrict__ dt_bi
         const int64_t t = end - tid;          // thread tid walks the tile backwards
         float dcum = 0.f, xdxu = 0.f, dt = 0.f, xdy = 0.f;
         if (t >= 0) {
-            xdxu = tok[bh * L + t];
-            xdy = tok[2 * BHL + bh * L + t];
+            const int64_t row = (b * L + t) * H + h;
+            xdxu = tok[row];
+            xdy = tok[2 * BHL + row];
             dt = dtf[bh * Lpad + t];
-            dcum = tok[BHL + bh * L + t] - dt * xdxu + (t == L - 1 ? hfdot : 0.f);
+            dcum = tok[BHL + row] - dt * xdxu + (t == L - 1 ? hfdot : 0.f);
         }
         // inclusive prefix over tid = suffix over t within the tile
         float v = dcum;
@@ -499,12 +493,9 @@ static cudaError_t backward_t(const BackwardArgs& a, cudaStream_t s) {
         if (e != cudaSuccess) return e;
     }
     const float* dtf = (const float*)(ws + l.off_dtf);
-    bwd_token_kernel<IoT, GT><<<grid_for(a.batch * a.L * H, 8), 256, 0, s>>>(
-        (const IoT*)a.x, (const IoT*)a.dy, (const IoT*)a.C, a.D, dtf, y1, y3, (GT*)a.dx, tok, a.batch, a.L, l.Lpad, H,
-        P, N, G, pw, slice_y);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    bwd_dbdc_kernel<GT><<<grid_for(a.batch * a.L * G * N, 256), 256, 0, s>>>(
-        dtf, y2, y3, (GT*)a.dB, (GT*)a.dC, a.batch, a.L, l.Lpad, H, N, G, pw, slice_y);
+    bwd_row_kernel<IoT, GT><<<grid_for(a.batch * a.L, 1), 256, 0, s>>>(
+        (const IoT*)a.x, (const IoT*)a.dy, (const IoT*)a.C, a.D, dtf, y1, y2, y3, (GT*)a.dx, (GT*)a.dB, (GT*)a.dC,
+        tok, a.batch, a.L, l.Lpad, H, P, N, G, pw, slice_y);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     bwd_decay_kernel<IoT, GT, StateT><<<(unsigned)BH, DTB, 0, s>>>(
         (const IoT*)a.dt_raw, a.dt_bias, a.A, dtf, tok, has_dfin ? dfin : nullptr, hfT, G0, (GT*)a.ddt_raw,
@@ -561,9 +552,9 @@ int backward_launches(const BackwardLayout& l, bool has_states) {
     // a scan is one launch on the tensor-core path, three on the CUDA-core one;
     // prep tokens (+ prep states); F: dt_cumsum, nblk scans, nblk - 1 flag
     // clears; R1: decay kernel and scan; R2: nblk clears and nblk scans; then
-    // four finishing kernels
+    // three finishing kernels (rows, decay gradient, parameters)
     const int st = l.tc_t ? 1 : 3, sm = l.tc_main ? 1 : 3;
-    return 1 + (has_states ? 1 : 0) + (int)(l.nblk * (st + 1)) + 1 + sm + (int)(l.nblk * (st + 1)) + 4;
+    return 1 + (has_states ? 1 : 0) + (int)(l.nblk * (st + 1)) + 1 + sm + (int)(l.nblk * (st + 1)) + 3;
 }
 
 }  // namespace ssd

@@ -250,10 +250,10 @@ def test_backward_workspace_and_launches():
     b, L, H, P, N = 2, 512, 4, 64, 128
     assert n >= 4 * b * L * H * P + 2 * 4 * b * L * H * N
     # tensor-core path: dstate 128 in two 64-column slices for the transposed scans
-    assert ssd.ssd_chunk_scan_bwd_launches(d, False) == 1 + 2 * 2 + 2 + 2 * 2 + 4
-    assert ssd.ssd_chunk_scan_bwd_launches(d, True) == 1 + 1 + 2 * 2 + 2 + 2 * 2 + 4
+    assert ssd.ssd_chunk_scan_bwd_launches(d, False) == 1 + 2 * 2 + 2 + 2 * 2 + 3
+    assert ssd.ssd_chunk_scan_bwd_launches(d, True) == 1 + 1 + 2 * 2 + 2 + 2 * 2 + 3
     # fp32 inputs: CUDA-core scans (three launches each), no slicing
-    assert ssd.ssd_chunk_scan_bwd_launches(desc(io_dtype=ssd.SSD_F32), False) == 1 + 4 + 1 + 3 + 4 + 4
+    assert ssd.ssd_chunk_scan_bwd_launches(desc(io_dtype=ssd.SSD_F32), False) == 1 + 4 + 1 + 3 + 4 + 3
     with pytest.raises(ssd.SsdError) as e:
         ssd.ssd_chunk_scan_bwd_workspace_size(desc(chunk=100))
     assert e.value.status == UNSUPPORTED
