@@ -274,6 +274,151 @@ bwd_row_kernel(const IoT* __restrict__ x, const IoT* __restrict__ dy, const IoT*
     }
 }
 
+// The same per-row work in 16-byte vectors for power-of-two headdim and dstate
+// (P/4 and N/4 powers of two, P <= 128): all threads of the block load a whole
+// row at once instead of a warp walking its heads one by one.  Per-head sums
+// are shuffle reductions over segments of P/4 (or min(32, N/4)) lanes; dB and
+// dC are summed over RSPLIT ranges of the group's heads, the partial sums
+// meeting in shared memory in a fixed order (bitwise deterministic).
+constexpr int ROW_THREADS = 256;
+
+template <typename T> struct Io4;
+template <> struct Io4<float> {
+    __device__ __forceinline__ static void load(const float* p, float v[4]) {
+        const float4 a = *reinterpret_cast<const float4*>(p);
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    }
+    __device__ __forceinline__ static void store(float* p, const float v[4]) {
+        *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+    }
+};
+template <> struct Io4<bf16> {
+    __device__ __forceinline__ static void load(const bf16* p, float v[4]) {
+        const uint2 a = *reinterpret_cast<const uint2*>(p);
+        v[0] = __uint_as_float(a.x << 16); v[1] = __uint_as_float(a.x & 0xffff0000u);
+        v[2] = __uint_as_float(a.y << 16); v[3] = __uint_as_float(a.y & 0xffff0000u);
+    }
+    __device__ __forceinline__ static void store(bf16* p, const float v[4]) {
+        __nv_bfloat162 lo = __floats2bfloat162_rn(v[0], v[1]), hi = __floats2bfloat162_rn(v[2], v[3]);
+        *reinterpret_cast<uint2*>(p) = make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
+    }
+};
+
+__device__ __forceinline__ float seg_sum(float v, int width) {
+    for (int o = width >> 1; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+template <typename IoT, typename GT>
+__global__ void __launch_bounds__(ROW_THREADS)
+bwd_row_vec_kernel(const IoT* __restrict__ x, const IoT* __restrict__ dy, const IoT* __restrict__ C,
+                   const float* __restrict__ D, const float* __restrict__ dtf, const float* __restrict__ y1,
+                   const float* __restrict__ y2, const float* __restrict__ y3, GT* __restrict__ dx,
+                   GT* __restrict__ dB, GT* __restrict__ dC, float* __restrict__ tok, int64_t batch, int64_t L,
+                   int64_t Lpad, int H, int P, int N, int G, int pw, int64_t slice_y) {
+    __shared__ __align__(16) float part[2][ROW_THREADS * 4];   // dB, dC partial sums [split][column]
+    const int tid = threadIdx.x;
+    const int hpg = H / G;
+    const int64_t rows = batch * L;
+    const int SP = P >> 2;                                   // lanes per head, dx phase
+    const int SN = (N >> 2) < 32 ? (N >> 2) : 32;            // lanes per head, C.(h dy) phase
+    const int VN = (N >> 2) / SN;                            // 4-vectors per lane there
+    const int ncol4 = (G * N) >> 2;                          // 4-vectors of a dB / dC row
+    int rsplit = ROW_THREADS / ncol4;                        // head ranges summed apart
+    if (rsplit < 1) rsplit = 1;
+    if (rsplit > hpg) rsplit = hpg;
+    for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+        const int64_t b = r / L, t = r - b * L;
+        const int64_t rr = b * L + (L - 1 - t);
+        // dx, x.dxu, x.dy
+        for (int h0 = 0; h0 < H; h0 += ROW_THREADS / SP) {
+            const int h = h0 + tid / SP, p4 = tid % SP;
+            float xdxu = 0.f, xdy = 0.f;
+            if (h < H) {
+                const int64_t row = r * H + h;
+                const float dt = dtf[(b * H + h) * Lpad + t];
+                const float dsk = D ? D[h] : 0.f;
+                float xv[4], dyv[4], u[4], o[4];
+                Io4<IoT>::load(x + row * P + 4 * p4, xv);
+                Io4<IoT>::load(dy + row * P + 4 * p4, dyv);
+                Io4<float>::load(y1 + (rr * H + h) * P + 4 * p4, u);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    o[e] = dt * u[e] + dsk * dyv[e];
+                    xdxu += xv[e] * u[e];
+                    xdy += xv[e] * dyv[e];
+                }
+                Io4<GT>::store(dx + row * P + 4 * p4, o);
+            }
+            xdxu = seg_sum(xdxu, SP);
+            xdy = seg_sum(xdy, SP);
+            if (h < H && p4 == 0) {
+                tok[r * H + h] = xdxu;
+                tok[2 * rows * H + r * H + h] = xdy;
+            }
+        }
+        // C . (h dy)
+        for (int h0 = 0; h0 < H; h0 += ROW_THREADS / SN) {
+            const int h = h0 + tid / SN, l4 = tid % SN;
+            float ydy = 0.f;
+            if (h < H) {
+                const IoT* Cg = C + (r * G + h / hpg) * N;
+                for (int i = 0; i < VN; ++i) {
+                    const int n = 4 * (l4 + SN * i), j = n / pw;
+                    float cv[4], yv[4];
+                    Io4<IoT>::load(Cg + n, cv);
+                    Io4<float>::load(y3 + j * slice_y + (r * H + h) * pw + (n - j * pw), yv);
+                    ydy += cv[0] * yv[0] + cv[1] * yv[1] + cv[2] * yv[2] + cv[3] * yv[3];
+                }
+            }
+            ydy = seg_sum(ydy, SN);
+            if (h < H && l4 == 0) tok[rows * H + r * H + h] = ydy;
+        }
+        // dB, dC: column vector c4 of the (g, n) row, head range sp
+        for (int i = tid; i < ncol4 * rsplit; i += ROW_THREADS) {
+            const int c4 = i % ncol4, sp = i / ncol4;
+            const int g = (4 * c4) / N, n = 4 * c4 - g * N, j = n / pw, k = n - j * pw;
+            const int q0 = (sp * hpg) / rsplit, q1 = ((sp + 1) * hpg) / rsplit;
+            float sb[4] = {0.f, 0.f, 0.f, 0.f}, sc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+            for (int q = q0; q < q1; ++q) {
+                const int h = g * hpg + q;
+                const float dt = dtf[(b * H + h) * Lpad + t];
+                float v2[4], v3[4];
+                Io4<float>::load(y2 + j * slice_y + (rr * H + h) * pw + k, v2);
+                Io4<float>::load(y3 + j * slice_y + (r * H + h) * pw + k, v3);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    sb[e] += dt * v2[e];
+                    sc[e] += v3[e];
+                }
+            }
+            if (rsplit == 1) {
+                Io4<GT>::store(dB + r * G * N + 4 * c4, sb);
+                Io4<GT>::store(dC + r * G * N + 4 * c4, sc);
+            } else {
+                Io4<float>::store(&part[0][4 * i], sb);
+                Io4<float>::store(&part[1][4 * i], sc);
+            }
+        }
+        if (rsplit > 1) {
+            __syncthreads();
+            for (int c = tid; c < 4 * ncol4; c += ROW_THREADS) {
+                float vb = 0.f, vc = 0.f;
+                for (int sp = 0; sp < rsplit; ++sp) {
+                    vb += part[0][sp * 4 * ncol4 + c];
+                    vc += part[1][sp * 4 * ncol4 + c];
+                }
+                dB[r * G * N + c] = from_f32<GT>(vb);
+                dC[r * G * N + c] = from_f32<GT>(vc);
+            }
+            __syncthreads();
+        }
+    }
+}
+
+static bool pow2(int v) { return v > 0 && (v & (v - 1)) == 0; }
+
 // One block per (b, h): <dfinal, h_final>, d init_state, then the suffix sum
 // of the log-decay gradient over the sequence (tiles of 256 tokens from the
 // end), d dt_raw, and this sequence's shares of dA, d dt_bias and dD.
@@ -493,9 +638,14 @@ static cudaError_t backward_t(const BackwardArgs& a, cudaStream_t s) {
         if (e != cudaSuccess) return e;
     }
     const float* dtf = (const float*)(ws + l.off_dtf);
-    bwd_row_kernel<IoT, GT><<<grid_for(a.batch * a.L, 1), 256, 0, s>>>(
-        (const IoT*)a.x, (const IoT*)a.dy, (const IoT*)a.C, a.D, dtf, y1, y2, y3, (GT*)a.dx, (GT*)a.dB, (GT*)a.dC,
-        tok, a.batch, a.L, l.Lpad, H, P, N, G, pw, slice_y);
+    if (pow2(P / 4) && P <= 128 && pow2(N / 4))
+        bwd_row_vec_kernel<IoT, GT><<<grid_for(a.batch * a.L, 1), ROW_THREADS, 0, s>>>(
+            (const IoT*)a.x, (const IoT*)a.dy, (const IoT*)a.C, a.D, dtf, y1, y2, y3, (GT*)a.dx, (GT*)a.dB,
+            (GT*)a.dC, tok, a.batch, a.L, l.Lpad, H, P, N, G, pw, slice_y);
+    else
+        bwd_row_kernel<IoT, GT><<<grid_for(a.batch * a.L, 1), 256, 0, s>>>(
+            (const IoT*)a.x, (const IoT*)a.dy, (const IoT*)a.C, a.D, dtf, y1, y2, y3, (GT*)a.dx, (GT*)a.dB,
+            (GT*)a.dC, tok, a.batch, a.L, l.Lpad, H, P, N, G, pw, slice_y);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     bwd_decay_kernel<IoT, GT, StateT><<<(unsigned)BH, DTB, 0, s>>>(
         (const IoT*)a.dt_raw, a.dt_bias, a.A, dtf, tok, has_dfin ? dfin : nullptr, hfT, G0, (GT*)a.ddt_raw,
