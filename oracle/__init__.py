@@ -24,6 +24,10 @@ C file's header:
   say that end-to-end training also needs the backward pass: "Mamba-3 : SSM
   optimise inference", opening paragraph; the gradients follow from the
   forward definition).
+- ``mamba3_recurrent`` -- the Mamba-3 recurrence: exponential-trapezoidal
+  input and a rotational (complex) state ("Mamba3", sections "New
+  discretisation scheme" and on complex-valued SSMs; "Mamba-3 : SSM optimise
+  inference", "Etats complexes via RoPE").
 - ``decode_step`` -- one token of the recurrent mode, in place on the state
   (same page, table "Evaluation criteria": O(1) recurrent step at inference).
 
@@ -80,6 +84,8 @@ def _load():
             lib.oracle_ssd_decode_step_mimo.restype = ctypes.c_int
             lib.oracle_ssd_backward.argtypes = sig6 + [_D] * 18 + [ctypes.c_int]
             lib.oracle_ssd_backward.restype = ctypes.c_int
+            lib.oracle_ssd_mamba3_recurrent.argtypes = sig6 + [_D] * 12 + [ctypes.c_int]
+            lib.oracle_ssd_mamba3_recurrent.restype = ctypes.c_int
             lib.oracle_round_bf16.argtypes = [ctypes.c_double]
             lib.oracle_round_bf16.restype = ctypes.c_double
             lib.oracle_round_bf16_array.argtypes = [_D, _D, _I64]
@@ -220,3 +226,24 @@ def backward(x, dt_raw, dt_bias, A, B, C, D, init_state, dy, dfinal=None, nthrea
     if rc != 0:
         raise ValueError("oracle_ssd_backward: invalid arguments")
     return out
+
+
+def mamba3_recurrent(x, dt_raw, dt_bias, A, B, C, D, lam=None, theta=None, init_state=None, nthreads=0):
+    """Mamba-3 sequential recurrence.  Shapes as ``recurrent``; lam [b,L,H] (the
+    trapezoid's mix, None = 1), theta [b,L,G,N/2] (rotation angle per step and
+    state pair, None = 0).  Returns (y, final_state) in float64."""
+    x, dt_raw, dt_bias, A, B, C, D, lam, theta, init_state = map(
+        _f64, (x, dt_raw, dt_bias, A, B, C, D, lam, theta, init_state))
+    b, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    assert dt_raw.shape == (b, L, H) and B.shape == C.shape == (b, L, G, N)
+    assert lam is None or lam.shape == (b, L, H)
+    assert theta is None or theta.shape == (b, L, G, N // 2)
+    y = np.empty((b, L, H, P))
+    fs = np.empty((b, H, N, P))
+    rc = _load().oracle_ssd_mamba3_recurrent(b, L, H, P, N, G, _ptr(x), _ptr(dt_raw), _ptr(dt_bias), _ptr(A),
+                                             _ptr(B), _ptr(C), _ptr(D), _ptr(lam), _ptr(theta), _ptr(init_state),
+                                             _ptr(y), _ptr(fs), int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle_ssd_mamba3_recurrent: invalid arguments")
+    return y, fs

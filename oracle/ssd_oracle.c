@@ -552,3 +552,91 @@ int oracle_ssd_backward(int64_t batch, int64_t seqlen, int64_t nheads, int64_t h
     free(part);
     return 0;
 }
+
+/* ------------------------------------------------------------------------ */
+/* 7. Mamba-3 recurrence: exponential-trapezoidal input, rotational state.   */
+/* ------------------------------------------------------------------------ */
+/* "Mamba3" (Telegram post), section "New discretisation scheme": the integral
+ * over a step is approximated from both ends of the interval with a learned
+ * mixing coefficient, which makes the recurrence an implicit convolution on
+ * the input.  Reading: over the step t-1 -> t of length dt_t the input term is
+ *     dt_t [ (1 - lam_t) exp(dt_t A) B_{t-1} x_{t-1}^T + lam_t B_t x_t^T ],
+ * the left end transported over the interval like the state (lam = 1 is
+ * Mamba-2's Euler input; there is no input before the first token).
+ * Same post, section on complex-valued SSMs, and "Mamba-3 : SSM optimise
+ * inference", section "Etats complexes via RoPE": the complex transition is a
+ * scaling and a rotation.  Reading: state rows (2k, 2k+1) form the pair k of
+ * a complex state component and the transition of step t rotates every pair
+ * by theta[t][g][k] (the same angle for every head of group g) and scales by
+ * exp(dt_t A):
+ *     h_t = exp(dt_t A) R(theta_t) (h_{t-1} + (1 - lam_t) dt_t B_{t-1} x_{t-1}^T)
+ *           + lam_t dt_t B_t x_t^T,
+ *     y_t = C_t^T h_t + D x_t,
+ * R rotating (h[2k], h[2k+1]) by the angle counter-clockwise.  lam [b][L][H]
+ * and theta [b][L][G][N/2] may each be NULL (lam = 1, theta = 0). */
+int oracle_ssd_mamba3_recurrent(int64_t batch, int64_t seqlen, int64_t nheads, int64_t headdim,
+                                int64_t dstate, int64_t ngroups, const double* x, const double* dt_raw,
+                                const double* dt_bias, const double* A, const double* B, const double* C,
+                                const double* D, const double* lam, const double* theta,
+                                const double* init_state, double* y, double* final_state, int nthreads) {
+    if (check_dims(batch, seqlen, nheads, headdim, dstate, ngroups)) return -1;
+    if (!x || !dt_raw || !A || !B || !C) return -1;
+    if (theta && dstate % 2 != 0) return -1;
+    const int64_t H = nheads, P = headdim, N = dstate, G = ngroups, L = seqlen;
+    const int64_t heads_per_group = H / G;
+    const int nt = set_threads(nthreads);
+    int64_t pair;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nt)
+    for (pair = 0; pair < batch * H; ++pair) {
+        const int64_t b = pair / H, h = pair % H, g = h / heads_per_group;
+        double* st = (double*)malloc(sizeof(double) * N * P);
+        if (init_state) memcpy(st, init_state + (b * H + h) * N * P, sizeof(double) * N * P);
+        else memset(st, 0, sizeof(double) * N * P);
+        const double bias = dt_bias ? dt_bias[h] : 0.0;
+        const double d_skip = D ? D[h] : 0.0;
+        for (int64_t t = 0; t < L; ++t) {
+            const double dt = sp(dt_raw[(b * L + t) * H + h] + bias);
+            const double decay = exp(dt * A[h]);
+            const double mix = lam ? lam[(b * L + t) * H + h] : 1.0;
+            const double* xt = x + ((b * L + t) * H + h) * P;
+            const double* Bt = B + ((b * L + t) * G + g) * N;
+            const double* Ct = C + ((b * L + t) * G + g) * N;
+            /* left end of the interval: the previous token's input, weighted 1 - lam_t */
+            if (t > 0) {
+                const double* xp = x + ((b * L + t - 1) * H + h) * P;
+                const double* Bp = B + ((b * L + t - 1) * G + g) * N;
+                for (int64_t n = 0; n < N; ++n)
+                    for (int64_t p = 0; p < P; ++p) st[n * P + p] += (1.0 - mix) * dt * Bp[n] * xp[p];
+            }
+            /* transition: rotate each pair of rows, then scale */
+            if (theta) {
+                for (int64_t k = 0; k < N / 2; ++k) {
+                    const double ang = theta[((b * L + t) * G + g) * (N / 2) + k];
+                    const double c = cos(ang), s = sin(ang);
+                    double* r0 = st + (2 * k) * P;
+                    double* r1 = st + (2 * k + 1) * P;
+                    for (int64_t p = 0; p < P; ++p) {
+                        const double u = r0[p], v = r1[p];
+                        r0[p] = c * u - s * v;
+                        r1[p] = s * u + c * v;
+                    }
+                }
+            }
+            for (int64_t i = 0; i < N * P; ++i) st[i] *= decay;
+            /* right end: the current token's input, weighted lam_t */
+            for (int64_t n = 0; n < N; ++n)
+                for (int64_t p = 0; p < P; ++p) st[n * P + p] += mix * dt * Bt[n] * xt[p];
+            if (y) {
+                double* yt = y + ((b * L + t) * H + h) * P;
+                for (int64_t p = 0; p < P; ++p) {
+                    double acc = 0.0;
+                    for (int64_t n = 0; n < N; ++n) acc += Ct[n] * st[n * P + p];
+                    yt[p] = acc + d_skip * xt[p];
+                }
+            }
+        }
+        if (final_state) memcpy(final_state + (b * H + h) * N * P, st, sizeof(double) * N * P);
+        free(st);
+    }
+    return 0;
+}

@@ -2,7 +2,8 @@
 
 Each case plants one slip in a temporary copy of the oracle's C source (on the
 CPU, never on a GPU), rebuilds it, and reruns the pins of
-``test_oracle_pins.py`` and ``test_oracle_bwd_pins.py`` against the mutant: at least one pin must fail.
+``test_oracle_pins.py``, ``test_oracle_bwd_pins.py`` and
+``test_oracle_mamba3_pins.py`` against the mutant: at least one pin must fail.
 """
 import importlib.util
 import os
@@ -11,6 +12,7 @@ import sys
 import pytest
 
 import tests.test_oracle_bwd_pins as bwd_pins
+import tests.test_oracle_mamba3_pins as m3_pins
 import tests.test_oracle_pins as pins
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -50,6 +52,11 @@ MUTATIONS = [
     ("bwd_dB_missing_dt", "dBt[n] = dt * gx;", "dBt[n] = gx;"),
     ("bwd_dC_reads_previous_state", "hy += hc[n * P + p] * dyt[p];", "hy += hp[n * P + p] * dyt[p];"),
     ("bwd_decay_path_of_dt_dropped", "const double ddt = gbx + Ah * dlogdecay;", "const double ddt = gbx;"),
+    ("m3_left_end_reads_current_token", "+= (1.0 - mix) * dt * Bp[n] * xp[p];", "+= (1.0 - mix) * dt * Bt[n] * xt[p];"),
+    ("m3_left_end_weight_swapped", "+= (1.0 - mix) * dt * Bp[n] * xp[p];", "+= mix * dt * Bp[n] * xp[p];"),
+    ("m3_rotation_not_orthogonal", "r0[p] = c * u - s * v;", "r0[p] = c * u + s * v;"),
+    ("m3_angle_indexed_by_head", "const double ang = theta[((b * L + t) * G + g) * (N / 2) + k];",
+     "const double ang = theta[((b * L + t) * G + h % G) * (N / 2) + k];"),
     ("bwd_wrong_segment_checkpoint", "memcpy(seg, ck + k * NP, sizeof(double) * NP);",
      "memcpy(seg, ck + (k > 0 ? k - 1 : 0) * NP, sizeof(double) * NP);"),
 ]
@@ -72,6 +79,13 @@ PIN_TESTS = [
     lambda: bwd_pins.test_backward_elementwise_finite_differences(2),
     lambda: bwd_pins.test_backward_directional_finite_differences(True, True),
     bwd_pins.test_backward_single_token_closed_form,
+    lambda: m3_pins.test_mamba3_reduces_to_mamba2(True),
+    m3_pins.test_trapezoid_impulse_response,
+    m3_pins.test_trapezoid_step_response_closed_form,
+    lambda: m3_pins.test_rotation_impulse_response(0.4),
+    m3_pins.test_common_rotation_of_B_and_C_is_invisible,
+    m3_pins.test_first_angle_acts_on_the_state_only,
+    m3_pins.test_angles_follow_the_group_map,
 ]
 
 
@@ -96,6 +110,7 @@ def test_pins_catch_mutation(tmp_path, monkeypatch, name, old, new):
     mutant = _load_mutant(tmp_path, name, old, new)
     monkeypatch.setattr(pins, "oracle", mutant)
     monkeypatch.setattr(bwd_pins, "oracle", mutant)
+    monkeypatch.setattr(m3_pins, "oracle", mutant)
     caught = 0
     for t in PIN_TESTS:
         try:
