@@ -12,7 +12,9 @@ with the same steps replayed from a checkpoint and a 16-token buffer
 (ssd_replay_step) under "decode"."replay" and rank-4 MIMO steps
 (ssd_state_update_mimo) on the same state under "decode"."mimo", and the
 backward pass of the prefill (ssd_chunk_scan_bwd, fp32 gradients, with a
-final-state gradient) under "backward".
+final-state gradient) under "backward", and the Mamba-3 prefill
+(ssd_chunk_scan_fwd_mamba3: trapezoidal input and rotational state) of the same
+layer under "mamba3".
 
 Timing: W untimed warm-up steps, then exactly K steps between a barrier +
 cudaDeviceSynchronize on both sides, CUDA events on the launching stream, max
@@ -589,6 +591,42 @@ def main():
                                   "roofline_time_us": 1e6 * max(bt_hbm, bt_tc),
                                   "kernel": "ssd_chunk_scan_bwd (three chunked scans + copies + finishing)"}}
 
+    # ---------------- Mamba-3 prefill (trapezoidal input + rotational state) on the same layer
+    ex = I.draw_mamba3_extras(s.batch, s.seqlen, s.nheads, s.ngroups, s.dstate, s.seed + rank)
+    m3_lam, m3_theta = to_dev(ex["lam"]), to_dev(ex["theta"])
+    m3ws = torch.empty(ssd.ssd_chunk_scan_mamba3_workspace_size(desc), dtype=torch.uint8, device=dev)
+    launches_per_m3 = ssd.ssd_chunk_scan_mamba3_launches(desc, True, True, True)
+
+    def mamba3(k):
+        d = sets[k % NSETS]
+        st = ssd.ssd_chunk_scan_fwd_mamba3(desc, d["x"].data_ptr(), d["dt_raw"].data_ptr(), d["dt_bias"].data_ptr(),
+                                           d["A"].data_ptr(), d["B"].data_ptr(), d["C"].data_ptr(),
+                                           d["D"].data_ptr(), m3_lam.data_ptr(), m3_theta.data_ptr(), 0,
+                                           y.data_ptr(), fs.data_ptr(), m3ws.data_ptr(), m3ws.numel(),
+                                           stream.cuda_stream)
+        if st:
+            raise ssd.SsdError(st, "ssd_chunk_scan_fwd_mamba3")
+
+    m3steps = max(3, min(args.steps, 10))
+    for k in range(args.warmup):
+        mamba3(k)
+    dist.barrier(pg)
+    torch.cuda.synchronize()
+    ev[0].record(stream)
+    for k in range(m3steps):
+        mamba3(k)
+    ev[1].record(stream)
+    torch.cuda.synchronize()
+    dist.barrier(pg)
+    m3ms = dist.max_over_ranks(pg, ev[0].elapsed_time(ev[1]) / m3steps)
+    st_err, detail = ssd.ssd_get_device_error(stream.cuda_stream)
+    if st_err:
+        raise RuntimeError(f"device error word {detail:#x} after the timed Mamba-3 prefill")
+    mamba3_line = {"tokens_per_s": tokens_rank * world / (m3ms * 1e-3), "ms_per_step": m3ms, "steps": m3steps,
+                   "launches_per_step": launches_per_m3, "vs_mamba2_prefill_time": m3ms / ms,
+                   "inputs": "lam ~ U[0,1] per (token, head), theta ~ U[-0.5,0.5] rad per (token, group, pair)",
+                   "path": "B, C turned by the cumulative angle in bf16 hi/lo pairs, three tensor-core scans"}
+
     # ---------------- end to end through the public API with host buffers
     e2e = None
     if rank == 0 or world > 1:
@@ -694,10 +732,11 @@ def main():
                            "l2": "3 rotating input sets (x 67 MB each); inputs larger than L2 across steps",
                            "kernel_path": "tensor cores" if path == 0 else "cuda cores"},
                 "tflops": tflops, "gbs": gbs, "roofline": roofline, "decode": decode_line,
-                "backward": backward_line,
+                "backward": backward_line, "mamba3": mamba3_line,
                 "cpu_baseline": cpu_baseline, "e2e": e2e, "workloads": workloads,
                 "gpu_launches": launches_per_prefill * args.steps + 2 * args.steps + rsteps,
                 "gpu_launches_backward": launches_per_bwd * bsteps,
+                "gpu_launches_mamba3": launches_per_m3 * m3steps,
                 "clocks": clk.summary()}
         print(json.dumps(line), flush=True)
     dist.finish(pg)

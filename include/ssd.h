@@ -255,6 +255,43 @@ ssd_status_t ssd_chunk_scan_bwd_workspace_size(const ssd_prefill_desc_t* desc, s
 ssd_status_t ssd_chunk_scan_bwd_launches(const ssd_prefill_desc_t* desc, int32_t has_states,
                                          int32_t* launches);
 
+/*
+ * Mamba-3 prefill: the chunked scan of the Mamba-3 recurrence, with an
+ * exponential-trapezoidal input ("Mamba3", section "New discretisation
+ * scheme": both ends of each step's interval, mixed by a learned coefficient)
+ * and a rotational (complex) state ("Mamba3", section on complex-valued SSMs;
+ * "Mamba-3 : SSM optimise inference", "Etats complexes via RoPE").  Per batch
+ * b and head h, with the state rows (2k, 2k+1) forming the rotating pair k:
+ *   h_t = exp(dt_t A) R(theta_t) (h_{t-1} + (1 - lam_t) dt_t B_{t-1} x_{t-1}^T)
+ *         + lam_t dt_t B_t x_t^T
+ *   y_t = C_t^T h_t + D x_t
+ * R(theta) turns (h[2k], h[2k+1]) counter-clockwise by theta[t][g][k]; there
+ * is no input before the first token.  Computed, as the pages suggest, by
+ * turning B and C with the cumulative angle and running the real chunked scan
+ * with the trapezoid's weights, then a per-token diagonal correction.
+ *
+ *  arguments as ssd_chunk_scan_fwd, plus
+ *  lam    [b][L][H]      fp32  nullable (= 1: Euler input, Mamba-2's)
+ *  theta  [b][L][G][N/2] fp32  nullable (= 0: real state)
+ *  With both NULL this is ssd_chunk_scan_fwd.
+ *  workspace >= ssd_chunk_scan_mamba3_workspace_size bytes, 256-byte aligned.
+ * Errors: as ssd_chunk_scan_fwd.
+ */
+ssd_status_t ssd_chunk_scan_fwd_mamba3(const ssd_prefill_desc_t* desc,
+                                       const void* x, const void* dt_raw, const float* dt_bias,
+                                       const float* A, const void* B, const void* C, const float* D,
+                                       const float* lam, const float* theta, const void* init_state,
+                                       void* y, void* final_state, void* workspace, size_t workspace_bytes,
+                                       void* stream);
+
+/* Workspace bytes ssd_chunk_scan_fwd_mamba3 needs for `desc`.  Pure host function. */
+ssd_status_t ssd_chunk_scan_mamba3_workspace_size(const ssd_prefill_desc_t* desc, size_t* bytes);
+
+/* Kernels one ssd_chunk_scan_fwd_mamba3 call launches (flags: lam given,
+ * theta given, final_state given).  Pure host function. */
+ssd_status_t ssd_chunk_scan_mamba3_launches(const ssd_prefill_desc_t* desc, int32_t has_lam, int32_t has_theta,
+                                            int32_t has_final_state, int32_t* launches);
+
 /* Size of the scratch array ssd_chunk_scan_fwd_noalloc uses (32 MiB per GPU). */
 #define SSD_NOALLOC_WORKSPACE_BYTES ((size_t)32 << 20)
 

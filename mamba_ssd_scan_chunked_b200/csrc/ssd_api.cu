@@ -242,6 +242,89 @@ ssd_status_t ssd_chunk_scan_fwd_varlen(const ssd_prefill_desc_t* d, const void* 
                    workspace_bytes, stream);
 }
 
+static Mamba3Layout m3_layout(const ssd_prefill_desc_t* d) {
+    return mamba3_layout(d->batch, d->seqlen, d->nheads, d->headdim, d->dstate, d->ngroups, d->chunk,
+                         d->io_dtype == SSD_BF16, prefill_path(d) == 0);
+}
+
+static ssd_status_t check_mamba3_desc(const ssd_prefill_desc_t* d) {
+    const ssd_status_t st = check_prefill_desc(d);
+    if (st != SSD_OK) return st;
+    // the rotation kernel's grid: (b, g, chunk, 4 pairs)
+    const int64_t nchunks = (d->seqlen + d->chunk - 1) / d->chunk;
+    if (d->batch * d->ngroups * nchunks * ((d->dstate / 2 + 3) / 4) >= ((int64_t)1 << 31)) return SSD_ERR_UNSUPPORTED;
+    return SSD_OK;
+}
+
+ssd_status_t ssd_chunk_scan_mamba3_workspace_size(const ssd_prefill_desc_t* desc, size_t* bytes) {
+    if (!bytes) return SSD_ERR_INVALID_ARG;
+    const ssd_status_t st = check_mamba3_desc(desc);
+    if (st != SSD_OK) return st;
+    *bytes = m3_layout(desc).total;
+    return SSD_OK;
+}
+
+ssd_status_t ssd_chunk_scan_fwd_mamba3(const ssd_prefill_desc_t* d, const void* x, const void* dt_raw,
+                                       const float* dt_bias, const float* A, const void* B, const void* C,
+                                       const float* D, const float* lam, const float* theta, const void* init_state,
+                                       void* y, void* final_state, void* workspace, size_t workspace_bytes,
+                                       void* stream) {
+    ssd_status_t st = check_mamba3_desc(d);
+    if (st != SSD_OK) return st;
+    if ((lam && !aligned16(lam)) || (theta && !aligned16(theta))) return SSD_ERR_ALIGNMENT;
+    const size_t tok = (size_t)d->batch * d->seqlen;
+    const size_t y_bytes = tok * d->nheads * d->headdim * dsize(d->y_dtype);
+    const size_t s_bytes = (size_t)d->batch * d->nheads * d->dstate * d->headdim * dsize(d->state_dtype);
+    if (overlaps(y, y_bytes, lam, tok * d->nheads * sizeof(float)) ||
+        overlaps(y, y_bytes, theta, tok * d->ngroups * (d->dstate / 2) * sizeof(float)) ||
+        overlaps(final_state, s_bytes, lam, tok * d->nheads * sizeof(float)) ||
+        overlaps(final_state, s_bytes, theta, tok * d->ngroups * (d->dstate / 2) * sizeof(float)))
+        return SSD_ERR_INVALID_ARG;
+    // empty problems, argument checks and the plain recurrence's cases: the
+    // forward call (with seqlen 0 the final state is the initial one either way)
+    if (d->batch == 0 || d->seqlen == 0 || (!lam && !theta))
+        return prefill(d, x, dt_raw, dt_bias, A, B, C, D, init_state, nullptr, y, final_state, workspace,
+                       workspace_bytes, stream);
+    if (!A || !x || !dt_raw || !B || !C || !y) return SSD_ERR_INVALID_ARG;
+    const void* ptrs[] = {x, dt_raw, dt_bias, A, B, C, D, init_state, y, final_state};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return SSD_ERR_ALIGNMENT;
+    const size_t x_bytes = tok * d->nheads * d->headdim * dsize(d->io_dtype);
+    const size_t bc_bytes = tok * d->ngroups * d->dstate * dsize(d->io_dtype);
+    if (overlaps(y, y_bytes, x, x_bytes) || overlaps(y, y_bytes, B, bc_bytes) || overlaps(y, y_bytes, C, bc_bytes) ||
+        overlaps(final_state, s_bytes, y, y_bytes) || overlaps(final_state, s_bytes, x, x_bytes))
+        return SSD_ERR_INVALID_ARG;
+    const Mamba3Layout lay = m3_layout(d);
+    if (!workspace || workspace_bytes < lay.total) return SSD_ERR_WORKSPACE;
+    if ((uintptr_t)workspace & 255u) return SSD_ERR_ALIGNMENT;
+    Mamba3Args a{};
+    a.batch = d->batch; a.L = d->seqlen; a.H = d->nheads; a.P = d->headdim; a.N = d->dstate;
+    a.G = d->ngroups; a.Q = d->chunk;
+    a.io_bf16 = d->io_dtype == SSD_BF16; a.y_bf16 = d->y_dtype == SSD_BF16;
+    a.state_bf16 = d->state_dtype == SSD_BF16; a.tc = prefill_path(d) == 0;
+    a.x = x; a.dt_raw = dt_raw; a.B = B; a.C = C; a.dt_bias = dt_bias; a.A = A; a.D = D;
+    a.lam = lam; a.theta = theta; a.init_state = init_state; a.y = y; a.final_state = final_state;
+    a.ws = (char*)workspace; a.lay = lay;
+    cudaError_t e = device_error_ptr(&a.dev_err);
+    if (e != cudaSuccess) return SSD_ERR_CUDA;
+    e = launch_mamba3(a, (cudaStream_t)stream);
+    return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
+}
+
+ssd_status_t ssd_chunk_scan_mamba3_launches(const ssd_prefill_desc_t* desc, int32_t has_lam, int32_t has_theta,
+                                            int32_t has_final_state, int32_t* launches) {
+    if (!launches) return SSD_ERR_INVALID_ARG;
+    const ssd_status_t st = check_mamba3_desc(desc);
+    if (st != SSD_OK) return st;
+    const bool tc = prefill_path(desc) == 0;
+    if (desc->batch == 0) *launches = 0;
+    else if (desc->seqlen == 0) *launches = has_final_state ? 1 : 0;
+    else if (!has_lam && !has_theta) *launches = 1 + (tc ? 1 : 3);
+    else *launches = mamba3_launches(tc, desc->io_dtype == SSD_BF16, has_lam != 0, has_theta != 0,
+                                     has_final_state != 0);
+    return SSD_OK;
+}
+
 // the descriptor of the transposed scans of the backward (headdim and dstate
 // swapped, one group per head, N cut into column slices)
 static ssd_prefill_desc_t transposed_desc(const ssd_prefill_desc_t* d, int64_t pw) {

@@ -126,6 +126,39 @@ cudaError_t launch_backward_empty(const BackwardArgs& a, cudaStream_t s);
 // kernels one ssd_chunk_scan_bwd call launches
 int backward_launches(const BackwardLayout& l, bool has_states);
 
+// Mamba-3 prefill (ssd_mamba3.cu): the forward's scan workspace plus the
+// rotated operands, angle sums, the diagonal correction and staging buffers.
+struct Mamba3Layout {
+    PrefillLayout scan;
+    size_t off_corr;               // fp32 [b*H][Lpad]
+    size_t off_Bt, off_Ct;         // io dtype [b][L][G][N], rotated by -Theta_t (bf16: the hi part)
+    size_t off_Btl, off_Ctl;       // bf16 inputs: the lo part of the same
+    size_t off_csum;               // fp64 [b][G][nchunks][N/2] angle sums per chunk
+    size_t off_thL;                // fp64 [b][G][N/2] angle at the last token
+    size_t off_y32[3];             // fp32 [b][L][H][P] scan outputs before the combination
+    size_t off_fsr;                // state dtype [b][H][N][P] rotated-frame final state (scan 1)
+    size_t off_fsr2;               // fp32 [b][H][N][P] the same of the B_lo scan
+    size_t total;
+};
+
+Mamba3Layout mamba3_layout(int64_t batch, int64_t L, int64_t H, int64_t P, int64_t N, int64_t G, int64_t Q,
+                           bool io_bf16, bool tc);
+
+struct Mamba3Args {
+    int64_t batch, L, H, P, N, G, Q;
+    bool io_bf16, y_bf16, state_bf16, tc;
+    const void *x, *dt_raw, *B, *C;
+    const float *dt_bias, *A, *D, *lam, *theta;
+    const void* init_state;
+    void *y, *final_state;
+    char* ws;
+    Mamba3Layout lay;
+    unsigned* dev_err;
+};
+
+cudaError_t launch_mamba3(const Mamba3Args& a, cudaStream_t s);
+int mamba3_launches(bool tc, bool io_bf16, bool has_lam, bool has_theta, bool has_final);
+
 // fault-injection bits set by ssd_debug_inject (read at every launch)
 uint32_t debug_faults();
 

@@ -129,6 +129,16 @@ def draw_output_grads(batch: int, seqlen: int, nheads: int, headdim: int, dstate
     return {"dy": to_storage(dy, dtype), "dfinal": to_storage(dfinal, state_dtype)}
 
 
+def draw_mamba3_extras(batch: int, seqlen: int, nheads: int, ngroups: int, dstate: int, seed: int) -> dict:
+    """Mamba-3 prefill inputs beyond Mamba-2's: the trapezoid's mix lam [b,L,H]
+    ~ U[0, 1] and the rotation angle per step and state pair theta [b,L,G,N/2]
+    ~ U[-0.5, 0.5] rad, both fp32."""
+    rng = np.random.default_rng([seed, 6])
+    lam = rng.uniform(0.0, 1.0, (batch, seqlen, nheads))
+    theta = rng.uniform(-0.5, 0.5, (batch, seqlen, ngroups, dstate // 2))
+    return {"lam": to_storage(lam, F32), "theta": to_storage(theta, F32)}
+
+
 def prefill_inputs(batch: int, seqlen: int, nheads: int, headdim: int, dstate: int,
                    ngroups: int, seed: int, dtype: str, batches=None) -> dict:
     """Whole prefill input set (or the listed batch elements, in that order)."""

@@ -27,7 +27,8 @@ STATUS = {0: "SSD_OK", 1: "SSD_ERR_INVALID_ARG", 2: "SSD_ERR_UNSUPPORTED", 3: "S
 # every symbol include/ssd.h declares
 EXPORTS = ("ssd_version", "ssd_status_string", "ssd_chunk_scan_workspace_size", "ssd_chunk_scan_path",
            "ssd_chunk_scan_fwd", "ssd_chunk_scan_fwd_varlen", "ssd_chunk_scan_fwd_noalloc",
-           "ssd_chunk_scan_bwd", "ssd_chunk_scan_bwd_workspace_size", "ssd_chunk_scan_bwd_launches", "ssd_state_update", "ssd_state_update_mimo",
+           "ssd_chunk_scan_bwd", "ssd_chunk_scan_bwd_workspace_size", "ssd_chunk_scan_bwd_launches",
+           "ssd_chunk_scan_fwd_mamba3", "ssd_chunk_scan_mamba3_workspace_size", "ssd_chunk_scan_mamba3_launches", "ssd_state_update", "ssd_state_update_mimo",
            "ssd_replay_buffer_size",
            "ssd_replay_step", "ssd_get_device_error", "ssd_debug_inject")
 
@@ -105,6 +106,14 @@ def lib():
             L.ssd_chunk_scan_bwd_launches.restype = ctypes.c_int
             L.ssd_chunk_scan_bwd_launches.argtypes = [ctypes.POINTER(PrefillDesc), ctypes.c_int32,
                                                       ctypes.POINTER(ctypes.c_int32)]
+            L.ssd_chunk_scan_fwd_mamba3.restype = ctypes.c_int
+            L.ssd_chunk_scan_fwd_mamba3.argtypes = [ctypes.POINTER(PrefillDesc)] + [_VP] * 13 + [ctypes.c_size_t, _VP]
+            L.ssd_chunk_scan_mamba3_workspace_size.restype = ctypes.c_int
+            L.ssd_chunk_scan_mamba3_workspace_size.argtypes = [ctypes.POINTER(PrefillDesc),
+                                                               ctypes.POINTER(ctypes.c_size_t)]
+            L.ssd_chunk_scan_mamba3_launches.restype = ctypes.c_int
+            L.ssd_chunk_scan_mamba3_launches.argtypes = [ctypes.POINTER(PrefillDesc)] + [ctypes.c_int32] * 3 + \
+                [ctypes.POINTER(ctypes.c_int32)]
             L.ssd_state_update.restype = ctypes.c_int
             L.ssd_state_update.argtypes = [ctypes.POINTER(DecodeDesc)] + [_VP] * 10
             L.ssd_state_update_mimo.restype = ctypes.c_int
@@ -172,6 +181,31 @@ def ssd_chunk_scan_bwd(desc, x, dt_raw, dt_bias, A, B, C, D, init_state, dy, dfi
             dinit_state, workspace)
     return lib().ssd_chunk_scan_bwd(ctypes.byref(desc), *(p or None for p in ptrs), int(workspace_bytes),
                                      stream or None)
+
+
+def ssd_chunk_scan_fwd_mamba3(desc, x, dt_raw, dt_bias, A, B, C, D, lam, theta, init_state, y, final_state,
+                              workspace, workspace_bytes, stream) -> int:
+    """Raw call of the Mamba-3 prefill; returns the status code (0 = enqueued)."""
+    ptrs = (x, dt_raw, dt_bias, A, B, C, D, lam, theta, init_state, y, final_state, workspace)
+    return lib().ssd_chunk_scan_fwd_mamba3(ctypes.byref(desc), *(p or None for p in ptrs), int(workspace_bytes),
+                                            stream or None)
+
+
+def ssd_chunk_scan_mamba3_workspace_size(desc: PrefillDesc) -> int:
+    n = ctypes.c_size_t(0)
+    st = lib().ssd_chunk_scan_mamba3_workspace_size(ctypes.byref(desc), ctypes.byref(n))
+    if st:
+        raise SsdError(st, "ssd_chunk_scan_mamba3_workspace_size")
+    return int(n.value)
+
+
+def ssd_chunk_scan_mamba3_launches(desc: PrefillDesc, has_lam: bool, has_theta: bool, has_final: bool) -> int:
+    n = ctypes.c_int32(0)
+    st = lib().ssd_chunk_scan_mamba3_launches(ctypes.byref(desc), int(bool(has_lam)), int(bool(has_theta)),
+                                              int(bool(has_final)), ctypes.byref(n))
+    if st:
+        raise SsdError(st, "ssd_chunk_scan_mamba3_launches")
+    return int(n.value)
 
 
 def ssd_chunk_scan_bwd_workspace_size(desc: PrefillDesc) -> int:
@@ -314,6 +348,36 @@ def chunk_scan_fwd(x, dt_raw, dt_bias, A, B, C, D, chunk, init_state=None, *, y=
                                        _ptr(workspace), workspace.numel(), _stream(stream))
     if st:
         raise SsdError(st, "ssd_chunk_scan_fwd")
+    return y, final_state
+
+
+def chunk_scan_fwd_mamba3(x, dt_raw, dt_bias, A, B, C, D, chunk, lam=None, theta=None, init_state=None, *,
+                          y_dtype=None, state_dtype=None, want_final_state=True, workspace=None, stream=None):
+    """Mamba-3 prefill (trapezoidal input mix ``lam`` [b,L,H] fp32, rotation
+    angles ``theta`` [b,L,G,N/2] fp32; either may be None).  Returns (y, final_state)."""
+    import torch
+    if state_dtype is None:
+        state_dtype = init_state.dtype if init_state is not None else torch.float32
+    desc = prefill_desc(x, B, chunk, y_dtype, state_dtype)
+    b, L, H, P = x.shape
+    N = B.shape[3]
+    for t in (x, dt_raw, B, C, dt_bias, A, D, lam, theta, init_state):
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("libssd takes contiguous CUDA tensors")
+    for t in (lam, theta):
+        if t is not None and t.dtype != torch.float32:
+            raise ValueError("lam and theta are fp32")
+    y = torch.empty((b, L, H, P), dtype=_torch_dtype(desc.y_dtype), device=x.device)
+    final_state = (torch.empty((b, H, N, P), dtype=_torch_dtype(desc.state_dtype), device=x.device)
+                   if want_final_state else None)
+    need = ssd_chunk_scan_mamba3_workspace_size(desc)
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
+    st = ssd_chunk_scan_fwd_mamba3(desc, _ptr(x), _ptr(dt_raw), _ptr(dt_bias), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                                   _ptr(lam), _ptr(theta), _ptr(init_state), _ptr(y), _ptr(final_state),
+                                   _ptr(workspace), workspace.numel(), _stream(stream))
+    if st:
+        raise SsdError(st, "ssd_chunk_scan_fwd_mamba3")
     return y, final_state
 
 

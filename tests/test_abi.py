@@ -29,7 +29,7 @@ def built():
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(ssd_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(ssd_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_header_matches_binding_exports():
@@ -276,3 +276,36 @@ def test_backward_host_validation_codes():
     assert bwd(d, workspace=ws + 16, workspace_bytes=need) == ALIGN
     assert bwd(desc(chunk=100)) == UNSUPPORTED
     assert bwd(desc(nheads=4, ngroups=3)) == INVALID
+
+
+def test_mamba3_workspace_launches_and_validation():
+    d = desc()
+    n = ssd.ssd_chunk_scan_mamba3_workspace_size(d)
+    assert n > ssd.ssd_chunk_scan_workspace_size(d)
+    # bf16, tensor-core path: angle sums + rotation, weights, three scans of the
+    # hi/lo operands (two after a flag clear), combination, final-state rotation
+    assert ssd.ssd_chunk_scan_mamba3_launches(d, True, True, True) == 2 + 1 + 1 + 2 * 2 + 1 + 1
+    assert ssd.ssd_chunk_scan_mamba3_launches(d, True, False, True) == 3
+    assert ssd.ssd_chunk_scan_mamba3_launches(d, False, True, False) == 2 + 1 + 1 + 2 * 2 + 1
+    assert ssd.ssd_chunk_scan_mamba3_launches(d, False, False, True) == 2       # the plain forward
+    assert ssd.ssd_chunk_scan_mamba3_launches(desc(io_dtype=ssd.SSD_F32), True, True, True) == 8
+
+    def call(dd, **kw):
+        p = dict(x=FAKE, dt_raw=FAKE + 0x1000000, dt_bias=0, A=FAKE + 0x2000000, B=FAKE + 0x3000000,
+                 C=FAKE + 0x4000000, D=0, lam=FAKE + 0x5000000, theta=FAKE + 0x6000000, init_state=0,
+                 y=FAKE + 0x10000000, final_state=0, workspace=0, workspace_bytes=0, stream=0)
+        p.update(kw)
+        return ssd.ssd_chunk_scan_fwd_mamba3(dd, p["x"], p["dt_raw"], p["dt_bias"], p["A"], p["B"], p["C"], p["D"],
+                                             p["lam"], p["theta"], p["init_state"], p["y"], p["final_state"],
+                                             p["workspace"], p["workspace_bytes"], p["stream"])
+
+    assert call(d) == WORKSPACE
+    assert call(d, lam=FAKE + 0x5000004) == ALIGN
+    assert call(d, theta=FAKE + 0x6000008) == ALIGN
+    assert call(d, y=FAKE + 0x5000000) == INVALID                # y overlaps lam
+    assert call(d, x=0) == INVALID
+    assert call(d, y=FAKE) == INVALID                            # y aliases x
+    assert call(d, workspace=FAKE + 0x40000000, workspace_bytes=n - 1) == WORKSPACE
+    assert call(d, workspace=FAKE + 0x40000010, workspace_bytes=n) == ALIGN
+    assert call(desc(chunk=100)) == UNSUPPORTED
+    assert call(desc(batch=0)) == OK                             # nothing to do, nothing launched

@@ -1,0 +1,80 @@
+"""GPU parity of ssd_chunk_scan_fwd_mamba3 (exponential-trapezoidal input,
+rotational state) against the float64 oracle's Mamba-3 recurrence, element by
+element on the same seeded inputs: y and the final state, max|err| / rms(oracle)
+within the bound of the input dtype.  Tensor-core shapes with ragged tails and
+every dstate, the CUDA-core fp32 path, sequences cut into runs, bf16 outputs
+and states, each of the two extensions alone, and the plain case (both absent)
+equal to ssd_chunk_scan_fwd bit for bit."""
+import numpy as np
+import pytest
+
+import oracle
+from mamba_ssd_scan_chunked_b200 import inputs as I
+from mamba_ssd_scan_chunked_b200 import ssd
+from tests.gpu_util import (TOL_BF16, TOL_F32, bf16_excess_metric, bf16_state_metric, metric, to_dev, to_host64,
+                            torch)
+
+pytestmark = pytest.mark.gpu
+
+
+def run_case(b, L, H, P, N, G, Q, io, use_lam, use_theta, with_init, seed=31, y_dtype="f32", state=I.F32):
+    t = torch()
+    inp = I.prefill_inputs(b, L, H, P, N, G, seed, io)
+    ex = I.draw_mamba3_extras(b, L, H, G, N, seed)
+    if with_init:
+        inp["init_state"] = np.stack([I.draw_decode_state(i, H, P, N, seed=seed + 1, dtype=state) for i in range(b)])
+    dev = {k: to_dev(v) for k, v in inp.items()}
+    lam = to_dev(ex["lam"]) if use_lam else None
+    theta = to_dev(ex["theta"]) if use_theta else None
+    yd = t.float32 if y_dtype == "f32" else t.bfloat16
+    y, fs = ssd.chunk_scan_fwd_mamba3(dev["x"], dev["dt_raw"], dev["dt_bias"], dev["A"], dev["B"], dev["C"], dev["D"],
+                                      Q, lam, theta, dev.get("init_state"), y_dtype=yd,
+                                      state_dtype=t.bfloat16 if state == I.BF16 else t.float32)
+    t.cuda.synchronize()
+    assert ssd.ssd_get_device_error(0)[0] == 0
+    f = {k: I.to_f64(v) for k, v in inp.items()}
+    y_ref, fs_ref = oracle.mamba3_recurrent(f["x"], f["dt_raw"], f["dt_bias"], f["A"], f["B"], f["C"], f["D"],
+                                            lam=I.to_f64(ex["lam"]) if use_lam else None,
+                                            theta=I.to_f64(ex["theta"]) if use_theta else None,
+                                            init_state=f.get("init_state"))
+    return to_host64(y), to_host64(fs), y_ref, fs_ref
+
+
+@pytest.mark.parametrize("b,L,H,P,N,G,Q,io,use_lam,use_theta,with_init", [
+    (2, 300, 4, 64, 128, 2, 128, I.BF16, True, True, True),     # tensor cores, ragged tail, both extensions
+    (2, 600, 2, 64, 64, 1, 256, I.BF16, True, False, False),    # trapezoid only, dstate 64
+    (1, 260, 2, 64, 256, 2, 128, I.BF16, False, True, True),    # rotation only, dstate 256
+    (2, 200, 3, 32, 16, 3, 64, I.F32, True, True, True),        # CUDA-core path, fp32
+    (1, 130, 2, 48, 24, 1, 32, I.F32, True, True, False),       # CUDA-core path, odd sizes
+])
+def test_mamba3_matches_oracle(b, L, H, P, N, G, Q, io, use_lam, use_theta, with_init):
+    y, fs, y_ref, fs_ref = run_case(b, L, H, P, N, G, Q, io, use_lam, use_theta, with_init)
+    tol = TOL_BF16 if io == I.BF16 else TOL_F32
+    assert metric(y, y_ref) <= tol
+    assert metric(fs, fs_ref) <= tol
+
+
+def test_mamba3_long_sequences_cut_into_runs():
+    """Two heads of 4096 tokens: the scans run in several runs with hand-offs,
+    and the cumulative angles grow far past 2 pi."""
+    y, fs, y_ref, fs_ref = run_case(1, 4096, 2, 64, 128, 1, 256, I.BF16, True, True, True)
+    assert metric(y, y_ref) <= TOL_BF16
+    assert metric(fs, fs_ref) <= TOL_BF16
+
+
+def test_mamba3_bf16_outputs_and_state():
+    y, fs, y_ref, fs_ref = run_case(2, 256, 4, 64, 128, 1, 128, I.BF16, True, True, True, y_dtype="bf16",
+                                    state=I.BF16)
+    assert bf16_excess_metric(y, y_ref) <= TOL_BF16
+    assert bf16_state_metric(fs, fs_ref) <= TOL_BF16
+
+
+def test_mamba3_without_extensions_is_the_forward_call():
+    t = torch()
+    inp = I.prefill_inputs(2, 300, 4, 64, 128, 2, 5, I.BF16)
+    dev = {k: to_dev(v) for k, v in inp.items()}
+    args = (dev["x"], dev["dt_raw"], dev["dt_bias"], dev["A"], dev["B"], dev["C"], dev["D"], 128)
+    y1, f1 = ssd.chunk_scan_fwd_mamba3(*args, y_dtype=t.float32)
+    y2, f2 = ssd.chunk_scan_fwd(*args, y_dtype=t.float32)
+    t.cuda.synchronize()
+    assert t.equal(y1, y2) and t.equal(f1, f2)
