@@ -234,6 +234,8 @@ ssd_status_t ssd_chunk_scan_fwd_varlen(const ssd_prefill_desc_t* desc,
  * The path (tensor-core or CUDA-core) follows ssd_chunk_scan_path for the
  * adjoint scan; the transposed scans (headdim N in 64-column slices, dstate
  * P) take the tensor-core path when bf16 inputs have headdim 64.
+ * Empty problems (batch 0 or seqlen 0) launch one kernel: dA, ddt_bias and dD
+ * are zeroed and dinit_state = dfinal_state (or zero); no workspace is needed.
  * Errors: as ssd_chunk_scan_fwd; the parameter gradients are plain fp32 sums
  * (deterministic: no atomics).
  */
