@@ -309,3 +309,19 @@ def test_mamba3_workspace_launches_and_validation():
     assert call(d, workspace=FAKE + 0x40000010, workspace_bytes=n) == ALIGN
     assert call(desc(chunk=100)) == UNSUPPORTED
     assert call(desc(batch=0)) == OK                             # nothing to do, nothing launched
+
+
+def test_binding_rejects_host_or_strided_tensors_before_any_cuda_call():
+    """The wrappers check devices, contiguity and the fp32 extras on the host."""
+    import torch
+    x = torch.zeros(1, 4, 2, 8, dtype=torch.bfloat16)
+    dt = torch.zeros(1, 4, 2, dtype=torch.bfloat16)
+    B = torch.zeros(1, 4, 1, 8, dtype=torch.bfloat16)
+    A = torch.zeros(2)
+    for call in (lambda: ssd.chunk_scan_fwd(x, dt, None, A, B, B, None, 16),
+                 lambda: ssd.chunk_scan_bwd(x, dt, None, A, B, B, None, 16, x),
+                 lambda: ssd.chunk_scan_fwd_mamba3(x, dt, None, A, B, B, None, 16),
+                 lambda: ssd.chunk_scan_fwd_mamba3(x, dt, None, A, B, B, None, 16,
+                                                   lam=torch.zeros(1, 4, 2).transpose(1, 2))):
+        with pytest.raises(ValueError):
+            call()
