@@ -28,6 +28,10 @@ C file's header:
   input and a rotational (complex) state ("Mamba3", sections "New
   discretisation scheme" and on complex-valued SSMs; "Mamba-3 : SSM optimise
   inference", "Etats complexes via RoPE").
+- ``mamba3_decode_step`` -- one token of the Mamba-3 recurrence (the state
+  plus the previous token's B and x, which the trapezoid's left end reads);
+  ``mimo_recurrent`` -- a sequence of MIMO tokens.  Both are references for
+  kernels not yet built, pinned like the rest.
 - ``decode_step`` -- one token of the recurrent mode, in place on the state
   (same page, table "Evaluation criteria": O(1) recurrent step at inference).
 
@@ -86,6 +90,10 @@ def _load():
             lib.oracle_ssd_backward.restype = ctypes.c_int
             lib.oracle_ssd_mamba3_recurrent.argtypes = sig6 + [_D] * 12 + [ctypes.c_int]
             lib.oracle_ssd_mamba3_recurrent.restype = ctypes.c_int
+            lib.oracle_ssd_mamba3_decode_step.argtypes = [_I64] * 5 + [_D] * 13 + [ctypes.c_int]
+            lib.oracle_ssd_mamba3_decode_step.restype = ctypes.c_int
+            lib.oracle_ssd_mimo_recurrent.argtypes = sig6 + [_I64] + [_D] * 10 + [ctypes.c_int]
+            lib.oracle_ssd_mimo_recurrent.restype = ctypes.c_int
             lib.oracle_round_bf16.argtypes = [ctypes.c_double]
             lib.oracle_round_bf16.restype = ctypes.c_double
             lib.oracle_round_bf16_array.argtypes = [_D, _D, _I64]
@@ -246,4 +254,42 @@ def mamba3_recurrent(x, dt_raw, dt_bias, A, B, C, D, lam=None, theta=None, init_
                                              _ptr(y), _ptr(fs), int(nthreads))
     if rc != 0:
         raise ValueError("oracle_ssd_mamba3_recurrent: invalid arguments")
+    return y, fs
+
+
+def mamba3_decode_step(state, B_prev, x_prev, x, dt_raw, dt_bias, A, B, C, D, lam=None, theta=None, nthreads=0):
+    """One Mamba-3 token in place on ``state`` [b,H,N,P] and the previous-token
+    buffers ``B_prev`` [b,G,N], ``x_prev`` [b,H,P] (float64, modified; zero
+    before the first token).  x [b,H,P], dt_raw [b,H], B, C [b,G,N], lam [b,H],
+    theta [b,G,N/2].  Returns y [b,H,P]."""
+    for a in (state, B_prev, x_prev):
+        if a.dtype != np.float64 or not a.flags.c_contiguous:
+            raise TypeError("state and buffers must be C-contiguous float64 arrays (updated in place)")
+    x, dt_raw, dt_bias, A, B, C, D, lam, theta = map(_f64, (x, dt_raw, dt_bias, A, B, C, D, lam, theta))
+    b, H, P = x.shape
+    G, N = B.shape[1], B.shape[2]
+    assert state.shape == (b, H, N, P) and B_prev.shape == B.shape and x_prev.shape == x.shape
+    y = np.empty((b, H, P))
+    rc = _load().oracle_ssd_mamba3_decode_step(b, H, P, N, G, _ptr(state), _ptr(B_prev), _ptr(x_prev), _ptr(x),
+                                               _ptr(dt_raw), _ptr(dt_bias), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                                               _ptr(lam), _ptr(theta), _ptr(y), int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle_ssd_mamba3_decode_step: invalid arguments")
+    return y
+
+
+def mimo_recurrent(x, dt_raw, dt_bias, A, B, C, D, init_state=None, nthreads=0):
+    """A sequence of MIMO tokens: x [b,L,H,R,P], dt_raw [b,L,H], B, C [b,L,G,R,N].
+    Returns (y [b,L,H,R,P], final_state [b,H,N,P])."""
+    x, dt_raw, dt_bias, A, B, C, D, init_state = map(_f64, (x, dt_raw, dt_bias, A, B, C, D, init_state))
+    b, L, H, R, P = x.shape
+    G, N = B.shape[2], B.shape[4]
+    assert B.shape == C.shape == (b, L, G, R, N) and dt_raw.shape == (b, L, H)
+    y = np.empty_like(x)
+    fs = np.empty((b, H, N, P))
+    rc = _load().oracle_ssd_mimo_recurrent(b, L, H, P, N, G, R, _ptr(x), _ptr(dt_raw), _ptr(dt_bias), _ptr(A),
+                                           _ptr(B), _ptr(C), _ptr(D), _ptr(init_state), _ptr(y), _ptr(fs),
+                                           int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle_ssd_mimo_recurrent: invalid arguments")
     return y, fs

@@ -640,3 +640,110 @@ int oracle_ssd_mamba3_recurrent(int64_t batch, int64_t seqlen, int64_t nheads, i
     }
     return 0;
 }
+
+/* ------------------------------------------------------------------------ */
+/* 8. Mamba-3 decode step and MIMO sequence (references for later kernels). */
+/* ------------------------------------------------------------------------ */
+/* One token of the Mamba-3 recurrence of section 7, in place.  The trapezoid's
+ * left end needs the previous token's input, so the decode state is the SSM
+ * state plus that token's B [b][G][N] and x [b][H][P] (zero before the first
+ * token); both are replaced by this token's.  lam [b][H], theta [b][G][N/2]
+ * nullable as in section 7. */
+int oracle_ssd_mamba3_decode_step(int64_t batch, int64_t nheads, int64_t headdim, int64_t dstate,
+                                  int64_t ngroups, double* state, double* B_prev, double* x_prev,
+                                  const double* x, const double* dt_raw, const double* dt_bias, const double* A,
+                                  const double* B, const double* C, const double* D, const double* lam,
+                                  const double* theta, double* y, int nthreads) {
+    if (check_dims(batch, 1, nheads, headdim, dstate, ngroups)) return -1;
+    if (!state || !B_prev || !x_prev || !x || !dt_raw || !A || !B || !C || !y) return -1;
+    if (theta && dstate % 2 != 0) return -1;
+    const int64_t H = nheads, P = headdim, N = dstate, G = ngroups;
+    const int64_t heads_per_group = H / G;
+    const int nt = set_threads(nthreads);
+    int64_t pair;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nt)
+    for (pair = 0; pair < batch * H; ++pair) {
+        const int64_t b = pair / H, h = pair % H, g = h / heads_per_group;
+        double* st = state + (b * H + h) * N * P;
+        const double dt = sp(dt_raw[b * H + h] + (dt_bias ? dt_bias[h] : 0.0));
+        const double decay = exp(dt * A[h]);
+        const double mix = lam ? lam[b * H + h] : 1.0;
+        const double* xp = x_prev + (b * H + h) * P;
+        const double* Bp = B_prev + (b * G + g) * N;
+        const double* xt = x + (b * H + h) * P;
+        const double* Bt = B + (b * G + g) * N;
+        const double* Ct = C + (b * G + g) * N;
+        for (int64_t n = 0; n < N; ++n)
+            for (int64_t p = 0; p < P; ++p) st[n * P + p] += (1.0 - mix) * dt * Bp[n] * xp[p];
+        if (theta) {
+            for (int64_t k = 0; k < N / 2; ++k) {
+                const double ang = theta[(b * G + g) * (N / 2) + k];
+                const double c = cos(ang), s = sin(ang);
+                for (int64_t p = 0; p < P; ++p) {
+                    const double u = st[(2 * k) * P + p], v = st[(2 * k + 1) * P + p];
+                    st[(2 * k) * P + p] = c * u - s * v;
+                    st[(2 * k + 1) * P + p] = s * u + c * v;
+                }
+            }
+        }
+        for (int64_t i = 0; i < N * P; ++i) st[i] *= decay;
+        for (int64_t n = 0; n < N; ++n)
+            for (int64_t p = 0; p < P; ++p) st[n * P + p] += mix * dt * Bt[n] * xt[p];
+        double* yt = y + (b * H + h) * P;
+        for (int64_t p = 0; p < P; ++p) {
+            double acc = 0.0;
+            for (int64_t n = 0; n < N; ++n) acc += Ct[n] * st[n * P + p];
+            yt[p] = acc + (D ? D[h] : 0.0) * xt[p];
+        }
+    }
+    /* the previous-token buffers take this token's inputs (after every head has read them) */
+    memcpy(x_prev, x, sizeof(double) * (size_t)(batch * H * P));
+    memcpy(B_prev, B, sizeof(double) * (size_t)(batch * G * N));
+    return 0;
+}
+
+/* A sequence of MIMO (rank-R) tokens: per token the step of
+ * oracle_ssd_decode_step_mimo, h_t = exp(dt_t A) h_{t-1} + dt_t sum_r B_{t,r} x_{t,r}^T,
+ * y_{t,r} = C_{t,r}^T h_t + D x_{t,r}.  x, y [b][L][H][R][P]; B, C [b][L][G][R][N]. */
+int oracle_ssd_mimo_recurrent(int64_t batch, int64_t seqlen, int64_t nheads, int64_t headdim, int64_t dstate,
+                              int64_t ngroups, int64_t rank, const double* x, const double* dt_raw,
+                              const double* dt_bias, const double* A, const double* B, const double* C,
+                              const double* D, const double* init_state, double* y, double* final_state,
+                              int nthreads) {
+    if (check_dims(batch, seqlen, nheads, headdim, dstate, ngroups) || rank < 1) return -1;
+    if (!x || !dt_raw || !A || !B || !C || !y) return -1;
+    const int64_t H = nheads, P = headdim, N = dstate, G = ngroups, L = seqlen, R = rank;
+    const int64_t heads_per_group = H / G;
+    const int nt = set_threads(nthreads);
+    int64_t pair;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nt)
+    for (pair = 0; pair < batch * H; ++pair) {
+        const int64_t b = pair / H, h = pair % H, g = h / heads_per_group;
+        double* st = (double*)malloc(sizeof(double) * N * P);
+        if (init_state) memcpy(st, init_state + (b * H + h) * N * P, sizeof(double) * N * P);
+        else memset(st, 0, sizeof(double) * N * P);
+        for (int64_t t = 0; t < L; ++t) {
+            const double dt = sp(dt_raw[(b * L + t) * H + h] + (dt_bias ? dt_bias[h] : 0.0));
+            const double decay = exp(dt * A[h]);
+            const double* Xt = x + ((b * L + t) * H + h) * R * P;
+            const double* Bt = B + ((b * L + t) * G + g) * R * N;
+            const double* Ct = C + ((b * L + t) * G + g) * R * N;
+            for (int64_t n = 0; n < N; ++n)
+                for (int64_t p = 0; p < P; ++p) {
+                    double in = 0.0;
+                    for (int64_t r = 0; r < R; ++r) in += Bt[r * N + n] * Xt[r * P + p];
+                    st[n * P + p] = decay * st[n * P + p] + dt * in;
+                }
+            double* Yt = y + ((b * L + t) * H + h) * R * P;
+            for (int64_t r = 0; r < R; ++r)
+                for (int64_t p = 0; p < P; ++p) {
+                    double acc = 0.0;
+                    for (int64_t n = 0; n < N; ++n) acc += Ct[r * N + n] * st[n * P + p];
+                    Yt[r * P + p] = acc + (D ? D[h] : 0.0) * Xt[r * P + p];
+                }
+        }
+        if (final_state) memcpy(final_state + (b * H + h) * N * P, st, sizeof(double) * N * P);
+        free(st);
+    }
+    return 0;
+}

@@ -143,3 +143,20 @@ def test_angles_follow_the_group_map():
     y_flat, _ = oracle.mamba3_recurrent(**dict(c, theta=None))
     assert rel(y_rot[:, :, 2:], y_flat[:, :, 2:]) < 1e-13      # heads 2, 3 read group 1
     assert rel(y_rot[:, :, :2], y_flat[:, :, :2]) > 1e-3
+
+
+# m8: the decode step (state + the previous token's B and x) stepped over a
+# sequence reproduces the sequence recurrence token by token
+def test_mamba3_decode_steps_equal_the_recurrence():
+    rng = np.random.default_rng(6)
+    c = mamba3_case(rng, b=2, L=17, H=4, P=3, N=6, G=2)
+    y_ref, f_ref = oracle.mamba3_recurrent(**c)
+    b, L, H, P = c["x"].shape
+    G, N = c["B"].shape[2:]
+    st = c["init_state"].copy()
+    Bp, xp = np.zeros((b, G, N)), np.zeros((b, H, P))
+    for t in range(L):
+        y = oracle.mamba3_decode_step(st, Bp, xp, c["x"][:, t], c["dt_raw"][:, t], c["dt_bias"], c["A"],
+                                      c["B"][:, t], c["C"][:, t], c["D"], c["lam"][:, t], c["theta"][:, t])
+        assert rel(y, y_ref[:, t]) < 1e-12
+    assert rel(st, f_ref) < 1e-12

@@ -57,6 +57,9 @@ MUTATIONS = [
     ("m3_rotation_not_orthogonal", "r0[p] = c * u - s * v;", "r0[p] = c * u + s * v;"),
     ("m3_angle_indexed_by_head", "const double ang = theta[((b * L + t) * G + g) * (N / 2) + k];",
      "const double ang = theta[((b * L + t) * G + h % G) * (N / 2) + k];"),
+    ("m3_decode_buffers_not_advanced", "memcpy(x_prev, x, sizeof(double) * (size_t)(batch * H * P));", ";"),
+    ("mimo_sequence_state_not_decayed", "st[n * P + p] = decay * st[n * P + p] + dt * in;",
+     "st[n * P + p] = st[n * P + p] + dt * in;"),
     ("bwd_wrong_segment_checkpoint", "memcpy(seg, ck + k * NP, sizeof(double) * NP);",
      "memcpy(seg, ck + (k > 0 ? k - 1 : 0) * NP, sizeof(double) * NP);"),
 ]
@@ -86,6 +89,8 @@ PIN_TESTS = [
     m3_pins.test_common_rotation_of_B_and_C_is_invisible,
     m3_pins.test_first_angle_acts_on_the_state_only,
     m3_pins.test_angles_follow_the_group_map,
+    m3_pins.test_mamba3_decode_steps_equal_the_recurrence,
+    lambda: pins.test_mimo_sequence_is_a_chain_of_mimo_steps(3),
 ]
 
 

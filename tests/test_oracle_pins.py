@@ -356,3 +356,28 @@ def test_mimo_bf16_state_rounding():
                                  round_state_bf16=True)
     assert np.array_equal(y1, y2)
     assert np.array_equal(rounded, oracle.round_bf16(exact))
+
+
+# p-mimo-seq: the MIMO sequence oracle is the (separately pinned) MIMO decode
+# step applied token by token, and at rank 1 the SISO recurrence
+@pytest.mark.parametrize("R", [1, 3])
+def test_mimo_sequence_is_a_chain_of_mimo_steps(R):
+    rng = np.random.default_rng(70 + R)
+    b, L, H, P, N, G = 2, 11, 4, 3, 5, 2
+    x = rng.standard_normal((b, L, H, R, P))
+    dt_raw = rng.standard_normal((b, L, H))
+    dt_bias = rng.uniform(-1, 0.5, H)
+    A = -rng.uniform(0.5, 3.0, H)
+    B = rng.standard_normal((b, L, G, R, N))
+    C = rng.standard_normal((b, L, G, R, N))
+    D = rng.standard_normal(H)
+    h0 = rng.standard_normal((b, H, N, P))
+    y, fs = oracle.mimo_recurrent(x, dt_raw, dt_bias, A, B, C, D, h0)
+    st = h0.copy()
+    for t in range(L):
+        yt = oracle.decode_step_mimo(st, x[:, t], dt_raw[:, t], dt_bias, A, B[:, t], C[:, t], D)
+        assert rel(y[:, t], yt) < 1e-13
+    assert rel(fs, st) < 1e-13
+    if R == 1:
+        y1, f1 = oracle.recurrent(x[:, :, :, 0], dt_raw, dt_bias, A, B[:, :, :, 0], C[:, :, :, 0], D, h0)
+        assert rel(y[:, :, :, 0], y1) < 1e-13 and rel(fs, f1) < 1e-13
