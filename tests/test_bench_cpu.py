@@ -1,0 +1,46 @@
+"""bench.py's algorithmic byte and flop counts (the roofline numerators),
+checked against counts written out tensor by tensor for the Mamba-2
+1.3B-shaped layer (batch 4 x 2048 tokens, 64 heads x P=64, N=128, one group,
+chunk 256) and the batch-256 decode.  No GPU is used."""
+import bench
+
+b, L, H, P, N, G, Q = 4, 2048, 64, 64, 128, 1, 256
+tok = b * L
+
+
+def test_prefill_bytes_tensor_by_tensor():
+    x = tok * H * P * 2                  # bf16
+    y = tok * H * P * 4                  # fp32
+    bc = 2 * tok * G * N * 2             # B and C, bf16
+    dt_raw = tok * H * 2
+    final = b * H * N * P * 4
+    assert bench.prefill_bytes(b, L, H, P, N, G, 2, 4, 4) == x + y + bc + dt_raw + final == 214_958_080
+
+
+def test_prefill_flops_per_chunk():
+    nc = L // Q
+    cb = G * 2 * Q * Q * N               # C B^T, once per group
+    mx = H * 2 * Q * Q * P               # the masked matrix times X
+    states = H * 4 * Q * N * P           # chunk state in and C h out
+    assert bench.prefill_flops(b, L, H, P, N, G, Q) == b * nc * (cb + mx + states)
+
+
+def test_backward_bytes_tensor_by_tensor():
+    reads = tok * H * P * 2 * 2 + tok * H * 2 + 2 * tok * G * N * 2 + b * H * N * P * 4   # x, dy, dt_raw, B, C, dfinal
+    writes = tok * H * P * 4 + tok * H * 4 + 2 * tok * G * N * 4                          # dx, ddt_raw, dB, dC (fp32)
+    assert bench.backward_bytes(b, L, H, P, N, G, 2, 4, 4) == reads + writes == 292_552_704
+
+
+def test_backward_flops_are_three_scans():
+    # the adjoint scan has the forward's shape; the two transposed scans have
+    # headdim N, dstate P and one group per head
+    main = bench.prefill_flops(b, L, H, P, N, G, Q)
+    transposed = bench.prefill_flops(b, L, H, N, P, H, Q)
+    assert bench.backward_flops(b, L, H, P, N, G, Q) == main + 2 * transposed
+
+
+def test_decode_bytes_state_read_and_write():
+    bd, Hd, Pd, Nd, Gd = 256, 128, 64, 128, 8
+    state = 2 * bd * Hd * Nd * Pd * 4
+    io = bd * Hd * Pd * (2 + 4) + 2 * bd * Gd * Nd * 2 + bd * Hd * 2
+    assert bench.decode_bytes(bd, Hd, Pd, Nd, Gd, 2, 4, 4) == state + io == 2_161_180_672
