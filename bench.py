@@ -39,6 +39,9 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+# kernel paths reported by ssd_chunk_scan_path
+PATH_NAMES = {0: "tensor cores", 1: "cuda cores", 2: "tensor cores, head pairs"}
+
 METRIC = "SSD prefill tokens/s + TFLOP/s; decode tokens/s + state GB/s (1 B200)"
 
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one
@@ -266,7 +269,7 @@ def measure_workloads(torch, ssd, I, dev, peaks, max_call_s=2.0):
         flops = prefill_flops(b, L, H, P, N, G, Q)
         t_hbm = nbytes / (hbm * 1e9)
         t_tc = flops / (peaks["bf16_tflops"] * 1e12)
-        out[sh.name] = {"kind": "prefill", "path": "tensor cores" if ssd.ssd_chunk_scan_path(desc) == 0 else "cuda cores",
+        out[sh.name] = {"kind": "prefill", "path": PATH_NAMES[ssd.ssd_chunk_scan_path(desc)],
                         "tokens_per_s": b * L / sec, "ms_per_call": sec * 1e3, "tflops": flops / sec / 1e12,
                         "gbs": nbytes / sec / 1e9, "bound": "hbm" if t_hbm >= t_tc else "tensor",
                         "frac": max(t_hbm, t_tc) / sec}
@@ -730,7 +733,7 @@ def main():
                            "chunk": s.chunk, "inputs": "bf16", "accumulate": "fp32", "y": "fp32",
                            "final_state": "fp32", "parallelism": f"dp{world}" if world > 1 else "single",
                            "l2": "3 rotating input sets (x 67 MB each); inputs larger than L2 across steps",
-                           "kernel_path": "tensor cores" if path == 0 else "cuda cores"},
+                           "kernel_path": PATH_NAMES[path]},
                 "tflops": tflops, "gbs": gbs, "roofline": roofline, "decode": decode_line,
                 "backward": backward_line, "mamba3": mamba3_line,
                 "cpu_baseline": cpu_baseline, "e2e": e2e, "workloads": workloads,

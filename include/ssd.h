@@ -150,7 +150,10 @@ ssd_status_t ssd_chunk_scan_workspace_size(const ssd_prefill_desc_t* desc, size_
  *       by TMA; fp32 accumulation and fp32 state passing): headdim 64,
  *       dstate 64, 128 or 256, chunk 128 or 256,
  *   1 = CUDA-core fp32 path (fp32 inputs, or shapes the tensor-core path does
- *       not cover).
+ *       not cover),
+ *   2 = the tensor-core path over pairs of heads of one group, which share
+ *       B, C and C B^T: dstate 128 with an even number of heads per group and
+ *       at least 148 (batch, head) sequences; same arithmetic as path 0.
  * Pure host function.
  */
 ssd_status_t ssd_chunk_scan_path(const ssd_prefill_desc_t* desc, int32_t* path);

@@ -92,7 +92,9 @@ static PrefillLayout prefill_layout(const ssd_prefill_desc_t* d, bool tc) {
 }
 
 static int prefill_path(const ssd_prefill_desc_t* d) {
-    return tc_path_supports(d->headdim, d->dstate, d->chunk, d->io_dtype == SSD_BF16) ? 0 : 1;
+    const bool bf = d->io_dtype == SSD_BF16;
+    if (!tc_path_supports(d->headdim, d->dstate, d->chunk, bf)) return 1;
+    return pair_path_supports(d->batch, d->nheads, d->headdim, d->dstate, d->ngroups, d->chunk, bf) ? 2 : 0;
 }
 
 // replay descriptor checks shared by ssd_replay_buffer_size and ssd_replay_step
@@ -156,7 +158,7 @@ ssd_status_t ssd_chunk_scan_workspace_size(const ssd_prefill_desc_t* desc, size_
     if (!bytes) return SSD_ERR_INVALID_ARG;
     const ssd_status_t st = check_prefill_desc(desc);
     if (st != SSD_OK) return st;
-    *bytes = prefill_layout(desc, prefill_path(desc) == 0).total;
+    *bytes = prefill_layout(desc, prefill_path(desc) != 1).total;
     return SSD_OK;
 }
 
@@ -189,7 +191,7 @@ static ssd_status_t prefill(const ssd_prefill_desc_t* d, const void* x, const vo
         overlaps(y, y_bytes, C, bc_bytes) || overlaps(final_state, s_bytes, y, y_bytes) ||
         overlaps(final_state, s_bytes, x, x_bytes))
         return SSD_ERR_INVALID_ARG;
-    const bool tc = prefill_path(d) == 0;
+    const bool tc = prefill_path(d) != 1;
     const PrefillLayout lay = prefill_layout(d, tc);
     if (d->batch == 0) return SSD_OK;
     if (d->seqlen > 0 && (!workspace || workspace_bytes < lay.total)) return SSD_ERR_WORKSPACE;
@@ -244,7 +246,7 @@ ssd_status_t ssd_chunk_scan_fwd_varlen(const ssd_prefill_desc_t* d, const void* 
 
 static Mamba3Layout m3_layout(const ssd_prefill_desc_t* d) {
     return mamba3_layout(d->batch, d->seqlen, d->nheads, d->headdim, d->dstate, d->ngroups, d->chunk,
-                         d->io_dtype == SSD_BF16, prefill_path(d) == 0);
+                         d->io_dtype == SSD_BF16, prefill_path(d) != 1);
 }
 
 static ssd_status_t check_mamba3_desc(const ssd_prefill_desc_t* d) {
@@ -301,7 +303,7 @@ ssd_status_t ssd_chunk_scan_fwd_mamba3(const ssd_prefill_desc_t* d, const void* 
     a.batch = d->batch; a.L = d->seqlen; a.H = d->nheads; a.P = d->headdim; a.N = d->dstate;
     a.G = d->ngroups; a.Q = d->chunk;
     a.io_bf16 = d->io_dtype == SSD_BF16; a.y_bf16 = d->y_dtype == SSD_BF16;
-    a.state_bf16 = d->state_dtype == SSD_BF16; a.tc = prefill_path(d) == 0;
+    a.state_bf16 = d->state_dtype == SSD_BF16; a.tc = prefill_path(d) != 1;
     a.x = x; a.dt_raw = dt_raw; a.B = B; a.C = C; a.dt_bias = dt_bias; a.A = A; a.D = D;
     a.lam = lam; a.theta = theta; a.init_state = init_state; a.y = y; a.final_state = final_state;
     a.ws = (char*)workspace; a.lay = lay;
@@ -316,7 +318,7 @@ ssd_status_t ssd_chunk_scan_mamba3_launches(const ssd_prefill_desc_t* desc, int3
     if (!launches) return SSD_ERR_INVALID_ARG;
     const ssd_status_t st = check_mamba3_desc(desc);
     if (st != SSD_OK) return st;
-    const bool tc = prefill_path(desc) == 0;
+    const bool tc = prefill_path(desc) != 1;
     if (desc->batch == 0) *launches = 0;
     else if (desc->seqlen == 0) *launches = has_final_state ? 1 : 0;
     else if (!has_lam && !has_theta) *launches = 1 + (tc ? 1 : 3);

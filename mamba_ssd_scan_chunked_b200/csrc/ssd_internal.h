@@ -85,6 +85,10 @@ bool tc_path_supports(int64_t P, int64_t N, int64_t Q, bool io_bf16);
 // runs per sequence of the tensor-core path (1 = every work item is a whole sequence)
 int64_t tc_runs(int64_t BH, int64_t nchunks, int64_t N);
 cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s);
+// tensor-core prefill over pairs of heads of one group (ssd_prefill_pair.cu);
+// launch_prefill_tc takes it for the shapes it covers
+bool pair_path_supports(int64_t batch, int64_t H, int64_t P, int64_t N, int64_t G, int64_t Q, bool io_bf16);
+cudaError_t launch_prefill_pair(const PrefillArgs& a, cudaStream_t s);
 
 // Backward pass of the prefill (ssd_backward.cu).  Workspace carve-up, all
 // offsets 256-byte aligned; "slice" strides separate the column slices of the

@@ -1,0 +1,679 @@
+// Tensor-core prefill of the SSD layer core for sm_100a, two heads at a time.
+//
+// The chunked contraction of the semiseparable matrix ("Mamba-2 vs
+// Transformers / SSD", section "Mamba-2 and the SSD paper: what changed in
+// practice": chunks processed in parallel, per-chunk states recombined; table
+// row "Blocked two-pass contraction").  Heads of one group share B and C, and
+// so share S = C B^T.  A work item here is a pair of heads (h0, h0+1) of one
+// group and one batch element, walked through its sequence in blocks of 128
+// tokens with both states kept in TMEM.  Per block, with r = decay cumsum *
+// log2(e) relative to the block start (per head):
+//
+//   S      = C B^T                         once for both heads (tcgen05, fp32 in TMEM)
+//   M_k    = S o [s<=l] 2^(r_l - r_s) dt_s  per head k (CUDA cores, TMEM -> regs -> TMEM)
+//   Yoff_k = C h_k                          (tcgen05; then scaled by 2^(r_l) in place)
+//   h_k'   = 2^(r_last) h_k + B^T (w o X_k) (tcgen05 onto the scaled state in TMEM)
+//   y_k    = Yoff_k + M_k X_k + D_k x       (tcgen05 onto Yoff, fp32 epilogue, TMA store)
+//
+// For a 16-token column group J lying wholly before the rows it meets, the
+// decay factor is split as 2^(r_l - r_J) * [2^(r_J - r_s) dt_s] (r_J = r at the
+// group's last token): one exponential per row and group, and one per token
+// shared by every row.  Both factors are <= 1 when the log-decays never
+// increase; a block where some head's cumsum does increase (A > 0 in some
+// token) takes the per-element form everywhere.
+//
+// Precision as in the single-head kernel: every operand computed in-kernel (M,
+// w o X, h) is contracted as a bf16 pair hi + lo against the exact bf16 input.
+//
+// Roles (one CTA per SM, persistent over its items c, c + grid, ...):
+//   warps 0-15  compute: warp w works on TMEM lanes 32*(w%4).. (tile rows) and
+//               the 16-column part w/4 of the state, Yoff and output tiles;
+//               warps with w%4 < 2 also form w o X, since their share of the
+//               causal mask transform is the smaller one
+//   warp 16     MMA issue (one elected lane, converged warp)
+//   warp 17     TMA: operand loads (C, B double-buffered one block ahead), the
+//               y stores, which it stages in the C/B buffers of the block just
+//               finished
+// Every wait on an mbarrier is bounded (2 s); the first one that gives up sets
+// the device error word and a CTA-wide abort word that ends every later wait
+// at once, so the launch always finishes.  No inter-CTA waits exist.
+#include "ssd_internal.h"
+#include "ssd_tc_common.cuh"
+
+namespace ssd {
+namespace pair {
+using namespace ::ssd::tc;
+
+constexpr int NS = 128;              // dstate of this kernel
+constexpr int PD = 64;               // headdim of this kernel
+constexpr int NCW = 16;              // compute warps
+constexpr int NCT = NCW * 32;
+constexpr int WARP_MMA = NCW, WARP_TMA = NCW + 1;
+constexpr int THREADS = NCT + 64;
+
+// TMEM columns (512 allocated)
+constexpr uint32_t COL_R0 = 0;      // S (fp32), turned in place into M of head 0 (bf16 hi|lo per K step)
+constexpr uint32_t COL_R1 = 128;    // M of head 1
+constexpr uint32_t COL_Y = 256;     // + 64 k: C h_k scaled, then + M_k X_k (fp32)
+constexpr uint32_t COL_ST = 384;    // + 64 k: state of head k (fp32, lane = state row)
+
+// shared memory (tiles 1024-byte aligned, 128-byte swizzle)
+constexpr uint32_t STAGE = 4 * TILE;             // C (K blocks 0, 1), B (K blocks 0, 1); later y staging
+constexpr uint32_t OFF_X = 2 * STAGE;            // x of head 0, head 1
+constexpr uint32_t OFF_W = OFF_X + 2 * TILE;     // per head: hi, lo of h (C h), then of w o X (state)
+constexpr uint32_t TILES = OFF_W + 4 * TILE;
+constexpr uint32_t OFF_DT = TILES;               // [2][128] dt, turned into u_s = log2(dt_s) - r_s
+constexpr uint32_t OFF_ACS = OFF_DT + 2 * SUB * 4;     // [2][128] chunk-local cumsum (natural log)
+constexpr int NFAC = 96;                         // tokens whose group can lie before a row block
+constexpr uint32_t OFF_FAC = OFF_ACS + 2 * SUB * 4;    // [2][96] 2^(r_J - r_s) dt_s
+constexpr uint32_t OFF_BAR = OFF_FAC + 2 * NFAC * 4;
+enum { B_CB0, B_CB1, B_X, B_T, B_S, B_OFF, B_ST, B_Y0, B_Y, B_H, B_WX, B_M, B_EPI, B_STG0, B_STG1, NBAR };
+constexpr uint32_t OFF_MISC = OFF_BAR + 8 * NBAR;      // TMEM base, abort word
+constexpr uint32_t SMEM = OFF_MISC + 16;
+static_assert(TILES % 1024 == 0 && OFF_BAR % 8 == 0, "alignment");
+static_assert(SMEM <= 232448, "shared memory per CTA");
+
+struct Params {
+    const float* dtw;          // [BH][Lpad] dt
+    const float* acsw;         // [BH][Lpad] chunk-local inclusive cumsum of dt*A
+    const void* init_state;    // [BH][N][P] state dtype or NULL
+    void* final_state;         // [BH][N][P] state dtype or NULL
+    const float* D;            // [H] or NULL
+    unsigned* dev_err;
+    long long Lpad;
+    int H, G, Q, nblk, npairs;
+    int state_bf16, y_bf16;
+};
+
+// bounded wait that gives up at once when another wait of the CTA has given up
+__device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, volatile int* abort) {
+    uint32_t spins = 0;
+    unsigned long long deadline = 0;
+    while (!mbar_try(bar, parity)) {
+        if ((++spins & 255u) == 0) {
+            if (*abort) return false;
+            const unsigned long long now = gtimer();
+            if (deadline == 0) {
+                deadline = now + WAIT_NS;
+            } else if (now > deadline) {
+                *abort = 1;
+                return false;
+            }
+        }
+    }
+    return true;
+}
+
+// hi/lo bf16 pairs of 2 x 4 fp32 values (element 2e in the low half of word e)
+__device__ __forceinline__ void split8(const float* v, uint32_t (&hw)[4], uint32_t (&lw)[4]) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        hw[e] = pack_bf16(v[2 * e], v[2 * e + 1]);
+        lw[e] = pack_bf16(v[2 * e] - bf16_lo(hw[e]), v[2 * e + 1] - bf16_hi(hw[e]));
+    }
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+ssd_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
+                const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmY, const Params p) {
+    extern __shared__ __align__(1024) uint8_t sm[];
+    const uint32_t base = smem_u32(sm);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    volatile int* s_abort = reinterpret_cast<volatile int*>(sm + OFF_MISC + 4);
+    auto bar = [&](int i) -> uint32_t { return base + OFF_BAR + 8u * (uint32_t)i; };
+
+    // the 128-byte swizzle of TMA and of the MMA descriptors assumes 1024-byte aligned tiles
+    if (base & 1023u) {
+        if (threadIdx.x == 0) atomicOr(p.dev_err, kErrAsyncTimeout);
+        return;
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;"
+                     ::"r"(base + OFF_MISC) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    if (threadIdx.x == NCT) {
+        //                          CB0 CB1 X  T  S  OFF ST Y0 Y  H    WX       M    EPI  STG0 STG1
+        const uint32_t cnt[NBAR] = {1, 1, 1, 1, 1, 1, 1, 1, 1, NCT, NCT / 2, NCT, NCT, NCT, NCT};
+        for (int i = 0; i < NBAR; ++i) mbar_init(bar(i), cnt[i]);
+        *s_abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + OFF_MISC);
+
+    // items of this CTA: blockIdx.x, + gridDim.x, ...; flat block counter jj over them
+    const int nitems = p.npairs > (int)blockIdx.x ? (p.npairs - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+    const int total = nitems * p.nblk;
+    const int hpg = p.H / p.G;
+    struct Item { int b, g, h0; };
+    auto item_of = [&](int i) -> Item {
+        const int it = (int)blockIdx.x + i * (int)gridDim.x;
+        const int pr = it % (hpg >> 1), bg = it / (hpg >> 1);
+        Item d;
+        d.g = bg % p.G;
+        d.b = bg / p.G;
+        d.h0 = d.g * hpg + 2 * pr;
+        return d;
+    };
+    unsigned err = 0;
+    auto wait = [&](int i, uint32_t ph) {
+        if (!wait_or_abort(bar(i), ph, s_abort)) err |= kErrAsyncTimeout;
+    };
+
+    if (warp == WARP_TMA) {
+        // ======================================================== TMA producer
+        const uint32_t lead = elect_one();
+        auto load_cb = [&](int t) {          // C, B of block t into stage t & 1 (+ its x into L2)
+            const Item d = item_of(t / p.nblk);
+            const int t0 = (t % p.nblk) * SUB;
+            const uint32_t st = base + (uint32_t)(t & 1) * STAGE, bb = bar(B_CB0 + (t & 1));
+            mbar_expect_tx(bb, 4 * TILE);
+            tma_load_4d(st, &tmC, 0, d.g, t0, d.b, bb);
+            tma_load_4d(st + TILE, &tmC, 64, d.g, t0, d.b, bb);
+            tma_load_4d(st + 2 * TILE, &tmB, 0, d.g, t0, d.b, bb);
+            tma_load_4d(st + 3 * TILE, &tmB, 64, d.g, t0, d.b, bb);
+            tma_prefetch_4d(&tmX, 0, d.h0, t0, d.b);
+            tma_prefetch_4d(&tmX, 0, d.h0 + 1, t0, d.b);
+        };
+        auto load_x = [&](int t) {
+            const Item d = item_of(t / p.nblk);
+            const int t0 = (t % p.nblk) * SUB;
+            mbar_expect_tx(bar(B_X), 2 * TILE);
+            tma_load_4d(base + OFF_X, &tmX, 0, d.h0, t0, d.b, bar(B_X));
+            tma_load_4d(base + OFF_X + TILE, &tmX, 0, d.h0 + 1, t0, d.b, bar(B_X));
+        };
+        auto load_t = [&](int t) {           // dt and cumsum of both heads
+            const Item d = item_of(t / p.nblk);
+            const long long o = (long long)(d.b * p.H + d.h0) * p.Lpad + (long long)(t % p.nblk) * SUB;
+            mbar_expect_tx(bar(B_T), 4 * SUB * 4);
+            bulk_load(base + OFF_DT, p.dtw + o, SUB * 4, bar(B_T));
+            bulk_load(base + OFF_DT + SUB * 4, p.dtw + o + p.Lpad, SUB * 4, bar(B_T));
+            bulk_load(base + OFF_ACS, p.acsw + o, SUB * 4, bar(B_T));
+            bulk_load(base + OFF_ACS + SUB * 4, p.acsw + o + p.Lpad, SUB * 4, bar(B_T));
+        };
+        if (lead && total > 0) {
+            load_cb(0);
+            if (total > 1) load_cb(1);
+            load_x(0);
+            // dt and the cumsum come from the decay kernel this launch may overlap
+            // (programmatic dependent launch): wait for it before reading them
+            asm volatile("griddepcontrol.wait;" ::: "memory");
+            load_t(0);
+        }
+        for (int jj = 0; jj < total; ++jj) {
+            const uint32_t ph = jj & 1;
+            wait(B_M, ph);                   // the block's dt / cumsum are consumed
+            if (lead && jj + 1 < total && !*s_abort) load_t(jj + 1);
+            wait(B_Y, ph);                   // its x is consumed
+            if (lead && jj + 1 < total && !*s_abort) load_x(jj + 1);
+            wait(B_STG0 + (jj & 1), (jj >> 1) & 1);   // y staged in the block's C/B stage
+            if (lead && !*s_abort) {
+                const Item d = item_of(jj / p.nblk);
+                const int t0 = (jj % p.nblk) * SUB;
+                const uint32_t st = base + (uint32_t)(jj & 1) * STAGE;
+#pragma unroll
+                for (int k = 0; k < 2; ++k) {
+                    tma_store_4d(&tmY, st + k * 2 * TILE, 0, d.h0 + k, t0, d.b);
+                    if (!p.y_bf16) tma_store_4d(&tmY, st + k * 2 * TILE + TILE, 32, d.h0 + k, t0, d.b);
+                }
+                bulk_commit();
+                bulk_wait_read0();           // the stage is free again
+                if (jj + 2 < total) load_cb(jj + 2);
+            }
+            __syncwarp();
+        }
+        if (lead) bulk_wait0();
+    } else if (warp == WARP_MMA) {
+        // ======================================================== MMA issue
+        const uint32_t lead = elect_one();
+        constexpr uint32_t ID_S = idesc_bf16(128, 128, false, false);   // C (K-major) x B^T (K-major)
+        constexpr uint32_t ID_N64 = idesc_bf16(128, PD, false, true);   // C x h (MN-major); M (TMEM) x X (MN-major)
+        constexpr uint32_t ID_ST = idesc_bf16(128, PD, true, true);     // B^T (MN-major) x wX (MN-major)
+        constexpr uint32_t KSTEP_K = 2, KBLOCK_K = TILE >> 4, KSTEP_MN = 2048 >> 4;
+        const uint64_t dX0 = sdesc(base + OFF_X, TILE, 1024), dX1 = sdesc(base + OFF_X + TILE, TILE, 1024);
+        const uint64_t dW00 = sdesc(base + OFF_W, TILE, 1024), dW01 = sdesc(base + OFF_W + TILE, TILE, 1024);
+        const uint64_t dW10 = sdesc(base + OFF_W + 2 * TILE, TILE, 1024);
+        const uint64_t dW11 = sdesc(base + OFF_W + 3 * TILE, TILE, 1024);
+        const uint32_t lead0 = lead;
+        for (int jj = 0; jj < total; ++jj) {
+            const uint32_t ph = jj & 1;
+            const uint32_t lead = lead0 && !*s_abort;     // once a wait gave up, issue nothing more
+            const uint32_t st = base + (uint32_t)(jj & 1) * STAGE;
+            const uint64_t dC = sdesc(st, 16, 1024), dBk = sdesc(st + 2 * TILE, 16, 1024);
+            const uint64_t dBm = sdesc(st + 2 * TILE, TILE, 1024);
+            // ---- S = C B^T into R0 once the previous block's head-0 Y has read M_0 there
+            wait(B_CB0 + (jj & 1), (jj >> 1) & 1);
+            if (jj > 0) wait(B_Y0, ph ^ 1u);
+            tc_fence_after();
+            __syncwarp();
+#pragma unroll
+            for (int k = 0; k < NS / 16; ++k) {
+                const uint32_t o = (uint32_t)(k >> 2) * KBLOCK_K + (uint32_t)(k & 3) * KSTEP_K;
+                if (k == 0) { if (lead) mma_ss<ID_S, 0>(tmem + COL_R0, dC + o, dBk + o);
+                } else if (lead) mma_ss<ID_S, 1>(tmem + COL_R0, dC + o, dBk + o);
+            }
+            if (lead) mma_commit(bar(B_S));
+            // ---- Yoff_k = C h_k,hi + C h_k,lo (h written by the compute warps; the
+            // previous epilogue has read the Y accumulators)
+            wait(B_H, ph);
+            if (jj > 0) wait(B_EPI, ph ^ 1u);
+            tc_fence_after();
+            __syncwarp();
+#pragma unroll
+            for (int k = 0; k < NS / 16; ++k) {
+                const uint32_t o = (uint32_t)(k >> 2) * KBLOCK_K + (uint32_t)(k & 3) * KSTEP_K;
+                if (k == 0) {
+                    if (lead) mma_ss<ID_N64, 0>(tmem + COL_Y, dC, dW00);
+                    if (lead) mma_ss<ID_N64, 0>(tmem + COL_Y + 64, dC, dW10);
+                } else {
+                    if (lead) mma_ss<ID_N64, 1>(tmem + COL_Y, dC + o, dW00 + k * KSTEP_MN);
+                    if (lead) mma_ss<ID_N64, 1>(tmem + COL_Y + 64, dC + o, dW10 + k * KSTEP_MN);
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < NS / 16; ++k) {
+                const uint32_t o = (uint32_t)(k >> 2) * KBLOCK_K + (uint32_t)(k & 3) * KSTEP_K;
+                if (lead) mma_ss<ID_N64, 1>(tmem + COL_Y, dC + o, dW01 + k * KSTEP_MN);
+                if (lead) mma_ss<ID_N64, 1>(tmem + COL_Y + 64, dC + o, dW11 + k * KSTEP_MN);
+            }
+            if (lead) mma_commit(bar(B_OFF));
+            // ---- state_k += B^T (w o X_k)_hi + B^T (w o X_k)_lo, onto 2^(r_last) h_k
+            wait(B_WX, ph);
+            tc_fence_after();
+            __syncwarp();
+#pragma unroll
+            for (int k = 0; k < SUB / 16; ++k) {
+                if (lead) mma_ss<ID_ST, 1>(tmem + COL_ST, dBm + k * KSTEP_MN, dW00 + k * KSTEP_MN);
+                if (lead) mma_ss<ID_ST, 1>(tmem + COL_ST + 64, dBm + k * KSTEP_MN, dW10 + k * KSTEP_MN);
+            }
+#pragma unroll
+            for (int k = 0; k < SUB / 16; ++k) {
+                if (lead) mma_ss<ID_ST, 1>(tmem + COL_ST, dBm + k * KSTEP_MN, dW01 + k * KSTEP_MN);
+                if (lead) mma_ss<ID_ST, 1>(tmem + COL_ST + 64, dBm + k * KSTEP_MN, dW11 + k * KSTEP_MN);
+            }
+            if (lead) mma_commit(bar(B_ST));
+            // ---- Y_k += M_k,hi X_k + M_k,lo X_k onto the scaled Yoff (A from TMEM)
+            wait(B_M, ph);
+            tc_fence_after();
+            __syncwarp();
+#pragma unroll
+            for (int k = 0; k < SUB / 16; ++k) {
+                if (lead) mma_ts<ID_N64, 1>(tmem + COL_Y, tmem + COL_R0 + 16 * k, dX0 + k * KSTEP_MN);
+                if (lead) mma_ts<ID_N64, 1>(tmem + COL_Y, tmem + COL_R0 + 16 * k + 8, dX0 + k * KSTEP_MN);
+            }
+            if (lead) mma_commit(bar(B_Y0));
+#pragma unroll
+            for (int k = 0; k < SUB / 16; ++k) {
+                if (lead) mma_ts<ID_N64, 1>(tmem + COL_Y + 64, tmem + COL_R1 + 16 * k, dX1 + k * KSTEP_MN);
+                if (lead) mma_ts<ID_N64, 1>(tmem + COL_Y + 64, tmem + COL_R1 + 16 * k + 8, dX1 + k * KSTEP_MN);
+            }
+            if (lead) mma_commit(bar(B_Y));
+            __syncwarp();
+        }
+    } else {
+        // ======================================================== compute warps
+        const int q = warp & 3, kq = warp >> 2;       // lane quarter, 16-column part
+        const int row = 32 * q + lane;                // TMEM lane = tile row
+        const uint32_t lo16 = (uint32_t)(32 * q) << 16;
+        const float NEG_INF = __int_as_float(0xff800000u);
+        float* s_u = reinterpret_cast<float*>(sm + OFF_DT);          // [2][128] dt -> u
+        const float* s_acs = reinterpret_cast<const float*>(sm + OFF_ACS);
+        float* s_fac = reinterpret_cast<float*>(sm + OFF_FAC);       // [2][96]
+        float prev_last[2] = {0.f, 0.f};
+        int it = -1, j = p.nblk - 1;
+        Item d{};
+        float Dk[2] = {0.f, 0.f};
+        for (int jj = 0; jj < total; ++jj) {
+            if (++j == p.nblk) {
+                j = 0;
+                d = item_of(++it);
+                Dk[0] = p.D ? p.D[d.h0] : 0.f;
+                Dk[1] = p.D ? p.D[d.h0 + 1] : 0.f;
+            }
+            const uint32_t ph = jj & 1;
+            const bool chunk_start = ((j * SUB) & (p.Q - 1)) == 0;   // the cumsum restarts at every chunk
+            const long long bh0 = (long long)d.b * p.H + d.h0;
+
+            // ---- per-token terms: r (log2, relative to the block start) of this
+            // thread's row, u_s = log2(dt_s) - r_s and the off-diagonal factors
+            wait(B_T, ph);
+            float r0[2], rl[2], rlast[2];
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                r0[k] = chunk_start ? 0.f : prev_last[k];
+                rl[k] = (s_acs[k * SUB + row] - r0[k]) * LOG2E;
+                rlast[k] = (s_acs[k * SUB + SUB - 1] - r0[k]) * LOG2E;
+            }
+            uint32_t inc = 0;                 // a log-decay that increases somewhere in the block
+            if (kq < 2) {
+                const int k = kq;
+                const float a_prev = row ? s_acs[k * SUB + row - 1] : r0[k];
+                inc = s_acs[k * SUB + row] > a_prev;
+                const float dtv = s_u[k * SUB + row];
+                const float u = (dtv > 0.f ? __log2f(dtv) : NEG_INF) - rl[k];
+                s_u[k * SUB + row] = u;       // in place: this thread alone reads and writes it
+                if (row < NFAC) s_fac[k * NFAC + row] = ex2((s_acs[k * SUB + (row | 15)] - r0[k]) * LOG2E + u);
+            }
+            prev_last[0] = s_acs[SUB - 1];
+            prev_last[1] = s_acs[2 * SUB - 1];
+            uint32_t direct;
+            asm volatile("{\n .reg .pred pi, po;\n setp.ne.u32 pi, %1, 0;\n bar.red.or.pred po, 1, %2, pi;\n"
+                         " selp.u32 %0, 1, 0, po;\n}\n"
+                         : "=r"(direct) : "r"(inc), "n"(NCT) : "memory");
+
+            // ---- h entering the block (the initial state, or what the previous
+            // block left in TMEM): 2^(r_last) h back into the state accumulator,
+            // h split hi -> W tile, lo -> W tile + TILE for C h
+            if (jj > 0) wait(B_ST, ph ^ 1u);  // previous state MMAs done (also frees W)
+            tc_fence_after();
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const uint32_t col = COL_ST + 64 * k + 16 * kq;
+                float hv[16];
+                if (j > 0) {
+                    uint32_t v[16];
+                    tmem_ld16(tmem + lo16 + col, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) hv[i] = __uint_as_float(v[i]);
+                } else if (p.init_state) {
+                    const long long o = ((bh0 + k) * NS + row) * PD + 16 * kq;
+                    if (p.state_bf16) {
+                        Vec16<bf16>::load(reinterpret_cast<const bf16*>(p.init_state) + o, hv);
+                        Vec16<bf16>::load(reinterpret_cast<const bf16*>(p.init_state) + o + 8, hv + 8);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 16; i += 4)
+                            Vec16<float>::load(reinterpret_cast<const float*>(p.init_state) + o + i, hv + i);
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) hv[i] = 0.f;
+                }
+                const float dl = ex2(rlast[k]);
+                uint32_t sc[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) sc[i] = __float_as_uint(dl * hv[i]);
+                tmem_st16(tmem + lo16 + col, sc);
+                uint8_t* wt = sm + OFF_W + k * 2 * TILE;
+#pragma unroll
+                for (int qq = 0; qq < 2; ++qq) {
+                    uint32_t hw[4], lw[4];
+                    split8(hv + 8 * qq, hw, lw);
+                    const uint32_t o = swz(row, 2 * kq + qq);
+                    *reinterpret_cast<uint4*>(wt + o) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                    *reinterpret_cast<uint4*>(wt + TILE + o) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+                }
+            }
+            tmem_wait_st();
+            fence_proxy_async();
+            tc_fence_before();
+            mbar_arrive(bar(B_H));
+
+            // ---- M_k = S o [s<=l] 2^(r_l - r_s) dt_s, written as bf16 hi/lo per K step:
+            // hi to columns [16g, 16g+8), lo to [16g+8, 16g+16) of R0 (head 0, in place
+            // over S) and R1 (head 1).  Quarter q needs column groups g < 2q+2; the
+            // rest is zero.  Groups g < 2q lie before every row of the quarter.
+            wait(B_S, ph);
+            tc_fence_after();
+#pragma unroll
+            for (int gi = 0; gi < 2; ++gi) {
+                const int g = kq + 4 * gi;
+                const uint32_t c0 = 16u * (uint32_t)g;
+                if (g >= 2 * q + 2) {
+                    uint32_t z[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) z[i] = 0u;
+                    tmem_st16(tmem + lo16 + COL_R0 + c0, z);
+                    tmem_st16(tmem + lo16 + COL_R1 + c0, z);
+                    continue;
+                }
+                uint32_t v[16];
+                tmem_ld16(tmem + lo16 + COL_R0 + c0, v);
+                tmem_wait_ld();
+                const bool before = g < 2 * q && !direct;
+#pragma unroll
+                for (int k = 0; k < 2; ++k) {
+                    uint32_t o[16];
+                    if (before) {
+                        const float f = ex2(rl[k] - (s_acs[k * SUB + c0 + 15] - r0[k]) * LOG2E);
+                        const float4* fb = reinterpret_cast<const float4*>(s_fac + k * NFAC + c0);
+#pragma unroll
+                        for (int i4 = 0; i4 < 4; ++i4) {
+                            const float4 bv = fb[i4];
+                            const float bb[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+                            for (int e = 0; e < 2; ++e) {
+                                const int i = 2 * i4 + e;
+                                const float m0 = __uint_as_float(v[2 * i]) * (f * bb[2 * e]);
+                                const float m1 = __uint_as_float(v[2 * i + 1]) * (f * bb[2 * e + 1]);
+                                const uint32_t hi = pack_bf16(m0, m1);
+                                o[i] = hi;
+                                o[8 + i] = pack_bf16(m0 - bf16_lo(hi), m1 - bf16_hi(hi));
+                            }
+                        }
+                    } else {
+                        const float4* uu = reinterpret_cast<const float4*>(s_u + k * SUB + c0);
+#pragma unroll
+                        for (int i4 = 0; i4 < 4; ++i4) {
+                            const float4 uv = uu[i4];
+                            const float ub[4] = {uv.x, uv.y, uv.z, uv.w};
+#pragma unroll
+                            for (int e = 0; e < 2; ++e) {
+                                const int i = 2 * i4 + e;
+                                const int s0 = (int)c0 + 2 * i;
+                                const float e0 = ex2(s0 <= row ? rl[k] + ub[2 * e] : NEG_INF);
+                                const float e1 = ex2(s0 + 1 <= row ? rl[k] + ub[2 * e + 1] : NEG_INF);
+                                const float m0 = __uint_as_float(v[2 * i]) * e0;
+                                const float m1 = __uint_as_float(v[2 * i + 1]) * e1;
+                                const uint32_t hi = pack_bf16(m0, m1);
+                                o[i] = hi;
+                                o[8 + i] = pack_bf16(m0 - bf16_lo(hi), m1 - bf16_hi(hi));
+                            }
+                        }
+                    }
+                    tmem_st16(tmem + lo16 + (k ? COL_R1 : COL_R0) + c0, o);
+                }
+            }
+
+            // ---- after C h: w o X into the W tiles (quarters 0 and 1: one token row of
+            // one head per thread), Yoff scaled by 2^(r_l), x kept for D x
+            wait(B_OFF, ph);
+            tc_fence_after();
+            if (q < 2) {
+                wait(B_X, ph);
+                const int t = kq * 64 + q * 32 + lane;
+                const int s_ = t & (SUB - 1), k = t >> 7;
+                const float wv = ex2(rlast[k] + s_u[k * SUB + s_]);
+                const uint8_t* xt = sm + OFF_X + k * TILE;
+                uint8_t* wt = sm + OFF_W + k * 2 * TILE;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const uint32_t o = swz(s_, c);
+                    const uint4 xv = *reinterpret_cast<const uint4*>(xt + o);
+                    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+                    float pv[8];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        pv[2 * e] = bf16_lo(xw[e]) * wv;
+                        pv[2 * e + 1] = bf16_hi(xw[e]) * wv;
+                    }
+                    uint32_t hw[4], lw[4];
+                    split8(pv, hw, lw);
+                    *reinterpret_cast<uint4*>(wt + o) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                    *reinterpret_cast<uint4*>(wt + TILE + o) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+                }
+                fence_proxy_async();
+                mbar_arrive(bar(B_WX));
+            }
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const uint32_t col = COL_Y + 64 * k + 16 * kq;
+                const float el = ex2(rl[k]);
+                uint32_t v[16];
+                tmem_ld16(tmem + lo16 + col, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(el * __uint_as_float(v[i]));
+                tmem_st16(tmem + lo16 + col, v);
+            }
+            if (q >= 2) wait(B_X, ph);
+            uint32_t xr[2][8];
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+#pragma unroll
+                for (int qq = 0; qq < 2; ++qq) {
+                    const uint4 xv = *reinterpret_cast<const uint4*>(sm + OFF_X + k * TILE + swz(row, 2 * kq + qq));
+                    xr[k][4 * qq] = xv.x; xr[k][4 * qq + 1] = xv.y; xr[k][4 * qq + 2] = xv.z; xr[k][4 * qq + 3] = xv.w;
+                }
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar(B_M));
+
+            // ---- after Y: the final state (last block), then y = Y + D x staged in the
+            // block's C/B stage (dead once every MMA of the block is done) for the TMA store
+            wait(B_Y, ph);
+            tc_fence_after();
+            if (j == p.nblk - 1 && p.final_state) {
+#pragma unroll
+                for (int k = 0; k < 2; ++k) {
+                    uint32_t sv[16];
+                    tmem_ld16(tmem + lo16 + COL_ST + 64 * k + 16 * kq, sv);
+                    tmem_wait_ld();
+                    float ho[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) ho[i] = __uint_as_float(sv[i]);
+                    const long long o = ((bh0 + k) * NS + row) * PD + 16 * kq;
+                    if (p.state_bf16) {
+                        bf16* fs = reinterpret_cast<bf16*>(p.final_state) + o;
+                        Vec16<bf16>::store(fs, ho);
+                        Vec16<bf16>::store(fs + 8, ho + 8);
+                    } else {
+                        float* fs = reinterpret_cast<float*>(p.final_state) + o;
+#pragma unroll
+                        for (int i = 0; i < 16; i += 4) Vec16<float>::store(fs + i, ho + i);
+                    }
+                }
+            }
+            uint32_t yv[2][16];
+            tmem_ld16(tmem + lo16 + COL_Y + 16 * kq, yv[0]);
+            tmem_ld16(tmem + lo16 + COL_Y + 64 + 16 * kq, yv[1]);
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(bar(B_EPI));          // the Y accumulators may be reused
+            uint8_t* stg = sm + (jj & 1) * STAGE;
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                float out[16];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    out[2 * e] = __uint_as_float(yv[k][2 * e]) + Dk[k] * bf16_lo(xr[k][e]);
+                    out[2 * e + 1] = __uint_as_float(yv[k][2 * e + 1]) + Dk[k] * bf16_hi(xr[k][e]);
+                }
+                uint8_t* tile = stg + k * 2 * TILE;
+                if (p.y_bf16) {
+#pragma unroll
+                    for (int qq = 0; qq < 2; ++qq)
+                        *reinterpret_cast<uint4*>(tile + swz(row, 2 * kq + qq)) = Vec16<bf16>::pack(out + 8 * qq);
+                } else {
+                    uint8_t* bx = tile + (kq >> 1) * TILE;     // columns 0-31 / 32-63: one box each
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+                        *reinterpret_cast<uint4*>(bx + swz(row, (kq & 1) * 4 + c)) = Vec16<float>::pack(out + 4 * c);
+                }
+            }
+            fence_proxy_async();
+            mbar_arrive(bar(B_STG0 + (jj & 1)));
+        }
+    }
+
+    if (err) atomicOr(p.dev_err, err);
+    tc_fence_before();
+    __syncthreads();
+    // after a wait gave up, copies or MMAs issued before it may still be in flight:
+    // let them drain (1 ms) before the shared memory and TMEM are released
+    if (*s_abort) {
+        const unsigned long long t_end = gtimer() + 1000000ull;
+        while (gtimer() < t_end) __nanosleep(1000);
+    }
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
+    }
+}
+
+}  // namespace pair
+
+bool pair_path_supports(int64_t batch, int64_t H, int64_t P, int64_t N, int64_t G, int64_t Q, bool io_bf16) {
+    // enough head pairs for every item to be a whole sequence on a part of 148 SMs
+    return io_bf16 && P == pair::PD && N == pair::NS && (Q == 128 || Q == 256) && (H / G) % 2 == 0 &&
+           batch * H >= 148;
+}
+
+cudaError_t launch_prefill_pair(const PrefillArgs& a, cudaStream_t s) {
+    using namespace pair;
+    if (!pair_path_supports(a.batch, a.H, a.P, a.N, a.G, a.Q, a.io_bf16)) return cudaErrorNotSupported;
+    CUtensorMap mx, mb, mc, my;
+    if (!tc::make_map(&my, a.y, (uint64_t)a.P, (uint64_t)a.H, (uint64_t)a.L, (uint64_t)a.batch, !a.y_bf16) ||
+        !tc::make_map(&mx, a.x, (uint64_t)a.P, (uint64_t)a.H, (uint64_t)a.L, (uint64_t)a.batch) ||
+        !tc::make_map(&mb, a.B, (uint64_t)a.N, (uint64_t)a.G, (uint64_t)a.L, (uint64_t)a.batch) ||
+        !tc::make_map(&mc, a.C, (uint64_t)a.N, (uint64_t)a.G, (uint64_t)a.L, (uint64_t)a.batch))
+        return cudaErrorInvalidValue;
+    static std::mutex mu;
+    static int sms_of[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        if (!sms_of[dev]) {
+            e = cudaFuncSetAttribute(ssd_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM);
+            if (e != cudaSuccess) return e;
+            int sms = 0;
+            e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+            if (e != cudaSuccess) return e;
+            sms_of[dev] = sms;
+        }
+    }
+    Params p{};
+    p.dtw = (const float*)(a.ws + a.lay.off_dt);
+    p.acsw = (const float*)(a.ws + a.lay.off_acs);
+    p.init_state = a.init_state;
+    p.final_state = a.final_state;
+    p.D = a.D;
+    p.dev_err = a.dev_err;
+    p.Lpad = a.lay.Lpad;
+    p.H = (int)a.H;
+    p.G = (int)a.G;
+    p.Q = (int)a.Q;
+    p.nblk = (int)((a.L + SUB - 1) / SUB);
+    const long long pairs = a.batch * a.H / 2;
+    const long long blocks = pairs * p.nblk;
+    if (pairs > 0x7fffffffLL || blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+    p.npairs = (int)pairs;
+    p.state_bf16 = a.state_bf16;
+    p.y_bf16 = a.y_bf16;
+    const unsigned grid = (unsigned)(pairs < sms_of[dev] ? pairs : sms_of[dev]);
+    // a programmatic dependent of the decay-cumsum kernel before it on the stream:
+    // the prologue and the first operand loads overlap that kernel; the producer
+    // waits for it (griddepcontrol.wait) before it reads dt and the cumsum
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(THREADS);
+    cfg.dynamicSmemBytes = SMEM;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, ssd_pair_kernel, mx, mb, mc, my, p);
+}
+
+}  // namespace ssd

@@ -46,26 +46,17 @@
 // word and a launch-wide abort word that ends every other hand-off wait at
 // once; the CTA then finishes its (in-bounds) work -- still waiting for its own
 // TMA and MMA completions -- and frees its TMEM.  Nothing traps.
-#include <cuda.h>
-#include <cudaTypedefs.h>
-
-#include <mutex>
-
-#include "ssd_common.cuh"
 #include "ssd_internal.h"
+#include "ssd_tc_common.cuh"
 
 namespace ssd {
 namespace tc {
 
-constexpr int SUB = 128;        // tokens per block (MMA M)
 constexpr int PD = 64;          // headdim handled by this path
 constexpr int NCOMPUTE = 256;   // compute threads of a pipeline: 8 warps; warps w and w+4 share TMEM lanes 32*(w%4)..+31
 // thread layout: warps 8p..8p+7 compute for pipeline p, then one control warp per
 // pipeline.  A warp may only touch TMEM lanes 32*(warp % 4), so compute warps
 // must start at a multiple of 4 warps: they come first.
-constexpr uint32_t TILE = SUB * 128;   // [128 rows x 64 bf16] SW128 tile = 16 KB
-constexpr float LOG2E = 1.4426950408889634f;
-constexpr unsigned long long WAIT_NS = 2000000000ull;   // bound of every device-side wait
 
 // TMEM columns of a pipeline
 constexpr uint32_t COL_R = 0;     // S (fp32 128) -> M hi|lo (bf16x2 64+64)
@@ -131,174 +122,6 @@ struct Params {
     int drop_publish;       // test hook: state items never publish (their successors time out)
 };
 
-// ---------------------------------------------------------------- PTX helpers
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-    return (uint32_t)__cvta_generic_to_shared(p);
-}
-__device__ __forceinline__ unsigned long long gtimer() {
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
-    return ok != 0;
-}
-__device__ __forceinline__ void fence_proxy_async() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_before() {
-    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* tm, int c0, int c1, int c2, int c3,
-                                            uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], [%6];"
-        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar)
-        : "memory");
-}
-// L2 prefetch of a tile (no shared-memory destination, no completion)
-__device__ __forceinline__ void tma_prefetch_4d(const CUtensorMap* tm, int c0, int c1, int c2, int c3) {
-    asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];"
-                 ::"l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(c2), "r"(c3) : "memory");
-}
-__device__ __forceinline__ void tma_store_4d(const CUtensorMap* tm, uint32_t src, int c0, int c1, int c2, int c3) {
-    asm volatile(
-        "cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];"
-        ::"l"(reinterpret_cast<uint64_t>(tm)), "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
-        : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-// 1-D bulk copy global -> shared (16-byte aligned addresses, size a multiple of 16)
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                 ::"r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
-}
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-__device__ __forceinline__ uint32_t elect_one() {
-    uint32_t p;
-    asm volatile("{\n .reg .pred P;\n elect.sync _|P, 0xffffffff;\n selp.u32 %0, 1, 0, P;\n}\n" : "=r"(p));
-    return p;
-}
-// 2^x on the SFU (approximate, flushes subnormal results to zero; 2^-inf = 0)
-__device__ __forceinline__ float ex2(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-// one tcgen05.mma (kind::f16, A and B from shared memory); IDESC and ACC are
-// compile-time constants so an issue costs the MMA and two address adds
-template <uint32_t IDESC, int ACC>
-__device__ __forceinline__ void mma_ss(uint32_t d, uint64_t a, uint64_t b) {
-    asm volatile(
-        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n"
-        ::"r"(d), "l"(a), "l"(b), "n"(IDESC), "n"(ACC) : "memory");
-}
-// one tcgen05.mma with the A operand in tensor memory
-template <uint32_t IDESC, int ACC>
-__device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a_tmem, uint64_t b) {
-    asm volatile(
-        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n"
-        ::"r"(d), "r"(a_tmem), "l"(b), "n"(IDESC), "n"(ACC) : "memory");
-}
-__device__ __forceinline__ void mma_commit(uint32_t bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
-}
-
-#define SSD_R8(i) "=r"(r[i]), "=r"(r[i + 1]), "=r"(r[i + 2]), "=r"(r[i + 3]), "=r"(r[i + 4]), "=r"(r[i + 5]), \
-                  "=r"(r[i + 6]), "=r"(r[i + 7])
-#define SSD_W8(i) "r"(r[i]), "r"(r[i + 1]), "r"(r[i + 2]), "r"(r[i + 3]), "r"(r[i + 4]), "r"(r[i + 5]), \
-                  "r"(r[i + 6]), "r"(r[i + 7])
-
-// 32 consecutive fp32 columns of this warp's 32 TMEM lanes (one row per thread)
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-        : SSD_R8(0), SSD_R8(8), SSD_R8(16), SSD_R8(24)
-        : "r"(taddr));
-}
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};"
-        ::"r"(taddr), SSD_W8(0), SSD_W8(8), SSD_W8(16), SSD_W8(24)
-        : "memory");
-}
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-        "%15}, [%16];"
-        : SSD_R8(0), SSD_R8(8)
-        : "r"(taddr));
-}
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-        "%15, %16};"
-        ::"r"(taddr), SSD_W8(0), SSD_W8(8)
-        : "memory");
-}
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-
-// Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version field.
-__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-    uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
-    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
-    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
-    d |= (uint64_t)1 << 46;
-    d |= (uint64_t)2 << 61;
-    return d;
-}
-// Instruction descriptor of kind::f16: bf16 x bf16 -> fp32, dense.
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int Nn, bool a_mn, bool b_mn) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
-           ((uint32_t)(Nn >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
-}
-
-// bf16 pair (lo element in the low half), round to nearest even
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-    __nv_bfloat162 t = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<uint32_t*>(&t);
-}
-__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
-
-// byte offset of 16-byte chunk `j` of row `r` in a 128-byte-swizzled tile
-__device__ __forceinline__ uint32_t swz(int r, int j) { return (uint32_t)(r * 128 + ((j ^ (r & 7)) << 4)); }
-
-// bounded wait on an mbarrier phase (a TMA or MMA completion); returns false
-// if it has not completed within WAIT_NS.  It never returns early on a chain
-// abort, so a CTA never leaves with its own copies or MMAs still in flight.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
-    uint32_t spins = 0;
-    unsigned long long deadline = 0;
-    while (!mbar_try(bar, parity)) {
-        if ((++spins & 1023u) == 0) {
-            const unsigned long long now = gtimer();
-            if (deadline == 0) deadline = now + WAIT_NS;
-            else if (now > deadline) return false;
-        }
-    }
-    return true;
-}
 
 // ---------------------------------------------------------------- the kernel
 // Persistent, one CTA per SM, Cfg::PIPES independent block pipelines per CTA.  A
@@ -929,36 +752,6 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
     }
 }
 
-// ---------------------------------------------------------------- host side
-static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    });
-    return fn;
-}
-
-// 4-D tensor map (inner, d1, d2, d3) with a {128 bytes, 1, 128, 1} box and
-// 128-byte swizzle: 64 bf16 or 32 fp32 elements per row of the box
-static bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t d1, uint64_t d2, uint64_t d3,
-                     bool fp32 = false) {
-    auto fn = encode_fn();
-    if (!fn) return false;
-    const uint64_t es = fp32 ? 4 : 2;
-    cuuint64_t dims[4] = {inner, d1, d2, d3};
-    cuuint64_t strides[3] = {inner * es, inner * d1 * es, inner * d1 * d2 * es};
-    cuuint32_t box[4] = {(cuuint32_t)(128 / es), 1, (cuuint32_t)SUB, 1};
-    cuuint32_t estr[4] = {1, 1, 1, 1};
-    return fn(m, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
-              const_cast<void*>(ptr), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
 
 template <int N>
 static cudaError_t launch_n(const PrefillArgs& a, cudaStream_t s) {
@@ -1061,6 +854,8 @@ bool tc_path_supports(int64_t P, int64_t N, int64_t Q, bool io_bf16) {
 
 cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
     if (!tc_path_supports(a.P, a.N, a.Q, a.io_bf16)) return cudaErrorNotSupported;
+    // pairs of heads sharing B and C, every item a whole sequence
+    if (pair_path_supports(a.batch, a.H, a.P, a.N, a.G, a.Q, a.io_bf16)) return launch_prefill_pair(a, s);
     switch (a.N) {
         case 64: return tc::launch_n<64>(a, s);
         case 128: return tc::launch_n<128>(a, s);

@@ -68,6 +68,11 @@ def test_workspace_size_and_path():
     assert n >= 2 * 4 * BH * Lpad + 4 * BH * 128 * 64
     assert ssd.ssd_chunk_scan_path(d) == 0                       # bf16, N=128: tensor cores
     assert ssd.ssd_chunk_scan_path(desc(io_dtype=ssd.SSD_F32)) == 1   # fp32: CUDA cores
+    # pairs of heads of a group once there are >= 148 sequences and an even number of heads per group
+    assert ssd.ssd_chunk_scan_path(desc(batch=2, nheads=74, ngroups=1)) == 2
+    assert ssd.ssd_chunk_scan_path(desc(batch=2, nheads=74, ngroups=74)) == 0      # one head per group
+    assert ssd.ssd_chunk_scan_path(desc(batch=1, nheads=146, ngroups=1)) == 0      # 146 sequences
+    assert ssd.ssd_chunk_scan_path(desc(batch=4, nheads=64, ngroups=1, dstate=64)) == 0
     # the CUDA-core path keeps one fp32 state per chunk
     n32 = ssd.ssd_chunk_scan_workspace_size(desc(io_dtype=ssd.SSD_F32))
     assert n32 >= 4 * BH * 2 * 128 * 64

@@ -55,6 +55,51 @@ def test_prefill_matches_oracle(case, with_init):
     assert metric(fs, fs_ref) <= tol
 
 
+# (b, L, H, G, chunk) of the head-pair kernel: dstate 128, an even number of heads
+# per group, >= 148 sequences
+PAIR_CASES = [
+    (1, 300, 148, 2, 256),    # 74 items, 3 blocks, ragged 44-token tail
+    (2, 520, 80, 4, 128),     # 80 items, chunk 128, an 8-token tail block
+    (1, 260, 400, 8, 128),    # 200 items on at most 148 CTAs: some CTAs take two
+]
+
+
+@pytest.mark.parametrize("case", PAIR_CASES, ids=lambda c: "b{}_L{}_H{}_G{}_Q{}".format(*c))
+@pytest.mark.parametrize("with_init", [False, True])
+def test_head_pair_path_matches_oracle(case, with_init):
+    b, L, H, G, Q = case
+    inp = shape_inputs(b, L, H, 64, 128, G, I.BF16, seed=41 + L)
+    assert path_of(inp, Q) == 2
+    h0 = random_state((b, H, 128, 64), 43 + L, I.F32) if with_init else None
+    y, fs = gpu_prefill(inp, Q, h0)
+    y_ref, fs_ref = oracle_prefill(inp, h0)
+    # same arithmetic as the single-head kernel: far inside the 2e-2 bound
+    assert metric(y, y_ref) < 2e-3
+    assert metric(fs, fs_ref) < 2e-3
+
+
+def test_head_pair_bf16_outputs_and_states():
+    inp = shape_inputs(2, 384, 80, 64, 128, 2, I.BF16, 23)
+    h0 = random_state((2, 80, 128, 64), 24, I.BF16)
+    y, fs = gpu_prefill(inp, 256, h0, y_dtype="bf16", state_dtype="bf16")
+    y_ref, fs_ref = oracle_prefill(inp, h0)
+    assert bf16_excess_metric(y, y_ref) <= TOL_BF16
+    assert bf16_excess_metric(fs, fs_ref) <= TOL_BF16
+
+
+def test_head_pair_positive_decay_exponent():
+    """A > 0 on some heads: the log-decay grows, and blocks of those pairs take the
+    per-element decay factors instead of the split ones."""
+    inp = shape_inputs(1, 400, 148, 64, 128, 2, I.BF16, 25)
+    A = inp["A"].copy()
+    A[[3, 4, 77]] = np.float32(0.02)
+    inp["A"] = A
+    y, fs = gpu_prefill(inp, 256)
+    y_ref, fs_ref = oracle_prefill(inp)
+    assert metric(y, y_ref) < 2e-3
+    assert metric(fs, fs_ref) < 2e-3
+
+
 @pytest.mark.parametrize("N", [64, 128, 256])
 def test_tensor_core_path_is_taken_for_bf16_headdim64(N):
     inp = shape_inputs(1, 256, 2, 64, N, 1, I.BF16, 3)
