@@ -310,14 +310,21 @@ ssd_status_t ssd_chunk_scan_mamba3_launches(const ssd_prefill_desc_t* desc, int3
  *
  * Arguments and results are exactly those of ssd_chunk_scan_fwd minus the
  * workspace.  The scratch is a fixed array of SSD_NOALLOC_WORKSPACE_BYTES in
- * the library's own device memory, reserved on every GPU that loads the
- * library until the process exits; nothing is allocated per call (no
+ * the library's own device memory; nothing is allocated per call (no
  * cudaMalloc, cudaFree or allocating library routine).
  *  - Problems whose ssd_chunk_scan_workspace_size exceeds the scratch are
  *    rejected with SSD_ERR_WORKSPACE before anything is launched (the 1.3B-
  *    shaped layer, batch 4 x 2048 tokens, needs about 12.6 MiB).
  *  - The first call with a given device current looks up the scratch's device
- *    address on that device; make that first call before any stream capture.
+ *    address on that device.  With the CUDA runtime's lazy module loading
+ *    (its default), that first lookup is also when the library's device code
+ *    is loaded on the device and the scratch is reserved, which may allocate
+ *    device memory and synchronise.  Make one warm-up call per device outside
+ *    any latency-critical region and before any stream capture; from then on
+ *    the scratch stays reserved on that device until the process exits.
+ *  - The address is kept for the life of the process: after cudaDeviceReset
+ *    (or anything else that destroys the device's primary context) it is
+ *    stale, so do not call this entry point again in that process.
  *  - Every call on a device shares the one scratch array, which keeps the last
  *    call's contents (the kernels reset what must start at zero themselves).
  *    Calls that overlap on the GPU -- on different streams, or from different

@@ -79,6 +79,9 @@ static PrefillLayout prefill_layout(const ssd_prefill_desc_t* d, bool tc) {
     off = align256(off + sizeof(float) * (size_t)BH * lay.Lpad);
     lay.off_acs = off;
     off = align256(off + sizeof(float) * (size_t)BH * lay.Lpad);
+    lay.off_acs_lo = off;
+    lay.has_lo = true;
+    off = align256(off + sizeof(float) * (size_t)BH * lay.Lpad);
     lay.off_states = off;
     const size_t state_elems = (size_t)d->dstate * d->headdim;
     // CUDA-core path: one state per chunk; tensor-core path: the entry state of

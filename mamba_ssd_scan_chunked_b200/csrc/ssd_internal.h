@@ -55,7 +55,9 @@ cudaError_t launch_mimo_step(const MimoArgs& a, cudaStream_t stream);
 struct PrefillLayout {
     int64_t nchunks;       // ceil(L / Q)
     int64_t Lpad;          // nchunks * Q
-    size_t off_dt, off_acs;        // fp32 [b][H][Lpad] each
+    size_t off_dt, off_acs;        // fp32 [b][H][Lpad] each; acs is the hi part of the cumsum
+    size_t off_acs_lo;             // fp32 [b][H][Lpad]: its lo part (when has_lo)
+    bool has_lo;                   // layouts of scans whose decays are written by other kernels have none
     size_t off_states;             // fp32 chunk states (CUDA-core path) or run-entry states
     size_t off_flags;              // int32 [b][H] run-entry states published + 64 control words
     size_t total;

@@ -6,8 +6,10 @@
 // buffers it was handed, for instance a plugin inside a host framework that
 // owns all device memory, or a latency-critical path where cudaMalloc (which
 // can synchronise the device) is not allowed.  This entry point instead uses a
-// fixed scratch array that lives in the library's own device memory, reserved
-// on every GPU that loads the library until the process exits.
+// fixed scratch array that lives in the library's own device memory.  It is
+// reserved on a device when the library's device code is loaded there (with
+// lazy module loading: at the first address lookup below) and stays until the
+// process exits.
 #include <mutex>
 
 #include "../../include/ssd.h"
@@ -24,7 +26,8 @@ static std::mutex g_noalloc_mutex;
 static void* g_noalloc_ptr[64];
 
 // Device address of the scratch on the current device (looked up on the first
-// call made with that device current, then cached).
+// call made with that device current, then cached for the life of the process:
+// a device reset would leave the cached address stale).
 static cudaError_t noalloc_scratch(void** out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);

@@ -34,6 +34,8 @@
 //   warp 17     TMA: operand loads (C, B double-buffered one block ahead), the
 //               y stores, which it stages in the C/B buffers of the block just
 //               finished
+// The per-token decay terms are read by the compute warps themselves, one block
+// ahead into registers, and turned into shared tables at the block's start.
 // Every wait on an mbarrier is bounded (2 s); the first one that gives up sets
 // the device error word and a CTA-wide abort word that ends every later wait
 // at once, so the launch always finishes.  No inter-CTA waits exist.
@@ -62,12 +64,13 @@ constexpr uint32_t STAGE = 4 * TILE;             // C (K blocks 0, 1), B (K bloc
 constexpr uint32_t OFF_X = 2 * STAGE;            // x of head 0, head 1
 constexpr uint32_t OFF_W = OFF_X + 2 * TILE;     // per head: hi, lo of h (C h), then of w o X (state)
 constexpr uint32_t TILES = OFF_W + 4 * TILE;
-constexpr uint32_t OFF_DT = TILES;               // [2][128] dt, turned into u_s = log2(dt_s) - r_s
-constexpr uint32_t OFF_ACS = OFF_DT + 2 * SUB * 4;     // [2][128] chunk-local cumsum (natural log)
+// per-token tables of the block (written by the compute warps; single buffer)
+constexpr uint32_t OFF_V = TILES;                // [2][128] v_s = log2(dt_s) + r_J - r_s (J: end of s's 16-token group)
 constexpr int NFAC = 96;                         // tokens whose group can lie before a row block
-constexpr uint32_t OFF_FAC = OFF_ACS + 2 * SUB * 4;    // [2][96] 2^(r_J - r_s) dt_s
-constexpr uint32_t OFF_BAR = OFF_FAC + 2 * NFAC * 4;
-enum { B_CB0, B_CB1, B_X, B_T, B_S, B_OFF, B_ST, B_Y0, B_Y, B_H, B_WX, B_M, B_EPI, B_STG0, B_STG1, NBAR };
+constexpr uint32_t OFF_FAC = OFF_V + 2 * SUB * 4;     // [2][96] 2^(v_s)
+constexpr uint32_t OFF_GE = OFF_FAC + 2 * NFAC * 4;   // [2][8] float2: cumsum (hi, lo) at the group ends
+constexpr uint32_t OFF_BAR = OFF_GE + 2 * 8 * 8;
+enum { B_CB0, B_CB1, B_X, B_S, B_OFF, B_ST, B_Y0, B_Y, B_H, B_WX, B_M, B_EPI, B_STG0, B_STG1, NBAR };
 constexpr uint32_t OFF_MISC = OFF_BAR + 8 * NBAR;      // TMEM base, abort word
 constexpr uint32_t SMEM = OFF_MISC + 16;
 static_assert(TILES % 1024 == 0 && OFF_BAR % 8 == 0, "alignment");
@@ -75,7 +78,8 @@ static_assert(SMEM <= 232448, "shared memory per CTA");
 
 struct Params {
     const float* dtw;          // [BH][Lpad] dt
-    const float* acsw;         // [BH][Lpad] chunk-local inclusive cumsum of dt*A
+    const float* acsw;         // [BH][Lpad] chunk-local inclusive cumsum of dt*A (hi part)
+    const float* acslo;        // [BH][Lpad] its lo part, or NULL (= 0)
     const void* init_state;    // [BH][N][P] state dtype or NULL
     void* final_state;         // [BH][N][P] state dtype or NULL
     const float* D;            // [H] or NULL
@@ -89,8 +93,8 @@ struct Params {
 __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, volatile int* abort) {
     uint32_t spins = 0;
     unsigned long long deadline = 0;
-    while (!mbar_try(bar, parity)) {
-        if ((++spins & 255u) == 0) {
+    while (!mbar_try_sleep(bar, parity, 100000u)) {
+        if ((++spins & 3u) == 0) {
             if (*abort) return false;
             const unsigned long long now = gtimer();
             if (deadline == 0) {
@@ -113,7 +117,8 @@ __device__ __forceinline__ void split8(const float* v, uint32_t (&hw)[4], uint32
     }
 }
 
-__global__ void __launch_bounds__(THREADS, 1)
+// 18 warps x 32 threads x 112 registers = 64512 of the SM's 65536
+__global__ void __maxnreg__(112)
 ssd_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmY, const Params p) {
     extern __shared__ __align__(1024) uint8_t sm[];
@@ -133,8 +138,8 @@ ssd_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     if (threadIdx.x == NCT) {
-        //                          CB0 CB1 X  T  S  OFF ST Y0 Y  H    WX       M    EPI  STG0 STG1
-        const uint32_t cnt[NBAR] = {1, 1, 1, 1, 1, 1, 1, 1, 1, NCT, NCT / 2, NCT, NCT, NCT, NCT};
+        //                          CB0 CB1 X  S  OFF ST Y0 Y  H    WX       M    EPI  STG0 STG1
+        const uint32_t cnt[NBAR] = {1, 1, 1, 1, 1, 1, 1, 1, NCT, NCT / 2, NCT, NCT, NCT, NCT};
         for (int i = 0; i < NBAR; ++i) mbar_init(bar(i), cnt[i]);
         *s_abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -185,29 +190,14 @@ ssd_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
             tma_load_4d(base + OFF_X, &tmX, 0, d.h0, t0, d.b, bar(B_X));
             tma_load_4d(base + OFF_X + TILE, &tmX, 0, d.h0 + 1, t0, d.b, bar(B_X));
         };
-        auto load_t = [&](int t) {           // dt and cumsum of both heads
-            const Item d = item_of(t / p.nblk);
-            const long long o = (long long)(d.b * p.H + d.h0) * p.Lpad + (long long)(t % p.nblk) * SUB;
-            mbar_expect_tx(bar(B_T), 4 * SUB * 4);
-            bulk_load(base + OFF_DT, p.dtw + o, SUB * 4, bar(B_T));
-            bulk_load(base + OFF_DT + SUB * 4, p.dtw + o + p.Lpad, SUB * 4, bar(B_T));
-            bulk_load(base + OFF_ACS, p.acsw + o, SUB * 4, bar(B_T));
-            bulk_load(base + OFF_ACS + SUB * 4, p.acsw + o + p.Lpad, SUB * 4, bar(B_T));
-        };
         if (lead && total > 0) {
             load_cb(0);
             if (total > 1) load_cb(1);
             load_x(0);
-            // dt and the cumsum come from the decay kernel this launch may overlap
-            // (programmatic dependent launch): wait for it before reading them
-            asm volatile("griddepcontrol.wait;" ::: "memory");
-            load_t(0);
         }
         for (int jj = 0; jj < total; ++jj) {
             const uint32_t ph = jj & 1;
-            wait(B_M, ph);                   // the block's dt / cumsum are consumed
-            if (lead && jj + 1 < total && !*s_abort) load_t(jj + 1);
-            wait(B_Y, ph);                   // its x is consumed
+            wait(B_Y, ph);                   // the block's x is consumed
             if (lead && jj + 1 < total && !*s_abort) load_x(jj + 1);
             wait(B_STG0 + (jj & 1), (jj >> 1) & 1);   // y staged in the block's C/B stage
             if (lead && !*s_abort) {
@@ -230,13 +220,14 @@ ssd_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
         // ======================================================== MMA issue
         const uint32_t lead = elect_one();
         constexpr uint32_t ID_S = idesc_bf16(128, 128, false, false);   // C (K-major) x B^T (K-major)
-        constexpr uint32_t ID_N64 = idesc_bf16(128, PD, false, true);   // C x h (MN-major); M (TMEM) x X (MN-major)
-        constexpr uint32_t ID_ST = idesc_bf16(128, PD, true, true);     // B^T (MN-major) x wX (MN-major)
+        constexpr uint32_t ID_Y = idesc_bf16(128, PD, false, true);     // M (TMEM) x X (MN-major)
+        // both heads at once: N = 128 columns = [head 0 | head 1] of the W tiles,
+        // whose 64-column halves lie 2 TILE apart (the leading byte offset)
+        constexpr uint32_t ID_OFF = idesc_bf16(128, 2 * PD, false, true);   // C (K-major) x [h_0 | h_1] (MN-major)
+        constexpr uint32_t ID_ST = idesc_bf16(128, 2 * PD, true, true);     // B^T (MN-major) x [wX_0 | wX_1]
         constexpr uint32_t KSTEP_K = 2, KBLOCK_K = TILE >> 4, KSTEP_MN = 2048 >> 4;
         const uint64_t dX0 = sdesc(base + OFF_X, TILE, 1024), dX1 = sdesc(base + OFF_X + TILE, TILE, 1024);
-        const uint64_t dW00 = sdesc(base + OFF_W, TILE, 1024), dW01 = sdesc(base + OFF_W + TILE, TILE, 1024);
-        const uint64_t dW10 = sdesc(base + OFF_W + 2 * TILE, TILE, 1024);
-        const uint64_t dW11 = sdesc(base + OFF_W + 3 * TILE, TILE, 1024);
+        const uint64_t dWhi = sdesc(base + OFF_W, 2 * TILE, 1024), dWlo = sdesc(base + OFF_W + TILE, 2 * TILE, 1024);
         const uint32_t lead0 = lead;
         for (int jj = 0; jj < total; ++jj) {
             const uint32_t ph = jj & 1;
@@ -265,19 +256,13 @@ ssd_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
 #pragma unroll
             for (int k = 0; k < NS / 16; ++k) {
                 const uint32_t o = (uint32_t)(k >> 2) * KBLOCK_K + (uint32_t)(k & 3) * KSTEP_K;
-                if (k == 0) {
-                    if (lead) mma_ss<ID_N64, 0>(tmem + COL_Y, dC, dW00);
-                    if (lead) mma_ss<ID_N64, 0>(tmem + COL_Y + 64, dC, dW10);
-                } else {
-                    if (lead) mma_ss<ID_N64, 1>(tmem + COL_Y, dC + o, dW00 + k * KSTEP_MN);
-                    if (lead) mma_ss<ID_N64, 1>(tmem + COL_Y + 64, dC + o, dW10 + k * KSTEP_MN);
-                }
+                if (k == 0) { if (lead) mma_ss<ID_OFF, 0>(tmem + COL_Y, dC, dWhi);
+                } else if (lead) mma_ss<ID_OFF, 1>(tmem + COL_Y, dC + o, dWhi + k * KSTEP_MN);
             }
 #pragma unroll
             for (int k = 0; k < NS / 16; ++k) {
                 const uint32_t o = (uint32_t)(k >> 2) * KBLOCK_K + (uint32_t)(k & 3) * KSTEP_K;
-                if (lead) mma_ss<ID_N64, 1>(tmem + COL_Y, dC + o, dW01 + k * KSTEP_MN);
-                if (lead) mma_ss<ID_N64, 1>(tmem + COL_Y + 64, dC + o, dW11 + k * KSTEP_MN);
+                if (lead) mma_ss<ID_OFF, 1>(tmem + COL_Y, dC + o, dWlo + k * KSTEP_MN);
             }
             if (lead) mma_commit(bar(B_OFF));
             // ---- state_k += B^T (w o X_k)_hi + B^T (w o X_k)_lo, onto 2^(r_last) h_k
@@ -285,15 +270,11 @@ ssd_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
             tc_fence_after();
             __syncwarp();
 #pragma unroll
-            for (int k = 0; k < SUB / 16; ++k) {
-                if (lead) mma_ss<ID_ST, 1>(tmem + COL_ST, dBm + k * KSTEP_MN, dW00 + k * KSTEP_MN);
-                if (lead) mma_ss<ID_ST, 1>(tmem + COL_ST + 64, dBm + k * KSTEP_MN, dW10 + k * KSTEP_MN);
-            }
+            for (int k = 0; k < SUB / 16; ++k)
+                if (lead) mma_ss<ID_ST, 1>(tmem + COL_ST, dBm + k * KSTEP_MN, dWhi + k * KSTEP_MN);
 #pragma unroll
-            for (int k = 0; k < SUB / 16; ++k) {
-                if (lead) mma_ss<ID_ST, 1>(tmem + COL_ST, dBm + k * KSTEP_MN, dW01 + k * KSTEP_MN);
-                if (lead) mma_ss<ID_ST, 1>(tmem + COL_ST + 64, dBm + k * KSTEP_MN, dW11 + k * KSTEP_MN);
-            }
+            for (int k = 0; k < SUB / 16; ++k)
+                if (lead) mma_ss<ID_ST, 1>(tmem + COL_ST, dBm + k * KSTEP_MN, dWlo + k * KSTEP_MN);
             if (lead) mma_commit(bar(B_ST));
             // ---- Y_k += M_k,hi X_k + M_k,lo X_k onto the scaled Yoff (A from TMEM)
             wait(B_M, ph);
@@ -301,14 +282,14 @@ ssd_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
             __syncwarp();
 #pragma unroll
             for (int k = 0; k < SUB / 16; ++k) {
-                if (lead) mma_ts<ID_N64, 1>(tmem + COL_Y, tmem + COL_R0 + 16 * k, dX0 + k * KSTEP_MN);
-                if (lead) mma_ts<ID_N64, 1>(tmem + COL_Y, tmem + COL_R0 + 16 * k + 8, dX0 + k * KSTEP_MN);
+                if (lead) mma_ts<ID_Y, 1>(tmem + COL_Y, tmem + COL_R0 + 16 * k, dX0 + k * KSTEP_MN);
+                if (lead) mma_ts<ID_Y, 1>(tmem + COL_Y, tmem + COL_R0 + 16 * k + 8, dX0 + k * KSTEP_MN);
             }
             if (lead) mma_commit(bar(B_Y0));
 #pragma unroll
             for (int k = 0; k < SUB / 16; ++k) {
-                if (lead) mma_ts<ID_N64, 1>(tmem + COL_Y + 64, tmem + COL_R1 + 16 * k, dX1 + k * KSTEP_MN);
-                if (lead) mma_ts<ID_N64, 1>(tmem + COL_Y + 64, tmem + COL_R1 + 16 * k + 8, dX1 + k * KSTEP_MN);
+                if (lead) mma_ts<ID_Y, 1>(tmem + COL_Y + 64, tmem + COL_R1 + 16 * k, dX1 + k * KSTEP_MN);
+                if (lead) mma_ts<ID_Y, 1>(tmem + COL_Y + 64, tmem + COL_R1 + 16 * k + 8, dX1 + k * KSTEP_MN);
             }
             if (lead) mma_commit(bar(B_Y));
             __syncwarp();
@@ -319,104 +300,144 @@ ssd_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
         const int row = 32 * q + lane;                // TMEM lane = tile row
         const uint32_t lo16 = (uint32_t)(32 * q) << 16;
         const float NEG_INF = __int_as_float(0xff800000u);
-        float* s_u = reinterpret_cast<float*>(sm + OFF_DT);          // [2][128] dt -> u
-        const float* s_acs = reinterpret_cast<const float*>(sm + OFF_ACS);
+        float* s_v = reinterpret_cast<float*>(sm + OFF_V);           // [2][128]
         float* s_fac = reinterpret_cast<float*>(sm + OFF_FAC);       // [2][96]
-        float prev_last[2] = {0.f, 0.f};
-        int it = -1, j = p.nblk - 1;
-        Item d{};
-        float Dk[2] = {0.f, 0.f};
-        for (int jj = 0; jj < total; ++jj) {
-            if (++j == p.nblk) {
-                j = 0;
-                d = item_of(++it);
-                Dk[0] = p.D ? p.D[d.h0] : 0.f;
-                Dk[1] = p.D ? p.D[d.h0 + 1] : 0.f;
-            }
-            const uint32_t ph = jj & 1;
-            const bool chunk_start = ((j * SUB) & (p.Q - 1)) == 0;   // the cumsum restarts at every chunk
-            const long long bh0 = (long long)d.b * p.H + d.h0;
+        float2* s_ge = reinterpret_cast<float2*>(sm + OFF_GE);       // [2][8]
+        // the workspace's dt and cumsum come from the decay kernel this launch may overlap
+        asm volatile("griddepcontrol.wait;" ::: "memory");
 
-            // ---- per-token terms: r (log2, relative to the block start) of this
-            // thread's row, u_s = log2(dt_s) - r_s and the off-diagonal factors
-            wait(B_T, ph);
-            float r0[2], rl[2], rlast[2];
+        // the cumsum of (bh, token t) as its (hi, lo) pair
+        auto cum = [&](long long bh, long long t) -> float2 {
+            const long long o = bh * p.Lpad + t;
+            return make_float2(__ldcg(p.acsw + o), p.acslo ? __ldcg(p.acslo + o) : 0.f);
+        };
+        // log2 of exp(a - b) for two cumsum pairs: the hi difference is exact when it is
+        // small next to the values, the only case where the factor is not negligible
+        auto dl2 = [](float2 a, float2 b) -> float { return ((a.x - b.x) + (a.y - b.y)) * LOG2E; };
+
+        // h entering a block, for both heads: the initial state (first block of an
+        // item) or the state the previous block left in TMEM.  2^(r_last) h goes back
+        // into the state accumulator; h is split hi -> W tile, lo -> W tile + TILE for C h.
+        auto h_enter = [&](bool first, long long bh, const float (&rlast)[2]) {
 #pragma unroll
             for (int k = 0; k < 2; ++k) {
-                r0[k] = chunk_start ? 0.f : prev_last[k];
-                rl[k] = (s_acs[k * SUB + row] - r0[k]) * LOG2E;
-                rlast[k] = (s_acs[k * SUB + SUB - 1] - r0[k]) * LOG2E;
-            }
-            uint32_t inc = 0;                 // a log-decay that increases somewhere in the block
-            if (kq < 2) {
-                const int k = kq;
-                const float a_prev = row ? s_acs[k * SUB + row - 1] : r0[k];
-                inc = s_acs[k * SUB + row] > a_prev;
-                const float dtv = s_u[k * SUB + row];
-                const float u = (dtv > 0.f ? __log2f(dtv) : NEG_INF) - rl[k];
-                s_u[k * SUB + row] = u;       // in place: this thread alone reads and writes it
-                if (row < NFAC) s_fac[k * NFAC + row] = ex2((s_acs[k * SUB + (row | 15)] - r0[k]) * LOG2E + u);
-            }
-            prev_last[0] = s_acs[SUB - 1];
-            prev_last[1] = s_acs[2 * SUB - 1];
-            uint32_t direct;
-            asm volatile("{\n .reg .pred pi, po;\n setp.ne.u32 pi, %1, 0;\n bar.red.or.pred po, 1, %2, pi;\n"
-                         " selp.u32 %0, 1, 0, po;\n}\n"
-                         : "=r"(direct) : "r"(inc), "n"(NCT) : "memory");
-
-            // ---- h entering the block (the initial state, or what the previous
-            // block left in TMEM): 2^(r_last) h back into the state accumulator,
-            // h split hi -> W tile, lo -> W tile + TILE for C h
-            if (jj > 0) wait(B_ST, ph ^ 1u);  // previous state MMAs done (also frees W)
-            tc_fence_after();
-#pragma unroll
-            for (int k = 0; k < 2; ++k) {
-                const uint32_t col = COL_ST + 64 * k + 16 * kq;
-                float hv[16];
-                if (j > 0) {
-                    uint32_t v[16];
-                    tmem_ld16(tmem + lo16 + col, v);
+                uint32_t hv[16];
+                if (!first) {
+                    tmem_ld16(tmem + lo16 + COL_ST + 64 * k + 16 * kq, hv);
                     tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) hv[i] = __uint_as_float(v[i]);
                 } else if (p.init_state) {
-                    const long long o = ((bh0 + k) * NS + row) * PD + 16 * kq;
+                    float f[16];
+                    const long long o = ((bh + k) * NS + row) * PD + 16 * kq;
                     if (p.state_bf16) {
-                        Vec16<bf16>::load(reinterpret_cast<const bf16*>(p.init_state) + o, hv);
-                        Vec16<bf16>::load(reinterpret_cast<const bf16*>(p.init_state) + o + 8, hv + 8);
+                        Vec16<bf16>::load(reinterpret_cast<const bf16*>(p.init_state) + o, f);
+                        Vec16<bf16>::load(reinterpret_cast<const bf16*>(p.init_state) + o + 8, f + 8);
                     } else {
 #pragma unroll
                         for (int i = 0; i < 16; i += 4)
-                            Vec16<float>::load(reinterpret_cast<const float*>(p.init_state) + o + i, hv + i);
+                            Vec16<float>::load(reinterpret_cast<const float*>(p.init_state) + o + i, f + i);
                     }
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) hv[i] = __float_as_uint(f[i]);
                 } else {
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) hv[i] = 0.f;
+                    for (int i = 0; i < 16; ++i) hv[i] = 0u;
                 }
                 const float dl = ex2(rlast[k]);
-                uint32_t sc[16];
+                const f32x2 dl2v = f2_pack(dl, dl);
+                uint32_t sc[16], hw[8], lw[8];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) sc[i] = __float_as_uint(dl * hv[i]);
-                tmem_st16(tmem + lo16 + col, sc);
+                for (int i = 0; i < 8; ++i) {
+                    const f32x2 h2 = f2_pack_u(hv[2 * i], hv[2 * i + 1]);
+                    float a, b;
+                    f2_unpack(f2_mul(dl2v, h2), a, b);
+                    sc[2 * i] = __float_as_uint(a);
+                    sc[2 * i + 1] = __float_as_uint(b);
+                    split2(h2, hw[i], lw[i]);
+                }
+                tmem_st16(tmem + lo16 + COL_ST + 64 * k + 16 * kq, sc);
                 uint8_t* wt = sm + OFF_W + k * 2 * TILE;
 #pragma unroll
                 for (int qq = 0; qq < 2; ++qq) {
-                    uint32_t hw[4], lw[4];
-                    split8(hv + 8 * qq, hw, lw);
                     const uint32_t o = swz(row, 2 * kq + qq);
-                    *reinterpret_cast<uint4*>(wt + o) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-                    *reinterpret_cast<uint4*>(wt + TILE + o) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+                    *reinterpret_cast<uint4*>(wt + o) = make_uint4(hw[4 * qq], hw[4 * qq + 1], hw[4 * qq + 2], hw[4 * qq + 3]);
+                    *reinterpret_cast<uint4*>(wt + TILE + o) =
+                        make_uint4(lw[4 * qq], lw[4 * qq + 1], lw[4 * qq + 2], lw[4 * qq + 3]);
                 }
             }
             tmem_wait_st();
             fence_proxy_async();
             tc_fence_before();
             mbar_arrive(bar(B_H));
+        };
+
+        // this thread's per-token data of a block, read from the workspace one block
+        // ahead: the cumsum of its row's token for both heads; for the table threads
+        // (kq < 2: head kq, token = row) also dt and the cumsum of the token before
+        struct Pre { float2 row[2]; float dt; float2 prev; };
+        auto fetch = [&](const Item& dd, int jb, Pre& r) {
+            const long long bh = (long long)dd.b * p.H + dd.h0;
+            const long long t = (long long)jb * SUB + row;
+            r.row[0] = cum(bh, t);
+            r.row[1] = cum(bh + 1, t);
+            if (kq < 2) {
+                r.dt = __ldcg(p.dtw + (bh + kq) * p.Lpad + t);
+                r.prev = row ? cum(bh + kq, t - 1) : make_float2(0.f, 0.f);
+            }
+        };
+
+        float2 ref[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};   // cumsum at the previous block's end
+        int it = 0, j = 0;
+        Item d = total > 0 ? item_of(0) : Item{};
+        Pre cur{};
+        if (total > 0) fetch(d, 0, cur);
+        for (int jj = 0; jj < total; ++jj) {
+            const uint32_t ph = jj & 1;
+            const bool chunk_start = ((j * SUB) & (p.Q - 1)) == 0;   // the cumsum restarts at every chunk
+            const long long bh0 = (long long)d.b * p.H + d.h0;
+            const float Dk[2] = {p.D ? p.D[d.h0] : 0.f, p.D ? p.D[d.h0 + 1] : 0.f};
+            int it_n = it, j_n = j + 1;
+            if (j_n == p.nblk) { j_n = 0; ++it_n; }
+            const bool has_next = jj + 1 < total;
+            const Item d_n = has_next ? (j_n == 0 ? item_of(it_n) : d) : d;
+            const long long bh0_n = (long long)d_n.b * p.H + d_n.h0;
+
+            // ---- per-token tables of the block.  Token s of head k: v_s = log2(dt_s)
+            // + log2 exp(acs_J - acs_s) with J the last token of s's 16-token group,
+            // and 2^(v_s); the cumsum pairs at the group ends
+            float2 r0[2];
+#pragma unroll
+            for (int k = 0; k < 2; ++k) r0[k] = chunk_start ? make_float2(0.f, 0.f) : ref[k];
+            uint32_t inc = 0;                 // a log-decay that increases somewhere in the block
+            if (kq < 2) {
+                const int k = kq;
+                const float2 me = cur.row[k];
+                inc = dl2(me, row ? cur.prev : r0[k]) > 0.f;
+                const float2 ge = make_float2(__shfl_sync(0xffffffffu, me.x, lane | 15),
+                                              __shfl_sync(0xffffffffu, me.y, lane | 15));
+                const float v = (cur.dt > 0.f ? __log2f(cur.dt) : NEG_INF) + dl2(ge, me);
+                s_v[k * SUB + row] = v;
+                if (row < NFAC) s_fac[k * NFAC + row] = ex2(v);
+                if ((row & 15) == 15) s_ge[k * 8 + (row >> 4)] = me;
+            }
+            uint32_t direct;
+            asm volatile("{\n .reg .pred pi, po;\n setp.ne.u32 pi, %1, 0;\n bar.red.or.pred po, 1, %2, pi;\n"
+                         " selp.u32 %0, 1, 0, po;\n}\n"
+                         : "=r"(direct) : "r"(inc), "n"(NCT) : "memory");
+            float rl[2], rlast[2];            // log2 decay of this row / of the whole block from its start
+            float2 g127[2];
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                g127[k] = s_ge[k * 8 + 7];
+                rl[k] = dl2(cur.row[k], r0[k]);
+                rlast[k] = dl2(g127[k], r0[k]);
+            }
+            if (jj == 0) h_enter(true, bh0, rlast);   // later blocks: entered during the previous one
 
             // ---- M_k = S o [s<=l] 2^(r_l - r_s) dt_s, written as bf16 hi/lo per K step:
             // hi to columns [16g, 16g+8), lo to [16g+8, 16g+16) of R0 (head 0, in place
             // over S) and R1 (head 1).  Quarter q needs column groups g < 2q+2; the
-            // rest is zero.  Groups g < 2q lie before every row of the quarter.
+            // rest is zero.  Groups g < 2q lie before every row of the quarter:
+            // factor 2^(r_l - r_J) 2^(v_s); the others 2^(r_l - r_J + v_s), masked.
             wait(B_S, ph);
             tc_fence_after();
 #pragma unroll
@@ -437,46 +458,45 @@ ssd_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                 const bool before = g < 2 * q && !direct;
 #pragma unroll
                 for (int k = 0; k < 2; ++k) {
+                    const float lf = dl2(cur.row[k], s_ge[k * 8 + g]);   // log2 decay from the group end to the row
                     uint32_t o[16];
                     if (before) {
-                        const float f = ex2(rl[k] - (s_acs[k * SUB + c0 + 15] - r0[k]) * LOG2E);
+                        const float f = ex2(lf);
+                        const f32x2 ff = f2_pack(f, f);
                         const float4* fb = reinterpret_cast<const float4*>(s_fac + k * NFAC + c0);
 #pragma unroll
                         for (int i4 = 0; i4 < 4; ++i4) {
                             const float4 bv = fb[i4];
-                            const float bb[4] = {bv.x, bv.y, bv.z, bv.w};
-#pragma unroll
-                            for (int e = 0; e < 2; ++e) {
-                                const int i = 2 * i4 + e;
-                                const float m0 = __uint_as_float(v[2 * i]) * (f * bb[2 * e]);
-                                const float m1 = __uint_as_float(v[2 * i + 1]) * (f * bb[2 * e + 1]);
-                                const uint32_t hi = pack_bf16(m0, m1);
-                                o[i] = hi;
-                                o[8 + i] = pack_bf16(m0 - bf16_lo(hi), m1 - bf16_hi(hi));
-                            }
+                            const f32x2 w01 = f2_mul(ff, f2_pack(bv.x, bv.y)), w23 = f2_mul(ff, f2_pack(bv.z, bv.w));
+                            split2(f2_mul(f2_pack_u(v[4 * i4], v[4 * i4 + 1]), w01), o[2 * i4], o[8 + 2 * i4]);
+                            split2(f2_mul(f2_pack_u(v[4 * i4 + 2], v[4 * i4 + 3]), w23), o[2 * i4 + 1], o[9 + 2 * i4]);
                         }
                     } else {
-                        const float4* uu = reinterpret_cast<const float4*>(s_u + k * SUB + c0);
+                        const float4* vv = reinterpret_cast<const float4*>(s_v + k * SUB + c0);
 #pragma unroll
                         for (int i4 = 0; i4 < 4; ++i4) {
-                            const float4 uv = uu[i4];
+                            const float4 uv = vv[i4];
                             const float ub[4] = {uv.x, uv.y, uv.z, uv.w};
+                            float e[4];
 #pragma unroll
-                            for (int e = 0; e < 2; ++e) {
-                                const int i = 2 * i4 + e;
-                                const int s0 = (int)c0 + 2 * i;
-                                const float e0 = ex2(s0 <= row ? rl[k] + ub[2 * e] : NEG_INF);
-                                const float e1 = ex2(s0 + 1 <= row ? rl[k] + ub[2 * e + 1] : NEG_INF);
-                                const float m0 = __uint_as_float(v[2 * i]) * e0;
-                                const float m1 = __uint_as_float(v[2 * i + 1]) * e1;
-                                const uint32_t hi = pack_bf16(m0, m1);
-                                o[i] = hi;
-                                o[8 + i] = pack_bf16(m0 - bf16_lo(hi), m1 - bf16_hi(hi));
-                            }
+                            for (int t = 0; t < 4; ++t)
+                                e[t] = ex2((int)c0 + 4 * i4 + t <= row ? lf + ub[t] : NEG_INF);
+                            split2(f2_mul(f2_pack_u(v[4 * i4], v[4 * i4 + 1]), f2_pack(e[0], e[1])),
+                                   o[2 * i4], o[8 + 2 * i4]);
+                            split2(f2_mul(f2_pack_u(v[4 * i4 + 2], v[4 * i4 + 3]), f2_pack(e[2], e[3])),
+                                   o[2 * i4 + 1], o[9 + 2 * i4]);
                         }
                     }
                     tmem_st16(tmem + lo16 + (k ? COL_R1 : COL_R0) + c0, o);
                 }
+            }
+            // the next block's per-token data, while this block's work goes on
+            Pre nxt{};
+            if (has_next) fetch(d_n, j_n, nxt);
+            float2 t127n[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+            if (has_next) {
+                t127n[0] = cum(bh0_n, (long long)j_n * SUB + SUB - 1);
+                t127n[1] = cum(bh0_n + 1, (long long)j_n * SUB + SUB - 1);
             }
 
             // ---- after C h: w o X into the W tiles (quarters 0 and 1: one token row of
@@ -487,7 +507,8 @@ ssd_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                 wait(B_X, ph);
                 const int t = kq * 64 + q * 32 + lane;
                 const int s_ = t & (SUB - 1), k = t >> 7;
-                const float wv = ex2(rlast[k] + s_u[k * SUB + s_]);
+                const float wv = ex2(dl2(s_ge[k * 8 + 7], s_ge[k * 8 + (s_ >> 4)]) + s_v[k * SUB + s_]);
+                const f32x2 w2 = f2_pack(wv, wv);
                 const uint8_t* xt = sm + OFF_X + k * TILE;
                 uint8_t* wt = sm + OFF_W + k * 2 * TILE;
 #pragma unroll
@@ -495,30 +516,33 @@ ssd_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                     const uint32_t o = swz(s_, c);
                     const uint4 xv = *reinterpret_cast<const uint4*>(xt + o);
                     const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-                    float pv[8];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        pv[2 * e] = bf16_lo(xw[e]) * wv;
-                        pv[2 * e + 1] = bf16_hi(xw[e]) * wv;
-                    }
                     uint32_t hw[4], lw[4];
-                    split8(pv, hw, lw);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) split2(f2_mul(bf16x2_to_f2(xw[e]), w2), hw[e], lw[e]);
                     *reinterpret_cast<uint4*>(wt + o) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
                     *reinterpret_cast<uint4*>(wt + TILE + o) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
                 }
                 fence_proxy_async();
                 mbar_arrive(bar(B_WX));
             }
-#pragma unroll
-            for (int k = 0; k < 2; ++k) {
-                const uint32_t col = COL_Y + 64 * k + 16 * kq;
-                const float el = ex2(rl[k]);
-                uint32_t v[16];
-                tmem_ld16(tmem + lo16 + col, v);
+            {
+                uint32_t v[2][16];
+                tmem_ld16(tmem + lo16 + COL_Y + 16 * kq, v[0]);
+                tmem_ld16(tmem + lo16 + COL_Y + 64 + 16 * kq, v[1]);
                 tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(el * __uint_as_float(v[i]));
-                tmem_st16(tmem + lo16 + col, v);
+                for (int k = 0; k < 2; ++k) {
+                    const float el = ex2(rl[k]);
+                    const f32x2 e2 = f2_pack(el, el);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        float a, b;
+                        f2_unpack(f2_mul(e2, f2_pack_u(v[k][2 * i], v[k][2 * i + 1])), a, b);
+                        v[k][2 * i] = __float_as_uint(a);
+                        v[k][2 * i + 1] = __float_as_uint(b);
+                    }
+                    tmem_st16(tmem + lo16 + COL_Y + 64 * k + 16 * kq, v[k]);
+                }
             }
             if (q >= 2) wait(B_X, ph);
             uint32_t xr[2][8];
@@ -534,19 +558,21 @@ ssd_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
             tc_fence_before();
             mbar_arrive(bar(B_M));
 
-            // ---- after Y: the final state (last block), then y = Y + D x staged in the
-            // block's C/B stage (dead once every MMA of the block is done) for the TMA store
-            wait(B_Y, ph);
+            // ---- once this block's state MMAs are done: the final state (last block of
+            // an item), then the next block's entering state -- ahead of this block's
+            // output, so that its C h can follow Y at once
+            if (has_next || j == p.nblk - 1) wait(B_ST, ph);
             tc_fence_after();
             if (j == p.nblk - 1 && p.final_state) {
+                uint32_t sv[2][16];
+                tmem_ld16(tmem + lo16 + COL_ST + 16 * kq, sv[0]);
+                tmem_ld16(tmem + lo16 + COL_ST + 64 + 16 * kq, sv[1]);
+                tmem_wait_ld();
 #pragma unroll
                 for (int k = 0; k < 2; ++k) {
-                    uint32_t sv[16];
-                    tmem_ld16(tmem + lo16 + COL_ST + 64 * k + 16 * kq, sv);
-                    tmem_wait_ld();
                     float ho[16];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) ho[i] = __uint_as_float(sv[i]);
+                    for (int i = 0; i < 16; ++i) ho[i] = __uint_as_float(sv[k][i]);
                     const long long o = ((bh0 + k) * NS + row) * PD + 16 * kq;
                     if (p.state_bf16) {
                         bf16* fs = reinterpret_cast<bf16*>(p.final_state) + o;
@@ -559,6 +585,18 @@ ssd_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                     }
                 }
             }
+            if (has_next) {
+                const bool cs_n = j_n == 0 || ((j_n * SUB) & (p.Q - 1)) == 0;
+                float rlast_n[2];
+#pragma unroll
+                for (int k = 0; k < 2; ++k) rlast_n[k] = dl2(t127n[k], cs_n ? make_float2(0.f, 0.f) : g127[k]);
+                h_enter(j_n == 0, bh0_n, rlast_n);
+            }
+
+            // ---- after Y: y = Y + D x staged in the block's C/B stage (dead once every
+            // MMA of the block is done) for the TMA store
+            wait(B_Y, ph);
+            tc_fence_after();
             uint32_t yv[2][16];
             tmem_ld16(tmem + lo16 + COL_Y + 16 * kq, yv[0]);
             tmem_ld16(tmem + lo16 + COL_Y + 64 + 16 * kq, yv[1]);
@@ -569,11 +607,11 @@ ssd_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
 #pragma unroll
             for (int k = 0; k < 2; ++k) {
                 float out[16];
+                const f32x2 dd = f2_pack(Dk[k], Dk[k]);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    out[2 * e] = __uint_as_float(yv[k][2 * e]) + Dk[k] * bf16_lo(xr[k][e]);
-                    out[2 * e + 1] = __uint_as_float(yv[k][2 * e + 1]) + Dk[k] * bf16_hi(xr[k][e]);
-                }
+                for (int e = 0; e < 8; ++e)
+                    f2_unpack(f2_fma(dd, bf16x2_to_f2(xr[k][e]), f2_pack_u(yv[k][2 * e], yv[k][2 * e + 1])),
+                              out[2 * e], out[2 * e + 1]);
                 uint8_t* tile = stg + k * 2 * TILE;
                 if (p.y_bf16) {
 #pragma unroll
@@ -588,6 +626,12 @@ ssd_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
             }
             fence_proxy_async();
             mbar_arrive(bar(B_STG0 + (jj & 1)));
+            ref[0] = g127[0];
+            ref[1] = g127[1];
+            cur = nxt;
+            it = it_n;
+            j = j_n;
+            d = d_n;
         }
     }
 
@@ -644,6 +688,7 @@ cudaError_t launch_prefill_pair(const PrefillArgs& a, cudaStream_t s) {
     Params p{};
     p.dtw = (const float*)(a.ws + a.lay.off_dt);
     p.acsw = (const float*)(a.ws + a.lay.off_acs);
+    p.acslo = a.lay.has_lo ? (const float*)(a.ws + a.lay.off_acs_lo) : nullptr;
     p.init_state = a.init_state;
     p.final_state = a.final_state;
     p.D = a.D;

@@ -6,7 +6,15 @@
 // recombined), per (batch b, head h), chunk c of Q tokens, l, s in [0, Q):
 //
 //   dt_cumsum   : dt_s = softplus(dt_raw_s + dt_bias), acs_l = sum_{k<=l} dt_k A
-//                 (chunk-local, inclusive).  Shared with the tensor-core path.
+//                 (chunk-local, inclusive), summed in fp64 and stored as an fp32
+//                 pair hi + lo.  Shared with the tensor-core path.
+//
+// Decay factors are exponentials of cumsum differences, exp(acs_l - acs_s).
+// With strong decays the cumsum of a chunk reaches magnitudes of 10^4, where
+// one fp32 rounding of acs is worth 1e-3 in the exponent; differences are
+// therefore formed as (hi_l - hi_s) + (lo_l - lo_s), which is exact in its
+// first term whenever the difference is small next to the values (the only
+// case where the factor is not negligibly small).
 //   chunk_state : S_c[n,p] = sum_s B_s[n] exp(acs_{Q-1} - acs_s) dt_s x_s[p]
 //   state_pass  : h_in[0] = init_state, h_in[c+1] = exp(acs_{Q-1}) h_in[c] + S_c
 //                 (sequential fp32 scan over chunks); final_state = h_in[nc]
@@ -37,9 +45,10 @@ template <typename IoT>
 __global__ void __launch_bounds__(256)
 dt_cumsum_kernel(const IoT* __restrict__ dt_raw, const float* __restrict__ dt_bias,
                  const float* __restrict__ A, float* __restrict__ dt_out,
-                 float* __restrict__ acs_out, int* __restrict__ flags, const int32_t* __restrict__ pad_left,
+                 float* __restrict__ acs_out, float* __restrict__ acs_lo_out, int* __restrict__ flags,
+                 const int32_t* __restrict__ pad_left,
                  int64_t L, int64_t Lpad, int H, int Q, int nflags, int nchunks, int hgroups) {
-    __shared__ float warp_tot[8][DT_HG];       // Q <= 256: at most 8 warps
+    __shared__ double warp_tot[8][DT_HG];      // Q <= 256: at most 8 warps
     const int hg = (int)(blockIdx.x % (unsigned)hgroups);
     const int c = (int)((blockIdx.x / (unsigned)hgroups) % (unsigned)nchunks);
     const int b = (int)(blockIdx.x / ((unsigned)hgroups * (unsigned)nchunks));
@@ -56,19 +65,20 @@ dt_cumsum_kernel(const IoT* __restrict__ dt_raw, const float* __restrict__ dt_bi
 #pragma unroll
     for (int k = 0; k < DT_HG; ++k)
         raw[k] = (live && h0 + k < H) ? to_f32(dt_raw[((int64_t)b * L + t) * H + h0 + k]) : 0.f;
-    float dt[DT_HG], v[DT_HG];
+    float dt[DT_HG];
+    double v[DT_HG];
 #pragma unroll
     for (int k = 0; k < DT_HG; ++k) {
         const int h = h0 + k;
         dt[k] = (live && h < H) ? softplus_f32(raw[k] + (dt_bias ? dt_bias[h] : 0.f)) : 0.f;
-        v[k] = h < H ? dt[k] * A[h] : 0.f;
+        v[k] = h < H ? (double)dt[k] * (double)A[h] : 0.0;   // the product of two fp32 values is exact
     }
-    // inclusive scan over the tokens, DT_HG columns at once
+    // inclusive scan over the tokens in fp64, DT_HG columns at once
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
 #pragma unroll
         for (int k = 0; k < DT_HG; ++k) {
-            const float u = __shfl_up_sync(0xffffffffu, v[k], o);
+            const double u = __shfl_up_sync(0xffffffffu, v[k], o);
             if (lane >= o) v[k] += u;
         }
     }
@@ -85,7 +95,9 @@ dt_cumsum_kernel(const IoT* __restrict__ dt_raw, const float* __restrict__ dt_bi
             if (h0 + k >= H) break;
             const int64_t o = ((int64_t)b * H + h0 + k) * Lpad + t;
             dt_out[o] = dt[k];
-            acs_out[o] = v[k];
+            const float hi = (float)v[k];
+            acs_out[o] = hi;
+            if (acs_lo_out) acs_lo_out[o] = (float)(v[k] - (double)hi);
         }
     }
     // reset the run hand-off flags and control words of this launch (a slice per block)
@@ -98,6 +110,7 @@ template <typename IoT>
 static cudaError_t launch_dt_t(const PrefillArgs& a, cudaStream_t s) {
     float* dt = (float*)(a.ws + a.lay.off_dt);
     float* acs = (float*)(a.ws + a.lay.off_acs);
+    float* acs_lo = a.lay.has_lo ? (float*)(a.ws + a.lay.off_acs_lo) : nullptr;
     int* flags = (int*)(a.ws + a.lay.off_flags);
     const int nflags = (int)(a.batch * a.H + 64);
     const int hgroups = (int)((a.H + DT_HG - 1) / DT_HG);
@@ -105,7 +118,8 @@ static cudaError_t launch_dt_t(const PrefillArgs& a, cudaStream_t s) {
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
     const unsigned threads = (unsigned)(a.Q < 32 ? 32 : a.Q);   // whole warps for the shuffles
     dt_cumsum_kernel<IoT><<<(unsigned)blocks, threads, 0, s>>>(
-        (const IoT*)a.dt_raw, a.dt_bias, a.A, dt, acs, flags, a.pad_left, a.L, a.lay.Lpad, (int)a.H, (int)a.Q, nflags,
+        (const IoT*)a.dt_raw, a.dt_bias, a.A, dt, acs, acs_lo, flags, a.pad_left, a.L, a.lay.Lpad, (int)a.H, (int)a.Q,
+        nflags,
         (int)a.lay.nchunks, hgroups);
     return cudaGetLastError();
 }
@@ -141,8 +155,8 @@ __device__ __forceinline__ void tile_fma(const float (*At)[TM + TPAD], const flo
 template <typename IoT>
 __global__ void __launch_bounds__(256)
 chunk_state_kernel(const IoT* __restrict__ x, const IoT* __restrict__ Bm, const float* __restrict__ dtw,
-                   const float* __restrict__ acsw, float* __restrict__ states, int64_t L, int64_t Lpad,
-                   int H, int P, int N, int G, int Q, int nchunks, int ntiles) {
+                   const float* __restrict__ acsw, const float* __restrict__ acslo, float* __restrict__ states,
+                   int64_t L, int64_t Lpad, int H, int P, int N, int G, int Q, int nchunks, int ntiles) {
     __shared__ __align__(16) float At[TK][TM + TPAD];   // [s][n]
     __shared__ __align__(16) float Bt[TK][TM + TPAD];   // [s][p] scaled by w_s
     __shared__ float ws[256];
@@ -156,8 +170,10 @@ chunk_state_kernel(const IoT* __restrict__ x, const IoT* __restrict__ Bm, const 
     const int64_t base_t = (int64_t)c * Q;
     const float* dtc = dtw + (int64_t)bh * Lpad + base_t;
     const float* acc_c = acsw + (int64_t)bh * Lpad + base_t;
-    const float a_last = acc_c[Q - 1];
-    for (int s = tid; s < Q; s += 256) ws[s] = expf(a_last - acc_c[s]) * dtc[s];
+    const float* acl_c = acslo ? acslo + (int64_t)bh * Lpad + base_t : nullptr;
+    const float a_last = acc_c[Q - 1], a_last_lo = acl_c ? acl_c[Q - 1] : 0.f;
+    for (int s = tid; s < Q; s += 256)
+        ws[s] = expf((a_last - acc_c[s]) + (a_last_lo - (acl_c ? acl_c[s] : 0.f))) * dtc[s];
     float acc[4][4] = {};
     for (int k0 = 0; k0 < Q; k0 += TK) {
         __syncthreads();
@@ -226,14 +242,14 @@ template <typename IoT, typename YT>
 __global__ void __launch_bounds__(256)
 chunk_scan_kernel(const IoT* __restrict__ x, const IoT* __restrict__ Bm, const IoT* __restrict__ Cm,
                   const float* __restrict__ Dv, const float* __restrict__ dtw,
-                  const float* __restrict__ acsw, const float* __restrict__ states,
-                  YT* __restrict__ y, int64_t L, int64_t Lpad, int H, int P, int N, int G, int Q,
-                  int nchunks, int ptiles) {
+                  const float* __restrict__ acsw, const float* __restrict__ acslo,
+                  const float* __restrict__ states, YT* __restrict__ y, int64_t L, int64_t Lpad, int H, int P,
+                  int N, int G, int Q, int nchunks, int ptiles) {
     __shared__ __align__(16) float At[TK][TM + TPAD];
     __shared__ __align__(16) float Bt[TK][TM + TPAD];
     __shared__ __align__(16) float Mt[TM][TM + TPAD];   // [s][l] masked decay matrix
     __shared__ __align__(16) float Xs[TM][TM + TPAD];   // [s][p]
-    __shared__ float acs_l[TM], acs_s[TM], dt_s[TM];
+    __shared__ float acs_l[TM], acs_s[TM], dt_s[TM], lo_l[TM], lo_s[TM];
     const int rtiles = (Q + TM - 1) / TM;
     const unsigned crt = (unsigned)(nchunks * rtiles);
     const int cr = (int)((blockIdx.x / (unsigned)ptiles) % crt);
@@ -244,10 +260,14 @@ chunk_scan_kernel(const IoT* __restrict__ x, const IoT* __restrict__ Bm, const I
     const int l0 = rt * TM;                       // chunk-local first row of the tile
     const int64_t base_t = (int64_t)c * Q;
     const float* acs = acsw + (int64_t)bh * Lpad + base_t;
+    const float* acl = acslo ? acslo + (int64_t)bh * Lpad + base_t : nullptr;
     const float* dtc = dtw + (int64_t)bh * Lpad + base_t;
     const float* hin = states + ((int64_t)bh * nchunks + c) * N * P;
     const int rows = min(TM, Q - l0);
-    if (tid < TM) acs_l[tid] = tid < rows ? acs[l0 + tid] : 0.f;
+    if (tid < TM) {
+        acs_l[tid] = tid < rows ? acs[l0 + tid] : 0.f;
+        lo_l[tid] = tid < rows && acl ? acl[l0 + tid] : 0.f;
+    }
 
     // off-diagonal term: acc = C_l^T h_in
     float acc[4][4] = {};
@@ -277,6 +297,7 @@ chunk_scan_kernel(const IoT* __restrict__ x, const IoT* __restrict__ Bm, const I
         __syncthreads();
         if (tid < TM) {
             acs_s[tid] = tid < cols ? acs[s0 + tid] : 0.f;
+            lo_s[tid] = tid < cols && acl ? acl[s0 + tid] : 0.f;
             dt_s[tid] = tid < cols ? dtc[s0 + tid] : 0.f;
         }
         float sc[4][4] = {};
@@ -301,7 +322,8 @@ chunk_scan_kernel(const IoT* __restrict__ x, const IoT* __restrict__ Bm, const I
             for (int j = 0; j < 4; ++j) {
                 const int li = ty * 4 + i, sj = tx * 4 + j;
                 const bool keep = (s0 + sj) <= (l0 + li) && sj < cols && li < rows;
-                Mt[sj][li] = keep ? sc[i][j] * expf(acs_l[li] - acs_s[sj]) * dt_s[sj] : 0.f;
+                Mt[sj][li] = keep ? sc[i][j] * expf((acs_l[li] - acs_s[sj]) + (lo_l[li] - lo_s[sj])) * dt_s[sj]
+                                  : 0.f;
             }
         for (int i = tid; i < TM * TM; i += 256) {
             const int sj = i / TM, pp = i % TM;
@@ -333,13 +355,14 @@ template <typename IoT, typename YT, typename StateT>
 static cudaError_t launch_simt_t(const PrefillArgs& a, cudaStream_t s) {
     const float* dt = (const float*)(a.ws + a.lay.off_dt);
     const float* acs = (const float*)(a.ws + a.lay.off_acs);
+    const float* acslo = a.lay.has_lo ? (const float*)(a.ws + a.lay.off_acs_lo) : nullptr;
     float* states = (float*)(a.ws + a.lay.off_states);
     const int nc = (int)a.lay.nchunks;
     const int H = (int)a.H, P = (int)a.P, N = (int)a.N, G = (int)a.G, Q = (int)a.Q;
     const unsigned BH = (unsigned)(a.batch * a.H);
     const unsigned tiles_np = (unsigned)(((N + TM - 1) / TM) * ((P + TM - 1) / TM));
     chunk_state_kernel<IoT><<<(unsigned)(nc * BH * tiles_np), 256, 0, s>>>(
-        (const IoT*)a.x, (const IoT*)a.B, dt, acs, states, a.L, a.lay.Lpad, H, P, N, G, Q, nc, (int)tiles_np);
+        (const IoT*)a.x, (const IoT*)a.B, dt, acs, acslo, states, a.L, a.lay.Lpad, H, P, N, G, Q, nc, (int)tiles_np);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const int NP = N * P;
@@ -350,7 +373,7 @@ static cudaError_t launch_simt_t(const PrefillArgs& a, cudaStream_t s) {
     const unsigned rtiles = (unsigned)((Q + TM - 1) / TM);
     const unsigned ptiles = (unsigned)((P + TM - 1) / TM);
     chunk_scan_kernel<IoT, YT><<<nc * rtiles * BH * ptiles, 256, 0, s>>>(
-        (const IoT*)a.x, (const IoT*)a.B, (const IoT*)a.C, a.D, dt, acs, states, (YT*)a.y, a.L,
+        (const IoT*)a.x, (const IoT*)a.B, (const IoT*)a.C, a.D, dt, acs, acslo, states, (YT*)a.y, a.L,
         a.lay.Lpad, H, P, N, G, Q, nc, (int)ptiles);
     return cudaGetLastError();
 }

@@ -41,6 +41,15 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
         : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
     return ok != 0;
 }
+// the same with a suspend-time hint: a thread whose phase is not complete sleeps
+// (issuing nothing) until the phase completes or about `ns` nanoseconds pass
+__device__ __forceinline__ bool mbar_try_sleep(uint32_t bar, uint32_t parity, uint32_t ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok) : "r"(bar), "r"(parity), "r"(ns) : "memory");
+    return ok != 0;
+}
 __device__ __forceinline__ void fence_proxy_async() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -169,6 +178,55 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
+// Packed pairs of fp32 values (sm_100 f32x2 arithmetic: one instruction acts on
+// both halves of a 64-bit register; round to nearest even like the scalar ops).
+typedef unsigned long long f32x2;
+__device__ __forceinline__ f32x2 f2_pack(float a, float b) {
+    f32x2 r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ f32x2 f2_pack_u(uint32_t a, uint32_t b) {
+    f32x2 r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(a), "r"(b));
+    return r;
+}
+__device__ __forceinline__ void f2_unpack(f32x2 v, float& a, float& b) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ f32x2 f2_mul(f32x2 a, f32x2 b) {
+    f32x2 r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ f32x2 f2_add(f32x2 a, f32x2 b) {
+    f32x2 r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ f32x2 f2_sub(f32x2 a, f32x2 b) {
+    f32x2 r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ f32x2 f2_fma(f32x2 a, f32x2 b, f32x2 c) {
+    f32x2 r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+// a pair (v0, v1) as the bf16 pairs hi = bf16(v), lo = bf16(v - hi) (element 0
+// in the low halves)
+__device__ __forceinline__ void split2(f32x2 v, uint32_t& hi, uint32_t& lo) {
+    float a, b;
+    f2_unpack(v, a, b);
+    hi = pack_bf16(a, b);
+    const f32x2 r = f2_sub(v, f2_pack(bf16_lo(hi), bf16_hi(hi)));
+    f2_unpack(r, a, b);
+    lo = pack_bf16(a, b);
+}
+// two bf16 values of one word as an fp32 pair
+__device__ __forceinline__ f32x2 bf16x2_to_f2(uint32_t w) { return f2_pack(bf16_lo(w), bf16_hi(w)); }
+
 // byte offset of 16-byte chunk `j` of row `r` in a 128-byte-swizzled tile
 __device__ __forceinline__ uint32_t swz(int r, int j) { return (uint32_t)(r * 128 + ((j ^ (r & 7)) << 4)); }
 
@@ -178,8 +236,8 @@ __device__ __forceinline__ uint32_t swz(int r, int j) { return (uint32_t)(r * 12
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
     uint32_t spins = 0;
     unsigned long long deadline = 0;
-    while (!mbar_try(bar, parity)) {
-        if ((++spins & 1023u) == 0) {
+    while (!mbar_try_sleep(bar, parity, 100000u)) {
+        if ((++spins & 15u) == 0) {
             const unsigned long long now = gtimer();
             if (deadline == 0) deadline = now + WAIT_NS;
             else if (now > deadline) return false;

@@ -26,7 +26,7 @@
  *    it; the blocked algorithm splits the sequence into chunks processed in
  *    parallel and recombines the per-chunk states.
  *
- * Readings where the pages are silent (every one is also listed in the design doc):
+ * Readings where the pages are silent:
  *  - y_t uses the state AFTER the token-t update (so the diagonal of the
  *    semiseparable mask is exp(0) = 1).
  *  - softplus(z) = log(1 + e^z), evaluated exactly (no threshold).
