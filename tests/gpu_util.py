@@ -51,8 +51,10 @@ def bf16_excess_metric(got: np.ndarray, ref: np.ndarray) -> float:
 # value and the oracle's float64 value fall on the two sides of a bf16 rounding
 # boundary, which independent rounding makes rare; a systematic bias of the
 # kernel's bf16 store (truncation, a wrong rounding mode) would move about half
-# of them.
-BF16_FLIP_SHARE_MAX = 0.05
+# of them.  Measured on the GPU tests: at most 2.6e-4 on states of 16k elements
+# or more (7.6e-5 after the batch-512 hand-off and 32 decode steps), and one
+# element of 512 on the smallest state.
+BF16_FLIP_SHARE_MAX = 0.01
 
 
 def bf16_flip_share(got: np.ndarray, ref: np.ndarray) -> float:

@@ -44,3 +44,23 @@ def test_decode_bytes_state_read_and_write():
     state = 2 * bd * Hd * Nd * Pd * 4
     io = bd * Hd * Pd * (2 + 4) + 2 * bd * Gd * Nd * 2 + bd * Hd * 2
     assert bench.decode_bytes(bd, Hd, Pd, Nd, Gd, 2, 4, 4) == state + io == 2_161_180_672
+
+
+def test_executed_flops_block_by_block():
+    # 128-token blocks; the head-pair kernel forms C B^T once per pair of heads, the
+    # single-head kernel once per head; per head C h, the chunk state and M X each
+    # run on the bf16 hi and lo parts of the operand computed in the kernel
+    nblk = L // 128
+    s = 2 * 128 * 128 * N
+    per_head = 2 * (2 * 128 * N * P) + 2 * (2 * 128 * N * P) + 2 * (2 * 128 * 128 * P)
+    assert bench.executed_flops(b, L, H, P, N, G, 2) == b * nblk * (H // 2 * s + H * per_head)
+    assert bench.executed_flops(b, L, H, P, N, G, 0) == b * nblk * (H * s + H * per_head)
+
+
+def test_handoff_prefill_bytes():
+    bb, LL, HH, GG = 512, 1024, 128, 8
+    t = bb * LL
+    x, y = t * HH * P * 2, t * HH * P * 4
+    bc, dt_raw = 2 * t * GG * N * 2, t * HH * 2
+    final = bb * HH * N * P * 2          # bf16 state handed to the decode steps
+    assert bench.prefill_bytes(bb, LL, HH, P, N, GG, 2, 4, 2) == x + y + bc + dt_raw + final

@@ -66,7 +66,8 @@ def test_mamba3_bf16_outputs_and_state():
     y, fs, y_ref, fs_ref = run_case(2, 256, 4, 64, 128, 1, 128, I.BF16, True, True, True, y_dtype="bf16",
                                     state=I.BF16)
     assert bf16_excess_metric(y, y_ref) <= TOL_BF16
-    assert bf16_state_metric(fs, fs_ref) <= TOL_BF16
+    # the final state is rounded to bf16 once, when stored: measured beyond its own rounding
+    assert bf16_excess_metric(fs, fs_ref) <= TOL_BF16
 
 
 def test_mamba3_without_extensions_is_the_forward_call():
