@@ -13,8 +13,8 @@ The line's value is prefill tokens/s; the same run reports:
 - "handoff_decode": the 32 ssd_state_update steps at batch 512 that the
   prefill's bf16 final state feeds (tokens/s, state GB/s);
 - "decode": K decode steps at batch 256 x 128 heads with an fp32 state, with
-  the same steps replayed from a checkpoint and a 16-token buffer ("replay")
-  and rank-4 MIMO steps ("mimo");
+  the same steps replayed from a checkpoint and a 16-token buffer ("replay"),
+  rank-4 MIMO steps ("mimo") and Mamba-3 steps ("mamba3");
 - "mamba2_1p3b": the Mamba-2 1.3B-shaped layer prefill (batch 4 x 2048 tokens,
   64 heads, 1 group), with its backward pass ("backward") and the Mamba-3
   prefill of the same layer ("mamba3");
@@ -53,6 +53,9 @@ METRIC = "SSD prefill tokens/s + TFLOP/s; decode tokens/s + state GB/s (1 B200)"
 # reports null until it is captured again (summaries under profiles/).
 NCU_TRAFFIC = {
     ("ssd_decode.cu", "decode_b256"): ("cba348ad46ab41a0", 1079097000 + 1024990000),
+    ("ssd_prefill_pair.cu", "mamba2_1p3b"): ("dff7966de41843dc", 77671424 + 89317120),
+    # captured with 32 of the 512 sequences and scaled by 16 (profiles/ssd_pair_kernel_handoff_prefill_b512.md)
+    ("ssd_prefill_pair.cu", "handoff_prefill"): ("dff7966de41843dc", (725146880 + 1084068352) * 16),
 }
 
 
@@ -319,6 +322,12 @@ def main():
     ap.add_argument("--no-workloads", action="store_true",
                     help="skip timing the other benchmark workloads (tiny fp32 prefill, long-sequence sweep)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) measurement")
+    ap.add_argument("--workload", choices=["handoff_prefill", "mamba2_1p3b"], default="handoff_prefill",
+                    help="the headline prefill workload (default: the batch-512 prefill, the largest single-GPU one)")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the headline workload's batch (a smaller case of the same shape, for profiling)")
+    ap.add_argument("--only-headline", action="store_true",
+                    help="time the headline prefill alone (for profiling one workload)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     rank = int(os.environ.get("RANK", "0"))
@@ -349,12 +358,17 @@ def main():
             raise RuntimeError(f"device error word {detail:#x} after {what}")
 
     # ================= headline: batch-512 prefill (each rank its own 512 sequences)
-    s = I.HANDOFF_PREFILL
+    s = I.HANDOFF_PREFILL if args.workload == "handoff_prefill" else I.MAMBA2_1P3B
     b, L, H, P, N, G, Q = s.batch, s.seqlen, s.nheads, s.headdim, s.dstate, s.ngroups, s.chunk
+    if args.batch > 0:
+        if not args.only_headline:
+            raise SystemExit("--batch is a profiling option: use it with --only-headline")
+        b = args.batch
+    sdt = bf16 if s is I.HANDOFF_PREFILL else torch.float32     # the hand-off keeps the final state in bf16
     inp = device_inputs(torch, dev, b, L, H, P, N, G, 4000 + rank, bf16)
     y = torch.empty((b, L, H, P), dtype=torch.float32, device=dev)
-    fs = torch.empty((b, H, N, P), dtype=bf16, device=dev)
-    desc = ssd.prefill_desc(inp["x"], inp["B"], Q, torch.float32, bf16)
+    fs = torch.empty((b, H, N, P), dtype=sdt, device=dev)
+    desc = ssd.prefill_desc(inp["x"], inp["B"], Q, torch.float32, sdt)
     path = ssd.ssd_chunk_scan_path(desc)
     ws = torch.empty(ssd.ssd_chunk_scan_workspace_size(desc), dtype=torch.uint8, device=dev)
 
@@ -373,12 +387,25 @@ def main():
     value = tokens_rank * world / (ms * 1e-3)
     flops = prefill_flops(b, L, H, P, N, G, Q)
     xflops = executed_flops(b, L, H, P, N, G, path)
-    nbytes = prefill_bytes(b, L, H, P, N, G, 2, 4, 2)
+    nbytes = prefill_bytes(b, L, H, P, N, G, 2, 4, 2 if sdt == bf16 else 4)
     roofline = roofline_of(nbytes, flops, ms * 1e-3, peaks, peak_kind)
-    roofline.update({"traffic": ncu_traffic("ssd_prefill_pair.cu", "handoff_prefill_b512"),
+    roofline.update({"traffic": ncu_traffic("ssd_prefill_pair.cu", args.workload),
                      "kernel": "ssd_chunk_scan_fwd (decay cumsum + tcgen05 head-pair chunk kernel)"})
+    if args.only_headline:
+        if rank == 0:
+            print(json.dumps({"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+                              "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+                              "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                              "config": {"workload": s.name, "global_batch": b * world, "seq_len": L,
+                                         "kernel_path": PATH_NAMES[path], "legs": "headline only"},
+                              "roofline": roofline, "gpu_launches": 2 * args.steps, "clocks": clk.summary()}),
+                  flush=True)
+        dist.finish(pg)
+        return
 
     # ---- the hand-off: the prefill's bf16 final state feeds 32 decode steps at batch 512
+    if s is not I.HANDOFF_PREFILL:
+        raise SystemExit("--workload mamba2_1p3b runs with --only-headline")
     dsh = I.HANDOFF_DECODE
     gen = torch.Generator(device=dev)
     gen.manual_seed(4100 + rank)
@@ -611,6 +638,34 @@ def main():
                            "roofline": {"bound": "hbm", "achieved": mgbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                                         "frac": mgbs / peaks["hbm_gbs"], "algorithmic_bytes_per_step": mbytes,
                                         "kernel": "mimo_step_kernel"}}
+    # ---- Mamba-3 decode steps on the same state: trapezoid mix lam and rotation angles
+    # theta given; the previous token's x and B are the previous step's inputs
+    ex3 = I.draw_mamba3_extras(dcfg.batch, nsteps_in, dcfg.nheads, dcfg.ngroups, dcfg.dstate, dcfg.seed)
+    m3lam = [torch.from_numpy(np.ascontiguousarray(ex3["lam"][:, t])).to(dev) for t in range(nsteps_in)]
+    m3th = [torch.from_numpy(np.ascontiguousarray(ex3["theta"][:, t])).to(dev) for t in range(nsteps_in)]
+
+    def mamba3_step(t):
+        d, dp = dsteps[t % nsteps_in], dsteps[(t - 1) % nsteps_in]
+        st = ssd.ssd_state_update_mamba3(ddesc, state.data_ptr(), d["x"].data_ptr(), dp["x"].data_ptr(),
+                                         d["dt_raw"].data_ptr(), prm["dt_bias"].data_ptr(), prm["A"].data_ptr(),
+                                         d["B"].data_ptr(), dp["B"].data_ptr(), d["C"].data_ptr(),
+                                         prm["D"].data_ptr(), m3lam[t % nsteps_in].data_ptr(),
+                                         m3th[t % nsteps_in].data_ptr(), yd.data_ptr(), stream.cuda_stream)
+        if st:
+            raise ssd.SsdError(st, "ssd_state_update_mamba3")
+
+    m3dms = timed(torch, stream, mamba3_step, dsteps_timed, args.warmup, pg, dist)
+    check("the timed Mamba-3 decode steps")
+    m3dbytes = (dbytes + dcfg.batch * dcfg.nheads * dcfg.headdim * 2 + dcfg.batch * dcfg.ngroups * dcfg.dstate * 2
+                + dcfg.batch * dcfg.nheads * 4 + dcfg.batch * dcfg.ngroups * dcfg.dstate // 2 * 4)
+    m3dgbs = m3dbytes / (m3dms * 1e-3) / 1e9
+    decode_line["mamba3"] = {"tokens_per_s": dcfg.batch * world / (m3dms * 1e-3), "ms_per_step": m3dms,
+                             "time_vs_state_update": m3dms / dms,
+                             "inputs": "lam ~ U[0,1] per (b, head), theta ~ U[-0.5,0.5] rad per (b, group, pair); "
+                                       "x_prev, B_prev = the previous step's x, B",
+                             "roofline": {"bound": "hbm", "achieved": m3dgbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                          "frac": m3dgbs / peaks["hbm_gbs"], "algorithmic_bytes_per_step": m3dbytes,
+                                          "kernel": "mamba3_step_kernel"}}
     del state, dsteps, yd, rbuf, mx_, mB, mC, my_
     torch.cuda.empty_cache()
 
@@ -759,7 +814,8 @@ def main():
                 "cpu_baseline": cpu_baseline, "e2e": e2e, "workloads": workloads,
                 "gpu_launches": 2 * args.steps,
                 "gpu_launches_other_legs": {"handoff_decode": dsh.steps, "decode": dsteps_timed,
-                                            "replay": 2 * rsteps, "mimo": dsteps_timed, "mamba2_1p3b": 2 * c1_steps,
+                                            "replay": 2 * rsteps, "mimo": dsteps_timed,
+                                            "mamba3_decode": dsteps_timed, "mamba2_1p3b": 2 * c1_steps,
                                             "backward": launches_per_bwd * bsteps, "mamba3": launches_per_m3 * m3steps},
                 "clocks": clk.summary()}
         print(json.dumps(line), flush=True)

@@ -387,6 +387,47 @@ ssd_status_t ssd_state_update_mimo(const ssd_mimo_desc_t* desc, void* state, con
                                    void* stream);
 
 /*
+ * Mamba-3 decode step, in place on the state: the exponential-trapezoidal
+ * input ("Mamba3" Telegram post, section "New discretisation scheme": the
+ * input is taken at both ends of the step and mixed by a learned weight) and
+ * the rotational state ("Mamba3", section on the complex-valued SSM; "Mamba-3 :
+ * SSM optimise inference", section "Etats complexes via RoPE": state pairs turn
+ * by data-dependent angles).  With dt = softplus(dt_raw + dt_bias), lam the mix
+ * and R(theta) turning state rows (2k, 2k+1) by theta[k]:
+ *
+ *   h <- exp(dt A) R(theta) (h + (1 - lam) dt B_prev x_prev^T) + lam dt B x^T
+ *   y  = C^T h + D x
+ *
+ * lam = 1 and theta = 0 give ssd_state_update.  The trapezoid reaches one token
+ * back, so the decode state is the SSM state plus the previous token's B and x;
+ * the caller passes those (its previous call's B and x) and keeps them: the call
+ * writes only the state and y.  The prefill's form is ssd_chunk_scan_fwd_mamba3.
+ *
+ *  desc   as ssd_state_update (io_dtype for x, x_prev, dt_raw, B, B_prev, C)
+ *  state  [b][H][N][P]  state_dtype  required, read and written in place
+ *  x      [b][H][P]     io_dtype     required
+ *  x_prev [b][H][P]     io_dtype     the previous token's x; NULL (with B_prev)
+ *                                     before the first token: no left end
+ *  dt_raw [b][H]        io_dtype     required
+ *  dt_bias, A, D [H]    fp32         dt_bias, D nullable
+ *  B, C   [b][G][N]     io_dtype     required
+ *  B_prev [b][G][N]     io_dtype     the previous token's B; NULL with x_prev
+ *  lam    [b][H]        fp32         nullable (= 1: Mamba-2's input)
+ *  theta  [b][G][N/2]   fp32         radians; nullable (= 0: no rotation)
+ *  y      [b][H][P]     y_dtype      required; must not overlap state, x or x_prev
+ * dstate must be even; headdim a power-of-two count of 16-byte state vectors
+ * that divides 32 (P <= 128 for fp32 states, <= 256 for bf16).
+ * Errors: SSD_ERR_INVALID_ARG (bad descriptor, NULL required pointer, only one
+ * of x_prev / B_prev, overlapping outputs), SSD_ERR_UNSUPPORTED (shape),
+ * SSD_ERR_ALIGNMENT, SSD_ERR_CUDA; nothing is launched on a host-side error.
+ */
+ssd_status_t ssd_state_update_mamba3(const ssd_decode_desc_t* desc, void* state, const void* x,
+                                     const void* x_prev, const void* dt_raw, const float* dt_bias,
+                                     const float* A, const void* B, const void* B_prev, const void* C,
+                                     const float* D, const float* lam, const float* theta, void* y,
+                                     void* stream);
+
+/*
  * Bytes of the replay buffer ssd_replay_step needs for `desc` (written to
  * *bytes).  Pure host function.  Errors: SSD_ERR_INVALID_ARG /
  * SSD_ERR_UNSUPPORTED as for ssd_replay_step.

@@ -459,6 +459,44 @@ ssd_status_t ssd_state_update(const ssd_decode_desc_t* d, void* state, const voi
     return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
 }
 
+ssd_status_t ssd_state_update_mamba3(const ssd_decode_desc_t* d, void* state, const void* x, const void* x_prev,
+                                     const void* dt_raw, const float* dt_bias, const float* A, const void* B,
+                                     const void* B_prev, const void* C, const float* D, const float* lam,
+                                     const float* theta, void* y, void* stream) {
+    if (!d) return SSD_ERR_INVALID_ARG;
+    if (d->batch < 0 || d->nheads < 1 || d->headdim < 1 || d->dstate < 1 || d->ngroups < 1 ||
+        d->nheads % d->ngroups != 0)
+        return SSD_ERR_INVALID_ARG;
+    if (!valid_dtype(d->io_dtype) || !valid_dtype(d->y_dtype) || !valid_dtype(d->state_dtype))
+        return SSD_ERR_INVALID_ARG;
+    if (d->headdim % 8 != 0 || d->dstate % 8 != 0 || d->headdim > 256 || d->dstate > 256)
+        return SSD_ERR_UNSUPPORTED;
+    if (!mamba3_step_supports(d->headdim, d->dstate, d->state_dtype == SSD_BF16)) return SSD_ERR_UNSUPPORTED;
+    if (d->batch * d->nheads > (int64_t)0x7fffffff) return SSD_ERR_UNSUPPORTED;
+    if (!state || !x || !dt_raw || !A || !B || !C || !y) return SSD_ERR_INVALID_ARG;
+    if ((x_prev == nullptr) != (B_prev == nullptr)) return SSD_ERR_INVALID_ARG;   // both or neither
+    const void* ptrs[] = {state, x, x_prev, dt_raw, dt_bias, A, B, B_prev, C, D, lam, theta, y};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return SSD_ERR_ALIGNMENT;
+    const size_t bh = (size_t)d->batch * d->nheads;
+    const size_t s_bytes = bh * d->dstate * d->headdim * dsize(d->state_dtype);
+    const size_t y_bytes = bh * d->headdim * dsize(d->y_dtype);
+    const size_t x_bytes = bh * d->headdim * dsize(d->io_dtype);
+    if (overlaps(y, y_bytes, state, s_bytes) || overlaps(y, y_bytes, x, x_bytes) ||
+        overlaps(state, s_bytes, x, x_bytes) || overlaps(y, y_bytes, x_prev, x_bytes) ||
+        overlaps(state, s_bytes, x_prev, x_bytes))
+        return SSD_ERR_INVALID_ARG;
+    if (d->batch == 0) return SSD_OK;
+    Mamba3StepArgs a{};
+    a.batch = d->batch; a.H = d->nheads; a.P = d->headdim; a.N = d->dstate; a.G = d->ngroups;
+    a.io_bf16 = d->io_dtype == SSD_BF16; a.y_bf16 = d->y_dtype == SSD_BF16;
+    a.state_bf16 = d->state_dtype == SSD_BF16;
+    a.state = state; a.x = x; a.x_prev = x_prev; a.dt_raw = dt_raw; a.B = B; a.B_prev = B_prev; a.C = C;
+    a.dt_bias = dt_bias; a.A = A; a.D = D; a.lam = lam; a.theta = theta; a.y = y;
+    const cudaError_t e = launch_mamba3_step(a, (cudaStream_t)stream);
+    return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
+}
+
 ssd_status_t ssd_state_update_mimo(const ssd_mimo_desc_t* d, void* state, const void* x, const void* dt_raw,
                                    const float* dt_bias, const float* A, const void* B, const void* C,
                                    const float* D, void* y, void* stream) {

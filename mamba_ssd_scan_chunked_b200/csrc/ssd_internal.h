@@ -19,6 +19,19 @@ struct DecodeArgs {
 
 cudaError_t launch_state_update(const DecodeArgs& a, cudaStream_t stream);
 
+// Mamba-3 decode step: trapezoidal input, rotational state (ssd_mamba3_decode.cu).
+struct Mamba3StepArgs {
+    int64_t batch, H, P, N, G;
+    bool io_bf16, y_bf16, state_bf16;
+    void* state;
+    const void *x, *x_prev, *dt_raw, *B, *B_prev, *C;   // x, x_prev [b][H][P]; B, B_prev, C [b][G][N]
+    const float *dt_bias, *A, *D, *lam, *theta;         // lam [b][H]; theta [b][G][N/2]
+    void* y;
+};
+
+bool mamba3_step_supports(int64_t P, int64_t N, bool state_bf16);
+cudaError_t launch_mamba3_step(const Mamba3StepArgs& a, cudaStream_t stream);
+
 // Replayed decode step: checkpoint + buffer of the last tokens (ssd_replay.cu).
 struct ReplayArgs {
     int64_t batch, H, P, N, G, K, fill;

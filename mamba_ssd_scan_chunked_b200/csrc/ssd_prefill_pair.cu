@@ -117,8 +117,9 @@ __device__ __forceinline__ void split8(const float* v, uint32_t (&hw)[4], uint32
     }
 }
 
-// 18 warps x 32 threads x 112 registers = 64512 of the SM's 65536
-__global__ void __maxnreg__(112)
+// 18 warps, 5 of them on one SM sub-partition (16384 registers each): at most 96
+// registers a thread, which the launch bounds give
+__global__ void __launch_bounds__(THREADS, 1)
 ssd_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmY, const Params p) {
     extern __shared__ __align__(1024) uint8_t sm[];
@@ -385,6 +386,33 @@ ssd_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
             }
         };
 
+        // w o X into the W tiles (quarters 0 and 1: one token row of one head per
+        // thread), once C h has read them; the state MMAs wait for it
+        auto do_wx = [&](uint32_t ph) {
+            wait(B_OFF, ph);
+            tc_fence_after();
+            wait(B_X, ph);
+            const int t = kq * 64 + q * 32 + lane;
+            const int s_ = t & (SUB - 1), k = t >> 7;
+            const float wv = ex2(dl2(s_ge[k * 8 + 7], s_ge[k * 8 + (s_ >> 4)]) + s_v[k * SUB + s_]);
+            const f32x2 w2 = f2_pack(wv, wv);
+            const uint8_t* xt = sm + OFF_X + k * TILE;
+            uint8_t* wt = sm + OFF_W + k * 2 * TILE;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const uint32_t o = swz(s_, c);
+                const uint4 xv = *reinterpret_cast<const uint4*>(xt + o);
+                const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+                uint32_t hw[4], lw[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) split2(f2_mul(bf16x2_to_f2(xw[e]), w2), hw[e], lw[e]);
+                *reinterpret_cast<uint4*>(wt + o) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                *reinterpret_cast<uint4*>(wt + TILE + o) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+            }
+            fence_proxy_async();
+            mbar_arrive(bar(B_WX));
+        };
+
         float2 ref[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};   // cumsum at the previous block's end
         int it = 0, j = 0;
         Item d = total > 0 ? item_of(0) : Item{};
@@ -409,9 +437,11 @@ ssd_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
             for (int k = 0; k < 2; ++k) r0[k] = chunk_start ? make_float2(0.f, 0.f) : ref[k];
             uint32_t inc = 0;                 // a log-decay that increases somewhere in the block
             if (kq < 2) {
+                // head kq; selected, not indexed, so that the registers stay registers
                 const int k = kq;
-                const float2 me = cur.row[k];
-                inc = dl2(me, row ? cur.prev : r0[k]) > 0.f;
+                const float2 me = k ? cur.row[1] : cur.row[0];
+                const float2 r0k = k ? r0[1] : r0[0];
+                inc = dl2(me, row ? cur.prev : r0k) > 0.f;
                 const float2 ge = make_float2(__shfl_sync(0xffffffffu, me.x, lane | 15),
                                               __shfl_sync(0xffffffffu, me.y, lane | 15));
                 const float v = (cur.dt > 0.f ? __log2f(cur.dt) : NEG_INF) + dl2(ge, me);
@@ -499,32 +529,11 @@ ssd_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                 t127n[1] = cum(bh0_n + 1, (long long)j_n * SUB + SUB - 1);
             }
 
-            // ---- after C h: w o X into the W tiles (quarters 0 and 1: one token row of
-            // one head per thread), Yoff scaled by 2^(r_l), x kept for D x
+            // ---- after C h: w o X into the W tiles (quarters 0 and 1), Yoff scaled by
+            // 2^(r_l), x kept for D x
             wait(B_OFF, ph);
             tc_fence_after();
-            if (q < 2) {
-                wait(B_X, ph);
-                const int t = kq * 64 + q * 32 + lane;
-                const int s_ = t & (SUB - 1), k = t >> 7;
-                const float wv = ex2(dl2(s_ge[k * 8 + 7], s_ge[k * 8 + (s_ >> 4)]) + s_v[k * SUB + s_]);
-                const f32x2 w2 = f2_pack(wv, wv);
-                const uint8_t* xt = sm + OFF_X + k * TILE;
-                uint8_t* wt = sm + OFF_W + k * 2 * TILE;
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const uint32_t o = swz(s_, c);
-                    const uint4 xv = *reinterpret_cast<const uint4*>(xt + o);
-                    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-                    uint32_t hw[4], lw[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) split2(f2_mul(bf16x2_to_f2(xw[e]), w2), hw[e], lw[e]);
-                    *reinterpret_cast<uint4*>(wt + o) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-                    *reinterpret_cast<uint4*>(wt + TILE + o) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-                }
-                fence_proxy_async();
-                mbar_arrive(bar(B_WX));
-            }
+            if (q < 2) do_wx(ph);
             {
                 uint32_t v[2][16];
                 tmem_ld16(tmem + lo16 + COL_Y + 16 * kq, v[0]);

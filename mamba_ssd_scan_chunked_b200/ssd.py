@@ -28,7 +28,8 @@ STATUS = {0: "SSD_OK", 1: "SSD_ERR_INVALID_ARG", 2: "SSD_ERR_UNSUPPORTED", 3: "S
 EXPORTS = ("ssd_version", "ssd_status_string", "ssd_chunk_scan_workspace_size", "ssd_chunk_scan_path",
            "ssd_chunk_scan_fwd", "ssd_chunk_scan_fwd_varlen", "ssd_chunk_scan_fwd_noalloc",
            "ssd_chunk_scan_bwd", "ssd_chunk_scan_bwd_workspace_size", "ssd_chunk_scan_bwd_launches",
-           "ssd_chunk_scan_fwd_mamba3", "ssd_chunk_scan_mamba3_workspace_size", "ssd_chunk_scan_mamba3_launches", "ssd_state_update", "ssd_state_update_mimo",
+           "ssd_chunk_scan_fwd_mamba3", "ssd_chunk_scan_mamba3_workspace_size", "ssd_chunk_scan_mamba3_launches",
+           "ssd_state_update", "ssd_state_update_mimo", "ssd_state_update_mamba3",
            "ssd_replay_buffer_size",
            "ssd_replay_step", "ssd_get_device_error", "ssd_debug_inject")
 
@@ -118,6 +119,8 @@ def lib():
             L.ssd_state_update.argtypes = [ctypes.POINTER(DecodeDesc)] + [_VP] * 10
             L.ssd_state_update_mimo.restype = ctypes.c_int
             L.ssd_state_update_mimo.argtypes = [ctypes.POINTER(MimoDesc)] + [_VP] * 10
+            L.ssd_state_update_mamba3.restype = ctypes.c_int
+            L.ssd_state_update_mamba3.argtypes = [ctypes.POINTER(DecodeDesc)] + [_VP] * 14
             L.ssd_replay_buffer_size.restype = ctypes.c_int
             L.ssd_replay_buffer_size.argtypes = [ctypes.POINTER(ReplayDesc), ctypes.POINTER(ctypes.c_size_t)]
             L.ssd_replay_step.restype = ctypes.c_int
@@ -241,6 +244,14 @@ def ssd_state_update_mimo(desc, state, x, dt_raw, dt_bias, A, B, C, D, y, stream
     """Raw call; returns the status code (0 = enqueued)."""
     return lib().ssd_state_update_mimo(ctypes.byref(desc), state or None, x or None, dt_raw or None, dt_bias or None,
                                        A or None, B or None, C or None, D or None, y or None, stream or None)
+
+
+def ssd_state_update_mamba3(desc, state, x, x_prev, dt_raw, dt_bias, A, B, B_prev, C, D, lam, theta, y,
+                            stream) -> int:
+    """Raw call; returns the status code (0 = enqueued)."""
+    return lib().ssd_state_update_mamba3(ctypes.byref(desc), state or None, x or None, x_prev or None, dt_raw or None,
+                                         dt_bias or None, A or None, B or None, B_prev or None, C or None, D or None,
+                                         lam or None, theta or None, y or None, stream or None)
 
 
 def ssd_replay_buffer_size(desc: ReplayDesc) -> int:
@@ -439,6 +450,30 @@ def state_update(state, x, dt_raw, dt_bias, A, B, C, D, *, y=None, y_dtype=None,
                           _ptr(D), _ptr(y), _stream(stream))
     if st:
         raise SsdError(st, "ssd_state_update")
+    return y
+
+
+def state_update_mamba3(state, x, dt_raw, dt_bias, A, B, C, D, *, x_prev=None, B_prev=None, lam=None, theta=None,
+                        y=None, y_dtype=None, stream=None):
+    """Mamba-3 decode step in place on ``state`` [b,H,N,P]: x, x_prev [b,H,P], dt_raw [b,H],
+    B, B_prev, C [b,G,N], lam [b,H] (fp32), theta [b,G,N/2] (fp32).  x_prev and B_prev
+    are the previous token's x and B (None before the first token).  Returns y."""
+    import torch
+    b, H, P = x.shape
+    G, N = B.shape[1], B.shape[2]
+    io = _dtype_code(x.dtype)
+    desc = DecodeDesc(b, H, P, N, G, io, _dtype_code(y_dtype) if y_dtype is not None else io,
+                      _dtype_code(state.dtype))
+    for t in (state, x, x_prev, dt_raw, B, B_prev, C, dt_bias, A, D, lam, theta, y):
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("libssd takes contiguous CUDA tensors")
+    if y is None:
+        y = torch.empty((b, H, P), dtype=_torch_dtype(desc.y_dtype), device=x.device)
+    st = ssd_state_update_mamba3(desc, _ptr(state), _ptr(x), _ptr(x_prev), _ptr(dt_raw), _ptr(dt_bias), _ptr(A),
+                                 _ptr(B), _ptr(B_prev), _ptr(C), _ptr(D), _ptr(lam), _ptr(theta), _ptr(y),
+                                 _stream(stream))
+    if st:
+        raise SsdError(st, "ssd_state_update_mamba3")
     return y
 
 

@@ -216,6 +216,34 @@ def test_mimo_host_validation_codes():
     assert call(md(batch=0)) == OK
 
 
+def test_mamba3_step_host_validation_codes():
+    def dd(**kw):
+        d = dict(batch=8, nheads=4, headdim=64, dstate=128, ngroups=2, io_dtype=ssd.SSD_BF16,
+                 y_dtype=ssd.SSD_F32, state_dtype=ssd.SSD_F32)
+        d.update(kw)
+        return ssd.DecodeDesc(**d)
+
+    def call(d, **ptrs):
+        p = dict(state=FAKE, x=FAKE + 0x1000000, x_prev=FAKE + 0x1800000, dt_raw=FAKE + 0x2000000, dt_bias=0,
+                 A=FAKE + 0x3000000, B=FAKE + 0x4000000, B_prev=FAKE + 0x4800000, C=FAKE + 0x5000000, D=0,
+                 lam=FAKE + 0x7000000, theta=FAKE + 0x7800000, y=FAKE + 0x6000000, stream=0)
+        p.update(ptrs)
+        return ssd.ssd_state_update_mamba3(d, p["state"], p["x"], p["x_prev"], p["dt_raw"], p["dt_bias"], p["A"],
+                                           p["B"], p["B_prev"], p["C"], p["D"], p["lam"], p["theta"], p["y"],
+                                           p["stream"])
+
+    assert call(dd(ngroups=3)) == INVALID
+    assert call(dd(), x_prev=0) == INVALID                 # the previous token's x without its B
+    assert call(dd(), B_prev=0) == INVALID
+    assert call(dd(dstate=24, headdim=96)) == UNSUPPORTED   # 24 fp32 vectors per row do not divide 32
+    assert call(dd(headdim=256)) == UNSUPPORTED            # fp32 state rows of 64 vectors
+    assert call(dd(), state=0) == INVALID
+    assert call(dd(), theta=FAKE + 0x7800004) == ALIGN
+    assert call(dd(), y=FAKE + 0x1800000) == INVALID       # y overlaps x_prev
+    assert call(dd(batch=0)) == OK
+    assert call(dd(batch=0), x_prev=0, B_prev=0, lam=0, theta=0) == OK
+
+
 def test_varlen_host_validation_codes():
     d = desc()
     need = ssd.ssd_chunk_scan_workspace_size(d)
