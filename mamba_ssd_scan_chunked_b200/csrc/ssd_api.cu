@@ -347,9 +347,11 @@ static ssd_status_t check_backward_desc(const ssd_prefill_desc_t* d, BackwardLay
     if (st != SSD_OK) return st;
     const BackwardLayout l = backward_layout(d->batch, d->seqlen, d->nheads, d->headdim, d->dstate, d->ngroups,
                                              d->chunk, d->io_dtype == SSD_BF16);
-    const ssd_prefill_desc_t t = transposed_desc(d, l.pw);
-    st = check_prefill_desc(&t);
-    if (st != SSD_OK) return st;
+    if (l.mode == 0) {
+        const ssd_prefill_desc_t t = transposed_desc(d, l.pw);
+        st = check_prefill_desc(&t);
+        if (st != SSD_OK) return st;
+    }
     if (d->batch * d->seqlen * d->nheads > ((int64_t)1 << 31) / 8) return SSD_ERR_UNSUPPORTED;
     if (lay) *lay = l;
     return SSD_OK;

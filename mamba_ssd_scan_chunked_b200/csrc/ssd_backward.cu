@@ -43,10 +43,47 @@ namespace ssd {
 
 static inline size_t al256(size_t v) { return (v + 255) & ~(size_t)255; }
 
+// the tensor-core block form (ssd_backward_tc.cu) for the shapes it covers
+constexpr bool kBwdTensorCoreBlocks = false;
+
 BackwardLayout backward_layout(int64_t batch, int64_t L, int64_t H, int64_t P, int64_t N, int64_t G, int64_t Q,
                                bool io_bf16) {
     BackwardLayout l{};
     const int64_t BH = batch * H;
+    const int64_t nb128 = (L + 127) / 128;
+    if (kBwdTensorCoreBlocks && bwd_tc_supports(H, P, N, G, io_bf16) && batch * (nb128 > 0 ? nb128 : 1) * G <= 65535 &&
+        BH * nb128 < ((int64_t)1 << 31)) {
+        // bf16 inputs, dstate 128, headdim 64, head pairs: the block form on tensor cores
+        l.mode = 2;
+        l.qb = 128;
+        l.nb = nb128;
+        size_t off = 0;
+        auto take = [&](size_t bytes) { const size_t o = off; off = al256(off + bytes); return o; };
+        const int64_t nbk = l.nb > 0 ? l.nb : 1;
+        const size_t st = (size_t)2 * 2 * BH * nbk * N * P;        // bf16 hi and lo
+        l.off_h0 = take(st);
+        l.off_ge = take(st);
+        l.off_part = take(sizeof(float) * 3 * (size_t)batch * nbk * H);
+        int64_t grid = 0, smax = 0;
+        bwd_tc_grid(batch, L, H, G, &grid, &smax);
+        l.off_dbc = take(sizeof(float) * (size_t)grid * smax * 2 * 128 * 128);
+        l.total = off;
+        return l;
+    }
+    if (!io_bf16) {
+        // fp32 inputs: the block form on CUDA cores
+        l.mode = 1;
+        l.qb = blk_block_size((int)P, (int)N);
+        l.nb = (L + l.qb - 1) / l.qb;
+        size_t off = 0;
+        auto take = [&](size_t bytes) { const size_t o = off; off = al256(off + bytes); return o; };
+        const size_t st = sizeof(float) * (size_t)BH * (l.nb > 0 ? l.nb : 1) * N * P;
+        l.off_h0 = take(st);
+        l.off_ge = take(st);
+        l.off_part = take(sizeof(float) * 3 * (size_t)batch * (l.nb > 0 ? l.nb : 1) * H);
+        l.total = off;
+        return l;
+    }
     l.nchunks = (L + Q - 1) / Q;
     l.Lpad = l.nchunks * Q;
     l.tc_main = tc_path_supports(P, N, Q, io_bf16);
@@ -527,6 +564,12 @@ __global__ void bwd_params_kernel(const float* __restrict__ part, float* __restr
 
 // ---------------------------------------------------------------- host side
 
+cudaError_t launch_backward_params(const float* part, float* dA, float* ddt_bias, float* dD, int64_t nseg, int H,
+                                   cudaStream_t s) {
+    bwd_params_kernel<<<(unsigned)((H + 127) / 128), 128, 0, s>>>(part, dA, ddt_bias, dD, nseg, H);
+    return cudaGetLastError();
+}
+
 static unsigned grid_for(int64_t work, int64_t per_block) {
     const int64_t g = (work + per_block - 1) / per_block;
     return (unsigned)(g < 1 ? 1 : (g > 148 * 16 ? 148 * 16 : g));
@@ -695,10 +738,14 @@ cudaError_t launch_backward_empty(const BackwardArgs& a, cudaStream_t s) {
 }
 
 cudaError_t launch_backward(const BackwardArgs& a, cudaStream_t s) {
+    if (a.lay.mode == 1) return launch_backward_blocks_cc(a, s);
+    if (a.lay.mode == 2) return launch_backward_tc(a, s);
     return a.io_bf16 ? backward_g<bf16>(a, s) : backward_g<float>(a, s);
 }
 
 int backward_launches(const BackwardLayout& l, bool has_states) {
+    if (l.mode == 1) return 3;                 // state passes, blocks, parameter sums
+    if (l.mode == 2) return 4;                 // state passes, blocks, dB / dC partial sums, parameter sums
     // a scan is one launch on the tensor-core path, three on the CUDA-core one;
     // prep tokens (+ prep states); F: dt_cumsum, nblk scans, nblk - 1 flag
     // clears; R1: decay kernel and scan; R2: nblk clears and nblk scans; then

@@ -109,6 +109,13 @@ cudaError_t launch_prefill_pair(const PrefillArgs& a, cudaStream_t s);
 // offsets 256-byte aligned; "slice" strides separate the column slices of the
 // transposed scans.
 struct BackwardLayout {
+    // 0: three chunked scans on rearranged operands; 1: block form on CUDA cores
+    // (ssd_backward_blocks.cu); 2: block form on tensor cores (ssd_backward_tc.cu)
+    int mode;
+    int64_t qb, nb;                // block form: tokens per block, blocks per sequence
+    size_t off_h0, off_ge;         // block form: entry states, end adjoints [b*H][nb][N] x
+                                   // (mode 1: fp32 [P]; mode 2: bf16 [2 (hi, lo)][P])
+    size_t off_dbc;                // mode 2: fp32 dB, dC partials [grid * smax][2][128][128]
     int64_t nchunks, Lpad;
     int64_t pw, nblk;              // column-slice width of the transposed scans, slices
     bool tc_main, tc_t;            // tensor-core path for the adjoint scan / transposed scans
@@ -140,6 +147,17 @@ struct BackwardArgs {
 };
 
 cudaError_t launch_backward(const BackwardArgs& a, cudaStream_t s);
+cudaError_t launch_backward_blocks_cc(const BackwardArgs& a, cudaStream_t s);
+// the tensor-core block form: shapes it covers, its CTAs and partial slots per CTA
+bool bwd_tc_supports(int64_t H, int64_t P, int64_t N, int64_t G, bool io_bf16);
+void bwd_tc_grid(int64_t batch, int64_t L, int64_t H, int64_t G, int64_t* grid, int64_t* smax);
+cudaError_t launch_backward_tc(const BackwardArgs& a, cudaStream_t s);
+// tokens per block of the CUDA-core block form, and its shared memory per block
+int blk_block_size(int P, int N);
+size_t blk_smem_bytes(int qb, int P, int N);
+// dA, d dt_bias, dD: part [nseg][H][3] summed over its nseg segments in order
+cudaError_t launch_backward_params(const float* part, float* dA, float* ddt_bias, float* dD, int64_t nseg, int H,
+                                   cudaStream_t s);
 // seqlen 0 (or batch 0): zero parameter gradients, d init_state = dfinal
 cudaError_t launch_backward_empty(const BackwardArgs& a, cudaStream_t s);
 // kernels one ssd_chunk_scan_bwd call launches

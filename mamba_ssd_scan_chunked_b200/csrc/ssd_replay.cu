@@ -185,10 +185,32 @@ replay_step_kernel(StateT* __restrict__ ckpt, IoT* __restrict__ xb, IoT* __restr
     if (!FLUSH) {
         if (lane <= fill) w = beta * cb[bg * 16 + lane];
     } else {
-        for (int s0 = 0; s0 < 16; ++s0) {      // unused slots K..15 get zero coefficients
-            const float bt = __shfl_sync(0xffffffffu, beta, s0);
-            const IoT* bs = s0 < fill ? Bb + (bg * K + s0) * N : bcur;
-            for (int n = lane; n < N; n += 32) gs[n * 17 + s0] = s0 < K ? bt * to_f32(bs[n]) : 0.f;
+        // g[n][s] for the 16 slots (unused slots K..15 get zero coefficients), the B_s
+        // rows read as 16-byte vectors, 8 per lane in flight at once
+        using BV = Vec16<IoT>;
+        constexpr int VE = BV::N;              // elements per vector
+        const int nvr = N / VE, nv = 16 * nvr;
+        for (int v0 = 0; v0 < nv; v0 += 8 * 32) {
+            uint4 raw[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int v = v0 + i * 32 + lane, s = v / nvr, c = v - s * nvr;
+                if (v < nv && s < K) {
+                    const IoT* bs = s < fill ? Bb + (bg * K + s) * N : bcur;
+                    raw[i] = *reinterpret_cast<const uint4*>(bs + c * VE);
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int v = v0 + i * 32 + lane, s = v / nvr, c = v - s * nvr;
+                const float bt = __shfl_sync(0xffffffffu, beta, s & 15);
+                if (v < nv) {
+                    float f[VE];
+                    if (s < K) BV::unpack(raw[i], f);
+#pragma unroll
+                    for (int e = 0; e < VE; ++e) gs[(c * VE + e) * 17 + s] = s < K ? bt * f[e] : 0.f;
+                }
+            }
         }
         __syncwarp();
     }

@@ -285,8 +285,11 @@ def test_backward_workspace_and_launches():
     # tensor-core path: dstate 128 in two 64-column slices for the transposed scans
     assert ssd.ssd_chunk_scan_bwd_launches(d, False) == 1 + 2 * 2 + 2 + 2 * 2 + 3
     assert ssd.ssd_chunk_scan_bwd_launches(d, True) == 1 + 1 + 2 * 2 + 2 + 2 * 2 + 3
-    # fp32 inputs: CUDA-core scans (three launches each), no slicing
-    assert ssd.ssd_chunk_scan_bwd_launches(desc(io_dtype=ssd.SSD_F32), False) == 1 + 4 + 1 + 3 + 4 + 3
+    # fp32 inputs: the block form on CUDA cores (state passes, blocks, parameter sums)
+    assert ssd.ssd_chunk_scan_bwd_launches(desc(io_dtype=ssd.SSD_F32), False) == 3
+    # its workspace: fp32 entry states and end adjoints of every 32-token block
+    nb = -(-L // 32)
+    assert ssd.ssd_chunk_scan_bwd_workspace_size(desc(io_dtype=ssd.SSD_F32)) >= 2 * 4 * b * H * nb * N * P
     with pytest.raises(ssd.SsdError) as e:
         ssd.ssd_chunk_scan_bwd_workspace_size(desc(chunk=100))
     assert e.value.status == UNSUPPORTED
