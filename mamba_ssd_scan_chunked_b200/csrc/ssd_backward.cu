@@ -43,15 +43,12 @@ namespace ssd {
 
 static inline size_t al256(size_t v) { return (v + 255) & ~(size_t)255; }
 
-// the tensor-core block form (ssd_backward_tc.cu) for the shapes it covers
-constexpr bool kBwdTensorCoreBlocks = false;
-
 BackwardLayout backward_layout(int64_t batch, int64_t L, int64_t H, int64_t P, int64_t N, int64_t G, int64_t Q,
                                bool io_bf16) {
     BackwardLayout l{};
     const int64_t BH = batch * H;
     const int64_t nb128 = (L + 127) / 128;
-    if (kBwdTensorCoreBlocks && bwd_tc_supports(H, P, N, G, io_bf16) && batch * (nb128 > 0 ? nb128 : 1) * G <= 65535 &&
+    if (bwd_tc_supports(H, P, N, G, io_bf16) && batch * (nb128 > 0 ? nb128 : 1) * G <= 65535 &&
         BH * nb128 < ((int64_t)1 << 31)) {
         // bf16 inputs, dstate 128, headdim 64, head pairs: the block form on tensor cores
         l.mode = 2;

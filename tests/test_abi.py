@@ -278,13 +278,20 @@ def bwd(d, **ptrs):
 def test_backward_workspace_and_launches():
     d = desc()
     n = ssd.ssd_chunk_scan_bwd_workspace_size(d)
-    # at least the forward's workspace plus the reversed copies and fp32 scan outputs
-    assert n > ssd.ssd_chunk_scan_workspace_size(d)
     b, L, H, P, N = 2, 512, 4, 64, 128
-    assert n >= 4 * b * L * H * P + 2 * 4 * b * L * H * N
-    # tensor-core path: dstate 128 in two 64-column slices for the transposed scans
-    assert ssd.ssd_chunk_scan_bwd_launches(d, False) == 1 + 2 * 2 + 2 + 2 * 2 + 3
-    assert ssd.ssd_chunk_scan_bwd_launches(d, True) == 1 + 1 + 2 * 2 + 2 + 2 * 2 + 3
+    # bf16, dstate 128, headdim 64, an even number of heads per group: the block
+    # form on tensor cores (state passes, block gradients, dB / dC partial sums,
+    # parameter sums); its workspace holds bf16 hi/lo entry states and end
+    # adjoints of every 128-token block
+    assert ssd.ssd_chunk_scan_bwd_launches(d, False) == 4
+    assert ssd.ssd_chunk_scan_bwd_launches(d, True) == 4
+    assert n >= 2 * 2 * 2 * b * H * (L // 128) * N * P
+    # other bf16 shapes: three chunked scans on tensor cores (dstate 256 in four
+    # 64-column slices for the transposed scans)
+    d256 = desc(dstate=256)
+    assert ssd.ssd_chunk_scan_bwd_launches(d256, False) == 1 + 4 * 2 + 2 + 4 * 2 + 3
+    n256 = ssd.ssd_chunk_scan_bwd_workspace_size(d256)
+    assert n256 >= 4 * b * L * H * P + 2 * 4 * b * L * H * 256
     # fp32 inputs: the block form on CUDA cores (state passes, blocks, parameter sums)
     assert ssd.ssd_chunk_scan_bwd_launches(desc(io_dtype=ssd.SSD_F32), False) == 3
     # its workspace: fp32 entry states and end adjoints of every 32-token block
