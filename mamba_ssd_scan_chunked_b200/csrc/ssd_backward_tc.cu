@@ -67,11 +67,12 @@ namespace st {
 constexpr int NCW = 8;                            // compute warps: head k = w / 4, lane quarter w % 4
 constexpr int NCT = NCW * 32;
 constexpr int THREADS = NCT + 32;                 // + the TMA / MMA warp
-constexpr uint32_t STAGE = 4 * TILE;              // N-side tiles (n 0-63, 64-127), P-side tile per head
-constexpr uint32_t OFF_W = 2 * STAGE;             // per head: (w o X) hi, lo
-constexpr uint32_t OFF_TOT = OFF_W + 4 * TILE;    // [2 heads][4 quarters] double: warp totals of the scan
+constexpr uint32_t OFF_N = 0;                     // 2 stages: N-side tiles (n 0-63, 64-127)
+constexpr uint32_t OFF_P = 4 * TILE;              // P-side tile per head (single buffer)
+constexpr uint32_t OFF_W = 6 * TILE;              // 2 buffers x 2 heads: (w o P-side) hi, lo
+constexpr uint32_t OFF_TOT = OFF_W + 8 * TILE;    // [2 heads][4 quarters] double: warp totals of the scan
 constexpr uint32_t OFF_BAR = OFF_TOT + 2 * 4 * 8;
-enum { B_FULL0, B_FULL1, B_WX, B_MMA, NBAR };
+enum { B_FULLN0, B_FULLN1, B_FULLP, B_PFREE, B_WX, B_MMA, NBAR };
 constexpr uint32_t OFF_MISC = OFF_BAR + 8 * NBAR;
 constexpr uint32_t SMEM = OFF_MISC + 16;
 static_assert(SMEM <= 232448, "shared memory per CTA");
@@ -91,6 +92,11 @@ struct Params {
 };
 }  // namespace st
 
+// Per block i of the walk: the compute warps form w o (x or dy) of block i into
+// W buffer i & 1 while the MMAs of block i - 1 still run, then wait for them,
+// write the state out as hi/lo and scale it by 2^(R_last) in TMEM; the MMAs of
+// block i follow.  The P-side tile is reloaded as soon as w o P of block i is
+// formed, the N-side tiles (B or C) two blocks ahead.
 __global__ void __launch_bounds__(st::THREADS, 1)
 bwd_states_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmDY,
                      const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmC,
@@ -111,7 +117,7 @@ bwd_states_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     if (threadIdx.x == NCT) {
-        const uint32_t cnt[NBAR] = {1, 1, NCT, 1};
+        const uint32_t cnt[NBAR] = {1, 1, 1, NCT, NCT, 1};
         for (int i = 0; i < NBAR; ++i) mbar_init(bar(i), cnt[i]);
         *s_abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -140,32 +146,40 @@ bwd_states_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
         const uint32_t lead = elect_one();
         const CUtensorMap* tmN = rev ? &tmC : &tmB;
         const CUtensorMap* tmP = rev ? &tmDY : &tmX;
-        auto load = [&](int i) {
+        auto load_n = [&](int i) {
             const int t0 = blk_of(i) * SUB;
-            const uint32_t stg = base + (uint32_t)(i & 1) * STAGE, bb = bar(B_FULL0 + (i & 1));
-            mbar_expect_tx(bb, 4 * TILE);
+            const uint32_t stg = base + OFF_N + (uint32_t)(i & 1) * 2 * TILE, bb = bar(B_FULLN0 + (i & 1));
+            mbar_expect_tx(bb, 2 * TILE);
             tma_load_4d(stg, tmN, 0, g, t0, b, bb);
             tma_load_4d(stg + TILE, tmN, 64, g, t0, b, bb);
-            tma_load_4d(stg + 2 * TILE, tmP, 0, h0, t0, b, bb);
-            tma_load_4d(stg + 3 * TILE, tmP, 0, h0 + 1, t0, b, bb);
+        };
+        auto load_p = [&](int i) {
+            const int t0 = blk_of(i) * SUB;
+            mbar_expect_tx(bar(B_FULLP), 2 * TILE);
+            tma_load_4d(base + OFF_P, tmP, 0, h0, t0, b, bar(B_FULLP));
+            tma_load_4d(base + OFF_P + TILE, tmP, 0, h0 + 1, t0, b, bar(B_FULLP));
         };
         if (lead) {
-            load(0);
-            if (nblk > 1) load(1);
+            load_n(0);
+            if (nblk > 1) load_n(1);
+            load_p(0);
         }
         __syncwarp();
         constexpr uint32_t ID = idesc_bf16(128, PD, true, true);   // N-side^T (MN-major) x w o P-side (MN-major)
         constexpr uint32_t KSTEP_MN = 2048 >> 4;
         for (int i = 0; i < nblk; ++i) {
-            const uint32_t stg = base + (uint32_t)(i & 1) * STAGE;
-            wait(B_WX, i & 1);               // states scaled, w o X written (implies the tiles landed)
+            wait(B_PFREE, i & 1);            // w o P of block i is formed: the P tile is free
+            if (lead && i + 1 < nblk && !*s_abort) load_p(i + 1);
+            __syncwarp();
+            wait(B_WX, i & 1);               // states written out and scaled
             tc_fence_after();
-            const uint64_t dN = sdesc(stg, TILE, 1024);
+            const uint64_t dN = sdesc(base + OFF_N + (uint32_t)(i & 1) * 2 * TILE, TILE, 1024);
             const bool go = lead && !*s_abort;
+            const uint32_t wb = base + OFF_W + (uint32_t)(i & 1) * 4 * TILE;
 #pragma unroll
             for (int k = 0; k < 2; ++k) {
-                const uint64_t dWh = sdesc(base + OFF_W + 2 * k * TILE, TILE, 1024);
-                const uint64_t dWl = sdesc(base + OFF_W + (2 * k + 1) * TILE, TILE, 1024);
+                const uint64_t dWh = sdesc(wb + 2 * k * TILE, TILE, 1024);
+                const uint64_t dWl = sdesc(wb + (2 * k + 1) * TILE, TILE, 1024);
 #pragma unroll
                 for (int kk = 0; kk < SUB / 16; ++kk) {
                     if (go) mma_ss<ID, 1>(tmem + 64 * k, dN + kk * KSTEP_MN, dWh + kk * KSTEP_MN);
@@ -174,8 +188,8 @@ bwd_states_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
             }
             if (go) mma_commit(bar(B_MMA));
             __syncwarp();
-            wait(B_MMA, i & 1);              // the stage and the w o X tiles are free again
-            if (lead && i + 2 < nblk && !*s_abort) load(i + 2);
+            wait(B_MMA, i & 1);              // the N stage is free again
+            if (lead && i + 2 < nblk && !*s_abort) load_n(i + 2);
             __syncwarp();
         }
     } else {
@@ -188,6 +202,10 @@ bwd_states_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
         const float Ah = p.A[h], bias = p.dt_bias ? p.dt_bias[h] : 0.f;
         double* s_tot = reinterpret_cast<double*>(sm + OFF_TOT);
         const uint16_t* dtr = reinterpret_cast<const uint16_t*>(p.dt_raw);
+        auto fetch = [&](int i) -> uint16_t {
+            const long long t = (long long)blk_of(i) * SUB + row;
+            return t < p.L ? dtr[(b * p.L + t) * p.H + h] : (uint16_t)0;
+        };
         // the starting value of the pass: init_state (forward) or dfinal (backward), else 0
         {
             const void* src = rev ? p.dfinal : p.init_state;
@@ -209,12 +227,13 @@ bwd_states_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
             tmem_wait_st();
         }
         uint16_t* out = rev ? p.ge : p.h0;
+        uint16_t dtr_next = fetch(0);
         for (int i = 0; i < nblk; ++i) {
             const int j = blk_of(i);
             const long long t = (long long)j * SUB + row;
             // dt and the block-local cumsum of dt A log2(e) (double), token s = row
-            float dt = 0.f;
-            if (t < p.L) dt = softplus_f32(__uint_as_float((uint32_t)dtr[(b * p.L + t) * p.H + h] << 16) + bias);
+            const float dt = t < p.L ? softplus_f32(__uint_as_float((uint32_t)dtr_next << 16) + bias) : 0.f;
+            if (i + 1 < nblk) dtr_next = fetch(i + 1);
             double v = (double)(dt * Ah) * (double)LOG2E;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
@@ -234,6 +253,32 @@ bwd_states_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
             const double R = v + off;
             const float wgt = rev ? ex2((float)R) : dt * ex2((float)(tot - R));
             const float scale = ex2((float)tot);
+            // w o (x or dy) of token `row` into W buffer i & 1 (the MMAs of block i - 2,
+            // which read it, completed before block i - 1's state was written out)
+            wait(B_FULLN0 + (i & 1), (i >> 1) & 1);
+            wait(B_FULLP, i & 1);
+            {
+                const uint8_t* src = sm + OFF_P + k * TILE;
+                uint8_t* dh = sm + OFF_W + (i & 1) * 4 * TILE + 2 * k * TILE;
+                uint8_t* dl = dh + TILE;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const uint32_t so = swz(row, c);
+                    const uint4 raw = *reinterpret_cast<const uint4*>(src + so);
+                    const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
+                    uint32_t hw[4], lw[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float a = bf16_lo(wv[e]) * wgt, bb = bf16_hi(wv[e]) * wgt;
+                        hw[e] = pack_bf16(a, bb);
+                        lw[e] = pack_bf16(a - bf16_lo(hw[e]), bb - bf16_hi(hw[e]));
+                    }
+                    *reinterpret_cast<uint4*>(dh + so) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                    *reinterpret_cast<uint4*>(dl + so) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+                }
+            }
+            fence_proxy_async();
+            mbar_arrive(bar(B_PFREE));
             // the previous block's update is complete: write the value out, scale it
             if (i > 0) wait(B_MMA, (i - 1) & 1);
             tc_fence_after();
@@ -264,29 +309,6 @@ bwd_states_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
                 }
                 tmem_wait_st();
             }
-            // w o (x or dy) of token `row`, as hi and lo tiles (MN-major B operand)
-            wait(B_FULL0 + (i & 1), (i >> 1) & 1);
-            {
-                const uint8_t* src = sm + (i & 1) * STAGE + (2 + k) * TILE;
-                uint8_t* dh = sm + OFF_W + 2 * k * TILE;
-                uint8_t* dl = dh + TILE;
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const uint32_t so = swz(row, c);
-                    const uint4 raw = *reinterpret_cast<const uint4*>(src + so);
-                    const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
-                    uint32_t hw[4], lw[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float a = bf16_lo(wv[e]) * wgt, bb = bf16_hi(wv[e]) * wgt;
-                        hw[e] = pack_bf16(a, bb);
-                        lw[e] = pack_bf16(a - bf16_lo(hw[e]), bb - bf16_hi(hw[e]));
-                    }
-                    *reinterpret_cast<uint4*>(dh + so) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-                    *reinterpret_cast<uint4*>(dl + so) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-                }
-            }
-            fence_proxy_async();
             tc_fence_before();
             mbar_arrive(bar(B_WX));
         }
@@ -323,28 +345,32 @@ bwd_states_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 128;" ::"r"(tmem) : "memory");
 }
 
+}  // namespace bwdtc
 
+namespace bwdtc {
 // ============================================================ 2. block gradients
 //
 // Unit u = ((b * nblk + j) * G + g) * hpg + q: head g*hpg + q of block j of
 // batch element b.  CTA c takes units [c U / grid, (c + 1) U / grid); a run of
 // its units with the same (b, j, g) is a segment, whose dB and dC accumulate in
 // TMEM over the segment's heads and leave as one partial.  Per unit (rows s or
-// l are the block's tokens, 128 TMEM lanes):
+// l are the block's tokens, 128 TMEM lanes), in issue order:
 //
 //   M1  S^T = B C^T                           -> TMEM S
 //   M2  X dY^T                                -> TMEM X
-//   C1  (w o X), (2^R o dY) as hi/lo tiles; x.dy; <Ge, h0> shares
-//   M3  dB += (w o X) Ge^T, dC += (2^R o dY) h0^T     (hi.hi + hi.lo + lo.hi)
 //   C2  transform: Mt = S^T e (in TMEM S as bf16 hi|lo), dS^T = dt_s e X dY^T
 //       (hi/lo tiles), e = 2^(R_l - R_s) [l >= s]; column and row sums of S dS
 //   M4  B Ge -> TMEM X[0:64], C h0 -> TMEM X[64:128]
-//   M5  dB += dS^T C, dC += dS B
 //   C3  u_l = 2^(R_l) dy_l . (C h0)_l, v_s = w_s x_s . (B Ge)_s
 //   M6  Mt dY -> TMEM X[64:128]
-//   C4  dxu = Mt dY + 2^(R_last - R_s) B Ge; dx; x . dxu; then d a, d dt_raw and
-//       the unit's shares of dA, d dt_bias, dD
+//   C4  dxu = Mt dY + 2^(R_last - R_s) B Ge; dx; x . dxu; d a, d dt_raw and the
+//       unit's shares of dA, d dt_bias, dD
+//   M5  dB += dS^T C, dC += dS B
+//   C1  (w o X), (2^R o dY) as hi/lo tiles over the consumed dS^T
+//   M3  dB += (w o X) Ge^T, dC += (2^R o dY) h0^T     (hi.hi + hi.lo + lo.hi)
 //   end of segment: TMEM dB, dC -> partial slot
+// The chain that gives dx and d a (M1 .. C4) does not wait for the dB, dC MMAs
+// (M5, M3), which run while the next unit's operands load.
 namespace mn {
 constexpr int NCW = 16;
 constexpr int NCT = NCW * 32;
@@ -353,21 +379,23 @@ constexpr int THREADS = NCT + 64;
 constexpr uint32_t COL_S = 0, COL_X = 128, COL_DB = 256, COL_DC = 384;
 constexpr uint32_t OFF_B = 0;                    // B tiles: n 0-63, n 64-127 (rows = tokens)
 constexpr uint32_t OFF_C = 2 * TILE;             // C tiles
-constexpr uint32_t OFF_X = 4 * TILE;             // x tile (rows = tokens, 64 p)
+constexpr uint32_t OFF_X = 4 * TILE;             // x tile (rows = tokens, 64 p); later the unit's scratch
 constexpr uint32_t OFF_DY = 5 * TILE;            // dy tile
 constexpr uint32_t OFF_H0 = 6 * TILE;            // h0 hi, lo (rows = n, 64 p)
 constexpr uint32_t OFF_GE = 8 * TILE;            // Ge hi, lo
-constexpr uint32_t OFF_WD = 10 * TILE;           // (w o X) hi, lo, (2^R o dY) hi, lo; later dS^T
-                                                 // hi (l 0-63, 64-127), lo (l 0-63, 64-127); then scratch
+constexpr uint32_t OFF_WD = 10 * TILE;           // dS^T hi (l 0-63, 64-127), lo (l 0-63, 64-127);
+                                                 // later (w o X) hi, lo, (2^R o dY) hi, lo
 constexpr uint32_t OFF_RT = 14 * TILE;           // float2 [128]: R (hi, lo) of the block's tokens
 constexpr uint32_t OFF_TOT = OFF_RT + 128 * 8;   // double [4]: scan totals of the lane quarters
 constexpr uint32_t OFF_BAR = OFF_TOT + 4 * 8;
-enum { F_BC, F_X, F_DY, F_HG, M_SX, C_WE, M_WE, C_T, M_BC, C_U, M_DX, C_E, C_FL, NBAR };
+enum { F_BC, F_X, F_DY, F_HG, M_SX, C_T, M_BC, C_U, M_DX, C_E, M_DS, C_WE, M_WE, C_FL, NBAR };
 constexpr uint32_t OFF_MISC = OFF_BAR + 8 * NBAR;
 constexpr uint32_t SMEM = OFF_MISC + 16;
 static_assert(SMEM <= 232448, "shared memory per CTA");
-// scratch in the OFF_WD region once dS^T is consumed: floats
+// scratch in the x tile (floats) once its values are in registers and M2 has run
 constexpr int SC_C = 0, SC_R = 512, SC_U = 1024, SC_V = 1536, SC_XDY = 2048, SC_XDXU = 2560, SC_K = 3072;
+constexpr int SC_END = 3584;
+static_assert(SC_END * 4 <= (int)TILE, "scratch fits the x tile");
 
 struct Params {
     const void* x;             // bf16 [b][L][H][P]
@@ -407,8 +435,8 @@ bwd_main_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     if (threadIdx.x == NCT) {
-        //                          BC X  DY HG SX WE   MWE T    MBC U    MDX E    FL
-        const uint32_t cnt[NBAR] = {1, 1, 1, 1, 1, NCT, 1, NCT, 1, NCT, 1, NCT, NCT};
+        //                          BC X  DY HG SX T    BC U    DX E    DS WE   MWE FL
+        const uint32_t cnt[NBAR] = {1, 1, 1, 1, 1, NCT, 1, NCT, 1, NCT, 1, NCT, 1, NCT};
         for (int i = 0; i < NBAR; ++i) mbar_init(bar(i), cnt[i]);
         *s_abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -427,8 +455,8 @@ bwd_main_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
         const long long u = u0 + i;
         Unit d;
         d.seg = u / hpg;
-        d.h = (int)(d.seg % p.G) * hpg + (int)(u % hpg);
         d.g = (int)(d.seg % p.G);
+        d.h = d.g * hpg + (int)(u % hpg);
         d.j = (int)((d.seg / p.G) % p.nblk);
         d.b = (int)(d.seg / p.G / p.nblk);
         d.first = i == 0 || u % hpg == 0;
@@ -449,47 +477,43 @@ bwd_main_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
             const Unit d = unit(i);
             const int t0 = d.j * SUB;
             const long long un = ((long long)d.b * p.H + d.h) * p.nblk + d.j;   // state unit (b, h, j)
-            if (d.first) {
-                if (i > 0) wait(M_DX, (i - 1) & 1);     // the previous segment's last dS MMAs are done
-                if (lead && !*s_abort) {
+            // x, dy: read by M2, M6 and into registers; the x tile was the previous unit's scratch
+            if (i > 0) { wait(M_DX, (i - 1) & 1); wait(C_E, (i - 1) & 1); }
+            if (lead && !*s_abort) {
+                mbar_expect_tx(bar(F_X), TILE);
+                tma_load_4d(base + OFF_X, &tmX, 0, d.h, t0, d.b, bar(F_X));
+                mbar_expect_tx(bar(F_DY), TILE);
+                tma_load_4d(base + OFF_DY, &tmDY, 0, d.h, t0, d.b, bar(F_DY));
+                if (i + 1 < nu) {                    // the next unit's x, dy into L2
+                    const Unit e = unit(i + 1);
+                    tma_prefetch_4d(&tmX, 0, e.h, e.j * SUB, e.b);
+                    tma_prefetch_4d(&tmDY, 0, e.h, e.j * SUB, e.b);
+                }
+            }
+            // h0, Ge (and at a segment's start B, C): the previous unit's MMAs are all done
+            if (i > 0) wait(M_WE, (i - 1) & 1);
+            if (lead && !*s_abort) {
+                if (d.first) {
                     mbar_expect_tx(bar(F_BC), 4 * TILE);
                     tma_load_4d(base + OFF_B, &tmB, 0, d.g, t0, d.b, bar(F_BC));
                     tma_load_4d(base + OFF_B + TILE, &tmB, 64, d.g, t0, d.b, bar(F_BC));
                     tma_load_4d(base + OFF_C, &tmC, 0, d.g, t0, d.b, bar(F_BC));
                     tma_load_4d(base + OFF_C + TILE, &tmC, 64, d.g, t0, d.b, bar(F_BC));
                 }
-                ++nseg;
-            }
-            // x: read by M2 and C1 of the previous unit
-            if (i > 0) { wait(M_SX, (i - 1) & 1); wait(C_WE, (i - 1) & 1); }
-            if (lead && !*s_abort) {
-                mbar_expect_tx(bar(F_X), TILE);
-                tma_load_4d(base + OFF_X, &tmX, 0, d.h, t0, d.b, bar(F_X));
-            }
-            // h0, Ge: read by M3, M4 (and C1) of the previous unit
-            if (i > 0) wait(M_BC, (i - 1) & 1);
-            if (lead && !*s_abort) {
                 mbar_expect_tx(bar(F_HG), 4 * TILE);
                 tma_load_4d(base + OFF_H0, &tmH0, 0, 0, 0, (int)un, bar(F_HG));
                 tma_load_4d(base + OFF_H0 + TILE, &tmH0, 0, 1, 0, (int)un, bar(F_HG));
                 tma_load_4d(base + OFF_GE, &tmGE, 0, 0, 0, (int)un, bar(F_HG));
                 tma_load_4d(base + OFF_GE + TILE, &tmGE, 0, 1, 0, (int)un, bar(F_HG));
             }
-            // dy: read by M2, C1, C3 and M6 of the previous unit
-            if (i > 0) { wait(M_DX, (i - 1) & 1); wait(C_U, (i - 1) & 1); }
-            if (lead && !*s_abort) {
-                mbar_expect_tx(bar(F_DY), TILE);
-                tma_load_4d(base + OFF_DY, &tmDY, 0, d.h, t0, d.b, bar(F_DY));
-            }
+            if (d.first) ++nseg;
             __syncwarp();
         }
         (void)nseg;
     } else if (warp == WARP_MMA) {
         // ======================================================== MMA issue
         const uint32_t lead0 = elect_one();
-        constexpr uint32_t ID_SS = idesc_bf16(128, 128, false, false);     // K-major x K-major, N = 128
-        constexpr uint32_t ID_XD = idesc_bf16(128, 128, false, false);     // X (K-major) x dY^T (K-major)
-        constexpr uint32_t ID_KN = idesc_bf16(128, 128, false, false);     // (w o X) x Ge^T: both K-major over p
+        constexpr uint32_t ID_KK = idesc_bf16(128, 128, false, false);     // K-major x K-major, N = 128
         constexpr uint32_t ID_P64 = idesc_bf16(128, PD, false, true);      // K-major x MN-major, N = 64
         constexpr uint32_t ID_DB = idesc_bf16(128, 128, false, true);      // dS^T (K-major) x C (MN-major)
         constexpr uint32_t ID_DC = idesc_bf16(128, 128, true, true);       // dS (MN-major) x B (MN-major)
@@ -506,7 +530,7 @@ bwd_main_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
             }
             wait(F_X, ph);
             wait(F_DY, ph);
-            if (i > 0) { wait(M_DX, ph ^ 1u); wait(C_E, ph ^ 1u); }   // TMEM S and X free
+            if (i > 0) wait(C_E, ph ^ 1u);           // TMEM X read (and TMEM S: M6 completed before)
             tc_fence_after();
             __syncwarp();
             // M1: S^T = B C^T (K = n, 8 steps); M2: X dY^T (K = p, 4 steps)
@@ -515,49 +539,21 @@ bwd_main_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
                     const uint32_t o = (uint32_t)(k >> 2) * KBLOCK_K + (uint32_t)(k & 3) * KSTEP_K;
-                    if (k == 0) { if (lead) mma_ss<ID_SS, 0>(tmem + COL_S, dB + o, dC + o);
-                    } else if (lead) mma_ss<ID_SS, 1>(tmem + COL_S, dB + o, dC + o);
+                    if (k == 0) { if (lead) mma_ss<ID_KK, 0>(tmem + COL_S, dB + o, dC + o);
+                    } else if (lead) mma_ss<ID_KK, 1>(tmem + COL_S, dB + o, dC + o);
                 }
                 const uint64_t dX = sdesc(base + OFF_X, 16, 1024), dY = sdesc(base + OFF_DY, 16, 1024);
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
                     const uint32_t o = (uint32_t)k * KSTEP_K;
-                    if (k == 0) { if (lead) mma_ss<ID_XD, 0>(tmem + COL_X, dX + o, dY + o);
-                    } else if (lead) mma_ss<ID_XD, 1>(tmem + COL_X, dX + o, dY + o);
+                    if (k == 0) { if (lead) mma_ss<ID_KK, 0>(tmem + COL_X, dX + o, dY + o);
+                    } else if (lead) mma_ss<ID_KK, 1>(tmem + COL_X, dX + o, dY + o);
                 }
                 if (lead) mma_commit(bar(M_SX));
             }
-            // M3: dB += (w o X) Ge^T, dC += (2^R o dY) h0^T (K = p, 4 steps; hi.hi, hi.lo, lo.hi)
-            wait(C_WE, ph);
-            wait(F_HG, ph);
-            if (d.first && nseg > 1) wait(C_FL, (nseg - 2) & 1);     // the previous partial is out
-            tc_fence_after();
-            __syncwarp();
-            {
-                const uint64_t wh = sdesc(base + OFF_WD, 16, 1024), wl = sdesc(base + OFF_WD + TILE, 16, 1024);
-                const uint64_t eh = sdesc(base + OFF_WD + 2 * TILE, 16, 1024);
-                const uint64_t el = sdesc(base + OFF_WD + 3 * TILE, 16, 1024);
-                const uint64_t gh = sdesc(base + OFF_GE, 16, 1024), gl = sdesc(base + OFF_GE + TILE, 16, 1024);
-                const uint64_t hh = sdesc(base + OFF_H0, 16, 1024), hl = sdesc(base + OFF_H0 + TILE, 16, 1024);
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const uint32_t o = (uint32_t)k * KSTEP_K;
-                    if (k == 0 && d.first) {
-                        if (lead) mma_ss<ID_KN, 0>(tmem + COL_DB, wh + o, gh + o);
-                        if (lead) mma_ss<ID_KN, 0>(tmem + COL_DC, eh + o, hh + o);
-                    } else {
-                        if (lead) mma_ss<ID_KN, 1>(tmem + COL_DB, wh + o, gh + o);
-                        if (lead) mma_ss<ID_KN, 1>(tmem + COL_DC, eh + o, hh + o);
-                    }
-                    if (lead) mma_ss<ID_KN, 1>(tmem + COL_DB, wh + o, gl + o);
-                    if (lead) mma_ss<ID_KN, 1>(tmem + COL_DB, wl + o, gh + o);
-                    if (lead) mma_ss<ID_KN, 1>(tmem + COL_DC, eh + o, hl + o);
-                    if (lead) mma_ss<ID_KN, 1>(tmem + COL_DC, el + o, hh + o);
-                }
-                if (lead) mma_commit(bar(M_WE));
-            }
             // M4: B Ge -> X[0:64], C h0 -> X[64:128] (K = n, 8 steps; Ge, h0 MN-major, hi + lo)
             wait(C_T, ph);
+            wait(F_HG, ph);
             tc_fence_after();
             __syncwarp();
             {
@@ -579,22 +575,6 @@ bwd_main_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
                 }
                 if (lead) mma_commit(bar(M_BC));
             }
-            // M5: dB += dS^T C (K = l), dC += dS B (K = s); dS^T hi/lo tiles in OFF_WD
-            {
-                const uint64_t dCm = sdesc(base + OFF_C, TILE, 1024), dBm = sdesc(base + OFF_B, TILE, 1024);
-#pragma unroll
-                for (int hl = 0; hl < 2; ++hl) {
-                    const uint32_t ds = base + OFF_WD + 2 * hl * TILE;
-                    const uint64_t aK = sdesc(ds, 16, 1024);       // dS^T as K-major A (rows s, K = l)
-                    const uint64_t aM = sdesc(ds, TILE, 1024);     // dS as MN-major A (M = l, K = s rows)
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        const uint32_t o = (uint32_t)(k >> 2) * KBLOCK_K + (uint32_t)(k & 3) * KSTEP_K;
-                        if (lead) mma_ss<ID_DB, 1>(tmem + COL_DB, aK + o, dCm + k * KSTEP_MN);
-                        if (lead) mma_ss<ID_DC, 1>(tmem + COL_DC, aM + k * KSTEP_MN, dBm + k * KSTEP_MN);
-                    }
-                }
-            }
             // M6: Mt dY -> X[64:128] (A = Mt hi|lo from TMEM S, K = l)
             wait(C_U, ph);
             tc_fence_after();
@@ -609,6 +589,53 @@ bwd_main_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
                 }
                 if (lead) mma_commit(bar(M_DX));
             }
+            // M5: dB += dS^T C (K = l), dC += dS B (K = s); the segment's first MMAs overwrite
+            if (d.first && nseg > 1) wait(C_FL, (nseg - 2) & 1);     // the previous partial is out
+            tc_fence_after();
+            __syncwarp();
+            {
+                const uint64_t dCm = sdesc(base + OFF_C, TILE, 1024), dBm = sdesc(base + OFF_B, TILE, 1024);
+#pragma unroll
+                for (int hl = 0; hl < 2; ++hl) {
+                    const uint32_t ds = base + OFF_WD + 2 * hl * TILE;
+                    const uint64_t aK = sdesc(ds, 16, 1024);       // dS^T as K-major A (rows s, K = l)
+                    const uint64_t aM = sdesc(ds, TILE, 1024);     // dS as MN-major A (M = l, K = s rows)
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const uint32_t o = (uint32_t)(k >> 2) * KBLOCK_K + (uint32_t)(k & 3) * KSTEP_K;
+                        if (hl == 0 && k == 0 && d.first) {
+                            if (lead) mma_ss<ID_DB, 0>(tmem + COL_DB, aK + o, dCm);
+                            if (lead) mma_ss<ID_DC, 0>(tmem + COL_DC, aM, dBm);
+                        } else {
+                            if (lead) mma_ss<ID_DB, 1>(tmem + COL_DB, aK + o, dCm + k * KSTEP_MN);
+                            if (lead) mma_ss<ID_DC, 1>(tmem + COL_DC, aM + k * KSTEP_MN, dBm + k * KSTEP_MN);
+                        }
+                    }
+                }
+                if (lead) mma_commit(bar(M_DS));
+            }
+            // M3: dB += (w o X) Ge^T, dC += (2^R o dY) h0^T (K = p, 4 steps; hi.hi, hi.lo, lo.hi)
+            wait(C_WE, ph);
+            tc_fence_after();
+            __syncwarp();
+            {
+                const uint64_t wh = sdesc(base + OFF_WD, 16, 1024), wl = sdesc(base + OFF_WD + TILE, 16, 1024);
+                const uint64_t eh = sdesc(base + OFF_WD + 2 * TILE, 16, 1024);
+                const uint64_t el = sdesc(base + OFF_WD + 3 * TILE, 16, 1024);
+                const uint64_t gh = sdesc(base + OFF_GE, 16, 1024), gl = sdesc(base + OFF_GE + TILE, 16, 1024);
+                const uint64_t hh = sdesc(base + OFF_H0, 16, 1024), hl = sdesc(base + OFF_H0 + TILE, 16, 1024);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const uint32_t o = (uint32_t)k * KSTEP_K;
+                    if (lead) mma_ss<ID_KK, 1>(tmem + COL_DB, wh + o, gh + o);
+                    if (lead) mma_ss<ID_KK, 1>(tmem + COL_DC, eh + o, hh + o);
+                    if (lead) mma_ss<ID_KK, 1>(tmem + COL_DB, wh + o, gl + o);
+                    if (lead) mma_ss<ID_KK, 1>(tmem + COL_DB, wl + o, gh + o);
+                    if (lead) mma_ss<ID_KK, 1>(tmem + COL_DC, eh + o, hl + o);
+                    if (lead) mma_ss<ID_KK, 1>(tmem + COL_DC, el + o, hh + o);
+                }
+                if (lead) mma_commit(bar(M_WE));
+            }
             __syncwarp();
         }
     } else {
@@ -618,27 +645,23 @@ bwd_main_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
         const uint32_t lo16 = (uint32_t)(32 * q) << 16;
         float2* s_rt = reinterpret_cast<float2*>(sm + OFF_RT);
         double* s_tot = reinterpret_cast<double*>(sm + OFF_TOT);
-        float* scr = reinterpret_cast<float*>(sm + OFF_WD);
+        float* scr = reinterpret_cast<float*>(sm + OFF_X);
         const uint16_t* dtr = reinterpret_cast<const uint16_t*>(p.dt_raw);
-        const uint16_t* xg = reinterpret_cast<const uint16_t*>(p.x);
-        const uint16_t* dyg = reinterpret_cast<const uint16_t*>(p.dy);
         auto csync = [&]() { asm volatile("bar.sync 1, %0;" ::"r"(NCT) : "memory"); };
-        int nseg = 0;
-        float dtr_next = 0.f;
-        auto fetch_dtr = [&](int i) -> float {
+        uint16_t dtr_next = 0;
+        auto fetch_dtr = [&](int i) -> uint16_t {
             const Unit d = unit(i);
             const long long t = (long long)d.j * SUB + row;
-            return t < p.L ? __uint_as_float((uint32_t)dtr[((long long)d.b * p.L + t) * p.H + d.h] << 16) : 0.f;
+            return t < p.L ? dtr[((long long)d.b * p.L + t) * p.H + d.h] : (uint16_t)0;
         };
         if (nu > 0) dtr_next = fetch_dtr(0);
         for (int i = 0; i < nu; ++i) {
             const Unit d = unit(i);
             const uint32_t ph = i & 1;
-            if (d.first) ++nseg;
             const long long t = (long long)d.j * SUB + row;
             const bool valid = t < p.L;
             const float Ah = p.A[d.h], bias = p.dt_bias ? p.dt_bias[d.h] : 0.f;
-            const float z = dtr_next + bias;
+            const float z = __uint_as_float((uint32_t)dtr_next << 16) + bias;
             const float dt = valid ? softplus_f32(z) : 0.f;
             if (i + 1 < nu) dtr_next = fetch_dtr(i + 1);
             // ---- P1: block-local cumsum R of dt A log2(e) (double), per token
@@ -649,7 +672,7 @@ bwd_main_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
                 if (lane >= o) v += w;
             }
             if (c == 0 && lane == 31) s_tot[q] = v;
-            csync();
+            csync();                                        // (also: every thread is past the previous unit)
             double off = 0.0, tot = 0.0;
 #pragma unroll
             for (int w = 0; w < 4; ++w) {
@@ -663,91 +686,62 @@ bwd_main_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
             const float er = ex2(Rhi + Rlo);               // 2^(R_s)
             const float wv = dt * wt;                      // w_s
             if (c == 0) s_rt[row] = make_float2(Rhi, Rlo);
-            // ---- C1: (w o X), (2^R o dY) hi/lo; x . dy; <Ge, h0>
+            // ---- x and dy of this row, columns 16c .. 16c + 15, into registers
             wait(F_X, ph);
             wait(F_DY, ph);
-            if (i > 0) wait(M_DX, ph ^ 1u);                 // the previous dS^T (and scratch) are consumed
-            csync();                                        // ... and every thread is past its scratch reads
+            uint32_t xr[8], yr[8];
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc) {
+                const uint32_t so = swz(row, 2 * c + cc);
+                const uint4 a4 = *reinterpret_cast<const uint4*>(sm + OFF_X + so);
+                const uint4 b4 = *reinterpret_cast<const uint4*>(sm + OFF_DY + so);
+                xr[4 * cc] = a4.x; xr[4 * cc + 1] = a4.y; xr[4 * cc + 2] = a4.z; xr[4 * cc + 3] = a4.w;
+                yr[4 * cc] = b4.x; yr[4 * cc + 1] = b4.y; yr[4 * cc + 2] = b4.z; yr[4 * cc + 3] = b4.w;
+            }
             float xdy = 0.f;
-            {
 #pragma unroll
-                for (int cc = 0; cc < 2; ++cc) {
-                    const int ch = 2 * c + cc;              // 16-byte chunk of the 128-byte row
-                    const uint32_t so = swz(row, ch);
-                    const uint4 xr = *reinterpret_cast<const uint4*>(sm + OFF_X + so);
-                    const uint4 yr = *reinterpret_cast<const uint4*>(sm + OFF_DY + so);
-                    const uint32_t xw[4] = {xr.x, xr.y, xr.z, xr.w}, yw[4] = {yr.x, yr.y, yr.z, yr.w};
-                    uint32_t ah[4], al[4], bh[4], bl[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float x0 = bf16_lo(xw[e]), x1 = bf16_hi(xw[e]);
-                        const float y0 = bf16_lo(yw[e]), y1 = bf16_hi(yw[e]);
-                        xdy = fmaf(x0, y0, fmaf(x1, y1, xdy));
-                        const float a0 = wv * x0, a1 = wv * x1, b0 = er * y0, b1 = er * y1;
-                        ah[e] = pack_bf16(a0, a1);
-                        al[e] = pack_bf16(a0 - bf16_lo(ah[e]), a1 - bf16_hi(ah[e]));
-                        bh[e] = pack_bf16(b0, b1);
-                        bl[e] = pack_bf16(b0 - bf16_lo(bh[e]), b1 - bf16_hi(bh[e]));
-                    }
-                    *reinterpret_cast<uint4*>(sm + OFF_WD + so) = make_uint4(ah[0], ah[1], ah[2], ah[3]);
-                    *reinterpret_cast<uint4*>(sm + OFF_WD + TILE + so) = make_uint4(al[0], al[1], al[2], al[3]);
-                    *reinterpret_cast<uint4*>(sm + OFF_WD + 2 * TILE + so) = make_uint4(bh[0], bh[1], bh[2], bh[3]);
-                    *reinterpret_cast<uint4*>(sm + OFF_WD + 3 * TILE + so) = make_uint4(bl[0], bl[1], bl[2], bl[3]);
-                }
-            }
-            wait(F_HG, ph);
-            float kp = 0.f;                                  // share of <Ge, h0>: row n = row, 16 columns
-            {
-#pragma unroll
-                for (int cc = 0; cc < 2; ++cc) {
-                    const uint32_t so = swz(row, 2 * c + cc);
-                    const uint4 gh = *reinterpret_cast<const uint4*>(sm + OFF_GE + so);
-                    const uint4 gl = *reinterpret_cast<const uint4*>(sm + OFF_GE + TILE + so);
-                    const uint4 hh = *reinterpret_cast<const uint4*>(sm + OFF_H0 + so);
-                    const uint4 hl = *reinterpret_cast<const uint4*>(sm + OFF_H0 + TILE + so);
-                    const uint32_t a[4] = {gh.x, gh.y, gh.z, gh.w}, a2[4] = {gl.x, gl.y, gl.z, gl.w};
-                    const uint32_t b[4] = {hh.x, hh.y, hh.z, hh.w}, b2[4] = {hl.x, hl.y, hl.z, hl.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        kp = fmaf(bf16_lo(a[e]) + bf16_lo(a2[e]), bf16_lo(b[e]) + bf16_lo(b2[e]), kp);
-                        kp = fmaf(bf16_hi(a[e]) + bf16_hi(a2[e]), bf16_hi(b[e]) + bf16_hi(b2[e]), kp);
-                    }
-                }
-            }
-            fence_proxy_async();
-            mbar_arrive(bar(C_WE));
-            // ---- C2: the transform of the tile (rows 32q.., columns 32c..)
+            for (int e = 0; e < 8; ++e) xdy = fmaf(bf16_lo(xr[e]), bf16_lo(yr[e]), fmaf(bf16_hi(xr[e]), bf16_hi(yr[e]), xdy));
+            // ---- C2: the transform of the tile (rows 32q.., columns 32c..); dS^T goes over
+            // the previous unit's (w o X), (2^R o dY) tiles
             wait(M_SX, ph);
-            wait(M_WE, ph);                                  // the WE tiles are consumed: dS^T may go there
+            if (i > 0) wait(M_WE, ph ^ 1u);
             tc_fence_after();
-            csync();                                         // the R table is complete
-            float csum = 0.f, rsum[2] = {0.f, 0.f};
+            csync();                                         // the R table is complete, x is in registers
+            float csum = 0.f, rsum[4];
 #pragma unroll
-            for (int ks = 0; ks < 2; ++ks) {
-                // one 16-column K step: columns lc .. lc + 15
-                const int lc = 32 * c + 16 * ks;
-                uint32_t sv[16], xv[16];
+            for (int ks2 = 0; ks2 < 2; ++ks2) {
+                // one 16-column K step: its S^T is read whole before Mt overwrites it in place
+                const int kb = 32 * c + 16 * ks2;
+                uint32_t sv[16];
                 if (c >= q) {
-                    tmem_ld16(tmem + lo16 + COL_S + lc, sv);
-                    tmem_ld16(tmem + lo16 + COL_X + lc, xv);
+                    tmem_ld16(tmem + lo16 + COL_S + kb, sv);
                     tmem_wait_ld();
                 }
-                float wcol[16];
 #pragma unroll
                 for (int h8 = 0; h8 < 2; ++h8) {
+                    // 8 columns lc .. lc + 7
+                    const int ch = 2 * ks2 + h8, lc = kb + 8 * h8;
+                    uint32_t xv[8];
+                    float wcol[8];
+                    if (c >= q) {
+                        asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                                     : "=r"(xv[0]), "=r"(xv[1]), "=r"(xv[2]), "=r"(xv[3]), "=r"(xv[4]), "=r"(xv[5]),
+                                       "=r"(xv[6]), "=r"(xv[7]) : "r"(tmem + lo16 + COL_X + lc));
+                        tmem_wait_ld();
+                    }
                     uint32_t mh[4], ml[4], dh[4], dl[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         float m2[2], g2[2];
 #pragma unroll
                         for (int z2 = 0; z2 < 2; ++z2) {
-                            const int kc = 8 * h8 + 2 * e + z2;      // column within the K step
+                            const int kc = 2 * e + z2;
                             const int l = lc + kc;
                             float m = 0.f, gd = 0.f, wcl = 0.f;
                             if (c >= q && l >= row) {
                                 const float2 rl = s_rt[l];
                                 const float f = ex2((rl.x - Rhi) + (rl.y - Rlo));
-                                const float sval = __uint_as_float(sv[kc]);
+                                const float sval = __uint_as_float(sv[8 * h8 + kc]);
                                 m = sval * f;
                                 gd = dt * f * __uint_as_float(xv[kc]);
                                 if (l > row) {
@@ -764,60 +758,66 @@ bwd_main_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
                         dh[e] = pack_bf16(g2[0], g2[1]);
                         dl[e] = pack_bf16(g2[0] - bf16_lo(dh[e]), g2[1] - bf16_hi(dh[e]));
                     }
-                    // Mt as the TMEM A operand: per K step 8 words hi, then 8 words lo
-                    tmem_st4(tmem + lo16 + COL_S + lc + 4 * h8, mh);
-                    tmem_st4(tmem + lo16 + COL_S + lc + 8 + 4 * h8, ml);
-                    // dS^T hi / lo: K block lc / 64, 16-byte chunk (lc % 64) / 8 + h8
-                    const uint32_t so = (uint32_t)(lc >> 6) * TILE + swz(row, ((lc & 63) >> 3) + h8);
+                    // Mt as the TMEM A operand: per 16-column K step 8 words hi, then 8 words lo
+                    tmem_st4(tmem + lo16 + COL_S + kb + 4 * h8, mh);
+                    tmem_st4(tmem + lo16 + COL_S + kb + 8 + 4 * h8, ml);
+                    // dS^T hi / lo: K block lc / 64, 16-byte chunk (lc % 64) / 8
+                    const uint32_t so = (uint32_t)(lc >> 6) * TILE + swz(row, (lc & 63) >> 3);
                     *reinterpret_cast<uint4*>(sm + OFF_WD + so) = make_uint4(dh[0], dh[1], dh[2], dh[3]);
                     *reinterpret_cast<uint4*>(sm + OFF_WD + 2 * TILE + so) = make_uint4(dl[0], dl[1], dl[2], dl[3]);
-                }
-                // row sums over this warp's 32 rows of the 16 columns: lanes i and i + 16
-                // end with column lc + (i & 15)
+                    // row sums over this warp's 32 rows of the 8 columns: lane i ends with column lc + (i & 7)
 #pragma unroll
-                for (int e = 0; e < 16; ++e) wcol[e] += __shfl_xor_sync(0xffffffffu, wcol[e], 16);
+                    for (int e = 0; e < 8; ++e) wcol[e] += __shfl_xor_sync(0xffffffffu, wcol[e], 16);
 #pragma unroll
-                for (int w = 8; w >= 1; w >>= 1) {
+                    for (int e = 0; e < 8; ++e) wcol[e] += __shfl_xor_sync(0xffffffffu, wcol[e], 8);
 #pragma unroll
-                    for (int e = 0; e < w; ++e) {
-                        const bool up = (lane & w) != 0;
-                        const float send = up ? wcol[e] : wcol[e + w];
-                        const float keep = up ? wcol[e + w] : wcol[e];
-                        wcol[e] = keep + __shfl_xor_sync(0xffffffffu, send, w);
+                    for (int w = 4; w >= 1; w >>= 1) {
+#pragma unroll
+                        for (int e = 0; e < w; ++e) {
+                            const bool up = (lane & w) != 0;
+                            const float send = up ? wcol[e] : wcol[e + w];
+                            const float keep = up ? wcol[e + w] : wcol[e];
+                            wcol[e] = keep + __shfl_xor_sync(0xffffffffu, send, w);
+                        }
                     }
+                    rsum[ch] = wcol[0];
                 }
-                rsum[ks] = wcol[0];
             }
             tmem_wait_st();
             fence_proxy_async();
             tc_fence_before();
             mbar_arrive(bar(C_T));
+            // ---- <Ge, h0> share: row n = row, columns 16c..
+            wait(F_HG, ph);
+            float kp = 0.f;
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc) {
+                const uint32_t so = swz(row, 2 * c + cc);
+                const uint4 gh = *reinterpret_cast<const uint4*>(sm + OFF_GE + so);
+                const uint4 gl = *reinterpret_cast<const uint4*>(sm + OFF_GE + TILE + so);
+                const uint4 hh = *reinterpret_cast<const uint4*>(sm + OFF_H0 + so);
+                const uint4 hl = *reinterpret_cast<const uint4*>(sm + OFF_H0 + TILE + so);
+                const uint32_t a1[4] = {gh.x, gh.y, gh.z, gh.w}, a2[4] = {gl.x, gl.y, gl.z, gl.w};
+                const uint32_t b1[4] = {hh.x, hh.y, hh.z, hh.w}, b2[4] = {hl.x, hl.y, hl.z, hl.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    kp = fmaf(bf16_lo(a1[e]) + bf16_lo(a2[e]), bf16_lo(b1[e]) + bf16_lo(b2[e]), kp);
+                    kp = fmaf(bf16_hi(a1[e]) + bf16_hi(a2[e]), bf16_hi(b1[e]) + bf16_hi(b2[e]), kp);
+                }
+            }
             // ---- C3: u, v from TMEM X (B Ge | C h0), columns 16c..
             wait(M_BC, ph);
             tc_fence_after();
             float u = 0.f, vv = 0.f;
-            uint32_t xpk[8];                                 // x of this row, columns 16c.., bf16 pairs
             {
-                uint32_t bg[16], ch[16];
+                uint32_t bg[16], chv[16];
                 tmem_ld16(tmem + lo16 + COL_X + 16 * c, bg);
-                tmem_ld16(tmem + lo16 + COL_X + 64 + 16 * c, ch);
-                const long long gofs = (((long long)d.b * p.L + (valid ? t : 0)) * p.H + d.h) * PD + 16 * c;
-                const uint4 x0 = valid ? *reinterpret_cast<const uint4*>(xg + gofs) : make_uint4(0, 0, 0, 0);
-                const uint4 x1 = valid ? *reinterpret_cast<const uint4*>(xg + gofs + 8) : make_uint4(0, 0, 0, 0);
-                xpk[0] = x0.x; xpk[1] = x0.y; xpk[2] = x0.z; xpk[3] = x0.w;
-                xpk[4] = x1.x; xpk[5] = x1.y; xpk[6] = x1.z; xpk[7] = x1.w;
+                tmem_ld16(tmem + lo16 + COL_X + 64 + 16 * c, chv);
                 tmem_wait_ld();
 #pragma unroll
-                for (int cc = 0; cc < 2; ++cc) {
-                    const uint4 yr = *reinterpret_cast<const uint4*>(sm + OFF_DY + swz(row, 2 * c + cc));
-                    const uint32_t yw[4] = {yr.x, yr.y, yr.z, yr.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int k = 8 * cc + 2 * e;
-                        u = fmaf(bf16_lo(yw[e]), __uint_as_float(ch[k]), fmaf(bf16_hi(yw[e]), __uint_as_float(ch[k + 1]), u));
-                        vv = fmaf(bf16_lo(xpk[4 * cc + e]), __uint_as_float(bg[k]),
-                                  fmaf(bf16_hi(xpk[4 * cc + e]), __uint_as_float(bg[k + 1]), vv));
-                    }
+                for (int e = 0; e < 8; ++e) {
+                    u = fmaf(bf16_lo(yr[e]), __uint_as_float(chv[2 * e]), fmaf(bf16_hi(yr[e]), __uint_as_float(chv[2 * e + 1]), u));
+                    vv = fmaf(bf16_lo(xr[e]), __uint_as_float(bg[2 * e]), fmaf(bf16_hi(xr[e]), __uint_as_float(bg[2 * e + 1]), vv));
                 }
             }
             tc_fence_before();
@@ -830,13 +830,6 @@ bwd_main_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
                 uint32_t bg[16], mt[16];
                 tmem_ld16(tmem + lo16 + COL_X + 16 * c, bg);
                 tmem_ld16(tmem + lo16 + COL_X + 64 + 16 * c, mt);
-                const long long gofs = (((long long)d.b * p.L + (valid ? t : 0)) * p.H + d.h) * PD + 16 * c;
-                uint4 y0 = make_uint4(0, 0, 0, 0), y1 = y0;
-                if (valid) {
-                    y0 = *reinterpret_cast<const uint4*>(dyg + gofs);
-                    y1 = *reinterpret_cast<const uint4*>(dyg + gofs + 8);
-                }
-                const uint32_t yw[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
                 tmem_wait_ld();
                 const float dsk = p.D ? p.D[d.h] : 0.f;
                 float o[16];
@@ -844,11 +837,12 @@ bwd_main_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
                 for (int e = 0; e < 8; ++e) {
                     const float du0 = fmaf(wt, __uint_as_float(bg[2 * e]), __uint_as_float(mt[2 * e]));
                     const float du1 = fmaf(wt, __uint_as_float(bg[2 * e + 1]), __uint_as_float(mt[2 * e + 1]));
-                    xdxu = fmaf(bf16_lo(xpk[e]), du0, fmaf(bf16_hi(xpk[e]), du1, xdxu));
-                    o[2 * e] = fmaf(dt, du0, dsk * bf16_lo(yw[e]));
-                    o[2 * e + 1] = fmaf(dt, du1, dsk * bf16_hi(yw[e]));
+                    xdxu = fmaf(bf16_lo(xr[e]), du0, fmaf(bf16_hi(xr[e]), du1, xdxu));
+                    o[2 * e] = fmaf(dt, du0, dsk * bf16_lo(yr[e]));
+                    o[2 * e + 1] = fmaf(dt, du1, dsk * bf16_hi(yr[e]));
                 }
                 if (valid) {
+                    const long long gofs = (((long long)d.b * p.L + t) * p.H + d.h) * PD + 16 * c;
                     if (p.grad_bf16) {
                         uint32_t w[8];
 #pragma unroll
@@ -863,31 +857,11 @@ bwd_main_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
                     }
                 }
             }
-            // ---- end of a segment: dB, dC partials (columns 32c..) -> slot
-            if (d.last) {
-                const long long slot = (long long)blockIdx.x * p.smax + (d.seg - seg0);
-                float* dst = p.dbc + slot * 2 * 128 * 128;
-#pragma unroll
-                for (int m = 0; m < 2; ++m) {
-                    uint32_t r[32];
-                    tmem_ld32(tmem + lo16 + (m ? COL_DC : COL_DB) + 32 * c, r);
-                    tmem_wait_ld();
-                    float4* o4 = reinterpret_cast<float4*>(dst + ((long long)m * 128 + row) * 128 + 32 * c);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        o4[e] = make_float4(__uint_as_float(r[4 * e]), __uint_as_float(r[4 * e + 1]),
-                                            __uint_as_float(r[4 * e + 2]), __uint_as_float(r[4 * e + 3]));
-                }
-                tc_fence_before();
-                mbar_arrive(bar(C_FL));
-            }
-            tc_fence_before();
-            mbar_arrive(bar(C_E));
-            // ---- the unit's token scalars into the scratch (dS^T is consumed: M_DX)
+            // ---- the unit's token scalars into the scratch (the x tile: M2 has read it)
             scr[SC_C + c * 128 + row] = csum;
-            if (lane < 16) {
-                scr[SC_R + q * 128 + 32 * c + lane] = rsum[0];
-                scr[SC_R + q * 128 + 32 * c + 16 + lane] = rsum[1];
+            if (lane < 8) {
+#pragma unroll
+                for (int ch = 0; ch < 4; ++ch) scr[SC_R + q * 128 + 32 * c + 8 * ch + lane] = rsum[ch];
             }
             scr[SC_U + c * 128 + row] = u;
             scr[SC_V + c * 128 + row] = vv;
@@ -922,8 +896,7 @@ bwd_main_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
                     if (lane >= o) { pd += a; pv += b2; }
                     if (lane + o < 32) su += cu;
                 }
-                float* wt3 = scr + SC_K;                     // reused: [4][3] warp totals
-                asm volatile("bar.sync 2, 128;" ::: "memory");   // every K share is read
+                float* wt3 = scr + SC_END;                   // [4][3] warp totals (after the scratch arrays)
                 if (lane == 31) { wt3[q * 3] = pd; wt3[q * 3 + 1] = pv; }
                 if (lane == 0) wt3[q * 3 + 2] = su;
                 asm volatile("bar.sync 2, 128;" ::: "memory");
@@ -948,13 +921,61 @@ bwd_main_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
                     sb += __shfl_xor_sync(0xffffffffu, sb, o);
                     sd += __shfl_xor_sync(0xffffffffu, sd, o);
                 }
-                asm volatile("bar.sync 2, 128;" ::: "memory");
+                asm volatile("bar.sync 2, 128;" ::: "memory");   // every warp total is read
                 if (lane == 0) { wt3[q * 3] = sa; wt3[q * 3 + 1] = sb; wt3[q * 3 + 2] = sd; }
                 asm volatile("bar.sync 2, 128;" ::: "memory");
                 if (q == 0 && lane < 3) {
                     const float tsum = wt3[lane] + wt3[3 + lane] + wt3[6 + lane] + wt3[9 + lane];
                     p.part[(((long long)d.b * p.nblk + d.j) * p.H + d.h) * 3 + lane] = tsum;
                 }
+            }
+            csync();                                         // the scratch is consumed
+            tc_fence_before();
+            mbar_arrive(bar(C_E));                           // TMEM X and the x tile are free
+            // ---- C1: (w o X), (2^R o dY) hi/lo over the consumed dS^T
+            wait(M_DS, ph);
+            {
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc) {
+                    const uint32_t so = swz(row, 2 * c + cc);
+                    uint32_t ah[4], al[4], bh[4], bl[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const uint32_t xw = xr[4 * cc + e], yw = yr[4 * cc + e];
+                        const float a0 = wv * bf16_lo(xw), a1 = wv * bf16_hi(xw);
+                        const float b0 = er * bf16_lo(yw), b1 = er * bf16_hi(yw);
+                        ah[e] = pack_bf16(a0, a1);
+                        al[e] = pack_bf16(a0 - bf16_lo(ah[e]), a1 - bf16_hi(ah[e]));
+                        bh[e] = pack_bf16(b0, b1);
+                        bl[e] = pack_bf16(b0 - bf16_lo(bh[e]), b1 - bf16_hi(bh[e]));
+                    }
+                    *reinterpret_cast<uint4*>(sm + OFF_WD + so) = make_uint4(ah[0], ah[1], ah[2], ah[3]);
+                    *reinterpret_cast<uint4*>(sm + OFF_WD + TILE + so) = make_uint4(al[0], al[1], al[2], al[3]);
+                    *reinterpret_cast<uint4*>(sm + OFF_WD + 2 * TILE + so) = make_uint4(bh[0], bh[1], bh[2], bh[3]);
+                    *reinterpret_cast<uint4*>(sm + OFF_WD + 3 * TILE + so) = make_uint4(bl[0], bl[1], bl[2], bl[3]);
+                }
+            }
+            fence_proxy_async();
+            mbar_arrive(bar(C_WE));
+            // ---- end of a segment: dB, dC partials (columns 32c..) -> slot
+            if (d.last) {
+                wait(M_WE, ph);
+                tc_fence_after();
+                const long long slot = (long long)blockIdx.x * p.smax + (d.seg - seg0);
+                float* dst = p.dbc + slot * 2 * 128 * 128;
+#pragma unroll
+                for (int m = 0; m < 2; ++m) {
+                    uint32_t r[32];
+                    tmem_ld32(tmem + lo16 + (m ? COL_DC : COL_DB) + 32 * c, r);
+                    tmem_wait_ld();
+                    float4* o4 = reinterpret_cast<float4*>(dst + ((long long)m * 128 + row) * 128 + 32 * c);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        o4[e] = make_float4(__uint_as_float(r[4 * e]), __uint_as_float(r[4 * e + 1]),
+                                            __uint_as_float(r[4 * e + 2]), __uint_as_float(r[4 * e + 3]));
+                }
+                tc_fence_before();
+                mbar_arrive(bar(C_FL));
             }
         }
     }
