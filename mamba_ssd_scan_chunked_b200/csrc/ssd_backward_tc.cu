@@ -83,8 +83,6 @@ struct Params {
     const float* A;            // [H]
     const void* init_state;    // state dtype [b*H][N][P] or NULL
     const void* dfinal;        // state dtype [b*H][N][P] or NULL
-    uint16_t* h0;              // bf16 [b*H][nblk][N][2][P]
-    uint16_t* ge;              // bf16 [b*H][nblk][N][2][P]
     void* dinit;               // state dtype [b*H][N][P] or NULL
     unsigned* dev_err;
     long long L;
@@ -94,12 +92,15 @@ struct Params {
 
 // Per block i of the walk: the compute warps form w o (x or dy) of block i into
 // W buffer i & 1 while the MMAs of block i - 1 still run, then wait for them,
-// write the state out as hi/lo and scale it by 2^(R_last) in TMEM; the MMAs of
-// block i follow.  The P-side tile is reloaded as soon as w o P of block i is
-// formed, the N-side tiles (B or C) two blocks ahead.
+// stage the state as hi/lo tiles in W buffer (i + 1) & 1 (which those MMAs have
+// just finished reading), scale it by 2^(R_last) in TMEM, and one thread per
+// head stores the two tiles with TMA; the MMAs of block i follow.  The P-side
+// tile is reloaded as soon as w o P of block i is formed, the N-side tiles (B
+// or C) two blocks ahead.
 __global__ void __launch_bounds__(st::THREADS, 1)
 bwd_states_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmDY,
                      const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmC,
+                     const __grid_constant__ CUtensorMap tmH0, const __grid_constant__ CUtensorMap tmGE,
                      const st::Params p) {
     using namespace st;
     extern __shared__ __align__(1024) uint8_t sm[];
@@ -226,7 +227,7 @@ bwd_states_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
             }
             tmem_wait_st();
         }
-        uint16_t* out = rev ? p.ge : p.h0;
+        const bool issuer = q == 0 && lane == 0;     // stores head k's tiles
         uint16_t dtr_next = fetch(0);
         for (int i = 0; i < nblk; ++i) {
             const int j = blk_of(i);
@@ -254,9 +255,12 @@ bwd_states_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
             const float wgt = rev ? ex2((float)R) : dt * ex2((float)(tot - R));
             const float scale = ex2((float)tot);
             // w o (x or dy) of token `row` into W buffer i & 1 (the MMAs of block i - 2,
-            // which read it, completed before block i - 1's state was written out)
+            // which read it, completed before block i - 1's state was written out; the
+            // TMA store of that state, staged there, has read it: waited by its issuer)
             wait(B_FULLN0 + (i & 1), (i >> 1) & 1);
             wait(B_FULLP, i & 1);
+            if (issuer) bulk_wait_read0();
+            asm volatile("bar.sync %0, %1;" ::"r"(1 + k), "r"(128) : "memory");
             {
                 const uint8_t* src = sm + OFF_P + k * TILE;
                 uint8_t* dh = sm + OFF_W + (i & 1) * 4 * TILE + 2 * k * TILE;
@@ -283,7 +287,7 @@ bwd_states_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
             if (i > 0) wait(B_MMA, (i - 1) & 1);
             tc_fence_after();
             {
-                uint16_t* o = out + ((bh * nblk + j) * NS + row) * (2 * PD);
+                uint8_t* sh = sm + OFF_W + ((i + 1) & 1) * 4 * TILE + 2 * k * TILE;   // staging: hi, lo tiles
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
                     uint32_t sv[32];
@@ -298,20 +302,29 @@ bwd_states_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
                         sv[2 * e] = __float_as_uint(a * scale);
                         sv[2 * e + 1] = __float_as_uint(bb * scale);
                     }
-                    uint4* oh = reinterpret_cast<uint4*>(o + 32 * c);
-                    uint4* ol = reinterpret_cast<uint4*>(o + PD + 32 * c);
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        oh[e] = make_uint4(hw[4 * e], hw[4 * e + 1], hw[4 * e + 2], hw[4 * e + 3]);
-                        ol[e] = make_uint4(lw[4 * e], lw[4 * e + 1], lw[4 * e + 2], lw[4 * e + 3]);
+                        const uint32_t so = swz(row, 4 * c + e);
+                        *reinterpret_cast<uint4*>(sh + so) = make_uint4(hw[4 * e], hw[4 * e + 1], hw[4 * e + 2], hw[4 * e + 3]);
+                        *reinterpret_cast<uint4*>(sh + TILE + so) = make_uint4(lw[4 * e], lw[4 * e + 1], lw[4 * e + 2], lw[4 * e + 3]);
                     }
                     tmem_st32(tmem + lo16 + 64 * k + 32 * c, sv);
                 }
                 tmem_wait_st();
+                fence_proxy_async();
+                asm volatile("bar.sync %0, %1;" ::"r"(1 + k), "r"(128) : "memory");
+                if (issuer && !*s_abort) {
+                    const int un = (int)(bh * nblk + j);
+                    const uint32_t sa = base + OFF_W + (uint32_t)((i + 1) & 1) * 4 * TILE + 2 * k * TILE;
+                    tma_store_4d(rev ? &tmGE : &tmH0, sa, 0, 0, 0, un);
+                    tma_store_4d(rev ? &tmGE : &tmH0, sa + TILE, 0, 1, 0, un);
+                    bulk_commit();
+                }
             }
             tc_fence_before();
             mbar_arrive(bar(B_WX));
         }
+        if (issuer) bulk_wait0();                   // the last tiles are written
         // the value after the whole sequence: d init_state (backward pass)
         wait(B_MMA, (nblk - 1) & 1);
         tc_fence_after();
@@ -682,6 +695,7 @@ bwd_main_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
             }
             const double R = v + off;
             const float Rhi = (float)R, Rlo = (float)(R - (double)Rhi);
+            const float totf = (float)tot;
             const float wt = ex2((float)(tot - R));        // 2^(R_last - R_s)
             const float er = ex2(Rhi + Rlo);               // 2^(R_s)
             const float wv = dt * wt;                      // w_s
@@ -787,6 +801,13 @@ bwd_main_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
             fence_proxy_async();
             tc_fence_before();
             mbar_arrive(bar(C_T));
+            // the row's shares into the scratch (the x tile: M2 has read it, x is in registers)
+            scr[SC_C + c * 128 + row] = csum;
+            if (lane < 8) {
+#pragma unroll
+                for (int ch = 0; ch < 4; ++ch) scr[SC_R + q * 128 + 32 * c + 8 * ch + lane] = rsum[ch];
+            }
+            scr[SC_XDY + c * 128 + row] = xdy;
             // ---- <Ge, h0> share: row n = row, columns 16c..
             wait(F_HG, ph);
             float kp = 0.f;
@@ -805,6 +826,7 @@ bwd_main_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
                     kp = fmaf(bf16_hi(a1[e]) + bf16_hi(a2[e]), bf16_hi(b1[e]) + bf16_hi(b2[e]), kp);
                 }
             }
+            scr[SC_K + c * 128 + row] = kp;
             // ---- C3: u, v from TMEM X (B Ge | C h0), columns 16c..
             wait(M_BC, ph);
             tc_fence_after();
@@ -820,6 +842,8 @@ bwd_main_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
                     vv = fmaf(bf16_lo(xr[e]), __uint_as_float(bg[2 * e]), fmaf(bf16_hi(xr[e]), __uint_as_float(bg[2 * e + 1]), vv));
                 }
             }
+            scr[SC_U + c * 128 + row] = u;
+            scr[SC_V + c * 128 + row] = vv;
             tc_fence_before();
             mbar_arrive(bar(C_U));
             // ---- C4: dxu, dx, x . dxu
@@ -857,17 +881,7 @@ bwd_main_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
                     }
                 }
             }
-            // ---- the unit's token scalars into the scratch (the x tile: M2 has read it)
-            scr[SC_C + c * 128 + row] = csum;
-            if (lane < 8) {
-#pragma unroll
-                for (int ch = 0; ch < 4; ++ch) scr[SC_R + q * 128 + 32 * c + 8 * ch + lane] = rsum[ch];
-            }
-            scr[SC_U + c * 128 + row] = u;
-            scr[SC_V + c * 128 + row] = vv;
-            scr[SC_XDY + c * 128 + row] = xdy;
             scr[SC_XDXU + c * 128 + row] = xdxu;
-            scr[SC_K + c * 128 + row] = kp;
             csync();
             // ---- d a, d dt_raw and the unit's parameter shares: warps c == 0, token = row
             if (c == 0) {
@@ -875,7 +889,7 @@ bwd_main_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
                 for (int e = lane; e < 512; e += 32) ksum += scr[SC_K + e];
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) ksum += __shfl_xor_sync(0xffffffffu, ksum, o);
-                const float K = ex2((float)tot) * ksum;
+                const float K = ex2(totf) * ksum;
                 float dk = 0.f, uu = 0.f, vs = 0.f, xd = 0.f, xu = 0.f;
 #pragma unroll
                 for (int w = 0; w < 4; ++w) {
@@ -1086,8 +1100,6 @@ cudaError_t launch_backward_tc(const BackwardArgs& a, cudaStream_t s) {
     sp.A = a.A;
     sp.init_state = a.init_state;
     sp.dfinal = a.dfinal;
-    sp.h0 = (uint16_t*)(a.ws + l.off_h0);
-    sp.ge = (uint16_t*)(a.ws + l.off_ge);
     sp.dinit = a.dinit;
     sp.dev_err = a.dev_err;
     sp.L = a.L;
@@ -1096,7 +1108,7 @@ cudaError_t launch_backward_tc(const BackwardArgs& a, cudaStream_t s) {
     sp.nblk = (int)nblk;
     sp.npairs = (int)(BH / 2);
     sp.state_bf16 = a.state_bf16;
-    bwd_states_tc_kernel<<<(unsigned)(2 * sp.npairs), st::THREADS, st::SMEM, s>>>(mx, mdy, mb, mc, sp);
+    bwd_states_tc_kernel<<<(unsigned)(2 * sp.npairs), st::THREADS, st::SMEM, s>>>(mx, mdy, mb, mc, mh0, mge, sp);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     // 2. block gradients
     int64_t grid = 0, smax = 0;
