@@ -661,22 +661,50 @@ bwd_main_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
         float* scr = reinterpret_cast<float*>(sm + OFF_X);
         const uint16_t* dtr = reinterpret_cast<const uint16_t*>(p.dt_raw);
         auto csync = [&]() { asm volatile("bar.sync 1, %0;" ::"r"(NCT) : "memory"); };
-        uint16_t dtr_next = 0;
-        auto fetch_dtr = [&](int i) -> uint16_t {
-            const Unit d = unit(i);
-            const long long t = (long long)d.j * SUB + row;
-            return t < p.L ? dtr[((long long)d.b * p.L + t) * p.H + d.h] : (uint16_t)0;
+        // the unit after d: (b, j, g, head in group) stepped as a counter
+        auto step = [&](Unit d) -> Unit {
+            Unit e = d;
+            int qh = d.h - d.g * hpg + 1;
+            e.first = qh == hpg;
+            if (qh == hpg) {
+                qh = 0;
+                ++e.seg;
+                if (++e.g == p.G) {
+                    e.g = 0;
+                    if (++e.j == p.nblk) { e.j = 0; ++e.b; }
+                }
+            }
+            e.h = e.g * hpg + qh;
+            e.last = qh == hpg - 1;
+            return e;
         };
-        if (nu > 0) dtr_next = fetch_dtr(0);
+        struct Pre { uint16_t dtr; float A, bias, D; };
+        auto fetch = [&](const Unit& d) -> Pre {
+            const long long t = (long long)d.j * SUB + row;
+            Pre r;
+            r.dtr = t < p.L ? dtr[((long long)d.b * p.L + t) * p.H + d.h] : (uint16_t)0;
+            r.A = p.A[d.h];
+            r.bias = p.dt_bias ? p.dt_bias[d.h] : 0.f;
+            r.D = p.D ? p.D[d.h] : 0.f;
+            return r;
+        };
+        Unit dn = unit(0);
+        Pre pn = fetch(dn);
         for (int i = 0; i < nu; ++i) {
-            const Unit d = unit(i);
+            Unit d = dn;
+            d.last = d.last || i == nu - 1;
+            d.first = d.first || i == 0;
+            const Pre pc = pn;
+            if (i + 1 < nu) {
+                dn = step(d);
+                pn = fetch(dn);
+            }
             const uint32_t ph = i & 1;
             const long long t = (long long)d.j * SUB + row;
             const bool valid = t < p.L;
-            const float Ah = p.A[d.h], bias = p.dt_bias ? p.dt_bias[d.h] : 0.f;
-            const float z = __uint_as_float((uint32_t)dtr_next << 16) + bias;
+            const float Ah = pc.A, bias = pc.bias;
+            const float z = __uint_as_float((uint32_t)pc.dtr << 16) + bias;
             const float dt = valid ? softplus_f32(z) : 0.f;
-            if (i + 1 < nu) dtr_next = fetch_dtr(i + 1);
             // ---- P1: block-local cumsum R of dt A log2(e) (double), per token
             double v = (double)(dt * Ah) * (double)LOG2E;
 #pragma unroll
@@ -721,29 +749,39 @@ bwd_main_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
             if (i > 0) wait(M_WE, ph ^ 1u);
             tc_fence_after();
             csync();                                         // the R table is complete, x is in registers
-            float csum = 0.f, rsum[4];
+            float csum = 0.f, rsum[4] = {0.f, 0.f, 0.f, 0.f};
+            float* tw = scr + warp * 256;                    // this warp's [32 rows][8] transpose buffer
+            if (c < q) {
+                // the tile lies wholly above the diagonal (l < s): zeros
+                const uint32_t zz[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+                for (int ch = 0; ch < 4; ++ch) {
+                    const int lc = 32 * c + 8 * ch, kb = lc & ~15, wo = (lc & 15) >> 1;
+                    tmem_st4(tmem + lo16 + COL_S + kb + wo, zz);
+                    tmem_st4(tmem + lo16 + COL_S + kb + 8 + wo, zz);
+                    const uint32_t so = (uint32_t)(lc >> 6) * TILE + swz(row, (lc & 63) >> 3);
+                    *reinterpret_cast<uint4*>(sm + OFF_WD + so) = make_uint4(0, 0, 0, 0);
+                    *reinterpret_cast<uint4*>(sm + OFF_WD + 2 * TILE + so) = make_uint4(0, 0, 0, 0);
+                }
+            } else {
 #pragma unroll
             for (int ks2 = 0; ks2 < 2; ++ks2) {
                 // one 16-column K step: its S^T is read whole before Mt overwrites it in place
                 const int kb = 32 * c + 16 * ks2;
                 uint32_t sv[16];
-                if (c >= q) {
-                    tmem_ld16(tmem + lo16 + COL_S + kb, sv);
-                    tmem_wait_ld();
-                }
+                tmem_ld16(tmem + lo16 + COL_S + kb, sv);
+                tmem_wait_ld();
 #pragma unroll
                 for (int h8 = 0; h8 < 2; ++h8) {
                     // 8 columns lc .. lc + 7
                     const int ch = 2 * ks2 + h8, lc = kb + 8 * h8;
                     uint32_t xv[8];
-                    float wcol[8];
-                    if (c >= q) {
-                        asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-                                     : "=r"(xv[0]), "=r"(xv[1]), "=r"(xv[2]), "=r"(xv[3]), "=r"(xv[4]), "=r"(xv[5]),
-                                       "=r"(xv[6]), "=r"(xv[7]) : "r"(tmem + lo16 + COL_X + lc));
-                        tmem_wait_ld();
-                    }
+                    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                                 : "=r"(xv[0]), "=r"(xv[1]), "=r"(xv[2]), "=r"(xv[3]), "=r"(xv[4]), "=r"(xv[5]),
+                                   "=r"(xv[6]), "=r"(xv[7]) : "r"(tmem + lo16 + COL_X + lc));
+                    tmem_wait_ld();
                     uint32_t mh[4], ml[4], dh[4], dl[4];
+                    float wcol[8];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         float m2[2], g2[2];
@@ -752,7 +790,7 @@ bwd_main_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
                             const int kc = 2 * e + z2;
                             const int l = lc + kc;
                             float m = 0.f, gd = 0.f, wcl = 0.f;
-                            if (c >= q && l >= row) {
+                            if (l >= row) {
                                 const float2 rl = s_rt[l];
                                 const float f = ex2((rl.x - Rhi) + (rl.y - Rlo));
                                 const float sval = __uint_as_float(sv[8 * h8 + kc]);
@@ -779,29 +817,28 @@ bwd_main_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
                     const uint32_t so = (uint32_t)(lc >> 6) * TILE + swz(row, (lc & 63) >> 3);
                     *reinterpret_cast<uint4*>(sm + OFF_WD + so) = make_uint4(dh[0], dh[1], dh[2], dh[3]);
                     *reinterpret_cast<uint4*>(sm + OFF_WD + 2 * TILE + so) = make_uint4(dl[0], dl[1], dl[2], dl[3]);
-                    // row sums over this warp's 32 rows of the 8 columns: lane i ends with column lc + (i & 7)
+                    // column sums of the 8 columns over this warp's 32 rows, through the
+                    // transpose buffer: lane i sums column i & 7 over rows 8 (i >> 3) ..
+                    *reinterpret_cast<float4*>(tw + lane * 8) = make_float4(wcol[0], wcol[1], wcol[2], wcol[3]);
+                    *reinterpret_cast<float4*>(tw + lane * 8 + 4) = make_float4(wcol[4], wcol[5], wcol[6], wcol[7]);
+                    __syncwarp();
+                    float cs = 0.f;
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) wcol[e] += __shfl_xor_sync(0xffffffffu, wcol[e], 16);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) wcol[e] += __shfl_xor_sync(0xffffffffu, wcol[e], 8);
-#pragma unroll
-                    for (int w = 4; w >= 1; w >>= 1) {
-#pragma unroll
-                        for (int e = 0; e < w; ++e) {
-                            const bool up = (lane & w) != 0;
-                            const float send = up ? wcol[e] : wcol[e + w];
-                            const float keep = up ? wcol[e + w] : wcol[e];
-                            wcol[e] = keep + __shfl_xor_sync(0xffffffffu, send, w);
-                        }
-                    }
-                    rsum[ch] = wcol[0];
+                    for (int r = 0; r < 8; ++r) cs += tw[(8 * (lane >> 3) + r) * 8 + (lane & 7)];
+                    cs += __shfl_xor_sync(0xffffffffu, cs, 8);
+                    cs += __shfl_xor_sync(0xffffffffu, cs, 16);
+                    rsum[ch] = cs;                           // lanes i and i ^ 8, i ^ 16, i ^ 24: column lc + (i & 7)
+                    __syncwarp();
                 }
+            }
             }
             tmem_wait_st();
             fence_proxy_async();
             tc_fence_before();
             mbar_arrive(bar(C_T));
-            // the row's shares into the scratch (the x tile: M2 has read it, x is in registers)
+            // the row's shares into the scratch (the x tile: M2 has read it, x is in registers,
+            // and every warp is done with its transform buffer)
+            csync();
             scr[SC_C + c * 128 + row] = csum;
             if (lane < 8) {
 #pragma unroll
@@ -855,7 +892,7 @@ bwd_main_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
                 tmem_ld16(tmem + lo16 + COL_X + 16 * c, bg);
                 tmem_ld16(tmem + lo16 + COL_X + 64 + 16 * c, mt);
                 tmem_wait_ld();
-                const float dsk = p.D ? p.D[d.h] : 0.f;
+                const float dsk = pc.D;
                 float o[16];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
