@@ -122,9 +122,25 @@ def backward_bytes(b, L, H, P, N, G, io_bytes, grad_bytes, state_bytes):
 
 
 def backward_flops(b, L, H, P, N, G, Q):
-    """The backward's three chunked scans: the state adjoint (the forward's
-    shape) and two transposed scans (headdim N, dstate P, one group per head)."""
+    """Algorithmic flops of the backward, counted as the three chunked scans it
+    amounts to: the state adjoint (the forward's shape) and two transposed scans
+    (headdim N, dstate P, one group per head)."""
     return prefill_flops(b, L, H, P, N, G, Q) + 2 * prefill_flops(b, L, H, N, P, H, Q)
+
+
+def backward_executed_flops(b, L, H, P, N, G):
+    """Tensor flops the block-form backward on tensor cores executes (128-token
+    blocks, hi/lo pairs): per (b, h, block) the block kernel's S^T, X dY^T (N =
+    128), B Ge and C h0 (hi + lo, N = 64), Mt dY (hi + lo), dS^T C and dS B (hi +
+    lo), the weighted-operand products (three per accumulator); per (b, h, block)
+    and direction one rank-128 state update (hi + lo)."""
+    sub = 128
+    nblk = -(-L // sub)
+    mm = lambda n, k: 2 * sub * n * k
+    per_unit = (mm(sub, N) + mm(sub, P) + 2 * 2 * mm(P, N) + 2 * mm(P, sub) + 2 * 2 * mm(N, sub)
+                + 3 * 2 * mm(N, P))
+    per_state = 2 * mm(P, sub) * (N // sub)
+    return b * H * nblk * (per_unit + 2 * per_state)
 
 
 def decode_bytes(b, H, P, N, G, io_bytes, y_bytes, state_bytes):
@@ -729,10 +745,14 @@ def main():
     bbytes = backward_bytes(c1.batch, c1.seqlen, c1.nheads, c1.headdim, c1.dstate, c1.ngroups, 2, 4, 4)
     bflops = backward_flops(c1.batch, c1.seqlen, c1.nheads, c1.headdim, c1.dstate, c1.ngroups, c1.chunk)
     broof = roofline_of(bbytes, bflops, bms * 1e-3, peaks, peak_kind)
-    broof["kernel"] = "ssd_chunk_scan_bwd (three chunked scans + copies + finishing)"
+    broof["kernel"] = ("ssd_chunk_scan_bwd (block form on tensor cores: state passes, block gradients, "
+                       "dB/dC partial sums, parameter sums)")
+    bexec = backward_executed_flops(c1.batch, c1.seqlen, c1.nheads, c1.headdim, c1.dstate, c1.ngroups)
     backward_line = {"tokens_per_s": t1 * world / (bms * 1e-3), "ms_per_step": bms, "steps": bsteps,
                      "launches_per_step": launches_per_bwd, "gradients": "fp32", "dfinal_state": "given",
-                     "gbs": bbytes / (bms * 1e-3) / 1e9, "tflops": bflops / (bms * 1e-3) / 1e12, "roofline": broof}
+                     "gbs": bbytes / (bms * 1e-3) / 1e9, "tflops": bflops / (bms * 1e-3) / 1e12,
+                     "executed_tflops": bexec / (bms * 1e-3) / 1e12, "executed_flops_per_call": bexec,
+                     "roofline": broof}
     del dyb, dfin, bws, gx, gdt, gB, gC, gpar
 
     # ---- Mamba-3 prefill (trapezoidal input + rotational state) of the same layer

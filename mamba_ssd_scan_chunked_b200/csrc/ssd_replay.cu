@@ -38,6 +38,7 @@ constexpr int RP_VEC = 4;
 constexpr int RP_U = 8;
 constexpr int RP_MINB = 8;
 constexpr int RP_MINB_FOLD = 4;             // the fold: 4 resident CTAs (measured 1..4)
+constexpr int RP_GS = 16;                   // floats per row of the fold's coefficient table
 
 // 4 consecutive elements of T, converted to and from fp32 (16 B fp32, 8 B bf16)
 template <typename T> struct Vec4;
@@ -119,8 +120,8 @@ replay_dots_kernel(const IoT* __restrict__ Bb, const IoT* __restrict__ Bm, const
     }
 }
 
-// Packed fp32 pairs (low half = first element) and the sm_100 paired FMA:
-// one instruction updates two columns of a state row.
+// Packed fp32 pairs (low half = first element) and the sm_100 paired FMA: one
+// instruction adds two consecutive buffered tokens' terms to a state element.
 __device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
     return (uint64_t)__float_as_uint(lo) | ((uint64_t)__float_as_uint(hi) << 32);
 }
@@ -129,11 +130,6 @@ __device__ __forceinline__ float f2hi(uint64_t v) { return __uint_as_float((uint
 __device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
     uint64_t d;
     asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-    return d;
-}
-__device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
-    uint64_t d;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
     return d;
 }
 
@@ -152,10 +148,10 @@ replay_step_kernel(StateT* __restrict__ ckpt, IoT* __restrict__ xb, IoT* __restr
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int bh = blockIdx.x * RP_WARPS + warp;
     if (bh >= BH) return;                      // whole warps; no block barrier follows
-    // per warp: C_t [N], then (flush) g[n][s] = beta_s B_s[n] for s < K, rows of
-    // 17 floats: an odd stride, so that 32 lanes writing consecutive n hit 32
-    // banks and the two rows a warp reads at once are in different banks
-    float* cs = rp_smem + (size_t)warp * (N + (FLUSH ? 17 * N : 0));
+    // per warp: C_t [N], then (flush) g[n][s] = beta_s B_s[n] for the 16 slots,
+    // rows of RP_GS floats (16-byte aligned rows, read as 4 float4; the two rows
+    // a warp reads at once fall in different banks)
+    float* cs = rp_smem + (size_t)warp * (N + (FLUSH ? RP_GS * N : 0));
     float* gs = cs + N;
     const int b = bh / H, h = bh % H, hpg = H / G, g = h / hpg;
     const size_t bg = (size_t)b * G + g;
@@ -208,7 +204,7 @@ replay_step_kernel(StateT* __restrict__ ckpt, IoT* __restrict__ xb, IoT* __restr
                     float f[VE];
                     if (s < K) BV::unpack(raw[i], f);
 #pragma unroll
-                    for (int e = 0; e < VE; ++e) gs[(c * VE + e) * 17 + s] = s < K ? bt * f[e] : 0.f;
+                    for (int e = 0; e < VE; ++e) gs[(c * VE + e) * RP_GS + s] = s < K ? bt * f[e] : 0.f;
                 }
             }
         }
@@ -238,21 +234,28 @@ replay_step_kernel(StateT* __restrict__ ckpt, IoT* __restrict__ xb, IoT* __restr
             }
         }
     } else {
-        // x_s of the K buffered tokens for this lane's columns (s == fill: x_t)
-        uint64_t xs[16][2];                    // x_s[cols] as fp32 pairs
+        // x of the 16 slots for this lane's 4 columns (slot fill: x_t; past it: zero), as
+        // pairs of consecutive slots per column: the paired FMA below adds slots 2k and
+        // 2k + 1 of one column at once, against the coefficient pair (g_2k, g_2k+1)
+        uint64_t xs2[8][RP_VEC];
 #pragma unroll
-        for (int s = 0; s < 16; ++s) {
-            float xv[RP_VEC];
-            if (s < fill) load4(xb + ((size_t)bh * K + s) * P + p0, xv);
-            else {                             // s == fill: this step's token; past K: zero
+        for (int k2 = 0; k2 < 8; ++k2) {
+            float xa[RP_VEC], xb2[RP_VEC];
 #pragma unroll
-                for (int j = 0; j < RP_VEC; ++j) xv[j] = s == fill ? xt[j] : 0.f;
+            for (int z = 0; z < 2; ++z) {
+                const int s = 2 * k2 + z;
+                float* xv = z ? xb2 : xa;
+                if (s < fill) load4(xb + ((size_t)bh * K + s) * P + p0, xv);
+                else {
+#pragma unroll
+                    for (int j = 0; j < RP_VEC; ++j) xv[j] = s == fill ? xt[j] : 0.f;
+                }
             }
-            xs[s][0] = f2pack(xv[0], xv[1]);
-            xs[s][1] = f2pack(xv[2], xv[3]);
+#pragma unroll
+            for (int j = 0; j < RP_VEC; ++j) xs2[k2][j] = f2pack(xa[j], xb2[j]);
         }
-        const uint64_t al2 = f2pack(alpha, alpha);
-        // h <- alpha h + sum_s g[n][s] x_s[cols]; acc = sum_n C[n] h_new[n][cols]
+        // h <- alpha h + sum_s g[n][s] x_s[cols] (even and odd slots summed apart, then
+        // added); acc = sum_n C[n] h_new[n][cols]
         for (int r0 = r_off; r0 < N; r0 += U * rstep) {
             float hv[U][RP_VEC];
 #pragma unroll
@@ -264,18 +267,22 @@ replay_step_kernel(StateT* __restrict__ ckpt, IoT* __restrict__ xb, IoT* __restr
             for (int u = 0; u < U; ++u) {
                 const int r = r0 + u * rstep;
                 if (r < N) {
-                    uint64_t v2[2] = {fmul2(al2, f2pack(hv[u][0], hv[u][1])), fmul2(al2, f2pack(hv[u][2], hv[u][3]))};
-                    const float* gr = gs + r * 17;
+                    const float4* g4 = reinterpret_cast<const float4*>(gs + r * RP_GS);
+                    uint64_t gp[8];
 #pragma unroll
-                    for (int t = 0; t < 16; ++t) {
-                        if (t < K) {
-                            const float gv = gr[t];
-                            const uint64_t g2 = f2pack(gv, gv);
-                            v2[0] = ffma2(g2, xs[t][0], v2[0]);
-                            v2[1] = ffma2(g2, xs[t][1], v2[1]);
-                        }
+                    for (int k4 = 0; k4 < 4; ++k4) {
+                        const float4 q4 = g4[k4];
+                        gp[2 * k4] = f2pack(q4.x, q4.y);
+                        gp[2 * k4 + 1] = f2pack(q4.z, q4.w);
                     }
-                    const float v[RP_VEC] = {f2lo(v2[0]), f2hi(v2[0]), f2lo(v2[1]), f2hi(v2[1])};
+                    float v[RP_VEC];
+#pragma unroll
+                    for (int j = 0; j < RP_VEC; ++j) {
+                        uint64_t a2 = f2pack(alpha * hv[u][j], 0.f);
+#pragma unroll
+                        for (int k2 = 0; k2 < 8; ++k2) a2 = ffma2(gp[k2], xs2[k2][j], a2);
+                        v[j] = f2lo(a2) + f2hi(a2);
+                    }
                     Vec4<StateT>::store(base + (size_t)r * P, v);   // bf16: rounded to nearest even
                     const float c = cs[r];
 #pragma unroll
@@ -339,7 +346,7 @@ static cudaError_t launch_rp(const ReplayArgs& a, cudaStream_t s) {
     const long long bh = a.batch * a.H;
     const unsigned grid = (unsigned)((bh + RP_WARPS - 1) / RP_WARPS);
     const bool flush = a.fill == a.K - 1;
-    const size_t smem = sizeof(float) * RP_WARPS * (size_t)a.N * (flush ? 18 : 1);
+    const size_t smem = sizeof(float) * RP_WARPS * (size_t)a.N * (flush ? 1 + RP_GS : 1);
     if (flush) {
         auto k = replay_step_kernel<StateT, IoT, YT, true>;
         if (smem > 48 * 1024) {

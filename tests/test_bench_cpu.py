@@ -57,6 +57,19 @@ def test_executed_flops_block_by_block():
     assert bench.executed_flops(b, L, H, P, N, G, 0) == b * nblk * (H * s + H * per_head)
 
 
+def test_backward_executed_flops_by_instruction():
+    # per (b, h, 128-token block): M = 128 MMAs with K = 16 steps, 2*M*N*K flops each;
+    # S^T (N 128, 8 steps), X dY^T (N 128, 4), B Ge and C h0 (N 64, 8, hi + lo each),
+    # Mt dY (N 64, 8, hi + lo), dS^T C and dS B (N 128, 8, hi + lo each), the weighted
+    # products (N 128, 4 steps, three per accumulator, two accumulators); per
+    # direction one state update (N 64, 8 steps, hi + lo)
+    nblk = L // 128
+    f = lambda n, steps: steps * 2 * 128 * n * 16
+    unit = f(128, 8) + f(128, 4) + 2 * 2 * f(64, 8) + 2 * f(64, 8) + 2 * 2 * f(128, 8) + 3 * 2 * f(128, 4)
+    state = 2 * f(64, 8)
+    assert bench.backward_executed_flops(b, L, H, P, N, G) == b * H * nblk * (unit + 2 * state)
+
+
 def test_handoff_prefill_bytes():
     bb, LL, HH, GG = 512, 1024, 128, 8
     t = bb * LL
