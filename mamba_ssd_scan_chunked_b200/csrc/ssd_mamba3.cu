@@ -240,35 +240,66 @@ m3_decay_kernel(const IoT* __restrict__ dt_raw, const float* __restrict__ dt_bia
 }
 
 // y_t = sum of the scans' outputs - c_t (C_t . B_t) x_t (corr NULL: no
-// correction; y2, y3 NULL: one scan); one block per token row, a warp per head.
-// y1 and y may be the same fp32 array (corrected in place).
+// correction; y2, y3 NULL: one scan); one block per token row.  C_t . B_t is
+// formed once per group (a warp per group, into shared memory), then the row's
+// H * P outputs go 4 at a time (16-byte loads of y1, y2, y3), every thread of
+// the block on consecutive vectors.  y1 and y may be the same fp32 array
+// (corrected in place: each vector is read before it is written, by one thread).
 template <typename IoT, typename YT>
 __global__ void __launch_bounds__(256)
 m3_combine_kernel(const float* y1, const float* __restrict__ y2, const float* __restrict__ y3,
                   const IoT* __restrict__ x, const IoT* __restrict__ B, const IoT* __restrict__ C,
                   const float* __restrict__ corr, YT* y, int64_t batch, int64_t L, int64_t Lpad, int H, int P, int N,
                   int G) {
+    __shared__ float s_cb[256];                // C_t . B_t per group (G <= 256; else formed per vector)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
     const int hpg = H / G;
+    const int vpr = H * P / 4;                 // 4-vectors of a token row (P is a multiple of 8)
     for (int64_t r = blockIdx.x; r < batch * L; r += gridDim.x) {
         const int64_t b = r / L, t = r - b * L;
-        for (int h = warp; h < H; h += nwarps) {
-            float f = 0.f;
-            if (corr) {
-                const int64_t grow = (r * G + h / hpg) * N;
+        const bool sh = corr && G <= 256;
+        if (sh) {
+            for (int g = warp; g < G; g += nwarps) {
+                const int64_t grow = (r * G + g) * N;
                 float cb = 0.f;
                 for (int n = lane; n < N; n += 32) cb += to_f32(C[grow + n]) * to_f32(B[grow + n]);
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) cb += __shfl_xor_sync(0xffffffffu, cb, o);
+                if (lane == 0) s_cb[g] = cb;
+            }
+            __syncthreads();
+        }
+        const int64_t row = r * H * P;
+        for (int i = threadIdx.x; i < vpr; i += blockDim.x) {
+            const int h = (4 * i) / P;
+            float4 v = reinterpret_cast<const float4*>(y1 + row)[i];
+            if (y2) {
+                const float4 v2 = reinterpret_cast<const float4*>(y2 + row)[i];
+                const float4 v3 = reinterpret_cast<const float4*>(y3 + row)[i];
+                v.x += v2.x + v3.x; v.y += v2.y + v3.y; v.z += v2.z + v3.z; v.w += v2.w + v3.w;
+            }
+            float f = 0.f;
+            if (corr) {
+                float cb;
+                if (sh) {
+                    cb = s_cb[h / hpg];
+                } else {                       // more groups than the table holds: per vector
+                    const int64_t grow = (r * G + h / hpg) * N;
+                    cb = 0.f;
+                    for (int n = 0; n < N; ++n) cb += to_f32(C[grow + n]) * to_f32(B[grow + n]);
+                }
                 f = corr[(b * H + h) * Lpad + t] * cb;
             }
-            const int64_t row = (r * H + h) * P;
-            for (int p = lane; p < P; p += 32) {
-                float v = y1[row + p];
-                if (y2) v += y2[row + p] + y3[row + p];
-                y[row + p] = from_f32<YT>(v - f * to_f32(x[row + p]));
-            }
+            float xv[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) xv[e] = to_f32(x[row + 4 * i + e]);
+            YT* o = y + row + 4 * i;
+            o[0] = from_f32<YT>(v.x - f * xv[0]);
+            o[1] = from_f32<YT>(v.y - f * xv[1]);
+            o[2] = from_f32<YT>(v.z - f * xv[2]);
+            o[3] = from_f32<YT>(v.w - f * xv[3]);
         }
+        if (sh) __syncthreads();               // s_cb is rewritten for the next row
     }
 }
 
