@@ -344,6 +344,8 @@ def main():
                     help="override the headline workload's batch (a smaller case of the same shape, for profiling)")
     ap.add_argument("--only-headline", action="store_true",
                     help="time the headline prefill alone (for profiling one workload)")
+    ap.add_argument("--layer-only", action="store_true",
+                    help="time the 1.3B-shaped layer's legs alone: prefill, backward, Mamba-3 prefill (for profiling)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     rank = int(os.environ.get("RANK", "0"))
@@ -368,10 +370,134 @@ def main():
     uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
     bf16 = torch.bfloat16
 
+    def to_dev(a):
+        if a.dtype == np.uint16:
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
     def check(what):
         st_err, detail = ssd.ssd_get_device_error(stream.cuda_stream)
         if st_err:
             raise RuntimeError(f"device error word {detail:#x} after {what}")
+
+    def prefill_call(d, yb, fb, wsb, desc_, strm=None):
+        st = ssd.ssd_chunk_scan_fwd(desc_, d["x"].data_ptr(), d["dt_raw"].data_ptr(), d["dt_bias"].data_ptr(),
+                                    d["A"].data_ptr(), d["B"].data_ptr(), d["C"].data_ptr(), d["D"].data_ptr(), 0,
+                                    yb.data_ptr(), fb.data_ptr(), wsb.data_ptr(), wsb.numel(),
+                                    (strm or stream).cuda_stream)
+        if st:
+            raise ssd.SsdError(st, "ssd_chunk_scan_fwd")
+
+
+    # ================= the Mamba-2 1.3B-shaped layer: prefill, backward, Mamba-3 prefill
+    def layer_legs():
+        c1 = I.MAMBA2_1P3B
+        my_batches = dist.shard(c1.batch * world, rank, world)
+        NSETS = 3       # rotating input sets (x 67 MB each) so no step finds its inputs in L2
+        sets = []
+        for k in range(NSETS):
+            batches = [bb + k * c1.batch * world for bb in my_batches]
+            sets.append({kk: to_dev(v) for kk, v in c1.inputs(batches=batches).items()})
+        y1 = torch.empty((c1.batch, c1.seqlen, c1.nheads, c1.headdim), dtype=torch.float32, device=dev)
+        f1 = torch.empty((c1.batch, c1.nheads, c1.dstate, c1.headdim), dtype=torch.float32, device=dev)
+        desc1 = ssd.prefill_desc(sets[0]["x"], sets[0]["B"], c1.chunk, torch.float32, torch.float32)
+        path1 = ssd.ssd_chunk_scan_path(desc1)
+        ws1 = torch.empty(ssd.ssd_chunk_scan_workspace_size(desc1), dtype=torch.uint8, device=dev)
+        c1_steps = max(args.steps, 2000)              # about 0.2 s of calls
+        c1clk = ClockSampler(uuid)
+        ms1 = timed(torch, stream, lambda k: prefill_call(sets[k % NSETS], y1, f1, ws1, desc1), c1_steps,
+                    args.warmup, pg, dist, c1clk)
+        check("the 1.3B-layer prefill")
+        t1 = c1.batch * c1.seqlen
+        fl1 = prefill_flops(c1.batch, c1.seqlen, c1.nheads, c1.headdim, c1.dstate, c1.ngroups, c1.chunk)
+        xf1 = executed_flops(c1.batch, c1.seqlen, c1.nheads, c1.headdim, c1.dstate, c1.ngroups, path1)
+        nb1 = prefill_bytes(c1.batch, c1.seqlen, c1.nheads, c1.headdim, c1.dstate, c1.ngroups, 2, 4, 4)
+        r1 = roofline_of(nb1, fl1, ms1 * 1e-3, peaks, peak_kind)
+        r1.update({"traffic": ncu_traffic("ssd_prefill_pair.cu", "mamba2_1p3b"),
+                   "kernel": "ssd_chunk_scan_fwd (decay cumsum + tcgen05 head-pair chunk kernel)"})
+        c1_line = {"workload": c1.name, "steps": c1_steps, "tokens_per_s": t1 * world / (ms1 * 1e-3), "ms_per_step": ms1,
+                   "tflops": fl1 / (ms1 * 1e-3) / 1e12, "executed_tflops": xf1 / (ms1 * 1e-3) / 1e12,
+                   "executed_flops_per_call": xf1, "gbs": nb1 / (ms1 * 1e-3) / 1e9, "kernel_path": PATH_NAMES[path1],
+                   "y": "fp32", "final_state": "fp32", "l2": "3 rotating input sets (x 67 MB each)",
+                   "roofline": r1, "clocks": c1clk.summary()}
+
+        # ---- backward pass of the same layer
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(1000 + rank)
+        dyb = torch.randn((c1.batch, c1.seqlen, c1.nheads, c1.headdim), generator=gen, device=dev).to(bf16)
+        dfin = 0.1 * torch.randn((c1.batch, c1.nheads, c1.dstate, c1.headdim), generator=gen, device=dev)
+        bws = torch.empty(ssd.ssd_chunk_scan_bwd_workspace_size(desc1), dtype=torch.uint8, device=dev)
+        gx = torch.empty((c1.batch, c1.seqlen, c1.nheads, c1.headdim), dtype=torch.float32, device=dev)
+        gdt = torch.empty((c1.batch, c1.seqlen, c1.nheads), dtype=torch.float32, device=dev)
+        gB = torch.empty((c1.batch, c1.seqlen, c1.ngroups, c1.dstate), dtype=torch.float32, device=dev)
+        gC = torch.empty_like(gB)
+        gpar = torch.empty((3, c1.nheads), dtype=torch.float32, device=dev)
+        launches_per_bwd = ssd.ssd_chunk_scan_bwd_launches(desc1, True)
+
+        def backward(k):
+            d = sets[k % NSETS]
+            st = ssd.ssd_chunk_scan_bwd(desc1, d["x"].data_ptr(), d["dt_raw"].data_ptr(), d["dt_bias"].data_ptr(),
+                                        d["A"].data_ptr(), d["B"].data_ptr(), d["C"].data_ptr(), d["D"].data_ptr(), 0,
+                                        dyb.data_ptr(), dfin.data_ptr(), gx.data_ptr(), gdt.data_ptr(),
+                                        gpar[0].data_ptr(), gpar[1].data_ptr(), gB.data_ptr(), gC.data_ptr(),
+                                        gpar[2].data_ptr(), 0, bws.data_ptr(), bws.numel(), stream.cuda_stream)
+            if st:
+                raise ssd.SsdError(st, "ssd_chunk_scan_bwd")
+
+        bsteps = max(10, min(args.steps, 50))
+        bms = timed(torch, stream, backward, bsteps, args.warmup, pg, dist)
+        check("the timed backward")
+        bbytes = backward_bytes(c1.batch, c1.seqlen, c1.nheads, c1.headdim, c1.dstate, c1.ngroups, 2, 4, 4)
+        bflops = backward_flops(c1.batch, c1.seqlen, c1.nheads, c1.headdim, c1.dstate, c1.ngroups, c1.chunk)
+        broof = roofline_of(bbytes, bflops, bms * 1e-3, peaks, peak_kind)
+        broof["kernel"] = ("ssd_chunk_scan_bwd (block form on tensor cores: state passes, block gradients, "
+                           "dB/dC partial sums, parameter sums)")
+        bexec = backward_executed_flops(c1.batch, c1.seqlen, c1.nheads, c1.headdim, c1.dstate, c1.ngroups)
+        backward_line = {"tokens_per_s": t1 * world / (bms * 1e-3), "ms_per_step": bms, "steps": bsteps,
+                         "launches_per_step": launches_per_bwd, "gradients": "fp32", "dfinal_state": "given",
+                         "gbs": bbytes / (bms * 1e-3) / 1e9, "tflops": bflops / (bms * 1e-3) / 1e12,
+                         "executed_tflops": bexec / (bms * 1e-3) / 1e12, "executed_flops_per_call": bexec,
+                         "roofline": broof}
+        del dyb, dfin, bws, gx, gdt, gB, gC, gpar
+
+        # ---- Mamba-3 prefill (trapezoidal input + rotational state) of the same layer
+        ex = I.draw_mamba3_extras(c1.batch, c1.seqlen, c1.nheads, c1.ngroups, c1.dstate, c1.seed + rank)
+        m3_lam, m3_theta = to_dev(ex["lam"]), to_dev(ex["theta"])
+        m3ws = torch.empty(ssd.ssd_chunk_scan_mamba3_workspace_size(desc1), dtype=torch.uint8, device=dev)
+        launches_per_m3 = ssd.ssd_chunk_scan_mamba3_launches(desc1, True, True, True)
+
+        def mamba3(k):
+            d = sets[k % NSETS]
+            st = ssd.ssd_chunk_scan_fwd_mamba3(desc1, d["x"].data_ptr(), d["dt_raw"].data_ptr(), d["dt_bias"].data_ptr(),
+                                               d["A"].data_ptr(), d["B"].data_ptr(), d["C"].data_ptr(),
+                                               d["D"].data_ptr(), m3_lam.data_ptr(), m3_theta.data_ptr(), 0,
+                                               y1.data_ptr(), f1.data_ptr(), m3ws.data_ptr(), m3ws.numel(),
+                                               stream.cuda_stream)
+            if st:
+                raise ssd.SsdError(st, "ssd_chunk_scan_fwd_mamba3")
+
+        m3steps = max(10, min(args.steps, 50))
+        m3ms = timed(torch, stream, mamba3, m3steps, args.warmup, pg, dist)
+        check("the timed Mamba-3 prefill")
+        mamba3_line = {"tokens_per_s": t1 * world / (m3ms * 1e-3), "ms_per_step": m3ms, "steps": m3steps,
+                       "launches_per_step": launches_per_m3, "vs_mamba2_prefill_time": m3ms / ms1,
+                       "inputs": "lam ~ U[0,1] per (token, head), theta ~ U[-0.5,0.5] rad per (token, group, pair)",
+                       "path": "B, C turned by the cumulative angle in bf16 hi/lo pairs, three tensor-core scans"}
+        c1_line["backward"] = backward_line
+        c1_line["mamba3"] = mamba3_line
+        del sets, y1, f1, ws1, m3ws
+        torch.cuda.empty_cache()
+        return c1_line
+
+    if args.layer_only:
+        # profiling: the 1.3B-shaped layer's legs alone (a few GB on the device)
+        c1_line = layer_legs()
+        if rank == 0:
+            print(json.dumps({"metric": METRIC, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                              "data": "synthetic", "legs": "1.3B-shaped layer only", "mamba2_1p3b": c1_line}),
+                  flush=True)
+        dist.finish(pg)
+        return
 
     # ================= headline: batch-512 prefill (each rank its own 512 sequences)
     s = I.HANDOFF_PREFILL if args.workload == "handoff_prefill" else I.MAMBA2_1P3B
@@ -387,14 +513,6 @@ def main():
     desc = ssd.prefill_desc(inp["x"], inp["B"], Q, torch.float32, sdt)
     path = ssd.ssd_chunk_scan_path(desc)
     ws = torch.empty(ssd.ssd_chunk_scan_workspace_size(desc), dtype=torch.uint8, device=dev)
-
-    def prefill_call(d, yb, fb, wsb, desc_, strm=None):
-        st = ssd.ssd_chunk_scan_fwd(desc_, d["x"].data_ptr(), d["dt_raw"].data_ptr(), d["dt_bias"].data_ptr(),
-                                    d["A"].data_ptr(), d["B"].data_ptr(), d["C"].data_ptr(), d["D"].data_ptr(), 0,
-                                    yb.data_ptr(), fb.data_ptr(), wsb.data_ptr(), wsb.numel(),
-                                    (strm or stream).cuda_stream)
-        if st:
-            raise ssd.SsdError(st, "ssd_chunk_scan_fwd")
 
     clk = ClockSampler(uuid)
     ms = timed(torch, stream, lambda k: prefill_call(inp, y, fs, ws, desc), args.steps, args.warmup, pg, dist, clk)
@@ -553,10 +671,6 @@ def main():
     state = torch.from_numpy(np.stack([I.draw_decode_state(bb, dcfg.nheads, dcfg.headdim, dcfg.dstate, dcfg.seed,
                                                            dcfg.state_dtype) for bb in dec_batches])).to(dev)
 
-    def to_dev(a):
-        if a.dtype == np.uint16:
-            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
-        return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
 
     prm = {k: to_dev(v) for k, v in I.draw_head_params(dcfg.nheads, dcfg.seed).items()}
     nsteps_in = 8
@@ -685,103 +799,7 @@ def main():
     del state, dsteps, yd, rbuf, mx_, mB, mC, my_
     torch.cuda.empty_cache()
 
-    # ================= the Mamba-2 1.3B-shaped layer: prefill, backward, Mamba-3 prefill
-    c1 = I.MAMBA2_1P3B
-    my_batches = dist.shard(c1.batch * world, rank, world)
-    NSETS = 3       # rotating input sets (x 67 MB each) so no step finds its inputs in L2
-    sets = []
-    for k in range(NSETS):
-        batches = [bb + k * c1.batch * world for bb in my_batches]
-        sets.append({kk: to_dev(v) for kk, v in c1.inputs(batches=batches).items()})
-    y1 = torch.empty((c1.batch, c1.seqlen, c1.nheads, c1.headdim), dtype=torch.float32, device=dev)
-    f1 = torch.empty((c1.batch, c1.nheads, c1.dstate, c1.headdim), dtype=torch.float32, device=dev)
-    desc1 = ssd.prefill_desc(sets[0]["x"], sets[0]["B"], c1.chunk, torch.float32, torch.float32)
-    path1 = ssd.ssd_chunk_scan_path(desc1)
-    ws1 = torch.empty(ssd.ssd_chunk_scan_workspace_size(desc1), dtype=torch.uint8, device=dev)
-    c1_steps = max(args.steps, 2000)              # about 0.2 s of calls
-    c1clk = ClockSampler(uuid)
-    ms1 = timed(torch, stream, lambda k: prefill_call(sets[k % NSETS], y1, f1, ws1, desc1), c1_steps,
-                args.warmup, pg, dist, c1clk)
-    check("the 1.3B-layer prefill")
-    t1 = c1.batch * c1.seqlen
-    fl1 = prefill_flops(c1.batch, c1.seqlen, c1.nheads, c1.headdim, c1.dstate, c1.ngroups, c1.chunk)
-    xf1 = executed_flops(c1.batch, c1.seqlen, c1.nheads, c1.headdim, c1.dstate, c1.ngroups, path1)
-    nb1 = prefill_bytes(c1.batch, c1.seqlen, c1.nheads, c1.headdim, c1.dstate, c1.ngroups, 2, 4, 4)
-    r1 = roofline_of(nb1, fl1, ms1 * 1e-3, peaks, peak_kind)
-    r1.update({"traffic": ncu_traffic("ssd_prefill_pair.cu", "mamba2_1p3b"),
-               "kernel": "ssd_chunk_scan_fwd (decay cumsum + tcgen05 head-pair chunk kernel)"})
-    c1_line = {"workload": c1.name, "steps": c1_steps, "tokens_per_s": t1 * world / (ms1 * 1e-3), "ms_per_step": ms1,
-               "tflops": fl1 / (ms1 * 1e-3) / 1e12, "executed_tflops": xf1 / (ms1 * 1e-3) / 1e12,
-               "executed_flops_per_call": xf1, "gbs": nb1 / (ms1 * 1e-3) / 1e9, "kernel_path": PATH_NAMES[path1],
-               "y": "fp32", "final_state": "fp32", "l2": "3 rotating input sets (x 67 MB each)",
-               "roofline": r1, "clocks": c1clk.summary()}
-
-    # ---- backward pass of the same layer
-    gen = torch.Generator(device=dev)
-    gen.manual_seed(1000 + rank)
-    dyb = torch.randn((c1.batch, c1.seqlen, c1.nheads, c1.headdim), generator=gen, device=dev).to(bf16)
-    dfin = 0.1 * torch.randn((c1.batch, c1.nheads, c1.dstate, c1.headdim), generator=gen, device=dev)
-    bws = torch.empty(ssd.ssd_chunk_scan_bwd_workspace_size(desc1), dtype=torch.uint8, device=dev)
-    gx = torch.empty((c1.batch, c1.seqlen, c1.nheads, c1.headdim), dtype=torch.float32, device=dev)
-    gdt = torch.empty((c1.batch, c1.seqlen, c1.nheads), dtype=torch.float32, device=dev)
-    gB = torch.empty((c1.batch, c1.seqlen, c1.ngroups, c1.dstate), dtype=torch.float32, device=dev)
-    gC = torch.empty_like(gB)
-    gpar = torch.empty((3, c1.nheads), dtype=torch.float32, device=dev)
-    launches_per_bwd = ssd.ssd_chunk_scan_bwd_launches(desc1, True)
-
-    def backward(k):
-        d = sets[k % NSETS]
-        st = ssd.ssd_chunk_scan_bwd(desc1, d["x"].data_ptr(), d["dt_raw"].data_ptr(), d["dt_bias"].data_ptr(),
-                                    d["A"].data_ptr(), d["B"].data_ptr(), d["C"].data_ptr(), d["D"].data_ptr(), 0,
-                                    dyb.data_ptr(), dfin.data_ptr(), gx.data_ptr(), gdt.data_ptr(),
-                                    gpar[0].data_ptr(), gpar[1].data_ptr(), gB.data_ptr(), gC.data_ptr(),
-                                    gpar[2].data_ptr(), 0, bws.data_ptr(), bws.numel(), stream.cuda_stream)
-        if st:
-            raise ssd.SsdError(st, "ssd_chunk_scan_bwd")
-
-    bsteps = max(10, min(args.steps, 50))
-    bms = timed(torch, stream, backward, bsteps, args.warmup, pg, dist)
-    check("the timed backward")
-    bbytes = backward_bytes(c1.batch, c1.seqlen, c1.nheads, c1.headdim, c1.dstate, c1.ngroups, 2, 4, 4)
-    bflops = backward_flops(c1.batch, c1.seqlen, c1.nheads, c1.headdim, c1.dstate, c1.ngroups, c1.chunk)
-    broof = roofline_of(bbytes, bflops, bms * 1e-3, peaks, peak_kind)
-    broof["kernel"] = ("ssd_chunk_scan_bwd (block form on tensor cores: state passes, block gradients, "
-                       "dB/dC partial sums, parameter sums)")
-    bexec = backward_executed_flops(c1.batch, c1.seqlen, c1.nheads, c1.headdim, c1.dstate, c1.ngroups)
-    backward_line = {"tokens_per_s": t1 * world / (bms * 1e-3), "ms_per_step": bms, "steps": bsteps,
-                     "launches_per_step": launches_per_bwd, "gradients": "fp32", "dfinal_state": "given",
-                     "gbs": bbytes / (bms * 1e-3) / 1e9, "tflops": bflops / (bms * 1e-3) / 1e12,
-                     "executed_tflops": bexec / (bms * 1e-3) / 1e12, "executed_flops_per_call": bexec,
-                     "roofline": broof}
-    del dyb, dfin, bws, gx, gdt, gB, gC, gpar
-
-    # ---- Mamba-3 prefill (trapezoidal input + rotational state) of the same layer
-    ex = I.draw_mamba3_extras(c1.batch, c1.seqlen, c1.nheads, c1.ngroups, c1.dstate, c1.seed + rank)
-    m3_lam, m3_theta = to_dev(ex["lam"]), to_dev(ex["theta"])
-    m3ws = torch.empty(ssd.ssd_chunk_scan_mamba3_workspace_size(desc1), dtype=torch.uint8, device=dev)
-    launches_per_m3 = ssd.ssd_chunk_scan_mamba3_launches(desc1, True, True, True)
-
-    def mamba3(k):
-        d = sets[k % NSETS]
-        st = ssd.ssd_chunk_scan_fwd_mamba3(desc1, d["x"].data_ptr(), d["dt_raw"].data_ptr(), d["dt_bias"].data_ptr(),
-                                           d["A"].data_ptr(), d["B"].data_ptr(), d["C"].data_ptr(),
-                                           d["D"].data_ptr(), m3_lam.data_ptr(), m3_theta.data_ptr(), 0,
-                                           y1.data_ptr(), f1.data_ptr(), m3ws.data_ptr(), m3ws.numel(),
-                                           stream.cuda_stream)
-        if st:
-            raise ssd.SsdError(st, "ssd_chunk_scan_fwd_mamba3")
-
-    m3steps = max(10, min(args.steps, 50))
-    m3ms = timed(torch, stream, mamba3, m3steps, args.warmup, pg, dist)
-    check("the timed Mamba-3 prefill")
-    mamba3_line = {"tokens_per_s": t1 * world / (m3ms * 1e-3), "ms_per_step": m3ms, "steps": m3steps,
-                   "launches_per_step": launches_per_m3, "vs_mamba2_prefill_time": m3ms / ms1,
-                   "inputs": "lam ~ U[0,1] per (token, head), theta ~ U[-0.5,0.5] rad per (token, group, pair)",
-                   "path": "B, C turned by the cumulative angle in bf16 hi/lo pairs, three tensor-core scans"}
-    c1_line["backward"] = backward_line
-    c1_line["mamba3"] = mamba3_line
-    del sets, y1, f1, ws1, m3ws
-    torch.cuda.empty_cache()
+    c1_line = layer_legs()
 
     # ================= the other workloads: tiny fp32 prefill, long-sequence / state-size sweep
     workloads = None

@@ -163,24 +163,63 @@ replay_step_kernel(StateT* __restrict__ ckpt, IoT* __restrict__ xb, IoT* __restr
     // state vectors in flight per lane (the fold holds x_s of 16 tokens as well)
     constexpr int U = FLUSH ? 4 : RP_U;
 
-    const float dt = softplus_f32(to_f32(dt_raw[bh]) + (dt_bias ? dt_bias[h] : 0.f));
-    const float cum_t = (fill > 0 ? cumb[(size_t)bh * K + fill - 1] : 0.f) + dt * A[h];
-    const float alpha = expf(cum_t);
+    // the prologue's independent loads first, so that they are in flight together:
+    // this step's dt_raw and head parameters, the buffered cumsum and dt of lane
+    // s's slot, C_t . B_s, C_t (N <= 256: at most 8 elements a lane), x_t
     const IoT* cg = Cm + bg * N;
     const IoT* bcur = Bm + bg * N;
-    for (int i = lane; i < N; i += 32) cs[i] = to_f32(cg[i]);
+    const float draw = to_f32(dt_raw[bh]), bias = dt_bias ? dt_bias[h] : 0.f, Ah = A[h];
+    const float cumf = fill > 0 ? cumb[(size_t)bh * K + fill - 1] : 0.f;
+    float cum_l = 0.f, dt_l = 0.f;
+    if (lane < fill) {
+        cum_l = cumb[(size_t)bh * K + lane];
+        dt_l = dtb[(size_t)bh * K + lane];
+    }
+    const float cbv = (!FLUSH && lane <= fill) ? cb[bg * 16 + lane] : 0.f;   // C_t . B_s (ordinary step)
+    float cv[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) cv[i] = lane + 32 * i < N ? to_f32(cg[lane + 32 * i]) : 0.f;
+    float xt[RP_VEC];
+    load4(x + (size_t)bh * P + p0, xt);
+    const float dt = softplus_f32(draw + bias);
+    const float cum_t = cumf + dt * Ah;
+    const float alpha = expf(cum_t);
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        if (lane + 32 * i < N) cs[lane + 32 * i] = cv[i];
     // lane s <= fill: token s of the buffer (s == fill: this step's token)
     float beta = 0.f;
     if (lane <= fill) {
-        const float cum_s = lane < fill ? cumb[(size_t)bh * K + lane] : cum_t;
-        const float dt_s = lane < fill ? dtb[(size_t)bh * K + lane] : dt;
+        const float cum_s = lane < fill ? cum_l : cum_t;
+        const float dt_s = lane < fill ? dt_l : dt;
         beta = expf(cum_t - cum_s) * dt_s;
     }
     __syncwarp();
     float w = 0.f;                             // lane s: beta_s (C_t . B_s)
-    if (!FLUSH) {
-        if (lane <= fill) w = beta * cb[bg * 16 + lane];
-    } else {
+    if (!FLUSH) w = beta * cbv;
+    uint64_t xs2[8][RP_VEC];                   // the fold's x pairs (below), loaded before the B rows
+    if (FLUSH) {
+        // x of the 16 slots for this lane's 4 columns (slot fill: x_t; past it: zero), as
+        // pairs of consecutive slots per column: the paired FMA below adds slots 2k and
+        // 2k + 1 of one column at once, against the coefficient pair (g_2k, g_2k+1)
+#pragma unroll
+        for (int k2 = 0; k2 < 8; ++k2) {
+            float xa[RP_VEC], xb2[RP_VEC];
+#pragma unroll
+            for (int z = 0; z < 2; ++z) {
+                const int s = 2 * k2 + z;
+                float* xv = z ? xb2 : xa;
+                if (s < fill) load4(xb + ((size_t)bh * K + s) * P + p0, xv);
+                else {
+#pragma unroll
+                    for (int j = 0; j < RP_VEC; ++j) xv[j] = s == fill ? xt[j] : 0.f;
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < RP_VEC; ++j) xs2[k2][j] = f2pack(xa[j], xb2[j]);
+        }
+    }
+    if (FLUSH) {
         // g[n][s] for the 16 slots (unused slots K..15 get zero coefficients), the B_s
         // rows read as 16-byte vectors, 8 per lane in flight at once
         using BV = Vec16<IoT>;
@@ -211,8 +250,6 @@ replay_step_kernel(StateT* __restrict__ ckpt, IoT* __restrict__ xb, IoT* __restr
         __syncwarp();
     }
 
-    float xt[RP_VEC];
-    load4(x + (size_t)bh * P + p0, xt);
     float acc[RP_VEC] = {0.f, 0.f, 0.f, 0.f};
     if (!FLUSH) {
         // read-only pass: acc = sum_n C[n] h_c[n][cols]
@@ -234,26 +271,6 @@ replay_step_kernel(StateT* __restrict__ ckpt, IoT* __restrict__ xb, IoT* __restr
             }
         }
     } else {
-        // x of the 16 slots for this lane's 4 columns (slot fill: x_t; past it: zero), as
-        // pairs of consecutive slots per column: the paired FMA below adds slots 2k and
-        // 2k + 1 of one column at once, against the coefficient pair (g_2k, g_2k+1)
-        uint64_t xs2[8][RP_VEC];
-#pragma unroll
-        for (int k2 = 0; k2 < 8; ++k2) {
-            float xa[RP_VEC], xb2[RP_VEC];
-#pragma unroll
-            for (int z = 0; z < 2; ++z) {
-                const int s = 2 * k2 + z;
-                float* xv = z ? xb2 : xa;
-                if (s < fill) load4(xb + ((size_t)bh * K + s) * P + p0, xv);
-                else {
-#pragma unroll
-                    for (int j = 0; j < RP_VEC; ++j) xv[j] = s == fill ? xt[j] : 0.f;
-                }
-            }
-#pragma unroll
-            for (int j = 0; j < RP_VEC; ++j) xs2[k2][j] = f2pack(xa[j], xb2[j]);
-        }
         // h <- alpha h + sum_s g[n][s] x_s[cols] (even and odd slots summed apart, then
         // added); acc = sum_n C[n] h_new[n][cols]
         for (int r0 = r_off; r0 < N; r0 += U * rstep) {
