@@ -63,15 +63,15 @@ Mamba3Layout mamba3_layout(int64_t batch, int64_t L, int64_t H, int64_t P, int64
 
 // Sum of the angles of every (b, g, chunk) and pair k, in float64.  Block =
 // (b, g, chunk); threads = (token lane, pair).
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(1024)
 m3_angle_sums_kernel(const float* __restrict__ theta, double* __restrict__ csum, int64_t L, int G, int K, int Q,
                      int nchunks) {
-    __shared__ double part[256];
+    __shared__ double part[1024];
     const int c = (int)(blockIdx.x % (unsigned)nchunks);
     const int64_t bg = blockIdx.x / (unsigned)nchunks;
     const int g = (int)(bg % G);
     const int64_t b = bg / G;
-    const int lanes = 256 / K;                  // K = N/2 <= 128, so at least 2
+    const int lanes = 1024 / K;                 // K = N/2 <= 128, so at least 8
     const int tid = threadIdx.x;
     double s = 0.0;
     if (tid < lanes * K) {
@@ -355,7 +355,7 @@ static cudaError_t mamba3_t(const Mamba3Args& a, cudaStream_t s) {
     IoT* Ctl = split ? (IoT*)(ws + l.off_Ctl) : nullptr;
     double* thL = (double*)(ws + l.off_thL);
     if (a.theta) {
-        m3_angle_sums_kernel<<<(unsigned)(a.batch * G * nchunks), 256, 0, s>>>(
+        m3_angle_sums_kernel<<<(unsigned)(a.batch * G * nchunks), 1024, 0, s>>>(
             a.theta, (double*)(ws + l.off_csum), a.L, G, K, Q, nchunks);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         const int KG = (K + 3) / 4;
