@@ -482,7 +482,10 @@ def main():
         mamba3_line = {"tokens_per_s": t1 * world / (m3ms * 1e-3), "ms_per_step": m3ms, "steps": m3steps,
                        "launches_per_step": launches_per_m3, "vs_mamba2_prefill_time": m3ms / ms1,
                        "inputs": "lam ~ U[0,1] per (token, head), theta ~ U[-0.5,0.5] rad per (token, group, pair)",
-                       "path": "B, C turned by the cumulative angle in bf16 hi/lo pairs, three tensor-core scans"}
+                       "path": ("B, C turned by the cumulative angle in bf16 hi/lo pairs, one head-pair scan taking "
+                                "the three products and the diagonal correction"
+                                if ssd.ssd_chunk_scan_path(desc1) == 2 else
+                                "B, C turned by the cumulative angle in bf16 hi/lo pairs, three tensor-core scans")}
         c1_line["backward"] = backward_line
         c1_line["mamba3"] = mamba3_line
         del sets, y1, f1, ws1, m3ws

@@ -326,7 +326,7 @@ ssd_status_t ssd_chunk_scan_mamba3_launches(const ssd_prefill_desc_t* desc, int3
     else if (desc->seqlen == 0) *launches = has_final_state ? 1 : 0;
     else if (!has_lam && !has_theta) *launches = 1 + (tc ? 1 : 3);
     else *launches = mamba3_launches(tc, desc->io_dtype == SSD_BF16, has_lam != 0, has_theta != 0,
-                                     has_final_state != 0);
+                                     has_final_state != 0, m3_layout(desc).fused);
     return SSD_OK;
 }
 

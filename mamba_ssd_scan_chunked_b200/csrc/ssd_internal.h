@@ -104,6 +104,11 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s);
 // launch_prefill_tc takes it for the shapes it covers
 bool pair_path_supports(int64_t batch, int64_t H, int64_t P, int64_t N, int64_t G, int64_t Q, bool io_bf16);
 cudaError_t launch_prefill_pair(const PrefillArgs& a, cudaStream_t s);
+// its Mamba-3 form: B, C are the turned operands as [b][L][G][2][N] bf16 (hi, lo),
+// dt and the cumsum slots of the workspace hold the trapezoid's weights and the
+// decay cumsum, dxc [BH][Lpad] the diagonal correction (or NULL); the initial
+// state is read as bf16 when init_bf16, the final one written per a.state_bf16
+cudaError_t launch_prefill_pair_mamba3(const PrefillArgs& a, const float* dxc, bool init_bf16, cudaStream_t s);
 
 // Backward pass of the prefill (ssd_backward.cu).  Workspace carve-up, all
 // offsets 256-byte aligned; "slice" strides separate the column slices of the
@@ -168,14 +173,16 @@ int backward_launches(const BackwardLayout& l, bool has_states);
 struct Mamba3Layout {
     PrefillLayout scan;
     size_t off_corr;               // fp32 [b*H][Lpad]
-    size_t off_Bt, off_Ct;         // io dtype [b][L][G][N], rotated by -Theta_t (bf16: the hi part)
-    size_t off_Btl, off_Ctl;       // bf16 inputs: the lo part of the same
+    size_t off_Bt, off_Ct;         // io dtype [b][L][G][N], rotated by -Theta_t (bf16: the hi part;
+                                   // fused: [b][L][G][2][N], hi then lo per group)
+    size_t off_Btl, off_Ctl;       // bf16 inputs: the lo part of the same (unused when fused)
     size_t off_csum;               // fp64 [b][G][nchunks][N/2] angle sums per chunk
     size_t off_thL;                // fp64 [b][G][N/2] angle at the last token
     size_t off_y32[3];             // fp32 [b][L][H][P] scan outputs before the combination
     size_t off_fsr;                // state dtype [b][H][N][P] rotated-frame final state (scan 1)
     size_t off_fsr2;               // fp32 [b][H][N][P] the same of the B_lo scan
     size_t total;
+    bool fused;                    // bf16 with the head-pair kernel: one scan of the turned hi/lo operands
 };
 
 Mamba3Layout mamba3_layout(int64_t batch, int64_t L, int64_t H, int64_t P, int64_t N, int64_t G, int64_t Q,
@@ -194,7 +201,7 @@ struct Mamba3Args {
 };
 
 cudaError_t launch_mamba3(const Mamba3Args& a, cudaStream_t s);
-int mamba3_launches(bool tc, bool io_bf16, bool has_lam, bool has_theta, bool has_final);
+int mamba3_launches(bool tc, bool io_bf16, bool has_lam, bool has_theta, bool has_final, bool fused);
 
 // fault-injection bits set by ssd_debug_inject (read at every launch)
 uint32_t debug_faults();

@@ -21,8 +21,10 @@
 // them once costs 0.067 x rms(y) on the test shapes (float64 model), so each is
 // stored as a bf16 pair hi + lo and, the scan being bilinear in (B, C), run as
 // scan(B_hi, C_hi) + scan(B_lo, C_hi) + scan(B_hi, C_lo) (the lo x lo term, about
-// 2^-18 relative, is dropped; the model then gives 9.8e-5).  fp32 inputs take
-// one scan.
+// 2^-18 relative, is dropped; the model then gives 9.8e-5).  Where the head-pair
+// kernel covers the shape, its Mamba-3 form takes all three products and the
+// correction in one scan (the turned operands then interleaved as
+// [b][L][G][2][N], hi then lo).  fp32 inputs take one scan.
 #include "../../include/ssd.h"
 #include "ssd_common.cuh"
 #include "ssd_internal.h"
@@ -46,14 +48,20 @@ Mamba3Layout mamba3_layout(int64_t batch, int64_t L, int64_t H, int64_t P, int64
     s.off_states = take(sizeof(float) * (size_t)N * P * BH * nstates);
     s.off_flags = take(sizeof(int) * ((size_t)BH + 64));
     const size_t e = io_bf16 ? 2 : 4, tok = (size_t)batch * L;
+    const size_t opb = e * tok * G * N;        // one turned operand
+    l.fused = io_bf16 && tc && pair_path_supports(batch, H, P, N, G, Q, io_bf16);
     l.off_corr = take(sizeof(float) * BH * s.Lpad);
-    l.off_Bt = take(e * tok * G * N);
-    l.off_Ct = take(e * tok * G * N);
-    l.off_Btl = take(e * tok * G * N);
-    l.off_Ctl = take(e * tok * G * N);
+    // bf16: hi and lo of each turned operand in one region (lo after hi, or
+    // interleaved per group in the fused form)
+    l.off_Bt = take(opb * (io_bf16 ? 2 : 1));
+    l.off_Ct = take(opb * (io_bf16 ? 2 : 1));
+    l.off_Btl = io_bf16 ? l.off_Bt + opb : 0;
+    l.off_Ctl = io_bf16 ? l.off_Ct + opb : 0;
     l.off_csum = take(sizeof(double) * (size_t)batch * G * s.nchunks * (N / 2));
     l.off_thL = take(sizeof(double) * (size_t)batch * G * (N / 2));
-    for (int i = 0; i < 3; ++i) l.off_y32[i] = take(sizeof(float) * tok * H * P);
+    // fp32 scan outputs before the combination: three for the split scans, one
+    // otherwise (the fused form writes y itself; lam without theta still combines)
+    for (int i = 0; i < 3; ++i) l.off_y32[i] = (i == 0 || !l.fused) ? take(sizeof(float) * tok * H * P) : 0;
     l.off_fsr = take(sizeof(float) * (size_t)BH * N * P);
     l.off_fsr2 = take(sizeof(float) * (size_t)BH * N * P);
     s.total = off;
@@ -99,7 +107,7 @@ __global__ void __launch_bounds__(256)
 m3_rotate_kernel(const IoT* __restrict__ B, const IoT* __restrict__ C, const float* __restrict__ theta,
                  const double* __restrict__ csum, IoT* __restrict__ Bt, IoT* __restrict__ Ct, IoT* __restrict__ Btl,
                  IoT* __restrict__ Ctl, double* __restrict__ thL, int64_t L, int G, int N, int Q, int nchunks,
-                 int KG) {
+                 int KG, int ostride) {
     __shared__ double wtot[8][4];
     __shared__ double carry[4];
     const int kg = (int)(blockIdx.x % (unsigned)KG);
@@ -147,6 +155,7 @@ m3_rotate_kernel(const IoT* __restrict__ B, const IoT* __restrict__ C, const flo
     for (int q = 0; q < 4; ++q) v[q] += carry[q];
     if (!live) return;
     const int64_t row = ((b * L + t) * G + g) * N;
+    const int64_t orow = ((b * L + t) * G + g) * ostride;     // N, or 2N with hi and lo interleaved
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
         if (k0 + q >= K) break;
@@ -158,8 +167,8 @@ m3_rotate_kernel(const IoT* __restrict__ B, const IoT* __restrict__ C, const flo
         const float c0 = to_f32(C[row + n0]), c1 = to_f32(C[row + n0 + 1]);
         // R(-Theta): (u, w) -> (cos u + sin w, -sin u + cos w); stored as hi (+ lo for bf16)
         const float r[4] = {cs * b0 + sn * b1, cs * b1 - sn * b0, cs * c0 + sn * c1, cs * c1 - sn * c0};
-        IoT* dst[4] = {Bt + row + n0, Bt + row + n0 + 1, Ct + row + n0, Ct + row + n0 + 1};
-        IoT* dlo[4] = {Btl + row + n0, Btl + row + n0 + 1, Ctl + row + n0, Ctl + row + n0 + 1};
+        IoT* dst[4] = {Bt + orow + n0, Bt + orow + n0 + 1, Ct + orow + n0, Ct + orow + n0 + 1};
+        IoT* dlo[4] = {Btl + orow + n0, Btl + orow + n0 + 1, Ctl + orow + n0, Ctl + orow + n0 + 1};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const IoT hi = from_f32<IoT>(r[i]);
@@ -170,9 +179,11 @@ m3_rotate_kernel(const IoT* __restrict__ B, const IoT* __restrict__ C, const flo
     }
 }
 
-// Scan weights w, chunk-local decay cumsum and the diagonal correction c, as
-// the forward's decay kernel lays them out ([b*H][Lpad]); also clears the
-// scan's hand-off flags.  Block = (b, chunk, 8 heads), thread = token.
+// Scan weights w, chunk-local decay cumsum and the diagonal correction's
+// coefficient c, as the forward's decay kernel lays them out ([b*H][Lpad]);
+// also clears the scan's hand-off flags.  Block = (b, chunk, 8 heads), thread =
+// token.  With B and C given (the fused form) the correction is written whole,
+// c_t (C_t . B_t), the dot product of the head's group formed by the thread.
 constexpr int M3_HG = 8;
 
 template <typename IoT>
@@ -180,7 +191,8 @@ __global__ void __launch_bounds__(256)
 m3_decay_kernel(const IoT* __restrict__ dt_raw, const float* __restrict__ dt_bias, const float* __restrict__ A,
                 const float* __restrict__ lam, float* __restrict__ w_out, float* __restrict__ acs_out,
                 float* __restrict__ corr_out, int* __restrict__ flags, int64_t L, int64_t Lpad, int H, int Q,
-                int nflags, int nchunks, int hgroups) {
+                int nflags, int nchunks, int hgroups, const IoT* __restrict__ Bcb, const IoT* __restrict__ Ccb,
+                int G, int N) {
     __shared__ float warp_tot[8][M3_HG];
     const int hg = (int)(blockIdx.x % (unsigned)hgroups);
     const int c = (int)((blockIdx.x / (unsigned)hgroups) % (unsigned)nchunks);
@@ -208,6 +220,33 @@ m3_decay_kernel(const IoT* __restrict__ dt_raw, const float* __restrict__ dt_bia
         cr[k] = (1.f - lmn) * dtn;            // 0 without lam, at the last token and past it
         w[k] = lm * dt + cr[k];
         v[k] = h < H ? dt * A[h] : 0.f;
+    }
+    if (Bcb && live) {
+        int gprev = -1;
+        float cb = 0.f;
+        const int hpg = H / G;
+#pragma unroll
+        for (int k = 0; k < M3_HG; ++k) {
+            const int h = h0 + k;
+            if (h >= H) break;
+            if (h / hpg != gprev) {
+                gprev = h / hpg;
+                const int64_t grow = ((b * L + t) * G + gprev) * N;
+                cb = 0.f;
+                if (sizeof(IoT) == 2 && (N & 7) == 0) {    // 16-byte rows of 8 bf16 (the arrays are 16-byte aligned)
+                    for (int n = 0; n < N; n += 8) {
+                        float cv[8], bv[8];
+                        Vec16<bf16>::load(reinterpret_cast<const bf16*>(Ccb + grow + n), cv);
+                        Vec16<bf16>::load(reinterpret_cast<const bf16*>(Bcb + grow + n), bv);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) cb += cv[i] * bv[i];
+                    }
+                } else {
+                    for (int n = 0; n < N; ++n) cb += to_f32(Ccb[grow + n]) * to_f32(Bcb[grow + n]);
+                }
+            }
+            cr[k] *= cb;
+        }
     }
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -305,9 +344,9 @@ m3_combine_kernel(const float* y1, const float* __restrict__ y2, const float* __
 
 // h_{L-1} = R(Theta_{L-1}) ~S_{L-1}: rows (2k, 2k+1) of every head of group g;
 // ~S_{L-1} = src (+ src2, the B_lo scan's final state, when split).
-template <typename StateT>
+template <typename SrcT, typename StateT>
 __global__ void __launch_bounds__(256)
-m3_unrotate_state_kernel(const StateT* __restrict__ src, const float* __restrict__ src2,
+m3_unrotate_state_kernel(const SrcT* __restrict__ src, const float* __restrict__ src2,
                          const double* __restrict__ thL, StateT* __restrict__ dst, int64_t batch, int H, int P, int N,
                          int G) {
     const int K = N / 2, hpg = H / G;
@@ -351,8 +390,11 @@ static cudaError_t mamba3_t(const Mamba3Args& a, cudaStream_t s) {
     cudaError_t e;
     IoT* Bt = (IoT*)(ws + l.off_Bt);
     IoT* Ct = (IoT*)(ws + l.off_Ct);
-    IoT* Btl = split ? (IoT*)(ws + l.off_Btl) : nullptr;
-    IoT* Ctl = split ? (IoT*)(ws + l.off_Ctl) : nullptr;
+    // the fused form (one head-pair scan of the turned hi/lo operands): hi and lo
+    // interleaved per group, [b][L][G][2][N]
+    const bool fused = split && l.fused;
+    IoT* Btl = split ? (fused ? Bt + N : (IoT*)(ws + l.off_Btl)) : nullptr;
+    IoT* Ctl = split ? (fused ? Ct + N : (IoT*)(ws + l.off_Ctl)) : nullptr;
     double* thL = (double*)(ws + l.off_thL);
     if (a.theta) {
         m3_angle_sums_kernel<<<(unsigned)(a.batch * G * nchunks), 1024, 0, s>>>(
@@ -361,7 +403,7 @@ static cudaError_t mamba3_t(const Mamba3Args& a, cudaStream_t s) {
         const int KG = (K + 3) / 4;
         m3_rotate_kernel<IoT><<<(unsigned)(a.batch * G * nchunks * KG), (unsigned)(Q < 32 ? 32 : Q), 0, s>>>(
             (const IoT*)a.B, (const IoT*)a.C, a.theta, (const double*)(ws + l.off_csum), Bt, Ct, Btl, Ctl, thL, a.L,
-            G, N, Q, nchunks, KG);
+            G, N, Q, nchunks, KG, fused ? 2 * N : N);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     {
@@ -369,8 +411,34 @@ static cudaError_t mamba3_t(const Mamba3Args& a, cudaStream_t s) {
         m3_decay_kernel<IoT><<<(unsigned)(a.batch * nchunks * hgroups), (unsigned)(Q < 32 ? 32 : Q), 0, s>>>(
             (const IoT*)a.dt_raw, a.dt_bias, a.A, a.lam, (float*)(ws + l.scan.off_dt), (float*)(ws + l.scan.off_acs),
             (float*)(ws + l.off_corr), (int*)(ws + l.scan.off_flags), a.L, l.scan.Lpad, H, Q, nflags, nchunks,
-            hgroups);
+            hgroups, fused && a.lam ? (const IoT*)a.B : nullptr, fused && a.lam ? (const IoT*)a.C : nullptr, G, N);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    if (fused) {
+        // one scan: the head-pair kernel's Mamba-3 form writes y (with D and the
+        // correction) and the turned final state in fp32 (rounded to the state
+        // dtype once, when turned back); the initial state enters the turned frame
+        // unchanged (no angle before the first token)
+        PrefillArgs p{};
+        p.batch = a.batch; p.L = a.L; p.H = a.H; p.P = a.P; p.N = a.N; p.G = a.G; p.Q = a.Q;
+        p.io_bf16 = true; p.y_bf16 = a.y_bf16; p.state_bf16 = false;
+        p.x = a.x; p.dt_raw = a.dt_raw; p.dt_bias = a.dt_bias; p.A = a.A;
+        p.B = Bt; p.C = Ct; p.D = a.D;
+        p.init_state = a.init_state; p.y = a.y; p.final_state = a.final_state ? (void*)(ws + l.off_fsr) : nullptr;
+        p.ws = ws; p.lay = l.scan; p.pad_left = nullptr; p.dev_err = a.dev_err; p.drop_publish = 0;
+        e = launch_prefill_pair_mamba3(p, a.lam ? (const float*)(ws + l.off_corr) : nullptr, a.state_bf16, s);
+        if (e != cudaSuccess) return e;
+        if (a.final_state) {
+            const unsigned grid = m3_grid(a.batch * H * K * P, 256);
+            if (a.state_bf16)
+                m3_unrotate_state_kernel<float, bf16><<<grid, 256, 0, s>>>(
+                    (const float*)(ws + l.off_fsr), nullptr, thL, (bf16*)a.final_state, a.batch, H, P, N, G);
+            else
+                m3_unrotate_state_kernel<float, float><<<grid, 256, 0, s>>>(
+                    (const float*)(ws + l.off_fsr), nullptr, thL, (float*)a.final_state, a.batch, H, P, N, G);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        }
+        return cudaSuccess;
     }
     // the scans: with lam or the split the outputs are combined (and corrected)
     // afterwards from fp32; with theta the final state is rotated back afterwards
@@ -427,10 +495,10 @@ static cudaError_t mamba3_t(const Mamba3Args& a, cudaStream_t s) {
         const unsigned grid = m3_grid(a.batch * H * K * P, 256);
         const float* src2 = split ? (const float*)(ws + l.off_fsr2) : nullptr;
         if (a.state_bf16)
-            m3_unrotate_state_kernel<bf16><<<grid, 256, 0, s>>>((const bf16*)(ws + l.off_fsr), src2, thL,
+            m3_unrotate_state_kernel<bf16, bf16><<<grid, 256, 0, s>>>((const bf16*)(ws + l.off_fsr), src2, thL,
                                                                (bf16*)a.final_state, a.batch, H, P, N, G);
         else
-            m3_unrotate_state_kernel<float><<<grid, 256, 0, s>>>((const float*)(ws + l.off_fsr), src2, thL,
+            m3_unrotate_state_kernel<float, float><<<grid, 256, 0, s>>>((const float*)(ws + l.off_fsr), src2, thL,
                                                                 (float*)a.final_state, a.batch, H, P, N, G);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
@@ -441,9 +509,11 @@ cudaError_t launch_mamba3(const Mamba3Args& a, cudaStream_t s) {
     return a.io_bf16 ? mamba3_t<bf16>(a, s) : mamba3_t<float>(a, s);
 }
 
-int mamba3_launches(bool tc, bool io_bf16, bool has_lam, bool has_theta, bool has_final) {
+int mamba3_launches(bool tc, bool io_bf16, bool has_lam, bool has_theta, bool has_final, bool fused) {
     const int scan = tc ? 1 : 3;
     const bool split = has_theta && io_bf16;
+    // the fused form: angle sums, rotation, weights, the head-pair scan, the final state turned back
+    if (split && fused) return 4 + (has_final ? 1 : 0);
     return (has_theta ? 2 : 0) + 1 + scan + (split ? 2 * (1 + scan) : 0) + ((has_lam || split) ? 1 : 0) +
            ((has_theta && has_final) ? 1 : 0);
 }

@@ -39,6 +39,22 @@
 // Every wait on an mbarrier is bounded (2 s); the first one that gives up sets
 // the device error word and a CTA-wide abort word that ends every later wait
 // at once, so the launch always finishes.  No inter-CTA waits exist.
+//
+// The Mamba-3 form (template flag M3) runs the whole Mamba-3 prefill in one
+// scan.  Its B and C are the operands turned by the cumulative angle, which are
+// no longer bf16 numbers; each comes as a bf16 pair hi + lo (groups 2g and
+// 2g + 1 of the operand arrays), and every product with them is taken as
+// hi x hi + hi x lo + lo x hi:
+//   S      = C_hi B_hi^T + C_hi B_lo^T + C_lo B_hi^T
+//   Yoff_k = C_hi h_hi + C_hi h_lo + C_lo h_hi
+//   h_k'  += B_hi^T wX_hi + B_hi^T wX_lo + B_lo^T wX_hi
+// (the lo x lo terms are about 2^-16 of the product and dropped).  The four
+// operand tiles fill both C/B stages, so there is one stage: C of the next
+// block is loaded once C h is done, B once the state MMAs are, and y goes
+// from the registers straight to global memory instead of through a staging
+// tile.  The epilogue also takes the trapezoid's diagonal correction,
+// y = Y + (D - c_t) x with c_t = (1 - lam_{t+1}) dt_{t+1} (C_t . B_t) per
+// token and head, from the workspace.
 #include "ssd_internal.h"
 #include "ssd_tc_common.cuh"
 
@@ -87,6 +103,11 @@ struct Params {
     long long Lpad;
     int H, G, Q, nblk, npairs;
     int state_bf16, y_bf16;
+    // the Mamba-3 form only
+    const float* dxc;          // [BH][Lpad] diagonal correction c_t, or NULL (= 0)
+    void* y;                   // [b][L][H][PD] y dtype
+    long long L;
+    int init_bf16;             // the initial state's dtype (the final state's is state_bf16)
 };
 
 // bounded wait that gives up at once when another wait of the CTA has given up
@@ -119,6 +140,7 @@ __device__ __forceinline__ void split8(const float* v, uint32_t (&hw)[4], uint32
 
 // 18 warps, 5 of them on one SM sub-partition (16384 registers each): at most 96
 // registers a thread, which the launch bounds give
+template <bool M3>
 __global__ void __launch_bounds__(THREADS, 1)
 ssd_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmY, const Params p) {
@@ -169,7 +191,62 @@ ssd_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
         if (!wait_or_abort(bar(i), ph, s_abort)) err |= kErrAsyncTimeout;
     };
 
-    if (warp == WARP_TMA) {
+    if (warp == WARP_TMA && M3) {
+        // ======================================================== TMA producer (Mamba-3 form)
+        // one stage: C hi, C lo at tiles 0-3 (K blocks 0, 1 each), B hi, B lo at 4-7
+        const uint32_t lead = elect_one();
+        auto load_c = [&](int t) {           // C of block t (+ x and the turned B, C of block t + 1 into L2)
+            const Item d = item_of(t / p.nblk);
+            const int t0 = (t % p.nblk) * SUB;
+            mbar_expect_tx(bar(B_CB0), 4 * TILE);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                tma_load_4d(base + (uint32_t)i * TILE, &tmC, 64 * (i & 1), 2 * d.g + (i >> 1), t0, d.b, bar(B_CB0));
+            if (t + 1 < total) {
+                const Item dn = item_of((t + 1) / p.nblk);
+                const int tn = ((t + 1) % p.nblk) * SUB;
+                tma_prefetch_4d(&tmX, 0, dn.h0, tn, dn.b);
+                tma_prefetch_4d(&tmX, 0, dn.h0 + 1, tn, dn.b);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    tma_prefetch_4d(&tmC, 64 * (i & 1), 2 * dn.g + (i >> 1), tn, dn.b);
+                    tma_prefetch_4d(&tmB, 64 * (i & 1), 2 * dn.g + (i >> 1), tn, dn.b);
+                }
+            }
+        };
+        auto load_b = [&](int t) {
+            const Item d = item_of(t / p.nblk);
+            const int t0 = (t % p.nblk) * SUB;
+            mbar_expect_tx(bar(B_CB1), 4 * TILE);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                tma_load_4d(base + (uint32_t)(4 + i) * TILE, &tmB, 64 * (i & 1), 2 * d.g + (i >> 1), t0, d.b,
+                            bar(B_CB1));
+        };
+        auto load_x = [&](int t) {
+            const Item d = item_of(t / p.nblk);
+            const int t0 = (t % p.nblk) * SUB;
+            mbar_expect_tx(bar(B_X), 2 * TILE);
+            tma_load_4d(base + OFF_X, &tmX, 0, d.h0, t0, d.b, bar(B_X));
+            tma_load_4d(base + OFF_X + TILE, &tmX, 0, d.h0 + 1, t0, d.b, bar(B_X));
+        };
+        if (lead && total > 0) {
+            load_c(0);
+            load_b(0);
+            load_x(0);
+        }
+        // C is free once C h is done (B_OFF), B once the state MMAs are (B_ST), x once Y is (B_Y)
+        for (int jj = 0; jj + 1 < total; ++jj) {
+            const uint32_t ph = jj & 1;
+            wait(B_OFF, ph);
+            if (lead && !*s_abort) load_c(jj + 1);
+            wait(B_ST, ph);
+            if (lead && !*s_abort) load_b(jj + 1);
+            wait(B_Y, ph);
+            if (lead && !*s_abort) load_x(jj + 1);
+            __syncwarp();
+        }
+    } else if (warp == WARP_TMA) {
         // ======================================================== TMA producer
         const uint32_t lead = elect_one();
         auto load_cb = [&](int t) {          // C, B of block t into stage t & 1 (+ its x into L2)
@@ -233,11 +310,21 @@ ssd_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
         for (int jj = 0; jj < total; ++jj) {
             const uint32_t ph = jj & 1;
             const uint32_t lead = lead0 && !*s_abort;     // once a wait gave up, issue nothing more
-            const uint32_t st = base + (uint32_t)(jj & 1) * STAGE;
-            const uint64_t dC = sdesc(st, 16, 1024), dBk = sdesc(st + 2 * TILE, 16, 1024);
-            const uint64_t dBm = sdesc(st + 2 * TILE, TILE, 1024);
+            // operand tiles: the stage of the block (C at tiles 0-1, B at 2-3); in
+            // the Mamba-3 form the one stage, C hi / C lo / B hi / B lo at tiles 0 / 2 / 4 / 6
+            const uint32_t st = M3 ? base : base + (uint32_t)(jj & 1) * STAGE;
+            const uint32_t offB = M3 ? 4 * TILE : 2 * TILE;
+            const uint64_t dC = sdesc(st, 16, 1024), dBk = sdesc(st + offB, 16, 1024);
+            const uint64_t dBm = sdesc(st + offB, TILE, 1024);
+            const uint64_t dCl = sdesc(st + 2 * TILE, 16, 1024), dBkl = sdesc(st + 6 * TILE, 16, 1024);
+            const uint64_t dBml = sdesc(st + 6 * TILE, TILE, 1024);
             // ---- S = C B^T into R0 once the previous block's head-0 Y has read M_0 there
-            wait(B_CB0 + (jj & 1), (jj >> 1) & 1);
+            if (M3) {
+                wait(B_CB0, ph);
+                wait(B_CB1, ph);
+            } else {
+                wait(B_CB0 + (jj & 1), (jj >> 1) & 1);
+            }
             if (jj > 0) wait(B_Y0, ph ^ 1u);
             tc_fence_after();
             __syncwarp();
@@ -246,6 +333,14 @@ ssd_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                 const uint32_t o = (uint32_t)(k >> 2) * KBLOCK_K + (uint32_t)(k & 3) * KSTEP_K;
                 if (k == 0) { if (lead) mma_ss<ID_S, 0>(tmem + COL_R0, dC + o, dBk + o);
                 } else if (lead) mma_ss<ID_S, 1>(tmem + COL_R0, dC + o, dBk + o);
+            }
+            if (M3) {
+#pragma unroll
+                for (int k = 0; k < NS / 16; ++k) {
+                    const uint32_t o = (uint32_t)(k >> 2) * KBLOCK_K + (uint32_t)(k & 3) * KSTEP_K;
+                    if (lead) mma_ss<ID_S, 1>(tmem + COL_R0, dC + o, dBkl + o);
+                    if (lead) mma_ss<ID_S, 1>(tmem + COL_R0, dCl + o, dBk + o);
+                }
             }
             if (lead) mma_commit(bar(B_S));
             // ---- Yoff_k = C h_k,hi + C h_k,lo (h written by the compute warps; the
@@ -265,6 +360,13 @@ ssd_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                 const uint32_t o = (uint32_t)(k >> 2) * KBLOCK_K + (uint32_t)(k & 3) * KSTEP_K;
                 if (lead) mma_ss<ID_OFF, 1>(tmem + COL_Y, dC + o, dWlo + k * KSTEP_MN);
             }
+            if (M3) {
+#pragma unroll
+                for (int k = 0; k < NS / 16; ++k) {
+                    const uint32_t o = (uint32_t)(k >> 2) * KBLOCK_K + (uint32_t)(k & 3) * KSTEP_K;
+                    if (lead) mma_ss<ID_OFF, 1>(tmem + COL_Y, dCl + o, dWhi + k * KSTEP_MN);
+                }
+            }
             if (lead) mma_commit(bar(B_OFF));
             // ---- state_k += B^T (w o X_k)_hi + B^T (w o X_k)_lo, onto 2^(r_last) h_k
             wait(B_WX, ph);
@@ -276,6 +378,11 @@ ssd_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
 #pragma unroll
             for (int k = 0; k < SUB / 16; ++k)
                 if (lead) mma_ss<ID_ST, 1>(tmem + COL_ST, dBm + k * KSTEP_MN, dWlo + k * KSTEP_MN);
+            if (M3) {
+#pragma unroll
+                for (int k = 0; k < SUB / 16; ++k)
+                    if (lead) mma_ss<ID_ST, 1>(tmem + COL_ST, dBml + k * KSTEP_MN, dWhi + k * KSTEP_MN);
+            }
             if (lead) mma_commit(bar(B_ST));
             // ---- Y_k += M_k,hi X_k + M_k,lo X_k onto the scaled Yoff (A from TMEM)
             wait(B_M, ph);
@@ -329,7 +436,7 @@ ssd_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                 } else if (p.init_state) {
                     float f[16];
                     const long long o = ((bh + k) * NS + row) * PD + 16 * kq;
-                    if (p.state_bf16) {
+                    if (M3 ? p.init_bf16 : p.state_bf16) {
                         Vec16<bf16>::load(reinterpret_cast<const bf16*>(p.init_state) + o, f);
                         Vec16<bf16>::load(reinterpret_cast<const bf16*>(p.init_state) + o + 8, f + 8);
                     } else {
@@ -374,12 +481,17 @@ ssd_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
         // this thread's per-token data of a block, read from the workspace one block
         // ahead: the cumsum of its row's token for both heads; for the table threads
         // (kq < 2: head kq, token = row) also dt and the cumsum of the token before
-        struct Pre { float2 row[2]; float dt; float2 prev; };
+        // (Mamba-3 form: also the diagonal correction of its row's token for both heads)
+        struct Pre { float2 row[2]; float dt; float2 prev; float dx[M3 ? 2 : 1]; };
         auto fetch = [&](const Item& dd, int jb, Pre& r) {
             const long long bh = (long long)dd.b * p.H + dd.h0;
             const long long t = (long long)jb * SUB + row;
             r.row[0] = cum(bh, t);
             r.row[1] = cum(bh + 1, t);
+            if (M3) {
+                r.dx[0] = p.dxc ? __ldcg(p.dxc + bh * p.Lpad + t) : 0.f;
+                r.dx[M3 ? 1 : 0] = p.dxc ? __ldcg(p.dxc + (bh + 1) * p.Lpad + t) : 0.f;
+            }
             if (kq < 2) {
                 r.dt = __ldcg(p.dtw + (bh + kq) * p.Lpad + t);
                 r.prev = row ? cum(bh + kq, t - 1) : make_float2(0.f, 0.f);
@@ -612,6 +724,39 @@ ssd_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(bar(B_EPI));          // the Y accumulators may be reused
+            if (M3) {
+                // y = Y + (D - c_t) x straight from the registers (16 columns of the row per head)
+                const long long t = (long long)j * SUB + row;
+                if (t < p.L) {
+#pragma unroll
+                    for (int k = 0; k < 2; ++k) {
+                        float out[16];
+                        const float dk = Dk[k] - cur.dx[M3 ? k : 0];
+                        const f32x2 dd = f2_pack(dk, dk);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            f2_unpack(f2_fma(dd, bf16x2_to_f2(xr[k][e]), f2_pack_u(yv[k][2 * e], yv[k][2 * e + 1])),
+                                      out[2 * e], out[2 * e + 1]);
+                        const long long o = (((long long)d.b * p.L + t) * p.H + d.h0 + k) * PD + 16 * kq;
+                        if (p.y_bf16) {
+                            bf16* yo = reinterpret_cast<bf16*>(p.y) + o;
+                            Vec16<bf16>::store(yo, out);
+                            Vec16<bf16>::store(yo + 8, out + 8);
+                        } else {
+                            float* yo = reinterpret_cast<float*>(p.y) + o;
+#pragma unroll
+                            for (int i = 0; i < 16; i += 4) Vec16<float>::store(yo + i, out + i);
+                        }
+                    }
+                }
+                ref[0] = g127[0];
+                ref[1] = g127[1];
+                cur = nxt;
+                it = it_n;
+                j = j_n;
+                d = d_n;
+                continue;
+            }
             uint8_t* stg = sm + (jj & 1) * STAGE;
 #pragma unroll
             for (int k = 0; k < 2; ++k) {
@@ -668,30 +813,33 @@ bool pair_path_supports(int64_t batch, int64_t H, int64_t P, int64_t N, int64_t 
            batch * H >= 148;
 }
 
-cudaError_t launch_prefill_pair(const PrefillArgs& a, cudaStream_t s) {
+// m3: the Mamba-3 form, B and C then [b][L][G][2][N] (hi, lo of the turned operands)
+static cudaError_t launch_pair(const PrefillArgs& a, bool m3, const float* dxc, bool init_bf16, cudaStream_t s) {
     using namespace pair;
     if (!pair_path_supports(a.batch, a.H, a.P, a.N, a.G, a.Q, a.io_bf16)) return cudaErrorNotSupported;
     CUtensorMap mx, mb, mc, my;
+    const uint64_t gops = (uint64_t)a.G * (m3 ? 2 : 1);    // groups of the B, C arrays
     if (!tc::make_map(&my, a.y, (uint64_t)a.P, (uint64_t)a.H, (uint64_t)a.L, (uint64_t)a.batch, !a.y_bf16) ||
         !tc::make_map(&mx, a.x, (uint64_t)a.P, (uint64_t)a.H, (uint64_t)a.L, (uint64_t)a.batch) ||
-        !tc::make_map(&mb, a.B, (uint64_t)a.N, (uint64_t)a.G, (uint64_t)a.L, (uint64_t)a.batch) ||
-        !tc::make_map(&mc, a.C, (uint64_t)a.N, (uint64_t)a.G, (uint64_t)a.L, (uint64_t)a.batch))
+        !tc::make_map(&mb, a.B, (uint64_t)a.N, gops, (uint64_t)a.L, (uint64_t)a.batch) ||
+        !tc::make_map(&mc, a.C, (uint64_t)a.N, gops, (uint64_t)a.L, (uint64_t)a.batch))
         return cudaErrorInvalidValue;
     static std::mutex mu;
-    static int sms_of[64] = {};
+    static int sms_of[64][2] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     {
         std::lock_guard<std::mutex> lk(mu);
-        if (!sms_of[dev]) {
-            e = cudaFuncSetAttribute(ssd_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM);
+        if (!sms_of[dev][m3]) {
+            e = cudaFuncSetAttribute(m3 ? ssd_pair_kernel<true> : ssd_pair_kernel<false>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM);
             if (e != cudaSuccess) return e;
             int sms = 0;
             e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
             if (e != cudaSuccess) return e;
-            sms_of[dev] = sms;
+            sms_of[dev][m3] = sms;
         }
     }
     Params p{};
@@ -713,7 +861,11 @@ cudaError_t launch_prefill_pair(const PrefillArgs& a, cudaStream_t s) {
     p.npairs = (int)pairs;
     p.state_bf16 = a.state_bf16;
     p.y_bf16 = a.y_bf16;
-    const unsigned grid = (unsigned)(pairs < sms_of[dev] ? pairs : sms_of[dev]);
+    p.dxc = dxc;
+    p.y = a.y;
+    p.L = a.L;
+    p.init_bf16 = init_bf16;
+    const unsigned grid = (unsigned)(pairs < sms_of[dev][m3] ? pairs : sms_of[dev][m3]);
     // a programmatic dependent of the decay-cumsum kernel before it on the stream:
     // the prologue and the first operand loads overlap that kernel; the producer
     // waits for it (griddepcontrol.wait) before it reads dt and the cumsum
@@ -727,7 +879,16 @@ cudaError_t launch_prefill_pair(const PrefillArgs& a, cudaStream_t s) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, ssd_pair_kernel, mx, mb, mc, my, p);
+    return m3 ? cudaLaunchKernelEx(&cfg, ssd_pair_kernel<true>, mx, mb, mc, my, p)
+              : cudaLaunchKernelEx(&cfg, ssd_pair_kernel<false>, mx, mb, mc, my, p);
+}
+
+cudaError_t launch_prefill_pair(const PrefillArgs& a, cudaStream_t s) {
+    return launch_pair(a, false, nullptr, a.state_bf16, s);
+}
+
+cudaError_t launch_prefill_pair_mamba3(const PrefillArgs& a, const float* dxc, bool init_bf16, cudaStream_t s) {
+    return launch_pair(a, true, dxc, init_bf16, s);
 }
 
 }  // namespace ssd

@@ -332,6 +332,14 @@ def test_mamba3_workspace_launches_and_validation():
     assert ssd.ssd_chunk_scan_mamba3_launches(d, False, True, False) == 2 + 1 + 1 + 2 * 2 + 1
     assert ssd.ssd_chunk_scan_mamba3_launches(d, False, False, True) == 2       # the plain forward
     assert ssd.ssd_chunk_scan_mamba3_launches(desc(io_dtype=ssd.SSD_F32), True, True, True) == 8
+    # 148 or more heads in all: the head-pair kernel's Mamba-3 form takes the three
+    # products and the correction in one scan (angle sums, rotation, weights, the
+    # scan, the final-state rotation)
+    dp = desc(nheads=80, ngroups=4)
+    assert ssd.ssd_chunk_scan_path(dp) == 2
+    assert ssd.ssd_chunk_scan_mamba3_launches(dp, True, True, True) == 5
+    assert ssd.ssd_chunk_scan_mamba3_launches(dp, False, True, False) == 4
+    assert ssd.ssd_chunk_scan_mamba3_launches(dp, True, False, True) == 3
 
     def call(dd, **kw):
         p = dict(x=FAKE, dt_raw=FAKE + 0x1000000, dt_bias=0, A=FAKE + 0x2000000, B=FAKE + 0x3000000,

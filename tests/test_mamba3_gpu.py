@@ -3,8 +3,9 @@ rotational state) against the float64 oracle's Mamba-3 recurrence, element by
 element on the same seeded inputs: y and the final state, max|err| / rms(oracle)
 within the bound of the input dtype.  Tensor-core shapes with ragged tails and
 every dstate, the CUDA-core fp32 path, sequences cut into runs, bf16 outputs
-and states, each of the two extensions alone, and the plain case (both absent)
-equal to ssd_chunk_scan_fwd bit for bit."""
+and states, each of the two extensions alone, the one-scan head-pair form (148
+heads or more), and the plain case (both absent) equal to ssd_chunk_scan_fwd bit
+for bit."""
 import numpy as np
 import pytest
 
@@ -52,6 +53,26 @@ def test_mamba3_matches_oracle(b, L, H, P, N, G, Q, io, use_lam, use_theta, with
     tol = TOL_BF16 if io == I.BF16 else TOL_F32
     assert metric(y, y_ref) <= tol
     assert metric(fs, fs_ref) <= tol
+
+
+@pytest.mark.parametrize("b,L,H,G,use_lam,use_theta,with_init,y_dtype,state", [
+    (2, 300, 80, 4, True, True, True, "f32", I.F32),      # ragged tail, both extensions, initial state
+    (1, 520, 160, 2, False, True, False, "f32", I.F32),  # rotation only, chunk-crossing blocks
+    (2, 256, 80, 8, True, True, True, "bf16", I.BF16),   # bf16 y and state
+])
+def test_mamba3_one_scan_head_pair_form(b, L, H, G, use_lam, use_theta, with_init, y_dtype, state):
+    """148 or more heads: one head-pair scan takes the turned operands as hi/lo
+    pairs (three products per contraction) and the trapezoid's diagonal
+    correction in its epilogue."""
+    y, fs, y_ref, fs_ref = run_case(b, L, H, 64, 128, G, 256 if L > 300 else 128, I.BF16, use_lam, use_theta,
+                                    with_init, y_dtype=y_dtype, state=state)
+    if y_dtype == "bf16":
+        assert bf16_excess_metric(y, y_ref) <= TOL_BF16
+        assert bf16_excess_metric(fs, fs_ref) <= TOL_BF16
+    else:
+        # the three products keep about 16 bits of the turned operands: far inside the bf16 bound
+        assert metric(y, y_ref) <= 1e-3
+        assert metric(fs, fs_ref) <= 1e-3
 
 
 def test_mamba3_long_sequences_cut_into_runs():
