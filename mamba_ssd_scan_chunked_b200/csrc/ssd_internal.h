@@ -106,9 +106,12 @@ bool pair_path_supports(int64_t batch, int64_t H, int64_t P, int64_t N, int64_t 
 cudaError_t launch_prefill_pair(const PrefillArgs& a, cudaStream_t s);
 // its Mamba-3 form: B, C are the turned operands as [b][L][G][2][N] bf16 (hi, lo),
 // dt and the cumsum slots of the workspace hold the trapezoid's weights and the
-// decay cumsum, dxc [BH][Lpad] the diagonal correction (or NULL); the initial
-// state is read as bf16 when init_bf16, the final one written per a.state_bf16
-cudaError_t launch_prefill_pair_mamba3(const PrefillArgs& a, const float* dxc, bool init_bf16, cudaStream_t s);
+// decay cumsum, dgw [BH][Lpad] the weight of each token's own term (or NULL: the
+// scan weight), rot [b][G][N/2] cos, sin of the last token's angle (the final
+// state is turned back by it as it is written); the initial state is read as
+// bf16 when init_bf16, the final one written per a.state_bf16
+cudaError_t launch_prefill_pair_mamba3(const PrefillArgs& a, const float* dgw, const float2* rot, bool init_bf16,
+                                       cudaStream_t s);
 
 // Backward pass of the prefill (ssd_backward.cu).  Workspace carve-up, all
 // offsets 256-byte aligned; "slice" strides separate the column slices of the
@@ -177,7 +180,7 @@ struct Mamba3Layout {
                                    // fused: [b][L][G][2][N], hi then lo per group)
     size_t off_Btl, off_Ctl;       // bf16 inputs: the lo part of the same (unused when fused)
     size_t off_csum;               // fp64 [b][G][nchunks][N/2] angle sums per chunk
-    size_t off_thL;                // fp64 [b][G][N/2] angle at the last token
+    size_t off_rotL;               // float2 [b][G][N/2] cos, sin of the angle at the last token
     size_t off_y32[3];             // fp32 [b][L][H][P] scan outputs before the combination
     size_t off_fsr;                // state dtype [b][H][N][P] rotated-frame final state (scan 1)
     size_t off_fsr2;               // fp32 [b][H][N][P] the same of the B_lo scan

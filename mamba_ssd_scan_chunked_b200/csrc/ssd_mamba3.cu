@@ -58,7 +58,7 @@ Mamba3Layout mamba3_layout(int64_t batch, int64_t L, int64_t H, int64_t P, int64
     l.off_Btl = io_bf16 ? l.off_Bt + opb : 0;
     l.off_Ctl = io_bf16 ? l.off_Ct + opb : 0;
     l.off_csum = take(sizeof(double) * (size_t)batch * G * s.nchunks * (N / 2));
-    l.off_thL = take(sizeof(double) * (size_t)batch * G * (N / 2));
+    l.off_rotL = take(sizeof(float2) * (size_t)batch * G * (N / 2));
     // fp32 scan outputs before the combination: three for the split scans, one
     // otherwise (the fused form writes y itself; lam without theta still combines)
     for (int i = 0; i < 3; ++i) l.off_y32[i] = (i == 0 || !l.fused) ? take(sizeof(float) * tok * H * P) : 0;
@@ -98,6 +98,51 @@ m3_angle_sums_kernel(const float* __restrict__ theta, double* __restrict__ csum,
     }
 }
 
+// The same sums with dstate a multiple of 8: block = (b, g, chunk, 4 pairs),
+// thread = token (one 16-byte load of its 4 angles), a block reduction.
+__global__ void __launch_bounds__(256)
+m3_angle_sums4_kernel(const float* __restrict__ theta, double* __restrict__ csum, int64_t L, int G, int K, int Q,
+                      int nchunks, int KG) {
+    __shared__ double wsum[8][4];
+    const int kg = (int)(blockIdx.x % (unsigned)KG);
+    const int64_t rest = blockIdx.x / (unsigned)KG;
+    const int c = (int)(rest % nchunks);
+    const int64_t bg = rest / nchunks;
+    const int g = (int)(bg % G);
+    const int64_t b = bg / G;
+    const int l = threadIdx.x, lane = l & 31, warp = l >> 5;
+    const int64_t t = (int64_t)c * Q + l;
+    double v[4] = {0.0, 0.0, 0.0, 0.0};
+    if (l < Q && t < L) {
+        const float4 a = *reinterpret_cast<const float4*>(theta + ((b * L + t) * G + g) * K + 4 * kg);
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+        for (int o = 16; o > 0; o >>= 1) v[q] += __shfl_xor_sync(0xffffffffu, v[q], o);
+    if (lane == 0)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) wsum[warp][q] = v[q];
+    __syncthreads();
+    if (l < 4) {
+        double tot = 0.0;
+        for (int w = 0; w < (int)(blockDim.x >> 5); ++w) tot += wsum[w][l];
+        csum[(bg * nchunks + c) * K + 4 * kg + l] = tot;
+    }
+}
+
+// 8 consecutive operand values (16-byte aligned) to fp32 and back
+__device__ __forceinline__ void ld8(const bf16* p, float* o) { Vec16<bf16>::load(p, o); }
+__device__ __forceinline__ void ld8(const float* p, float* o) {
+    Vec16<float>::load(p, o);
+    Vec16<float>::load(p + 4, o + 4);
+}
+__device__ __forceinline__ void st8(bf16* p, const float* v) { Vec16<bf16>::store(p, v); }
+__device__ __forceinline__ void st8(float* p, const float* v) {
+    Vec16<float>::store(p, v);
+    Vec16<float>::store(p + 4, v + 4);
+}
+
 // ~B = R(-Theta_t) B, ~C = R(-Theta_t) C.  Block = (b, g, chunk, 4 pairs),
 // thread = token: the cumulative angle is the previous chunks' sums (warp 0,
 // lanes over chunks) plus a block scan over the chunk's tokens, in float64.
@@ -106,7 +151,7 @@ template <typename IoT>
 __global__ void __launch_bounds__(256)
 m3_rotate_kernel(const IoT* __restrict__ B, const IoT* __restrict__ C, const float* __restrict__ theta,
                  const double* __restrict__ csum, IoT* __restrict__ Bt, IoT* __restrict__ Ct, IoT* __restrict__ Btl,
-                 IoT* __restrict__ Ctl, double* __restrict__ thL, int64_t L, int G, int N, int Q, int nchunks,
+                 IoT* __restrict__ Ctl, float2* __restrict__ rotL, int64_t L, int G, int N, int Q, int nchunks,
                  int KG, int ostride) {
     __shared__ double wtot[8][4];
     __shared__ double carry[4];
@@ -133,10 +178,16 @@ m3_rotate_kernel(const IoT* __restrict__ B, const IoT* __restrict__ C, const flo
 #pragma unroll
             for (int q = 0; q < 4; ++q) carry[q] = cv[q];
     }
-    double v[4];
+    const bool vec = (N & 7) == 0;            // 4 whole pairs: 16-byte loads and stores
+    double v[4] = {0.0, 0.0, 0.0, 0.0};
+    if (vec && live) {
+        const float4 a = *reinterpret_cast<const float4*>(theta + ((b * L + t) * G + g) * K + k0);
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    } else if (!vec) {
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
-        v[q] = (live && k0 + q < K) ? (double)theta[((b * L + t) * G + g) * K + k0 + q] : 0.0;
+        for (int q = 0; q < 4; ++q)
+            v[q] = (live && k0 + q < K) ? (double)theta[((b * L + t) * G + g) * K + k0 + q] : 0.0;
+    }
     for (int o = 1; o < 32; o <<= 1) {
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
@@ -156,6 +207,34 @@ m3_rotate_kernel(const IoT* __restrict__ B, const IoT* __restrict__ C, const flo
     if (!live) return;
     const int64_t row = ((b * L + t) * G + g) * N;
     const int64_t orow = ((b * L + t) * G + g) * ostride;     // N, or 2N with hi and lo interleaved
+    if (vec) {
+        const int n0 = 2 * k0;
+        float bv[8], cv[8], r[2][8];
+        ld8(B + row + n0, bv);
+        ld8(C + row + n0, cv);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            double sd, cd;
+            sincos(v[q], &sd, &cd);
+            const float cs = (float)cd, sn = (float)sd;
+            r[0][2 * q] = cs * bv[2 * q] + sn * bv[2 * q + 1];
+            r[0][2 * q + 1] = cs * bv[2 * q + 1] - sn * bv[2 * q];
+            r[1][2 * q] = cs * cv[2 * q] + sn * cv[2 * q + 1];
+            r[1][2 * q + 1] = cs * cv[2 * q + 1] - sn * cv[2 * q];
+            if (t == L - 1) rotL[bg * K + k0 + q] = make_float2(cs, sn);
+        }
+        st8(Bt + orow + n0, r[0]);
+        st8(Ct + orow + n0, r[1]);
+        if (Btl) {
+#pragma unroll
+            for (int i = 0; i < 2; ++i)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) r[i][e] -= to_f32(from_f32<IoT>(r[i][e]));
+            st8(Btl + orow + n0, r[0]);
+            st8(Ctl + orow + n0, r[1]);
+        }
+        return;
+    }
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
         if (k0 + q >= K) break;
@@ -175,15 +254,15 @@ m3_rotate_kernel(const IoT* __restrict__ B, const IoT* __restrict__ C, const flo
             *dst[i] = hi;
             if (Btl) *dlo[i] = from_f32<IoT>(r[i] - to_f32(hi));
         }
-        if (t == L - 1) thL[bg * K + k0 + q] = v[q];
+        if (t == L - 1) rotL[bg * K + k0 + q] = make_float2(cs, sn);
     }
 }
 
 // Scan weights w, chunk-local decay cumsum and the diagonal correction's
 // coefficient c, as the forward's decay kernel lays them out ([b*H][Lpad]);
 // also clears the scan's hand-off flags.  Block = (b, chunk, 8 heads), thread =
-// token.  With B and C given (the fused form) the correction is written whole,
-// c_t (C_t . B_t), the dot product of the head's group formed by the thread.
+// token.  With diag_w (the fused form) the third output is instead the weight of
+// a token's own term, lam_t dt_t = w_t - c_t.
 constexpr int M3_HG = 8;
 
 template <typename IoT>
@@ -191,8 +270,7 @@ __global__ void __launch_bounds__(256)
 m3_decay_kernel(const IoT* __restrict__ dt_raw, const float* __restrict__ dt_bias, const float* __restrict__ A,
                 const float* __restrict__ lam, float* __restrict__ w_out, float* __restrict__ acs_out,
                 float* __restrict__ corr_out, int* __restrict__ flags, int64_t L, int64_t Lpad, int H, int Q,
-                int nflags, int nchunks, int hgroups, const IoT* __restrict__ Bcb, const IoT* __restrict__ Ccb,
-                int G, int N) {
+                int nflags, int nchunks, int hgroups, int diag_w) {
     __shared__ float warp_tot[8][M3_HG];
     const int hg = (int)(blockIdx.x % (unsigned)hgroups);
     const int c = (int)((blockIdx.x / (unsigned)hgroups) % (unsigned)nchunks);
@@ -220,33 +298,7 @@ m3_decay_kernel(const IoT* __restrict__ dt_raw, const float* __restrict__ dt_bia
         cr[k] = (1.f - lmn) * dtn;            // 0 without lam, at the last token and past it
         w[k] = lm * dt + cr[k];
         v[k] = h < H ? dt * A[h] : 0.f;
-    }
-    if (Bcb && live) {
-        int gprev = -1;
-        float cb = 0.f;
-        const int hpg = H / G;
-#pragma unroll
-        for (int k = 0; k < M3_HG; ++k) {
-            const int h = h0 + k;
-            if (h >= H) break;
-            if (h / hpg != gprev) {
-                gprev = h / hpg;
-                const int64_t grow = ((b * L + t) * G + gprev) * N;
-                cb = 0.f;
-                if (sizeof(IoT) == 2 && (N & 7) == 0) {    // 16-byte rows of 8 bf16 (the arrays are 16-byte aligned)
-                    for (int n = 0; n < N; n += 8) {
-                        float cv[8], bv[8];
-                        Vec16<bf16>::load(reinterpret_cast<const bf16*>(Ccb + grow + n), cv);
-                        Vec16<bf16>::load(reinterpret_cast<const bf16*>(Bcb + grow + n), bv);
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) cb += cv[i] * bv[i];
-                    }
-                } else {
-                    for (int n = 0; n < N; ++n) cb += to_f32(Ccb[grow + n]) * to_f32(Bcb[grow + n]);
-                }
-            }
-            cr[k] *= cb;
-        }
+        if (diag_w) cr[k] = lm * dt;
     }
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -343,30 +395,28 @@ m3_combine_kernel(const float* y1, const float* __restrict__ y2, const float* __
 }
 
 // h_{L-1} = R(Theta_{L-1}) ~S_{L-1}: rows (2k, 2k+1) of every head of group g;
-// ~S_{L-1} = src (+ src2, the B_lo scan's final state, when split).
+// ~S_{L-1} = src (+ src2, the B_lo scan's final state, when split).  Block =
+// (b, h); rotL holds cos, sin of the last token's angle per (b, g, pair).
 template <typename SrcT, typename StateT>
 __global__ void __launch_bounds__(256)
 m3_unrotate_state_kernel(const SrcT* __restrict__ src, const float* __restrict__ src2,
-                         const double* __restrict__ thL, StateT* __restrict__ dst, int64_t batch, int H, int P, int N,
-                         int G) {
+                         const float2* __restrict__ rotL, StateT* __restrict__ dst, int H, int P, int N, int G) {
     const int K = N / 2, hpg = H / G;
-    const int64_t n_all = batch * H * K * P;
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n_all; i += (int64_t)gridDim.x * blockDim.x) {
-        const int p = (int)(i % P);
-        const int k = (int)((i / P) % K);
-        const int64_t bh = i / ((int64_t)K * P);
-        const int h = (int)(bh % H);
-        const int64_t b = bh / H;
-        double sd, cd;
-        sincos(thL[(b * G + h / hpg) * K + k], &sd, &cd);
+    const int64_t bh = blockIdx.x;
+    const int h = (int)(bh % H);
+    const int64_t b = bh / H;
+    const float2* rr = rotL + (b * G + h / hpg) * K;
+    for (int i = threadIdx.x; i < K * P; i += blockDim.x) {
+        const int k = i / P, p = i - k * P;
+        const float2 cs = rr[k];
         const int64_t o0 = (bh * N + 2 * k) * P + p, o1 = o0 + P;
         float u = to_f32(src[o0]), v = to_f32(src[o1]);
         if (src2) {
             u += src2[o0];
             v += src2[o1];
         }
-        dst[o0] = from_f32<StateT>((float)cd * u - (float)sd * v);
-        dst[o1] = from_f32<StateT>((float)sd * u + (float)cd * v);
+        dst[o0] = from_f32<StateT>(cs.x * u - cs.y * v);
+        dst[o1] = from_f32<StateT>(cs.y * u + cs.x * v);
     }
 }
 
@@ -395,14 +445,18 @@ static cudaError_t mamba3_t(const Mamba3Args& a, cudaStream_t s) {
     const bool fused = split && l.fused;
     IoT* Btl = split ? (fused ? Bt + N : (IoT*)(ws + l.off_Btl)) : nullptr;
     IoT* Ctl = split ? (fused ? Ct + N : (IoT*)(ws + l.off_Ctl)) : nullptr;
-    double* thL = (double*)(ws + l.off_thL);
+    float2* rotL = (float2*)(ws + l.off_rotL);
     if (a.theta) {
-        m3_angle_sums_kernel<<<(unsigned)(a.batch * G * nchunks), 1024, 0, s>>>(
-            a.theta, (double*)(ws + l.off_csum), a.L, G, K, Q, nchunks);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
         const int KG = (K + 3) / 4;
+        if ((N & 7) == 0)
+            m3_angle_sums4_kernel<<<(unsigned)(a.batch * G * nchunks * KG), (unsigned)(Q < 32 ? 32 : Q), 0, s>>>(
+                a.theta, (double*)(ws + l.off_csum), a.L, G, K, Q, nchunks, KG);
+        else
+            m3_angle_sums_kernel<<<(unsigned)(a.batch * G * nchunks), 1024, 0, s>>>(
+                a.theta, (double*)(ws + l.off_csum), a.L, G, K, Q, nchunks);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
         m3_rotate_kernel<IoT><<<(unsigned)(a.batch * G * nchunks * KG), (unsigned)(Q < 32 ? 32 : Q), 0, s>>>(
-            (const IoT*)a.B, (const IoT*)a.C, a.theta, (const double*)(ws + l.off_csum), Bt, Ct, Btl, Ctl, thL, a.L,
+            (const IoT*)a.B, (const IoT*)a.C, a.theta, (const double*)(ws + l.off_csum), Bt, Ct, Btl, Ctl, rotL, a.L,
             G, N, Q, nchunks, KG, fused ? 2 * N : N);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
@@ -411,34 +465,23 @@ static cudaError_t mamba3_t(const Mamba3Args& a, cudaStream_t s) {
         m3_decay_kernel<IoT><<<(unsigned)(a.batch * nchunks * hgroups), (unsigned)(Q < 32 ? 32 : Q), 0, s>>>(
             (const IoT*)a.dt_raw, a.dt_bias, a.A, a.lam, (float*)(ws + l.scan.off_dt), (float*)(ws + l.scan.off_acs),
             (float*)(ws + l.off_corr), (int*)(ws + l.scan.off_flags), a.L, l.scan.Lpad, H, Q, nflags, nchunks,
-            hgroups, fused && a.lam ? (const IoT*)a.B : nullptr, fused && a.lam ? (const IoT*)a.C : nullptr, G, N);
+            hgroups, fused ? 1 : 0);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     if (fused) {
         // one scan: the head-pair kernel's Mamba-3 form writes y (with D and the
-        // correction) and the turned final state in fp32 (rounded to the state
-        // dtype once, when turned back); the initial state enters the turned frame
+        // trapezoid's own-token weights lam dt) and the final state, turned back
+        // from fp32 as it is stored; the initial state enters the turned frame
         // unchanged (no angle before the first token)
         PrefillArgs p{};
         p.batch = a.batch; p.L = a.L; p.H = a.H; p.P = a.P; p.N = a.N; p.G = a.G; p.Q = a.Q;
-        p.io_bf16 = true; p.y_bf16 = a.y_bf16; p.state_bf16 = false;
+        p.io_bf16 = true; p.y_bf16 = a.y_bf16; p.state_bf16 = a.state_bf16;
         p.x = a.x; p.dt_raw = a.dt_raw; p.dt_bias = a.dt_bias; p.A = a.A;
         p.B = Bt; p.C = Ct; p.D = a.D;
-        p.init_state = a.init_state; p.y = a.y; p.final_state = a.final_state ? (void*)(ws + l.off_fsr) : nullptr;
+        p.init_state = a.init_state; p.y = a.y; p.final_state = a.final_state;
         p.ws = ws; p.lay = l.scan; p.pad_left = nullptr; p.dev_err = a.dev_err; p.drop_publish = 0;
-        e = launch_prefill_pair_mamba3(p, a.lam ? (const float*)(ws + l.off_corr) : nullptr, a.state_bf16, s);
-        if (e != cudaSuccess) return e;
-        if (a.final_state) {
-            const unsigned grid = m3_grid(a.batch * H * K * P, 256);
-            if (a.state_bf16)
-                m3_unrotate_state_kernel<float, bf16><<<grid, 256, 0, s>>>(
-                    (const float*)(ws + l.off_fsr), nullptr, thL, (bf16*)a.final_state, a.batch, H, P, N, G);
-            else
-                m3_unrotate_state_kernel<float, float><<<grid, 256, 0, s>>>(
-                    (const float*)(ws + l.off_fsr), nullptr, thL, (float*)a.final_state, a.batch, H, P, N, G);
-            if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        }
-        return cudaSuccess;
+        return launch_prefill_pair_mamba3(p, a.lam ? (const float*)(ws + l.off_corr) : nullptr, rotL, a.state_bf16,
+                                          s);
     }
     // the scans: with lam or the split the outputs are combined (and corrected)
     // afterwards from fp32; with theta the final state is rotated back afterwards
@@ -492,14 +535,14 @@ static cudaError_t mamba3_t(const Mamba3Args& a, cudaStream_t s) {
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     if (unrotate) {
-        const unsigned grid = m3_grid(a.batch * H * K * P, 256);
+        const unsigned grid = (unsigned)(a.batch * H);
         const float* src2 = split ? (const float*)(ws + l.off_fsr2) : nullptr;
         if (a.state_bf16)
-            m3_unrotate_state_kernel<bf16, bf16><<<grid, 256, 0, s>>>((const bf16*)(ws + l.off_fsr), src2, thL,
-                                                               (bf16*)a.final_state, a.batch, H, P, N, G);
+            m3_unrotate_state_kernel<bf16, bf16><<<grid, 256, 0, s>>>((const bf16*)(ws + l.off_fsr), src2, rotL,
+                                                                     (bf16*)a.final_state, H, P, N, G);
         else
-            m3_unrotate_state_kernel<float, float><<<grid, 256, 0, s>>>((const float*)(ws + l.off_fsr), src2, thL,
-                                                                (float*)a.final_state, a.batch, H, P, N, G);
+            m3_unrotate_state_kernel<float, float><<<grid, 256, 0, s>>>((const float*)(ws + l.off_fsr), src2, rotL,
+                                                                      (float*)a.final_state, H, P, N, G);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     return cudaSuccess;
@@ -512,8 +555,8 @@ cudaError_t launch_mamba3(const Mamba3Args& a, cudaStream_t s) {
 int mamba3_launches(bool tc, bool io_bf16, bool has_lam, bool has_theta, bool has_final, bool fused) {
     const int scan = tc ? 1 : 3;
     const bool split = has_theta && io_bf16;
-    // the fused form: angle sums, rotation, weights, the head-pair scan, the final state turned back
-    if (split && fused) return 4 + (has_final ? 1 : 0);
+    // the fused form: angle sums, rotation, weights, the head-pair scan (which turns the final state back)
+    if (split && fused) return 4;
     return (has_theta ? 2 : 0) + 1 + scan + (split ? 2 * (1 + scan) : 0) + ((has_lam || split) ? 1 : 0) +
            ((has_theta && has_final) ? 1 : 0);
 }

@@ -52,9 +52,10 @@
 // operand tiles fill both C/B stages, so there is one stage: C of the next
 // block is loaded once C h is done, B once the state MMAs are, and y goes
 // from the registers straight to global memory instead of through a staging
-// tile.  The epilogue also takes the trapezoid's diagonal correction,
-// y = Y + (D - c_t) x with c_t = (1 - lam_{t+1}) dt_{t+1} (C_t . B_t) per
-// token and head, from the workspace.
+// tile.  The trapezoid's weights w_s stand where dt_s stands in the forward;
+// a token's own term takes lam_t dt_t instead (the diagonal of M, with the
+// exact C_t . B_t of S's diagonal), and the final state is turned back by the
+// last token's angle as it is written (rows 2k, 2k+1 are lanes of one warp).
 #include "ssd_internal.h"
 #include "ssd_tc_common.cuh"
 
@@ -102,13 +103,15 @@ struct Params {
     unsigned* dev_err;
     long long Lpad;
     int H, G, Q, nblk, npairs;
-    int state_bf16, y_bf16;
-    // the Mamba-3 form only
-    const float* dxc;          // [BH][Lpad] diagonal correction c_t, or NULL (= 0)
+    int state_bf16, y_bf16;    // Mamba-3 form: state_bf16 bit 0 the final state's dtype, bit 1 the initial one's
+    // the Mamba-3 form only (the struct stays within 128 bytes: a larger one costs
+    // the kernel registers)
+    const float* dgw;          // [BH][Lpad] weight of a token's own term (lam dt), or NULL (= the scan weight)
+    const float2* rot;         // [b][G][NS/2] cos, sin of the last token's angle per pair
     void* y;                   // [b][L][H][PD] y dtype
-    long long L;
-    int init_bf16;             // the initial state's dtype (the final state's is state_bf16)
+    int L;
 };
+static_assert(sizeof(Params) <= 128, "kernel parameter struct");
 
 // bounded wait that gives up at once when another wait of the CTA has given up
 __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, volatile int* abort) {
@@ -436,7 +439,7 @@ ssd_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                 } else if (p.init_state) {
                     float f[16];
                     const long long o = ((bh + k) * NS + row) * PD + 16 * kq;
-                    if (M3 ? p.init_bf16 : p.state_bf16) {
+                    if (M3 ? (p.state_bf16 & 2) : p.state_bf16) {
                         Vec16<bf16>::load(reinterpret_cast<const bf16*>(p.init_state) + o, f);
                         Vec16<bf16>::load(reinterpret_cast<const bf16*>(p.init_state) + o + 8, f + 8);
                     } else {
@@ -481,16 +484,16 @@ ssd_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
         // this thread's per-token data of a block, read from the workspace one block
         // ahead: the cumsum of its row's token for both heads; for the table threads
         // (kq < 2: head kq, token = row) also dt and the cumsum of the token before
-        // (Mamba-3 form: also the diagonal correction of its row's token for both heads)
-        struct Pre { float2 row[2]; float dt; float2 prev; float dx[M3 ? 2 : 1]; };
+        // (Mamba-3 form: also the weight of its row's own term for both heads)
+        struct Pre { float2 row[2]; float dt; float2 prev; float dg[M3 ? 2 : 1]; };
         auto fetch = [&](const Item& dd, int jb, Pre& r) {
             const long long bh = (long long)dd.b * p.H + dd.h0;
             const long long t = (long long)jb * SUB + row;
             r.row[0] = cum(bh, t);
             r.row[1] = cum(bh + 1, t);
-            if (M3) {
-                r.dx[0] = p.dxc ? __ldcg(p.dxc + bh * p.Lpad + t) : 0.f;
-                r.dx[M3 ? 1 : 0] = p.dxc ? __ldcg(p.dxc + (bh + 1) * p.Lpad + t) : 0.f;
+            if (M3 && p.dgw) {
+                r.dg[0] = __ldcg(p.dgw + bh * p.Lpad + t);
+                r.dg[M3 ? 1 : 0] = __ldcg(p.dgw + (bh + 1) * p.Lpad + t);
             }
             if (kq < 2) {
                 r.dt = __ldcg(p.dtw + (bh + kq) * p.Lpad + t);
@@ -623,6 +626,12 @@ ssd_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
 #pragma unroll
                             for (int t = 0; t < 4; ++t)
                                 e[t] = ex2((int)c0 + 4 * i4 + t <= row ? lf + ub[t] : NEG_INF);
+                            if (M3 && p.dgw) {
+                                // the row's own token: lam dt in place of the scan weight
+#pragma unroll
+                                for (int t = 0; t < 4; ++t)
+                                    if ((int)c0 + 4 * i4 + t == row) e[t] = cur.dg[M3 ? k : 0];
+                            }
                             split2(f2_mul(f2_pack_u(v[4 * i4], v[4 * i4 + 1]), f2_pack(e[0], e[1])),
                                    o[2 * i4], o[8 + 2 * i4]);
                             split2(f2_mul(f2_pack_u(v[4 * i4 + 2], v[4 * i4 + 3]), f2_pack(e[2], e[3])),
@@ -689,13 +698,24 @@ ssd_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                 tmem_ld16(tmem + lo16 + COL_ST + 16 * kq, sv[0]);
                 tmem_ld16(tmem + lo16 + COL_ST + 64 + 16 * kq, sv[1]);
                 tmem_wait_ld();
+                float2 cs = make_float2(1.f, 0.f);
+                if (M3) cs = p.rot[((long long)d.b * p.G + d.g) * (NS / 2) + (row >> 1)];
 #pragma unroll
                 for (int k = 0; k < 2; ++k) {
                     float ho[16];
 #pragma unroll
                     for (int i = 0; i < 16; ++i) ho[i] = __uint_as_float(sv[k][i]);
+                    if (M3) {
+                        // h = R(Theta_last) ~h: row 2k' -> c u - s w, row 2k'+1 -> s u + c w
+                        // (u, w the rows 2k', 2k'+1 of the turned state: this lane and its neighbour)
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const float other = __shfl_xor_sync(0xffffffffu, ho[i], 1);
+                            ho[i] = (row & 1) ? fmaf(cs.y, other, cs.x * ho[i]) : fmaf(-cs.y, other, cs.x * ho[i]);
+                        }
+                    }
                     const long long o = ((bh0 + k) * NS + row) * PD + 16 * kq;
-                    if (p.state_bf16) {
+                    if (M3 ? (p.state_bf16 & 1) : p.state_bf16) {
                         bf16* fs = reinterpret_cast<bf16*>(p.final_state) + o;
                         Vec16<bf16>::store(fs, ho);
                         Vec16<bf16>::store(fs + 8, ho + 8);
@@ -731,8 +751,7 @@ ssd_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
 #pragma unroll
                     for (int k = 0; k < 2; ++k) {
                         float out[16];
-                        const float dk = Dk[k] - cur.dx[M3 ? k : 0];
-                        const f32x2 dd = f2_pack(dk, dk);
+                        const f32x2 dd = f2_pack(Dk[k], Dk[k]);
 #pragma unroll
                         for (int e = 0; e < 8; ++e)
                             f2_unpack(f2_fma(dd, bf16x2_to_f2(xr[k][e]), f2_pack_u(yv[k][2 * e], yv[k][2 * e + 1])),
@@ -814,7 +833,8 @@ bool pair_path_supports(int64_t batch, int64_t H, int64_t P, int64_t N, int64_t 
 }
 
 // m3: the Mamba-3 form, B and C then [b][L][G][2][N] (hi, lo of the turned operands)
-static cudaError_t launch_pair(const PrefillArgs& a, bool m3, const float* dxc, bool init_bf16, cudaStream_t s) {
+static cudaError_t launch_pair(const PrefillArgs& a, bool m3, const float* dgw, const float2* rot, bool init_bf16,
+                               cudaStream_t s) {
     using namespace pair;
     if (!pair_path_supports(a.batch, a.H, a.P, a.N, a.G, a.Q, a.io_bf16)) return cudaErrorNotSupported;
     CUtensorMap mx, mb, mc, my;
@@ -859,12 +879,13 @@ static cudaError_t launch_pair(const PrefillArgs& a, bool m3, const float* dxc, 
     const long long blocks = pairs * p.nblk;
     if (pairs > 0x7fffffffLL || blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
     p.npairs = (int)pairs;
-    p.state_bf16 = a.state_bf16;
+    p.state_bf16 = m3 ? (a.state_bf16 ? 1 : 0) | (init_bf16 ? 2 : 0) : a.state_bf16;
     p.y_bf16 = a.y_bf16;
-    p.dxc = dxc;
+    p.dgw = dgw;
+    p.rot = rot;
     p.y = a.y;
-    p.L = a.L;
-    p.init_bf16 = init_bf16;
+    if (a.L > 0x7fffffffLL) return cudaErrorInvalidValue;
+    p.L = (int)a.L;
     const unsigned grid = (unsigned)(pairs < sms_of[dev][m3] ? pairs : sms_of[dev][m3]);
     // a programmatic dependent of the decay-cumsum kernel before it on the stream:
     // the prologue and the first operand loads overlap that kernel; the producer
@@ -884,11 +905,13 @@ static cudaError_t launch_pair(const PrefillArgs& a, bool m3, const float* dxc, 
 }
 
 cudaError_t launch_prefill_pair(const PrefillArgs& a, cudaStream_t s) {
-    return launch_pair(a, false, nullptr, a.state_bf16, s);
+    return launch_pair(a, false, nullptr, nullptr, a.state_bf16, s);
 }
 
-cudaError_t launch_prefill_pair_mamba3(const PrefillArgs& a, const float* dxc, bool init_bf16, cudaStream_t s) {
-    return launch_pair(a, true, dxc, init_bf16, s);
+cudaError_t launch_prefill_pair_mamba3(const PrefillArgs& a, const float* dgw, const float2* rot, bool init_bf16,
+                                       cudaStream_t s) {
+    if (a.final_state && !rot) return cudaErrorInvalidValue;
+    return launch_pair(a, true, dgw, rot, init_bf16, s);
 }
 
 }  // namespace ssd

@@ -333,11 +333,11 @@ def test_mamba3_workspace_launches_and_validation():
     assert ssd.ssd_chunk_scan_mamba3_launches(d, False, False, True) == 2       # the plain forward
     assert ssd.ssd_chunk_scan_mamba3_launches(desc(io_dtype=ssd.SSD_F32), True, True, True) == 8
     # 148 or more heads in all: the head-pair kernel's Mamba-3 form takes the three
-    # products and the correction in one scan (angle sums, rotation, weights, the
-    # scan, the final-state rotation)
+    # products and the trapezoid's own-token weights in one scan, and turns the
+    # final state back as it stores it (angle sums, rotation, weights, the scan)
     dp = desc(nheads=80, ngroups=4)
     assert ssd.ssd_chunk_scan_path(dp) == 2
-    assert ssd.ssd_chunk_scan_mamba3_launches(dp, True, True, True) == 5
+    assert ssd.ssd_chunk_scan_mamba3_launches(dp, True, True, True) == 4
     assert ssd.ssd_chunk_scan_mamba3_launches(dp, False, True, False) == 4
     assert ssd.ssd_chunk_scan_mamba3_launches(dp, True, False, True) == 3
 
