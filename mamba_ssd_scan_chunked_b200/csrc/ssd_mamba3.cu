@@ -280,25 +280,65 @@ m3_decay_kernel(const IoT* __restrict__ dt_raw, const float* __restrict__ dt_bia
     const int64_t t = (int64_t)c * Q + l;
     const bool live = l < Q && t < L, next = l < Q && t + 1 < L;
     float v[M3_HG], w[M3_HG], cr[M3_HG];
+    // dt and lam of this token for the block's heads (16-byte loads when the 8 heads
+    // are whole and aligned), then those of the next token from the next thread;
+    // the last thread of a warp or of the chunk reads the next token itself
+    auto load8 = [&](int64_t tt, float (&dtv)[M3_HG], float (&lmv)[M3_HG]) {
+        const bool whole = (H & 7) == 0;
+        if (whole) {
+            float raw[M3_HG];
+            if (sizeof(IoT) == 2) {
+                Vec16<bf16>::load(reinterpret_cast<const bf16*>(dt_raw) + (b * L + tt) * H + h0, raw);
+            } else {
+                Vec16<float>::load(reinterpret_cast<const float*>(dt_raw) + (b * L + tt) * H + h0, raw);
+                Vec16<float>::load(reinterpret_cast<const float*>(dt_raw) + (b * L + tt) * H + h0 + 4, raw + 4);
+            }
+            if (lam) {
+                Vec16<float>::load(lam + (b * L + tt) * H + h0, lmv);
+                Vec16<float>::load(lam + (b * L + tt) * H + h0 + 4, lmv + 4);
+            }
+#pragma unroll
+            for (int k = 0; k < M3_HG; ++k) {
+                dtv[k] = softplus_f32(raw[k] + (dt_bias ? dt_bias[h0 + k] : 0.f));
+                if (!lam) lmv[k] = 1.f;
+            }
+        } else {
+#pragma unroll
+            for (int k = 0; k < M3_HG; ++k) {
+                const int h = h0 + k;
+                dtv[k] = 0.f;
+                lmv[k] = 1.f;
+                if (h < H) {
+                    dtv[k] = softplus_f32(to_f32(dt_raw[(b * L + tt) * H + h]) + (dt_bias ? dt_bias[h] : 0.f));
+                    if (lam) lmv[k] = lam[(b * L + tt) * H + h];
+                }
+            }
+        }
+    };
+    float dt[M3_HG], lm[M3_HG], dtn[M3_HG], lmn[M3_HG];
+#pragma unroll
+    for (int k = 0; k < M3_HG; ++k) { dt[k] = 0.f; lm[k] = 1.f; dtn[k] = 0.f; lmn[k] = 1.f; }
+    if (live) load8(t, dt, lm);
+    const bool edge = lane == 31 || l == Q - 1;
+#pragma unroll
+    for (int k = 0; k < M3_HG; ++k) {
+        dtn[k] = __shfl_down_sync(0xffffffffu, dt[k], 1);
+        lmn[k] = __shfl_down_sync(0xffffffffu, lm[k], 1);
+    }
+    if (edge) {
+#pragma unroll
+        for (int k = 0; k < M3_HG; ++k) { dtn[k] = 0.f; lmn[k] = 1.f; }
+        if (next) load8(t + 1, dtn, lmn);
+    }
 #pragma unroll
     for (int k = 0; k < M3_HG; ++k) {
         const int h = h0 + k;
-        float dt = 0.f, dtn = 0.f, lm = 1.f, lmn = 1.f;
-        if (h < H) {
-            const float bias = dt_bias ? dt_bias[h] : 0.f;
-            if (live) {
-                dt = softplus_f32(to_f32(dt_raw[(b * L + t) * H + h]) + bias);
-                if (lam) lm = lam[(b * L + t) * H + h];
-            }
-            if (next && lam) {
-                dtn = softplus_f32(to_f32(dt_raw[(b * L + t + 1) * H + h]) + bias);
-                lmn = lam[(b * L + t + 1) * H + h];
-            }
-        }
-        cr[k] = (1.f - lmn) * dtn;            // 0 without lam, at the last token and past it
-        w[k] = lm * dt + cr[k];
-        v[k] = h < H ? dt * A[h] : 0.f;
-        if (diag_w) cr[k] = lm * dt;
+        if (h >= H) { dt[k] = 0.f; dtn[k] = 0.f; lm[k] = 1.f; lmn[k] = 1.f; }
+        if (!lam) { lm[k] = 1.f; lmn[k] = 1.f; }
+        cr[k] = (1.f - lmn[k]) * dtn[k];      // 0 without lam, at the last token and past it
+        w[k] = lm[k] * dt[k] + cr[k];
+        v[k] = h < H ? dt[k] * A[h] : 0.f;
+        if (diag_w) cr[k] = lm[k] * dt[k];
     }
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
