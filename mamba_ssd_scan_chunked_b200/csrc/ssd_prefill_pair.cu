@@ -27,9 +27,8 @@
 //
 // Roles (one CTA per SM, persistent over its items c, c + grid, ...):
 //   warps 0-15  compute: warp w works on TMEM lanes 32*(w%4).. (tile rows) and
-//               the 16-column part w/4 of the state, Yoff and output tiles;
-//               warps with w%4 < 2 also form w o X, since their share of the
-//               causal mask transform is the smaller one
+//               the 16-column part w/4 of the state, Yoff, x, w o X and
+//               output tiles (x is read from shared memory once, for w o X and D x)
 //   warp 16     MMA issue (one elected lane, converged warp)
 //   warp 17     TMA: operand loads (C, B double-buffered one block ahead), the
 //               y stores, which it stages in the C/B buffers of the block just
@@ -165,7 +164,7 @@ ssd_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
     }
     if (threadIdx.x == NCT) {
         //                          CB0 CB1 X  S  OFF ST Y0 Y  H    WX       M    EPI  STG0 STG1
-        const uint32_t cnt[NBAR] = {1, 1, 1, 1, 1, 1, 1, 1, NCT, NCT / 2, NCT, NCT, NCT, NCT};
+        const uint32_t cnt[NBAR] = {1, 1, 1, 1, 1, 1, 1, 1, NCT, M3 ? NCT / 2 : NCT, NCT, NCT, NCT, NCT};
         for (int i = 0; i < NBAR; ++i) mbar_init(bar(i), cnt[i]);
         *s_abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -501,11 +500,9 @@ ssd_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
             }
         };
 
-        // w o X into the W tiles (quarters 0 and 1: one token row of one head per
-        // thread), once C h has read them; the state MMAs wait for it
+        // Mamba-3 form (whose epilogue holds more registers): w o X by quarters 0 and 1,
+        // one token row of one head per thread, read from the x tiles
         auto do_wx = [&](uint32_t ph) {
-            wait(B_OFF, ph);
-            tc_fence_after();
             wait(B_X, ph);
             const int t = kq * 64 + q * 32 + lane;
             const int s_ = t & (SUB - 1), k = t >> 7;
@@ -537,7 +534,6 @@ ssd_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
             const uint32_t ph = jj & 1;
             const bool chunk_start = ((j * SUB) & (p.Q - 1)) == 0;   // the cumsum restarts at every chunk
             const long long bh0 = (long long)d.b * p.H + d.h0;
-            const float Dk[2] = {p.D ? p.D[d.h0] : 0.f, p.D ? p.D[d.h0 + 1] : 0.f};
             int it_n = it, j_n = j + 1;
             if (j_n == p.nblk) { j_n = 0; ++it_n; }
             const bool has_next = jj + 1 < total;
@@ -641,40 +637,13 @@ ssd_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                     tmem_st16(tmem + lo16 + (k ? COL_R1 : COL_R0) + c0, o);
                 }
             }
-            // the next block's per-token data, while this block's work goes on
-            Pre nxt{};
-            if (has_next) fetch(d_n, j_n, nxt);
-            float2 t127n[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-            if (has_next) {
-                t127n[0] = cum(bh0_n, (long long)j_n * SUB + SUB - 1);
-                t127n[1] = cum(bh0_n + 1, (long long)j_n * SUB + SUB - 1);
-            }
 
-            // ---- after C h: w o X into the W tiles (quarters 0 and 1), Yoff scaled by
-            // 2^(r_l), x kept for D x
+            // ---- after C h: w o X of this thread's row and 16 columns (both heads, from
+            // the x it keeps for D x) into the W tiles; then Yoff scaled by 2^(r_l)
             wait(B_OFF, ph);
             tc_fence_after();
-            if (q < 2) do_wx(ph);
-            {
-                uint32_t v[2][16];
-                tmem_ld16(tmem + lo16 + COL_Y + 16 * kq, v[0]);
-                tmem_ld16(tmem + lo16 + COL_Y + 64 + 16 * kq, v[1]);
-                tmem_wait_ld();
-#pragma unroll
-                for (int k = 0; k < 2; ++k) {
-                    const float el = ex2(rl[k]);
-                    const f32x2 e2 = f2_pack(el, el);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        float a, b;
-                        f2_unpack(f2_mul(e2, f2_pack_u(v[k][2 * i], v[k][2 * i + 1])), a, b);
-                        v[k][2 * i] = __float_as_uint(a);
-                        v[k][2 * i + 1] = __float_as_uint(b);
-                    }
-                    tmem_st16(tmem + lo16 + COL_Y + 64 * k + 16 * kq, v[k]);
-                }
-            }
-            if (q >= 2) wait(B_X, ph);
+            if (M3 && q < 2) do_wx(ph);
+            if (!M3 || q >= 2) wait(B_X, ph);
             uint32_t xr[2][8];
 #pragma unroll
             for (int k = 0; k < 2; ++k) {
@@ -684,9 +653,53 @@ ssd_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                     xr[k][4 * qq] = xv.x; xr[k][4 * qq + 1] = xv.y; xr[k][4 * qq + 2] = xv.z; xr[k][4 * qq + 3] = xv.w;
                 }
             }
+#pragma unroll
+            for (int k = 0; k < 2 && !M3; ++k) {
+                // w_s = 2^(r_last - r_s) dt_s for the row's token s
+                const float wv = ex2(dl2(s_ge[k * 8 + 7], s_ge[k * 8 + (row >> 4)]) + s_v[k * SUB + row]);
+                const f32x2 w2 = f2_pack(wv, wv);
+                uint8_t* wt = sm + OFF_W + k * 2 * TILE;
+#pragma unroll
+                for (int qq = 0; qq < 2; ++qq) {
+                    uint32_t hw[4], lw[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) split2(f2_mul(bf16x2_to_f2(xr[k][4 * qq + e]), w2), hw[e], lw[e]);
+                    const uint32_t o = swz(row, 2 * kq + qq);
+                    *reinterpret_cast<uint4*>(wt + o) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                    *reinterpret_cast<uint4*>(wt + TILE + o) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+                }
+            }
+            if (!M3) {
+                fence_proxy_async();
+                mbar_arrive(bar(B_WX));
+            }
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                uint32_t v[16];
+                tmem_ld16(tmem + lo16 + COL_Y + 64 * k + 16 * kq, v);
+                tmem_wait_ld();
+                const float el = ex2(rl[k]);
+                const f32x2 e2 = f2_pack(el, el);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    float a, b;
+                    f2_unpack(f2_mul(e2, f2_pack_u(v[2 * i], v[2 * i + 1])), a, b);
+                    v[2 * i] = __float_as_uint(a);
+                    v[2 * i + 1] = __float_as_uint(b);
+                }
+                tmem_st16(tmem + lo16 + COL_Y + 64 * k + 16 * kq, v);
+            }
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(bar(B_M));
+            // the next block's per-token data, while this block's MMAs run
+            Pre nxt{};
+            if (has_next) fetch(d_n, j_n, nxt);
+            float2 t127n[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+            if (has_next) {
+                t127n[0] = cum(bh0_n, (long long)j_n * SUB + SUB - 1);
+                t127n[1] = cum(bh0_n + 1, (long long)j_n * SUB + SUB - 1);
+            }
 
             // ---- once this block's state MMAs are done: the final state (last block of
             // an item), then the next block's entering state -- ahead of this block's
@@ -744,6 +757,7 @@ ssd_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(bar(B_EPI));          // the Y accumulators may be reused
+            const float Dk[2] = {p.D ? __ldg(p.D + d.h0) : 0.f, p.D ? __ldg(p.D + d.h0 + 1) : 0.f};
             if (M3) {
                 // y = Y + (D - c_t) x straight from the registers (16 columns of the row per head)
                 const long long t = (long long)j * SUB + row;
