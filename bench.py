@@ -856,8 +856,11 @@ def main():
                 "gpu_launches": 2 * args.steps,
                 "gpu_launches_other_legs": {"handoff_decode": dsh.steps, "decode": dsteps_timed,
                                             "replay": 2 * rsteps, "mimo": dsteps_timed,
-                                            "mamba3_decode": dsteps_timed, "mamba2_1p3b": 2 * c1_steps,
-                                            "backward": launches_per_bwd * bsteps, "mamba3": launches_per_m3 * m3steps},
+                                            "mamba3_decode": dsteps_timed, "mamba2_1p3b": 2 * c1_line["steps"],
+                                            "backward": (c1_line["backward"]["launches_per_step"] *
+                                                         c1_line["backward"]["steps"]),
+                                            "mamba3": (c1_line["mamba3"]["launches_per_step"] *
+                                                       c1_line["mamba3"]["steps"])},
                 "clocks": clk.summary()}
         print(json.dumps(line), flush=True)
     dist.finish(pg)

@@ -77,3 +77,30 @@ def test_handoff_prefill_bytes():
     bc, dt_raw = 2 * t * GG * N * 2, t * HH * 2
     final = bb * HH * N * P * 2          # bf16 state handed to the decode steps
     assert bench.prefill_bytes(bb, LL, HH, P, N, GG, 2, 4, 2) == x + y + bc + dt_raw + final
+
+
+def test_main_reads_no_name_bound_only_inside_the_layer_legs():
+    """bench.main() nests the 1.3B-layer legs in a function (so that --layer-only
+    can run them alone); a name bound only inside it is undefined outside, which
+    only a full GPU run would otherwise reveal."""
+    import ast
+    tree = ast.parse(open(bench.__file__).read())
+    main = next(n for n in tree.body if isinstance(n, ast.FunctionDef) and n.name == "main")
+    inner = next(n for n in ast.walk(main) if isinstance(n, ast.FunctionDef) and n.name == "layer_legs")
+    inner_ids = {id(n) for n in ast.walk(inner)}
+
+    def bound(nodes):
+        out = set()
+        for n in nodes:
+            if isinstance(n, ast.Name) and isinstance(n.ctx, ast.Store):
+                out.add(n.id)
+            elif isinstance(n, ast.arg):
+                out.add(n.arg)
+            elif isinstance(n, (ast.FunctionDef, ast.Import, ast.ImportFrom)):
+                out |= {n.name} if isinstance(n, ast.FunctionDef) else {a.asname or a.name for a in n.names}
+        return out
+
+    outer_nodes = [n for n in ast.walk(main) if id(n) not in inner_ids]
+    only_inner = bound(n for stmt in inner.body for n in ast.walk(stmt)) - bound(outer_nodes) - {inner.name}
+    read_outside = {n.id for n in outer_nodes if isinstance(n, ast.Name) and isinstance(n.ctx, ast.Load)}
+    assert not (only_inner & read_outside), sorted(only_inner & read_outside)
