@@ -53,9 +53,9 @@ METRIC = "SSD prefill tokens/s + TFLOP/s; decode tokens/s + state GB/s (1 B200)"
 # reports null until it is captured again (summaries under profiles/).
 NCU_TRAFFIC = {
     ("ssd_decode.cu", "decode_b256"): ("cba348ad46ab41a0", 1079097000 + 1024990000),
-    ("ssd_prefill_pair.cu", "mamba2_1p3b"): ("5ba6bd034334ce0e", 77948416 + 88473856),
+    ("ssd_prefill_pair.cu", "mamba2_1p3b"): ("b35367f961e75b78", 77953536 + 87025152),
     # captured with 32 of the 512 sequences and scaled by 16 (profiles/ssd_pair_kernel_handoff_prefill_b512.md)
-    ("ssd_prefill_pair.cu", "handoff_prefill"): ("5ba6bd034334ce0e", (729124864 + 1091180800) * 16),
+    ("ssd_prefill_pair.cu", "handoff_prefill"): ("b35367f961e75b78", (729406976 + 1091555328) * 16),
 }
 
 

@@ -759,26 +759,62 @@ ssd_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
             mbar_arrive(bar(B_EPI));          // the Y accumulators may be reused
             const float Dk[2] = {p.D ? __ldg(p.D + d.h0) : 0.f, p.D ? __ldg(p.D + d.h0 + 1) : 0.f};
             if (M3) {
-                // y = Y + (D - c_t) x straight from the registers (16 columns of the row per head)
+                // y = Y + D x straight from the registers (16 columns of the row per head).
+                // fp32: the 16-byte pieces are first transposed within lane quads
+                // (lane 4i+c then holds piece c of rows 4i..4i+3 of the warp), so that
+                // each store instruction writes 8 rows of 64 contiguous bytes, not 32
+                // rows of 16
                 const long long t = (long long)j * SUB + row;
-                if (t < p.L) {
+                const long long tq = (long long)j * SUB + 32 * q + (lane & ~3);
+                const int jq = lane & 3;
 #pragma unroll
-                    for (int k = 0; k < 2; ++k) {
-                        float out[16];
-                        const f32x2 dd = f2_pack(Dk[k], Dk[k]);
+                for (int k = 0; k < 2; ++k) {
+                    float out[16];
+                    const f32x2 dd = f2_pack(Dk[k], Dk[k]);
 #pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            f2_unpack(f2_fma(dd, bf16x2_to_f2(xr[k][e]), f2_pack_u(yv[k][2 * e], yv[k][2 * e + 1])),
-                                      out[2 * e], out[2 * e + 1]);
-                        const long long o = (((long long)d.b * p.L + t) * p.H + d.h0 + k) * PD + 16 * kq;
-                        if (p.y_bf16) {
-                            bf16* yo = reinterpret_cast<bf16*>(p.y) + o;
+                    for (int e = 0; e < 8; ++e)
+                        f2_unpack(f2_fma(dd, bf16x2_to_f2(xr[k][e]), f2_pack_u(yv[k][2 * e], yv[k][2 * e + 1])),
+                                  out[2 * e], out[2 * e + 1]);
+                    if (p.y_bf16) {
+                        if (t < p.L) {
+                            bf16* yo = reinterpret_cast<bf16*>(p.y) + (((long long)d.b * p.L + t) * p.H + d.h0 + k) * PD +
+                                       16 * kq;
                             Vec16<bf16>::store(yo, out);
                             Vec16<bf16>::store(yo + 8, out + 8);
-                        } else {
-                            float* yo = reinterpret_cast<float*>(p.y) + o;
+                        }
+                    } else {
+                        float4 ch[4];
 #pragma unroll
-                            for (int i = 0; i < 16; i += 4) Vec16<float>::store(yo + i, out + i);
+                        for (int c = 0; c < 4; ++c)
+                            ch[c] = make_float4(out[4 * c], out[4 * c + 1], out[4 * c + 2], out[4 * c + 3]);
+                        // swap 2x2 blocks of pieces with lane ^ 2, then single pieces with lane ^ 1
+#pragma unroll
+                        for (int u = 0; u < 2; ++u) {
+                            const bool hi = jq & 2;
+                            const float4 v = hi ? ch[u] : ch[2 + u];
+                            const float4 r = make_float4(__shfl_xor_sync(0xffffffffu, v.x, 2),
+                                                         __shfl_xor_sync(0xffffffffu, v.y, 2),
+                                                         __shfl_xor_sync(0xffffffffu, v.z, 2),
+                                                         __shfl_xor_sync(0xffffffffu, v.w, 2));
+                            if (hi) ch[u] = r; else ch[2 + u] = r;
+                        }
+#pragma unroll
+                        for (int u = 0; u < 2; ++u) {
+                            const bool odd = jq & 1;
+                            const float4 v = odd ? ch[2 * u] : ch[2 * u + 1];
+                            const float4 r = make_float4(__shfl_xor_sync(0xffffffffu, v.x, 1),
+                                                         __shfl_xor_sync(0xffffffffu, v.y, 1),
+                                                         __shfl_xor_sync(0xffffffffu, v.z, 1),
+                                                         __shfl_xor_sync(0xffffffffu, v.w, 1));
+                            if (odd) ch[2 * u] = r; else ch[2 * u + 1] = r;
+                        }
+#pragma unroll
+                        for (int m = 0; m < 4; ++m) {
+                            if (tq + m < p.L) {
+                                float* yo = reinterpret_cast<float*>(p.y) +
+                                            (((long long)d.b * p.L + tq + m) * p.H + d.h0 + k) * PD + 16 * kq + 4 * jq;
+                                *reinterpret_cast<float4*>(yo) = ch[m];
+                            }
                         }
                     }
                 }
