@@ -309,6 +309,18 @@ def _stream(stream) -> int:
     return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
 
 
+def _expect(t, shape, name, dtype=None):
+    """The C ABI takes bare pointers and sizes from the descriptor, so a tensor of
+    another shape or dtype than the descriptor implies would be read or written
+    out of bounds: refuse it here (None passes: optional arguments)."""
+    if t is None:
+        return
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected {dtype}")
+
+
 def prefill_desc(x, B, chunk, y_dtype=None, state_dtype=None) -> PrefillDesc:
     import torch
     b, L, H, P = x.shape
@@ -323,6 +335,18 @@ def workspace_bytes(x, B, chunk, y_dtype=None, state_dtype=None) -> int:
     return ssd_chunk_scan_workspace_size(prefill_desc(x, B, chunk, y_dtype, state_dtype))
 
 
+def _check_prefill_args(desc, x, dt_raw, dt_bias, A, B, C, D, init_state):
+    import torch
+    b, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    _expect(dt_raw, (b, L, H), "dt_raw", x.dtype)
+    _expect(B, (b, L, G, N), "B", x.dtype)
+    _expect(C, (b, L, G, N), "C", x.dtype)
+    for name, t in (("dt_bias", dt_bias), ("A", A), ("D", D)):
+        _expect(t, (H,), name, torch.float32)
+    _expect(init_state, (b, H, N, P), "init_state", _torch_dtype(desc.state_dtype))
+
+
 def chunk_scan_fwd(x, dt_raw, dt_bias, A, B, C, D, chunk, init_state=None, *, y=None, final_state=None,
                    y_dtype=None, state_dtype=None, want_final_state=True, workspace=None, pad_left=None, stream=None):
     """Chunked prefill scan.  Shapes: x [b,L,H,P], dt_raw [b,L,H], B/C [b,L,G,N], dt_bias/A/D [H] (fp32);
@@ -332,11 +356,18 @@ def chunk_scan_fwd(x, dt_raw, dt_bias, A, B, C, D, chunk, init_state=None, *, y=
     when not given; ``state_dtype`` defaults to init_state's dtype, else fp32.
     """
     import torch
+    if y_dtype is None and y is not None:
+        y_dtype = y.dtype
     if state_dtype is None:
-        state_dtype = init_state.dtype if init_state is not None else torch.float32
+        state_dtype = (init_state.dtype if init_state is not None else
+                       final_state.dtype if final_state is not None else torch.float32)
     desc = prefill_desc(x, B, chunk, y_dtype, state_dtype)
     b, L, H, P = x.shape
-    N = B.shape[3]
+    G, N = B.shape[2], B.shape[3]
+    _check_prefill_args(desc, x, dt_raw, dt_bias, A, B, C, D, init_state)
+    _expect(y, (b, L, H, P), "y", _torch_dtype(desc.y_dtype))
+    _expect(final_state, (b, H, N, P), "final_state", _torch_dtype(desc.state_dtype))
+    _expect(pad_left, (b,), "pad_left")
     for t in (x, dt_raw, B, C, dt_bias, A, D, init_state, y, final_state):
         if t is not None and (not t.is_cuda or not t.is_contiguous()):
             raise ValueError("libssd takes contiguous CUDA tensors")
@@ -371,7 +402,10 @@ def chunk_scan_fwd_mamba3(x, dt_raw, dt_bias, A, B, C, D, chunk, lam=None, theta
         state_dtype = init_state.dtype if init_state is not None else torch.float32
     desc = prefill_desc(x, B, chunk, y_dtype, state_dtype)
     b, L, H, P = x.shape
-    N = B.shape[3]
+    G, N = B.shape[2], B.shape[3]
+    _check_prefill_args(desc, x, dt_raw, dt_bias, A, B, C, D, init_state)
+    _expect(lam, (b, L, H), "lam")
+    _expect(theta, (b, L, G, N // 2), "theta")
     for t in (x, dt_raw, B, C, dt_bias, A, D, lam, theta, init_state):
         if t is not None and (not t.is_cuda or not t.is_contiguous()):
             raise ValueError("libssd takes contiguous CUDA tensors")
@@ -407,6 +441,9 @@ def chunk_scan_bwd(x, dt_raw, dt_bias, A, B, C, D, chunk, dy, init_state=None, d
     desc = prefill_desc(x, B, chunk, grad_dtype, state_dtype)
     b, L, H, P = x.shape
     G, N = B.shape[2], B.shape[3]
+    _check_prefill_args(desc, x, dt_raw, dt_bias, A, B, C, D, init_state)
+    _expect(dy, (b, L, H, P), "dy", x.dtype)
+    _expect(dfinal_state, (b, H, N, P), "dfinal_state", _torch_dtype(desc.state_dtype))
     for t in (x, dt_raw, B, C, dt_bias, A, D, init_state, dy, dfinal_state):
         if t is not None and (not t.is_cuda or not t.is_contiguous()):
             raise ValueError("libssd takes contiguous CUDA tensors")
@@ -433,11 +470,28 @@ def chunk_scan_bwd(x, dt_raw, dt_bias, A, B, C, D, chunk, dy, init_state=None, d
     return out
 
 
+def _check_decode_args(state, x, dt_raw, dt_bias, A, B, C, D, y, y_dtype, bshape=None):
+    import torch
+    b, H = x.shape[0], x.shape[1]
+    P = x.shape[-1]
+    G, N = B.shape[1], B.shape[-1]
+    _expect(state, (b, H, N, P), "state")
+    _expect(dt_raw, (b, H), "dt_raw", x.dtype)
+    _expect(B, bshape or (b, G, N), "B", x.dtype)
+    _expect(C, bshape or (b, G, N), "C", x.dtype)
+    for name, t in (("dt_bias", dt_bias), ("A", A), ("D", D)):
+        _expect(t, (H,), name, torch.float32)
+    _expect(y, tuple(x.shape), "y", y_dtype)
+
+
 def state_update(state, x, dt_raw, dt_bias, A, B, C, D, *, y=None, y_dtype=None, stream=None):
     """Decode step in place on ``state`` [b,H,N,P].  x [b,H,P], dt_raw [b,H], B/C [b,G,N].  Returns y."""
     import torch
     b, H, P = x.shape
     G, N = B.shape[1], B.shape[2]
+    if y_dtype is None and y is not None:
+        y_dtype = y.dtype
+    _check_decode_args(state, x, dt_raw, dt_bias, A, B, C, D, y, y_dtype)
     io = _dtype_code(x.dtype)
     desc = DecodeDesc(b, H, P, N, G, io, _dtype_code(y_dtype) if y_dtype is not None else io,
                       _dtype_code(state.dtype))
@@ -461,6 +515,13 @@ def state_update_mamba3(state, x, dt_raw, dt_bias, A, B, C, D, *, x_prev=None, B
     import torch
     b, H, P = x.shape
     G, N = B.shape[1], B.shape[2]
+    if y_dtype is None and y is not None:
+        y_dtype = y.dtype
+    _check_decode_args(state, x, dt_raw, dt_bias, A, B, C, D, y, y_dtype)
+    _expect(x_prev, (b, H, P), "x_prev", x.dtype)
+    _expect(B_prev, (b, G, N), "B_prev", x.dtype)
+    _expect(lam, (b, H), "lam")
+    _expect(theta, (b, G, N // 2), "theta")
     io = _dtype_code(x.dtype)
     desc = DecodeDesc(b, H, P, N, G, io, _dtype_code(y_dtype) if y_dtype is not None else io,
                       _dtype_code(state.dtype))
@@ -497,7 +558,12 @@ def replay_step(checkpoint, buffer, fill, capacity, x, dt_raw, dt_bias, A, B, C,
     """Replayed decode step: checkpoint [b,H,N,P] + buffer (``replay_buffer``) holding ``fill``
     tokens; x [b,H,P], dt_raw [b,H], B/C [b,G,N].  Returns (y, next fill)."""
     import torch
+    if y_dtype is None and y is not None:
+        y_dtype = y.dtype
+    _check_decode_args(checkpoint, x, dt_raw, dt_bias, A, B, C, D, y, y_dtype)
     desc = replay_desc(checkpoint, x, B, capacity, y_dtype)
+    if buffer is not None and buffer.numel() * buffer.element_size() < ssd_replay_buffer_size(desc):
+        raise ValueError("buffer: smaller than ssd_replay_buffer_size")
     for t in (checkpoint, buffer, x, dt_raw, B, C, dt_bias, A, D, y):
         if t is not None and (not t.is_cuda or not t.is_contiguous()):
             raise ValueError("libssd takes contiguous CUDA tensors")
@@ -516,6 +582,9 @@ def state_update_mimo(state, x, dt_raw, dt_bias, A, B, C, D, *, y=None, y_dtype=
     import torch
     b, H, R, P = x.shape
     G, N = B.shape[1], B.shape[3]
+    if y_dtype is None and y is not None:
+        y_dtype = y.dtype
+    _check_decode_args(state, x, dt_raw, dt_bias, A, B, C, D, y, y_dtype, bshape=(b, G, R, N))
     io = _dtype_code(x.dtype)
     desc = MimoDesc(b, H, P, N, G, R, io, _dtype_code(y_dtype) if y_dtype is not None else io,
                     _dtype_code(state.dtype))

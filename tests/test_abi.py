@@ -376,3 +376,49 @@ def test_binding_rejects_host_or_strided_tensors_before_any_cuda_call():
                                                    lam=torch.zeros(1, 4, 2).transpose(1, 2))):
         with pytest.raises(ValueError):
             call()
+
+
+def test_binding_rejects_outputs_and_inputs_the_descriptor_does_not_describe():
+    """The C ABI sizes every buffer from the descriptor; the wrappers refuse a
+    tensor of another shape or dtype (a bf16 final state given where the
+    descriptor says fp32 would be written past its end), before any CUDA call,
+    and take y's and the final state's dtypes from the tensors given."""
+    import torch
+    b, L, H, P, N, G = 1, 4, 2, 8, 8, 1
+    x = torch.zeros(b, L, H, P, dtype=torch.bfloat16)
+    dt = torch.zeros(b, L, H, dtype=torch.bfloat16)
+    B = torch.zeros(b, L, G, N, dtype=torch.bfloat16)
+    A = torch.zeros(H)
+    bad = [
+        dict(final_state=torch.zeros(b, H, N, P, dtype=torch.bfloat16), state_dtype=torch.float32),
+        dict(y=torch.zeros(b, L, H, P, dtype=torch.float32), y_dtype=torch.bfloat16),
+        dict(y=torch.zeros(b, L, H, P + 1)),
+        dict(final_state=torch.zeros(b, H, N + 1, P)),
+    ]
+    for kw in bad:
+        with pytest.raises(ValueError, match="y|final_state"):
+            ssd.chunk_scan_fwd(x, dt, None, A, B, B, None, 16, **kw)
+    with pytest.raises(ValueError, match="dt_raw"):
+        ssd.chunk_scan_fwd(x, dt.float(), None, A, B, B, None, 16)
+    with pytest.raises(ValueError, match="C"):
+        ssd.chunk_scan_fwd(x, dt, None, A, B, B[:, :, :, :4].contiguous(), None, 16)
+    with pytest.raises(ValueError, match="A"):
+        ssd.chunk_scan_fwd(x, dt, None, torch.zeros(H + 1), B, B, None, 16)
+    with pytest.raises(ValueError, match="dy"):
+        ssd.chunk_scan_bwd(x, dt, None, A, B, B, None, 16, x[:, :2].contiguous())
+    with pytest.raises(ValueError, match="theta"):
+        ssd.chunk_scan_fwd_mamba3(x, dt, None, A, B, B, None, 16, theta=torch.zeros(b, L, G, N))
+    # decode: state, y and the step's operands
+    st = torch.zeros(b, H, N, P)
+    xd, dtd, Bd = torch.zeros(b, H, P, dtype=torch.bfloat16), torch.zeros(b, H, dtype=torch.bfloat16), \
+        torch.zeros(b, G, N, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="state"):
+        ssd.state_update(torch.zeros(b, H, N, P + 1), xd, dtd, None, A, Bd, Bd, None)
+    with pytest.raises(ValueError, match="y"):
+        ssd.state_update(st, xd, dtd, None, A, Bd, Bd, None, y=torch.zeros(b, H, P), y_dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="B_prev"):
+        ssd.state_update_mamba3(st, xd, dtd, None, A, Bd, Bd, None, B_prev=torch.zeros(b, G, N + 2,
+                                                                                        dtype=torch.bfloat16))
+    # well-formed host tensors still reach the device check
+    with pytest.raises(ValueError, match="CUDA"):
+        ssd.chunk_scan_fwd(x, dt, None, A, B, B, None, 16, final_state=torch.zeros(b, H, N, P, dtype=torch.bfloat16))
