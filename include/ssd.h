@@ -273,7 +273,10 @@ ssd_status_t ssd_chunk_scan_bwd_launches(const ssd_prefill_desc_t* desc, int32_t
  * R(theta) turns (h[2k], h[2k+1]) counter-clockwise by theta[t][g][k]; there
  * is no input before the first token.  Computed, as the pages suggest, by
  * turning B and C with the cumulative angle and running the real chunked scan
- * with the trapezoid's weights, then a per-token diagonal correction.
+ * with the trapezoid's weights (a token's own term weighted lam dt): with bf16
+ * inputs and the head-pair shapes (N = 128, P = 64, an even number of heads per
+ * group, batch * nheads >= 148) in one scan over the turned operands' bf16
+ * hi/lo pairs, otherwise as three scans and a combination.
  *
  *  arguments as ssd_chunk_scan_fwd, plus
  *  lam    [b][L][H]      fp32  nullable (= 1: Euler input, Mamba-2's)
